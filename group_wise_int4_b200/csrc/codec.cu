@@ -1,0 +1,456 @@
+// Group-wise int4/int8 compression and decompression (FlexGen source walkthrough,
+// section 6.3: compress / decompress of a CompressionConfig(num_bits, group_size,
+// group_dim, symmetric=False) with a packed uint8 data tensor and an fp16 per-group
+// scale).
+//
+// Both directions are pure HBM streams (2 + bits/8 + 4/group_size bytes per element),
+// so the kernels are shaped for bandwidth: 16-byte vector loads that bypass L1,
+// streaming stores, several independent vectors in flight per thread, and a
+// grid-stride loop sized to the SM count.
+//
+// Two layouts:
+//   contiguous - the group dimension is the last one: the tensor is a flat sequence of
+//                groups; gs/8 lanes share a group and reduce min/max with shuffles.
+//   strided    - the group dimension has inner extent `inner` > 1 after it: a thread
+//                owns 8 adjacent columns (one 16-byte vector per row), scans the
+//                group's rows once for min/max and once more (from L2) to quantise.
+#include "quant.cuh"
+
+namespace flexq {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+// ---------------------------------------------------------------------------------
+// contiguous compress: G groups of GS fp16, codes G x (GS*BITS/8) bytes, meta G half2
+template <int BITS, int GS>
+__global__ void __launch_bounds__(kThreads) compress_contig_kernel(const __half* __restrict__ x,
+                                                                   uint8_t* __restrict__ codes,
+                                                                   uint32_t* __restrict__ meta,
+                                                                   int64_t G) {
+    constexpr int L = GS / 8;      // lanes per group
+    constexpr int GPW = 32 / L;    // groups per warp and step
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % L;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+    const int64_t stride = nwarps * GPW;
+
+    for (int64_t base = warp * GPW; base < G; base += stride * kUnroll) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = base + u * stride + lane / L;
+            v[u] = g < G ? ld_stream_v4(x + g * GS + sub * 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = base + u * stride + lane / L;
+            __half2 hmn, hmx;
+            minmax8(v[u], hmn, hmx);
+            float mn = hmin_of(hmn), mx = hmax_of(hmx);
+#pragma unroll
+            for (int off = 1; off < L; off <<= 1) {
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            }
+            const __half s16 = group_scale16<BITS>(mn, mx);
+            const float s = __half2float(s16);
+            if (g < G) {
+                if (BITS == 4) {
+                    st_stream_u32(codes + g * (GS / 2) + sub * 4, quant8_4bit(v[u], mn, s));
+                } else {
+                    st_stream_v2(codes + g * GS + sub * 8, quant8_8bit(v[u], mn, s));
+                }
+                if (sub == 0) meta[g] = pack_half2_bits(__float2half_rn(mn), s16);
+            }
+        }
+    }
+}
+
+// contiguous decompress: one thread per 16 bytes of codes (32 values at 4 bits,
+// 16 values at 8 bits).
+template <int BITS, int GS>
+__global__ void __launch_bounds__(kThreads) decompress_contig_kernel(const uint8_t* __restrict__ codes,
+                                                                     const uint32_t* __restrict__ meta,
+                                                                     __half* __restrict__ y,
+                                                                     int64_t chunks) {
+    constexpr int EPT = 128 / BITS;  // values per 16-byte chunk
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
+    for (int64_t base = tid; base < chunks; base += nthreads * kUnroll) {
+        uint4 c[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t ch = base + u * nthreads;
+            c[u] = ch < chunks ? ld_stream_v4(codes + ch * 16) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t ch = base + u * nthreads;
+            if (ch >= chunks) continue;
+            const int64_t e0 = ch * EPT;
+            // a chunk lies inside one group when EPT <= GS (always: EPT <= 32 <= GS)
+            const uint32_t m = __ldg(meta + e0 / GS);
+            const float mn = h2f_lo(m);
+            const float step = group_step(__ushort_as_half(static_cast<unsigned short>(m >> 16)));
+            const uint32_t w[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+            uint32_t out[EPT / 2];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (BITS == 4) {
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        const uint32_t byte = (w[k] >> (8 * b)) & 0xFFu;
+                        out[k * 4 + b] = pack_half2_bits(dequant_one(byte & 15u, step, mn),
+                                                         dequant_one(byte >> 4, step, mn));
+                    }
+                } else {
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) {
+                        const uint32_t pair = (w[k] >> (16 * b)) & 0xFFFFu;
+                        out[k * 2 + b] = pack_half2_bits(dequant_one(pair & 0xFFu, step, mn),
+                                                         dequant_one(pair >> 8, step, mn));
+                    }
+                }
+            }
+            uint4* dst = reinterpret_cast<uint4*>(y + e0);
+#pragma unroll
+            for (int q = 0; q < EPT / 8; ++q)
+                st_stream_v4(dst + q, make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// strided compress: x viewed as [outer][ng*GS][inner]; a work item is (o, g, 8 columns)
+// (VEC = 8) or (o, g, 1 column) (VEC = 1, ragged widths or unaligned pointers).
+template <int BITS, int GS, int VEC>
+__global__ void __launch_bounds__(kThreads) compress_strided_kernel(const __half* __restrict__ x,
+                                                                    uint8_t* __restrict__ codes,
+                                                                    uint32_t* __restrict__ meta,
+                                                                    int64_t outer, int64_t ng,
+                                                                    int64_t inner) {
+    const int64_t cols = inner / VEC;
+    const int64_t items = outer * ng * cols;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
+    constexpr int CB = GS * BITS / 8;  // code rows per group
+    for (int64_t it = tid; it < items; it += nthreads) {
+        const int64_t cv = it % cols;
+        const int64_t og = it / cols;  // o * ng + g
+        const int64_t c0 = cv * VEC;
+        const __half* src = x + og * GS * inner + c0;
+        float mn[VEC], mx[VEC];
+        if (VEC == 8) {
+            __half2 m2[4], M2[4];
+            {
+                const uint4 v = ld_stream_v4(src);
+                const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) m2[k] = M2[k] = h[k];
+            }
+#pragma unroll 8
+            for (int r = 1; r < GS; ++r) {
+                const uint4 v = *reinterpret_cast<const uint4*>(src + r * inner);
+                const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    m2[k] = __hmin2(m2[k], h[k]);
+                    M2[k] = __hmax2(M2[k], h[k]);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                mn[2 * k] = __low2float(m2[k]);
+                mn[2 * k + 1] = __high2float(m2[k]);
+                mx[2 * k] = __low2float(M2[k]);
+                mx[2 * k + 1] = __high2float(M2[k]);
+            }
+        } else {
+            mn[0] = mx[0] = __half2float(src[0]);
+            for (int r = 1; r < GS; ++r) {
+                const float v = __half2float(src[r * inner]);
+                mn[0] = fminf(mn[0], v);
+                mx[0] = fmaxf(mx[0], v);
+            }
+        }
+        float s[VEC];
+        uint32_t mw[VEC];
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) {
+            const __half s16 = group_scale16<BITS>(mn[k], mx[k]);
+            s[k] = __half2float(s16);
+            mw[k] = pack_half2_bits(__float2half_rn(mn[k]), s16);
+        }
+        uint8_t* dst = codes + og * CB * inner + c0;
+        if (VEC == 8) {
+#pragma unroll 4
+            for (int r = 0; r < GS; r += (BITS == 4 ? 2 : 1)) {
+                const uint4 a = *reinterpret_cast<const uint4*>(src + r * inner);
+                const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
+                uint32_t lo = 0, hi = 0;
+                if (BITS == 4) {
+                    const uint4 b = *reinterpret_cast<const uint4*>(src + (r + 1) * inner);
+                    const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t q0 = quant_one<4>(h2f_lo(wa[k]), mn[2 * k], s[2 * k]) |
+                                            (quant_one<4>(h2f_lo(wb[k]), mn[2 * k], s[2 * k]) << 4);
+                        const uint32_t q1 = quant_one<4>(h2f_hi(wa[k]), mn[2 * k + 1], s[2 * k + 1]) |
+                                            (quant_one<4>(h2f_hi(wb[k]), mn[2 * k + 1], s[2 * k + 1]) << 4);
+                        const uint32_t two = q0 | (q1 << 8);
+                        if (k < 2) lo |= two << (16 * k); else hi |= two << (16 * (k - 2));
+                    }
+                    st_stream_v2(dst + (r / 2) * inner, make_uint2(lo, hi));
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t two = quant_one<8>(h2f_lo(wa[k]), mn[2 * k], s[2 * k]) |
+                                             (quant_one<8>(h2f_hi(wa[k]), mn[2 * k + 1], s[2 * k + 1]) << 8);
+                        if (k < 2) lo |= two << (16 * k); else hi |= two << (16 * (k - 2));
+                    }
+                    st_stream_v2(dst + r * inner, make_uint2(lo, hi));
+                }
+            }
+            uint32_t* md = meta + og * inner + c0;
+            st_stream_v4(md, make_uint4(mw[0], mw[1], mw[2], mw[3]));
+            st_stream_v4(md + 4, make_uint4(mw[4], mw[5], mw[6], mw[7]));
+        } else {
+            for (int r = 0; r < GS; r += (BITS == 4 ? 2 : 1)) {
+                uint32_t q = quant_one<BITS>(__half2float(src[r * inner]), mn[0], s[0]);
+                if (BITS == 4) q |= quant_one<4>(__half2float(src[(r + 1) * inner]), mn[0], s[0]) << 4;
+                dst[(BITS == 4 ? r / 2 : r) * inner] = static_cast<uint8_t>(q);
+            }
+            meta[og * inner + c0] = mw[0];
+        }
+    }
+}
+
+template <int BITS, int GS, int VEC>
+__global__ void __launch_bounds__(kThreads) decompress_strided_kernel(const uint8_t* __restrict__ codes,
+                                                                      const uint32_t* __restrict__ meta,
+                                                                      __half* __restrict__ y,
+                                                                      int64_t outer, int64_t ng,
+                                                                      int64_t inner) {
+    const int64_t cols = inner / VEC;
+    const int64_t items = outer * ng * cols;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
+    constexpr int CB = GS * BITS / 8;
+    for (int64_t it = tid; it < items; it += nthreads) {
+        const int64_t cv = it % cols;
+        const int64_t og = it / cols;
+        const int64_t c0 = cv * VEC;
+        float mn[VEC], step[VEC];
+        const uint32_t* ms = meta + og * inner + c0;
+        if (VEC == 8) {
+            const uint4 a = ld_stream_v4(ms);
+            const uint4 b = ld_stream_v4(ms + 4);
+            const uint32_t m[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                mn[k] = h2f_lo(m[k]);
+                step[k] = group_step(__ushort_as_half(static_cast<unsigned short>(m[k] >> 16)));
+            }
+        } else {
+            mn[0] = h2f_lo(ms[0]);
+            step[0] = group_step(__ushort_as_half(static_cast<unsigned short>(ms[0] >> 16)));
+        }
+        const uint8_t* src = codes + og * CB * inner + c0;
+        __half* dst = y + og * GS * inner + c0;
+        if (VEC == 8) {
+#pragma unroll 4
+            for (int j = 0; j < CB; ++j) {
+                uint2 cw;
+                asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                             : "=r"(cw.x), "=r"(cw.y)
+                             : "l"(src + j * inner));
+                const uint32_t w[2] = {cw.x, cw.y};
+                if (BITS == 4) {
+                    uint32_t r0[4], r1[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t b0 = (w[k / 2] >> (16 * (k % 2))) & 0xFFu;
+                        const uint32_t b1 = (w[k / 2] >> (16 * (k % 2) + 8)) & 0xFFu;
+                        r0[k] = pack_half2_bits(dequant_one(b0 & 15u, step[2 * k], mn[2 * k]),
+                                                dequant_one(b1 & 15u, step[2 * k + 1], mn[2 * k + 1]));
+                        r1[k] = pack_half2_bits(dequant_one(b0 >> 4, step[2 * k], mn[2 * k]),
+                                                dequant_one(b1 >> 4, step[2 * k + 1], mn[2 * k + 1]));
+                    }
+                    st_stream_v4(dst + (2 * j) * inner, make_uint4(r0[0], r0[1], r0[2], r0[3]));
+                    st_stream_v4(dst + (2 * j + 1) * inner, make_uint4(r1[0], r1[1], r1[2], r1[3]));
+                } else {
+                    uint32_t r0[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t b0 = (w[k / 2] >> (16 * (k % 2))) & 0xFFu;
+                        const uint32_t b1 = (w[k / 2] >> (16 * (k % 2) + 8)) & 0xFFu;
+                        r0[k] = pack_half2_bits(dequant_one(b0, step[2 * k], mn[2 * k]),
+                                                dequant_one(b1, step[2 * k + 1], mn[2 * k + 1]));
+                    }
+                    st_stream_v4(dst + j * inner, make_uint4(r0[0], r0[1], r0[2], r0[3]));
+                }
+            }
+        } else {
+            for (int j = 0; j < CB; ++j) {
+                const uint32_t b = src[j * inner];
+                if (BITS == 4) {
+                    dst[(2 * j) * inner] = dequant_one(b & 15u, step[0], mn[0]);
+                    dst[(2 * j + 1) * inner] = dequant_one(b >> 4, step[0], mn[0]);
+                } else {
+                    dst[j * inner] = dequant_one(b, step[0], mn[0]);
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------
+struct Geometry {
+    int64_t outer = 1, ng = 0, inner = 1, n = 0;
+    int gd = 0;
+};
+
+int validate(int32_t ndim, const int64_t* shape, const flexq_config& cfg, Geometry& geo) {
+    FLEX_REQUIRE(shape != nullptr, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(ndim >= 1 && ndim <= 4, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(cfg.symmetric == 0, FLEX_ERR_UNSUPPORTED);
+    FLEX_REQUIRE(cfg.num_bits == 4 || cfg.num_bits == 8, FLEX_ERR_UNSUPPORTED);
+    FLEX_REQUIRE(cfg.group_size == 32 || cfg.group_size == 64 || cfg.group_size == 128,
+                 FLEX_ERR_UNSUPPORTED);
+    int gd = cfg.group_dim;
+    if (gd < 0) gd += ndim;
+    FLEX_REQUIRE(gd >= 0 && gd < ndim, FLEX_ERR_INVALID_ARG);
+    int64_t n = 1;
+    for (int i = 0; i < ndim; ++i) {
+        FLEX_REQUIRE(shape[i] >= 0, FLEX_ERR_INVALID_ARG);
+        n *= shape[i];
+    }
+    FLEX_REQUIRE(shape[gd] % cfg.group_size == 0, FLEX_ERR_SHAPE);
+    geo.gd = gd;
+    geo.n = n;
+    geo.outer = 1;
+    for (int i = 0; i < gd; ++i) geo.outer *= shape[i];
+    geo.inner = 1;
+    for (int i = gd + 1; i < ndim; ++i) geo.inner *= shape[i];
+    geo.ng = shape[gd] / cfg.group_size;
+    return FLEX_OK;
+}
+
+unsigned grid_for(int64_t work_threads) {
+    const int64_t cap = static_cast<int64_t>(sm_count()) * (2048 / kThreads);
+    int64_t blocks = (work_threads + kThreads - 1) / kThreads;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return static_cast<unsigned>(blocks);
+}
+
+template <int BITS, int GS>
+int launch_compress(const Geometry& g, const __half* x, uint8_t* codes, uint32_t* meta,
+                    cudaStream_t st) {
+    if (g.inner == 1) {
+        const int64_t G = g.outer * g.ng;
+        const int64_t lanes = G * (GS / 8);
+        compress_contig_kernel<BITS, GS><<<grid_for((lanes + kUnroll - 1) / kUnroll), kThreads, 0, st>>>(
+            x, codes, meta, G);
+    } else {
+        const bool vec = (g.inner % 8 == 0);
+        const int64_t items = g.outer * g.ng * (vec ? g.inner / 8 : g.inner);
+        if (vec)
+            compress_strided_kernel<BITS, GS, 8><<<grid_for(items), kThreads, 0, st>>>(x, codes, meta, g.outer,
+                                                                                     g.ng, g.inner);
+        else
+            compress_strided_kernel<BITS, GS, 1><<<grid_for(items), kThreads, 0, st>>>(x, codes, meta, g.outer,
+                                                                                     g.ng, g.inner);
+    }
+    return launch_status();
+}
+
+template <int BITS, int GS>
+int launch_decompress(const Geometry& g, const uint8_t* codes, const uint32_t* meta, __half* y,
+                      cudaStream_t st) {
+    if (g.inner == 1) {
+        const int64_t chunks = g.n * BITS / 8 / 16;
+        decompress_contig_kernel<BITS, GS><<<grid_for((chunks + kUnroll - 1) / kUnroll), kThreads, 0, st>>>(
+            codes, meta, y, chunks);
+    } else {
+        const bool vec = (g.inner % 8 == 0);
+        const int64_t items = g.outer * g.ng * (vec ? g.inner / 8 : g.inner);
+        if (vec)
+            decompress_strided_kernel<BITS, GS, 8><<<grid_for(items), kThreads, 0, st>>>(codes, meta, y, g.outer,
+                                                                                       g.ng, g.inner);
+        else
+            decompress_strided_kernel<BITS, GS, 1><<<grid_for(items), kThreads, 0, st>>>(codes, meta, y, g.outer,
+                                                                                       g.ng, g.inner);
+    }
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace flexq
+
+using namespace flexq;
+
+extern "C" int64_t flexq_codes_bytes(int32_t ndim, const int64_t* shape, flexq_config cfg) {
+    Geometry g;
+    const int rc = validate(ndim, shape, cfg, g);
+    if (rc != FLEX_OK) return rc;
+    return g.n * cfg.num_bits / 8;
+}
+
+extern "C" int64_t flexq_meta_bytes(int32_t ndim, const int64_t* shape, flexq_config cfg) {
+    Geometry g;
+    const int rc = validate(ndim, shape, cfg, g);
+    if (rc != FLEX_OK) return rc;
+    return g.outer * g.ng * g.inner * 4;
+}
+
+extern "C" int flexq_compress(const void* x, int32_t ndim, const int64_t* shape, flexq_config cfg,
+                              void* codes, void* meta, void* stream) {
+    Geometry g;
+    const int rc = validate(ndim, shape, cfg, g);
+    if (rc != FLEX_OK) return rc;
+    if (g.n == 0) return FLEX_OK;
+    FLEX_REQUIRE(x && codes && meta, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(aligned16(x) && aligned16(codes) && aligned16(meta), FLEX_ERR_ALIGN);
+    const cudaStream_t st = as_stream(stream);
+    const __half* xh = static_cast<const __half*>(x);
+    uint8_t* c = static_cast<uint8_t*>(codes);
+    uint32_t* m = static_cast<uint32_t*>(meta);
+#define CALL_C(B, S) launch_compress<B, S>(g, xh, c, m, st)
+    if (cfg.num_bits == 4) {
+        if (cfg.group_size == 32) return CALL_C(4, 32);
+        if (cfg.group_size == 64) return CALL_C(4, 64);
+        return CALL_C(4, 128);
+    }
+    if (cfg.group_size == 32) return CALL_C(8, 32);
+    if (cfg.group_size == 64) return CALL_C(8, 64);
+    return CALL_C(8, 128);
+#undef CALL_C
+}
+
+extern "C" int flexq_decompress(const void* codes, const void* meta, int32_t ndim, const int64_t* shape,
+                                flexq_config cfg, void* y, void* stream) {
+    Geometry g;
+    const int rc = validate(ndim, shape, cfg, g);
+    if (rc != FLEX_OK) return rc;
+    if (g.n == 0) return FLEX_OK;
+    FLEX_REQUIRE(y && codes && meta, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(aligned16(y) && aligned16(codes) && aligned16(meta), FLEX_ERR_ALIGN);
+    const cudaStream_t st = as_stream(stream);
+    const uint8_t* c = static_cast<const uint8_t*>(codes);
+    const uint32_t* m = static_cast<const uint32_t*>(meta);
+    __half* yh = static_cast<__half*>(y);
+#define CALL_D(B, S) launch_decompress<B, S>(g, c, m, yh, st)
+    if (cfg.num_bits == 4) {
+        if (cfg.group_size == 32) return CALL_D(4, 32);
+        if (cfg.group_size == 64) return CALL_D(4, 64);
+        return CALL_D(4, 128);
+    }
+    if (cfg.group_size == 32) return CALL_D(8, 32);
+    if (cfg.group_size == 64) return CALL_D(8, 64);
+    return CALL_D(8, 128);
+#undef CALL_D
+}

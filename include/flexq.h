@@ -1,0 +1,206 @@
+/*
+ * flexq.h - C ABI of the B200 (sm_100a) group-wise int4 OPT layer library.
+ *
+ * What it computes comes from the FlexGen pages:
+ *   - FlexGen source walkthrough, section 6.3 "4-bit group-wise quantisation of
+ *     weights and KV cache": CompressionConfig(num_bits, group_size, group_dim,
+ *     symmetric), compress / decompress, two 4-bit codes per uint8 in a data tensor of
+ *     shape shape[:group_dim] + (num_groups*(group_size//2),) + shape[group_dim+1:],
+ *     and an fp16 per-group scale tensor; weights use (4, 64) and the KV cache
+ *     (4, 64) grouped along the head dimension.
+ *   - FlexGen source-reading notes, "Pytorch Backend": prefill attention is `mha`,
+ *     the decode step is `mha_gen`; "Flex Opt": every step runs load_cache,
+ *     compute_layer, store_cache, in that order.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc / torch CUDA memory) unless
+ *     a parameter says otherwise. The caller owns and allocates every buffer:
+ *     inputs, outputs, codes, metadata, caches and workspaces. The library keeps no
+ *     per-call state; its only global state is one device status word per device,
+ *     created on first use (see flex_get_status).
+ *   - fp16 means IEEE binary16, "half2" a pair of binary16 stored as 4 bytes.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call only enqueues work on `stream` and returns; none synchronises,
+ *     except flex_get_status.
+ *   - Return value: FLEX_OK (0) or a negative FLEX_ERR_*. Argument errors are found
+ *     on the host before anything is enqueued; nothing is written then. No C++
+ *     exception crosses this boundary.
+ *   - Pointers must be 16-byte aligned. Outputs must not alias inputs unless stated.
+ *   - Non-finite inputs (NaN, Inf) give unspecified results.
+ */
+#ifndef FLEXQ_H
+#define FLEXQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------------ */
+#define FLEX_OK               0
+#define FLEX_ERR_INVALID_ARG (-1)  /* null pointer, negative size, bad rank       */
+#define FLEX_ERR_UNSUPPORTED (-2)  /* bits not 4/8, group not 32/64/128,
+                                      symmetric != 0, head_dim not 64/128, ...    */
+#define FLEX_ERR_SHAPE       (-3)  /* dim not a multiple of group_size,
+                                      pos >= max_seq, seq > max_seq, ...          */
+#define FLEX_ERR_ALIGN       (-4)  /* pointer not 16-byte aligned                 */
+#define FLEX_ERR_WORKSPACE   (-5)  /* workspace missing or too small              */
+#define FLEX_ERR_CUDA        (-6)  /* a CUDA launch or runtime call failed        */
+#define FLEX_ERR_TIMEOUT     (-7)  /* a device-side bounded wait gave up          */
+
+/* ---- compression configuration (CompressionConfig of section 6.3) ------------ */
+typedef struct {
+    int32_t num_bits;    /* 4 or 8                                                 */
+    int32_t group_size;  /* 32, 64 or 128                                          */
+    int32_t group_dim;   /* dimension the groups run along; negative counts back  */
+    int32_t symmetric;   /* must be 0: the min/max (asymmetric) form               */
+} flexq_config;
+
+/* A compressed tensor: the pages' (data, scale, config) triple.
+ *   codes: uint8, shape shape[:gd] + (ng*gs*bits/8,) + shape[gd+1:], row-major.
+ *          4-bit: byte j of a group = q[2j] | q[2j+1] << 4 (pairs along group_dim).
+ *   meta : half2 {min, scale} per group, shape shape[:gd] + (ng,) + shape[gd+1:].
+ *          scale = fp16((2^b - 1) / (max - min)), 0 for a constant group,
+ *          65504 where that quotient overflows fp16.                              */
+typedef struct {
+    const void*  codes;
+    const void*  meta;
+    int32_t      ndim;      /* 1..4 */
+    int64_t      shape[4];  /* logical (uncompressed) shape */
+    flexq_config cfg;
+} flexq_tensor;
+
+/* ---- codec (compress / decompress of section 6.3) ------------------------------ */
+
+/* Bytes of the codes / metadata buffers for a tensor of `shape` (rank ndim) under
+ * `cfg`. Returns a negative FLEX_ERR_* if the configuration or shape is invalid. */
+int64_t flexq_codes_bytes(int32_t ndim, const int64_t* shape, flexq_config cfg);
+int64_t flexq_meta_bytes(int32_t ndim, const int64_t* shape, flexq_config cfg);
+
+/* compress: x (fp16, row-major, `shape`) -> codes + meta, per group of group_size
+ * elements along group_dim:
+ *   min, max of the group; scale16 = fp16((2^b-1) / (max - min)) (0 if max == min,
+ *   65504 on overflow); q = clamp(rint((x - min) * scale16), 0, 2^b - 1), the
+ *   subtraction and the product each rounded in fp32, ties to even.
+ * Bit-exact and deterministic. Any rank 1..4; the group dimension may be the
+ * contiguous one or a strided one. Tensors of any size (64-bit indexing). */
+int flexq_compress(const void* x, int32_t ndim, const int64_t* shape, flexq_config cfg,
+                   void* codes, void* meta, void* stream);
+
+/* decompress: codes + meta -> y (fp16, `shape`):
+ *   y = fp16(fp32(fp32(q * fp32(1/scale16)) + min)), or y = min when scale16 == 0. */
+int flexq_decompress(const void* codes, const void* meta, int32_t ndim, const int64_t* shape,
+                     flexq_config cfg, void* y, void* stream);
+
+/* ---- OPT decoder layer ------------------------------------------------------- */
+
+/* Parameters of one OPT pre-LayerNorm decoder layer.
+ *   Weights are compressed with {4 or 8 bits, group 64, group_dim 1} and stored
+ *   [out][in] (grouped along the input dimension, the contiguous one):
+ *     w_qkv [3h][h]  rows ordered [q; k; v], feature = head*head_dim + j
+ *     w_o   [h][h], w_fc1 [ffn][h], w_fc2 [h][ffn]
+ *   Biases and LayerNorm parameters are plain fp16 vectors.                      */
+typedef struct {
+    int32_t h, n_heads, head_dim, ffn;
+    const void *ln1_g, *ln1_b, *ln2_g, *ln2_b;   /* fp16 [h]                        */
+    flexq_tensor w_qkv, w_o, w_fc1, w_fc2;       /* compressed weights              */
+    const void *b_qkv, *b_o, *b_fc1, *b_fc2;     /* fp16 [3h], [h], [ffn], [h]      */
+} flex_layer;
+
+/* Compressed KV cache of one layer (section 6.3: KV grouped along the head dim).
+ *   k_codes, v_codes: uint8 [batch][n_heads][max_seq][head_dim*bits/8]
+ *   k_meta,  v_meta : half2 [batch][n_heads][max_seq][head_dim/group_size]
+ *   cfg: num_bits 4 or 8, group_size 32/64 (dividing head_dim), group_dim = 3.   */
+typedef struct {
+    void *k_codes, *k_meta, *v_codes, *v_meta;
+    int32_t batch, n_heads, head_dim, max_seq;
+    flexq_config cfg;
+} flex_kv_cache;
+
+/* Workspace bytes that flex_prefill_layer (seq > 1) or flex_decode_layer (seq == 1)
+ * needs for `batch` sequences of `seq` tokens. Negative FLEX_ERR_* on bad args. */
+int64_t flex_workspace_bytes(const flex_layer* L, int32_t batch, int32_t seq);
+
+/* Prefill (`mha` path): x_in fp16 [batch][seq][h] -> x_out fp16 [batch][seq][h].
+ *   a = LN1(x); q,k,v = a Wqkv^T + b (q scaled by head_dim^-1/2); causal softmax
+ *   attention on the fresh fp16 q/k/v; h1 = x + o Wo^T + b_o;
+ *   out = h1 + ReLU(LN2(h1) W1^T + b1) W2^T + b2   (LayerNorm eps 1e-5).
+ * Writes the quantised fp16 keys/values of tokens [0, seq) into cache slots
+ * [0, seq) (store_cache). seq <= cache->max_seq, batch == cache->batch.
+ * ws: device workspace of at least flex_workspace_bytes(L, batch, seq) bytes;
+ * x_in and x_out must not alias. */
+int flex_prefill_layer(const flex_layer* L, const flex_kv_cache* cache, const void* x_in,
+                       void* x_out, int32_t batch, int32_t seq, void* ws, int64_t ws_bytes,
+                       void* stream);
+
+/* Decode step (`mha_gen` path) at position pos: x_in fp16 [batch][h] -> x_out fp16.
+ *   Same layer; the new token attends to the dequantised cache slots [0, pos) and
+ *   to its own fresh key/value; its quantised key/value are then in slot pos.
+ * pos < cache->max_seq; batch <= cache->batch (sequences 0..batch-1 of the cache).
+ * ws: at least flex_workspace_bytes(L, batch, 1) bytes. */
+int flex_decode_layer(const flex_layer* L, const flex_kv_cache* cache, const void* x_in,
+                      void* x_out, int32_t batch, int32_t pos, void* ws, int64_t ws_bytes,
+                      void* stream);
+
+/* ---- hot-path steps, callable one by one ------------------------------------- */
+
+/* store_cache: quantise k_new / v_new (fp16 [batch][n_heads][head_dim], rows of
+ * `row_stride` elements between consecutive sequences; head h of sequence b starts
+ * at b*row_stride + h*head_dim) into cache slot pos of sequences 0..batch-1.
+ * Same quantiser as flexq_compress with group_dim = head dim. */
+int flex_append_kv(const flex_kv_cache* cache, const void* k_new, const void* v_new,
+                   int64_t row_stride, int32_t batch, int32_t pos, void* stream);
+
+/* Decode attention (`mha_gen` core): per sequence b < batch and head:
+ *   o = softmax([q.k_0 .. q.k_{pos-1}, q.k_new]) [v_0 .. v_{pos-1}, v_new]
+ * with k_j, v_j the dequantised cache slots [0, pos). q, k_new, v_new: fp16 rows of
+ * `row_stride` elements per sequence, head h at offset h*head_dim (q is used as
+ * given: callers pre-scale it). o: fp16 [batch][n_heads*head_dim].
+ * ws: at least flex_decode_attention_ws_bytes(cache, batch, pos) bytes. */
+int64_t flex_decode_attention_ws_bytes(const flex_kv_cache* cache, int32_t batch, int32_t pos);
+int flex_decode_attention(const flex_kv_cache* cache, const void* q, const void* k_new,
+                          const void* v_new, int64_t row_stride, void* o, int32_t batch,
+                          int32_t pos, void* ws, int64_t ws_bytes, void* stream);
+
+/* Prefill attention (`mha` core): causal softmax attention on fresh fp16 q, k, v,
+ * each [batch][seq][n_heads][head_dim] inside rows of `row_stride` elements per
+ * token (token t of sequence b at (b*seq + t)*row_stride). o: fp16
+ * [batch][seq][n_heads*head_dim]. head_dim 64 or 128. */
+int flex_prefill_attention(const void* q, const void* k, const void* v, int64_t row_stride,
+                           void* o, int32_t batch, int32_t seq, int32_t n_heads,
+                           int32_t head_dim, void* stream);
+
+/* Dequant-fused weight GEMM: y[m][n] = epi( sum_k x[m][k] * W^[n][k] + bias[n] )
+ *   x fp16 [M][K] row-major, W compressed [N][K] (group 64 along K, 4 or 8 bits),
+ *   bias fp16 [N] or NULL, residual fp16 [M][N] or NULL (added after bias),
+ *   epilogue: FLEX_EPI_NONE, FLEX_EPI_RELU (after bias), FLEX_EPI_RESIDUAL.
+ *   y fp16 [M][N]; y may alias residual. ws: flex_gemm_ws_bytes(M, N, K) bytes.  */
+#define FLEX_EPI_NONE     0
+#define FLEX_EPI_RELU     1
+#define FLEX_EPI_RESIDUAL 2
+int64_t flex_gemm_ws_bytes(int32_t M, int32_t N, int32_t K);
+int flex_dequant_gemm(const void* x, const flexq_tensor* W, const void* bias,
+                      const void* residual, void* y, int32_t M, int32_t epilogue,
+                      void* ws, int64_t ws_bytes, void* stream);
+
+/* LayerNorm over rows of h fp16 values: y = (x - mean)/sqrt(var + 1e-5) * g + b,
+ * biased variance, fp32 statistics. x, y fp16 [rows][h]; may alias. */
+int flex_layernorm(const void* x, const void* g, const void* b, void* y, int64_t rows,
+                   int32_t h, void* stream);
+
+/* ---- status ------------------------------------------------------------------ */
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device: FLEX_OK, or FLEX_ERR_TIMEOUT if a kernel's bounded wait gave up
+ * since the last call, or FLEX_ERR_CUDA if the stream reports an error. */
+int flex_get_status(void* stream);
+
+/* Static English text for a status code. */
+const char* flex_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLEXQ_H */

@@ -396,13 +396,18 @@ int decode_attn_nsplit(int pairs, int pos) {
     int ns = (target + pairs - 1) / pairs;
     const int max_by_len = (pos + 31) / 32;          // at least 32 keys per split
     if (ns > max_by_len) ns = max_by_len;
-    const int min_by_smem = (pos + 8191) / 8192;
-    if (ns < min_by_smem) ns = min_by_smem;
     return ns < 1 ? 1 : ns;
 }
 
 int64_t decode_attn_ws_bytes(int pairs, int head_dim, int pos) {
     const int ns = decode_attn_nsplit(pairs, pos);
+    return static_cast<int64_t>(pairs) * (ns > 0 ? ns : 1) * (head_dim + 2) * 4;
+}
+
+// Bound on decode_attn_ws_bytes over every pos.
+int64_t decode_attn_ws_bound(int pairs, int head_dim) {
+    const int target = 4 * sm_count();
+    const int ns = (target + pairs - 1) / pairs;
     return static_cast<int64_t>(pairs) * (ns > 0 ? ns : 1) * (head_dim + 2) * 4;
 }
 

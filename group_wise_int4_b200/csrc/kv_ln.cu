@@ -14,18 +14,20 @@
 namespace flexq {
 namespace {
 
-// One group of GS values per GS/8 lanes; groups enumerate (tensor, sequence, head, g).
+// One group of GS values per GS/8 lanes; groups enumerate (tensor, sequence, token,
+// head, group). Token t of sequence b comes from row (b*seq + t) of the source and goes
+// to cache slot pos0 + t.
 template <int BITS, int GS>
 __global__ void __launch_bounds__(256) append_kv_kernel(const __half* __restrict__ k_new,
                                                         const __half* __restrict__ v_new,
                                                         int64_t row_stride, uint8_t* __restrict__ k_codes,
                                                         uint32_t* __restrict__ k_meta,
                                                         uint8_t* __restrict__ v_codes,
-                                                        uint32_t* __restrict__ v_meta, int batch,
-                                                        int n_heads, int head_dim, int max_seq, int pos) {
+                                                        uint32_t* __restrict__ v_meta, int batch, int seq,
+                                                        int n_heads, int head_dim, int max_seq, int pos0) {
     constexpr int L = GS / 8;
     const int gph = head_dim / GS;                              // groups per head
-    const int64_t per_tensor = static_cast<int64_t>(batch) * n_heads * gph;
+    const int64_t per_tensor = static_cast<int64_t>(batch) * seq * n_heads * gph;
     const int64_t total = 2 * per_tensor;
     const int lane = threadIdx.x & 31;
     const int sub = lane % L;
@@ -33,12 +35,14 @@ __global__ void __launch_bounds__(256) append_kv_kernel(const __half* __restrict
     const bool valid = gidx < total;
     const int64_t g = valid ? gidx : 0;
     const int which = static_cast<int>(g / per_tensor);        // 0 = key, 1 = value
-    const int64_t r = g % per_tensor;
+    int64_t r = g % per_tensor;
     const int gi = static_cast<int>(r % gph);
-    const int64_t bh = r / gph;                                 // b * n_heads + head
-    const int64_t b = bh / n_heads;
-    const int head = static_cast<int>(bh % n_heads);
-    const __half* src = (which == 0 ? k_new : v_new) + b * row_stride + head * head_dim + gi * GS + sub * 8;
+    r /= gph;
+    const int head = static_cast<int>(r % n_heads);
+    r /= n_heads;                                               // b * seq + t
+    const int t = static_cast<int>(r % seq);
+    const int64_t b = r / seq;
+    const __half* src = (which == 0 ? k_new : v_new) + r * row_stride + head * head_dim + gi * GS + sub * 8;
     uint4 v = make_uint4(0, 0, 0, 0);
     if (valid) v = *reinterpret_cast<const uint4*>(src);
     __half2 hmn, hmx;
@@ -52,7 +56,7 @@ __global__ void __launch_bounds__(256) append_kv_kernel(const __half* __restrict
     const __half s16 = group_scale16<BITS>(mn, mx);
     const float s = __half2float(s16);
     if (!valid) return;
-    const int64_t slot = bh * max_seq + pos;                    // [b][nh][max_seq]
+    const int64_t slot = (b * n_heads + head) * max_seq + pos0 + t;   // [b][nh][max_seq]
     uint8_t* codes = (which == 0 ? k_codes : v_codes) + slot * (head_dim * BITS / 8) + gi * (GS * BITS / 8);
     uint32_t* meta = (which == 0 ? k_meta : v_meta) + slot * gph + gi;
     if (BITS == 4)
@@ -138,10 +142,11 @@ __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const __half* __r
 }  // namespace
 
 int append_kv_launch(const flex_kv_cache* c, const void* k_new, const void* v_new, int64_t row_stride,
-                     int batch, int pos, cudaStream_t st) {
+                     int batch, int seq, int pos0, cudaStream_t st) {
     const int gs = c->cfg.group_size;
-    const int64_t groups = 2LL * batch * c->n_heads * (c->head_dim / gs);
+    const int64_t groups = 2LL * batch * seq * c->n_heads * (c->head_dim / gs);
     const int64_t threads = groups * (gs / 8);
+    if (threads == 0) return FLEX_OK;
     const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
     const __half* k = static_cast<const __half*>(k_new);
     const __half* v = static_cast<const __half*>(v_new);
@@ -149,9 +154,9 @@ int append_kv_launch(const flex_kv_cache* c, const void* k_new, const void* v_ne
     uint8_t* vc = static_cast<uint8_t*>(c->v_codes);
     uint32_t* km = static_cast<uint32_t*>(c->k_meta);
     uint32_t* vm = static_cast<uint32_t*>(c->v_meta);
-#define APPEND(B, G)                                                                                    \
-    append_kv_kernel<B, G><<<blocks, 256, 0, st>>>(k, v, row_stride, kc, km, vc, vm, batch, c->n_heads, \
-                                                   c->head_dim, c->max_seq, pos)
+#define APPEND(B, G)                                                                                          \
+    append_kv_kernel<B, G><<<blocks, 256, 0, st>>>(k, v, row_stride, kc, km, vc, vm, batch, seq, c->n_heads, \
+                                                   c->head_dim, c->max_seq, pos0)
     if (c->cfg.num_bits == 4) {
         if (gs == 32) APPEND(4, 32); else if (gs == 64) APPEND(4, 64); else APPEND(4, 128);
     } else {
@@ -200,7 +205,7 @@ extern "C" int flex_append_kv(const flex_kv_cache* cache, const void* k_new, con
     FLEX_REQUIRE(row_stride >= static_cast<int64_t>(cache->n_heads) * cache->head_dim, FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(row_stride % 8 == 0, FLEX_ERR_ALIGN);
     FLEX_REQUIRE(aligned16(k_new) && aligned16(v_new), FLEX_ERR_ALIGN);
-    return append_kv_launch(cache, k_new, v_new, row_stride, batch, pos, as_stream(stream));
+    return append_kv_launch(cache, k_new, v_new, row_stride, batch, 1, pos, as_stream(stream));
 }
 
 extern "C" int flex_layernorm(const void* x, const void* g, const void* b, void* y, int64_t rows, int32_t h,

@@ -1,0 +1,167 @@
+// OPT decoder layer: prefill (`mha` path) and decode step (`mha_gen` path).
+//
+// FlexGen source-reading notes, "Flex Opt": per token, layer and gpu-batch the loop
+// runs load_weight, load_cache, load_hidden, compute_layer, store_hidden, store_cache;
+// compute_layer is the pre-LayerNorm OPT block. Here everything is resident on one
+// GPU, so loading is a no-op and a layer call is the fixed launch sequence
+//
+//   LN1 -> QKV GEMM (+bias, q * d^-1/2) -> attention -> store_cache -> out-proj GEMM
+//   (+bias, +x) -> LN2 -> fc1 GEMM (+bias, ReLU) -> fc2 GEMM (+bias, +h1)
+//
+// on one stream, without host synchronisation, so a caller can capture it in a CUDA
+// graph. All intermediates live in the caller's workspace.
+#include "common.cuh"
+
+namespace flexq {
+
+int validate_cache(const flex_kv_cache* c);
+int validate_weight(const flexq_tensor* W);
+int layernorm_launch(const void* x, const void* g, const void* b, void* y, int64_t rows, int h, cudaStream_t st);
+int append_kv_launch(const flex_kv_cache* c, const void* k_new, const void* v_new, int64_t row_stride, int batch,
+                     int seq, int pos0, cudaStream_t st);
+int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new, const void* v_new,
+                       int64_t row_stride, void* o, int batch, int pos, void* ws, cudaStream_t st);
+int64_t decode_attn_ws_bound(int pairs, int head_dim);
+int prefill_attn_launch(const void* q, const void* k, const void* v, int64_t row_stride, void* o, int batch,
+                        int seq, int n_heads, int head_dim, cudaStream_t st);
+int64_t gemm_ws_bytes(int M, int N, int K, int bits);
+int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const void* residual, void* y, int M,
+                int relu, int nq, float qscale, void* ws, int64_t ws_bytes, cudaStream_t st);
+
+namespace {
+
+inline int64_t align256(int64_t v) { return (v + 255) / 256 * 256; }
+
+struct WsLayout {
+    int64_t a, qkv, o, h1, a2, f, attn, gemm, total, gemm_bytes;
+};
+
+int check_weight_shape(const flexq_tensor& W, int64_t n, int64_t k) {
+    const int rc = validate_weight(&W);
+    if (rc != FLEX_OK) return rc;
+    FLEX_REQUIRE(W.shape[0] == n && W.shape[1] == k, FLEX_ERR_SHAPE);
+    return FLEX_OK;
+}
+
+int validate_layer(const flex_layer* L) {
+    FLEX_REQUIRE(L != nullptr, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(L->h > 0 && L->n_heads > 0 && L->head_dim > 0 && L->ffn > 0, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(L->head_dim == 64 || L->head_dim == 128, FLEX_ERR_UNSUPPORTED);
+    FLEX_REQUIRE(static_cast<int64_t>(L->n_heads) * L->head_dim == L->h, FLEX_ERR_SHAPE);
+    FLEX_REQUIRE(L->h % 256 == 0 && L->ffn % 256 == 0 && L->h <= 12288, FLEX_ERR_SHAPE);
+    FLEX_REQUIRE(L->ln1_g && L->ln1_b && L->ln2_g && L->ln2_b, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(L->b_qkv && L->b_o && L->b_fc1 && L->b_fc2, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(aligned16(L->ln1_g) && aligned16(L->ln1_b) && aligned16(L->ln2_g) && aligned16(L->ln2_b) &&
+                     aligned16(L->b_qkv) && aligned16(L->b_o) && aligned16(L->b_fc1) && aligned16(L->b_fc2),
+                 FLEX_ERR_ALIGN);
+    int rc = check_weight_shape(L->w_qkv, 3LL * L->h, L->h);
+    if (rc == FLEX_OK) rc = check_weight_shape(L->w_o, L->h, L->h);
+    if (rc == FLEX_OK) rc = check_weight_shape(L->w_fc1, L->ffn, L->h);
+    if (rc == FLEX_OK) rc = check_weight_shape(L->w_fc2, L->h, L->ffn);
+    return rc;
+}
+
+WsLayout layout(const flex_layer* L, int batch, int seq) {
+    const int64_t T = static_cast<int64_t>(batch) * seq;
+    WsLayout w{};
+    int64_t off = 0;
+    w.a = off;    off += align256(T * L->h * 2);
+    w.qkv = off;  off += align256(T * 3 * L->h * 2);
+    w.o = off;    off += align256(T * L->h * 2);
+    w.h1 = off;   off += align256(T * L->h * 2);
+    w.a2 = off;   off += align256(T * L->h * 2);
+    w.f = off;    off += align256(T * L->ffn * 2);
+    w.attn = off;
+    if (seq == 1) off += align256(decode_attn_ws_bound(batch * L->n_heads, L->head_dim));
+    w.gemm = off;
+    const int M = static_cast<int>(T);
+    int64_t g = 0;
+    const int bits[4] = {L->w_qkv.cfg.num_bits, L->w_o.cfg.num_bits, L->w_fc1.cfg.num_bits, L->w_fc2.cfg.num_bits};
+    const int64_t nk[4][2] = {{3LL * L->h, L->h}, {L->h, L->h}, {L->ffn, L->h}, {L->h, L->ffn}};
+    for (int i = 0; i < 4; ++i) {
+        const int64_t b = gemm_ws_bytes(M, static_cast<int>(nk[i][0]), static_cast<int>(nk[i][1]), bits[i]);
+        if (b > g) g = b;
+    }
+    w.gemm_bytes = g;
+    off += align256(g);
+    w.total = off;
+    return w;
+}
+
+int run_layer(const flex_layer* L, const flex_kv_cache* C, const void* x_in, void* x_out, int batch, int seq, int pos,
+              void* ws, int64_t ws_bytes, cudaStream_t st) {
+    const WsLayout w = layout(L, batch, seq);
+    FLEX_REQUIRE(ws != nullptr && ws_bytes >= w.total, FLEX_ERR_WORKSPACE);
+    FLEX_REQUIRE(aligned16(ws), FLEX_ERR_ALIGN);
+    char* base = static_cast<char*>(ws);
+    void* a = base + w.a;
+    __half* qkv = reinterpret_cast<__half*>(base + w.qkv);
+    void* o = base + w.o;
+    void* h1 = base + w.h1;
+    void* a2 = base + w.a2;
+    void* f = base + w.f;
+    void* gws = base + w.gemm;
+    const int64_t T = static_cast<int64_t>(batch) * seq;
+    const int M = static_cast<int>(T);
+    const int h = L->h;
+    const float qscale = 1.0f / sqrtf(static_cast<float>(L->head_dim));
+    int rc = layernorm_launch(x_in, L->ln1_g, L->ln1_b, a, T, h, st);
+    if (rc == FLEX_OK) rc = gemm_launch(a, &L->w_qkv, L->b_qkv, nullptr, qkv, M, 0, h, qscale, gws, w.gemm_bytes, st);
+    if (rc != FLEX_OK) return rc;
+    if (seq == 1) {
+        rc = decode_attn_launch(C, qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, pos, base + w.attn, st);
+        if (rc == FLEX_OK) rc = append_kv_launch(C, qkv + h, qkv + 2 * h, 3LL * h, batch, 1, pos, st);
+    } else {
+        rc = prefill_attn_launch(qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, seq, L->n_heads, L->head_dim, st);
+        if (rc == FLEX_OK) rc = append_kv_launch(C, qkv + h, qkv + 2 * h, 3LL * h, batch, seq, 0, st);
+    }
+    if (rc == FLEX_OK) rc = gemm_launch(o, &L->w_o, L->b_o, x_in, h1, M, 0, 0, 1.f, gws, w.gemm_bytes, st);
+    if (rc == FLEX_OK) rc = layernorm_launch(h1, L->ln2_g, L->ln2_b, a2, T, h, st);
+    if (rc == FLEX_OK) rc = gemm_launch(a2, &L->w_fc1, L->b_fc1, nullptr, f, M, 1, 0, 1.f, gws, w.gemm_bytes, st);
+    if (rc == FLEX_OK) rc = gemm_launch(f, &L->w_fc2, L->b_fc2, h1, x_out, M, 0, 0, 1.f, gws, w.gemm_bytes, st);
+    return rc;
+}
+
+int check_cache_for_layer(const flex_layer* L, const flex_kv_cache* C) {
+    const int rc = validate_cache(C);
+    if (rc != FLEX_OK) return rc;
+    FLEX_REQUIRE(C->n_heads == L->n_heads && C->head_dim == L->head_dim, FLEX_ERR_SHAPE);
+    return FLEX_OK;
+}
+
+}  // namespace
+}  // namespace flexq
+
+using namespace flexq;
+
+extern "C" int64_t flex_workspace_bytes(const flex_layer* L, int32_t batch, int32_t seq) {
+    const int rc = validate_layer(L);
+    if (rc != FLEX_OK) return rc;
+    FLEX_REQUIRE(batch > 0 && seq > 0, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(static_cast<int64_t>(batch) * seq < (1LL << 31), FLEX_ERR_SHAPE);
+    return layout(L, batch, seq).total;
+}
+
+extern "C" int flex_prefill_layer(const flex_layer* L, const flex_kv_cache* cache, const void* x_in, void* x_out,
+                                  int32_t batch, int32_t seq, void* ws, int64_t ws_bytes, void* stream) {
+    int rc = validate_layer(L);
+    if (rc == FLEX_OK) rc = check_cache_for_layer(L, cache);
+    if (rc != FLEX_OK) return rc;
+    FLEX_REQUIRE(x_in && x_out && x_in != x_out, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(aligned16(x_in) && aligned16(x_out), FLEX_ERR_ALIGN);
+    FLEX_REQUIRE(batch > 0 && batch == cache->batch, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(seq > 0 && seq <= cache->max_seq, FLEX_ERR_SHAPE);
+    return run_layer(L, cache, x_in, x_out, batch, seq, 0, ws, ws_bytes, as_stream(stream));
+}
+
+extern "C" int flex_decode_layer(const flex_layer* L, const flex_kv_cache* cache, const void* x_in, void* x_out,
+                                 int32_t batch, int32_t pos, void* ws, int64_t ws_bytes, void* stream) {
+    int rc = validate_layer(L);
+    if (rc == FLEX_OK) rc = check_cache_for_layer(L, cache);
+    if (rc != FLEX_OK) return rc;
+    FLEX_REQUIRE(x_in && x_out && x_in != x_out, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(aligned16(x_in) && aligned16(x_out), FLEX_ERR_ALIGN);
+    FLEX_REQUIRE(batch > 0 && batch <= cache->batch, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(pos >= 0 && pos < cache->max_seq, FLEX_ERR_SHAPE);
+    return run_layer(L, cache, x_in, x_out, batch, 1, pos, ws, ws_bytes, as_stream(stream));
+}

@@ -1,0 +1,123 @@
+"""Parity of the tcgen05 dequant-fused GEMM (flex_dequant_gemm, through the C ABI)
+with the oracle: y = epilogue(x W^T + b) with W^ the oracle's dequantised weight,
+float64 products. Tolerance: the method's max|err| <= 1e-2 max|ref| + 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+import group_wise_int4_b200 as fq
+import synth
+from oracle import codec as oc
+from _helpers import assert_layer_close, to_np, sync_status
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_gemm(x, w16, bias, residual, epi, bits, rows=None):
+    w = w16 if rows is None else w16[rows]
+    c, m = oc.compress(np.ascontiguousarray(w), bits, 64, 1)
+    wd = oc.decompress(c, m, w.shape, bits, 64, 1).astype(np.float64)
+    y = x.astype(np.float64) @ wd.T
+    if bias is not None:
+        y += (bias if rows is None else bias[rows]).astype(np.float64)
+    if epi == fq.FLEX_EPI_RELU:
+        y = np.maximum(y, 0)
+    if epi == fq.FLEX_EPI_RESIDUAL:
+        y += (residual if rows is None else residual[:, rows]).astype(np.float64)
+    return y
+
+
+def _run(M, N, K, epi, bits=4, seed=0, with_bias=True):
+    x = synth.activations((M, K), seed)
+    w = synth.normal_f16((N, K), seed + 1, 0.02)
+    b = synth.normal_f16((N,), seed + 2, 0.02) if with_bias else None
+    r = synth.activations((M, N), seed + 3) if epi == fq.FLEX_EPI_RESIDUAL else None
+    W = fq.CompressedWeight(w.cuda(), bits, 64)
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    ws = torch.zeros(max(16, fq.flex_gemm_ws_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
+    fq.flex_dequant_gemm(x.cuda(), W, None if b is None else b.cuda(), None if r is None else r.cuda(), y, M, epi, ws)
+    sync_status()
+    return x.numpy(), w.numpy(), None if b is None else b.numpy(), None if r is None else r.numpy(), y, ws
+
+
+CASES = [(1, 256, 256), (4, 256, 512), (17, 384, 768), (32, 512, 2048), (48, 256, 256), (64, 768, 512),
+         (144, 512, 1024), (250, 256, 512), (256, 384, 256), (300, 256, 512), (1000, 384, 768)]
+
+
+@pytest.mark.parametrize("M,N,K", CASES)
+def test_gemm_bias(M, N, K):
+    x, w, b, _, y, _ = _run(M, N, K, fq.FLEX_EPI_NONE, seed=M)
+    assert_layer_close(y, _oracle_gemm(x, w, b, None, fq.FLEX_EPI_NONE, 4), f"gemm {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(4, 256, 512), (144, 512, 1024), (700, 256, 256)])
+def test_gemm_relu(M, N, K):
+    x, w, b, _, y, _ = _run(M, N, K, fq.FLEX_EPI_RELU, seed=M + 7)
+    ref = _oracle_gemm(x, w, b, None, fq.FLEX_EPI_RELU, 4)
+    assert_layer_close(y, ref, "relu")
+    assert float(y.min()) >= 0
+
+
+@pytest.mark.parametrize("M,N,K", [(5, 256, 768), (144, 384, 512), (513, 256, 256)])
+def test_gemm_residual(M, N, K):
+    x, w, b, r, y, _ = _run(M, N, K, fq.FLEX_EPI_RESIDUAL, seed=M + 9)
+    assert_layer_close(y, _oracle_gemm(x, w, b, r, fq.FLEX_EPI_RESIDUAL, 4), "residual")
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 256, 512), (200, 256, 768)])
+def test_gemm_8bit_no_bias(M, N, K):
+    x, w, _, _, y, _ = _run(M, N, K, fq.FLEX_EPI_NONE, bits=8, seed=M + 11, with_bias=False)
+    assert_layer_close(y, _oracle_gemm(x, w, None, None, fq.FLEX_EPI_NONE, 8), "8-bit")
+
+
+def test_gemm_repeatable_and_workspace_left_clean():
+    """Split-K reduces in a fixed order: two calls give identical bits; the
+    workspace's tickets are back to zero after each call."""
+    M, N, K = 16, 512, 4096
+    x, w, b, _, y1, ws = _run(M, N, K, fq.FLEX_EPI_NONE, seed=5)
+    W = fq.CompressedWeight(torch.from_numpy(w).cuda(), 4, 64)
+    y2 = torch.empty_like(y1)
+    fq.flex_dequant_gemm(torch.from_numpy(x).cuda(), W, torch.from_numpy(b).cuda(), None, y2, M, 0, ws)
+    sync_status()
+    assert torch.equal(y1, y2)
+    nt = N // 128
+    assert int(ws[: 4 * nt].view(torch.int32).abs().sum()) == 0
+
+
+@pytest.mark.parametrize("name,M,N,K", [("opt-1.3b qkv decode", 32, 6144, 2048),
+                                        ("opt-1.3b fc2 decode", 32, 2048, 8192),
+                                        ("opt-30b fc1 gpu-batch", 48, 28672, 7168),
+                                        ("opt-175b fc1 decode", 144, 49152, 12288),
+                                        ("opt-1.3b qkv prefill", 16384, 6144, 2048)])
+def test_gemm_full_size_sampled(name, M, N, K):
+    """Full-size shapes in the launch configuration the layer uses; the oracle checks
+    sampled output features (all tokens) - it needs only those weight rows."""
+    x = synth.activations((M, K), 40, device="cuda")
+    w = synth.normal_f16((N, K), 41, 0.02, device="cuda")
+    b = synth.normal_f16((N,), 42, 0.02, device="cuda")
+    W = fq.CompressedWeight(w, 4, 64)
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    ws = torch.zeros(max(16, fq.flex_gemm_ws_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
+    fq.flex_dequant_gemm(x, W, b, None, y, M, 0, ws)
+    sync_status()
+    rng = np.random.default_rng(N)
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 1], rng.integers(0, N, 24)]))
+    mrows = np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, 64)])) if M > 256 else np.arange(M)
+    xs = to_np(x[torch.from_numpy(mrows).cuda()])
+    ref = _oracle_gemm(xs, to_np(w), to_np(b), None, 0, 4, rows=rows)
+    got = y[torch.from_numpy(mrows).cuda()][:, torch.from_numpy(rows).cuda()]
+    assert_layer_close(got, ref, name)
+    assert bool(torch.isfinite(y).all())
+
+
+def test_gemm_bad_args():
+    w = torch.zeros((256, 512), dtype=torch.float16, device="cuda")
+    W = fq.CompressedWeight(w)
+    y = torch.empty((4, 256), dtype=torch.float16, device="cuda")
+    x = torch.zeros((4, 512), dtype=torch.float16, device="cuda")
+    with pytest.raises(fq.FlexError) as e:
+        fq.flex_dequant_gemm(x, W, None, None, y, 4, fq.FLEX_EPI_NONE, None)
+    assert e.value.code == fq.FLEX_ERR_WORKSPACE
+    with pytest.raises(fq.FlexError) as e:
+        fq.flex_dequant_gemm(x, W, None, None, y, 4, fq.FLEX_EPI_RESIDUAL, None)
+    assert e.value.code == fq.FLEX_ERR_INVALID_ARG

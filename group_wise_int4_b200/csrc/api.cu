@@ -4,7 +4,9 @@
 // variable whose address is looked up once per device. Kernels with bounded waits
 // record FLEX_ERR_TIMEOUT there instead of trapping; flex_get_status reads and clears
 // it.
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 
@@ -24,6 +26,17 @@ int current_device() {
     return dev < kMaxDevices ? dev : -1;
 }
 }  // namespace
+
+bool smem_attr_needed(const void* kernel, int bytes) {
+    static std::map<std::pair<const void*, int>, int> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(g_mu);
+    int& have = done[std::make_pair(kernel, dev)];
+    if (have >= bytes) return false;
+    have = bytes;
+    return true;
+}
 
 int sm_count() {
     const int dev = current_device();

@@ -1,10 +1,10 @@
 // Attention of the OPT layer.
 //
-// Decode (`mha_gen`, FlexGen source-reading notes, "Pytorch Backend"): one new token per
+// Decode (`mha_gen`, the source-notes page «FlexGen» (PtirisNote), "Pytorch Backend"): one new token per
 // sequence attends to the compressed cache slots [0, pos) - written by earlier
 // store_cache calls - and to its own fresh key/value (the loop runs load_cache,
 // compute_layer, store_cache, so the current token's key/value are not in the cache
-// yet). The int4 cache (FlexGen source walkthrough, section 6.3: 4 bits, group 64
+// yet). The int4 cache (the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南», section 6.3: 4 bits, group 64
 // along the head dimension) is streamed once and dequantised in registers; the sum
 // over a group is factored as  sum_i q_i * (c_i*step + min) = step*sum_i q_i c_i +
 // min*sum_i q_i,  and likewise for the value side, so each code costs one extract and
@@ -24,161 +24,6 @@ namespace flexq {
 namespace {
 
 constexpr int DA_THREADS = 128;
-
-// ---------------------------------------------------------------------------------
-// decode attention, split-KV partials
-template <int D, int BITS, int GS>
-__global__ void __launch_bounds__(DA_THREADS) decode_attn_split_kernel(
-    const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
-    const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
-    const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
-    float* __restrict__ part) {
-    constexpr int KB = D * BITS / 8;        // code bytes per key
-    constexpr int TPK = KB / 4;             // threads per key (one u32 of codes each)
-    constexpr int EPT = 32 / BITS;          // dims per thread
-    constexpr int KPI = DA_THREADS / TPK;   // keys per iteration
-    constexpr int GPK = D / GS;             // groups per key
-    const int pair = blockIdx.x;            // b * n_heads + head
-    const int split = blockIdx.y;
-    const int nsplit = gridDim.y;
-    const int b = pair / n_heads, head = pair % n_heads;
-    const int tid = threadIdx.x;
-    const int kl = tid / TPK, wl = tid % TPK;
-    const int d0 = wl * EPT;
-    const int grp = d0 / GS;
-
-    float qv[EPT];
-    float qsum = 0.f;
-    {
-        const __half* qp = q + static_cast<int64_t>(b) * row_stride + head * D + d0;
-#pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            qv[e] = __half2float(qp[e]);
-            qsum += qv[e];
-        }
-    }
-    const int j0 = split * chunk;
-    const int j1 = min(pos, j0 + chunk);
-    const int64_t slot0 = static_cast<int64_t>(pair) * max_seq;
-
-    float m = -FLT_MAX, l = 0.f, U = 0.f;
-    float acc[EPT];
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) acc[e] = 0.f;
-
-    // the trip count is uniform across the CTA: lanes past the end of the split load
-    // nothing and skip the update, but still take part in the shuffles
-    for (int jb = j0; jb < j1; jb += KPI) {
-        const int j = jb + kl;
-        const bool valid = j < j1;
-        const int64_t slot = slot0 + (valid ? j : j0);
-        const uint32_t kw = __ldg(reinterpret_cast<const uint32_t*>(k_codes + slot * KB) + wl);
-        const uint32_t vw = __ldg(reinterpret_cast<const uint32_t*>(v_codes + slot * KB) + wl);
-        const uint32_t km = __ldg(k_meta + slot * GPK + grp);
-        const uint32_t vm = __ldg(v_meta + slot * GPK + grp);
-        float dot = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            const uint32_t c = (kw >> (BITS * e)) & ((1u << BITS) - 1u);
-            dot = fmaf(qv[e], static_cast<float>(c), dot);
-        }
-        const float kstep = group_step(__ushort_as_half(static_cast<unsigned short>(km >> 16)));
-        const float kmn = h2f_lo(km);
-        float s = (kstep == 0.f) ? kmn * qsum : fmaf(kstep, dot, kmn * qsum);
-#pragma unroll
-        for (int off = TPK / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (!valid) continue;
-        if (s > m) {
-            const float alpha = __expf(m - s);
-            m = s;
-            l *= alpha;
-            U *= alpha;
-#pragma unroll
-            for (int e = 0; e < EPT; ++e) acc[e] *= alpha;
-        }
-        const float p = __expf(s - m);
-        l += p;
-        const float vstep = group_step(__ushort_as_half(static_cast<unsigned short>(vm >> 16)));
-        const float vmn = h2f_lo(vm);
-        const float w = p * vstep;
-        U = fmaf(p, vmn, U);
-#pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            const uint32_t c = (vw >> (BITS * e)) & ((1u << BITS) - 1u);
-            acc[e] = fmaf(w, static_cast<float>(c), acc[e]);
-        }
-    }
-
-    // merge the KPI key lanes of this CTA
-    __shared__ float sm_m[KPI], sm_l[KPI];
-    __shared__ float sm_o[KPI][D];
-    if (wl == 0) {
-        sm_m[kl] = m;
-        sm_l[kl] = l;
-    }
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) sm_o[kl][d0 + e] = acc[e] + U;
-    __syncthreads();
-    float M = -FLT_MAX;
-#pragma unroll
-    for (int i = 0; i < KPI; ++i) M = fmaxf(M, sm_m[i]);
-    float* out = part + (static_cast<int64_t>(pair) * nsplit + split) * (D + 2);
-    for (int d = tid; d < D; d += DA_THREADS) {
-        float o = 0.f;
-#pragma unroll
-        for (int i = 0; i < KPI; ++i) {
-            const float f = sm_l[i] > 0.f ? __expf(sm_m[i] - M) : 0.f;
-            o = fmaf(f, sm_o[i][d], o);
-        }
-        out[2 + d] = o;
-    }
-    if (tid == 0) {
-        float L = 0.f;
-#pragma unroll
-        for (int i = 0; i < KPI; ++i) L += sm_l[i] > 0.f ? __expf(sm_m[i] - M) * sm_l[i] : 0.f;
-        out[0] = M;
-        out[1] = L;
-    }
-}
-
-// combine the split partials with the fresh key/value of the current token
-template <int D>
-__global__ void __launch_bounds__(D) decode_attn_combine_kernel(const __half* __restrict__ q,
-                                                                const __half* __restrict__ k_new,
-                                                                const __half* __restrict__ v_new,
-                                                                int64_t row_stride, int n_heads,
-                                                                int nsplit,
-                                                                const float* __restrict__ part,
-                                                                __half* __restrict__ o) {
-    const int pair = blockIdx.x;
-    const int b = pair / n_heads, head = pair % n_heads;
-    const int d = threadIdx.x;
-    const int64_t off = static_cast<int64_t>(b) * row_stride + head * D + d;
-    float s = __half2float(q[off]) * __half2float(k_new[off]);
-#pragma unroll
-    for (int w = 16; w > 0; w >>= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
-    __shared__ float red[D / 32];
-    if ((d & 31) == 0) red[d >> 5] = s;
-    __syncthreads();
-    float snew = 0.f;
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) snew += red[i];
-    const float* pp = part + static_cast<int64_t>(pair) * nsplit * (D + 2);
-    float M = snew;
-    for (int i = 0; i < nsplit; ++i)
-        if (pp[i * (D + 2) + 1] > 0.f) M = fmaxf(M, pp[i * (D + 2)]);
-    const float fn = __expf(snew - M);
-    float L = fn;
-    float acc = fn * __half2float(v_new[off]);
-    for (int i = 0; i < nsplit; ++i) {
-        const float* p = pp + i * (D + 2);
-        if (!(p[1] > 0.f)) continue;
-        const float f = __expf(p[0] - M);
-        L = fmaf(f, p[1], L);
-        acc = fmaf(f, p[2 + d], acc);
-    }
-    o[static_cast<int64_t>(b) * n_heads * D + head * D + d] = __float2half_rn(acc / L);
-}
 
 // ---------------------------------------------------------------------------------
 // prefill attention (causal), mma.sync m16n8k16
@@ -220,6 +65,772 @@ __device__ __forceinline__ uint32_t pack_f2h2(float lo, float hi) {
     return pack_half2_bits(__float2half_rn(lo), __float2half_rn(hi));
 }
 
+// ---------------------------------------------------------------------------------
+// decode attention, split-KV partials.
+//
+// A thread owns 16 bytes of every key it touches (32 dims at 4 bits, 16 at 8 bits);
+// TPK = key bytes / 16 threads share a key. Each CTA iteration covers DA_U keys per
+// thread: all their code and metadata loads are issued first (memory-level
+// parallelism), then the scores, one online-softmax update for the block, and the
+// value accumulation.
+constexpr int DA_U = 8;
+
+// Exact integer -> float of a code: place it in the mantissa of 2^23 and subtract 2^23
+// (an integer-pipe OR and one fp32 add, instead of the slower conversion unit).
+__device__ __forceinline__ float code_f(uint32_t w, int shift, uint32_t mask) {
+    return __int_as_float(0x4B000000u | ((w >> shift) & mask)) - 8388608.0f;
+}
+
+template <int D, int BITS, int GS>
+__global__ void __launch_bounds__(DA_THREADS) decode_attn_split_kernel(
+    const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
+    const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
+    const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
+    float* __restrict__ part) {
+    constexpr int KB = D * BITS / 8;        // code bytes per key
+    constexpr int TPK = KB / 16;            // threads per key (16 bytes each)
+    constexpr int EPT = 128 / BITS;         // dims per thread
+    constexpr int KPI = DA_THREADS / TPK;   // keys per CTA and unroll step
+    constexpr int GPK = D / GS;             // groups per key
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    pdl_wait();
+    pdl_trigger();
+    const int pair = blockIdx.x;            // b * n_heads + head
+    const int split = blockIdx.y;
+    const int nsplit = gridDim.y;
+    const int b = pair / n_heads, head = pair % n_heads;
+    const int tid = threadIdx.x;
+    const int kl = tid / TPK, wl = tid % TPK;
+    const int d0 = wl * EPT;
+    const int grp = d0 / GS;
+
+    float qv[EPT];
+    float qsum = 0.f;
+    {
+        const uint4* qp = reinterpret_cast<const uint4*>(q + static_cast<int64_t>(b) * row_stride + head * D + d0);
+#pragma unroll
+        for (int v = 0; v < EPT / 8; ++v) {
+            const uint4 w = qp[v];
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                qv[8 * v + 2 * k] = h2f_lo(ww[k]);
+                qv[8 * v + 2 * k + 1] = h2f_hi(ww[k]);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) qsum += qv[e];
+    }
+    const int j0 = split * chunk;
+    const int j1 = min(pos, j0 + chunk);
+    const int64_t slot0 = static_cast<int64_t>(pair) * max_seq;
+
+    float m = -FLT_MAX, l = 0.f, U = 0.f;
+    float acc[EPT];
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) acc[e] = 0.f;
+
+    // the trip count is uniform across the CTA: lanes past the end of the split load
+    // slot j0 instead and skip the update, but still take part in the shuffles
+    for (int jb = j0; jb < j1; jb += DA_U * KPI) {
+        uint4 kc[DA_U], vc[DA_U];
+        uint32_t km[DA_U], vm[DA_U];
+#pragma unroll
+        for (int u = 0; u < DA_U; ++u) {
+            const int j = jb + u * KPI + kl;
+            const int64_t slot = slot0 + (j < j1 ? j : j0);
+            kc[u] = __ldg(reinterpret_cast<const uint4*>(k_codes + slot * KB) + wl);
+            vc[u] = __ldg(reinterpret_cast<const uint4*>(v_codes + slot * KB) + wl);
+            km[u] = __ldg(k_meta + slot * GPK + grp);
+            vm[u] = __ldg(v_meta + slot * GPK + grp);
+        }
+        float s[DA_U];
+        float bmax = -FLT_MAX;
+#pragma unroll
+        for (int u = 0; u < DA_U; ++u) {
+            const uint32_t w[4] = {kc[u].x, kc[u].y, kc[u].z, kc[u].w};
+            float dot = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) dot = fmaf(qv[e], code_f(w[e * BITS / 32], (e * BITS) % 32, MASK), dot);
+            const float kstep = group_step(__ushort_as_half(static_cast<unsigned short>(km[u] >> 16)));
+            const float kmn = h2f_lo(km[u]);
+            float su = fmaf(kstep, dot, kmn * qsum);
+#pragma unroll
+            for (int off = TPK / 2; off > 0; off >>= 1) su += __shfl_xor_sync(0xffffffffu, su, off);
+            const int j = jb + u * KPI + kl;
+            s[u] = j < j1 ? su : -FLT_MAX;
+            bmax = fmaxf(bmax, s[u]);
+        }
+        if (bmax > m) {
+            const float alpha = __expf(m - bmax);
+            m = bmax;
+            l *= alpha;
+            U *= alpha;
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) acc[e] *= alpha;
+        }
+#pragma unroll
+        for (int u = 0; u < DA_U; ++u) {
+            if (s[u] == -FLT_MAX) continue;
+            const float p = __expf(s[u] - m);
+            l += p;
+            const float vstep = group_step(__ushort_as_half(static_cast<unsigned short>(vm[u] >> 16)));
+            const float w = p * vstep;
+            U = fmaf(p, h2f_lo(vm[u]), U);
+            const uint32_t vw[4] = {vc[u].x, vc[u].y, vc[u].z, vc[u].w};
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) acc[e] = fmaf(w, code_f(vw[e * BITS / 32], (e * BITS) % 32, MASK), acc[e]);
+        }
+    }
+
+    // merge the KPI key lanes of this CTA
+    __shared__ float sm_m[KPI], sm_l[KPI];
+    __shared__ float sm_o[KPI][D + 1];
+    if (wl == 0) {
+        sm_m[kl] = m;
+        sm_l[kl] = l;
+    }
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) sm_o[kl][d0 + e] = acc[e] + U;
+    __syncthreads();
+    float M = -FLT_MAX;
+    for (int i = 0; i < KPI; ++i) M = fmaxf(M, sm_m[i]);
+    float* out = part + (static_cast<int64_t>(pair) * nsplit + split) * (D + 2);
+    for (int d = tid; d < D; d += DA_THREADS) {
+        float o = 0.f;
+        for (int i = 0; i < KPI; ++i) {
+            const float f = sm_l[i] > 0.f ? __expf(sm_m[i] - M) : 0.f;
+            o = fmaf(f, sm_o[i][d], o);
+        }
+        out[2 + d] = o;
+    }
+    if (tid == 0) {
+        float L = 0.f;
+        for (int i = 0; i < KPI; ++i) L += sm_l[i] > 0.f ? __expf(sm_m[i] - M) * sm_l[i] : 0.f;
+        out[0] = M;
+        out[1] = L;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// decode attention on the tensor cores (4-bit cache), mma.sync m16n8k16, fp32 accumulate.
+//
+// Each warp walks 16-key tiles of its (sequence, head) range. Codes enter the MMA raw,
+// as the exact fp16 values 1024 + c (one LOP3 per two codes); the dequantisation is
+// applied to the small results instead of to every element:
+//   scores: the 8 columns of the QK MMA are the key groups (B[dim][n] = q[dim] when
+//           dim is in group n, else 0), so one pass gives S[j][n] = sum_{dim in n}
+//           (1024 + c_j[dim]) q[dim] and
+//           s_j = sum_n step_jn (S[j][n] - 1024 Q_n) + min_jn Q_n,  Q_n = sum_{dim in n} q;
+//   values: B[j][n] = w_jn = p_j step_jn (fp16), so D'[dim][n] = 1024 W_n +
+//           sum_j w_jn c_j[dim] and o[dim] = D'[dim][g] - 1024 W_g + sum_j p_j min_jg
+//           with g the group of dim and W_g = sum_j w_jg.
+// Both MMAs are free to permute the K dimension (dims for QK, keys for PV) as long as A
+// and B agree; the layouts below are chosen so that every thread loads contiguous code
+// bytes and builds its fragments with PRMT / LOP3 only.
+__device__ __forceinline__ uint32_t nib_pair(uint32_t x) {
+    // (x & 0x000F000F) | 0x64006400: two 4-bit codes as the fp16 pair (1024 + lo, 1024 + hi)
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(0x000F000Fu), "r"(0x64006400u));
+    return r;
+}
+__device__ __forceinline__ uint32_t byte_pair(uint32_t a, uint32_t b, uint32_t byte) {
+    // byte `byte` of a into bits 0..7, byte `byte` of b into bits 16..23
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(byte | ((4u + byte) << 8)));
+    return r;
+}
+__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
+    return pack_half2_bits(__float2half_rn(lo), __float2half_rn(hi));
+}
+// a[n] for a runtime n without dynamic register indexing (which would go to local memory)
+template <int N>
+__device__ __forceinline__ float pick(const float (&a)[N], int n) {
+    float r = a[0];
+#pragma unroll
+    for (int i = 1; i < N; ++i) r = (n == i) ? a[i] : r;
+    return r;
+}
+
+template <int D>
+struct MmaTile {                            // one 16-key tile's loads for one thread
+    uint32_t kg[D / 32], kg8[D / 32];       // QK side: keys g, g+8, this thread's D/4 dims
+    uint32_t kmg[2], kmg8[2];               // K metadata of keys g, g+8, groups 2t, 2t+1
+    uint32_t vw[4][D / 64 > 0 ? D / 64 : 1];// PV side: keys 2t, 2t+1, 2t+8, 2t+9, dims D/8*g..
+    uint32_t vmv[4];                        // V metadata of those keys, group g
+};
+
+template <int D, int GS>
+__device__ __forceinline__ void mma_tile_load(MmaTile<D>& T, int jt, int j0, int j1, int64_t slot0, int g, int t,
+                                              const uint8_t* __restrict__ k_codes, const uint32_t* __restrict__ k_meta,
+                                              const uint8_t* __restrict__ v_codes,
+                                              const uint32_t* __restrict__ v_meta) {
+    constexpr int G = D / GS, KB = D / 2, KW = D / 32, VW = D / 64;
+    auto slot_of = [&](int jj) { return slot0 + (jj < j1 ? jj : j0); };   // past the range: a valid slot
+    const int64_t sg = slot_of(jt + g), sg8 = slot_of(jt + g + 8);
+    const uint32_t* pg = reinterpret_cast<const uint32_t*>(k_codes + sg * KB) + t * KW;
+    const uint32_t* pg8 = reinterpret_cast<const uint32_t*>(k_codes + sg8 * KB) + t * KW;
+    if (KW == 4) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(pg));
+        const uint4 c = __ldg(reinterpret_cast<const uint4*>(pg8));
+        T.kg[0] = a.x; T.kg[1 % KW] = a.y; T.kg[2 % KW] = a.z; T.kg[3 % KW] = a.w;
+        T.kg8[0] = c.x; T.kg8[1 % KW] = c.y; T.kg8[2 % KW] = c.z; T.kg8[3 % KW] = c.w;
+    } else {
+        const uint2 a = __ldg(reinterpret_cast<const uint2*>(pg));
+        const uint2 c = __ldg(reinterpret_cast<const uint2*>(pg8));
+        T.kg[0] = a.x; T.kg[1 % KW] = a.y;
+        T.kg8[0] = c.x; T.kg8[1 % KW] = c.y;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const bool has = 2 * t + u < G;
+        T.kmg[u] = has ? __ldg(k_meta + sg * G + 2 * t + u) : 0u;
+        T.kmg8[u] = has ? __ldg(k_meta + sg8 * G + 2 * t + u) : 0u;
+    }
+    const int kv[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int64_t vs = slot_of(jt + kv[u]);
+        const uint32_t* pv = reinterpret_cast<const uint32_t*>(v_codes + vs * KB) + g * VW;
+        if (VW == 2) {
+            const uint2 a = __ldg(reinterpret_cast<const uint2*>(pv));
+            T.vw[u][0] = a.x;
+            T.vw[u][1 % (VW > 0 ? VW : 1)] = a.y;
+        } else {
+            T.vw[u][0] = __ldg(pv);
+        }
+        T.vmv[u] = (g < G) ? __ldg(v_meta + vs * G + g) : 0u;
+    }
+}
+
+template <int D, int GS>
+__global__ void __launch_bounds__(DA_THREADS) decode_attn_mma_kernel(
+    const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
+    const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
+    const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
+    float* __restrict__ part) {
+    constexpr int G = D / GS;              // groups per key: 1, 2 or 4
+    constexpr int NKS = D / 16;            // QK k-steps
+    constexpr int NMT = D / 16;            // PV M-tiles
+    constexpr int NW = DA_THREADS / 32;
+    constexpr float C1024 = 1024.f;
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int pair = blockIdx.x, split = blockIdx.y, nsplit = gridDim.y;
+    const int b = pair / n_heads, head = pair % n_heads;
+    const int64_t slot0 = static_cast<int64_t>(pair) * max_seq;
+    const int j0 = split * chunk;
+    const int j1 = min(pos, j0 + chunk);
+
+    // ---- query: per-group sums and the masked B operand of the QK MMA
+    const __half* qp = q + static_cast<int64_t>(b) * row_stride + head * D;
+    float Qg[G];
+#pragma unroll
+    for (int n = 0; n < G; ++n) Qg[n] = 0.f;
+#pragma unroll
+    for (int v = 0; v < D / 8; ++v) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(qp) + v);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) Qg[(8 * v) / GS] += h2f_lo(ww[k]) + h2f_hi(ww[k]);
+    }
+    // thread t's QK dims: [t*D/4, (t+1)*D/4); k-step ks uses word ks/2, nibbles e0, e0+1
+    // (e0 = 2*(ks%2)); slot pair (2t, 2t+1) <- dims (base, base+4), (2t+8, 2t+9) <- (base+1, base+5)
+    const int tgrp = (t * (D / 4)) / GS;
+    uint32_t bq[NKS][2];
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks) {
+        const int base = t * (D / 4) + 8 * (ks / 2) + 2 * (ks % 2);
+        if (g == tgrp) {
+            bq[ks][0] = pack_half2_bits(qp[base], qp[base + 4]);
+            bq[ks][1] = pack_half2_bits(qp[base + 1], qp[base + 5]);
+        } else {
+            bq[ks][0] = bq[ks][1] = 0u;
+        }
+    }
+
+    float m = -FLT_MAX;                    // running max (warp-uniform)
+    float lsum = 0.f;                      // lanes t == 0: their keys' share of the running sum
+    float Wrun = 0.f, Urun = 0.f;          // quads g < G: group g's sum_j w_jg, sum_j p_j min_jg
+    float oacc[NMT][4];
+#pragma unroll
+    for (int i = 0; i < NMT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+
+    const int ntiles = (j1 - j0 + 15) / 16;
+    MmaTile<D> cur, nxt;
+    if (warp < ntiles) mma_tile_load<D, GS>(cur, j0 + warp * 16, j0, j1, slot0, g, t, k_codes, k_meta, v_codes, v_meta);
+    for (int tile = warp; tile < ntiles; tile += NW) {
+        const int jt = j0 + tile * 16;
+        // prefetch the warp's next tile while this one is computed
+        if (tile + NW < ntiles)
+            mma_tile_load<D, GS>(nxt, jt + NW * 16, j0, j1, slot0, g, t, k_codes, k_meta, v_codes, v_meta);
+
+        // ---- scores: S[key][group] on the tensor cores
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < NKS; ++ks) {
+            const int w = ks / 2, e0 = 2 * (ks % 2);
+            const uint32_t a[4] = {nib_pair(cur.kg[w] >> (4 * e0)), nib_pair(cur.kg8[w] >> (4 * e0)),
+                                   nib_pair(cur.kg[w] >> (4 * e0 + 4)), nib_pair(cur.kg8[w] >> (4 * e0 + 4))};
+            mma16816(sacc, a, bq[ks][0], bq[ks][1]);
+        }
+        // lane (g, t) holds columns 2t, 2t+1 of keys g (sacc[0..1]) and g+8 (sacc[2..3])
+        float sg_part = 0.f, sg8_part = 0.f;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int n = 2 * t + u;
+            if (n < G) {
+                const float Qn = pick(Qg, n);
+                const float st0 = group_step(__ushort_as_half(static_cast<unsigned short>(cur.kmg[u] >> 16)));
+                const float st1 = group_step(__ushort_as_half(static_cast<unsigned short>(cur.kmg8[u] >> 16)));
+                sg_part += fmaf(st0, sacc[u] - C1024 * Qn, h2f_lo(cur.kmg[u]) * Qn);
+                sg8_part += fmaf(st1, sacc[2 + u] - C1024 * Qn, h2f_lo(cur.kmg8[u]) * Qn);
+            }
+        }
+        if (G == 4) {
+            sg_part += __shfl_xor_sync(0xffffffffu, sg_part, 1);
+            sg8_part += __shfl_xor_sync(0xffffffffu, sg8_part, 1);
+        }
+        // every lane of quad g takes the scores of keys g, g+8 from the quad's lane t = 0
+        sg_part = __shfl_sync(0xffffffffu, sg_part, lane & ~3);
+        sg8_part = __shfl_sync(0xffffffffu, sg8_part, lane & ~3);
+        const float s_lo = (jt + g < j1) ? sg_part : -FLT_MAX;
+        const float s_hi = (jt + g + 8 < j1) ? sg8_part : -FLT_MAX;
+        float tmax = fmaxf(s_lo, s_hi);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
+        if (tmax > m) {                    // warp-uniform
+            const float alpha = __expf(m - tmax);
+            m = tmax;
+            lsum *= alpha;
+            Wrun *= alpha;
+            Urun *= alpha;
+#pragma unroll
+            for (int i = 0; i < NMT; ++i) {
+                oacc[i][0] *= alpha;
+                oacc[i][1] *= alpha;
+                oacc[i][2] *= alpha;
+                oacc[i][3] *= alpha;
+            }
+        }
+        const float p_lo = s_lo == -FLT_MAX ? 0.f : __expf(s_lo - m);
+        const float p_hi = s_hi == -FLT_MAX ? 0.f : __expf(s_hi - m);
+        if (t == 0) lsum += p_lo + p_hi;
+        // ---- PV: B[key][n] = p_key * step_key,n in lanes (n, t'): keys 2t', 2t'+1, 2t'+8, 2t'+9
+        const float pA = __shfl_sync(0xffffffffu, p_lo, 8 * t);        // key 2t
+        const float pAh = __shfl_sync(0xffffffffu, p_hi, 8 * t);       // key 2t+8
+        const float pB = __shfl_sync(0xffffffffu, p_lo, 8 * t + 4);    // key 2t+1
+        const float pBh = __shfl_sync(0xffffffffu, p_hi, 8 * t + 4);   // key 2t+9
+        uint32_t bv0 = 0u, bv1 = 0u;
+        float wt = 0.f, ut = 0.f;
+        if (g < G) {
+            const float pk[4] = {pA, pB, pAh, pBh};
+            float wv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float stp = group_step(__ushort_as_half(static_cast<unsigned short>(cur.vmv[u] >> 16)));
+                wv[u] = __half2float(__float2half_rn(pk[u] * stp));
+                wt += wv[u];
+                ut = fmaf(pk[u], h2f_lo(cur.vmv[u]), ut);
+            }
+            bv0 = half2_bits(wv[0], wv[1]);
+            bv1 = half2_bits(wv[2], wv[3]);
+        }
+        wt += __shfl_xor_sync(0xffffffffu, wt, 1);
+        wt += __shfl_xor_sync(0xffffffffu, wt, 2);
+        ut += __shfl_xor_sync(0xffffffffu, ut, 1);
+        ut += __shfl_xor_sync(0xffffffffu, ut, 2);
+        Wrun += wt;
+        Urun += ut;
+#pragma unroll
+        for (int mt = 0; mt < NMT; ++mt) {
+            const int wi = mt / 4, by = mt % 4;
+            const uint32_t x1 = byte_pair(cur.vw[0][wi], cur.vw[1][wi], by);
+            const uint32_t x2 = byte_pair(cur.vw[2][wi], cur.vw[3][wi], by);
+            const uint32_t a[4] = {nib_pair(x1), nib_pair(x1 >> 4), nib_pair(x2), nib_pair(x2 >> 4)};
+            mma16816(oacc[mt], a, bv0, bv1);
+        }
+        cur = nxt;
+    }
+
+    // ---- warp result: o[dim] = D'[dim][grp] - 1024 W_grp + U_grp, l = sum of lsum
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    __shared__ float sm_m[NW], sm_l[NW];
+    __shared__ float sm_o[NW][D];
+    // W/U of every group, from lanes (n, 0)
+    float Wg[G], Ug[G];
+#pragma unroll
+    for (int n = 0; n < G; ++n) {
+        Wg[n] = __shfl_sync(0xffffffffu, Wrun, 4 * n);
+        Ug[n] = __shfl_sync(0xffffffffu, Urun, 4 * n);
+    }
+#pragma unroll
+    for (int mt = 0; mt < NMT; ++mt) {
+        const int wi = mt / 4, by = mt % 4;
+        const int dlo = (D / 8) * g + 8 * wi + 2 * by;          // row g ; row g+8 is dlo + 1
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int dim = dlo + hr;
+            const int n = dim / GS;
+            if (n / 2 == t) {
+                // static register indices only (a runtime index would move oacc to local memory)
+                const float v = (n % 2) ? oacc[mt][2 * hr + 1] : oacc[mt][2 * hr];
+                sm_o[warp][dim] = v - C1024 * pick(Wg, n) + pick(Ug, n);
+            }
+        }
+    }
+    if (lane == 0) {
+        sm_m[warp] = m;
+        sm_l[warp] = lsum;
+    }
+    __syncthreads();
+    float M = -FLT_MAX;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) M = fmaxf(M, sm_m[i]);
+    float* out = part + (static_cast<int64_t>(pair) * nsplit + split) * (D + 2);
+    for (int d = threadIdx.x; d < D; d += DA_THREADS) {
+        float o = 0.f;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+            const float f = sm_l[i] > 0.f ? __expf(sm_m[i] - M) : 0.f;
+            o = fmaf(f, sm_o[i][d], o);
+        }
+        out[2 + d] = o;
+    }
+    if (threadIdx.x == 0) {
+        float L = 0.f;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) L += sm_l[i] > 0.f ? __expf(sm_m[i] - M) * sm_l[i] : 0.f;
+        out[0] = M;
+        out[1] = L;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// decode attention on the tensor cores with the key range staged in shared memory.
+// Same arithmetic as decode_attn_mma_kernel; the codes and metadata of 64-key chunks
+// are copied with cp.async into a DA_NS-deep ring (all threads of the CTA take part),
+// so DA_NS - 1 chunks are always in flight. In every chunk warp w owns tile w (keys
+// 16w..16w+15) and keeps its own online-softmax state across chunks.
+constexpr int DA_CHUNK = 64;
+constexpr int DA_NS = 4;
+
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool pred) {
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    const int n = pred ? 4 : 0;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(s), "l"(gmem), "r"(n) : "memory");
+}
+
+template <int D, int GS>
+__global__ void __launch_bounds__(DA_THREADS) decode_attn_staged_kernel(
+    const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
+    const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
+    const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
+    float* __restrict__ part) {
+    constexpr int G = D / GS;              // groups per key: 1, 2 or 4
+    constexpr int KB = D / 2;              // code bytes per key
+    constexpr int NKS = D / 16;            // QK k-steps
+    constexpr int NMT = D / 16;            // PV M-tiles
+    constexpr int NW = DA_THREADS / 32;    // warps = tiles per chunk
+    constexpr int CODE_BYTES = DA_CHUNK * KB;
+    constexpr int META_WORDS = DA_CHUNK * G;
+    constexpr int STAGE = 2 * CODE_BYTES + 2 * META_WORDS * 4;
+    constexpr float C1024 = 1024.f;
+    static_assert(NW * 16 == DA_CHUNK, "one 16-key tile per warp and chunk");
+    __shared__ __align__(16) uint8_t ring[DA_NS][STAGE];
+    pdl_wait();
+    pdl_trigger();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int pair = blockIdx.x, split = blockIdx.y, nsplit = gridDim.y;
+    const int b = pair / n_heads, head = pair % n_heads;
+    const int64_t slot0 = static_cast<int64_t>(pair) * max_seq;
+    const int j0 = split * chunk;
+    const int j1 = min(pos, j0 + chunk);
+    const int nchunks = (j1 - j0 + DA_CHUNK - 1) / DA_CHUNK;
+
+    // copy chunk c into ring slot c % DA_NS (keys past j1 are zero-filled, never read)
+    auto load_chunk = [&](int c) {
+        uint8_t* st = ring[c % DA_NS];
+        const int jc = j0 + c * DA_CHUNK;
+        const int n = min(DA_CHUNK, j1 - jc);
+        for (int u = threadIdx.x; u < CODE_BYTES / 16; u += DA_THREADS) {
+            const int key = (u * 16) / KB;
+            const bool ok = key < n;
+            const int64_t off = (slot0 + (ok ? jc : j0)) * KB + u * 16;
+            cp_async16(st + u * 16, k_codes + off, ok);
+            cp_async16(st + CODE_BYTES + u * 16, v_codes + off, ok);
+        }
+        for (int u = threadIdx.x; u < META_WORDS; u += DA_THREADS) {
+            const int key = u / G;
+            const bool ok = key < n;
+            const int64_t off = (slot0 + (ok ? jc : j0)) * G + u;
+            cp_async4(st + 2 * CODE_BYTES + u * 4, k_meta + off, ok);
+            cp_async4(st + 2 * CODE_BYTES + META_WORDS * 4 + u * 4, v_meta + off, ok);
+        }
+    };
+#pragma unroll
+    for (int c = 0; c < DA_NS - 1; ++c) {
+        if (c < nchunks) load_chunk(c);
+        cp_async_commit();
+    }
+
+    // ---- query: per-group sums and the masked B operand of the QK MMA
+    const __half* qp = q + static_cast<int64_t>(b) * row_stride + head * D;
+    float Qg[G];
+#pragma unroll
+    for (int n = 0; n < G; ++n) Qg[n] = 0.f;
+#pragma unroll
+    for (int v = 0; v < D / 8; ++v) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(qp) + v);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) Qg[(8 * v) / GS] += h2f_lo(ww[k]) + h2f_hi(ww[k]);
+    }
+    const int tgrp = (t * (D / 4)) / GS;
+    uint32_t bq[NKS][2];
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks) {
+        const int base = t * (D / 4) + 8 * (ks / 2) + 2 * (ks % 2);
+        if (g == tgrp) {
+            bq[ks][0] = pack_half2_bits(qp[base], qp[base + 4]);
+            bq[ks][1] = pack_half2_bits(qp[base + 1], qp[base + 5]);
+        } else {
+            bq[ks][0] = bq[ks][1] = 0u;
+        }
+    }
+
+    float m = -FLT_MAX, lsum = 0.f, Wrun = 0.f, Urun = 0.f;
+    float oacc[NMT][4];
+#pragma unroll
+    for (int i = 0; i < NMT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+
+    for (int c = 0; c < nchunks; ++c) {
+        if (c + DA_NS - 1 < nchunks) load_chunk(c + DA_NS - 1);
+        cp_async_commit();
+        cp_async_wait<DA_NS - 1>();
+        __syncthreads();
+        const uint8_t* st = ring[c % DA_NS];
+        const uint8_t* kc = st + warp * 16 * KB;                     // this warp's tile
+        const uint8_t* vc = st + CODE_BYTES + warp * 16 * KB;
+        const uint32_t* km = reinterpret_cast<const uint32_t*>(st + 2 * CODE_BYTES) + warp * 16 * G;
+        const uint32_t* vm = reinterpret_cast<const uint32_t*>(st + 2 * CODE_BYTES + META_WORDS * 4) + warp * 16 * G;
+        const int jt = j0 + c * DA_CHUNK + warp * 16;
+
+        // ---- scores
+        uint32_t kg[D / 32], kg8[D / 32];
+        if (D == 128) {
+            const uint4 a = *reinterpret_cast<const uint4*>(kc + g * KB + t * (D / 8));
+            const uint4 e = *reinterpret_cast<const uint4*>(kc + (g + 8) * KB + t * (D / 8));
+            kg[0] = a.x; kg[1 % (D / 32)] = a.y; kg[2 % (D / 32)] = a.z; kg[3 % (D / 32)] = a.w;
+            kg8[0] = e.x; kg8[1 % (D / 32)] = e.y; kg8[2 % (D / 32)] = e.z; kg8[3 % (D / 32)] = e.w;
+        } else {
+            const uint2 a = *reinterpret_cast<const uint2*>(kc + g * KB + t * (D / 8));
+            const uint2 e = *reinterpret_cast<const uint2*>(kc + (g + 8) * KB + t * (D / 8));
+            kg[0] = a.x; kg[1 % (D / 32)] = a.y;
+            kg8[0] = e.x; kg8[1 % (D / 32)] = e.y;
+        }
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < NKS; ++ks) {
+            const int w = ks / 2, e0 = 2 * (ks % 2);
+            const uint32_t a[4] = {nib_pair(kg[w] >> (4 * e0)), nib_pair(kg8[w] >> (4 * e0)),
+                                   nib_pair(kg[w] >> (4 * e0 + 4)), nib_pair(kg8[w] >> (4 * e0 + 4))};
+            mma16816(sacc, a, bq[ks][0], bq[ks][1]);
+        }
+        float sg_part = 0.f, sg8_part = 0.f;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int n = 2 * t + u;
+            if (n < G) {
+                const uint32_t m0 = km[g * G + n], m8 = km[(g + 8) * G + n];
+                const float Qn = pick(Qg, n);
+                const float st0 = group_step(__ushort_as_half(static_cast<unsigned short>(m0 >> 16)));
+                const float st8 = group_step(__ushort_as_half(static_cast<unsigned short>(m8 >> 16)));
+                sg_part += fmaf(st0, sacc[u] - C1024 * Qn, h2f_lo(m0) * Qn);
+                sg8_part += fmaf(st8, sacc[2 + u] - C1024 * Qn, h2f_lo(m8) * Qn);
+            }
+        }
+        if (G == 4) {
+            sg_part += __shfl_xor_sync(0xffffffffu, sg_part, 1);
+            sg8_part += __shfl_xor_sync(0xffffffffu, sg8_part, 1);
+        }
+        sg_part = __shfl_sync(0xffffffffu, sg_part, lane & ~3);
+        sg8_part = __shfl_sync(0xffffffffu, sg8_part, lane & ~3);
+        const float s_lo = (jt + g < j1) ? sg_part : -FLT_MAX;
+        const float s_hi = (jt + g + 8 < j1) ? sg8_part : -FLT_MAX;
+        float tmax = fmaxf(s_lo, s_hi);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
+        if (tmax > m) {                    // warp-uniform
+            const float alpha = __expf(m - tmax);
+            m = tmax;
+            lsum *= alpha;
+            Wrun *= alpha;
+            Urun *= alpha;
+#pragma unroll
+            for (int i = 0; i < NMT; ++i) {
+                oacc[i][0] *= alpha;
+                oacc[i][1] *= alpha;
+                oacc[i][2] *= alpha;
+                oacc[i][3] *= alpha;
+            }
+        }
+        const float p_lo = s_lo == -FLT_MAX ? 0.f : __expf(s_lo - m);
+        const float p_hi = s_hi == -FLT_MAX ? 0.f : __expf(s_hi - m);
+        if (t == 0) lsum += p_lo + p_hi;
+        // ---- values
+        const float pA = __shfl_sync(0xffffffffu, p_lo, 8 * t);
+        const float pAh = __shfl_sync(0xffffffffu, p_hi, 8 * t);
+        const float pB = __shfl_sync(0xffffffffu, p_lo, 8 * t + 4);
+        const float pBh = __shfl_sync(0xffffffffu, p_hi, 8 * t + 4);
+        uint32_t bv0 = 0u, bv1 = 0u;
+        float wt = 0.f, ut = 0.f;
+        if (g < G) {
+            const float pk[4] = {pA, pB, pAh, pBh};
+            float wv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t mv = vm[(2 * t + (u & 1) + 8 * (u >> 1)) * G + g];
+                const float stp = group_step(__ushort_as_half(static_cast<unsigned short>(mv >> 16)));
+                wv[u] = __half2float(__float2half_rn(pk[u] * stp));
+                wt += wv[u];
+                ut = fmaf(pk[u], h2f_lo(mv), ut);
+            }
+            bv0 = half2_bits(wv[0], wv[1]);
+            bv1 = half2_bits(wv[2], wv[3]);
+        }
+        wt += __shfl_xor_sync(0xffffffffu, wt, 1);
+        wt += __shfl_xor_sync(0xffffffffu, wt, 2);
+        ut += __shfl_xor_sync(0xffffffffu, ut, 1);
+        ut += __shfl_xor_sync(0xffffffffu, ut, 2);
+        Wrun += wt;
+        Urun += ut;
+        // PV side: thread g holds dims [g*D/8, (g+1)*D/8) of keys 2t, 2t+1, 2t+8, 2t+9,
+        // i.e. D/16 code bytes of each key starting at byte g*D/16
+        uint32_t vw[4][D / 64];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (D == 128) {
+                const uint2 a = *reinterpret_cast<const uint2*>(vc + (2 * t + (u & 1) + 8 * (u >> 1)) * KB + g * (D / 16));
+                vw[u][0] = a.x;
+                vw[u][1 % (D / 64)] = a.y;
+            } else {
+                vw[u][0] = *reinterpret_cast<const uint32_t*>(vc + (2 * t + (u & 1) + 8 * (u >> 1)) * KB + g * (D / 16));
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < NMT; ++mt) {
+            const int wi = mt / 4, by = mt % 4;
+            const uint32_t x1 = byte_pair(vw[0][wi], vw[1][wi], by);
+            const uint32_t x2 = byte_pair(vw[2][wi], vw[3][wi], by);
+            const uint32_t a[4] = {nib_pair(x1), nib_pair(x1 >> 4), nib_pair(x2), nib_pair(x2 >> 4)};
+            mma16816(oacc[mt], a, bv0, bv1);
+        }
+        __syncthreads();                   // the slot is refilled by the next iteration
+    }
+    cp_async_wait<0>();
+
+    // ---- warp result and CTA merge (as in decode_attn_mma_kernel)
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    __shared__ float sm_m[NW], sm_l[NW];
+    __shared__ float sm_o[NW][D];
+    float Wg[G], Ug[G];
+#pragma unroll
+    for (int n = 0; n < G; ++n) {
+        Wg[n] = __shfl_sync(0xffffffffu, Wrun, 4 * n);
+        Ug[n] = __shfl_sync(0xffffffffu, Urun, 4 * n);
+    }
+#pragma unroll
+    for (int mt = 0; mt < NMT; ++mt) {
+        const int wi = mt / 4, by = mt % 4;
+        const int dlo = (D / 8) * g + 8 * wi + 2 * by;
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int dim = dlo + hr;
+            const int n = dim / GS;
+            if (n / 2 == t) {
+                // static register indices only (a runtime index would move oacc to local memory)
+                const float v = (n % 2) ? oacc[mt][2 * hr + 1] : oacc[mt][2 * hr];
+                sm_o[warp][dim] = v - C1024 * pick(Wg, n) + pick(Ug, n);
+            }
+        }
+    }
+    if (lane == 0) {
+        sm_m[warp] = m;
+        sm_l[warp] = lsum;
+    }
+    __syncthreads();
+    float M = -FLT_MAX;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) M = fmaxf(M, sm_m[i]);
+    float* out = part + (static_cast<int64_t>(pair) * nsplit + split) * (D + 2);
+    for (int d = threadIdx.x; d < D; d += DA_THREADS) {
+        float o = 0.f;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+            const float f = sm_l[i] > 0.f ? __expf(sm_m[i] - M) : 0.f;
+            o = fmaf(f, sm_o[i][d], o);
+        }
+        out[2 + d] = o;
+    }
+    if (threadIdx.x == 0) {
+        float L = 0.f;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) L += sm_l[i] > 0.f ? __expf(sm_m[i] - M) * sm_l[i] : 0.f;
+        out[0] = M;
+        out[1] = L;
+    }
+}
+
+// combine the split partials with the fresh key/value of the current token
+template <int D>
+__global__ void __launch_bounds__(D) decode_attn_combine_kernel(const __half* __restrict__ q,
+                                                                const __half* __restrict__ k_new,
+                                                                const __half* __restrict__ v_new,
+                                                                int64_t row_stride, int n_heads,
+                                                                int nsplit,
+                                                                const float* __restrict__ part,
+                                                                __half* __restrict__ o, int perm) {
+    pdl_wait();
+    pdl_trigger();
+    const int pair = blockIdx.x;
+    const int b = pair / n_heads, head = pair % n_heads;
+    const int d = threadIdx.x;
+    const int64_t off = static_cast<int64_t>(b) * row_stride + head * D + d;
+    float s = __half2float(q[off]) * __half2float(k_new[off]);
+#pragma unroll
+    for (int w = 16; w > 0; w >>= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
+    __shared__ float red[D / 32];
+    if ((d & 31) == 0) red[d >> 5] = s;
+    __syncthreads();
+    float snew = 0.f;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) snew += red[i];
+    const float* pp = part + static_cast<int64_t>(pair) * nsplit * (D + 2);
+    float M = snew;
+    for (int i = 0; i < nsplit; ++i)
+        if (pp[i * (D + 2) + 1] > 0.f) M = fmaxf(M, pp[i * (D + 2)]);
+    const float fn = __expf(snew - M);
+    float L = fn;
+    float acc = fn * __half2float(v_new[off]);
+    for (int i = 0; i < nsplit; ++i) {
+        const float* p = pp + i * (D + 2);
+        if (!(p[1] > 0.f)) continue;
+        const float f = __expf(p[0] - M);
+        L = fmaf(f, p[1], L);
+        acc = fmaf(f, p[2 + d], acc);
+    }
+    // perm: interleaved 8-block order for the next GEMM (element k -> 2(k%4) + (k/4)%2)
+    const int dd = perm ? ((d & ~7) | ((d & 3) << 1) | ((d >> 2) & 1)) : d;
+    o[static_cast<int64_t>(b) * n_heads * D + head * D + dd] = __float2half_rn(acc / L);
+}
+
 template <int D>
 __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* __restrict__ q,
                                                                   const __half* __restrict__ k,
@@ -228,6 +839,8 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* 
                                                                   __half* __restrict__ o, int seq,
                                                                   int n_heads) {
     constexpr int LD = D + 8;                  // padded smem row (halves): conflict-free ldmatrix
+    pdl_wait();
+    pdl_trigger();
     constexpr int CPR = D / 8;                 // 16-byte chunks per row
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __half* sQ = reinterpret_cast<__half*>(smem_raw);
@@ -394,7 +1007,7 @@ int decode_attn_nsplit(int pairs, int pos) {
     if (pos <= 0) return 0;
     const int target = 4 * sm_count();
     int ns = (target + pairs - 1) / pairs;
-    const int max_by_len = (pos + 31) / 32;          // at least 32 keys per split
+    const int max_by_len = (pos + 127) / 128;        // at least 128 keys per split
     if (ns > max_by_len) ns = max_by_len;
     return ns < 1 ? 1 : ns;
 }
@@ -412,7 +1025,7 @@ int64_t decode_attn_ws_bound(int pairs, int head_dim) {
 }
 
 int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new, const void* v_new,
-                       int64_t row_stride, void* o, int batch, int pos, void* ws, cudaStream_t st) {
+                       int64_t row_stride, void* o, int batch, int pos, void* ws, bool perm, cudaStream_t st) {
     const int pairs = batch * c->n_heads;
     const int ns = decode_attn_nsplit(pairs, pos);
     const int chunk = ns > 0 ? (pos + ns - 1) / ns : 0;
@@ -425,12 +1038,16 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
     if (ns > 0) {
         const dim3 grid(pairs, ns);
 #define SPLIT(D_, B_, G_)                                                                                 \
-    decode_attn_split_kernel<D_, B_, G_><<<grid, DA_THREADS, 0, st>>>(qh, row_stride, kc, km, vc, vm,     \
-                                                                      c->n_heads, c->max_seq, pos, chunk, \
-                                                                      part)
+    launch_k(decode_attn_split_kernel<D_, B_, G_>, grid, dim3(DA_THREADS), 0, st, true, qh, row_stride, kc, km, vc, \
+             vm, c->n_heads, c->max_seq, pos, chunk, part)
+#define MMA(D_, G_)                                                                                      \
+    launch_k(decode_attn_staged_kernel<D_, G_>, grid, dim3(DA_THREADS), 0, st, true, qh, row_stride, kc, km, vc, vm, \
+             c->n_heads, c->max_seq, pos, chunk, part)
         const int D = c->head_dim, B = c->cfg.num_bits, G = c->cfg.group_size;
-        if (D == 64 && B == 4 && G == 64) SPLIT(64, 4, 64);
-        else if (D == 64 && B == 4 && G == 32) SPLIT(64, 4, 32);
+        if (D == 64 && B == 4 && G == 64) MMA(64, 64);
+        else if (D == 64 && B == 4 && G == 32) MMA(64, 32);
+        else if (D == 128 && B == 4 && G == 64) MMA(128, 64);
+        else if (D == 128 && B == 4 && G == 32) MMA(128, 32);
         else if (D == 64 && B == 8 && G == 64) SPLIT(64, 8, 64);
         else if (D == 64 && B == 8 && G == 32) SPLIT(64, 8, 32);
         else if (D == 128 && B == 4 && G == 64) SPLIT(128, 4, 64);
@@ -438,14 +1055,17 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
         else if (D == 128 && B == 8 && G == 64) SPLIT(128, 8, 64);
         else SPLIT(128, 8, 32);
 #undef SPLIT
+#undef MMA
     }
     const __half* kn = static_cast<const __half*>(k_new);
     const __half* vn = static_cast<const __half*>(v_new);
     __half* oh = static_cast<__half*>(o);
     if (c->head_dim == 64)
-        decode_attn_combine_kernel<64><<<pairs, 64, 0, st>>>(qh, kn, vn, row_stride, c->n_heads, ns, part, oh);
+        launch_k(decode_attn_combine_kernel<64>, dim3(pairs), dim3(64), 0, st, true, qh, kn, vn, row_stride,
+                 c->n_heads, ns, static_cast<const float*>(part), oh, perm ? 1 : 0);
     else
-        decode_attn_combine_kernel<128><<<pairs, 128, 0, st>>>(qh, kn, vn, row_stride, c->n_heads, ns, part, oh);
+        launch_k(decode_attn_combine_kernel<128>, dim3(pairs), dim3(128), 0, st, true, qh, kn, vn, row_stride,
+                 c->n_heads, ns, static_cast<const float*>(part), oh, perm ? 1 : 0);
     return launch_status();
 }
 
@@ -461,11 +1081,13 @@ int prefill_attn_launch(const void* q, const void* k, const void* v, int64_t row
     const __half* vh = static_cast<const __half*>(v);
     __half* oh = static_cast<__half*>(o);
     if (head_dim == 64) {
-        cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        prefill_attn_kernel<64><<<grid, PA_THREADS, smem, st>>>(qh, kh, vh, row_stride, oh, seq, n_heads);
+        set_smem_once(prefill_attn_kernel<64>, (int)smem);
+        launch_k(prefill_attn_kernel<64>, grid, dim3(PA_THREADS), smem, st, true, qh, kh, vh, row_stride, oh, seq,
+                 n_heads);
     } else {
-        cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        prefill_attn_kernel<128><<<grid, PA_THREADS, smem, st>>>(qh, kh, vh, row_stride, oh, seq, n_heads);
+        set_smem_once(prefill_attn_kernel<128>, (int)smem);
+        launch_k(prefill_attn_kernel<128>, grid, dim3(PA_THREADS), smem, st, true, qh, kh, vh, row_stride, oh, seq,
+                 n_heads);
     }
     return launch_status();
 }
@@ -495,7 +1117,7 @@ extern "C" int flex_decode_attention(const flex_kv_cache* cache, const void* q, 
     const int64_t need = decode_attn_ws_bytes(batch * cache->n_heads, cache->head_dim, pos);
     FLEX_REQUIRE(ws != nullptr && ws_bytes >= need, FLEX_ERR_WORKSPACE);
     FLEX_REQUIRE(aligned16(ws), FLEX_ERR_ALIGN);
-    return decode_attn_launch(cache, q, k_new, v_new, row_stride, o, batch, pos, ws, as_stream(stream));
+    return decode_attn_launch(cache, q, k_new, v_new, row_stride, o, batch, pos, ws, false, as_stream(stream));
 }
 
 extern "C" int flex_prefill_attention(const void* q, const void* k, const void* v, int64_t row_stride, void* o,

@@ -1,4 +1,4 @@
-// Group-wise int4/int8 compression and decompression (FlexGen source walkthrough,
+// Group-wise int4/int8 compression and decompression (the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南»,
 // section 6.3: compress / decompress of a CompressionConfig(num_bits, group_size,
 // group_dim, symmetric=False) with a packed uint8 data tensor and an fp16 per-group
 // scale).

@@ -28,6 +28,40 @@ inline int launch_status() {
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device), so that it is
+// not called again while a stream is being captured into a graph.
+bool smem_attr_needed(const void* kernel, int bytes);
+template <typename K>
+inline void set_smem_once(K kernel, int bytes) {
+    if (smem_attr_needed(reinterpret_cast<const void*>(kernel), bytes))
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// Launch `kernel` on `st`, with programmatic stream serialisation when pdl is true.
+template <typename... KArgs, typename... Args>
+inline void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                     Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// store_cache fused into the QKV projection's epilogue (see gemm.cu).
+struct KvFuse {
+    const flex_kv_cache* cache;
+    int h;       // hidden size: features [h, 2h) keys, [2h, 3h) values
+    int seq;     // tokens per sequence in this call
+    int pos0;    // cache slot of token 0
+};
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 // Device status word of the current device (created on first use; see flex_get_status).
@@ -67,6 +101,14 @@ __device__ __forceinline__ uint32_t pack_half2_bits(__half lo, __half hi) {
     return static_cast<uint32_t>(__half_as_ushort(lo)) |
            (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
 }
+
+// Programmatic dependent launch: a kernel launched with launch_k(..., pdl = true) may
+// start while its predecessor in the stream is still running. pdl_wait() blocks until
+// the predecessor grid has completed and its writes are visible (it returns at once
+// when there is no such dependency); pdl_trigger() lets this kernel's own dependents
+// start their prologues.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void set_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);

@@ -2,7 +2,7 @@
 //
 //   y[m][n] = epilogue( sum_k x[m][k] * W^[n][k] + bias[n] )
 //
-// W is a group-wise compressed weight (FlexGen source walkthrough, section 6.3:
+// W is a group-wise compressed weight (the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南», section 6.3:
 // 4-bit codes, group 64, per-group fp16 {min, scale}), stored [N][K] and grouped along
 // K, so a 64-wide K chunk is exactly one group per row. The kernel never materialises
 // W^ in global memory:
@@ -24,6 +24,7 @@
 // depend on scheduling. Every mbarrier wait is bounded: on expiry the CTA records
 // FLEX_ERR_TIMEOUT in the device status word, drains its own copies and MMAs, frees
 // TMEM and exits.
+#include "quant.cuh"
 #include "tc.cuh"
 
 namespace flexq {
@@ -36,6 +37,7 @@ constexpr int kThreads = 384;      // 12 warps
 constexpr int kDequantThreads = 256;
 constexpr int kNSA = 4;            // dequantised A stages
 constexpr int kMetaChunks = 4;     // groups per metadata tile
+constexpr int kDoneRing = 8;       // mma_done barriers (>= kNSA and >= every activation ring depth)
 
 struct GemmParams {
     const __half* bias;
@@ -50,13 +52,20 @@ struct GemmParams {
     int nq;                // columns n < nq are multiplied by qscale
     float qscale;
     int relu;
+    int yperm;             // write y in the interleaved 8-block order
     int nsx, nsc;          // activation / code ring depths
     uint32_t off_x, off_c, off_m, off_bar;
     uint32_t tmem_cols;
+    // fused store_cache (QKV projection): output features [kv_h, 2 kv_h) are the keys and
+    // [2 kv_h, 3 kv_h) the values; token m = b * kv_seq + t goes to cache slot kv_pos0 + t
+    // of sequence b. kv_codes[0] == nullptr: off.
+    uint8_t* kv_codes[2];
+    uint32_t* kv_meta[2];
+    int kv_h, kv_hd, kv_nh, kv_max_seq, kv_seq, kv_pos0, kv_bits, kv_gs;
 };
 
 struct Bars {
-    uint32_t codes_full, codes_empty, x_full, x_empty, a_full, a_empty, meta_full, meta_empty, acc_full, drain;
+    uint32_t codes_full, codes_empty, x_full, a_full, mma_done, acc_full, drain;
 };
 
 __device__ __forceinline__ uint32_t dequant_pair(uint32_t raw_pair_bits, uint32_t step2, uint32_t mn2) {
@@ -89,19 +98,121 @@ __device__ __forceinline__ uint4 dequant8_4bit(uint32_t w, uint32_t step2, uint3
     return make_uint4(prmt(p0, p1, 0x5410u), prmt(p2, p3, 0x5410u), prmt(p0, p1, 0x7632u), prmt(p2, p3, 0x7632u));
 }
 
+// Same 8 codes, left in the pair order the unpack produces: (e0,e4) (e1,e5) (e2,e6)
+// (e3,e7), i.e. positions [e0 e4 e1 e5 e2 e6 e3 e7]. The activation operand must then
+// use the same order inside every 8-block of K (the "interleaved" activation layout the
+// layer kernels write), and the MMA sees matching K positions on both sides.
+__device__ __forceinline__ uint4 dequant8_4bit_il(uint32_t w, uint32_t step2, uint32_t mn2) {
+    return make_uint4(dequant_pair(lop_nib(w), step2, mn2), dequant_pair(lop_nib(w >> 4), step2, mn2),
+                      dequant_pair(lop_nib(w >> 8), step2, mn2), dequant_pair(lop_nib(w >> 12), step2, mn2));
+}
+
+__device__ __forceinline__ uint32_t lop_byte(uint32_t x) {
+    // (x & 0x00FF00FF) | 0x64006400
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(0x00FF00FFu), "r"(0x64006400u));
+    return r;
+}
+
+// 8 codes of 8 bits (two u32: k0..k3, k4..k7) -> 8 fp16 in the interleaved order.
+__device__ __forceinline__ uint4 dequant8_8bit_il(uint32_t w0, uint32_t w1, uint32_t step2, uint32_t mn2) {
+    return make_uint4(dequant_pair(lop_byte(prmt(w0, w1, 0x0400u)), step2, mn2),
+                      dequant_pair(lop_byte(prmt(w0, w1, 0x0501u)), step2, mn2),
+                      dequant_pair(lop_byte(prmt(w0, w1, 0x0602u)), step2, mn2),
+                      dequant_pair(lop_byte(prmt(w0, w1, 0x0703u)), step2, mn2));
+}
+
 // 4 codes of 8 bits (one u32) -> 4 fp16 as two half2.
 __device__ __forceinline__ uint2 dequant4_8bit(uint32_t w, uint32_t step2, uint32_t mn2) {
     const uint32_t hi = 0x64646464u;
     return make_uint2(dequant_pair(prmt(w, hi, 0x4140u), step2, mn2), dequant_pair(prmt(w, hi, 0x4342u), step2, mn2));
 }
 
+// Fused store_cache for 8 token columns of the epilogue. Thread (warp, lane) holds output
+// feature n (= one dimension of one head) for the columns col..col+7, already rounded to
+// fp16. A quantisation group is gs consecutive features: one warp (gs = 32) or the two
+// warps of a pair (gs = 64: warps 4/5, 6/7, 8/9, 10/11 hold rows 0-63 / 64-127 of the
+// same column half). min/max are reduced over the group, then every thread quantises its
+// own value with the shared quantiser (bit-identical to flexq_compress of the same
+// fp16 values); even lanes write the byte of two 4-bit codes, the group's first row its
+// {min, scale}.
 template <int BITS>
+__device__ __forceinline__ void kv_store8_bits(const GemmParams& p, const __half (&o16)[8], int col, int m0, int n0,
+                                               int n, int warp, int lane, uint32_t* kv_red) {
+    const int sec = (n0 - p.kv_h) / p.kv_h;                // 0 keys, 1 values
+    const int f = n - p.kv_h - sec * p.kv_h;
+    const int head = f / p.kv_hd, dim = f % p.kv_hd;
+    // min / max of the 8 columns as 4 half2 pairs
+    __half2 mn2[4], mx2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mn2[k] = mx2[k] = __halves2half2(o16[2 * k], o16[2 * k + 1]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t a = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t*>(&mn2[k]), off);
+            const uint32_t b = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t*>(&mx2[k]), off);
+            mn2[k] = __hmin2(mn2[k], *reinterpret_cast<const __half2*>(&a));
+            mx2[k] = __hmax2(mx2[k], *reinterpret_cast<const __half2*>(&b));
+        }
+    if (p.kv_gs == 64) {
+        const int w = warp - 4, pairbar = 2 + (w >> 1);
+        if (lane == 0)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                kv_red[(w * 4 + k) * 2] = *reinterpret_cast<uint32_t*>(&mn2[k]);
+                kv_red[(w * 4 + k) * 2 + 1] = *reinterpret_cast<uint32_t*>(&mx2[k]);
+            }
+        asm volatile("bar.sync %0, 64;" ::"r"(pairbar) : "memory");
+        const int pw = w ^ 1;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t a = kv_red[(pw * 4 + k) * 2], b = kv_red[(pw * 4 + k) * 2 + 1];
+            mn2[k] = __hmin2(mn2[k], *reinterpret_cast<const __half2*>(&a));
+            mx2[k] = __hmax2(mx2[k], *reinterpret_cast<const __half2*>(&b));
+        }
+        asm volatile("bar.sync %0, 64;" ::"r"(pairbar) : "memory");   // kv_red is reused by the next call
+    }
+    uint8_t* codes = p.kv_codes[sec];
+    uint32_t* meta = p.kv_meta[sec];
+    const int gph = p.kv_hd / p.kv_gs;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int m = m0 + col + j;
+        const float mn = (j & 1) ? __high2float(mn2[j >> 1]) : __low2float(mn2[j >> 1]);
+        const float mx = (j & 1) ? __high2float(mx2[j >> 1]) : __low2float(mx2[j >> 1]);
+        const __half s16 = group_scale16<BITS>(mn, mx);
+        const uint32_t q = quant_one<BITS>(__half2float(o16[j]), mn, __half2float(s16));
+        const uint32_t qn = __shfl_down_sync(0xffffffffu, q, 1);
+        if (m >= p.M) continue;
+        const int b = m / p.kv_seq, t = m - b * p.kv_seq;
+        const int64_t slot = (static_cast<int64_t>(b) * p.kv_nh + head) * p.kv_max_seq + p.kv_pos0 + t;
+        if (BITS == 4) {
+            if ((lane & 1) == 0) codes[slot * (p.kv_hd / 2) + dim / 2] = static_cast<uint8_t>(q | (qn << 4));
+        } else {
+            codes[slot * p.kv_hd + dim] = static_cast<uint8_t>(q);
+        }
+        if (dim % p.kv_gs == 0) meta[slot * gph + dim / p.kv_gs] = pack_half2_bits(__float2half_rn(mn), s16);
+    }
+}
+
+__device__ __forceinline__ void kv_store8(const GemmParams& p, const __half (&o16)[8], int col, int m0, int n0, int n,
+                                          int warp, int lane, uint32_t* kv_red) {
+    if (p.kv_bits == 4)
+        kv_store8_bits<4>(p, o16, col, m0, n0, n, warp, lane, kv_red);
+    else
+        kv_store8_bits<8>(p, o16, col, m0, n0, n, warp, lane, kv_red);
+}
+
+template <int BITS, bool XPERM>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                               const __grid_constant__ CUtensorMap tm_meta,
                                                               const __grid_constant__ CUtensorMap tm_x,
                                                               const GemmParams p) {
-    constexpr int CB = kBM * kBK * BITS / 8;     // code bytes per stage
-    constexpr int CROW = kBK * BITS / 8;         // code bytes per row and stage
+    constexpr int CROW = kBK * BITS / 8;          // code bytes per row and K chunk (32 or 64)
+    constexpr int CPS = 128 / CROW;               // K chunks per code stage (4 or 2)
+    constexpr int CSTAGE = kBM * 128;             // code bytes per stage: 128 rows x 128 B
+    constexpr int MSTAGE = kBM * kMetaChunks * 4; // metadata bytes per stage: 128 rows x 4 groups
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -110,8 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kBM, m0 = blockIdx.y * p.BN, split = blockIdx.z;
     const int nk_total = p.K / kBK;
-    const int c_begin = split * p.cps;
-    const int nk = min(nk_total, c_begin + p.cps) - c_begin;
+    const int c_begin = split * p.cps;                            // multiple of kMetaChunks
+    const int nk = min(nk_total, c_begin + p.cps) - c_begin;      // multiple of kMetaChunks
+    const int nstages = nk / CPS;
 
     const uint32_t sA = base, sX = base + p.off_x, sC = base + p.off_c, sM = base + p.off_m;
     const uint32_t sb = base + p.off_bar;
@@ -120,35 +232,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     B.codes_full = sb;
     B.codes_empty = B.codes_full + 8 * NSC;
     B.x_full = B.codes_empty + 8 * NSC;
-    B.x_empty = B.x_full + 8 * NSX;
-    B.a_full = B.x_empty + 8 * NSX;
-    B.a_empty = B.a_full + 8 * kNSA;
-    B.meta_full = B.a_empty + 8 * kNSA;
-    B.meta_empty = B.meta_full + 16;
-    B.acc_full = B.meta_empty + 16;
+    B.a_full = B.x_full + 8 * NSX;
+    B.mma_done = B.a_full + 8 * kNSA;
+    B.acc_full = B.mma_done + 8 * kDoneRing;
     B.drain = B.acc_full + 8;
     const uint32_t misc = B.drain + 8;                        // tmem slot, abort flag, last flag
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (misc - base));
     volatile int* abort = reinterpret_cast<volatile int*>(gbase + (misc - base) + 4);
     volatile int* last_flag = reinterpret_cast<volatile int*>(gbase + (misc - base) + 8);
+    uint32_t* kv_red = reinterpret_cast<uint32_t*>(gbase + (misc - base) + 16);   // [8 warps][4 pairs][2]
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSC; ++s) {
             tc::bar_init(B.codes_full + 8 * s, 1);
             tc::bar_init(B.codes_empty + 8 * s, kDequantThreads);
         }
-        for (int s = 0; s < NSX; ++s) {
-            tc::bar_init(B.x_full + 8 * s, 1);
-            tc::bar_init(B.x_empty + 8 * s, 1);
-        }
-        for (int s = 0; s < kNSA; ++s) {
-            tc::bar_init(B.a_full + 8 * s, kDequantThreads);
-            tc::bar_init(B.a_empty + 8 * s, 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            tc::bar_init(B.meta_full + 8 * s, 1);
-            tc::bar_init(B.meta_empty + 8 * s, kDequantThreads);
-        }
+        for (int s = 0; s < NSX; ++s) tc::bar_init(B.x_full + 8 * s, 1);
+        for (int s = 0; s < kNSA; ++s) tc::bar_init(B.a_full + 8 * s, kDequantThreads);
+        for (int s = 0; s < kDoneRing; ++s) tc::bar_init(B.mma_done + 8 * s, 1);
         tc::bar_init(B.acc_full, 1);
         tc::bar_init(B.drain, 1);
         *abort = 0;
@@ -168,36 +269,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();                                   // the activations come from the previous kernel
 
     if (warp == 0) {
-        // ---------------- codes + metadata producer ----------------
+        // ---------------- code + metadata producer: one stage = CPS chunks ----------------
         if (lane == 0) {
-            int i = 0, mi = 0;   // code tiles and metadata tiles issued
-            for (; i < nk; ++i) {
-                const int c = c_begin + i;
-                if (i % kMetaChunks == 0) {
-                    const int blk = i / kMetaChunks, sm = blk & 1;
-                    if (!tc::bar_wait(B.meta_empty + 8 * sm, ((blk >> 1) & 1) ^ 1, abort, p.status)) break;
-                    tc::bar_arrive_expect_tx(B.meta_full + 8 * sm, kBM * kMetaChunks * 4);
-                    tc::tma_load_2d(sM + sm * (kBM * kMetaChunks * 4), &tm_meta, c, n0, B.meta_full + 8 * sm);
-                    ++mi;
-                }
-                const int s = i % NSC;
-                if (!tc::bar_wait(B.codes_empty + 8 * s, ((i / NSC) & 1) ^ 1, abort, p.status)) break;
-                tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CB);
-                tc::tma_load_2d(sC + s * CB, &tm_codes, c * CROW, n0, B.codes_full + 8 * s);
+            int st = 0;
+            for (; st < nstages; ++st) {
+                const int s = st % NSC;
+                if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ((st / NSC) & 1) ^ 1, abort, p.status)) break;
+                const int c = c_begin + st * CPS;
+                tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CSTAGE + MSTAGE);
+                tc::tma_load_2d(sC + s * CSTAGE, &tm_codes, c * CROW, n0, B.codes_full + 8 * s);
+                tc::tma_load_2d(sM + s * MSTAGE, &tm_meta, c & ~(kMetaChunks - 1), n0, B.codes_full + 8 * s);
             }
             // drain: every copy this thread issued has landed before the CTA can exit
-            const int issued = i;
-            for (int s = 0; s < NSC && s < issued; ++s) {
-                const int last = s + ((issued - 1 - s) / NSC) * NSC;
+            for (int s = 0; s < NSC && s < st; ++s) {
+                const int last = s + ((st - 1 - s) / NSC) * NSC;
                 volatile int never = 0;
                 tc::bar_wait(B.codes_full + 8 * s, (last / NSC) & 1, &never, p.status);
-            }
-            for (int sm = 0; sm < 2 && sm < mi; ++sm) {
-                const int last = sm + ((mi - 1 - sm) / 2) * 2;
-                volatile int never = 0;
-                tc::bar_wait(B.meta_full + 8 * sm, (last >> 1) & 1, &never, p.status);
             }
         }
         __syncwarp();
@@ -207,7 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             int i = 0;
             for (; i < nk; ++i) {
                 const int s = i % NSX;
-                if (!tc::bar_wait(B.x_empty + 8 * s, ((i / NSX) & 1) ^ 1, abort, p.status)) break;
+                // slot s last held chunk i - NSX: wait until its MMAs are done
+                if (i >= NSX) {
+                    const int pc = i - NSX;
+                    if (!tc::bar_wait(B.mma_done + 8 * (pc % kDoneRing), (pc / kDoneRing) & 1, abort, p.status)) break;
+                }
                 tc::bar_arrive_expect_tx(B.x_full + 8 * s, p.BN * 128);
                 tc::tma_load_2d(sX + s * (p.BN * 128), &tm_x, (c_begin + i) * kBK, m0, B.x_full + 8 * s);
             }
@@ -234,72 +328,114 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk)
                     tc::mma_f16(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_commit(B.a_empty + 8 * sa);
-                tc::mma_commit(B.x_empty + 8 * sx);
+                // exactly one commit per chunk: a commit covers the MMAs issued since the
+                // previous one, so a second commit here would complete at once. Both rings
+                // that reuse this chunk's operands (A and activations) wait on mma_done;
+                // the last chunk's commit is the accumulator-ready signal.
+                tc::mma_commit(i + 1 < nk ? B.mma_done + 8 * (i % kDoneRing) : B.acc_full);
             }
-            if (ok) {
-                tc::mma_commit(B.acc_full);
-            } else {
+            if (!ok) {
                 // nothing of ours may still run on the tensor cores at exit
                 tc::mma_commit(B.drain);
                 volatile int never = 0;
                 tc::bar_wait(B.drain, 0, &never, p.status);
+            } else {
+                // every commit's mbarrier arrival must have landed before the CTA exits: a
+                // late arrival would hit the barriers of the next CTA on this SM, which
+                // live at the same shared-memory addresses
+                volatile int never = 0;
+                const int last = nk - 1;                 // committed to acc_full (waited in the epilogue)
+                for (int c = last - kDoneRing > 0 ? last - kDoneRing : 0; c < last; ++c)
+                    tc::bar_wait(B.mma_done + 8 * (c % kDoneRing), (c / kDoneRing) & 1, &never, p.status);
+                tc::bar_wait(B.acc_full, 0, &never, p.status);
             }
         }
         __syncwarp();
     } else if (warp >= 4) {
         // ---------------- dequantisation ----------------
+        // thread (row, half): for every K chunk, half of the row's codes (16 code bytes at
+        // 4 bits, 32 at 8 bits) -> 32 fp16 = 4 of the row's 8 16-byte chunks of A
         const int dt = threadIdx.x - 128;
         const int row = dt & 127, half_ = dt >> 7;
+        const int sw = row & 7;
         bool ok = true;
-        uint4 mrow = make_uint4(0, 0, 0, 0);
-        for (int i = 0; i < nk; ++i) {
-            if (i % kMetaChunks == 0) {
-                const int blk = i / kMetaChunks;
-                if (!tc::bar_wait(B.meta_full + 8 * (blk & 1), (blk >> 1) & 1, abort, p.status)) { ok = false; break; }
-                mrow = *reinterpret_cast<const uint4*>(gbase + (sM - base) + (blk & 1) * (kBM * kMetaChunks * 4) + row * 16);
-            }
-            const int sc = i % NSC;
-            if (!tc::bar_wait(B.codes_full + 8 * sc, (i / NSC) & 1, abort, p.status)) { ok = false; break; }
-            const uint8_t* crow = gbase + (sC - base) + sc * CB + row * CROW + half_ * (CROW / 2);
-            uint4 cw0 = *reinterpret_cast<const uint4*>(crow);
-            uint4 cw1 = make_uint4(0, 0, 0, 0);
-            if (BITS == 8) cw1 = *reinterpret_cast<const uint4*>(crow + 16);
-            tc::bar_arrive(B.codes_empty + 8 * sc);
-            if (i % kMetaChunks == kMetaChunks - 1 || i == nk - 1) tc::bar_arrive(B.meta_empty + 8 * ((i / kMetaChunks) & 1));
-
-            const uint32_t mw = (i % 4 == 0) ? mrow.x : (i % 4 == 1) ? mrow.y : (i % 4 == 2) ? mrow.z : mrow.w;
-            const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
-            const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
-            const __half step = __float2half_rn(sc32 > 0.f ? 1.0f / sc32 : 0.f);
-            const __half2 step2h = __half2half2(step), mn2h = __half2half2(mn);
-            const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&step2h);
-            const uint32_t mn2 = *reinterpret_cast<const uint32_t*>(&mn2h);
-
-            const int sa = i % kNSA;
-            if (!tc::bar_wait(B.a_empty + 8 * sa, ((i / kNSA) & 1) ^ 1, abort, p.status)) { ok = false; break; }
-            uint8_t* arow = gbase + sa * (kBM * 128) + row * 128;
-            const int sw = row & 7;
-            if (BITS == 4) {
-                const uint32_t w[4] = {cw0.x, cw0.y, cw0.z, cw0.w};
+        int i = 0;                                  // K chunk index within the split
+        for (int st = 0; st < nstages && ok; ++st) {
+            const int s = st % NSC;
+            if (!tc::bar_wait(B.codes_full + 8 * s, (st / NSC) & 1, abort, p.status)) { ok = false; break; }
+            // codes of this stage (the tile was stored with the 128-byte swizzle: 16-byte
+            // unit u of row r sits at unit u ^ (r % 8))
+            const uint8_t* crow = gbase + (sC - base) + s * CSTAGE + row * 128;
+            uint4 cw[CPS][BITS / 4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 v = dequant8_4bit(w[j], step2, mn2);
-                    *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = v;
-                }
-            } else {
-                const uint32_t w[8] = {cw0.x, cw0.y, cw0.z, cw0.w, cw1.x, cw1.y, cw1.z, cw1.w};
+            for (int c = 0; c < CPS; ++c)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint2 a = dequant4_8bit(w[2 * j], step2, mn2);
-                    const uint2 b = dequant4_8bit(w[2 * j + 1], step2, mn2);
-                    *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+                for (int v = 0; v < BITS / 4; ++v) {
+                    const int u = c * (CROW / 16) + half_ * (BITS / 4) + v;
+                    cw[c][v] = *reinterpret_cast<const uint4*>(crow + ((u ^ sw) << 4));
                 }
+            const uint4 mrow = *reinterpret_cast<const uint4*>(gbase + (sM - base) + s * MSTAGE + row * 16);
+            const uint32_t mwv[4] = {mrow.x, mrow.y, mrow.z, mrow.w};
+            const int moff = (c_begin + st * CPS) & (kMetaChunks - 1);
+#pragma unroll
+            for (int c = 0; c < CPS; ++c, ++i) {
+                const uint32_t mw = mwv[(moff + c) & 3];
+                const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
+                const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
+                // step = fp16(1/scale); a constant group (scale 0) gets step 0 and decodes to min
+                const __half step = __float2half_rn(sc32 > 0.f ? __frcp_rn(sc32) : 0.f);
+                const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
+                const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
+                const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
+                const int sa = i % kNSA;
+                // slot sa last held chunk i - kNSA: wait until its MMAs are done
+                if (i >= kNSA) {
+                    const int pc = i - kNSA;
+                    if (!tc::bar_wait(B.mma_done + 8 * (pc % kDoneRing), (pc / kDoneRing) & 1, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                uint8_t* arow = gbase + sa * (kBM * 128) + row * 128;
+                if (BITS == 4) {
+                    const uint32_t w[4] = {cw[c][0].x, cw[c][0].y, cw[c][0].z, cw[c][0].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2) : dequant8_4bit(w[j], step2, mnv2);
+                        *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = v;
+                    }
+                } else {
+                    const uint4 c0 = cw[c][0], c1 = cw[c][BITS / 4 - 1];
+                    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 v;
+                        if (XPERM) {
+                            v = dequant8_8bit_il(w[2 * j], w[2 * j + 1], step2, mnv2);
+                        } else {
+                            const uint2 a = dequant4_8bit(w[2 * j], step2, mnv2);
+                            const uint2 b = dequant4_8bit(w[2 * j + 1], step2, mnv2);
+                            v = make_uint4(a.x, a.y, b.x, b.y);
+                        }
+                        *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = v;
+                    }
+                }
+                tc::fence_proxy_async_smem();
+                tc::bar_arrive(B.a_full + 8 * sa);
             }
-            tc::fence_proxy_async_smem();
-            tc::bar_arrive(B.a_full + 8 * sa);
+            // release the code stage only once all of its values have been consumed (the
+            // next TMA into this slot must not overtake these shared-memory reads)
+            if (ok) tc::bar_arrive(B.codes_empty + 8 * s);
         }
         // ---------------- epilogue ----------------
+        pdl_trigger();                            // dependents may start their prologue
+        const int lq = warp & 3, ch = (warp - 4) >> 2;
+        const int irow = lq * 32 + lane;
+        const int n = n0 + irow;
+        const float bias_n = p.bias ? __half2float(p.bias[n]) : 0.f;   // issued before the waits
+        const float scale_n = n < p.nq ? p.qscale : 1.f;
+        // interleaved output: element k of every 8-block goes to position 2(k%4) + (k/4)%2
+        const int n_out = p.yperm ? ((n & ~7) | ((n & 3) << 1) | ((n >> 2) & 1)) : n;
         asm volatile("bar.sync 1, 256;" ::: "memory");
         if (ok && !*abort) ok = tc::bar_wait(B.acc_full, 0, abort, p.status);
         // one decision for all 256 threads (they share the named barriers below)
@@ -314,28 +450,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             : "memory");
         if (all_ok) {
             tc::fence_after_sync();
-            const int lq = warp & 3, ch = (warp - 4) >> 2;
-            const int irow = lq * 32 + lane;
-            const int n = n0 + irow;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16);
             const int cbeg = ch * (p.BN / 2), cend = cbeg + p.BN / 2;
-            const float bias_n = p.bias ? __half2float(p.bias[n]) : 0.f;
-            const float scale_n = n < p.nq ? p.qscale : 1.f;
-            auto finish = [&](int col, float v) {
-                const int m = m0 + col;
-                if (m >= p.M) return;
-                v = (v + bias_n) * scale_n;
-                if (p.relu) v = fmaxf(v, 0.f);
-                const int64_t o = static_cast<int64_t>(m) * p.N + n;
-                if (p.residual) v += __half2float(p.residual[o]);
-                p.y[o] = __float2half_rn(v);
+            // 8 columns at a time: residual loads issued together, then the stores
+            // fused store_cache: this tile lies inside the key or the value block (h % 128 == 0)
+            const bool kv_on = p.kv_codes[0] != nullptr && n0 >= p.kv_h;
+            auto finish8 = [&](int col, const float (&v)[8]) {
+                float r[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int m = m0 + col + j;
+                    r[j] = (p.residual && m < p.M) ? __half2float(p.residual[static_cast<int64_t>(m) * p.N + n]) : 0.f;
+                }
+                __half o16[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int m = m0 + col + j;
+                    float x = (v[j] + bias_n) * scale_n;
+                    if (p.relu) x = fmaxf(x, 0.f);
+                    o16[j] = __float2half_rn(x + r[j]);
+                    if (m < p.M) p.y[static_cast<int64_t>(m) * p.N + n_out] = o16[j];
+                }
+                if (kv_on) kv_store8(p, o16, col, m0, n0, n, warp, lane, kv_red);
             };
             if (p.splits == 1) {
                 for (int col = cbeg; col < cend; col += 8) {
                     float v[8];
                     tc::tmem_ld8(taddr + col, v);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) finish(col + j, v[j]);
+                    finish8(col, v);
                 }
             } else {
                 const int tile = blockIdx.y * gridDim.x + blockIdx.x;
@@ -353,11 +495,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 if (*last_flag) {
                     __threadfence();
                     const float* all = p.part + static_cast<int64_t>(tile) * p.splits * p.BN * kBM;
-                    for (int col = cbeg; col < cend; ++col) {
-                        float acc = 0.f;
-                        for (int s = 0; s < p.splits; ++s)
-                            acc += __ldcg(all + (static_cast<int64_t>(s) * p.BN + col) * kBM + irow);
-                        finish(col, acc);
+                    for (int col = cbeg; col < cend; col += 8) {
+                        float acc[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+                        // up to 4 splits' 8 values in flight at once, summed in split order
+                        for (int s0 = 0; s0 < p.splits; s0 += 4) {
+                            float t[4][8];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    t[u][j] = (s0 + u < p.splits)
+                                                  ? __ldcg(all + (static_cast<int64_t>(s0 + u) * p.BN + col + j) * kBM + irow)
+                                                  : 0.f;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) acc[j] += t[u][j];
+                        }
+                        finish8(col, acc);
                     }
                     if (dt == 0) p.counters[tile] = 0;
                 }
@@ -416,13 +573,12 @@ Plan make_plan(int M, int N, int K, int bits) {
     P.splits = splits;
     P.cps = cps;
     P.nsx = P.BN <= 64 ? 6 : (P.BN <= 160 ? 4 : 3);
-    P.nsc = bits == 4 ? 8 : 4;
-    const uint32_t cb = kBM * kBK * bits / 8;
+    P.nsc = P.BN <= 160 ? 4 : 2;                  // code stages of 128 rows x 128 B (+ metadata)
     P.off_x = kNSA * kBM * 128;
     P.off_c = P.off_x + P.nsx * P.BN * 128;
-    P.off_m = P.off_c + P.nsc * cb;
-    P.off_bar = P.off_m + 2 * kBM * kMetaChunks * 4;
-    uint32_t smem = P.off_bar + 8 * (2 * P.nsc + 2 * P.nsx + 2 * kNSA + 4 + 2) + 16 + 1024;
+    P.off_m = P.off_c + P.nsc * kBM * 128;
+    P.off_bar = P.off_m + P.nsc * kBM * kMetaChunks * 4;
+    uint32_t smem = P.off_bar + 8 * (2 * P.nsc + P.nsx + kNSA + kDoneRing + 2) + 16 + 256 + 1024;
     if (smem < 120 * 1024) smem = 120 * 1024;   // at most one CTA per SM: TMEM is never contended
     P.smem = smem;
     uint32_t cols = 32;
@@ -467,15 +623,17 @@ int validate_weight(const flexq_tensor* W) {
 
 // y = epilogue(x W^T + bias); see flex_dequant_gemm. nq/qscale: columns n < nq scaled.
 int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const void* residual, void* y, int M,
-                int relu, int nq, float qscale, void* ws, int64_t ws_bytes, cudaStream_t st) {
+                int relu, int nq, float qscale, bool xperm, bool yperm, void* ws, int64_t ws_bytes, cudaStream_t st,
+                const KvFuse* kv) {
     if (M == 0) return FLEX_OK;
     const int N = static_cast<int>(W->shape[0]), K = static_cast<int>(W->shape[1]);
     const int bits = W->cfg.num_bits;
     const Plan P = make_plan(M, N, K, bits);
     if (P.ws_bytes > 0 && (ws == nullptr || ws_bytes < P.ws_bytes)) return FLEX_ERR_WORKSPACE;
     CUtensorMap tm_codes, tm_meta, tm_x;
+    // code tiles: 128 rows x 128 bytes (4 K chunks at 4 bits, 2 at 8 bits), 128-byte swizzle
     int rc = make_tmap_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, static_cast<uint64_t>(K) * bits / 8,
-                          N, static_cast<uint64_t>(K) * bits / 8, kBK * bits / 8, kBM, CU_TENSOR_MAP_SWIZZLE_NONE);
+                          N, static_cast<uint64_t>(K) * bits / 8, 128, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != FLEX_OK) return rc;
     rc = make_tmap_2d(&tm_meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, W->meta, K / kBK, N,
                       static_cast<uint64_t>(K / kBK) * 4, kMetaChunks, kBM, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -499,6 +657,7 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     gp.nq = nq;
     gp.qscale = qscale;
     gp.relu = relu;
+    gp.yperm = yperm ? 1 : 0;
     gp.nsx = P.nsx;
     gp.nsc = P.nsc;
     gp.off_x = P.off_x;
@@ -506,14 +665,32 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     gp.off_m = P.off_m;
     gp.off_bar = P.off_bar;
     gp.tmem_cols = P.tmem_cols;
-    const dim3 grid(P.tiles_n, P.tiles_m, P.splits);
-    if (bits == 4) {
-        cudaFuncSetAttribute(gemm_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
-        gemm_tc_kernel<4><<<grid, kThreads, P.smem, st>>>(tm_codes, tm_meta, tm_x, gp);
-    } else {
-        cudaFuncSetAttribute(gemm_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
-        gemm_tc_kernel<8><<<grid, kThreads, P.smem, st>>>(tm_codes, tm_meta, tm_x, gp);
+    if (kv != nullptr) {
+        gp.kv_codes[0] = static_cast<uint8_t*>(kv->cache->k_codes);
+        gp.kv_codes[1] = static_cast<uint8_t*>(kv->cache->v_codes);
+        gp.kv_meta[0] = static_cast<uint32_t*>(kv->cache->k_meta);
+        gp.kv_meta[1] = static_cast<uint32_t*>(kv->cache->v_meta);
+        gp.kv_h = kv->h;
+        gp.kv_hd = kv->cache->head_dim;
+        gp.kv_nh = kv->cache->n_heads;
+        gp.kv_max_seq = kv->cache->max_seq;
+        gp.kv_seq = kv->seq;
+        gp.kv_pos0 = kv->pos0;
+        gp.kv_bits = kv->cache->cfg.num_bits;
+        gp.kv_gs = kv->cache->cfg.group_size;
     }
+    const dim3 grid(P.tiles_n, P.tiles_m, P.splits);
+#define GEMM_LAUNCH(B_, XP_)                                                                 \
+    do {                                                                                     \
+        set_smem_once(gemm_tc_kernel<B_, XP_>, 227 * 1024);                                  \
+        launch_k(gemm_tc_kernel<B_, XP_>, grid, dim3(kThreads), P.smem, st, true, tm_codes, tm_meta, tm_x, gp); \
+    } while (0)
+    if (bits == 4) {
+        if (xperm) GEMM_LAUNCH(4, true); else GEMM_LAUNCH(4, false);
+    } else {
+        if (xperm) GEMM_LAUNCH(8, true); else GEMM_LAUNCH(8, false);
+    }
+#undef GEMM_LAUNCH
     return launch_status();
 }
 
@@ -541,5 +718,6 @@ extern "C" int flex_dequant_gemm(const void* x, const flexq_tensor* W, const voi
                  FLEX_ERR_ALIGN);
     FLEX_REQUIRE(ws == nullptr || aligned16(ws), FLEX_ERR_ALIGN);
     return gemm_launch(x, W, bias, epilogue == FLEX_EPI_RESIDUAL ? residual : nullptr, y, M,
-                       epilogue == FLEX_EPI_RELU ? 1 : 0, 0, 1.0f, ws, ws_bytes, as_stream(stream));
+                       epilogue == FLEX_EPI_RELU ? 1 : 0, 0, 1.0f, false, false, ws, ws_bytes, as_stream(stream),
+                       nullptr);
 }

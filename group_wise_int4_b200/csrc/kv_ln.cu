@@ -1,7 +1,7 @@
 // store_cache (flex_append_kv) and LayerNorm.
 //
-// store_cache: FlexGen source-reading notes, "Flex Opt" - the step's new key/value are
-// written to the cache after compute_layer; FlexGen source walkthrough, section 6.3 -
+// store_cache: the source-notes page «FlexGen» (PtirisNote), "Flex Opt" - the step's new key/value are
+// written to the cache after compute_layer; the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南», section 6.3 -
 // with --compress-cache they are stored group-wise quantised, 4 bits, group 64, along
 // the head dimension. The arithmetic is the shared quantiser (quant.cuh), so slot
 // contents equal flexq_compress of the same fp16 values bit for bit.
@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(256) append_kv_kernel(const __half* __restrict
                                                         uint32_t* __restrict__ v_meta, int batch, int seq,
                                                         int n_heads, int head_dim, int max_seq, int pos0) {
     constexpr int L = GS / 8;
+    pdl_wait();
+    pdl_trigger();
     const int gph = head_dim / GS;                              // groups per head
     const int64_t per_tensor = static_cast<int64_t>(batch) * seq * n_heads * gph;
     const int64_t total = 2 * per_tensor;
@@ -84,11 +86,17 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
     return t;
 }
 
+// PERM: write each 8-value block in the interleaved order [x0 x4 x1 x5 x2 x6 x3 x7] that
+// the GEMM's unpack produces for the weights (see gemm.cu), so that the GEMM needs no
+// re-pairing of its dequantised operand.
+template <bool PERM>
 __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const __half* __restrict__ x,
                                                                const __half* __restrict__ g,
                                                                const __half* __restrict__ b,
                                                                __half* __restrict__ y, int h) {
     __shared__ float red[LN_THREADS / 32];
+    pdl_wait();
+    pdl_trigger();
     const int64_t row = blockIdx.x;
     const int nvec = h / 8;
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * h);
@@ -135,7 +143,16 @@ __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const __half* __r
             const float hi = (h2f_hi(w[k]) - mean) * rstd * h2f_hi(gw[k]) + h2f_hi(bw[k]);
             o[k] = pack_half2_bits(__float2half_rn(lo), __float2half_rn(hi));
         }
-        yr[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        if (PERM) {
+            uint32_t t[4];
+            asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(t[0]) : "r"(o[0]), "r"(o[2]));
+            asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(t[1]) : "r"(o[0]), "r"(o[2]));
+            asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(t[2]) : "r"(o[1]), "r"(o[3]));
+            asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(t[3]) : "r"(o[1]), "r"(o[3]));
+            yr[c] = make_uint4(t[0], t[1], t[2], t[3]);
+        } else {
+            yr[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     }
 }
 
@@ -154,9 +171,9 @@ int append_kv_launch(const flex_kv_cache* c, const void* k_new, const void* v_ne
     uint8_t* vc = static_cast<uint8_t*>(c->v_codes);
     uint32_t* km = static_cast<uint32_t*>(c->k_meta);
     uint32_t* vm = static_cast<uint32_t*>(c->v_meta);
-#define APPEND(B, G)                                                                                          \
-    append_kv_kernel<B, G><<<blocks, 256, 0, st>>>(k, v, row_stride, kc, km, vc, vm, batch, seq, c->n_heads, \
-                                                   c->head_dim, c->max_seq, pos0)
+#define APPEND(B, G)                                                                                    \
+    launch_k(append_kv_kernel<B, G>, dim3(blocks), dim3(256), 0, st, true, k, v, row_stride, kc, km, vc, vm, \
+             batch, seq, c->n_heads, c->head_dim, c->max_seq, pos0)
     if (c->cfg.num_bits == 4) {
         if (gs == 32) APPEND(4, 32); else if (gs == 64) APPEND(4, 64); else APPEND(4, 128);
     } else {
@@ -182,12 +199,18 @@ int validate_cache(const flex_kv_cache* c) {
     return FLEX_OK;
 }
 
-int layernorm_launch(const void* x, const void* g, const void* b, void* y, int64_t rows, int h,
+int layernorm_launch(const void* x, const void* g, const void* b, void* y, int64_t rows, int h, bool perm,
                      cudaStream_t st) {
     if (rows == 0) return FLEX_OK;
-    layernorm_kernel<<<static_cast<unsigned>(rows), LN_THREADS, 0, st>>>(
-        static_cast<const __half*>(x), static_cast<const __half*>(g), static_cast<const __half*>(b),
-        static_cast<__half*>(y), h);
+    const __half* xh = static_cast<const __half*>(x);
+    const __half* gh = static_cast<const __half*>(g);
+    const __half* bh = static_cast<const __half*>(b);
+    __half* yh = static_cast<__half*>(y);
+    const dim3 grid(static_cast<unsigned>(rows));
+    if (perm)
+        launch_k(layernorm_kernel<true>, grid, dim3(LN_THREADS), 0, st, true, xh, gh, bh, yh, h);
+    else
+        launch_k(layernorm_kernel<false>, grid, dim3(LN_THREADS), 0, st, true, xh, gh, bh, yh, h);
     return launch_status();
 }
 
@@ -214,5 +237,5 @@ extern "C" int flex_layernorm(const void* x, const void* g, const void* b, void*
     FLEX_REQUIRE(rows >= 0 && h > 0, FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(h % 8 == 0 && h <= LN_THREADS * LN_VPT * 8, FLEX_ERR_UNSUPPORTED);
     FLEX_REQUIRE(aligned16(x) && aligned16(g) && aligned16(b) && aligned16(y), FLEX_ERR_ALIGN);
-    return layernorm_launch(x, g, b, y, rows, h, as_stream(stream));
+    return layernorm_launch(x, g, b, y, rows, h, false, as_stream(stream));
 }

@@ -1,6 +1,6 @@
 // OPT decoder layer: prefill (`mha` path) and decode step (`mha_gen` path).
 //
-// FlexGen source-reading notes, "Flex Opt": per token, layer and gpu-batch the loop
+// the source-notes page «FlexGen» (PtirisNote), "Flex Opt": per token, layer and gpu-batch the loop
 // runs load_weight, load_cache, load_hidden, compute_layer, store_hidden, store_cache;
 // compute_layer is the pre-LayerNorm OPT block. Here everything is resident on one
 // GPU, so loading is a no-op and a layer call is the fixed launch sequence
@@ -16,17 +16,19 @@ namespace flexq {
 
 int validate_cache(const flex_kv_cache* c);
 int validate_weight(const flexq_tensor* W);
-int layernorm_launch(const void* x, const void* g, const void* b, void* y, int64_t rows, int h, cudaStream_t st);
+int layernorm_launch(const void* x, const void* g, const void* b, void* y, int64_t rows, int h, bool perm,
+                     cudaStream_t st);
 int append_kv_launch(const flex_kv_cache* c, const void* k_new, const void* v_new, int64_t row_stride, int batch,
                      int seq, int pos0, cudaStream_t st);
 int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new, const void* v_new,
-                       int64_t row_stride, void* o, int batch, int pos, void* ws, cudaStream_t st);
+                       int64_t row_stride, void* o, int batch, int pos, void* ws, bool perm, cudaStream_t st);
 int64_t decode_attn_ws_bound(int pairs, int head_dim);
 int prefill_attn_launch(const void* q, const void* k, const void* v, int64_t row_stride, void* o, int batch,
                         int seq, int n_heads, int head_dim, cudaStream_t st);
 int64_t gemm_ws_bytes(int M, int N, int K, int bits);
 int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const void* residual, void* y, int M,
-                int relu, int nq, float qscale, void* ws, int64_t ws_bytes, cudaStream_t st);
+                int relu, int nq, float qscale, bool xperm, bool yperm, void* ws, int64_t ws_bytes, cudaStream_t st,
+                const KvFuse* kv);
 
 namespace {
 
@@ -105,20 +107,28 @@ int run_layer(const flex_layer* L, const flex_kv_cache* C, const void* x_in, voi
     const int M = static_cast<int>(T);
     const int h = L->h;
     const float qscale = 1.0f / sqrtf(static_cast<float>(L->head_dim));
-    int rc = layernorm_launch(x_in, L->ln1_g, L->ln1_b, a, T, h, st);
-    if (rc == FLEX_OK) rc = gemm_launch(a, &L->w_qkv, L->b_qkv, nullptr, qkv, M, 0, h, qscale, gws, w.gemm_bytes, st);
+    // a, a2, f and the decode attention output are written in the interleaved 8-block
+    // order that the GEMM's unpack produces for its weights (see gemm.cu); h1, qkv and
+    // the prefill attention output stay in natural order.
+    const bool dec = (seq == 1);
+    // the QKV epilogue also quantises the new keys/values into their cache slots
+    // (store_cache): slot pos for a decode step, slots [0, seq) for a prompt
+    const KvFuse kv{C, h, seq, dec ? pos : 0};
+    int rc = layernorm_launch(x_in, L->ln1_g, L->ln1_b, a, T, h, true, st);
+    if (rc == FLEX_OK)
+        rc = gemm_launch(a, &L->w_qkv, L->b_qkv, nullptr, qkv, M, 0, h, qscale, true, false, gws, w.gemm_bytes, st, &kv);
     if (rc != FLEX_OK) return rc;
-    if (seq == 1) {
-        rc = decode_attn_launch(C, qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, pos, base + w.attn, st);
-        if (rc == FLEX_OK) rc = append_kv_launch(C, qkv + h, qkv + 2 * h, 3LL * h, batch, 1, pos, st);
-    } else {
+    if (dec)
+        rc = decode_attn_launch(C, qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, pos, base + w.attn, true, st);
+    else
         rc = prefill_attn_launch(qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, seq, L->n_heads, L->head_dim, st);
-        if (rc == FLEX_OK) rc = append_kv_launch(C, qkv + h, qkv + 2 * h, 3LL * h, batch, seq, 0, st);
-    }
-    if (rc == FLEX_OK) rc = gemm_launch(o, &L->w_o, L->b_o, x_in, h1, M, 0, 0, 1.f, gws, w.gemm_bytes, st);
-    if (rc == FLEX_OK) rc = layernorm_launch(h1, L->ln2_g, L->ln2_b, a2, T, h, st);
-    if (rc == FLEX_OK) rc = gemm_launch(a2, &L->w_fc1, L->b_fc1, nullptr, f, M, 1, 0, 1.f, gws, w.gemm_bytes, st);
-    if (rc == FLEX_OK) rc = gemm_launch(f, &L->w_fc2, L->b_fc2, h1, x_out, M, 0, 0, 1.f, gws, w.gemm_bytes, st);
+    if (rc == FLEX_OK)
+        rc = gemm_launch(o, &L->w_o, L->b_o, x_in, h1, M, 0, 0, 1.f, dec, false, gws, w.gemm_bytes, st, nullptr);
+    if (rc == FLEX_OK) rc = layernorm_launch(h1, L->ln2_g, L->ln2_b, a2, T, h, true, st);
+    if (rc == FLEX_OK)
+        rc = gemm_launch(a2, &L->w_fc1, L->b_fc1, nullptr, f, M, 1, 0, 1.f, true, true, gws, w.gemm_bytes, st, nullptr);
+    if (rc == FLEX_OK)
+        rc = gemm_launch(f, &L->w_fc2, L->b_fc2, h1, x_out, M, 0, 0, 1.f, true, false, gws, w.gemm_bytes, st, nullptr);
     return rc;
 }
 

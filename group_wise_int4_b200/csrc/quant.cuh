@@ -2,7 +2,7 @@
 // (compression, store_cache, the fused QKV epilogue) so that all of them produce the
 // same bits.
 //
-// FlexGen source walkthrough, section 6.3: per group of group_size values along
+// the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南», section 6.3: per group of group_size values along
 // group_dim keep {min, scale} with an fp16 scale and store unsigned num_bits codes;
 // q = round((x - min) * (2^b - 1) / (max - min)).  Every fp32 operation below is an
 // explicitly rounded intrinsic, so the compiler cannot contract or reorder it.

@@ -27,14 +27,18 @@ __device__ __forceinline__ void bar_arrive(uint32_t bar) {
 __device__ __forceinline__ void bar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
+// try_wait with a suspend-time hint: a waiting thread sleeps (up to the hint, in ns)
+// until the phase completes instead of spinning and taking issue slots from the
+// warps that do the work.
+constexpr uint32_t kSuspendHintNs = 200000;
 __device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -44,22 +48,28 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-// Wait for the phase of `bar` with the given parity to complete. Gives up after
-// kWaitLimitNs (or at once when *abort is set by another role of the CTA): then it
-// records FLEX_ERR_TIMEOUT in the device status word, raises *abort and returns false.
+// Wait for the phase of `bar` with the given parity to complete. The common path is a
+// try_wait loop (each try_wait sleeps until the phase completes or the hint runs out);
+// every 16 polls it checks *abort (raised by another role of the CTA) and the elapsed
+// time.
+// After kWaitLimitNs it records FLEX_ERR_TIMEOUT in the device status word, raises
+// *abort and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
     if (bar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 64; ++i)
-            if (bar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort = 1;
-            set_status(status, FLEX_ERR_TIMEOUT);
-            return false;
+    uint64_t t0 = 0;
+    for (uint32_t n = 1;; ++n) {
+        if (bar_try_wait(bar, parity)) return true;
+        if ((n & 15u) == 0) {
+            if (*abort) return false;
+            const uint64_t t = globaltimer_ns();
+            if (t0 == 0) {
+                t0 = t;
+            } else if (t - t0 > kWaitLimitNs) {
+                *abort = 1;
+                set_status(status, FLEX_ERR_TIMEOUT);
+                return false;
+            }
         }
     }
 }

@@ -70,6 +70,25 @@ def test_gemm_8bit_no_bias(M, N, K):
     assert_layer_close(y, _oracle_gemm(x, w, None, None, fq.FLEX_EPI_NONE, 8), "8-bit")
 
 
+@pytest.mark.parametrize("M,N,K", [(32, 19200, 4096), (512, 9472, 2048), (144, 19200, 2048)])
+def test_gemm_ring_reuse(M, N, K):
+    """Enough tiles for a single K split, so every shared-memory ring wraps around
+    several times (the code/metadata stages, the activation and the dequantised rings)."""
+    x = synth.activations((M, K), 60, device="cuda")
+    w = synth.normal_f16((N, K), 61, 0.02, device="cuda")
+    b = synth.normal_f16((N,), 62, 0.02, device="cuda")
+    W = fq.CompressedWeight(w, 4, 64)
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    ws = torch.zeros(max(16, fq.flex_gemm_ws_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
+    fq.flex_dequant_gemm(x, W, b, None, y, M, 0, ws)
+    sync_status()
+    rows = np.array([0, 1, 127, 128, 5000 % N, N - 129, N - 1])
+    mrows = np.unique(np.array([0, M // 2, M - 1]))
+    ref = _oracle_gemm(to_np(x[torch.from_numpy(mrows).cuda()]), to_np(w), to_np(b), None, 0, 4, rows=rows)
+    got = y[torch.from_numpy(mrows).cuda()][:, torch.from_numpy(rows).cuda()]
+    assert_layer_close(got, ref, f"ring reuse {M}x{N}x{K}")
+
+
 def test_gemm_repeatable_and_workspace_left_clean():
     """Split-K reduces in a fixed order: two calls give identical bits; the
     workspace's tickets are back to zero after each call."""

@@ -1,6 +1,6 @@
 """Pins of the oracle quantiser against what the pages and the mathematics fix.
 
-Sources: FlexGen source walkthrough, section 6.3 (configuration, packed shape, fp16
+Sources: the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南», section 6.3 (configuration, packed shape, fp16
 scale, "about 70% less weight memory"); the min/max formula of the method. None of
 these tests re-types the oracle's own formula: they check hand-worked values,
 closed forms, bounds, exact-rational brute force and layout invariants.

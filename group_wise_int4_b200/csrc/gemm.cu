@@ -33,8 +33,13 @@ namespace {
 
 constexpr int kBM = 128;           // weight rows per CTA (MMA M)
 constexpr int kBK = 64;            // K per stage = one quantisation group
-constexpr int kThreads = 384;      // 12 warps
-constexpr int kDequantThreads = 256;
+// 14 warps. Warps 0-3: code TMA, activation TMA, MMA issue, spare. Dequantisation: the 8
+// warps 4, 5, 7, 8, 9, 11, 12, 13 - none on the MMA warp's SM sub-partition (warp % 4 ==
+// 2), so the single MMA-issuing thread is never starved of issue slots. Epilogue: warps
+// 4-11 (each TMEM lane quarter needs warps with warp % 4 equal to it).
+constexpr int kThreads = 448;
+constexpr int kTeamThreads = 256;
+constexpr int kDequantThreads = kTeamThreads;
 constexpr int kNSA = 4;            // dequantised A stages
 constexpr int kMetaChunks = 4;     // groups per metadata tile
 constexpr int kDoneRing = 8;       // mma_done barriers (>= kNSA and >= every activation ring depth)
@@ -353,17 +358,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         __syncwarp();
     } else if (warp >= 4) {
         // ---------------- dequantisation ----------------
-        // thread (row, half): for every K chunk, half of the row's codes (16 code bytes at
-        // 4 bits, 32 at 8 bits) -> 32 fp16 = 4 of the row's 8 16-byte chunks of A
-        const int dt = threadIdx.x - 128;
+        // thread (row, half) turns half of the row's codes of a K chunk (16 code bytes at
+        // 4 bits, 32 at 8 bits) into 32 fp16 = 4 of the row's 8 16-byte units of A; the
+        // chunks of a code stage are unpacked in pairs behind one proxy fence.
+        const bool deq = (warp < 14) && ((warp & 3) != 2);
+        const int rank = (warp - 4) - (warp > 6) - (warp > 10);       // 0..7 for the dequant warps
+        const int dt = rank * 32 + lane;
         const int row = dt & 127, half_ = dt >> 7;
         const int sw = row & 7;
+        constexpr int CPP = CPS >= 2 ? 2 : 1;           // chunks per fence
         bool ok = true;
-        int i = 0;                                  // K chunk index within the split
-        for (int st = 0; st < nstages && ok; ++st) {
+        for (int st = 0; deq && st < nstages && ok; ++st) {
             const int s = st % NSC;
             if (!tc::bar_wait(B.codes_full + 8 * s, (st / NSC) & 1, abort, p.status)) { ok = false; break; }
-            // codes of this stage (the tile was stored with the 128-byte swizzle: 16-byte
+            // codes of the stage (the tile was stored with the 128-byte swizzle: 16-byte
             // unit u of row r sits at unit u ^ (r % 8))
             const uint8_t* crow = gbase + (sC - base) + s * CSTAGE + row * 128;
             uint4 cw[CPS][BITS / 4];
@@ -378,55 +386,65 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const uint32_t mwv[4] = {mrow.x, mrow.y, mrow.z, mrow.w};
             const int moff = (c_begin + st * CPS) & (kMetaChunks - 1);
 #pragma unroll
-            for (int c = 0; c < CPS; ++c, ++i) {
-                const uint32_t mw = mwv[(moff + c) & 3];
-                const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
-                const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
-                // step = fp16(1/scale); a constant group (scale 0) gets step 0 and decodes to min
-                const __half step = __float2half_rn(sc32 > 0.f ? __frcp_rn(sc32) : 0.f);
-                const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
-                const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
-                const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
-                const int sa = i % kNSA;
-                // slot sa last held chunk i - kNSA: wait until its MMAs are done
-                if (i >= kNSA) {
-                    const int pc = i - kNSA;
-                    if (!tc::bar_wait(B.mma_done + 8 * (pc % kDoneRing), (pc / kDoneRing) & 1, abort, p.status)) {
-                        ok = false;
-                        break;
+            for (int c0 = 0; c0 < CPS; c0 += CPP) {
+                // the A slots of these chunks must have been consumed by the MMAs
+#pragma unroll
+                for (int c = c0; c < c0 + CPP; ++c) {
+                    const int i = st * CPS + c;
+                    if (i >= kNSA) {
+                        const int pc = i - kNSA;
+                        if (!tc::bar_wait(B.mma_done + 8 * (pc % kDoneRing), (pc / kDoneRing) & 1, abort, p.status))
+                            ok = false;
                     }
                 }
-                uint8_t* arow = gbase + sa * (kBM * 128) + row * 128;
-                if (BITS == 4) {
-                    const uint32_t w[4] = {cw[c][0].x, cw[c][0].y, cw[c][0].z, cw[c][0].w};
+                if (!ok) break;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2) : dequant8_4bit(w[j], step2, mnv2);
-                        *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = v;
-                    }
-                } else {
-                    const uint4 c0 = cw[c][0], c1 = cw[c][BITS / 4 - 1];
-                    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                for (int c = c0; c < c0 + CPP; ++c) {
+                    const int i = st * CPS + c;
+                    const uint32_t mw = mwv[(moff + c) & 3];
+                    const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
+                    const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
+                    // step = fp16(1/scale); a constant group (scale 0) gets step 0 and decodes to min
+                    const __half step = __float2half_rn(sc32 > 0.f ? __frcp_rn(sc32) : 0.f);
+                    const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
+                    const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
+                    const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
+                    uint8_t* arow = gbase + (i % kNSA) * (kBM * 128) + row * 128;
+                    if (BITS == 4) {
+                        const uint32_t w[4] = {cw[c][0].x, cw[c][0].y, cw[c][0].z, cw[c][0].w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint4 v;
-                        if (XPERM) {
-                            v = dequant8_8bit_il(w[2 * j], w[2 * j + 1], step2, mnv2);
-                        } else {
-                            const uint2 a = dequant4_8bit(w[2 * j], step2, mnv2);
-                            const uint2 b = dequant4_8bit(w[2 * j + 1], step2, mnv2);
-                            v = make_uint4(a.x, a.y, b.x, b.y);
+                        for (int j = 0; j < 4; ++j) {
+                            const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2) : dequant8_4bit(w[j], step2, mnv2);
+                            *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = v;
                         }
-                        *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = v;
+                    } else {
+                        const uint4 q0 = cw[c][0], q1 = cw[c][BITS / 4 - 1];
+                        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint4 v;
+                            if (XPERM) {
+                                v = dequant8_8bit_il(w[2 * j], w[2 * j + 1], step2, mnv2);
+                            } else {
+                                const uint2 a = dequant4_8bit(w[2 * j], step2, mnv2);
+                                const uint2 b = dequant4_8bit(w[2 * j + 1], step2, mnv2);
+                                v = make_uint4(a.x, a.y, b.x, b.y);
+                            }
+                            *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = v;
+                        }
                     }
                 }
                 tc::fence_proxy_async_smem();
-                tc::bar_arrive(B.a_full + 8 * sa);
+#pragma unroll
+                for (int c = c0; c < c0 + CPP; ++c) tc::bar_arrive(B.a_full + 8 * ((st * CPS + c) % kNSA));
             }
             // release the code stage only once all of its values have been consumed (the
             // next TMA into this slot must not overtake these shared-memory reads)
             if (ok) tc::bar_arrive(B.codes_empty + 8 * s);
         }
+        if (warp >= 12) {
+            // not an epilogue warp
+        } else {
         // ---------------- epilogue ----------------
         pdl_trigger();                            // dependents may start their prologue
         const int lq = warp & 3, ch = (warp - 4) >> 2;
@@ -520,6 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 }
             }
         }
+    }
     }
 
     tc::fence_before_sync();

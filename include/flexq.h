@@ -2,13 +2,13 @@
  * flexq.h - C ABI of the B200 (sm_100a) group-wise int4 OPT layer library.
  *
  * What it computes comes from the FlexGen pages:
- *   - FlexGen source walkthrough, section 6.3 "4-bit group-wise quantisation of
+ *   - the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南», section 6.3 "4-bit group-wise quantisation of
  *     weights and KV cache": CompressionConfig(num_bits, group_size, group_dim,
  *     symmetric), compress / decompress, two 4-bit codes per uint8 in a data tensor of
  *     shape shape[:group_dim] + (num_groups*(group_size//2),) + shape[group_dim+1:],
  *     and an fp16 per-group scale tensor; weights use (4, 64) and the KV cache
  *     (4, 64) grouped along the head dimension.
- *   - FlexGen source-reading notes, "Pytorch Backend": prefill attention is `mha`,
+ *   - the source-notes page «FlexGen» (PtirisNote), "Pytorch Backend": prefill attention is `mha`,
  *     the decode step is `mha_gen`; "Flex Opt": every step runs load_cache,
  *     compute_layer, store_cache, in that order.
  *

@@ -8,12 +8,12 @@ no code, header, table or helper with the CUDA library under
 
 Sources (the web pages on FlexGen's group-wise int4 method):
 
-* FlexGen source walkthrough, section 6.3 "4-bit group-wise quantisation of weights
+* the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南», section 6.3 "4-bit group-wise quantisation of weights
   and KV cache": the compression configuration (num_bits 4, group_size 64,
   group_dim 0 for weights and 2 for the cache, asymmetric), the packed data shape
   ``shape[:group_dim] + (num_groups * (group_size // 2),) + shape[group_dim+1:]``
   with two 4-bit codes per uint8, and a per-group fp16 scale tensor.
-* FlexGen source-reading notes, "Pytorch Backend" and "Flex Opt": prefill attention
+* the source-notes page «FlexGen» (PtirisNote), "Pytorch Backend" and "Flex Opt": prefill attention
   is ``mha``, the decode step is ``mha_gen``; the generation loop runs load_cache,
   compute_layer and then store_cache, so a decode step attends to the cache of the
   earlier tokens plus its own fresh key and value, and its own key/value are

@@ -1,6 +1,6 @@
 """Group-wise asymmetric min/max quantiser (oracle; test infrastructure only).
 
-Statement followed: FlexGen source walkthrough, section 6.3 - ``compress`` splits a
+Statement followed: the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南», section 6.3 - ``compress`` splits a
 tensor along ``group_dim`` into groups of ``group_size`` elements, keeps per group a
 fp16 scale, and stores ``num_bits``-bit unsigned codes, two 4-bit codes per uint8,
 in a data tensor of shape

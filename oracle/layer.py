@@ -1,10 +1,10 @@
 """OPT decoder layer, prefill (``mha``) and decode step (``mha_gen``) - oracle; test
 infrastructure only.
 
-Statement followed: FlexGen source-reading notes, "Pytorch Backend" (``mha`` is the
+Statement followed: the source-notes page «FlexGen» (PtirisNote), "Pytorch Backend" (``mha`` is the
 prefill attention, ``mha_gen`` the decode attention) and "Flex Opt" (each
 generation step runs load_cache, compute_layer, store_cache, so the key/value of
-the current token are stored after the layer has run); FlexGen source walkthrough,
+the current token are stored after the layer has run); the walkthrough page «FlexGen 单 GPU 高吞吐大模型推理引擎：论文解读与源码实战指南»,
 section 6.3 (the KV cache is compressed with 4 bits, group 64, grouped along the
 head dimension). The layer itself is the OPT pre-LayerNorm block:
 

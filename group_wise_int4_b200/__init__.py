@@ -28,6 +28,9 @@ FLEX_ERR_ALIGN = -4
 FLEX_ERR_WORKSPACE = -5
 FLEX_ERR_CUDA = -6
 FLEX_ERR_TIMEOUT = -7
+FLEX_ERR_SCRATCH_LIMIT = -8
+
+FLEX_DECODE_ATTENTION_STATIC_MAX_BYTES = 8 << 20
 
 FLEX_EPI_NONE = 0
 FLEX_EPI_RELU = 1
@@ -84,6 +87,8 @@ _SIGS = {
     "flex_decode_attention_ws_bytes": (_I64, [ctypes.POINTER(flex_kv_cache), _I32, _I32]),
     "flex_decode_attention": (_I32, [ctypes.POINTER(flex_kv_cache), _P, _P, _P, _I64, _P, _I32, _I32,
                                      _P, _I64, _P]),
+    "flex_decode_attention_noalloc": (_I32, [ctypes.POINTER(flex_kv_cache), _P, _P, _P, _I64, _P, _I32,
+                                             _I32, _P]),
     "flex_prefill_attention": (_I32, [_P, _P, _P, _I64, _P, _I32, _I32, _I32, _I32, _P]),
     "flex_gemm_ws_bytes": (_I64, [_I32, _I32, _I32]),
     "flex_dequant_gemm": (_I32, [_P, ctypes.POINTER(flexq_tensor), _P, _P, _P, _I32, _I32, _P, _I64, _P]),
@@ -323,6 +328,16 @@ def flex_decode_attention(cache: FlexKVCache, q, k_new, v_new, row_stride, o, ba
                                      int(ws.numel() * ws.element_size()) if ws is not None else 0,
                                      ctypes.c_void_p(_stream(stream)))
     _check(rc, "flex_decode_attention")
+
+
+def flex_decode_attention_noalloc(cache: FlexKVCache, q, k_new, v_new, row_stride, o, batch, pos,
+                                  stream=None):
+    """flex_decode_attention with the library's built-in scratch instead of a workspace
+    (no device allocation; calls that may overlap on one device race on that scratch)."""
+    rc = lib().flex_decode_attention_noalloc(ctypes.byref(cache.struct()), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                             int(row_stride), _ptr(o), int(batch), int(pos),
+                                             ctypes.c_void_p(_stream(stream)))
+    _check(rc, "flex_decode_attention_noalloc")
 
 
 def flex_prefill_attention(q, k, v, row_stride, o, batch, seq, n_heads, head_dim, stream=None):

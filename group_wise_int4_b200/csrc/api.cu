@@ -87,6 +87,7 @@ extern "C" const char* flex_status_string(int32_t status) {
         case FLEX_ERR_WORKSPACE: return "workspace missing or too small";
         case FLEX_ERR_CUDA: return "CUDA error";
         case FLEX_ERR_TIMEOUT: return "device wait timed out";
+        case FLEX_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the built-in buffer holds";
         default: return "unknown status";
     }
 }

@@ -18,6 +18,8 @@
 // fp32 accumulation), online softmax in registers.
 #include <float.h>
 
+#include <mutex>
+
 #include "quant.cuh"
 
 namespace flexq {
@@ -1130,4 +1132,56 @@ extern "C" int flex_prefill_attention(const void* q, const void* k, const void* 
                  FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(o), FLEX_ERR_ALIGN);
     return prefill_attn_launch(q, k, v, row_stride, o, batch, seq, n_heads, head_dim, as_stream(stream));
+}
+
+// ---- decode attention with library-owned scratch ---------------------------------------
+//
+// Same kernels and launch as flex_decode_attention; only the split-KV partials live in a
+// buffer inside this library instead of a caller-supplied workspace, so the call itself
+// allocates nothing. Every partial the combine kernel reads is written earlier in the same
+// call by the split kernel, so the buffer needs no clearing, at load time or between calls.
+namespace flexq {
+namespace {
+
+constexpr int64_t kDecodeScratchBytes = FLEX_DECODE_ATTENTION_STATIC_MAX_BYTES;
+__device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+constexpr int kScratchDevices = 64;
+void* g_decode_scratch_ptr[kScratchDevices];
+std::mutex g_decode_scratch_mu;
+
+// Device address of this device's copy of g_decode_scratch, looked up on the first call
+// made with the device current and cached for the life of the process. nullptr if the
+// lookup fails.
+void* decode_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kScratchDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_decode_scratch_mu);
+    if (g_decode_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        g_decode_scratch_ptr[dev] = p;
+    }
+    return g_decode_scratch_ptr[dev];
+}
+
+}  // namespace
+}  // namespace flexq
+
+extern "C" int flex_decode_attention_noalloc(const flex_kv_cache* cache, const void* q, const void* k_new,
+                                             const void* v_new, int64_t row_stride, void* o, int32_t batch,
+                                             int32_t pos, void* stream) {
+    const int rc = validate_cache(cache);
+    if (rc != FLEX_OK) return rc;
+    FLEX_REQUIRE(q && k_new && v_new && o, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(batch > 0 && batch <= cache->batch, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(pos >= 0 && pos < cache->max_seq, FLEX_ERR_SHAPE);
+    FLEX_REQUIRE(row_stride >= static_cast<int64_t>(cache->n_heads) * cache->head_dim, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(aligned16(q) && aligned16(k_new) && aligned16(v_new) && aligned16(o), FLEX_ERR_ALIGN);
+    const int64_t need = decode_attn_ws_bytes(batch * cache->n_heads, cache->head_dim, pos);
+    FLEX_REQUIRE(need <= kDecodeScratchBytes, FLEX_ERR_SCRATCH_LIMIT);
+    void* scratch = decode_scratch();
+    FLEX_REQUIRE(scratch != nullptr, FLEX_ERR_CUDA);
+    return decode_attn_launch(cache, q, k_new, v_new, row_stride, o, batch, pos, scratch, false,
+                              as_stream(stream));
 }

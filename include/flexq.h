@@ -48,6 +48,9 @@ extern "C" {
 #define FLEX_ERR_WORKSPACE   (-5)  /* workspace missing or too small              */
 #define FLEX_ERR_CUDA        (-6)  /* a CUDA launch or runtime call failed        */
 #define FLEX_ERR_TIMEOUT     (-7)  /* a device-side bounded wait gave up          */
+#define FLEX_ERR_SCRATCH_LIMIT (-8) /* problem needs more scratch than the library's
+                                       built-in buffer holds (see
+                                       flex_decode_attention_noalloc)             */
 
 /* ---- compression configuration (CompressionConfig of section 6.3) ------------ */
 typedef struct {
@@ -162,6 +165,31 @@ int64_t flex_decode_attention_ws_bytes(const flex_kv_cache* cache, int32_t batch
 int flex_decode_attention(const flex_kv_cache* cache, const void* q, const void* k_new,
                           const void* v_new, int64_t row_stride, void* o, int32_t batch,
                           int32_t pos, void* ws, int64_t ws_bytes, void* stream);
+
+/* Decode attention that allocates nothing and takes no workspace. The pages have no
+ * counterpart: it is a library convenience for callers that cannot hand over device
+ * memory, e.g. a plain C host program that owns only the cache and activation buffers
+ * and has no device allocator, or an out-of-memory handler that must make progress
+ * when no more device memory can be had. Arguments, layouts and results are those of
+ * flex_decode_attention; the split-KV partials go to a buffer compiled into the
+ * library (FLEX_DECODE_ATTENTION_STATIC_MAX_BYTES per device, held for the life of
+ * the process once the library's device code is loaded).
+ *   - Limit: a call whose partials, flex_decode_attention_ws_bytes(cache, batch, pos),
+ *     exceed FLEX_DECODE_ATTENTION_STATIC_MAX_BYTES returns FLEX_ERR_SCRATCH_LIMIT and
+ *     launches nothing (8 MiB covers e.g. 144 sequences x 96 heads of 128).
+ *   - Set-up: the first call on a device, made with that device current, looks up the
+ *     buffer's device address with a CUDA runtime query (with lazy module loading the
+ *     driver may load the library's device code, buffer included, at that moment);
+ *     make that first call before any stream capture begins on the device.
+ *   - Nothing in the buffer has to start at zero: each call writes every partial it
+ *     reads.
+ *   - One buffer per device, shared by all calls: two calls on one device that may run
+ *     at the same time (different streams with no ordering between them) race on it and
+ *     give wrong results. Calls issued on one stream are ordered and safe. */
+#define FLEX_DECODE_ATTENTION_STATIC_MAX_BYTES (8LL << 20)
+int flex_decode_attention_noalloc(const flex_kv_cache* cache, const void* q, const void* k_new,
+                                  const void* v_new, int64_t row_stride, void* o, int32_t batch,
+                                  int32_t pos, void* stream);
 
 /* Prefill attention (`mha` core): causal softmax attention on fresh fp16 q, k, v,
  * each [batch][seq][n_heads][head_dim] inside rows of `row_stride` elements per

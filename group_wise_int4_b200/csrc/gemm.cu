@@ -57,6 +57,11 @@ struct GemmParams {
     int nq;                // columns n < nq are multiplied by qscale
     float qscale;
     int relu;
+    // weights may be read before the previous kernel on the stream has completed: set
+    // only by the layer calls, whose kernels never write weights (every kernel of this
+    // library signals its dependents only after its own wait, so everything before the
+    // immediately preceding kernel is complete whenever this grid runs)
+    int early_w;
     int yperm;             // write y in the interleaved 8-block order
     int nsx, nsc;          // activation / code ring depths
     uint32_t off_x, off_c, off_m, off_bar;
@@ -274,11 +279,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();                                   // the activations come from the previous kernel
+    // Dependencies on the previous kernel (programmatic dependent launch): the
+    // activation producer and the epilogue wait for it before touching global memory;
+    // the code producer also waits unless early_w; the MMA and dequant roles only touch
+    // shared memory and TMEM.
 
     if (warp == 0) {
         // ---------------- code + metadata producer: one stage = CPS chunks ----------------
         if (lane == 0) {
+            if (!p.early_w) pdl_wait();
             int st = 0;
             for (; st < nstages; ++st) {
                 const int s = st % NSC;
@@ -299,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     } else if (warp == 1) {
         // ---------------- activation producer ----------------
         if (lane == 0) {
+            pdl_wait();                           // the activations come from the previous kernel
             int i = 0;
             for (; i < nk; ++i) {
                 const int s = i % NSX;
@@ -446,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             // not an epilogue warp
         } else {
         // ---------------- epilogue ----------------
+        pdl_wait();                               // residual, bias, y and workspace
         pdl_trigger();                            // dependents may start their prologue
         const int lq = warp & 3, ch = (warp - 4) >> 2;
         const int irow = lq * 32 + lane;
@@ -643,7 +654,7 @@ int validate_weight(const flexq_tensor* W) {
 // y = epilogue(x W^T + bias); see flex_dequant_gemm. nq/qscale: columns n < nq scaled.
 int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const void* residual, void* y, int M,
                 int relu, int nq, float qscale, bool xperm, bool yperm, void* ws, int64_t ws_bytes, cudaStream_t st,
-                const KvFuse* kv) {
+                const KvFuse* kv, bool early_w) {
     if (M == 0) return FLEX_OK;
     const int N = static_cast<int>(W->shape[0]), K = static_cast<int>(W->shape[1]);
     const int bits = W->cfg.num_bits;
@@ -676,6 +687,7 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     gp.nq = nq;
     gp.qscale = qscale;
     gp.relu = relu;
+    gp.early_w = early_w ? 1 : 0;
     gp.yperm = yperm ? 1 : 0;
     gp.nsx = P.nsx;
     gp.nsc = P.nsc;
@@ -738,5 +750,5 @@ extern "C" int flex_dequant_gemm(const void* x, const flexq_tensor* W, const voi
     FLEX_REQUIRE(ws == nullptr || aligned16(ws), FLEX_ERR_ALIGN);
     return gemm_launch(x, W, bias, epilogue == FLEX_EPI_RESIDUAL ? residual : nullptr, y, M,
                        epilogue == FLEX_EPI_RELU ? 1 : 0, 0, 1.0f, false, false, ws, ws_bytes, as_stream(stream),
-                       nullptr);
+                       nullptr, false);
 }

@@ -28,7 +28,7 @@ int prefill_attn_launch(const void* q, const void* k, const void* v, int64_t row
 int64_t gemm_ws_bytes(int M, int N, int K, int bits);
 int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const void* residual, void* y, int M,
                 int relu, int nq, float qscale, bool xperm, bool yperm, void* ws, int64_t ws_bytes, cudaStream_t st,
-                const KvFuse* kv);
+                const KvFuse* kv, bool early_w);
 
 namespace {
 
@@ -116,19 +116,19 @@ int run_layer(const flex_layer* L, const flex_kv_cache* C, const void* x_in, voi
     const KvFuse kv{C, h, seq, dec ? pos : 0};
     int rc = layernorm_launch(x_in, L->ln1_g, L->ln1_b, a, T, h, true, st);
     if (rc == FLEX_OK)
-        rc = gemm_launch(a, &L->w_qkv, L->b_qkv, nullptr, qkv, M, 0, h, qscale, true, false, gws, w.gemm_bytes, st, &kv);
+        rc = gemm_launch(a, &L->w_qkv, L->b_qkv, nullptr, qkv, M, 0, h, qscale, true, false, gws, w.gemm_bytes, st, &kv, true);
     if (rc != FLEX_OK) return rc;
     if (dec)
         rc = decode_attn_launch(C, qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, pos, base + w.attn, true, st);
     else
         rc = prefill_attn_launch(qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, seq, L->n_heads, L->head_dim, st);
     if (rc == FLEX_OK)
-        rc = gemm_launch(o, &L->w_o, L->b_o, x_in, h1, M, 0, 0, 1.f, dec, false, gws, w.gemm_bytes, st, nullptr);
+        rc = gemm_launch(o, &L->w_o, L->b_o, x_in, h1, M, 0, 0, 1.f, dec, false, gws, w.gemm_bytes, st, nullptr, true);
     if (rc == FLEX_OK) rc = layernorm_launch(h1, L->ln2_g, L->ln2_b, a2, T, h, true, st);
     if (rc == FLEX_OK)
-        rc = gemm_launch(a2, &L->w_fc1, L->b_fc1, nullptr, f, M, 1, 0, 1.f, true, true, gws, w.gemm_bytes, st, nullptr);
+        rc = gemm_launch(a2, &L->w_fc1, L->b_fc1, nullptr, f, M, 1, 0, 1.f, true, true, gws, w.gemm_bytes, st, nullptr, true);
     if (rc == FLEX_OK)
-        rc = gemm_launch(f, &L->w_fc2, L->b_fc2, h1, x_out, M, 0, 0, 1.f, true, false, gws, w.gemm_bytes, st, nullptr);
+        rc = gemm_launch(f, &L->w_fc2, L->b_fc2, h1, x_out, M, 0, 0, 1.f, true, false, gws, w.gemm_bytes, st, nullptr, true);
     return rc;
 }
 

@@ -7,14 +7,21 @@
 // K, so a 64-wide K chunk is exactly one group per row. The kernel never materialises
 // W^ in global memory:
 //
-//   warp 0      TMA: int4 code tiles [128 rows][32 B] and metadata tiles
-//               [128 rows][4 groups] into shared-memory rings
-//   warp 1      TMA: activation tiles [BN rows][64] fp16 with the 128-byte swizzle
-//   warp 2      allocates the TMEM accumulator and issues tcgen05.mma (one thread)
-//   warps 4-11  unpack the codes in shared memory to fp16 (q*step + min, one half2 FMA
-//               per pair) in the canonical K-major 128-byte-swizzled layout, then run
-//               the epilogue from TMEM (bias, 1/sqrt(d) on the query columns, ReLU,
-//               residual, fp16 store)
+//   warp 0      TMA: code tiles [128 rows][128 B] (one step = 4 K chunks at 4 bits, 2
+//               at 8 bits) and metadata tiles [128 rows][4 groups] into a shared ring
+//   warp 1      TMA: activation tiles [BN rows][64] fp16 with the 128-byte swizzle, a
+//               step (or half a step for BN > 128) per stage
+//   warp 2      allocates all 512 TMEM columns and issues tcgen05.mma (one thread):
+//               A (the dequantised weights) from TMEM, B (activations) from shared
+//               memory, one wait and one commit per step
+//   warps 4-11  unpack the codes to fp16 (q*step + min, one half2 FMA per pair) and
+//               store them into the step's A slot in TMEM (tcgen05.st), then run the
+//               epilogue from the TMEM accumulator (bias, 1/sqrt(d) on the query
+//               columns, ReLU, residual, fp16 store, fused store_cache)
+//
+// TMEM: columns [0, 256) hold the fp32 accumulator (BN <= 256 columns), [256, 512) the
+// A slots (two steps at 4 bits), so dequantisation of step j+1 overlaps the MMAs of
+// step j and the dequantised weights never go through shared memory.
 //
 // Swap-AB orientation: the weight rows are the MMA's M side (128 per CTA) and the
 // activation rows (batch in decode, tokens in prefill) its N side (BN = 16..256), so a
@@ -33,16 +40,16 @@ namespace {
 
 constexpr int kBM = 128;           // weight rows per CTA (MMA M)
 constexpr int kBK = 64;            // K per stage = one quantisation group
-// 14 warps. Warps 0-3: code TMA, activation TMA, MMA issue, spare. Dequantisation: the 8
-// warps 4, 5, 7, 8, 9, 11, 12, 13 - none on the MMA warp's SM sub-partition (warp % 4 ==
-// 2), so the single MMA-issuing thread is never starved of issue slots. Epilogue: warps
-// 4-11 (each TMEM lane quarter needs warps with warp % 4 equal to it).
-constexpr int kThreads = 448;
-constexpr int kTeamThreads = 256;
-constexpr int kDequantThreads = kTeamThreads;
-constexpr int kNSA = 4;            // dequantised A stages
+// 12 warps: 0 code TMA, 1 activation TMA, 2 TMEM allocation and MMA issue, 3 spare,
+// 4-11 dequantisation into TMEM and then the epilogue (a warp reaches only the TMEM lane
+// quarter warp % 4, so each quarter has two of them, one per K half).
+constexpr int kThreads = 384;
+constexpr int kDequantThreads = 256;
 constexpr int kMetaChunks = 4;     // groups per metadata tile
-constexpr int kDoneRing = 8;       // mma_done barriers (>= kNSA and >= every activation ring depth)
+constexpr int kDoneRing = 8;       // mma_done barriers, one per step (more than any ring's look-ahead)
+constexpr int kTmemCols = 512;     // whole TMEM of the SM (one CTA per SM)
+constexpr int kACol0 = 256;        // TMEM columns [0, 256): accumulator; [256, 512): dequantised A slots
+constexpr int kACols = kTmemCols - kACol0;
 
 struct GemmParams {
     const __half* bias;
@@ -64,6 +71,7 @@ struct GemmParams {
     int early_w;
     int yperm;             // write y in the interleaved 8-block order
     int nsx, nsc;          // activation / code ring depths
+    int xu;                // K chunks per activation stage
     uint32_t off_x, off_c, off_m, off_bar;
     uint32_t tmem_cols;
     // fused store_cache (QKV projection): output features [kv_h, 2 kv_h) are the keys and
@@ -220,9 +228,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                                                               const __grid_constant__ CUtensorMap tm_x,
                                                               const GemmParams p) {
     constexpr int CROW = kBK * BITS / 8;          // code bytes per row and K chunk (32 or 64)
-    constexpr int CPS = 128 / CROW;               // K chunks per code stage (4 or 2)
+    constexpr int KU = 128 / CROW;                // K chunks per step = per code stage (4 or 2)
     constexpr int CSTAGE = kBM * 128;             // code bytes per stage: 128 rows x 128 B
     constexpr int MSTAGE = kBM * kMetaChunks * 4; // metadata bytes per stage: 128 rows x 4 groups
+    constexpr int SLOT_COLS = KU * 32;            // TMEM columns of one A slot: KU chunks x 64 fp16
+    constexpr int NSLOT = kACols / SLOT_COLS;     // A slots (2 at 4 bits, 4 at 8 bits)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -233,17 +243,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int nk_total = p.K / kBK;
     const int c_begin = split * p.cps;                            // multiple of kMetaChunks
     const int nk = min(nk_total, c_begin + p.cps) - c_begin;      // multiple of kMetaChunks
-    const int nstages = nk / CPS;
+    const int nsteps = nk / KU;
+    const int XU = p.xu;                                          // K chunks per activation stage
+    const int nxu = nk / XU;
 
-    const uint32_t sA = base, sX = base + p.off_x, sC = base + p.off_c, sM = base + p.off_m;
+    const uint32_t sX = base, sC = base + p.off_c, sM = base + p.off_m;
     const uint32_t sb = base + p.off_bar;
     const int NSX = p.nsx, NSC = p.nsc;
+    const uint32_t xbytes = static_cast<uint32_t>(p.BN) * 128;   // one activation chunk: BN rows x 64 fp16
     Bars B;
     B.codes_full = sb;
     B.codes_empty = B.codes_full + 8 * NSC;
     B.x_full = B.codes_empty + 8 * NSC;
     B.a_full = B.x_full + 8 * NSX;
-    B.mma_done = B.a_full + 8 * kNSA;
+    B.mma_done = B.a_full + 8 * NSLOT;
     B.acc_full = B.mma_done + 8 * kDoneRing;
     B.drain = B.acc_full + 8;
     const uint32_t misc = B.drain + 8;                        // tmem slot, abort flag, last flag
@@ -258,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             tc::bar_init(B.codes_empty + 8 * s, kDequantThreads);
         }
         for (int s = 0; s < NSX; ++s) tc::bar_init(B.x_full + 8 * s, 1);
-        for (int s = 0; s < kNSA; ++s) tc::bar_init(B.a_full + 8 * s, kDequantThreads);
+        for (int s = 0; s < NSLOT; ++s) tc::bar_init(B.a_full + 8 * s, kDequantThreads);
         for (int s = 0; s < kDoneRing; ++s) tc::bar_init(B.mma_done + 8 * s, 1);
         tc::bar_init(B.acc_full, 1);
         tc::bar_init(B.drain, 1);
@@ -267,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         tc::bar_fence_init();
     }
     if (warp == 2) {
-        tc::tmem_alloc(misc, p.tmem_cols);
+        tc::tmem_alloc(misc, kTmemCols);
         tc::tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
@@ -278,21 +291,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *tmem_slot;             // accumulator: columns [0, BN); A slots from kACol0
     // Dependencies on the previous kernel (programmatic dependent launch): the
     // activation producer and the epilogue wait for it before touching global memory;
     // the code producer also waits unless early_w; the MMA and dequant roles only touch
     // shared memory and TMEM.
 
     if (warp == 0) {
-        // ---------------- code + metadata producer: one stage = CPS chunks ----------------
+        // ---------------- code + metadata producer: one stage = one step of KU chunks ----------------
         if (lane == 0) {
             if (!p.early_w) pdl_wait();
             int st = 0;
-            for (; st < nstages; ++st) {
+            for (; st < nsteps; ++st) {
                 const int s = st % NSC;
                 if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ((st / NSC) & 1) ^ 1, abort, p.status)) break;
-                const int c = c_begin + st * CPS;
+                const int c = c_begin + st * KU;
                 tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CSTAGE + MSTAGE);
                 tc::tma_load_2d(sC + s * CSTAGE, &tm_codes, c * CROW, n0, B.codes_full + 8 * s);
                 tc::tma_load_2d(sM + s * MSTAGE, &tm_meta, c & ~(kMetaChunks - 1), n0, B.codes_full + 8 * s);
@@ -306,21 +319,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- activation producer ----------------
+        // ---------------- activation producer: one stage = XU chunks ----------------
         if (lane == 0) {
             pdl_wait();                           // the activations come from the previous kernel
-            int i = 0;
-            for (; i < nk; ++i) {
-                const int s = i % NSX;
-                // slot s last held chunk i - NSX: wait until its MMAs are done
-                if (i >= NSX) {
-                    const int pc = i - NSX;
-                    if (!tc::bar_wait(B.mma_done + 8 * (pc % kDoneRing), (pc / kDoneRing) & 1, abort, p.status)) break;
+            int u = 0;
+            for (; u < nxu; ++u) {
+                const int s = u % NSX;
+                if (u >= NSX) {
+                    // the stage last held unit u - NSX: wait for the MMAs of the step that read it
+                    const int pj = ((u - NSX) * XU) / KU;
+                    if (!tc::bar_wait(B.mma_done + 8 * (pj % kDoneRing), (pj / kDoneRing) & 1, abort, p.status))
+                        break;
                 }
-                tc::bar_arrive_expect_tx(B.x_full + 8 * s, p.BN * 128);
-                tc::tma_load_2d(sX + s * (p.BN * 128), &tm_x, (c_begin + i) * kBK, m0, B.x_full + 8 * s);
+                tc::bar_arrive_expect_tx(B.x_full + 8 * s, XU * xbytes);
+                for (int c = 0; c < XU; ++c)
+                    tc::tma_load_2d(sX + (s * XU + c) * xbytes, &tm_x, (c_begin + u * XU + c) * kBK, m0,
+                                    B.x_full + 8 * s);
             }
-            const int issued = i;
+            const int issued = u;
             for (int s = 0; s < NSX && s < issued; ++s) {
                 const int last = s + ((issued - 1 - s) / NSX) * NSX;
                 volatile int never = 0;
@@ -329,25 +345,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
         __syncwarp();
     } else if (warp == 2) {
-        // ---------------- MMA issuer ----------------
+        // ---------------- MMA issuer: one wait per step of KU chunks, one commit per step ----------------
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_f16_f32(kBM, p.BN);
             bool ok = true;
-            for (int i = 0; i < nk; ++i) {
-                const int sa = i % kNSA, sx = i % NSX;
-                if (!tc::bar_wait(B.a_full + 8 * sa, (i / kNSA) & 1, abort, p.status)) { ok = false; break; }
-                if (!tc::bar_wait(B.x_full + 8 * sx, (i / NSX) & 1, abort, p.status)) { ok = false; break; }
+            for (int j = 0; j < nsteps && ok; ++j) {
+                const int sa = j % NSLOT;
+                if (!tc::bar_wait(B.a_full + 8 * sa, (j / NSLOT) & 1, abort, p.status)) { ok = false; break; }
                 tc::fence_after_sync();
-                const uint64_t ad = tc::desc_k_sw128(sA + sa * (kBM * 128));
-                const uint64_t bd = tc::desc_k_sw128(sX + sx * (p.BN * 128));
+                const uint32_t a_tm = tmem + kACol0 + sa * SLOT_COLS;
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                    tc::mma_f16(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-                // exactly one commit per chunk: a commit covers the MMAs issued since the
-                // previous one, so a second commit here would complete at once. Both rings
-                // that reuse this chunk's operands (A and activations) wait on mma_done;
-                // the last chunk's commit is the accumulator-ready signal.
-                tc::mma_commit(i + 1 < nk ? B.mma_done + 8 * (i % kDoneRing) : B.acc_full);
+                for (int c = 0; c < KU; ++c) {
+                    const int i = j * KU + c;
+                    const int u = i / XU, xs = u % NSX;
+                    if (i % XU == 0 && !tc::bar_wait(B.x_full + 8 * xs, (u / NSX) & 1, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint64_t bd = tc::desc_k_sw128(sX + (xs * XU + (i % XU)) * xbytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc::mma_f16_ts(tmem, a_tm + c * 32 + kk * 8, bd + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (!ok) break;
+                // exactly one commit per step: a commit covers the MMAs issued since the
+                // previous one, so a second commit here would complete at once. The A slot
+                // and the activation stages of this step are reused once it lands; the
+                // last step's commit is the accumulator-ready signal.
+                tc::mma_commit(j + 1 < nsteps ? B.mma_done + 8 * (j % kDoneRing) : B.acc_full);
             }
             if (!ok) {
                 // nothing of ours may still run on the tensor cores at exit
@@ -359,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 // late arrival would hit the barriers of the next CTA on this SM, which
                 // live at the same shared-memory addresses
                 volatile int never = 0;
-                const int last = nk - 1;                 // committed to acc_full (waited in the epilogue)
+                const int last = nsteps - 1;             // committed to acc_full (waited in the epilogue)
                 for (int c = last - kDoneRing > 0 ? last - kDoneRing : 0; c < last; ++c)
                     tc::bar_wait(B.mma_done + 8 * (c % kDoneRing), (c / kDoneRing) & 1, &never, p.status);
                 tc::bar_wait(B.acc_full, 0, &never, p.status);
@@ -367,94 +392,94 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
         __syncwarp();
     } else if (warp >= 4) {
-        // ---------------- dequantisation ----------------
-        // thread (row, half) turns half of the row's codes of a K chunk (16 code bytes at
-        // 4 bits, 32 at 8 bits) into 32 fp16 = 4 of the row's 8 16-byte units of A; the
-        // chunks of a code stage are unpacked in pairs behind one proxy fence.
-        const bool deq = (warp < 14) && ((warp & 3) != 2);
-        const int rank = (warp - 4) - (warp > 6) - (warp > 10);       // 0..7 for the dequant warps
-        const int dt = rank * 32 + lane;
-        const int row = dt & 127, half_ = dt >> 7;
+        // ---------------- dequantisation into TMEM ----------------
+        // Warp w writes TMEM lanes 32 (w % 4) .. +31 (a warp may only access its own lane
+        // quarter): thread (row = 32 (w % 4) + lane, half h) turns half of the row's codes
+        // of each K chunk (16 code bytes at 4 bits, 32 at 8 bits) into 32 fp16 = 16
+        // columns of the step's A slot.
+        const int q = warp & 3, h = (warp - 4) >> 2;
+        const int row = q * 32 + lane;
         const int sw = row & 7;
-        constexpr int CPP = CPS >= 2 ? 2 : 1;           // chunks per fence
+        const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + h * 16;
         bool ok = true;
-        for (int st = 0; deq && st < nstages && ok; ++st) {
+        for (int st = 0; st < nsteps && ok; ++st) {
             const int s = st % NSC;
             if (!tc::bar_wait(B.codes_full + 8 * s, (st / NSC) & 1, abort, p.status)) { ok = false; break; }
             // codes of the stage (the tile was stored with the 128-byte swizzle: 16-byte
             // unit u of row r sits at unit u ^ (r % 8))
-            const uint8_t* crow = gbase + (sC - base) + s * CSTAGE + row * 128;
-            uint4 cw[CPS][BITS / 4];
+            const uint32_t crow = sC + s * CSTAGE + row * 128;
+            uint4 cw[KU][BITS / 4];
 #pragma unroll
-            for (int c = 0; c < CPS; ++c)
+            for (int c = 0; c < KU; ++c)
 #pragma unroll
                 for (int v = 0; v < BITS / 4; ++v) {
-                    const int u = c * (CROW / 16) + half_ * (BITS / 4) + v;
-                    cw[c][v] = *reinterpret_cast<const uint4*>(crow + ((u ^ sw) << 4));
+                    const int u = c * (CROW / 16) + h * (BITS / 4) + v;
+                    cw[c][v] = tc::lds128(crow + ((u ^ sw) << 4));
                 }
-            const uint4 mrow = *reinterpret_cast<const uint4*>(gbase + (sM - base) + s * MSTAGE + row * 16);
-            const uint32_t mwv[4] = {mrow.x, mrow.y, mrow.z, mrow.w};
-            const int moff = (c_begin + st * CPS) & (kMetaChunks - 1);
-#pragma unroll
-            for (int c0 = 0; c0 < CPS; c0 += CPP) {
-                // the A slots of these chunks must have been consumed by the MMAs
-#pragma unroll
-                for (int c = c0; c < c0 + CPP; ++c) {
-                    const int i = st * CPS + c;
-                    if (i >= kNSA) {
-                        const int pc = i - kNSA;
-                        if (!tc::bar_wait(B.mma_done + 8 * (pc % kDoneRing), (pc / kDoneRing) & 1, abort, p.status))
-                            ok = false;
-                    }
+            const uint4 mrow = tc::lds128(sM + s * MSTAGE + row * 16);
+            const int moff = (c_begin + st * KU) & (kMetaChunks - 1);
+            // the A slot must have been read by the MMAs of step st - NSLOT
+            const int sa = st % NSLOT;
+            if (st >= NSLOT) {
+                const int pj = st - NSLOT;
+                if (!tc::bar_wait(B.mma_done + 8 * (pj % kDoneRing), (pj / kDoneRing) & 1, abort, p.status)) {
+                    ok = false;
+                    break;
                 }
-                if (!ok) break;
-#pragma unroll
-                for (int c = c0; c < c0 + CPP; ++c) {
-                    const int i = st * CPS + c;
-                    const uint32_t mw = mwv[(moff + c) & 3];
-                    const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
-                    const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
-                    // step = fp16(1/scale); a constant group (scale 0) gets step 0 and decodes to min
-                    const __half step = __float2half_rn(sc32 > 0.f ? __frcp_rn(sc32) : 0.f);
-                    const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
-                    const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
-                    const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
-                    uint8_t* arow = gbase + (i % kNSA) * (kBM * 128) + row * 128;
-                    if (BITS == 4) {
-                        const uint32_t w[4] = {cw[c][0].x, cw[c][0].y, cw[c][0].z, cw[c][0].w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2) : dequant8_4bit(w[j], step2, mnv2);
-                            *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = v;
-                        }
-                    } else {
-                        const uint4 q0 = cw[c][0], q1 = cw[c][BITS / 4 - 1];
-                        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint4 v;
-                            if (XPERM) {
-                                v = dequant8_8bit_il(w[2 * j], w[2 * j + 1], step2, mnv2);
-                            } else {
-                                const uint2 a = dequant4_8bit(w[2 * j], step2, mnv2);
-                                const uint2 b = dequant4_8bit(w[2 * j + 1], step2, mnv2);
-                                v = make_uint4(a.x, a.y, b.x, b.y);
-                            }
-                            *reinterpret_cast<uint4*>(arow + (((half_ * 4 + j) ^ sw) << 4)) = v;
-                        }
-                    }
-                }
-                tc::fence_proxy_async_smem();
-#pragma unroll
-                for (int c = c0; c < c0 + CPP; ++c) tc::bar_arrive(B.a_full + 8 * ((st * CPS + c) % kNSA));
+                tc::fence_after_sync();
             }
-            // release the code stage only once all of its values have been consumed (the
-            // next TMA into this slot must not overtake these shared-memory reads)
-            if (ok) tc::bar_arrive(B.codes_empty + 8 * s);
+#pragma unroll
+            for (int c = 0; c < KU; ++c) {
+                // group (moff + c) % 4 of the metadata tile (a select: a runtime array index
+                // would put the words in local memory)
+                const int mi = (moff + c) & 3;
+                const uint32_t mw = mi == 0 ? mrow.x : (mi == 1 ? mrow.y : (mi == 2 ? mrow.z : mrow.w));
+                const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
+                const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
+                // step = fp16(1/scale); a constant group (scale 0) gets step 0 and decodes to min
+                const __half step = __float2half_rn(sc32 > 0.f ? __frcp_rn(sc32) : 0.f);
+                const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
+                const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
+                const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
+                uint32_t r[16];
+                if (BITS == 4) {
+                    const uint32_t w[4] = {cw[c][0].x, cw[c][0].y, cw[c][0].z, cw[c][0].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2) : dequant8_4bit(w[j], step2, mnv2);
+                        r[4 * j] = v.x;
+                        r[4 * j + 1] = v.y;
+                        r[4 * j + 2] = v.z;
+                        r[4 * j + 3] = v.w;
+                    }
+                } else {
+                    const uint4 q0 = cw[c][0], q1 = cw[c][BITS / 4 - 1];
+                    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 v;
+                        if (XPERM) {
+                            v = dequant8_8bit_il(w[2 * j], w[2 * j + 1], step2, mnv2);
+                        } else {
+                            const uint2 a = dequant4_8bit(w[2 * j], step2, mnv2);
+                            const uint2 b = dequant4_8bit(w[2 * j + 1], step2, mnv2);
+                            v = make_uint4(a.x, a.y, b.x, b.y);
+                        }
+                        r[4 * j] = v.x;
+                        r[4 * j + 1] = v.y;
+                        r[4 * j + 2] = v.z;
+                        r[4 * j + 3] = v.w;
+                    }
+                }
+                tc::tmem_st16(t_row + sa * SLOT_COLS + c * 32, r);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            tc::bar_arrive(B.a_full + 8 * sa);
+            // the code stage's values are all consumed: the next TMA may refill it
+            tc::bar_arrive(B.codes_empty + 8 * s);
         }
-        if (warp >= 12) {
-            // not an epilogue warp
-        } else {
+        const int et = (warp - 4) * 32 + lane;    // 0..255 over the epilogue warps
         // ---------------- epilogue ----------------
         pdl_wait();                               // residual, bias, y and workspace
         pdl_trigger();                            // dependents may start their prologue
@@ -519,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 }
                 __threadfence();
                 asm volatile("bar.sync 1, 256;" ::: "memory");
-                if (dt == 0) *last_flag = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+                if (et == 0) *last_flag = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
                 asm volatile("bar.sync 1, 256;" ::: "memory");
                 if (*last_flag) {
                     __threadfence();
@@ -545,18 +570,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                         }
                         finish8(col, acc);
                     }
-                    if (dt == 0) p.counters[tile] = 0;
+                    if (et == 0) p.counters[tile] = 0;
                 }
             }
         }
-    }
     }
 
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 2) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, p.tmem_cols);
+        tc::tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -578,7 +602,7 @@ EncodeTiledFn encode_fn() {
 }
 
 struct Plan {
-    int BN, tiles_n, tiles_m, splits, cps, nsx, nsc;
+    int BN, tiles_n, tiles_m, splits, cps, nsx, nsc, xu;
     uint32_t off_x, off_c, off_m, off_bar, smem, tmem_cols;
     int64_t ws_bytes, counters_bytes;
 };
@@ -602,18 +626,27 @@ Plan make_plan(int M, int N, int K, int bits) {
     splits = (nk + cps - 1) / cps;
     P.splits = splits;
     P.cps = cps;
-    P.nsx = P.BN <= 64 ? 6 : (P.BN <= 160 ? 4 : 3);
-    P.nsc = P.BN <= 160 ? 4 : 2;                  // code stages of 128 rows x 128 B (+ metadata)
-    P.off_x = kNSA * kBM * 128;
-    P.off_c = P.off_x + P.nsx * P.BN * 128;
+    // activation stages: a whole step (KU chunks) when it fits in 64 KB, else half a step;
+    // up to 128 KB of them, 2..6 deep
+    const int ku = 128 / (kBK * bits / 8);
+    int xu = ku;
+    while (xu > 1 && xu * P.BN * 128 > 64 * 1024) xu >>= 1;
+    const uint32_t xstage = static_cast<uint32_t>(xu) * P.BN * 128;
+    int nsx = static_cast<int>((128u * 1024u) / xstage);
+    if (nsx > 6) nsx = 6;
+    if (nsx < 2) nsx = 2;
+    P.xu = xu;
+    P.nsx = nsx;
+    P.nsc = 4;                                    // code stages of 128 rows x 128 B (+ metadata)
+    P.off_x = 0;
+    P.off_c = nsx * xstage;
     P.off_m = P.off_c + P.nsc * kBM * 128;
     P.off_bar = P.off_m + P.nsc * kBM * kMetaChunks * 4;
-    uint32_t smem = P.off_bar + 8 * (2 * P.nsc + P.nsx + kNSA + kDoneRing + 2) + 16 + 256 + 1024;
-    if (smem < 120 * 1024) smem = 120 * 1024;   // at most one CTA per SM: TMEM is never contended
+    const int nslot = kACols / (ku * 32);
+    uint32_t smem = P.off_bar + 8 * (2 * P.nsc + P.nsx + nslot + kDoneRing + 2) + 16 + 256 + 1024;
+    if (smem < 120 * 1024) smem = 120 * 1024;   // at most one CTA per SM: the CTA takes all of TMEM
     P.smem = smem;
-    uint32_t cols = 32;
-    while (cols < static_cast<uint32_t>(P.BN)) cols <<= 1;
-    P.tmem_cols = cols;
+    P.tmem_cols = kTmemCols;
     P.counters_bytes = ((static_cast<int64_t>(tiles) * 4 + 255) / 256) * 256;
     P.ws_bytes = splits > 1 ? P.counters_bytes + static_cast<int64_t>(tiles) * splits * P.BN * kBM * 4 : 0;
     return P;
@@ -691,6 +724,7 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     gp.yperm = yperm ? 1 : 0;
     gp.nsx = P.nsx;
     gp.nsc = P.nsc;
+    gp.xu = P.xu;
     gp.off_x = P.off_x;
     gp.off_c = P.off_c;
     gp.off_m = P.off_m;

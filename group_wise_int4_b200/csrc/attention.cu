@@ -24,6 +24,21 @@
 
 namespace flexq {
 namespace {
+// 1/scale of a group with the hardware reciprocal (rcp.approx, relative error below
+// 2^-22): attention uses the step only inside fp32 sums checked against a tolerance,
+// so the correctly rounded division of the codec is not needed here. Scale 0 (a
+// constant group) gives step 0.
+__device__ __forceinline__ float group_step_fast(__half s16) {
+    const float s = __half2float(s16);
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    return s > 0.0f ? r : 0.0f;
+}
+}  // namespace
+}  // namespace flexq
+
+namespace flexq {
+namespace {
 
 constexpr int DA_THREADS = 128;
 
@@ -154,7 +169,7 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_split_kernel(
             float dot = 0.f;
 #pragma unroll
             for (int e = 0; e < EPT; ++e) dot = fmaf(qv[e], code_f(w[e * BITS / 32], (e * BITS) % 32, MASK), dot);
-            const float kstep = group_step(__ushort_as_half(static_cast<unsigned short>(km[u] >> 16)));
+            const float kstep = group_step_fast(__ushort_as_half(static_cast<unsigned short>(km[u] >> 16)));
             const float kmn = h2f_lo(km[u]);
             float su = fmaf(kstep, dot, kmn * qsum);
 #pragma unroll
@@ -176,7 +191,7 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_split_kernel(
             if (s[u] == -FLT_MAX) continue;
             const float p = __expf(s[u] - m);
             l += p;
-            const float vstep = group_step(__ushort_as_half(static_cast<unsigned short>(vm[u] >> 16)));
+            const float vstep = group_step_fast(__ushort_as_half(static_cast<unsigned short>(vm[u] >> 16)));
             const float w = p * vstep;
             U = fmaf(p, h2f_lo(vm[u]), U);
             const uint32_t vw[4] = {vc[u].x, vc[u].y, vc[u].z, vc[u].w};
@@ -385,8 +400,8 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_mma_kernel(
             const int n = 2 * t + u;
             if (n < G) {
                 const float Qn = pick(Qg, n);
-                const float st0 = group_step(__ushort_as_half(static_cast<unsigned short>(cur.kmg[u] >> 16)));
-                const float st1 = group_step(__ushort_as_half(static_cast<unsigned short>(cur.kmg8[u] >> 16)));
+                const float st0 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(cur.kmg[u] >> 16)));
+                const float st1 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(cur.kmg8[u] >> 16)));
                 sg_part += fmaf(st0, sacc[u] - C1024 * Qn, h2f_lo(cur.kmg[u]) * Qn);
                 sg8_part += fmaf(st1, sacc[2 + u] - C1024 * Qn, h2f_lo(cur.kmg8[u]) * Qn);
             }
@@ -432,7 +447,7 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_mma_kernel(
             float wv[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float stp = group_step(__ushort_as_half(static_cast<unsigned short>(cur.vmv[u] >> 16)));
+                const float stp = group_step_fast(__ushort_as_half(static_cast<unsigned short>(cur.vmv[u] >> 16)));
                 wv[u] = __half2float(__float2half_rn(pk[u] * stp));
                 wt += wv[u];
                 ut = fmaf(pk[u], h2f_lo(cur.vmv[u]), ut);
@@ -651,8 +666,8 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_staged_kernel(
             if (n < G) {
                 const uint32_t m0 = km[g * G + n], m8 = km[(g + 8) * G + n];
                 const float Qn = pick(Qg, n);
-                const float st0 = group_step(__ushort_as_half(static_cast<unsigned short>(m0 >> 16)));
-                const float st8 = group_step(__ushort_as_half(static_cast<unsigned short>(m8 >> 16)));
+                const float st0 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(m0 >> 16)));
+                const float st8 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(m8 >> 16)));
                 sg_part += fmaf(st0, sacc[u] - C1024 * Qn, h2f_lo(m0) * Qn);
                 sg8_part += fmaf(st8, sacc[2 + u] - C1024 * Qn, h2f_lo(m8) * Qn);
             }
@@ -698,7 +713,7 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_staged_kernel(
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const uint32_t mv = vm[(2 * t + (u & 1) + 8 * (u >> 1)) * G + g];
-                const float stp = group_step(__ushort_as_half(static_cast<unsigned short>(mv >> 16)));
+                const float stp = group_step_fast(__ushort_as_half(static_cast<unsigned short>(mv >> 16)));
                 wv[u] = __half2float(__float2half_rn(pk[u] * stp));
                 wt += wv[u];
                 ut = fmaf(pk[u], h2f_lo(mv), ut);

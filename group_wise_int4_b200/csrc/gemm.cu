@@ -26,11 +26,19 @@
 // Swap-AB orientation: the weight rows are the MMA's M side (128 per CTA) and the
 // activation rows (batch in decode, tokens in prefill) its N side (BN = 16..256), so a
 // decode batch of a few sequences still fills an M=128 instruction. Small grids are
-// split along K; each split writes fp32 partials and the last CTA of a tile (atomic
-// ticket) reduces them in a fixed order and runs the epilogue, so results do not
-// depend on scheduling. Every mbarrier wait is bounded: on expiry the CTA records
-// FLEX_ERR_TIMEOUT in the device status word, drains its own copies and MMAs, frees
-// TMEM and exits.
+// split along K into up to 8 splits per tile. When every tile's splits fit on the GPU
+// at once as one thread-block cluster each, they are launched so: each split leaves its
+// fp32 partial tile in its own shared memory and the CTAs of the cluster each finish a
+// share of the tile, reading all partials over distributed shared memory. Otherwise
+// the splits write fp32 partials to the workspace and the last CTA of a tile (atomic
+// ticket) finishes it. Both add the partials in split order, so results do not depend
+// on scheduling. Every mbarrier wait is bounded: on
+// expiry the CTA records FLEX_ERR_TIMEOUT in the device status word, drains its own
+// copies and MMAs, frees TMEM and exits (still taking part in the cluster barriers).
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "quant.cuh"
 #include "tc.cuh"
 
@@ -50,13 +58,12 @@ constexpr int kDoneRing = 8;       // mma_done barriers, one per step (more than
 constexpr int kTmemCols = 512;     // whole TMEM of the SM (one CTA per SM)
 constexpr int kACol0 = 256;        // TMEM columns [0, 256): accumulator; [256, 512): dequantised A slots
 constexpr int kACols = kTmemCols - kACol0;
+constexpr int kMaxSplits = 8;      // K splits of a tile form one cluster (portable size)
 
 struct GemmParams {
     const __half* bias;
     const __half* residual;
     __half* y;
-    float* part;
-    int* counters;
     int* status;
     int M, N, K;
     int BN;
@@ -72,6 +79,13 @@ struct GemmParams {
     int yperm;             // write y in the interleaved 8-block order
     int nsx, nsc;          // activation / code ring depths
     int xu;                // K chunks per activation stage
+    int nacc, acc_stride;  // independent TMEM accumulators and their column spacing
+    // K splits (splits > 1): cluster = 1 reduces them through distributed shared memory
+    // inside one thread-block cluster per tile; cluster = 0 through fp32 partials in the
+    // workspace, the last CTA of a tile (atomic ticket) finishing it
+    int cluster;
+    float* part;
+    int* counters;
     uint32_t off_x, off_c, off_m, off_bar;
     uint32_t tmem_cols;
     // fused store_cache (QKV projection): output features [kv_h, 2 kv_h) are the keys and
@@ -92,6 +106,15 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t raw_pair_bits, uint32_
     __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&raw_pair_bits), *reinterpret_cast<const __half2*>(&bias2));
     v = __hfma2(v, *reinterpret_cast<const __half2*>(&step2), *reinterpret_cast<const __half2*>(&mn2));
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Hardware reciprocal (rcp.approx, relative error below 2^-22); the result is rounded
+// to fp16 right after, so it matches the correctly rounded reciprocal except at rare
+// fp16 rounding ties.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t lop_nib(uint32_t w) {
@@ -292,6 +315,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;             // accumulator: columns [0, BN); A slots from kACol0
+
+    // epilogue mapping (warps 4-11): TMEM lane quarter lq = row block, column half ch
+    const int lq = warp & 3, ch = (warp - 4) >> 2;
+    const int irow = lq * 32 + lane;
+    const int n = n0 + irow;
+    const float scale_n = n < p.nq ? p.qscale : 1.f;
+    // interleaved output: element k of every 8-block goes to position 2(k%4) + (k/4)%2
+    const int n_out = p.yperm ? ((n & ~7) | ((n & 3) << 1) | ((n >> 2) & 1)) : n;
+    // fused store_cache: this tile lies inside the key or the value block (h % 128 == 0)
+    const bool kv_on = p.kv_codes[0] != nullptr && n0 >= p.kv_h;
+    float bias_n = 0.f;                           // read by the epilogue after its PDL wait
+    uint32_t all_ok = 0;                          // epilogue warps: the main loop completed
+    // bias, q-scale, ReLU, residual, fp16 store (and store_cache) of 8 columns of row n
+    auto finish8 = [&](int col, const float (&v)[8]) {
+        float r[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int m = m0 + col + j;
+            r[j] = (p.residual && m < p.M) ? __half2float(p.residual[static_cast<int64_t>(m) * p.N + n]) : 0.f;
+        }
+        __half o16[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int m = m0 + col + j;
+            float x = (v[j] + bias_n) * scale_n;
+            if (p.relu) x = fmaxf(x, 0.f);
+            o16[j] = __float2half_rn(x + r[j]);
+            if (m < p.M) p.y[static_cast<int64_t>(m) * p.N + n_out] = o16[j];
+        }
+        if (kv_on) kv_store8(p, o16, col, m0, n0, n, warp, lane, kv_red);
+    };
     // Dependencies on the previous kernel (programmatic dependent launch): the
     // activation producer and the epilogue wait for it before touching global memory;
     // the code producer also waits unless early_w; the MMA and dequant roles only touch
@@ -301,14 +355,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         // ---------------- code + metadata producer: one stage = one step of KU chunks ----------------
         if (lane == 0) {
             if (!p.early_w) pdl_wait();
-            int st = 0;
+            // ring position kept incrementally (stage s, phase bit ph): no integer division
+            // by the runtime ring depth on this thread's path
+            int st = 0, s = 0;
+            uint32_t ph = 0;
             for (; st < nsteps; ++st) {
-                const int s = st % NSC;
-                if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ((st / NSC) & 1) ^ 1, abort, p.status)) break;
+                if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ph ^ 1, abort, p.status)) break;
                 const int c = c_begin + st * KU;
                 tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CSTAGE + MSTAGE);
                 tc::tma_load_2d(sC + s * CSTAGE, &tm_codes, c * CROW, n0, B.codes_full + 8 * s);
                 tc::tma_load_2d(sM + s * MSTAGE, &tm_meta, c & ~(kMetaChunks - 1), n0, B.codes_full + 8 * s);
+                if (++s == NSC) { s = 0; ph ^= 1; }
             }
             // drain: every copy this thread issued has landed before the CTA can exit
             for (int s = 0; s < NSC && s < st; ++s) {
@@ -322,9 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         // ---------------- activation producer: one stage = XU chunks ----------------
         if (lane == 0) {
             pdl_wait();                           // the activations come from the previous kernel
-            int u = 0;
+            int u = 0, s = 0;
             for (; u < nxu; ++u) {
-                const int s = u % NSX;
                 if (u >= NSX) {
                     // the stage last held unit u - NSX: wait for the MMAs of the step that read it
                     const int pj = ((u - NSX) * XU) / KU;
@@ -335,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 for (int c = 0; c < XU; ++c)
                     tc::tma_load_2d(sX + (s * XU + c) * xbytes, &tm_x, (c_begin + u * XU + c) * kBK, m0,
                                     B.x_full + 8 * s);
+                if (++s == NSX) s = 0;
             }
             const int issued = u;
             for (int s = 0; s < NSX && s < issued; ++s) {
@@ -347,25 +404,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     } else if (warp == 2) {
         // ---------------- MMA issuer: one wait per step of KU chunks, one commit per step ----------------
         if (lane == 0) {
+            // This single thread issues every MMA, so its own instruction latency is the
+            // issue rate: everything below is precomputed or advanced incrementally (no
+            // integer division by a runtime value in the loop).
             const uint32_t idesc = tc::idesc_f16_f32(kBM, p.BN);
+            // k-step kk of every chunk accumulates into accumulator kk % nacc (nacc = 1, 2
+            // or 4), so consecutive MMAs do not wait for each other's results; the
+            // epilogue adds the accumulators
+            const uint32_t amask = static_cast<uint32_t>(p.nacc - 1);
+            uint32_t d_tm[kBK / 16];
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) d_tm[kk] = tmem + (kk & amask) * static_cast<uint32_t>(p.acc_stride);
+            int xs = 0;
+            uint32_t xph = 0;
             bool ok = true;
             for (int j = 0; j < nsteps && ok; ++j) {
                 const int sa = j % NSLOT;
                 if (!tc::bar_wait(B.a_full + 8 * sa, (j / NSLOT) & 1, abort, p.status)) { ok = false; break; }
                 tc::fence_after_sync();
                 const uint32_t a_tm = tmem + kACol0 + sa * SLOT_COLS;
+                for (int c0 = 0; c0 < KU && ok; c0 += XU) {
+                    if (!tc::bar_wait(B.x_full + 8 * xs, xph, abort, p.status)) { ok = false; break; }
+                    const uint32_t xb = sX + static_cast<uint32_t>(xs * XU) * xbytes;
+                    for (int c2 = 0; c2 < XU; ++c2) {
+                        const int c = c0 + c2;
+                        const uint64_t bd = tc::desc_k_sw128(xb + c2 * xbytes);
+                        const bool first = (j == 0 && c == 0);
 #pragma unroll
-                for (int c = 0; c < KU; ++c) {
-                    const int i = j * KU + c;
-                    const int u = i / XU, xs = u % NSX;
-                    if (i % XU == 0 && !tc::bar_wait(B.x_full + 8 * xs, (u / NSX) & 1, abort, p.status)) {
-                        ok = false;
-                        break;
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            tc::mma_f16_ts(d_tm[kk], a_tm + c * 32 + kk * 8, bd + 2 * kk, idesc,
+                                           (first && static_cast<uint32_t>(kk) <= amask) ? 0u : 1u);
                     }
-                    const uint64_t bd = tc::desc_k_sw128(sX + (xs * XU + (i % XU)) * xbytes);
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc::mma_f16_ts(tmem, a_tm + c * 32 + kk * 8, bd + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                    if (++xs == NSX) { xs = 0; xph ^= 1; }
                 }
                 if (!ok) break;
                 // exactly one commit per step: a commit covers the MMAs issued since the
@@ -402,9 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         const int sw = row & 7;
         const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + h * 16;
         bool ok = true;
+        int s = 0;
+        uint32_t cph = 0;
         for (int st = 0; st < nsteps && ok; ++st) {
-            const int s = st % NSC;
-            if (!tc::bar_wait(B.codes_full + 8 * s, (st / NSC) & 1, abort, p.status)) { ok = false; break; }
+            if (!tc::bar_wait(B.codes_full + 8 * s, cph, abort, p.status)) { ok = false; break; }
             // codes of the stage (the tile was stored with the 128-byte swizzle: 16-byte
             // unit u of row r sits at unit u ^ (r % 8))
             const uint32_t crow = sC + s * CSTAGE + row * 128;
@@ -437,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
                 const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
                 // step = fp16(1/scale); a constant group (scale 0) gets step 0 and decodes to min
-                const __half step = __float2half_rn(sc32 > 0.f ? __frcp_rn(sc32) : 0.f);
+                const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
                 const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
                 const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
                 const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
@@ -478,22 +549,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             tc::bar_arrive(B.a_full + 8 * sa);
             // the code stage's values are all consumed: the next TMA may refill it
             tc::bar_arrive(B.codes_empty + 8 * s);
+            if (++s == NSC) { s = 0; cph ^= 1; }
         }
-        const int et = (warp - 4) * 32 + lane;    // 0..255 over the epilogue warps
         // ---------------- epilogue ----------------
-        pdl_wait();                               // residual, bias, y and workspace
+        pdl_wait();                               // residual, bias and y
         pdl_trigger();                            // dependents may start their prologue
-        const int lq = warp & 3, ch = (warp - 4) >> 2;
-        const int irow = lq * 32 + lane;
-        const int n = n0 + irow;
-        const float bias_n = p.bias ? __half2float(p.bias[n]) : 0.f;   // issued before the waits
-        const float scale_n = n < p.nq ? p.qscale : 1.f;
-        // interleaved output: element k of every 8-block goes to position 2(k%4) + (k/4)%2
-        const int n_out = p.yperm ? ((n & ~7) | ((n & 3) << 1) | ((n >> 2) & 1)) : n;
+        bias_n = p.bias ? __half2float(p.bias[n]) : 0.f;
         asm volatile("bar.sync 1, 256;" ::: "memory");
         if (ok && !*abort) ok = tc::bar_wait(B.acc_full, 0, abort, p.status);
         // one decision for all 256 threads (they share the named barriers below)
-        uint32_t all_ok;
         asm volatile(
             "{\n\t.reg .pred p, q;\n\t"
             "setp.ne.u32 p, %1, 0;\n\t"
@@ -506,39 +570,40 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             tc::fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16);
             const int cbeg = ch * (p.BN / 2), cend = cbeg + p.BN / 2;
-            // 8 columns at a time: residual loads issued together, then the stores
-            // fused store_cache: this tile lies inside the key or the value block (h % 128 == 0)
-            const bool kv_on = p.kv_codes[0] != nullptr && n0 >= p.kv_h;
-            auto finish8 = [&](int col, const float (&v)[8]) {
-                float r[8];
+            // 8 columns of row n: the sum of the accumulators, in accumulator order
+            auto acc8 = [&](int col, float (&v)[8]) {
+                tc::tmem_ld8(taddr + col, v);
+                for (int a = 1; a < p.nacc; ++a) {
+                    float w[8];
+                    tc::tmem_ld8(taddr + a * p.acc_stride + col, w);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int m = m0 + col + j;
-                    r[j] = (p.residual && m < p.M) ? __half2float(p.residual[static_cast<int64_t>(m) * p.N + n]) : 0.f;
+                    for (int j = 0; j < 8; ++j) v[j] += w[j];
                 }
-                __half o16[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int m = m0 + col + j;
-                    float x = (v[j] + bias_n) * scale_n;
-                    if (p.relu) x = fmaxf(x, 0.f);
-                    o16[j] = __float2half_rn(x + r[j]);
-                    if (m < p.M) p.y[static_cast<int64_t>(m) * p.N + n_out] = o16[j];
-                }
-                if (kv_on) kv_store8(p, o16, col, m0, n0, n, warp, lane, kv_red);
             };
             if (p.splits == 1) {
                 for (int col = cbeg; col < cend; col += 8) {
                     float v[8];
-                    tc::tmem_ld8(taddr + col, v);
+                    acc8(col, v);
                     finish8(col, v);
                 }
+            } else if (p.cluster) {
+                // this split's fp32 partial tile into this CTA's shared memory, column-major
+                // [BN][128] (it reuses the activation ring: every MMA has completed)
+                for (int col = cbeg; col < cend; col += 8) {
+                    float v[8];
+                    acc8(col, v);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) tc::st_shared_f32(sX + ((col + j) * kBM + irow) * 4, v[j]);
+                }
             } else {
+                // partial tile to the workspace; the last split of the tile to arrive adds
+                // all partials in split order and finishes the tile
+                const int et = (warp - 4) * 32 + lane;
                 const int tile = blockIdx.y * gridDim.x + blockIdx.x;
                 float* mine = p.part + (static_cast<int64_t>(tile) * p.splits + split) * p.BN * kBM;
                 for (int col = cbeg; col < cend; col += 8) {
                     float v[8];
-                    tc::tmem_ld8(taddr + col, v);
+                    acc8(col, v);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) mine[(col + j) * kBM + irow] = v[j];
                 }
@@ -553,18 +618,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                         float acc[8];
 #pragma unroll
                         for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-                        // up to 4 splits' 8 values in flight at once, summed in split order
-                        for (int s0 = 0; s0 < p.splits; s0 += 4) {
-                            float t[4][8];
+                        // up to 8 splits' 8 values in flight at once, added in split order
+                        for (int s0 = 0; s0 < p.splits; s0 += 8) {
+                            float t[8][8];
 #pragma unroll
-                            for (int u = 0; u < 4; ++u)
+                            for (int u = 0; u < 8; ++u)
 #pragma unroll
                                 for (int j = 0; j < 8; ++j)
                                     t[u][j] = (s0 + u < p.splits)
                                                   ? __ldcg(all + (static_cast<int64_t>(s0 + u) * p.BN + col + j) * kBM + irow)
                                                   : 0.f;
 #pragma unroll
-                            for (int u = 0; u < 4; ++u)
+                            for (int u = 0; u < 8; ++u)
 #pragma unroll
                                 for (int j = 0; j < 8; ++j) acc[j] += t[u][j];
                         }
@@ -574,6 +639,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 }
             }
         }
+    }
+
+    if (p.splits > 1 && p.cluster) {
+        // ---------------- split-K reduction across the cluster ----------------
+        // The K splits of a tile are one thread-block cluster. After the barrier every
+        // split's partial tile is visible; CTA r finishes the 8-column groups v with
+        // v % splits == r, adding the partials in split order (deterministic), and the
+        // second barrier keeps every CTA's shared memory alive until its peers are done.
+        // All threads of every CTA take part in both barriers.
+        tc::cluster_sync();
+        if (warp >= 4 && all_ok) {
+            const int S = p.splits;
+            const int rank = static_cast<int>(tc::cluster_rank());
+            int idx = 0;
+            for (int v = rank; v < p.BN / 8; v += S, ++idx) {
+                if ((idx & 1) != ch) continue;    // the two column halves alternate
+                const int col = v * 8;
+                float acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+                for (int sp = 0; sp < S; ++sp) {
+                    const uint32_t peer = tc::map_peer(sX + (col * kBM + irow) * 4, static_cast<uint32_t>(sp));
+                    float t[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) t[j] = tc::ld_peer_f32(peer + j * kBM * 4);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[j] += t[j];
+                }
+                finish8(col, acc);
+            }
+        }
+        tc::cluster_sync();
     }
 
     tc::fence_before_sync();
@@ -601,8 +698,40 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// Thread-block clusters of `splits` CTAs of this kernel that can be resident at once on
+// the current device (cached per device and size); 0 if the query fails.
+int max_active_clusters(int splits, uint32_t smem) {
+    static std::map<std::tuple<int, int, uint32_t>, int> cache;
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(dev, splits, smem);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    set_smem_once(gemm_tc_kernel<4, true>, 227 * 1024);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, splits);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<4, true>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    cache[key] = n;
+    return n;
+}
+
 struct Plan {
-    int BN, tiles_n, tiles_m, splits, cps, nsx, nsc, xu;
+    int BN, tiles_n, tiles_m, splits, cps, nsx, nsc, xu, nacc, acc_stride, cluster;
     uint32_t off_x, off_c, off_m, off_bar, smem, tmem_cols;
     int64_t ws_bytes, counters_bytes;
 };
@@ -619,6 +748,7 @@ Plan make_plan(int M, int N, int K, int bits) {
     int splits = 1;
     if (tiles < sms) splits = sms / tiles;
     int max_splits = nk / kMetaChunks;
+    if (max_splits > kMaxSplits) max_splits = kMaxSplits;
     if (max_splits < 1) max_splits = 1;
     if (splits > max_splits) splits = max_splits;
     int cps = (nk + splits - 1) / splits;
@@ -647,8 +777,16 @@ Plan make_plan(int M, int N, int K, int bits) {
     if (smem < 120 * 1024) smem = 120 * 1024;   // at most one CTA per SM: the CTA takes all of TMEM
     P.smem = smem;
     P.tmem_cols = kTmemCols;
+    // up to 4 accumulators in TMEM columns [0, 256), 32-column aligned
+    P.acc_stride = ((P.BN + 31) / 32) * 32;
+    P.nacc = kACol0 / P.acc_stride >= 4 ? 4 : (kACol0 / P.acc_stride >= 2 ? 2 : 1);   // a power of two
+    // split-K: through distributed shared memory when every tile's cluster can be
+    // resident at once (one wave), else through workspace partials and a ticket
+    P.cluster = (splits > 1 && max_active_clusters(splits, P.smem) >= tiles) ? 1 : 0;
     P.counters_bytes = ((static_cast<int64_t>(tiles) * 4 + 255) / 256) * 256;
-    P.ws_bytes = splits > 1 ? P.counters_bytes + static_cast<int64_t>(tiles) * splits * P.BN * kBM * 4 : 0;
+    P.ws_bytes = (splits > 1 && !P.cluster)
+                     ? P.counters_bytes + static_cast<int64_t>(tiles) * splits * P.BN * kBM * 4
+                     : 0;
     return P;
 }
 
@@ -708,8 +846,6 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     gp.bias = static_cast<const __half*>(bias);
     gp.residual = static_cast<const __half*>(residual);
     gp.y = static_cast<__half*>(y);
-    gp.counters = static_cast<int*>(ws);
-    gp.part = reinterpret_cast<float*>(static_cast<char*>(ws) + P.counters_bytes);
     gp.status = status_word();
     gp.M = M;
     gp.N = N;
@@ -725,6 +861,11 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     gp.nsx = P.nsx;
     gp.nsc = P.nsc;
     gp.xu = P.xu;
+    gp.cluster = P.cluster;
+    gp.counters = static_cast<int*>(ws);
+    gp.part = reinterpret_cast<float*>(static_cast<char*>(ws) + P.counters_bytes);
+    gp.nacc = P.nacc;
+    gp.acc_stride = P.acc_stride;
     gp.off_x = P.off_x;
     gp.off_c = P.off_c;
     gp.off_m = P.off_m;
@@ -745,10 +886,25 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
         gp.kv_gs = kv->cache->cfg.group_size;
     }
     const dim3 grid(P.tiles_n, P.tiles_m, P.splits);
+    // programmatic dependent launch, and the K splits of a tile as one cluster
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = P.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = P.splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.cluster ? 2 : 1;
 #define GEMM_LAUNCH(B_, XP_)                                                                 \
     do {                                                                                     \
         set_smem_once(gemm_tc_kernel<B_, XP_>, 227 * 1024);                                  \
-        launch_k(gemm_tc_kernel<B_, XP_>, grid, dim3(kThreads), P.smem, st, true, tm_codes, tm_meta, tm_x, gp); \
+        cudaLaunchKernelEx(&cfg, gemm_tc_kernel<B_, XP_>, tm_codes, tm_meta, tm_x, gp);      \
     } while (0)
     if (bits == 4) {
         if (xperm) GEMM_LAUNCH(4, true); else GEMM_LAUNCH(4, false);

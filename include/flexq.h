@@ -203,7 +203,11 @@ int flex_prefill_attention(const void* q, const void* k, const void* v, int64_t 
  *   x fp16 [M][K] row-major, W compressed [N][K] (group 64 along K, 4 or 8 bits),
  *   bias fp16 [N] or NULL, residual fp16 [M][N] or NULL (added after bias),
  *   epilogue: FLEX_EPI_NONE, FLEX_EPI_RELU (after bias), FLEX_EPI_RESIDUAL.
- *   y fp16 [M][N]; y may alias residual. ws: flex_gemm_ws_bytes(M, N, K) bytes.  */
+ *   y fp16 [M][N]; y may alias residual. ws: flex_gemm_ws_bytes(M, N, K) bytes of
+ *   device memory, zero-filled before its first use (its tickets return to zero after
+ *   every call); the size depends on the device. It is 0, and ws may be NULL, when the
+ *   K splits of a tile reduce through distributed shared memory (thread-block
+ *   clusters) or the GEMM is not split.                                          */
 #define FLEX_EPI_NONE     0
 #define FLEX_EPI_RELU     1
 #define FLEX_EPI_RESIDUAL 2

@@ -232,33 +232,32 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_split_kernel(
 // ---------------------------------------------------------------------------------
 // decode attention on the tensor cores (4-bit cache), mma.sync m16n8k16, fp32 accumulate.
 //
-// Each warp walks 16-key tiles of its (sequence, head) range. Codes enter the MMA raw,
-// as the exact fp16 values 1024 + c (one LOP3 per two codes); the dequantisation is
-// applied to the small results instead of to every element:
-//   scores: the 8 columns of the QK MMA are the key groups (B[dim][n] = q[dim] when
-//           dim is in group n, else 0), so one pass gives S[j][n] = sum_{dim in n}
-//           (1024 + c_j[dim]) q[dim] and
-//           s_j = sum_n step_jn (S[j][n] - 1024 Q_n) + min_jn Q_n,  Q_n = sum_{dim in n} q;
-//   values: B[j][n] = w_jn = p_j step_jn (fp16), so D'[dim][n] = 1024 W_n +
-//           sum_j w_jn c_j[dim] and o[dim] = D'[dim][g] - 1024 W_g + sum_j p_j min_jg
-//           with g the group of dim and W_g = sum_j w_jg.
-// Both MMAs are free to permute the K dimension (dims for QK, keys for PV) as long as A
-// and B agree; the layouts below are chosen so that every thread loads contiguous code
-// bytes and builds its fragments with PRMT / LOP3 only.
-__device__ __forceinline__ uint32_t nib_pair(uint32_t x) {
-    // (x & 0x000F000F) | 0x64006400: two 4-bit codes as the fp16 pair (1024 + lo, 1024 + hi)
+// Codes enter the MMAs raw, as exact fp16 values built with one LOP3 per two codes:
+// the low nibble of a byte (the even dim) as 1024 + c, the high nibble (the odd dim)
+// as 1024 + 16 c, so no shifts are needed. The group dequantisation x^ = step c + min
+// (step = 1/scale) is applied to the small results instead of to every element:
+//   scores: the query operand holds q[dim] for even dims and q[dim]/16 for odd ones,
+//           in column n = the dim's group (zero elsewhere), so the QK MMA gives per
+//           key j and group n  R[j][n] = sum_{dim in n} c_j[dim] q[dim] + QC_n  with
+//           QC_n = 1024 sum_{even dim in n} q + 64 sum_{odd dim in n} q, and
+//           s_j = sum_n step_jn (R[j][n] - QC_n) + min_jn Q_n,  Q_n = sum_{dim in n} q;
+//   values: the PV MMA multiplies the transposed codes by B[j][n] = w_jn = fp16(p_j
+//           step_jn), so for dim d of group n: D'[d] = 1024 W_n + f_d sum_j w_jn c_j[d]
+//           (f_d = 1 for even, 16 for odd dims) and
+//           o[d] = (D'[d] - 1024 W_n) / f_d + U_n,  W_n = sum_j w_jn,  U_n = sum_j p_j min_jn.
+// Both MMAs are free to permute their K dimension (dims for QK, keys for PV) as long as
+// A and B agree; the layouts below let every thread load contiguous code bytes.
+__device__ __forceinline__ uint32_t nib_lo(uint32_t x) {
+    // (x & 0x000F000F) | 0x64006400: low nibbles of bytes 0 and 2 as fp16 1024 + c
     uint32_t r;
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(0x000F000Fu), "r"(0x64006400u));
     return r;
 }
-__device__ __forceinline__ uint32_t byte_pair(uint32_t a, uint32_t b, uint32_t byte) {
-    // byte `byte` of a into bits 0..7, byte `byte` of b into bits 16..23
+__device__ __forceinline__ uint32_t nib_hi(uint32_t x) {
+    // (x & 0x00F000F0) | 0x64006400: high nibbles of bytes 0 and 2 as fp16 1024 + 16 c
     uint32_t r;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(byte | ((4u + byte) << 8)));
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(0x00F000F0u), "r"(0x64006400u));
     return r;
-}
-__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
-    return pack_half2_bits(__float2half_rn(lo), __float2half_rn(hi));
 }
 // a[n] for a runtime n without dynamic register indexing (which would go to local memory)
 template <int N>
@@ -268,296 +267,44 @@ __device__ __forceinline__ float pick(const float (&a)[N], int n) {
     for (int i = 1; i < N; ++i) r = (n == i) ? a[i] : r;
     return r;
 }
-
-template <int D>
-struct MmaTile {                            // one 16-key tile's loads for one thread
-    uint32_t kg[D / 32], kg8[D / 32];       // QK side: keys g, g+8, this thread's D/4 dims
-    uint32_t kmg[2], kmg8[2];               // K metadata of keys g, g+8, groups 2t, 2t+1
-    uint32_t vw[4][D / 64 > 0 ? D / 64 : 1];// PV side: keys 2t, 2t+1, 2t+8, 2t+9, dims D/8*g..
-    uint32_t vmv[4];                        // V metadata of those keys, group g
-};
-
-template <int D, int GS>
-__device__ __forceinline__ void mma_tile_load(MmaTile<D>& T, int jt, int j0, int j1, int64_t slot0, int g, int t,
-                                              const uint8_t* __restrict__ k_codes, const uint32_t* __restrict__ k_meta,
-                                              const uint8_t* __restrict__ v_codes,
-                                              const uint32_t* __restrict__ v_meta) {
-    constexpr int G = D / GS, KB = D / 2, KW = D / 32, VW = D / 64;
-    auto slot_of = [&](int jj) { return slot0 + (jj < j1 ? jj : j0); };   // past the range: a valid slot
-    const int64_t sg = slot_of(jt + g), sg8 = slot_of(jt + g + 8);
-    const uint32_t* pg = reinterpret_cast<const uint32_t*>(k_codes + sg * KB) + t * KW;
-    const uint32_t* pg8 = reinterpret_cast<const uint32_t*>(k_codes + sg8 * KB) + t * KW;
-    if (KW == 4) {
-        const uint4 a = __ldg(reinterpret_cast<const uint4*>(pg));
-        const uint4 c = __ldg(reinterpret_cast<const uint4*>(pg8));
-        T.kg[0] = a.x; T.kg[1 % KW] = a.y; T.kg[2 % KW] = a.z; T.kg[3 % KW] = a.w;
-        T.kg8[0] = c.x; T.kg8[1 % KW] = c.y; T.kg8[2 % KW] = c.z; T.kg8[3 % KW] = c.w;
-    } else {
-        const uint2 a = __ldg(reinterpret_cast<const uint2*>(pg));
-        const uint2 c = __ldg(reinterpret_cast<const uint2*>(pg8));
-        T.kg[0] = a.x; T.kg[1 % KW] = a.y;
-        T.kg8[0] = c.x; T.kg8[1 % KW] = c.y;
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const bool has = 2 * t + u < G;
-        T.kmg[u] = has ? __ldg(k_meta + sg * G + 2 * t + u) : 0u;
-        T.kmg8[u] = has ? __ldg(k_meta + sg8 * G + 2 * t + u) : 0u;
-    }
-    const int kv[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int64_t vs = slot_of(jt + kv[u]);
-        const uint32_t* pv = reinterpret_cast<const uint32_t*>(v_codes + vs * KB) + g * VW;
-        if (VW == 2) {
-            const uint2 a = __ldg(reinterpret_cast<const uint2*>(pv));
-            T.vw[u][0] = a.x;
-            T.vw[u][1 % (VW > 0 ? VW : 1)] = a.y;
-        } else {
-            T.vw[u][0] = __ldg(pv);
-        }
-        T.vmv[u] = (g < G) ? __ldg(v_meta + vs * G + g) : 0u;
-    }
+__device__ __forceinline__ uint32_t prmt_sel(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
 }
-
-template <int D, int GS>
-__global__ void __launch_bounds__(DA_THREADS) decode_attn_mma_kernel(
-    const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
-    const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
-    const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
-    float* __restrict__ part) {
-    constexpr int G = D / GS;              // groups per key: 1, 2 or 4
-    constexpr int NKS = D / 16;            // QK k-steps
-    constexpr int NMT = D / 16;            // PV M-tiles
-    constexpr int NW = DA_THREADS / 32;
-    constexpr float C1024 = 1024.f;
-    pdl_wait();
-    pdl_trigger();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int pair = blockIdx.x, split = blockIdx.y, nsplit = gridDim.y;
-    const int b = pair / n_heads, head = pair % n_heads;
-    const int64_t slot0 = static_cast<int64_t>(pair) * max_seq;
-    const int j0 = split * chunk;
-    const int j1 = min(pos, j0 + chunk);
-
-    // ---- query: per-group sums and the masked B operand of the QK MMA
-    const __half* qp = q + static_cast<int64_t>(b) * row_stride + head * D;
-    float Qg[G];
-#pragma unroll
-    for (int n = 0; n < G; ++n) Qg[n] = 0.f;
-#pragma unroll
-    for (int v = 0; v < D / 8; ++v) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(qp) + v);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) Qg[(8 * v) / GS] += h2f_lo(ww[k]) + h2f_hi(ww[k]);
-    }
-    // thread t's QK dims: [t*D/4, (t+1)*D/4); k-step ks uses word ks/2, nibbles e0, e0+1
-    // (e0 = 2*(ks%2)); slot pair (2t, 2t+1) <- dims (base, base+4), (2t+8, 2t+9) <- (base+1, base+5)
-    const int tgrp = (t * (D / 4)) / GS;
-    uint32_t bq[NKS][2];
-#pragma unroll
-    for (int ks = 0; ks < NKS; ++ks) {
-        const int base = t * (D / 4) + 8 * (ks / 2) + 2 * (ks % 2);
-        if (g == tgrp) {
-            bq[ks][0] = pack_half2_bits(qp[base], qp[base + 4]);
-            bq[ks][1] = pack_half2_bits(qp[base + 1], qp[base + 5]);
-        } else {
-            bq[ks][0] = bq[ks][1] = 0u;
-        }
-    }
-
-    float m = -FLT_MAX;                    // running max (warp-uniform)
-    float lsum = 0.f;                      // lanes t == 0: their keys' share of the running sum
-    float Wrun = 0.f, Urun = 0.f;          // quads g < G: group g's sum_j w_jg, sum_j p_j min_jg
-    float oacc[NMT][4];
-#pragma unroll
-    for (int i = 0; i < NMT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-
-    const int ntiles = (j1 - j0 + 15) / 16;
-    MmaTile<D> cur, nxt;
-    if (warp < ntiles) mma_tile_load<D, GS>(cur, j0 + warp * 16, j0, j1, slot0, g, t, k_codes, k_meta, v_codes, v_meta);
-    for (int tile = warp; tile < ntiles; tile += NW) {
-        const int jt = j0 + tile * 16;
-        // prefetch the warp's next tile while this one is computed
-        if (tile + NW < ntiles)
-            mma_tile_load<D, GS>(nxt, jt + NW * 16, j0, j1, slot0, g, t, k_codes, k_meta, v_codes, v_meta);
-
-        // ---- scores: S[key][group] on the tensor cores
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < NKS; ++ks) {
-            const int w = ks / 2, e0 = 2 * (ks % 2);
-            const uint32_t a[4] = {nib_pair(cur.kg[w] >> (4 * e0)), nib_pair(cur.kg8[w] >> (4 * e0)),
-                                   nib_pair(cur.kg[w] >> (4 * e0 + 4)), nib_pair(cur.kg8[w] >> (4 * e0 + 4))};
-            mma16816(sacc, a, bq[ks][0], bq[ks][1]);
-        }
-        // lane (g, t) holds columns 2t, 2t+1 of keys g (sacc[0..1]) and g+8 (sacc[2..3])
-        float sg_part = 0.f, sg8_part = 0.f;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int n = 2 * t + u;
-            if (n < G) {
-                const float Qn = pick(Qg, n);
-                const float st0 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(cur.kmg[u] >> 16)));
-                const float st1 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(cur.kmg8[u] >> 16)));
-                sg_part += fmaf(st0, sacc[u] - C1024 * Qn, h2f_lo(cur.kmg[u]) * Qn);
-                sg8_part += fmaf(st1, sacc[2 + u] - C1024 * Qn, h2f_lo(cur.kmg8[u]) * Qn);
-            }
-        }
-        if (G == 4) {
-            sg_part += __shfl_xor_sync(0xffffffffu, sg_part, 1);
-            sg8_part += __shfl_xor_sync(0xffffffffu, sg8_part, 1);
-        }
-        // every lane of quad g takes the scores of keys g, g+8 from the quad's lane t = 0
-        sg_part = __shfl_sync(0xffffffffu, sg_part, lane & ~3);
-        sg8_part = __shfl_sync(0xffffffffu, sg8_part, lane & ~3);
-        const float s_lo = (jt + g < j1) ? sg_part : -FLT_MAX;
-        const float s_hi = (jt + g + 8 < j1) ? sg8_part : -FLT_MAX;
-        float tmax = fmaxf(s_lo, s_hi);
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
-        if (tmax > m) {                    // warp-uniform
-            const float alpha = __expf(m - tmax);
-            m = tmax;
-            lsum *= alpha;
-            Wrun *= alpha;
-            Urun *= alpha;
-#pragma unroll
-            for (int i = 0; i < NMT; ++i) {
-                oacc[i][0] *= alpha;
-                oacc[i][1] *= alpha;
-                oacc[i][2] *= alpha;
-                oacc[i][3] *= alpha;
-            }
-        }
-        const float p_lo = s_lo == -FLT_MAX ? 0.f : __expf(s_lo - m);
-        const float p_hi = s_hi == -FLT_MAX ? 0.f : __expf(s_hi - m);
-        if (t == 0) lsum += p_lo + p_hi;
-        // ---- PV: B[key][n] = p_key * step_key,n in lanes (n, t'): keys 2t', 2t'+1, 2t'+8, 2t'+9
-        const float pA = __shfl_sync(0xffffffffu, p_lo, 8 * t);        // key 2t
-        const float pAh = __shfl_sync(0xffffffffu, p_hi, 8 * t);       // key 2t+8
-        const float pB = __shfl_sync(0xffffffffu, p_lo, 8 * t + 4);    // key 2t+1
-        const float pBh = __shfl_sync(0xffffffffu, p_hi, 8 * t + 4);   // key 2t+9
-        uint32_t bv0 = 0u, bv1 = 0u;
-        float wt = 0.f, ut = 0.f;
-        if (g < G) {
-            const float pk[4] = {pA, pB, pAh, pBh};
-            float wv[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float stp = group_step_fast(__ushort_as_half(static_cast<unsigned short>(cur.vmv[u] >> 16)));
-                wv[u] = __half2float(__float2half_rn(pk[u] * stp));
-                wt += wv[u];
-                ut = fmaf(pk[u], h2f_lo(cur.vmv[u]), ut);
-            }
-            bv0 = half2_bits(wv[0], wv[1]);
-            bv1 = half2_bits(wv[2], wv[3]);
-        }
-        wt += __shfl_xor_sync(0xffffffffu, wt, 1);
-        wt += __shfl_xor_sync(0xffffffffu, wt, 2);
-        ut += __shfl_xor_sync(0xffffffffu, ut, 1);
-        ut += __shfl_xor_sync(0xffffffffu, ut, 2);
-        Wrun += wt;
-        Urun += ut;
-#pragma unroll
-        for (int mt = 0; mt < NMT; ++mt) {
-            const int wi = mt / 4, by = mt % 4;
-            const uint32_t x1 = byte_pair(cur.vw[0][wi], cur.vw[1][wi], by);
-            const uint32_t x2 = byte_pair(cur.vw[2][wi], cur.vw[3][wi], by);
-            const uint32_t a[4] = {nib_pair(x1), nib_pair(x1 >> 4), nib_pair(x2), nib_pair(x2 >> 4)};
-            mma16816(oacc[mt], a, bv0, bv1);
-        }
-        cur = nxt;
-    }
-
-    // ---- warp result: o[dim] = D'[dim][grp] - 1024 W_grp + U_grp, l = sum of lsum
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-    __shared__ float sm_m[NW], sm_l[NW];
-    __shared__ float sm_o[NW][D];
-    // W/U of every group, from lanes (n, 0)
-    float Wg[G], Ug[G];
-#pragma unroll
-    for (int n = 0; n < G; ++n) {
-        Wg[n] = __shfl_sync(0xffffffffu, Wrun, 4 * n);
-        Ug[n] = __shfl_sync(0xffffffffu, Urun, 4 * n);
-    }
-#pragma unroll
-    for (int mt = 0; mt < NMT; ++mt) {
-        const int wi = mt / 4, by = mt % 4;
-        const int dlo = (D / 8) * g + 8 * wi + 2 * by;          // row g ; row g+8 is dlo + 1
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int dim = dlo + hr;
-            const int n = dim / GS;
-            if (n / 2 == t) {
-                // static register indices only (a runtime index would move oacc to local memory)
-                const float v = (n % 2) ? oacc[mt][2 * hr + 1] : oacc[mt][2 * hr];
-                sm_o[warp][dim] = v - C1024 * pick(Wg, n) + pick(Ug, n);
-            }
-        }
-    }
-    if (lane == 0) {
-        sm_m[warp] = m;
-        sm_l[warp] = lsum;
-    }
-    __syncthreads();
-    float M = -FLT_MAX;
-#pragma unroll
-    for (int i = 0; i < NW; ++i) M = fmaxf(M, sm_m[i]);
-    float* out = part + (static_cast<int64_t>(pair) * nsplit + split) * (D + 2);
-    for (int d = threadIdx.x; d < D; d += DA_THREADS) {
-        float o = 0.f;
-#pragma unroll
-        for (int i = 0; i < NW; ++i) {
-            const float f = sm_l[i] > 0.f ? __expf(sm_m[i] - M) : 0.f;
-            o = fmaf(f, sm_o[i][d], o);
-        }
-        out[2 + d] = o;
-    }
-    if (threadIdx.x == 0) {
-        float L = 0.f;
-#pragma unroll
-        for (int i = 0; i < NW; ++i) L += sm_l[i] > 0.f ? __expf(sm_m[i] - M) * sm_l[i] : 0.f;
-        out[0] = M;
-        out[1] = L;
-    }
-}
-
-// ---------------------------------------------------------------------------------
-// decode attention on the tensor cores with the key range staged in shared memory.
-// Same arithmetic as decode_attn_mma_kernel; the codes and metadata of 64-key chunks
-// are copied with cp.async into a DA_NS-deep ring (all threads of the CTA take part),
-// so DA_NS - 1 chunks are always in flight. In every chunk warp w owns tile w (keys
-// 16w..16w+15) and keeps its own online-softmax state across chunks.
-constexpr int DA_CHUNK = 64;
-constexpr int DA_NS = 4;
-
 __device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool pred) {
     const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
     const int n = pred ? 4 : 0;
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(s), "l"(gmem), "r"(n) : "memory");
 }
 
+// One CTA (4 warps) streams the key range [j0, j1) of one (sequence, head) in stages of
+// DT_KEYS keys through a cp.async ring (3 stages deep at head_dim 64, 2 at 128); in a stage warp w owns keys
+// [32 w, 32 w + 32) as two 16-key tiles, with one online-softmax update per stage.
+// Writes the split's partial {max, sum, unnormalised output} for the combine kernel.
+constexpr int DT_KEYS = 128;
+
 template <int D, int GS>
-__global__ void __launch_bounds__(DA_THREADS) decode_attn_staged_kernel(
+__global__ void __launch_bounds__(DA_THREADS) decode_attn_tc_kernel(
     const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
     const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
     const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
     float* __restrict__ part) {
     constexpr int G = D / GS;              // groups per key: 1, 2 or 4
     constexpr int KB = D / 2;              // code bytes per key
-    constexpr int NKS = D / 16;            // QK k-steps
-    constexpr int NMT = D / 16;            // PV M-tiles
-    constexpr int NW = DA_THREADS / 32;    // warps = tiles per chunk
-    constexpr int CODE_BYTES = DA_CHUNK * KB;
-    constexpr int META_WORDS = DA_CHUNK * G;
-    constexpr int STAGE = 2 * CODE_BYTES + 2 * META_WORDS * 4;
-    constexpr float C1024 = 1024.f;
-    static_assert(NW * 16 == DA_CHUNK, "one 16-key tile per warp and chunk");
-    __shared__ __align__(16) uint8_t ring[DA_NS][STAGE];
+    constexpr int KW = D / 32;             // QK: code words per key and thread (D/4 dims)
+    constexpr int VW = D / 64;             // PV: code words per key and thread (D/8 dims)
+    constexpr int NMT = D / 16;            // PV M-tiles (16 dims each)
+    constexpr int NW = DA_THREADS / 32;
+    constexpr int CODE = DT_KEYS * KB;     // code bytes of a stage (keys or values)
+    constexpr int META = DT_KEYS * G;      // metadata words of a stage (keys or values)
+    constexpr int STAGE = 2 * CODE + 2 * META * 4;
+    constexpr int DT_NS = D == 128 ? 2 : 3;   // stages in flight (static shared memory < 48 KB)
+    static_assert(NW * 32 == DT_KEYS, "32 keys per warp and stage");
+    static_assert(CODE % (16 * DA_THREADS) == 0 && META % DA_THREADS == 0, "whole copy rounds");
+    __shared__ __align__(16) uint8_t ring[DT_NS][STAGE];
+    __shared__ float sm_m[NW], sm_l[NW];
+    __shared__ float sm_o[NW][D];
     pdl_wait();
     pdl_trigger();
 
@@ -567,215 +314,267 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_staged_kernel(
     const int b = pair / n_heads, head = pair % n_heads;
     const int64_t slot0 = static_cast<int64_t>(pair) * max_seq;
     const int j0 = split * chunk;
-    const int j1 = min(pos, j0 + chunk);
-    const int nchunks = (j1 - j0 + DA_CHUNK - 1) / DA_CHUNK;
+    const int nkeys = min(pos, j0 + chunk) - j0;                  // keys of this split (> 0)
+    const int nst = (nkeys + DT_KEYS - 1) / DT_KEYS;
 
-    // copy chunk c into ring slot c % DA_NS (keys past j1 are zero-filled, never read)
-    auto load_chunk = [&](int c) {
-        uint8_t* st = ring[c % DA_NS];
-        const int jc = j0 + c * DA_CHUNK;
-        const int n = min(DA_CHUNK, j1 - jc);
-        for (int u = threadIdx.x; u < CODE_BYTES / 16; u += DA_THREADS) {
-            const int key = (u * 16) / KB;
-            const bool ok = key < n;
-            const int64_t off = (slot0 + (ok ? jc : j0)) * KB + u * 16;
-            cp_async16(st + u * 16, k_codes + off, ok);
-            cp_async16(st + CODE_BYTES + u * 16, v_codes + off, ok);
+    // ---- stage copies: every thread moves CODE/16/128 16-byte units of each code tensor
+    // and META/128 metadata words of each metadata tensor; keys past the range are
+    // zero-filled (a zero scale gives step 0, so they contribute nothing)
+    const uint8_t* kc_src = k_codes + (slot0 + j0) * KB;
+    const uint8_t* vc_src = v_codes + (slot0 + j0) * KB;
+    const uint32_t* km_src = k_meta + (slot0 + j0) * G;
+    const uint32_t* vm_src = v_meta + (slot0 + j0) * G;
+    auto load_stage = [&](int s) {
+        uint8_t* st = ring[s % DT_NS];
+        const int kbase = s * DT_KEYS;
+#pragma unroll
+        for (int i = 0; i < CODE / (16 * DA_THREADS); ++i) {
+            const int u = threadIdx.x + i * DA_THREADS;
+            const bool ok = kbase + (u * 16) / KB < nkeys;
+            const int64_t off = ok ? static_cast<int64_t>(kbase) * KB + u * 16 : 0;
+            cp_async16(st + u * 16, kc_src + off, ok);
+            cp_async16(st + CODE + u * 16, vc_src + off, ok);
         }
-        for (int u = threadIdx.x; u < META_WORDS; u += DA_THREADS) {
-            const int key = u / G;
-            const bool ok = key < n;
-            const int64_t off = (slot0 + (ok ? jc : j0)) * G + u;
-            cp_async4(st + 2 * CODE_BYTES + u * 4, k_meta + off, ok);
-            cp_async4(st + 2 * CODE_BYTES + META_WORDS * 4 + u * 4, v_meta + off, ok);
+#pragma unroll
+        for (int i = 0; i < META / DA_THREADS; ++i) {
+            const int u = threadIdx.x + i * DA_THREADS;
+            const bool ok = kbase + u / G < nkeys;
+            const int64_t off = ok ? static_cast<int64_t>(kbase) * G + u : 0;
+            cp_async4(st + 2 * CODE + u * 4, km_src + off, ok);
+            cp_async4(st + 2 * CODE + META * 4 + u * 4, vm_src + off, ok);
         }
     };
 #pragma unroll
-    for (int c = 0; c < DA_NS - 1; ++c) {
-        if (c < nchunks) load_chunk(c);
+    for (int s = 0; s < DT_NS - 1; ++s) {
+        if (s < nst) load_stage(s);
         cp_async_commit();
     }
 
-    // ---- query: per-group sums and the masked B operand of the QK MMA
+    // ---- query: group sums and the QK B operand (this thread's D/4 dims, column g)
     const __half* qp = q + static_cast<int64_t>(b) * row_stride + head * D;
-    float Qg[G];
+    float Qg[G], QC[G];
 #pragma unroll
-    for (int n = 0; n < G; ++n) Qg[n] = 0.f;
+    for (int n = 0; n < G; ++n) Qg[n] = QC[n] = 0.f;
 #pragma unroll
     for (int v = 0; v < D / 8; ++v) {
         const uint4 w = __ldg(reinterpret_cast<const uint4*>(qp) + v);
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) Qg[(8 * v) / GS] += h2f_lo(ww[k]) + h2f_hi(ww[k]);
+        for (int k = 0; k < 4; ++k) {
+            const float lo = h2f_lo(ww[k]), hi = h2f_hi(ww[k]);     // even, odd dim
+            Qg[(8 * v) / GS] += lo + hi;
+            QC[(8 * v) / GS] += 1024.f * lo + 64.f * hi;
+        }
     }
-    const int tgrp = (t * (D / 4)) / GS;
-    uint32_t bq[NKS][2];
+    const int tgrp = (t * (D / 4)) / GS;   // group of this thread's QK dims
+    const __half sixteenth = __float2half(0.0625f);
+    uint32_t bq[2 * KW][2];
 #pragma unroll
-    for (int ks = 0; ks < NKS; ++ks) {
-        const int base = t * (D / 4) + 8 * (ks / 2) + 2 * (ks % 2);
+    for (int ks = 0; ks < 2 * KW; ++ks) {
+        // k-step ks uses word ks/2; its registers hold dims (d, d+4) and (d+1, d+5)
+        const int d = t * (D / 4) + 8 * (ks / 2) + 2 * (ks % 2);
         if (g == tgrp) {
-            bq[ks][0] = pack_half2_bits(qp[base], qp[base + 4]);
-            bq[ks][1] = pack_half2_bits(qp[base + 1], qp[base + 5]);
+            bq[ks][0] = pack_half2_bits(qp[d], qp[d + 4]);
+            bq[ks][1] = pack_half2_bits(__hmul(qp[d + 1], sixteenth), __hmul(qp[d + 5], sixteenth));
         } else {
             bq[ks][0] = bq[ks][1] = 0u;
         }
     }
 
-    float m = -FLT_MAX, lsum = 0.f, Wrun = 0.f, Urun = 0.f;
+    // ---- PV: owner lanes of the w values and the lanes they are gathered from.
+    // Lane (g, t) owns group own_n of key g + 8 own_h (G = 1: t < 2; G = 2: all; G = 4:
+    // both halves of group t).
+    const int own_n = (G == 4) ? t : t % G;
+    const int own_h = (G == 4) ? 0 : t / G;
+    const bool owner = (G == 4) || (t < 2 * G);
+    // b0 needs keys 2t, 2t+1 (half 0) and b1 keys 2t+8, 2t+9 (half 1), group g
+    const int gn = g < G ? g : 0;
+    const int src_a0 = 4 * (2 * t) + gn;                              // half 0: owner t = n
+    const int src_a1 = 4 * (2 * t + 1) + gn;
+    const int src_b0 = 4 * (2 * t) + ((G == 4) ? gn : G + gn);        // half 1: t = G + n (G < 4)
+    const int src_b1 = 4 * (2 * t + 1) + ((G == 4) ? gn : G + gn);
+
+    float m = -FLT_MAX, lsum = 0.f, Wl = 0.f, Ul = 0.f;
     float oacc[NMT][4];
 #pragma unroll
     for (int i = 0; i < NMT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
 
-    for (int c = 0; c < nchunks; ++c) {
-        if (c + DA_NS - 1 < nchunks) load_chunk(c + DA_NS - 1);
+    for (int s = 0; s < nst; ++s) {
+        if (s + DT_NS - 1 < nst) load_stage(s + DT_NS - 1);
         cp_async_commit();
-        cp_async_wait<DA_NS - 1>();
+        cp_async_wait<DT_NS - 1>();
         __syncthreads();
-        const uint8_t* st = ring[c % DA_NS];
-        const uint8_t* kc = st + warp * 16 * KB;                     // this warp's tile
-        const uint8_t* vc = st + CODE_BYTES + warp * 16 * KB;
-        const uint32_t* km = reinterpret_cast<const uint32_t*>(st + 2 * CODE_BYTES) + warp * 16 * G;
-        const uint32_t* vm = reinterpret_cast<const uint32_t*>(st + 2 * CODE_BYTES + META_WORDS * 4) + warp * 16 * G;
-        const int jt = j0 + c * DA_CHUNK + warp * 16;
-
-        // ---- scores
-        uint32_t kg[D / 32], kg8[D / 32];
-        if (D == 128) {
-            const uint4 a = *reinterpret_cast<const uint4*>(kc + g * KB + t * (D / 8));
-            const uint4 e = *reinterpret_cast<const uint4*>(kc + (g + 8) * KB + t * (D / 8));
-            kg[0] = a.x; kg[1 % (D / 32)] = a.y; kg[2 % (D / 32)] = a.z; kg[3 % (D / 32)] = a.w;
-            kg8[0] = e.x; kg8[1 % (D / 32)] = e.y; kg8[2 % (D / 32)] = e.z; kg8[3 % (D / 32)] = e.w;
-        } else {
-            const uint2 a = *reinterpret_cast<const uint2*>(kc + g * KB + t * (D / 8));
-            const uint2 e = *reinterpret_cast<const uint2*>(kc + (g + 8) * KB + t * (D / 8));
-            kg[0] = a.x; kg[1 % (D / 32)] = a.y;
-            kg8[0] = e.x; kg8[1 % (D / 32)] = e.y;
-        }
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int kw0 = s * DT_KEYS + warp * 32;                 // the warp's first key
+        if (kw0 < nkeys) {
+            const uint8_t* st = ring[s % DT_NS];
+            const uint32_t* kmeta = reinterpret_cast<const uint32_t*>(st + 2 * CODE) + warp * 32 * G;
+            const uint32_t* vmeta = reinterpret_cast<const uint32_t*>(st + 2 * CODE + META * 4) + warp * 32 * G;
+            // ---- scores of the two tiles: keys (tile 16 + g) and (tile 16 + g + 8)
+            float sc[2][2];
 #pragma unroll
-        for (int ks = 0; ks < NKS; ++ks) {
-            const int w = ks / 2, e0 = 2 * (ks % 2);
-            const uint32_t a[4] = {nib_pair(kg[w] >> (4 * e0)), nib_pair(kg8[w] >> (4 * e0)),
-                                   nib_pair(kg[w] >> (4 * e0 + 4)), nib_pair(kg8[w] >> (4 * e0 + 4))};
-            mma16816(sacc, a, bq[ks][0], bq[ks][1]);
-        }
-        float sg_part = 0.f, sg8_part = 0.f;
+            for (int tile = 0; tile < 2; ++tile) {
+                const uint8_t* kc = st + (warp * 32 + tile * 16) * KB + t * (D / 8);
+                uint32_t x0[KW], x8[KW];
+                if (KW == 4) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(kc + g * KB);
+                    const uint4 c = *reinterpret_cast<const uint4*>(kc + (g + 8) * KB);
+                    x0[0] = a.x; x0[1 % KW] = a.y; x0[2 % KW] = a.z; x0[3 % KW] = a.w;
+                    x8[0] = c.x; x8[1 % KW] = c.y; x8[2 % KW] = c.z; x8[3 % KW] = c.w;
+                } else {
+                    const uint2 a = *reinterpret_cast<const uint2*>(kc + g * KB);
+                    const uint2 c = *reinterpret_cast<const uint2*>(kc + (g + 8) * KB);
+                    x0[0] = a.x; x0[1 % KW] = a.y;
+                    x8[0] = c.x; x8[1 % KW] = c.y;
+                }
+                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int n = 2 * t + u;
-            if (n < G) {
-                const uint32_t m0 = km[g * G + n], m8 = km[(g + 8) * G + n];
-                const float Qn = pick(Qg, n);
-                const float st0 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(m0 >> 16)));
-                const float st8 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(m8 >> 16)));
-                sg_part += fmaf(st0, sacc[u] - C1024 * Qn, h2f_lo(m0) * Qn);
-                sg8_part += fmaf(st8, sacc[2 + u] - C1024 * Qn, h2f_lo(m8) * Qn);
+                for (int w = 0; w < KW; ++w) {
+                    const uint32_t y0 = x0[w] >> 8, y8 = x8[w] >> 8;
+                    const uint32_t a0[4] = {nib_lo(x0[w]), nib_lo(x8[w]), nib_hi(x0[w]), nib_hi(x8[w])};
+                    mma16816(sacc, a0, bq[2 * w][0], bq[2 * w][1]);
+                    const uint32_t a1[4] = {nib_lo(y0), nib_lo(y8), nib_hi(y0), nib_hi(y8)};
+                    mma16816(sacc, a1, bq[2 * w + 1][0], bq[2 * w + 1][1]);
+                }
+                // per key: sum over the groups this lane holds (columns 2t, 2t+1)
+                float s0 = 0.f, s8 = 0.f;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int n = 2 * t + u;
+                    if (n < G) {
+                        const uint32_t m0 = kmeta[(tile * 16 + g) * G + n], m8 = kmeta[(tile * 16 + g + 8) * G + n];
+                        const float qc = pick(QC, n), qg = pick(Qg, n);
+                        const float st0 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(m0 >> 16)));
+                        const float st8 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(m8 >> 16)));
+                        s0 += fmaf(st0, sacc[u] - qc, h2f_lo(m0) * qg);
+                        s8 += fmaf(st8, sacc[2 + u] - qc, h2f_lo(m8) * qg);
+                    }
+                }
+                if (G == 4) {
+                    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+                    s8 += __shfl_xor_sync(0xffffffffu, s8, 1);
+                }
+                s0 = __shfl_sync(0xffffffffu, s0, lane & ~3);
+                s8 = __shfl_sync(0xffffffffu, s8, lane & ~3);
+                const int kt = kw0 + tile * 16;
+                sc[tile][0] = (kt + g < nkeys) ? s0 : -FLT_MAX;
+                sc[tile][1] = (kt + g + 8 < nkeys) ? s8 : -FLT_MAX;
             }
-        }
-        if (G == 4) {
-            sg_part += __shfl_xor_sync(0xffffffffu, sg_part, 1);
-            sg8_part += __shfl_xor_sync(0xffffffffu, sg8_part, 1);
-        }
-        sg_part = __shfl_sync(0xffffffffu, sg_part, lane & ~3);
-        sg8_part = __shfl_sync(0xffffffffu, sg8_part, lane & ~3);
-        const float s_lo = (jt + g < j1) ? sg_part : -FLT_MAX;
-        const float s_hi = (jt + g + 8 < j1) ? sg8_part : -FLT_MAX;
-        float tmax = fmaxf(s_lo, s_hi);
+            // ---- one online-softmax update for the 32 keys
+            float tmax = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
-        if (tmax > m) {                    // warp-uniform
-            const float alpha = __expf(m - tmax);
-            m = tmax;
-            lsum *= alpha;
-            Wrun *= alpha;
-            Urun *= alpha;
+            for (int off = 4; off < 32; off <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
+            if (tmax > m) {                        // warp-uniform
+                const float alpha = __expf(m - tmax);
+                m = tmax;
+                lsum *= alpha;
+                Wl *= alpha;
+                Ul *= alpha;
 #pragma unroll
-            for (int i = 0; i < NMT; ++i) {
-                oacc[i][0] *= alpha;
-                oacc[i][1] *= alpha;
-                oacc[i][2] *= alpha;
-                oacc[i][3] *= alpha;
+                for (int i = 0; i < NMT; ++i) {
+                    oacc[i][0] *= alpha;
+                    oacc[i][1] *= alpha;
+                    oacc[i][2] *= alpha;
+                    oacc[i][3] *= alpha;
+                }
             }
-        }
-        const float p_lo = s_lo == -FLT_MAX ? 0.f : __expf(s_lo - m);
-        const float p_hi = s_hi == -FLT_MAX ? 0.f : __expf(s_hi - m);
-        if (t == 0) lsum += p_lo + p_hi;
-        // ---- values
-        const float pA = __shfl_sync(0xffffffffu, p_lo, 8 * t);
-        const float pAh = __shfl_sync(0xffffffffu, p_hi, 8 * t);
-        const float pB = __shfl_sync(0xffffffffu, p_lo, 8 * t + 4);
-        const float pBh = __shfl_sync(0xffffffffu, p_hi, 8 * t + 4);
-        uint32_t bv0 = 0u, bv1 = 0u;
-        float wt = 0.f, ut = 0.f;
-        if (g < G) {
-            const float pk[4] = {pA, pB, pAh, pBh};
-            float wv[4];
+            float pr[2][2];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t mv = vm[(2 * t + (u & 1) + 8 * (u >> 1)) * G + g];
-                const float stp = group_step_fast(__ushort_as_half(static_cast<unsigned short>(mv >> 16)));
-                wv[u] = __half2float(__float2half_rn(pk[u] * stp));
-                wt += wv[u];
-                ut = fmaf(pk[u], h2f_lo(mv), ut);
+            for (int tile = 0; tile < 2; ++tile)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) pr[tile][h] = sc[tile][h] == -FLT_MAX ? 0.f : __expf(sc[tile][h] - m);
+            if (t == 0) lsum += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+            // ---- values
+#pragma unroll
+            for (int tile = 0; tile < 2; ++tile) {
+                // owner lanes: w = fp16(p step) of (key g + 8 h, group n); running W, U
+                uint32_t wb[2] = {0u, 0u};
+#pragma unroll
+                for (int hh = 0; hh < ((G == 4) ? 2 : 1); ++hh) {
+                    const int h = (G == 4) ? hh : own_h;
+                    if (owner) {
+                        const uint32_t mv = vmeta[(tile * 16 + g + 8 * h) * G + own_n];
+                        const float stp = group_step_fast(__ushort_as_half(static_cast<unsigned short>(mv >> 16)));
+                        const float pk = h ? pr[tile][1] : pr[tile][0];
+                        const __half w16 = __float2half_rn(pk * stp);
+                        Wl += __half2float(w16);
+                        Ul = fmaf(pk, h2f_lo(mv), Ul);
+                        wb[hh] = static_cast<uint32_t>(__half_as_ushort(w16));
+                    }
+                }
+                // gather the B operand: keys 2t, 2t+1 (b0) and 2t+8, 2t+9 (b1) of group g
+                const uint32_t lo_a = __shfl_sync(0xffffffffu, wb[0], src_a0);
+                const uint32_t lo_b = __shfl_sync(0xffffffffu, wb[0], src_a1);
+                const uint32_t hi_a = __shfl_sync(0xffffffffu, wb[(G == 4) ? 1 : 0], src_b0);
+                const uint32_t hi_b = __shfl_sync(0xffffffffu, wb[(G == 4) ? 1 : 0], src_b1);
+                const uint32_t b0 = g < G ? (lo_a | (lo_b << 16)) : 0u;
+                const uint32_t b1 = g < G ? (hi_a | (hi_b << 16)) : 0u;
+                // A: transposed codes; thread g holds D/16 bytes (dims D/8 g ..) of keys
+                // 2t, 2t+1, 2t+8, 2t+9
+                const uint8_t* vc = st + CODE + (warp * 32 + tile * 16) * KB + g * (D / 16);
+                uint32_t vk[4][VW > 0 ? VW : 1];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int key = 2 * t + (u & 1) + 8 * (u >> 1);
+                    if (VW == 2) {
+                        const uint2 a = *reinterpret_cast<const uint2*>(vc + key * KB);
+                        vk[u][0] = a.x;
+                        vk[u][1 % (VW > 0 ? VW : 1)] = a.y;
+                    } else {
+                        vk[u][0] = *reinterpret_cast<const uint32_t*>(vc + key * KB);
+                    }
+                }
+#pragma unroll
+                for (int mt = 0; mt < NMT; ++mt) {
+                    const int wi = mt / 4, by = mt % 4;
+                    // byte `by` of key 2t -> bytes 0,1 and of key 2t+1 -> bytes 2,3
+                    const uint32_t sel = static_cast<uint32_t>(by * 0x11 + (4 + by) * 0x1100);
+                    const uint32_t x1 = prmt_sel(vk[0][wi], vk[1][wi], sel);
+                    const uint32_t x2 = prmt_sel(vk[2][wi], vk[3][wi], sel);
+                    const uint32_t a[4] = {nib_lo(x1), nib_hi(x1), nib_lo(x2), nib_hi(x2)};
+                    mma16816(oacc[mt], a, b0, b1);
+                }
             }
-            bv0 = half2_bits(wv[0], wv[1]);
-            bv1 = half2_bits(wv[2], wv[3]);
-        }
-        wt += __shfl_xor_sync(0xffffffffu, wt, 1);
-        wt += __shfl_xor_sync(0xffffffffu, wt, 2);
-        ut += __shfl_xor_sync(0xffffffffu, ut, 1);
-        ut += __shfl_xor_sync(0xffffffffu, ut, 2);
-        Wrun += wt;
-        Urun += ut;
-        // PV side: thread g holds dims [g*D/8, (g+1)*D/8) of keys 2t, 2t+1, 2t+8, 2t+9,
-        // i.e. D/16 code bytes of each key starting at byte g*D/16
-        uint32_t vw[4][D / 64];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (D == 128) {
-                const uint2 a = *reinterpret_cast<const uint2*>(vc + (2 * t + (u & 1) + 8 * (u >> 1)) * KB + g * (D / 16));
-                vw[u][0] = a.x;
-                vw[u][1 % (D / 64)] = a.y;
-            } else {
-                vw[u][0] = *reinterpret_cast<const uint32_t*>(vc + (2 * t + (u & 1) + 8 * (u >> 1)) * KB + g * (D / 16));
-            }
-        }
-#pragma unroll
-        for (int mt = 0; mt < NMT; ++mt) {
-            const int wi = mt / 4, by = mt % 4;
-            const uint32_t x1 = byte_pair(vw[0][wi], vw[1][wi], by);
-            const uint32_t x2 = byte_pair(vw[2][wi], vw[3][wi], by);
-            const uint32_t a[4] = {nib_pair(x1), nib_pair(x1 >> 4), nib_pair(x2), nib_pair(x2 >> 4)};
-            mma16816(oacc[mt], a, bv0, bv1);
         }
         __syncthreads();                   // the slot is refilled by the next iteration
     }
     cp_async_wait<0>();
 
-    // ---- warp result and CTA merge (as in decode_attn_mma_kernel)
+    // ---- warp result: W_n, U_n per group (sum over the owner lanes), then the rows
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-    __shared__ float sm_m[NW], sm_l[NW];
-    __shared__ float sm_o[NW][D];
-    float Wg[G], Ug[G];
+    for (int off = 4; off < 32; off <<= 1) {
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+        Wl += __shfl_xor_sync(0xffffffffu, Wl, off);
+        Ul += __shfl_xor_sync(0xffffffffu, Ul, off);
+    }
+    if (G == 1) {                          // owners t = 0, 1 (t = 2, 3 hold 0)
+        Wl += __shfl_xor_sync(0xffffffffu, Wl, 1);
+        Ul += __shfl_xor_sync(0xffffffffu, Ul, 1);
+        Wl += __shfl_xor_sync(0xffffffffu, Wl, 2);
+        Ul += __shfl_xor_sync(0xffffffffu, Ul, 2);
+    } else if (G == 2) {                   // owners of group t % 2: t and t ^ 2
+        Wl += __shfl_xor_sync(0xffffffffu, Wl, 2);
+        Ul += __shfl_xor_sync(0xffffffffu, Ul, 2);
+    }
+    // now lane t of every quad holds W, U of group t (G = 1: all lanes hold group 0)
+    float Wn[2], Un[2];                    // groups 2t and 2t + 1
 #pragma unroll
-    for (int n = 0; n < G; ++n) {
-        Wg[n] = __shfl_sync(0xffffffffu, Wrun, 4 * n);
-        Ug[n] = __shfl_sync(0xffffffffu, Urun, 4 * n);
+    for (int u = 0; u < 2; ++u) {
+        const int n = (2 * t + u) < G ? 2 * t + u : 0;
+        Wn[u] = __shfl_sync(0xffffffffu, Wl, (lane & ~3) | (G == 1 ? 0 : n));
+        Un[u] = __shfl_sync(0xffffffffu, Ul, (lane & ~3) | (G == 1 ? 0 : n));
     }
 #pragma unroll
     for (int mt = 0; mt < NMT; ++mt) {
-        const int wi = mt / 4, by = mt % 4;
-        const int dlo = (D / 8) * g + 8 * wi + 2 * by;
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int dim = dlo + hr;
-            const int n = dim / GS;
-            if (n / 2 == t) {
-                // static register indices only (a runtime index would move oacc to local memory)
-                const float v = (n % 2) ? oacc[mt][2 * hr + 1] : oacc[mt][2 * hr];
-                sm_o[warp][dim] = v - C1024 * pick(Wg, n) + pick(Ug, n);
-            }
+        const int de = 2 * (g * (D / 16) + mt);        // even dim of row g; row g + 8 is de + 1
+        const int n = de / GS;
+        if (n / 2 == t) {
+            // static register indices only (a runtime index would move oacc to local memory)
+            const bool odd_col = (n % 2) != 0;
+            const float ev = odd_col ? oacc[mt][1] : oacc[mt][0];
+            const float od = odd_col ? oacc[mt][3] : oacc[mt][2];
+            const float W = odd_col ? Wn[1] : Wn[0], U = odd_col ? Un[1] : Un[0];
+            sm_o[warp][de] = ev - 1024.f * W + U;
+            sm_o[warp][de + 1] = (od - 1024.f * W) * 0.0625f + U;
         }
     }
     if (lane == 0) {
@@ -1058,7 +857,7 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
     launch_k(decode_attn_split_kernel<D_, B_, G_>, grid, dim3(DA_THREADS), 0, st, true, qh, row_stride, kc, km, vc, \
              vm, c->n_heads, c->max_seq, pos, chunk, part)
 #define MMA(D_, G_)                                                                                      \
-    launch_k(decode_attn_staged_kernel<D_, G_>, grid, dim3(DA_THREADS), 0, st, true, qh, row_stride, kc, km, vc, vm, \
+    launch_k(decode_attn_tc_kernel<D_, G_>, grid, dim3(DA_THREADS), 0, st, true, qh, row_stride, kc, km, vc, vm, \
              c->n_heads, c->max_seq, pos, chunk, part)
         const int D = c->head_dim, B = c->cfg.num_bits, G = c->cfg.group_size;
         if (D == 64 && B == 4 && G == 64) MMA(64, 64);

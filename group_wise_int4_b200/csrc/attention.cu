@@ -281,15 +281,21 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool pre
 // One CTA (4 warps) streams the key range [j0, j1) of one (sequence, head) in stages of
 // DT_KEYS keys through a cp.async ring (3 stages deep at head_dim 64, 2 at 128); in a stage warp w owns keys
 // [32 w, 32 w + 32) as two 16-key tiles, with one online-softmax update per stage.
-// Writes the split's partial {max, sum, unnormalised output} for the combine kernel.
+// Writes the split's partial {max, sum, unnormalised output} for the combine kernel;
+// with a single split (gridDim.y == 1) it does the combine step itself: it folds in the
+// fresh key/value of the current token and writes the normalised output o (in the
+// interleaved 8-block order when perm != 0).
 constexpr int DT_KEYS = 128;
 
+// 7 CTAs per SM at head_dim 64 (all 1024 CTAs of a 32 x 32-head decode in one wave),
+// 4 at head_dim 128
 template <int D, int GS>
-__global__ void __launch_bounds__(DA_THREADS) decode_attn_tc_kernel(
+__global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : 4) decode_attn_tc_kernel(
     const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
     const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
     const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
-    float* __restrict__ part) {
+    float* __restrict__ part, const __half* __restrict__ k_new, const __half* __restrict__ v_new,
+    __half* __restrict__ o, int perm) {
     constexpr int G = D / GS;              // groups per key: 1, 2 or 4
     constexpr int KB = D / 2;              // code bytes per key
     constexpr int KW = D / 32;             // QK: code words per key and thread (D/4 dims)
@@ -305,6 +311,7 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_tc_kernel(
     __shared__ __align__(16) uint8_t ring[DT_NS][STAGE];
     __shared__ float sm_m[NW], sm_l[NW];
     __shared__ float sm_o[NW][D];
+    __shared__ float sm_red[NW];
     pdl_wait();
     pdl_trigger();
 
@@ -315,6 +322,7 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_tc_kernel(
     const int64_t slot0 = static_cast<int64_t>(pair) * max_seq;
     const int j0 = split * chunk;
     const int nkeys = min(pos, j0 + chunk) - j0;                  // keys of this split (> 0)
+    static_assert(D <= DA_THREADS, "one thread per output dim");
     const int nst = (nkeys + DT_KEYS - 1) / DT_KEYS;
 
     // ---- stage copies: every thread moves CODE/16/128 16-byte units of each code tensor
@@ -582,18 +590,50 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_tc_kernel(
         sm_l[warp] = lsum;
     }
     __syncthreads();
+    if (nsplit == 1) {
+        // single split: the combine step here. Fresh score q . k_new (one dim per thread).
+        const int d = threadIdx.x;
+        const int64_t off = static_cast<int64_t>(b) * row_stride + head * D + d;
+        float sn = d < D ? __half2float(qp[d]) * __half2float(k_new[off]) : 0.f;
+#pragma unroll
+        for (int w = 16; w > 0; w >>= 1) sn += __shfl_xor_sync(0xffffffffu, sn, w);
+        if (lane == 0) sm_red[warp] = sn;
+        __syncthreads();
+        float snew = 0.f;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) snew += sm_red[i];
+        float M = snew;
+#pragma unroll
+        for (int i = 0; i < NW; ++i)
+            if (sm_l[i] > 0.f) M = fmaxf(M, sm_m[i]);
+        if (d < D) {
+            const float fn = __expf(snew - M);
+            float L = fn, acc = fn * __half2float(v_new[off]);
+#pragma unroll
+            for (int i = 0; i < NW; ++i) {
+                if (!(sm_l[i] > 0.f)) continue;
+                const float f = __expf(sm_m[i] - M);
+                L = fmaf(f, sm_l[i], L);
+                acc = fmaf(f, sm_o[i][d], acc);
+            }
+            // perm: interleaved 8-block order for the next GEMM (element k -> 2(k%4) + (k/4)%2)
+            const int dd = perm ? ((d & ~7) | ((d & 3) << 1) | ((d >> 2) & 1)) : d;
+            o[static_cast<int64_t>(b) * n_heads * D + head * D + dd] = __float2half_rn(acc / L);
+        }
+        return;
+    }
     float M = -FLT_MAX;
 #pragma unroll
     for (int i = 0; i < NW; ++i) M = fmaxf(M, sm_m[i]);
     float* out = part + (static_cast<int64_t>(pair) * nsplit + split) * (D + 2);
     for (int d = threadIdx.x; d < D; d += DA_THREADS) {
-        float o = 0.f;
+        float acc = 0.f;
 #pragma unroll
         for (int i = 0; i < NW; ++i) {
             const float f = sm_l[i] > 0.f ? __expf(sm_m[i] - M) : 0.f;
-            o = fmaf(f, sm_o[i][d], o);
+            acc = fmaf(f, sm_o[i][d], acc);
         }
-        out[2 + d] = o;
+        out[2 + d] = acc;
     }
     if (threadIdx.x == 0) {
         float L = 0.f;
@@ -851,6 +891,12 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
     const uint8_t* vc = static_cast<const uint8_t*>(c->v_codes);
     const uint32_t* km = static_cast<const uint32_t*>(c->k_meta);
     const uint32_t* vm = static_cast<const uint32_t*>(c->v_meta);
+    const __half* kn = static_cast<const __half*>(k_new);
+    const __half* vn = static_cast<const __half*>(v_new);
+    __half* oh = static_cast<__half*>(o);
+    const int D = c->head_dim, B = c->cfg.num_bits, G = c->cfg.group_size;
+    // 4-bit caches with a single split finish in the split kernel (no combine launch)
+    bool combined = false;
     if (ns > 0) {
         const dim3 grid(pairs, ns);
 #define SPLIT(D_, B_, G_)                                                                                 \
@@ -858,30 +904,30 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
              vm, c->n_heads, c->max_seq, pos, chunk, part)
 #define MMA(D_, G_)                                                                                      \
     launch_k(decode_attn_tc_kernel<D_, G_>, grid, dim3(DA_THREADS), 0, st, true, qh, row_stride, kc, km, vc, vm, \
-             c->n_heads, c->max_seq, pos, chunk, part)
-        const int D = c->head_dim, B = c->cfg.num_bits, G = c->cfg.group_size;
-        if (D == 64 && B == 4 && G == 64) MMA(64, 64);
-        else if (D == 64 && B == 4 && G == 32) MMA(64, 32);
-        else if (D == 128 && B == 4 && G == 64) MMA(128, 64);
-        else if (D == 128 && B == 4 && G == 32) MMA(128, 32);
-        else if (D == 64 && B == 8 && G == 64) SPLIT(64, 8, 64);
-        else if (D == 64 && B == 8 && G == 32) SPLIT(64, 8, 32);
-        else if (D == 128 && B == 4 && G == 64) SPLIT(128, 4, 64);
-        else if (D == 128 && B == 4 && G == 32) SPLIT(128, 4, 32);
-        else if (D == 128 && B == 8 && G == 64) SPLIT(128, 8, 64);
-        else SPLIT(128, 8, 32);
+             c->n_heads, c->max_seq, pos, chunk, part, kn, vn, oh, perm ? 1 : 0)
+        if (B == 4) {
+            if (D == 64 && G == 64) MMA(64, 64);
+            else if (D == 64) MMA(64, 32);
+            else if (G == 64) MMA(128, 64);
+            else MMA(128, 32);
+            combined = (ns == 1);
+        } else {
+            if (D == 64 && G == 64) SPLIT(64, 8, 64);
+            else if (D == 64) SPLIT(64, 8, 32);
+            else if (G == 64) SPLIT(128, 8, 64);
+            else SPLIT(128, 8, 32);
+        }
 #undef SPLIT
 #undef MMA
     }
-    const __half* kn = static_cast<const __half*>(k_new);
-    const __half* vn = static_cast<const __half*>(v_new);
-    __half* oh = static_cast<__half*>(o);
-    if (c->head_dim == 64)
-        launch_k(decode_attn_combine_kernel<64>, dim3(pairs), dim3(64), 0, st, true, qh, kn, vn, row_stride,
-                 c->n_heads, ns, static_cast<const float*>(part), oh, perm ? 1 : 0);
-    else
-        launch_k(decode_attn_combine_kernel<128>, dim3(pairs), dim3(128), 0, st, true, qh, kn, vn, row_stride,
-                 c->n_heads, ns, static_cast<const float*>(part), oh, perm ? 1 : 0);
+    if (!combined) {
+        if (D == 64)
+            launch_k(decode_attn_combine_kernel<64>, dim3(pairs), dim3(64), 0, st, true, qh, kn, vn, row_stride,
+                     c->n_heads, ns, static_cast<const float*>(part), oh, perm ? 1 : 0);
+        else
+            launch_k(decode_attn_combine_kernel<128>, dim3(pairs), dim3(128), 0, st, true, qh, kn, vn, row_stride,
+                     c->n_heads, ns, static_cast<const float*>(part), oh, perm ? 1 : 0);
+    }
     return launch_status();
 }
 

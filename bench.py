@@ -255,7 +255,13 @@ def run_flexq(args):
         for g in graphs:
             g.replay()
 
-    launches_per_layer_step = 8               # LN1, QKV(+store_cache), attn split, attn combine, out, LN2, fc1, fc2
+    # LN1, QKV (+store_cache), attention, out, LN2, fc1, fc2, plus the attention combine
+    # when a (sequence, head) key range is split across CTAs (the library splits when the
+    # pairs alone fill fewer than 4 CTAs per SM; a split keeps at least 128 keys)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    pairs = b * nh
+    splits = [max(1, min((4 * sms + pairs - 1) // pairs, (s + t + 127) // 128)) for t in range(nsteps)]
+    launches_per_token = [L * (7 if ns == 1 else 8) for ns in splits]
     units_per_step = b * nsteps * L
 
     for _ in range(args.warmup):
@@ -340,7 +346,7 @@ def run_flexq(args):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(host_in.numel() * 2),
                 "d2h_bytes_per_step": int(host_out.numel() * 2)},
-        "gpu_launches": launches_per_layer_step * L * nsteps * args.steps,
+        "gpu_launches": sum(launches_per_token) * args.steps,
         "clocks": clocks,
         "peaks": peaks,
         "parts": parts,
@@ -446,8 +452,9 @@ def measure_parts(fq, torch, synth, cfg, layers, caches, ws_dec, stream, peaks, 
     # per kernel (the four GEMMs are launches of one kernel, gemm_tc_kernel): time per
     # layer step, and bytes and duration per launch averaged over its launches
     gemms = ["gemm_qkv", "gemm_out", "gemm_fc1", "gemm_fc2"]
+    gemm_kernel = "gemv_kernel" if b <= 8 else "gemm_tc_kernel"    # the library's dispatch by batch
     per_kernel = {
-        "gemm_tc_kernel": dict(launches=4, ms=sum(kern[g]["ms"] for g in gemms),
+        gemm_kernel: dict(launches=4, ms=sum(kern[g]["ms"] for g in gemms),
                                bytes=sum(kern[g]["bytes"] for g in gemms), source=["gemm.cu", "tc.cuh"]),
         "decode_attention": dict(launches=2, ms=kern["decode_attention"]["ms"],
                                  bytes=kern["decode_attention"]["bytes"], source=["attention.cu"]),

@@ -48,10 +48,12 @@ namespace {
 
 constexpr int kBM = 128;           // weight rows per CTA (MMA M)
 constexpr int kBK = 64;            // K per stage = one quantisation group
-// 12 warps: 0 code TMA, 1 activation TMA, 2 TMEM allocation and MMA issue, 3 spare,
-// 4-11 dequantisation into TMEM and then the epilogue (a warp reaches only the TMEM lane
-// quarter warp % 4, so each quarter has two of them, one per K half).
-constexpr int kThreads = 384;
+// 14 warps: 0 code TMA, 1 activation TMA, 2 TMEM allocation, 4-11 dequantisation into
+// TMEM and then the epilogue (a warp reaches only the TMEM lane quarter warp % 4, so each
+// quarter has two of them, one per K half). One thread each of warps 2, 3, 12, 13
+// issues the MMAs of one accumulator (as many issuers as accumulators), so the issue
+// latency of tcgen05.mma is paid in parallel.
+constexpr int kThreads = 448;
 constexpr int kDequantThreads = 256;
 constexpr int kMetaChunks = 4;     // groups per metadata tile
 constexpr int kDoneRing = 8;       // mma_done barriers, one per step (more than any ring's look-ahead)
@@ -59,6 +61,10 @@ constexpr int kTmemCols = 512;     // whole TMEM of the SM (one CTA per SM)
 constexpr int kACol0 = 256;        // TMEM columns [0, 256): accumulator; [256, 512): dequantised A slots
 constexpr int kACols = kTmemCols - kACol0;
 constexpr int kMaxSplits = 8;      // K splits of a tile form one cluster (portable size)
+// Split-K tickets: a fixed region at the start of every GEMM workspace (the partials
+// follow it), so that GEMMs of different tile counts sharing one workspace never write
+// partials over each other's tickets. Split plans have at most 2 * SMs tiles.
+constexpr int64_t kTicketBytes = 2048;
 
 struct GemmParams {
     const __half* bias;
@@ -97,7 +103,7 @@ struct GemmParams {
 };
 
 struct Bars {
-    uint32_t codes_full, codes_empty, x_full, a_full, mma_done, acc_full, drain;
+    uint32_t codes_full, codes_empty, x_full, a_full, mma_done, acc_full, drain;   // drain: one per issuer
 };
 
 __device__ __forceinline__ uint32_t dequant_pair(uint32_t raw_pair_bits, uint32_t step2, uint32_t mn2) {
@@ -245,6 +251,18 @@ __device__ __forceinline__ void kv_store8(const GemmParams& p, const __half (&o1
         kv_store8_bits<8>(p, o16, col, m0, n0, n, warp, lane, kv_red);
 }
 
+// The MMAs of one K chunk (4 k-steps of 16) that belong to issuer ii of NI: k-steps ii,
+// ii + NI, ... into accumulator d_acc (unrolled, so the issue loop has no branches).
+template <int NI>
+__device__ __forceinline__ void issue_ksteps(uint32_t d_acc, uint32_t a_chunk, uint64_t b_desc, uint32_t idesc, int ii,
+                                             bool first) {
+#pragma unroll
+    for (int q = 0; q < kBK / 16 / NI; ++q) {
+        const int kk = ii + q * NI;
+        tc::mma_f16_ts(d_acc, a_chunk + kk * 8, b_desc + 2 * kk, idesc, (first && q == 0) ? 0u : 1u);
+    }
+}
+
 template <int BITS, bool XPERM>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                               const __grid_constant__ CUtensorMap tm_meta,
@@ -282,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     B.mma_done = B.a_full + 8 * NSLOT;
     B.acc_full = B.mma_done + 8 * kDoneRing;
     B.drain = B.acc_full + 8;
-    const uint32_t misc = B.drain + 8;                        // tmem slot, abort flag, last flag
+    const uint32_t misc = B.drain + 8 * 4;                    // tmem slot, abort flag, last flag
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (misc - base));
     volatile int* abort = reinterpret_cast<volatile int*>(gbase + (misc - base) + 4);
     volatile int* last_flag = reinterpret_cast<volatile int*>(gbase + (misc - base) + 8);
@@ -295,9 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
         for (int s = 0; s < NSX; ++s) tc::bar_init(B.x_full + 8 * s, 1);
         for (int s = 0; s < NSLOT; ++s) tc::bar_init(B.a_full + 8 * s, kDequantThreads);
-        for (int s = 0; s < kDoneRing; ++s) tc::bar_init(B.mma_done + 8 * s, 1);
-        tc::bar_init(B.acc_full, 1);
-        tc::bar_init(B.drain, 1);
+        // every issuer commits each step once
+        for (int s = 0; s < kDoneRing; ++s) tc::bar_init(B.mma_done + 8 * s, p.nacc);
+        tc::bar_init(B.acc_full, p.nacc);
+        for (int i = 0; i < 4; ++i) tc::bar_init(B.drain + 8 * i, 1);
         *abort = 0;
         *last_flag = 0;
         tc::bar_fence_init();
@@ -401,20 +420,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
         }
         __syncwarp();
-    } else if (warp == 2) {
-        // ---------------- MMA issuer: one wait per step of KU chunks, one commit per step ----------------
-        if (lane == 0) {
-            // This single thread issues every MMA, so its own instruction latency is the
-            // issue rate: everything below is precomputed or advanced incrementally (no
-            // integer division by a runtime value in the loop).
+    } else if (warp == 2 || warp == 3 || warp >= 12) {
+        // ---------------- MMA issuers: one per accumulator ----------------
+        // Issuer ii issues the k-steps kk = ii, ii + nacc, ... of every chunk into
+        // accumulator ii, with one wait per step (A slot) and per activation stage and one
+        // commit per step. Each thread's loop is free of integer division by runtime
+        // values: its instruction latency is part of the issue rate.
+        const int ii = warp == 2 ? 0 : (warp == 3 ? 1 : warp - 10);
+        if (lane == 0 && ii < p.nacc) {
+            const int NI = p.nacc;
             const uint32_t idesc = tc::idesc_f16_f32(kBM, p.BN);
-            // k-step kk of every chunk accumulates into accumulator kk % nacc (nacc = 1, 2
-            // or 4), so consecutive MMAs do not wait for each other's results; the
-            // epilogue adds the accumulators
-            const uint32_t amask = static_cast<uint32_t>(p.nacc - 1);
-            uint32_t d_tm[kBK / 16];
-#pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) d_tm[kk] = tmem + (kk & amask) * static_cast<uint32_t>(p.acc_stride);
+            const uint32_t d_acc = tmem + static_cast<uint32_t>(ii * p.acc_stride);
             int xs = 0;
             uint32_t xph = 0;
             bool ok = true;
@@ -430,25 +446,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                         const int c = c0 + c2;
                         const uint64_t bd = tc::desc_k_sw128(xb + c2 * xbytes);
                         const bool first = (j == 0 && c == 0);
-#pragma unroll
-                        for (int kk = 0; kk < kBK / 16; ++kk)
-                            tc::mma_f16_ts(d_tm[kk], a_tm + c * 32 + kk * 8, bd + 2 * kk, idesc,
-                                           (first && static_cast<uint32_t>(kk) <= amask) ? 0u : 1u);
+                        if (NI == 4) issue_ksteps<4>(d_acc, a_tm + c * 32, bd, idesc, ii, first);
+                        else if (NI == 2) issue_ksteps<2>(d_acc, a_tm + c * 32, bd, idesc, ii, first);
+                        else issue_ksteps<1>(d_acc, a_tm + c * 32, bd, idesc, ii, first);
                     }
                     if (++xs == NSX) { xs = 0; xph ^= 1; }
                 }
                 if (!ok) break;
-                // exactly one commit per step: a commit covers the MMAs issued since the
-                // previous one, so a second commit here would complete at once. The A slot
-                // and the activation stages of this step are reused once it lands; the
-                // last step's commit is the accumulator-ready signal.
+                // exactly one commit per step and issuer: a commit covers the MMAs this
+                // thread issued since its previous one, so a second commit here would
+                // complete at once. The A slot and the activation stages of this step are
+                // reused once every issuer's commit has landed; the last step's commits
+                // are the accumulator-ready signal.
                 tc::mma_commit(j + 1 < nsteps ? B.mma_done + 8 * (j % kDoneRing) : B.acc_full);
             }
             if (!ok) {
-                // nothing of ours may still run on the tensor cores at exit
-                tc::mma_commit(B.drain);
+                // nothing of this thread's may still run on the tensor cores at exit
+                tc::mma_commit(B.drain + 8 * ii);
                 volatile int never = 0;
-                tc::bar_wait(B.drain, 0, &never, p.status);
+                tc::bar_wait(B.drain + 8 * ii, 0, &never, p.status);
             } else {
                 // every commit's mbarrier arrival must have landed before the CTA exits: a
                 // late arrival would hit the barriers of the next CTA on this SM, which
@@ -682,6 +698,304 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------------------------------
+// Small-batch path (up to 8 activation rows, 4-bit weights): dequant-fused GEMV on
+// mma.sync m16n8k16 (the kernel handles up to 32 rows; the dispatch uses it up to 8).
+//
+// A CTA (4 warps) owns kGvRows = 64 weight rows and a range of K groups (all of K, or
+// 1/splits of it); warp w owns rows 16w .. 16w+15. The group's codes, metadata and
+// activation slice pass through a kGvStages-deep cp.async ring in shared memory, so
+// several groups are always in flight. A warp turns each 32-bit word of codes into 4
+// fp16 pairs in registers (lop3, hsub2, hfma2; the pairs come out in the order (e0,e4)
+// (e1,e5) (e2,e6) (e3,e7)) and uses them directly as A fragments - thread (g, t) holds
+// K positions [16t, 16t+16) of rows g and g+8 - with the activations of the same K
+// positions as B fragments (an interleaved activation row gives them as plain 16-byte
+// loads). No single issuing thread and no staging of dequantised weights.
+// With K splits each split writes its partial tile to the workspace and the last split
+// of a tile to finish (atomic ticket) adds them in split order, so results do not
+// depend on scheduling. The epilogue is the GEMM's (bias, q-scale, ReLU, residual,
+// interleaved output, fused store_cache).
+constexpr int kGvWarps = 4;
+constexpr int kGvThreads = kGvWarps * 32;
+constexpr int kGvRows = 16 * kGvWarps;     // 64 weight rows per CTA
+constexpr int kGvStages = 3;               // stages of 4 groups (256 K) in flight
+
+struct GemvParams {
+    const uint8_t* codes;                  // [N][K/2]
+    const uint32_t* meta;                  // [N][K/64] half2 {min, scale}
+    const __half* x;                       // [M][K]
+    const __half* bias;
+    const __half* residual;
+    __half* y;
+    float* part;                           // split partials [tiles][splits][kGvRows][32]
+    int* counters;                         // [tiles] tickets
+    int M, N, K, splits, gps;              // gps: groups per split
+    int nq;
+    float qscale;
+    int relu, yperm, xperm, early_w;
+    uint8_t* kv_codes[2];
+    uint32_t* kv_meta[2];
+    int kv_h, kv_hd, kv_nh, kv_max_seq, kv_seq, kv_pos0, kv_bits, kv_gs;
+};
+
+__device__ __forceinline__ void hmma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void gv_cp16(uint32_t dst, const void* src, bool pred) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(pred ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void gv_cp4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void gv_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void gv_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(kGvStages - 2) : "memory");
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128v(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+
+// Epilogue of the small-batch path for activation row m and weight rows n0 + 8c .. +7:
+// bias, q-scale, ReLU, residual, fp16 store (interleaved 8-block order when yperm) and
+// the fused store_cache. The 8 lanes sharing m are consecutive (item = 8 m + c); rows
+// past M return without touching anything.
+__device__ __forceinline__ void gemv_finish(const GemvParams& p, int n0, int c, int m, int lane, const float (&v)[8]) {
+    const bool valid = m < p.M;
+    const int nb = n0 + 8 * c;
+    __half o16[8];
+    if (valid) {
+        const uint4 bv = p.bias ? __ldg(reinterpret_cast<const uint4*>(p.bias + nb)) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 rv = p.residual ? *reinterpret_cast<const uint4*>(p.residual + static_cast<int64_t>(m) * p.N + nb)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w}, rw[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float bi = (i & 1) ? h2f_hi(bw[i >> 1]) : h2f_lo(bw[i >> 1]);
+            const float ri = (i & 1) ? h2f_hi(rw[i >> 1]) : h2f_lo(rw[i >> 1]);
+            float xo = (v[i] + bi) * (nb + i < p.nq ? p.qscale : 1.f);
+            if (p.relu) xo = fmaxf(xo, 0.f);
+            o16[i] = __float2half_rn(xo + ri);
+        }
+        // interleaved output: element k of the 8-block goes to position 2(k%4) + (k/4)%2
+        __half op[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) op[p.yperm ? (2 * (i & 3) + ((i >> 2) & 1)) : i] = o16[i];
+        *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m) * p.N + nb) =
+            make_uint4(pack_half2_bits(op[0], op[1]), pack_half2_bits(op[2], op[3]), pack_half2_bits(op[4], op[5]),
+                       pack_half2_bits(op[6], op[7]));
+    }
+    if (p.kv_codes[0] != nullptr && n0 >= p.kv_h && valid) {
+        // fused store_cache: the 8 values are dims [dim, dim+8) of one head; a group of gs
+        // dims is the gs/8 lanes of consecutive c for this m (all 8 lanes of m are here)
+        const uint4 nv = make_uint4(pack_half2_bits(o16[0], o16[1]), pack_half2_bits(o16[2], o16[3]),
+                                    pack_half2_bits(o16[4], o16[5]), pack_half2_bits(o16[6], o16[7]));
+        const int sec = (n0 - p.kv_h) / p.kv_h;                 // 0 keys, 1 values
+        const int f = nb - p.kv_h - sec * p.kv_h;
+        const int head = f / p.kv_hd, dim = f % p.kv_hd;
+        __half2 mn2, mx2;
+        minmax8(nv, mn2, mx2);
+        float mn = hmin_of(mn2), mx = hmax_of(mx2);
+        const unsigned lanes = 0xFFu << (lane & 24);
+        const unsigned gmask = p.kv_gs == 64 ? 7u : 3u;
+        for (unsigned off = 1; off <= gmask; off <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(lanes, mn, off));
+            mx = fmaxf(mx, __shfl_xor_sync(lanes, mx, off));
+        }
+        const int b = m / p.kv_seq, tt = m - b * p.kv_seq;
+        const int64_t slot = (static_cast<int64_t>(b) * p.kv_nh + head) * p.kv_max_seq + p.kv_pos0 + tt;
+        uint8_t* codes = p.kv_codes[sec];
+        uint32_t* meta = p.kv_meta[sec];
+        const int gph = p.kv_hd / p.kv_gs;
+        if (p.kv_bits == 4) {
+            const __half s16 = group_scale16<4>(mn, mx);
+            *reinterpret_cast<uint32_t*>(codes + slot * (p.kv_hd / 2) + dim / 2) = quant8_4bit(nv, mn, __half2float(s16));
+            if (dim % p.kv_gs == 0) meta[slot * gph + dim / p.kv_gs] = pack_half2_bits(__float2half_rn(mn), s16);
+        } else {
+            const __half s16 = group_scale16<8>(mn, mx);
+            *reinterpret_cast<uint2*>(codes + slot * p.kv_hd + dim) = quant8_8bit(nv, mn, __half2float(s16));
+            if (dim % p.kv_gs == 0) meta[slot * gph + dim / p.kv_gs] = pack_half2_bits(__float2half_rn(mn), s16);
+        }
+    }
+}
+
+template <int NT>                          // n-tiles of 8 activation rows (M <= 8 NT)
+__global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p) {
+    constexpr int MC = 8 * NT;             // activation rows of the tile
+    // stage = 4 groups (256 K): codes [64 rows][128 B + 16 pad], metadata [64][4 groups],
+    // activations [MC rows][4 groups][128 B + 16 pad] (the pads spread the fragment loads
+    // over all banks)
+    constexpr int CROW = 128 + 16;
+    constexpr int XSEG = 128 + 16;
+    constexpr int CODES = kGvRows * CROW;
+    constexpr int META = kGvRows * 16;
+    constexpr int STAGE = CODES + META + MC * 4 * XSEG;
+    extern __shared__ __align__(16) uint8_t gv_smem[];
+    __shared__ int last;
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(gv_smem));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int tile = blockIdx.x, split = blockIdx.y;
+    const int n0 = tile * kGvRows;
+    const int ngroups = p.K / 64;
+    const int gb = split * p.gps;                       // multiple of 4
+    const int nst = (min(ngroups, gb + p.gps) - gb) / 4;  // stages of this CTA (> 0)
+    const int64_t krow = p.K / 2;                       // code bytes per weight row
+
+    auto load_weights = [&](int i) {       // groups gb + 4i .. +3 into stage i % kGvStages
+        const uint32_t st = sbase + (i % kGvStages) * STAGE;
+        const int G = gb + 4 * i;
+#pragma unroll
+        for (int j = 0; j < (kGvRows * 8) / kGvThreads; ++j) {
+            const int u = threadIdx.x + j * kGvThreads, row = u >> 3, c16 = u & 7;
+            gv_cp16(st + row * CROW + c16 * 16, p.codes + (n0 + row) * krow + G * 32 + c16 * 16, true);
+        }
+        if (threadIdx.x < kGvRows)
+            gv_cp16(st + CODES + threadIdx.x * 16, p.meta + static_cast<int64_t>(n0 + threadIdx.x) * ngroups + G, true);
+    };
+    auto load_x = [&](int i) {
+        const uint32_t st = sbase + (i % kGvStages) * STAGE + CODES + META;
+        const int G = gb + 4 * i;
+#pragma unroll
+        for (int j = 0; j < (MC * 32) / kGvThreads; ++j) {
+            const int u = threadIdx.x + j * kGvThreads;
+            const int m = u >> 5, q = (u >> 3) & 3, c16 = u & 7;
+            const bool ok = m < p.M;
+            gv_cp16(st + (m * 4 + q) * XSEG + c16 * 16,
+                    p.x + static_cast<int64_t>(ok ? m : 0) * p.K + (G + q) * 64 + c16 * 8, ok);
+        }
+    };
+    // weights do not depend on the previous kernel: inside a layer call their first
+    // stages are requested before the programmatic-launch wait
+    if (p.early_w) {
+#pragma unroll
+        for (int i = 0; i < kGvStages - 1; ++i)
+            if (i < nst) load_weights(i);
+    }
+    pdl_wait();                            // the activations come from the previous kernel
+    pdl_trigger();
+#pragma unroll
+    for (int i = 0; i < kGvStages - 1; ++i) {
+        if (i < nst) {
+            if (!p.early_w) load_weights(i);
+            load_x(i);
+        }
+        gv_commit();
+    }
+
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    // thread (g, t): rows r0 and r0 + 8 of the tile, group t of every stage (its 64 K
+    // positions, 8 code words per row); the MMA's K order is free as long as A and B agree
+    const int r0 = 16 * warp + g;
+    for (int i = 0; i < nst; ++i) {
+        if (i + kGvStages - 1 < nst) {
+            load_weights(i + kGvStages - 1);
+            load_x(i + kGvStages - 1);
+        }
+        gv_commit();
+        gv_wait();
+        __syncthreads();
+        const uint32_t st = sbase + (i % kGvStages) * STAGE;
+        const uint4 ca0 = lds128v(st + r0 * CROW + t * 32), ca1 = lds128v(st + r0 * CROW + t * 32 + 16);
+        const uint4 cb0 = lds128v(st + (r0 + 8) * CROW + t * 32), cb1 = lds128v(st + (r0 + 8) * CROW + t * 32 + 16);
+        const uint32_t mw0 = lds32(st + CODES + r0 * 16 + t * 4), mw1 = lds32(st + CODES + (r0 + 8) * 16 + t * 4);
+        uint32_t s2[2], m2[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint32_t mwr = r ? mw1 : mw0;
+            const __half mn = __ushort_as_half(static_cast<unsigned short>(mwr & 0xFFFFu));
+            const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mwr >> 16)));
+            const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
+            const __half2 sh = __half2half2(step), mh = __half2half2(mn);
+            s2[r] = *reinterpret_cast<const uint32_t*>(&sh);
+            m2[r] = *reinterpret_cast<const uint32_t*>(&mh);
+        }
+        const uint32_t wa[8] = {ca0.x, ca0.y, ca0.z, ca0.w, ca1.x, ca1.y, ca1.z, ca1.w};
+        const uint32_t wb[8] = {cb0.x, cb0.y, cb0.z, cb0.w, cb1.x, cb1.y, cb1.z, cb1.w};
+        const uint32_t xs = st + CODES + META + (g * 4 + t) * XSEG;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            // K positions 8w .. 8w+7 of group t: A pairs (e0,e4) (e1,e5) (e2,e6) (e3,e7)
+            const uint4 d0 = dequant8_4bit_il(wa[w], s2[0], m2[0]);    // row r0
+            const uint4 d1 = dequant8_4bit_il(wb[w], s2[1], m2[1]);    // row r0 + 8
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                // activations of row 8 nt + g at the same K positions, as the pairs
+                // (k0,k4) (k1,k5) (k2,k6) (k3,k7)
+                uint4 xv = lds128v(xs + nt * 8 * 4 * XSEG + w * 16);
+                if (!p.xperm)
+                    xv = make_uint4(prmt(xv.x, xv.z, 0x5410u), prmt(xv.x, xv.z, 0x7632u), prmt(xv.y, xv.w, 0x5410u),
+                                    prmt(xv.y, xv.w, 0x7632u));
+                hmma16816(acc[nt], d0.x, d1.x, d0.y, d1.y, xv.x, xv.y);
+                hmma16816(acc[nt], d0.z, d1.z, d0.w, d1.w, xv.z, xv.w);
+            }
+        }
+        __syncthreads();                   // the stage is refilled by the next iteration
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+    // ---- the tile (64 rows x MC activation rows) through shared memory: [64][MC + 1]
+    float* red = reinterpret_cast<float*>(gv_smem);
+    __syncthreads();
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[(r0 + 8 * (j >> 1)) * (MC + 1) + 8 * nt + 2 * t + (j & 1)] = acc[nt][j];
+    __syncthreads();
+    // (activation row m, rows 8c .. 8c+7): 8 MC items, 2 per thread at MC = 32
+    for (int item = threadIdx.x; item < 8 * MC; item += kGvThreads) {
+        const int c = item & 7, m = item >> 3;
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = red[(8 * c + i) * (MC + 1) + m];
+        if (p.splits > 1) {
+            float* mine = p.part + (static_cast<int64_t>(tile) * p.splits + split) * kGvRows * 32;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mine[(8 * c + i) * 32 + m] = v[i];
+        } else {
+            gemv_finish(p, n0, c, m, lane, v);
+        }
+    }
+    if (p.splits == 1) return;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const float* all = p.part + static_cast<int64_t>(tile) * p.splits * kGvRows * 32;
+    for (int item = threadIdx.x; item < 8 * MC; item += kGvThreads) {
+        const int c = item & 7, m = item >> 3;
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+        for (int sp = 0; sp < p.splits; ++sp)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] += __ldcg(all + (static_cast<int64_t>(sp) * kGvRows + 8 * c + i) * 32 + m);
+        gemv_finish(p, n0, c, m, lane, v);
+    }
+    if (threadIdx.x == 0) p.counters[tile] = 0;
+}
+
+// ---------------------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -773,7 +1087,7 @@ Plan make_plan(int M, int N, int K, int bits) {
     P.off_m = P.off_c + P.nsc * kBM * 128;
     P.off_bar = P.off_m + P.nsc * kBM * kMetaChunks * 4;
     const int nslot = kACols / (ku * 32);
-    uint32_t smem = P.off_bar + 8 * (2 * P.nsc + P.nsx + nslot + kDoneRing + 2) + 16 + 256 + 1024;
+    uint32_t smem = P.off_bar + 8 * (2 * P.nsc + P.nsx + nslot + kDoneRing + 1 + 4) + 16 + 256 + 1024;
     if (smem < 120 * 1024) smem = 120 * 1024;   // at most one CTA per SM: the CTA takes all of TMEM
     P.smem = smem;
     P.tmem_cols = kTmemCols;
@@ -783,10 +1097,38 @@ Plan make_plan(int M, int N, int K, int bits) {
     // split-K: through distributed shared memory when every tile's cluster can be
     // resident at once (one wave), else through workspace partials and a ticket
     P.cluster = (splits > 1 && max_active_clusters(splits, P.smem) >= tiles) ? 1 : 0;
-    P.counters_bytes = ((static_cast<int64_t>(tiles) * 4 + 255) / 256) * 256;
+    P.counters_bytes = kTicketBytes;
     P.ws_bytes = (splits > 1 && !P.cluster)
                      ? P.counters_bytes + static_cast<int64_t>(tiles) * splits * P.BN * kBM * 4
                      : 0;
+    return P;
+}
+
+// The register-dequant GEMV serves int4 weights for up to 8 activation rows; from 9 rows
+// on the tcgen05 GEMM is faster (measured: each GEMV warp's mma.sync accumulation chains
+// are latency-bound at 2-4 n-tiles).
+bool gemv_eligible(int M, int N, int bits) { return bits == 4 && M >= 1 && M <= 8 && N % kGvRows == 0; }
+
+struct GemvPlan {
+    int nt, tiles, splits, gps;
+    uint32_t smem;
+    int64_t ws_bytes, counters_bytes;
+};
+
+GemvPlan gemv_plan(int M, int N, int K) {
+    GemvPlan P{};
+    P.nt = (M + 7) / 8;
+    P.tiles = N / kGvRows;
+    const int nstages = K / 256;          // stages of 4 groups
+    // split K while the grid fits two CTAs per SM and every split keeps >= 2 stages
+    int splits = 1;
+    while (P.tiles * (splits + 1) <= 2 * sm_count() && nstages / (splits + 1) >= 2) ++splits;
+    const int sps = (nstages + splits - 1) / splits;   // stages per split
+    P.gps = 4 * sps;
+    P.splits = (nstages + sps - 1) / sps;
+    P.smem = static_cast<uint32_t>((kGvRows * 144 + kGvRows * 16 + 8 * P.nt * 4 * 144) * kGvStages);
+    P.counters_bytes = kTicketBytes;
+    P.ws_bytes = P.splits > 1 ? P.counters_bytes + static_cast<int64_t>(P.tiles) * P.splits * kGvRows * 32 * 4 : 0;
     return P;
 }
 
@@ -806,7 +1148,67 @@ int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, 
     return r == CUDA_SUCCESS ? FLEX_OK : FLEX_ERR_CUDA;
 }
 
-int64_t gemm_ws_bytes(int M, int N, int K, int bits) { return make_plan(M, N, K, bits).ws_bytes; }
+int64_t gemm_ws_bytes(int M, int N, int K, int bits) {
+    return gemv_eligible(M, N, bits) ? gemv_plan(M, N, K).ws_bytes : make_plan(M, N, K, bits).ws_bytes;
+}
+
+namespace {
+int gemv_launch(const void* x, const flexq_tensor* W, const void* bias, const void* residual, void* y, int M,
+                int relu, int nq, float qscale, bool xperm, bool yperm, void* ws, int64_t ws_bytes, cudaStream_t st,
+                const KvFuse* kv, bool early_w) {
+    const int N = static_cast<int>(W->shape[0]), K = static_cast<int>(W->shape[1]);
+    const GemvPlan P = gemv_plan(M, N, K);
+    if (P.ws_bytes > 0 && (ws == nullptr || ws_bytes < P.ws_bytes)) return FLEX_ERR_WORKSPACE;
+    GemvParams gp{};
+    gp.codes = static_cast<const uint8_t*>(W->codes);
+    gp.meta = static_cast<const uint32_t*>(W->meta);
+    gp.x = static_cast<const __half*>(x);
+    gp.bias = static_cast<const __half*>(bias);
+    gp.residual = static_cast<const __half*>(residual);
+    gp.y = static_cast<__half*>(y);
+    gp.counters = static_cast<int*>(ws);
+    gp.part = reinterpret_cast<float*>(static_cast<char*>(ws) + P.counters_bytes);
+    gp.M = M;
+    gp.N = N;
+    gp.K = K;
+    gp.splits = P.splits;
+    gp.gps = P.gps;
+    gp.nq = nq;
+    gp.qscale = qscale;
+    gp.relu = relu;
+    gp.yperm = yperm ? 1 : 0;
+    gp.xperm = xperm ? 1 : 0;
+    gp.early_w = early_w ? 1 : 0;
+    if (kv != nullptr) {
+        gp.kv_codes[0] = static_cast<uint8_t*>(kv->cache->k_codes);
+        gp.kv_codes[1] = static_cast<uint8_t*>(kv->cache->v_codes);
+        gp.kv_meta[0] = static_cast<uint32_t*>(kv->cache->k_meta);
+        gp.kv_meta[1] = static_cast<uint32_t*>(kv->cache->v_meta);
+        gp.kv_h = kv->h;
+        gp.kv_hd = kv->cache->head_dim;
+        gp.kv_nh = kv->cache->n_heads;
+        gp.kv_max_seq = kv->cache->max_seq;
+        gp.kv_seq = kv->seq;
+        gp.kv_pos0 = kv->pos0;
+        gp.kv_bits = kv->cache->cfg.num_bits;
+        gp.kv_gs = kv->cache->cfg.group_size;
+    }
+    const dim3 grid(P.tiles, P.splits);
+#define GEMV_LAUNCH(NT_)                                                                            \
+    do {                                                                                            \
+        set_smem_once(gemv_kernel<NT_>, static_cast<int>(P.smem));                                  \
+        launch_k(gemv_kernel<NT_>, grid, dim3(kGvThreads), P.smem, st, true, gp);                   \
+    } while (0)
+    switch (P.nt) {
+        case 1: GEMV_LAUNCH(1); break;
+        case 2: GEMV_LAUNCH(2); break;
+        case 3: GEMV_LAUNCH(3); break;
+        default: GEMV_LAUNCH(4); break;
+    }
+#undef GEMV_LAUNCH
+    return launch_status();
+}
+}  // namespace
 
 int validate_weight(const flexq_tensor* W) {
     FLEX_REQUIRE(W != nullptr && W->codes && W->meta, FLEX_ERR_INVALID_ARG);
@@ -829,6 +1231,9 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     if (M == 0) return FLEX_OK;
     const int N = static_cast<int>(W->shape[0]), K = static_cast<int>(W->shape[1]);
     const int bits = W->cfg.num_bits;
+    // small batches of int4 weights: the register-dequant GEMV on mma.sync
+    if (gemv_eligible(M, N, bits))
+        return gemv_launch(x, W, bias, residual, y, M, relu, nq, qscale, xperm, yperm, ws, ws_bytes, st, kv, early_w);
     const Plan P = make_plan(M, N, K, bits);
     if (P.ws_bytes > 0 && (ws == nullptr || ws_bytes < P.ws_bytes)) return FLEX_ERR_WORKSPACE;
     CUtensorMap tm_codes, tm_meta, tm_x;

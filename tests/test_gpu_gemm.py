@@ -89,18 +89,22 @@ def test_gemm_ring_reuse(M, N, K):
     assert_layer_close(got, ref, f"ring reuse {M}x{N}x{K}")
 
 
-def test_gemm_split_k_repeatable_without_workspace():
-    """Split-K (here 8 splits of 4 tiles, one cluster per tile) reduces in split order
-    through distributed shared memory: two calls give identical bits, and the GEMM
-    needs no workspace."""
-    M, N, K = 16, 512, 4096
-    assert fq.flex_gemm_ws_bytes(M, N, K) == 0
+@pytest.mark.parametrize("M", [4, 16, 48])
+def test_gemm_split_k_repeatable(M):
+    """Split-K reduces in split order (M = 4: the small-batch GEMV; M = 16, 48: the
+    tensor-core GEMM): two calls give identical bits, and a workspace, where one is
+    needed, has its tickets back at zero after each call."""
+    N, K = 512, 4096
     x, w, b, _, y1, ws = _run(M, N, K, fq.FLEX_EPI_NONE, seed=5)
     W = fq.CompressedWeight(torch.from_numpy(w).cuda(), 4, 64)
     y2 = torch.empty_like(y1)
-    fq.flex_dequant_gemm(torch.from_numpy(x).cuda(), W, torch.from_numpy(b).cuda(), None, y2, M, 0, None)
+    need = fq.flex_gemm_ws_bytes(M, N, K)
+    fq.flex_dequant_gemm(torch.from_numpy(x).cuda(), W, torch.from_numpy(b).cuda(), None, y2, M, 0,
+                         ws if need > 0 else None)
     sync_status()
     assert torch.equal(y1, y2)
+    if need > 0:
+        assert int(ws[:256].view(torch.int32).abs().sum()) == 0
 
 
 @pytest.mark.parametrize("name,M,N,K", [("opt-1.3b qkv decode", 32, 6144, 2048),
@@ -146,3 +150,24 @@ def test_gemm_bad_args():
     with pytest.raises(fq.FlexError) as e:
         fq.flex_dequant_gemm(x, W, None, None, y, 4, fq.FLEX_EPI_RESIDUAL, None)
     assert e.value.code == fq.FLEX_ERR_INVALID_ARG
+
+
+def test_gemm_sequence_shares_one_workspace():
+    """GEMMs of different tile counts and split counts run back to back on one
+    workspace, as inside a layer call: every result matches its own run on a fresh
+    workspace (a GEMM's partials must never land on another's tickets)."""
+    shapes = [(32, 6144, 2048), (32, 2048, 2048), (32, 8192, 2048), (32, 2048, 8192), (48, 2048, 2048),
+              (48, 6144, 2048)]
+    need = max(fq.flex_gemm_ws_bytes(*s) for s in shapes)
+    shared = torch.zeros(max(16, need), dtype=torch.uint8, device="cuda")
+    for rep in range(2):
+        for i, (M, N, K) in enumerate(shapes):
+            x = synth.activations((M, K), 60 + i, device="cuda")
+            W = fq.CompressedWeight(synth.normal_f16((N, K), 70 + i, 0.02, device="cuda"))
+            y1 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+            y2 = torch.empty_like(y1)
+            fq.flex_dequant_gemm(x, W, None, None, y1, M, 0, shared)
+            fresh = torch.zeros(max(16, fq.flex_gemm_ws_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
+            fq.flex_dequant_gemm(x, W, None, None, y2, M, 0, fresh)
+            sync_status()
+            assert torch.equal(y1, y2), (rep, M, N, K)

@@ -452,7 +452,7 @@ def measure_parts(fq, torch, synth, cfg, layers, caches, ws_dec, stream, peaks, 
     # per kernel (the four GEMMs are launches of one kernel, gemm_tc_kernel): time per
     # layer step, and bytes and duration per launch averaged over its launches
     gemms = ["gemm_qkv", "gemm_out", "gemm_fc1", "gemm_fc2"]
-    gemm_kernel = "gemv_kernel" if b <= 8 else "gemm_tc_kernel"    # the library's dispatch by batch
+    gemm_kernel = "gemv_kernel" if b <= 32 else "gemm_tc_kernel"   # the library's dispatch by batch
     per_kernel = {
         gemm_kernel: dict(launches=4, ms=sum(kern[g]["ms"] for g in gemms),
                                bytes=sum(kern[g]["bytes"] for g in gemms), source=["gemm.cu", "tc.cuh"]),

@@ -698,8 +698,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------------------------------
-// Small-batch path (up to 8 activation rows, 4-bit weights): dequant-fused GEMV on
-// mma.sync m16n8k16 (the kernel handles up to 32 rows; the dispatch uses it up to 8).
+// Small-batch path (up to 32 activation rows, 4-bit weights): dequant-fused GEMV on
+// mma.sync m16n8k16.
 //
 // A CTA (4 warps) owns kGvRows = 64 weight rows and a range of K groups (all of K, or
 // 1/splits of it); warp w owns rows 16w .. 16w+15. The group's codes, metadata and
@@ -899,9 +899,13 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
         gv_commit();
     }
 
-    float acc[NT][4];
+    // two accumulator sets (the two MMAs of every code word go to different sets), so
+    // each set's dependent mma.sync chain is half as long
+    float acc[NT][4], acc2[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[nt][j] = acc2[nt][j] = 0.f;
     // thread (g, t): rows r0 and r0 + 8 of the tile, group t of every stage (its 64 K
     // positions, 8 code words per row); the MMA's K order is free as long as A and B agree
     const int r0 = 16 * warp + g;
@@ -945,12 +949,16 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
                     xv = make_uint4(prmt(xv.x, xv.z, 0x5410u), prmt(xv.x, xv.z, 0x7632u), prmt(xv.y, xv.w, 0x5410u),
                                     prmt(xv.y, xv.w, 0x7632u));
                 hmma16816(acc[nt], d0.x, d1.x, d0.y, d1.y, xv.x, xv.y);
-                hmma16816(acc[nt], d0.z, d1.z, d0.w, d1.w, xv.z, xv.w);
+                hmma16816(acc2[nt], d0.z, d1.z, d0.w, d1.w, xv.z, xv.w);
             }
         }
         __syncthreads();                   // the stage is refilled by the next iteration
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[nt][j] += acc2[nt][j];
 
     // ---- the tile (64 rows x MC activation rows) through shared memory: [64][MC + 1]
     float* red = reinterpret_cast<float*>(gv_smem);
@@ -1104,10 +1112,9 @@ Plan make_plan(int M, int N, int K, int bits) {
     return P;
 }
 
-// The register-dequant GEMV serves int4 weights for up to 8 activation rows; from 9 rows
-// on the tcgen05 GEMM is faster (measured: each GEMV warp's mma.sync accumulation chains
-// are latency-bound at 2-4 n-tiles).
-bool gemv_eligible(int M, int N, int bits) { return bits == 4 && M >= 1 && M <= 8 && N % kGvRows == 0; }
+// The register-dequant GEMV serves int4 weights for up to 32 activation rows (one tile
+// of n-tiles); larger batches and prefill go to the tcgen05 GEMM.
+bool gemv_eligible(int M, int N, int bits) { return bits == 4 && M >= 1 && M <= 32 && N % kGvRows == 0; }
 
 struct GemvPlan {
     int nt, tiles, splits, gps;

@@ -91,7 +91,7 @@ def test_gemm_ring_reuse(M, N, K):
 
 @pytest.mark.parametrize("M", [4, 16, 48])
 def test_gemm_split_k_repeatable(M):
-    """Split-K reduces in split order (M = 4: the small-batch GEMV; M = 16, 48: the
+    """Split-K reduces in split order (M = 4, 16: the small-batch GEMV; M = 48: the
     tensor-core GEMM): two calls give identical bits, and a workspace, where one is
     needed, has its tickets back at zero after each call."""
     N, K = 512, 4096

@@ -434,8 +434,10 @@ def measure_parts(fq, torch, synth, cfg, layers, caches, ws_dec, stream, peaks, 
                                           "gemm_fc2": (h, ffn, xf, o, 0)}.items():
         wkey = {"gemm_qkv": "w_qkv", "gemm_out": "w_o", "gemm_fc1": "w_fc1", "gemm_fc2": "w_fc2"}[name]
         kern[name] = dict(
+            # the layer hands every GEMM its activations in the interleaved 8-block order
             ms=time_cycle(lambda l, n=n, xin=xin, yout=yout, epi=epi, wkey=wkey:
-                          fq.flex_dequant_gemm(xin, layers[l].w[wkey], None, None, yout, b, epi, gws, stream=stream)),
+                          fq.flex_dequant_gemm(xin, layers[l].w[wkey], None, None, yout, b,
+                                               epi | fq.FLEX_GEMM_X_INTERLEAVED, gws, stream=stream)),
             bytes=n * k * per + b * k * 2 + b * n * 2, launches_per_layer_step=1, source=["gemm.cu", "tc.cuh"])
     kern["store_cache"] = dict(
         ms=time_cycle(lambda l: fq.flex_append_kv(caches[l], x[:, h:], x[:, 2 * h:], 3 * h, b, pos, stream=stream)),

@@ -32,6 +32,8 @@ FLEX_ERR_SCRATCH_LIMIT = -8
 
 FLEX_DECODE_ATTENTION_STATIC_MAX_BYTES = 8 << 20
 
+FLEX_GEMM_X_INTERLEAVED = 0x10
+
 FLEX_EPI_NONE = 0
 FLEX_EPI_RELU = 1
 FLEX_EPI_RESIDUAL = 2

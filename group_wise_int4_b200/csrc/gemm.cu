@@ -1344,6 +1344,8 @@ extern "C" int flex_dequant_gemm(const void* x, const flexq_tensor* W, const voi
     if (rc != FLEX_OK) return rc;
     FLEX_REQUIRE(x && y, FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(M >= 0, FLEX_ERR_INVALID_ARG);
+    const bool xil = (epilogue & FLEX_GEMM_X_INTERLEAVED) != 0;
+    epilogue &= ~FLEX_GEMM_X_INTERLEAVED;
     FLEX_REQUIRE(epilogue == FLEX_EPI_NONE || epilogue == FLEX_EPI_RELU || epilogue == FLEX_EPI_RESIDUAL,
                  FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(epilogue != FLEX_EPI_RESIDUAL || residual != nullptr, FLEX_ERR_INVALID_ARG);
@@ -1351,6 +1353,6 @@ extern "C" int flex_dequant_gemm(const void* x, const flexq_tensor* W, const voi
                  FLEX_ERR_ALIGN);
     FLEX_REQUIRE(ws == nullptr || aligned16(ws), FLEX_ERR_ALIGN);
     return gemm_launch(x, W, bias, epilogue == FLEX_EPI_RESIDUAL ? residual : nullptr, y, M,
-                       epilogue == FLEX_EPI_RELU ? 1 : 0, 0, 1.0f, false, false, ws, ws_bytes, as_stream(stream),
+                       epilogue == FLEX_EPI_RELU ? 1 : 0, 0, 1.0f, xil, false, ws, ws_bytes, as_stream(stream),
                        nullptr, false);
 }

@@ -211,6 +211,10 @@ int flex_prefill_attention(const void* q, const void* k, const void* v, int64_t 
 #define FLEX_EPI_NONE     0
 #define FLEX_EPI_RELU     1
 #define FLEX_EPI_RESIDUAL 2
+/* OR-ed into `epilogue`: x is stored with every 8-element block of K interleaved as
+ * [k0, k4, k1, k5, k2, k6, k3, k7] - the layout the layer calls hand from one kernel to
+ * the next (and in which the GEMM needs no permutation of its own). */
+#define FLEX_GEMM_X_INTERLEAVED 0x10
 int64_t flex_gemm_ws_bytes(int32_t M, int32_t N, int32_t K);
 int flex_dequant_gemm(const void* x, const flexq_tensor* W, const void* bias,
                       const void* residual, void* y, int32_t M, int32_t epilogue,

@@ -171,3 +171,30 @@ def test_gemm_sequence_shares_one_workspace():
             fq.flex_dequant_gemm(x, W, None, None, y2, M, 0, fresh)
             sync_status()
             assert torch.equal(y1, y2), (rep, M, N, K)
+
+
+def _interleave8(x):
+    """Every 8-block of the last dim as [k0, k4, k1, k5, k2, k6, k3, k7]."""
+    s = x.shape
+    b = x.reshape(*s[:-1], s[-1] // 8, 2, 4).transpose(-1, -2)
+    return b.reshape(s).contiguous()
+
+
+@pytest.mark.parametrize("M,N,K", [(32, 2048, 2048), (7, 512, 1024), (48, 1024, 2048)])
+def test_gemm_interleaved_activations(M, N, K):
+    """FLEX_GEMM_X_INTERLEAVED: the same logical activations stored in the interleaved
+    8-block order give the natural-order result (bit for bit on the small-batch path,
+    whose operands are identical; within rounding on the tensor-core GEMM, whose K order
+    changes)."""
+    x = synth.activations((M, K), 80, device="cuda")
+    W = fq.CompressedWeight(synth.normal_f16((N, K), 81, 0.02, device="cuda"))
+    y1 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    y2 = torch.empty_like(y1)
+    ws = torch.zeros(max(16, fq.flex_gemm_ws_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
+    fq.flex_dequant_gemm(x, W, None, None, y1, M, fq.FLEX_EPI_NONE, ws)
+    fq.flex_dequant_gemm(_interleave8(x), W, None, None, y2, M, fq.FLEX_EPI_NONE | fq.FLEX_GEMM_X_INTERLEAVED, ws)
+    sync_status()
+    if M <= 32:
+        assert torch.equal(y1, y2)
+    else:
+        assert (y1.float() - y2.float()).abs().max().item() <= 1e-2 * y1.float().abs().max().item() + 1e-3

@@ -701,23 +701,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // Small-batch path (up to 32 activation rows, 4-bit weights): dequant-fused GEMV on
 // mma.sync m16n8k16.
 //
-// A CTA (4 warps) owns kGvRows = 64 weight rows and a range of K groups (all of K, or
-// 1/splits of it); warp w owns rows 16w .. 16w+15. The group's codes, metadata and
-// activation slice pass through a kGvStages-deep cp.async ring in shared memory, so
-// several groups are always in flight. A warp turns each 32-bit word of codes into 4
+// A CTA owns kGvRows = 64 weight rows and a range of K groups (all of K, or 1/splits of
+// it). Its warps form a 4 x kGvKq grid: warp (rb, kq) owns rows 16rb .. 16rb+15 and the
+// kq-th share of the 8 code words of every group, so each warp's dependent chain per
+// stage is 8/kGvKq words long and the SM holds enough warps to hide the latencies. The
+// group's codes, metadata and activation slice pass through a kGvStages-deep cp.async
+// ring in shared memory, so several groups are always in flight. A warp turns each
+// 32-bit word of codes into 4
 // fp16 pairs in registers (lop3, hsub2, hfma2; the pairs come out in the order (e0,e4)
 // (e1,e5) (e2,e6) (e3,e7)) and uses them directly as A fragments - thread (g, t) holds
 // K positions [16t, 16t+16) of rows g and g+8 - with the activations of the same K
 // positions as B fragments (an interleaved activation row gives them as plain 16-byte
 // loads). No single issuing thread and no staging of dequantised weights.
-// With K splits each split writes its partial tile to the workspace and the last split
-// of a tile to finish (atomic ticket) adds them in split order, so results do not
-// depend on scheduling. The epilogue is the GEMM's (bias, q-scale, ReLU, residual,
+// The kGvKq partial tiles of a CTA are added in shared memory. With K splits each split
+// writes its partial tile to the workspace and the last split of a tile to finish
+// (atomic ticket) adds them in split order, so results do not depend on scheduling. The epilogue is the GEMM's (bias, q-scale, ReLU, residual,
 // interleaved output, fused store_cache).
-constexpr int kGvWarps = 4;
-constexpr int kGvThreads = kGvWarps * 32;
-constexpr int kGvRows = 16 * kGvWarps;     // 64 weight rows per CTA
-constexpr int kGvStages = 3;               // stages of 4 groups (256 K) in flight
+constexpr int kGvRowWarps = 4;             // warps across the rows (16 rows each)
+constexpr int kGvKq = 4;                   // warps across the 8 code words of a group
+constexpr int kGvWords = 8 / kGvKq;        // code words per warp per group
+constexpr int kGvThreads = kGvRowWarps * kGvKq * 32;
+constexpr int kGvCtasPerSm = 1;
+constexpr int kGvRows = 16 * kGvRowWarps;  // 64 weight rows per CTA
+constexpr int kGvStages = 5;               // ring of stages of 4 groups (256 K)
+static_assert(8 * 32 <= kGvThreads, "every epilogue item (activation row, 8 rows) has its own thread");
 
 struct GemvParams {
     const uint8_t* codes;                  // [N][K/2]
@@ -732,6 +739,7 @@ struct GemvParams {
     int nq;
     float qscale;
     int relu, yperm, xperm, early_w;
+    int cluster;                           // K splits reduced inside a thread-block cluster
     uint8_t* kv_codes[2];
     uint32_t* kv_meta[2];
     int kv_h, kv_hd, kv_nh, kv_max_seq, kv_seq, kv_pos0, kv_bits, kv_gs;
@@ -775,15 +783,14 @@ __device__ __forceinline__ uint4 lds128v(uint32_t a) {
 // Epilogue of the small-batch path for activation row m and weight rows n0 + 8c .. +7:
 // bias, q-scale, ReLU, residual, fp16 store (interleaved 8-block order when yperm) and
 // the fused store_cache. The 8 lanes sharing m are consecutive (item = 8 m + c); rows
-// past M return without touching anything.
-__device__ __forceinline__ void gemv_finish(const GemvParams& p, int n0, int c, int m, int lane, const float (&v)[8]) {
+// past M return without touching anything. bv / rv are the 8 bias and residual values,
+// loaded by the caller ahead of time (zeros where there are none).
+__device__ __forceinline__ void gemv_finish(const GemvParams& p, int n0, int c, int m, int lane, const float (&v)[8],
+                                            const uint4 bv, const uint4 rv) {
     const bool valid = m < p.M;
     const int nb = n0 + 8 * c;
     __half o16[8];
     if (valid) {
-        const uint4 bv = p.bias ? __ldg(reinterpret_cast<const uint4*>(p.bias + nb)) : make_uint4(0u, 0u, 0u, 0u);
-        const uint4 rv = p.residual ? *reinterpret_cast<const uint4*>(p.residual + static_cast<int64_t>(m) * p.N + nb)
-                                    : make_uint4(0u, 0u, 0u, 0u);
         const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w}, rw[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -836,7 +843,7 @@ __device__ __forceinline__ void gemv_finish(const GemvParams& p, int n0, int c, 
 }
 
 template <int NT>                          // n-tiles of 8 activation rows (M <= 8 NT)
-__global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p) {
+__global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm) gemv_kernel(const GemvParams p) {
     constexpr int MC = 8 * NT;             // activation rows of the tile
     // stage = 4 groups (256 K): codes [64 rows][128 B + 16 pad], metadata [64][4 groups],
     // activations [MC rows][4 groups][128 B + 16 pad] (the pads spread the fragment loads
@@ -851,6 +858,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
     const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(gv_smem));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
+    const int rb = warp % kGvRowWarps, kq = warp / kGvRowWarps;
     const int tile = blockIdx.x, split = blockIdx.y;
     const int n0 = tile * kGvRows;
     const int ngroups = p.K / 64;
@@ -862,9 +870,10 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
         const uint32_t st = sbase + (i % kGvStages) * STAGE;
         const int G = gb + 4 * i;
 #pragma unroll
-        for (int j = 0; j < (kGvRows * 8) / kGvThreads; ++j) {
+        for (int j = 0; j < (kGvRows * 8 + kGvThreads - 1) / kGvThreads; ++j) {
             const int u = threadIdx.x + j * kGvThreads, row = u >> 3, c16 = u & 7;
-            gv_cp16(st + row * CROW + c16 * 16, p.codes + (n0 + row) * krow + G * 32 + c16 * 16, true);
+            if ((kGvRows * 8) % kGvThreads == 0 || u < kGvRows * 8)
+                gv_cp16(st + row * CROW + c16 * 16, p.codes + (n0 + row) * krow + G * 32 + c16 * 16, true);
         }
         if (threadIdx.x < kGvRows)
             gv_cp16(st + CODES + threadIdx.x * 16, p.meta + static_cast<int64_t>(n0 + threadIdx.x) * ngroups + G, true);
@@ -873,12 +882,13 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
         const uint32_t st = sbase + (i % kGvStages) * STAGE + CODES + META;
         const int G = gb + 4 * i;
 #pragma unroll
-        for (int j = 0; j < (MC * 32) / kGvThreads; ++j) {
+        for (int j = 0; j < (MC * 32 + kGvThreads - 1) / kGvThreads; ++j) {
             const int u = threadIdx.x + j * kGvThreads;
             const int m = u >> 5, q = (u >> 3) & 3, c16 = u & 7;
             const bool ok = m < p.M;
-            gv_cp16(st + (m * 4 + q) * XSEG + c16 * 16,
-                    p.x + static_cast<int64_t>(ok ? m : 0) * p.K + (G + q) * 64 + c16 * 8, ok);
+            if ((MC * 32) % kGvThreads == 0 || u < MC * 32)
+                gv_cp16(st + (m * 4 + q) * XSEG + c16 * 16,
+                        p.x + static_cast<int64_t>(ok ? m : 0) * p.K + (G + q) * 64 + c16 * 8, ok);
         }
     };
     // weights do not depend on the previous kernel: inside a layer call their first
@@ -888,8 +898,19 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
         for (int i = 0; i < kGvStages - 1; ++i)
             if (i < nst) load_weights(i);
     }
+    // this thread's epilogue item, if any: rows n0 + 8 (tid % 8) .. +7 of activation row
+    // m_fin (the cluster reduction gives rank r the rows m = r, r + S, ...); its bias
+    // (a weight) is fetched now, its residual once the previous kernel has finished
+    const int c_fin = threadIdx.x & 7;
+    const int m_fin = (p.splits > 1 && p.cluster) ? split + p.splits * (threadIdx.x >> 3) : (threadIdx.x >> 3);
+    const bool has_fin = m_fin < p.M && (p.splits > 1 && p.cluster ? true : threadIdx.x < 8 * MC);
+    const uint4 bias_v = (has_fin && p.bias) ? __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * c_fin))
+                                             : make_uint4(0u, 0u, 0u, 0u);
     pdl_wait();                            // the activations come from the previous kernel
     pdl_trigger();
+    const uint4 res_v = (has_fin && p.residual)
+                            ? *reinterpret_cast<const uint4*>(p.residual + static_cast<int64_t>(m_fin) * p.N + n0 + 8 * c_fin)
+                            : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int i = 0; i < kGvStages - 1; ++i) {
         if (i < nst) {
@@ -906,9 +927,10 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[nt][j] = acc2[nt][j] = 0.f;
-    // thread (g, t): rows r0 and r0 + 8 of the tile, group t of every stage (its 64 K
-    // positions, 8 code words per row); the MMA's K order is free as long as A and B agree
-    const int r0 = 16 * warp + g;
+    // thread (g, t): rows r0 and r0 + 8 of the tile, group t of every stage, code words
+    // [kq kGvWords, (kq + 1) kGvWords) of it (8 K positions each); the MMA's K order is
+    // free as long as A and B agree
+    const int r0 = 16 * rb + g;
     for (int i = 0; i < nst; ++i) {
         if (i + kGvStages - 1 < nst) {
             load_weights(i + kGvStages - 1);
@@ -918,8 +940,23 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
         gv_wait();
         __syncthreads();
         const uint32_t st = sbase + (i % kGvStages) * STAGE;
-        const uint4 ca0 = lds128v(st + r0 * CROW + t * 32), ca1 = lds128v(st + r0 * CROW + t * 32 + 16);
-        const uint4 cb0 = lds128v(st + (r0 + 8) * CROW + t * 32), cb1 = lds128v(st + (r0 + 8) * CROW + t * 32 + 16);
+        uint32_t wa[kGvWords], wb[kGvWords];
+        {
+            const uint32_t ra = st + r0 * CROW + t * 32 + kq * kGvWords * 4, rbb = ra + 8 * CROW;
+#pragma unroll
+            for (int v = 0; v < kGvWords; v += 4) {
+                if (kGvWords >= 4) {
+                    const uint4 a = lds128v(ra + 4 * v), b = lds128v(rbb + 4 * v);
+                    wa[v] = a.x; wa[v + 1] = a.y; wa[v + 2] = a.z; wa[v + 3] = a.w;
+                    wb[v] = b.x; wb[v + 1] = b.y; wb[v + 2] = b.z; wb[v + 3] = b.w;
+                }
+            }
+            if (kGvWords == 2) {
+                const uint2 a = lds64(ra), b = lds64(rbb);
+                wa[0] = a.x; wa[kGvWords - 1] = a.y; wb[0] = b.x; wb[kGvWords - 1] = b.y;
+            }
+            if (kGvWords == 1) { wa[0] = lds32(ra); wb[0] = lds32(rbb); }
+        }
         const uint32_t mw0 = lds32(st + CODES + r0 * 16 + t * 4), mw1 = lds32(st + CODES + (r0 + 8) * 16 + t * 4);
         uint32_t s2[2], m2[2];
 #pragma unroll
@@ -932,11 +969,9 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
             s2[r] = *reinterpret_cast<const uint32_t*>(&sh);
             m2[r] = *reinterpret_cast<const uint32_t*>(&mh);
         }
-        const uint32_t wa[8] = {ca0.x, ca0.y, ca0.z, ca0.w, ca1.x, ca1.y, ca1.z, ca1.w};
-        const uint32_t wb[8] = {cb0.x, cb0.y, cb0.z, cb0.w, cb1.x, cb1.y, cb1.z, cb1.w};
-        const uint32_t xs = st + CODES + META + (g * 4 + t) * XSEG;
+        const uint32_t xs = st + CODES + META + (g * 4 + t) * XSEG + kq * kGvWords * 16;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
+        for (int w = 0; w < kGvWords; ++w) {
             // K positions 8w .. 8w+7 of group t: A pairs (e0,e4) (e1,e5) (e2,e6) (e3,e7)
             const uint4 d0 = dequant8_4bit_il(wa[w], s2[0], m2[0]);    // row r0
             const uint4 d1 = dequant8_4bit_il(wb[w], s2[1], m2[1]);    // row r0 + 8
@@ -960,45 +995,106 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(const GemvParams p)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[nt][j] += acc2[nt][j];
 
-    // ---- the tile (64 rows x MC activation rows) through shared memory: [64][MC + 1]
+    // ---- the tile (64 rows x MC activation rows) through shared memory: one
+    // [64][MC + 1] partial per word share kq, added in kq order
     float* red = reinterpret_cast<float*>(gv_smem);
+    constexpr int RED = kGvRows * (MC + 1);
+    static_assert(kGvKq * RED * 4 <= STAGE * kGvStages, "reduction tile exceeds the ring");
     __syncthreads();
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) red[(r0 + 8 * (j >> 1)) * (MC + 1) + 8 * nt + 2 * t + (j & 1)] = acc[nt][j];
+        for (int j = 0; j < 4; ++j)
+            red[kq * RED + (r0 + 8 * (j >> 1)) * (MC + 1) + 8 * nt + 2 * t + (j & 1)] = acc[nt][j];
     __syncthreads();
-    // (activation row m, rows 8c .. 8c+7): 8 MC items, 2 per thread at MC = 32
+    // (activation row m, rows 8c .. 8c+7): 8 MC items
     for (int item = threadIdx.x; item < 8 * MC; item += kGvThreads) {
         const int c = item & 7, m = item >> 3;
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = red[(8 * c + i) * (MC + 1) + m];
-        if (p.splits > 1) {
+#pragma unroll
+        for (int q = 1; q < kGvKq; ++q)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] += red[q * RED + (8 * c + i) * (MC + 1) + m];
+        if (p.splits == 1) {
+            gemv_finish(p, n0, c, m, lane, v, bias_v, res_v);
+        } else if (p.cluster) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) red[(8 * c + i) * (MC + 1) + m] = v[i];   // this item's own elements
+        } else {
             float* mine = p.part + (static_cast<int64_t>(tile) * p.splits + split) * kGvRows * 32;
 #pragma unroll
             for (int i = 0; i < 8; ++i) mine[(8 * c + i) * 32 + m] = v[i];
-        } else {
-            gemv_finish(p, n0, c, m, lane, v);
         }
     }
     if (p.splits == 1) return;
-    __threadfence();
+    if (p.cluster) {
+        // The K splits of a tile are one cluster (rank = split). After the barrier every
+        // split's summed partial tile (the kq = 0 slot of its `red`) is visible; rank r
+        // finishes activation rows m = r, r + S, ... adding the partials in split order,
+        // and the second barrier keeps every CTA's shared memory alive until its peers
+        // are done. Every thread of every CTA takes part in both barriers.
+        tc::cluster_sync();
+        const int S = p.splits;
+        if (has_fin) {
+            const int m = m_fin, c = c_fin;
+            const uint32_t own = static_cast<uint32_t>(__cvta_generic_to_shared(red + (8 * c) * (MC + 1) + m));
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = 0.f;
+            for (int sp0 = 0; sp0 < S; sp0 += 4) {
+                float t4[4][8];
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const uint32_t peer = tc::map_peer(own, static_cast<uint32_t>(sp0 + s4 < S ? sp0 + s4 : 0));
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        t4[s4][i] = sp0 + s4 < S ? tc::ld_peer_f32(peer + i * (MC + 1) * 4) : 0.f;
+                }
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] += t4[s4][i];
+            }
+            gemv_finish(p, n0, c, m, lane, v, bias_v, res_v);
+        }
+        tc::cluster_sync();
+        return;
+    }
+    // ticket: the barrier orders every thread's partial stores before thread 0's fence
+    // and atomic (release); the last split's thread 0 fences again before the barrier
+    // that lets its CTA read the other splits' partials (acquire)
     __syncthreads();
-    if (threadIdx.x == 0) last = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+    if (threadIdx.x == 0) {
+        __threadfence();
+        last = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+        if (last) __threadfence();
+    }
     __syncthreads();
     if (!last) return;
-    __threadfence();
     const float* all = p.part + static_cast<int64_t>(tile) * p.splits * kGvRows * 32;
     for (int item = threadIdx.x; item < 8 * MC; item += kGvThreads) {
         const int c = item & 7, m = item >> 3;
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = 0.f;
-        for (int sp = 0; sp < p.splits; ++sp)
+        // four splits' loads in flight at a time, added in split order
+        for (int sp0 = 0; sp0 < p.splits; sp0 += 4) {
+            float t4[4][8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] += __ldcg(all + (static_cast<int64_t>(sp) * kGvRows + 8 * c + i) * 32 + m);
-        gemv_finish(p, n0, c, m, lane, v);
+            for (int s4 = 0; s4 < 4; ++s4)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    t4[s4][i] = sp0 + s4 < p.splits
+                                    ? __ldcg(all + (static_cast<int64_t>(sp0 + s4) * kGvRows + 8 * c + i) * 32 + m)
+                                    : 0.f;
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] += t4[s4][i];
+        }
+        gemv_finish(p, n0, c, m, lane, v, bias_v, res_v);
     }
     if (threadIdx.x == 0) p.counters[tile] = 0;
 }
@@ -1117,25 +1213,63 @@ Plan make_plan(int M, int N, int K, int bits) {
 bool gemv_eligible(int M, int N, int bits) { return bits == 4 && M >= 1 && M <= 32 && N % kGvRows == 0; }
 
 struct GemvPlan {
-    int nt, tiles, splits, gps;
+    int nt, tiles, splits, gps, cluster;
     uint32_t smem;
     int64_t ws_bytes, counters_bytes;
 };
+
+// Clusters of `splits` GEMV CTAs that can be resident at once (cached per device, size
+// and shared memory); 0 if the query fails.
+int gemv_max_active_clusters(int splits, uint32_t smem) {
+    static std::map<std::tuple<int, int, uint32_t>, int> cache;
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(dev, splits, smem);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    set_smem_once(gemv_kernel<4>, static_cast<int>(smem));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, splits, 1);
+    cfg.blockDim = dim3(kGvThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = splits;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemv_kernel<4>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    cache[key] = n;
+    return n;
+}
 
 GemvPlan gemv_plan(int M, int N, int K) {
     GemvPlan P{};
     P.nt = (M + 7) / 8;
     P.tiles = N / kGvRows;
     const int nstages = K / 256;          // stages of 4 groups
-    // split K while the grid fits two CTAs per SM and every split keeps >= 2 stages
+    // split K while the grid fits kGvCtasPerSm CTAs per SM and every split keeps >= 2 stages
     int splits = 1;
-    while (P.tiles * (splits + 1) <= 2 * sm_count() && nstages / (splits + 1) >= 2) ++splits;
+    while (P.tiles * (splits + 1) <= kGvCtasPerSm * sm_count() && nstages / (splits + 1) >= 2) ++splits;
     const int sps = (nstages + splits - 1) / splits;   // stages per split
     P.gps = 4 * sps;
     P.splits = (nstages + sps - 1) / sps;
     P.smem = static_cast<uint32_t>((kGvRows * 144 + kGvRows * 16 + 8 * P.nt * 4 * 144) * kGvStages);
+    // K splits: reduced through distributed shared memory when the splits of every tile
+    // fit one portable cluster and all clusters are resident at once, else through
+    // workspace partials and a ticket
+    P.cluster = (P.splits > 1 && P.splits <= kMaxSplits && gemv_max_active_clusters(P.splits, P.smem) >= P.tiles) ? 1 : 0;
     P.counters_bytes = kTicketBytes;
-    P.ws_bytes = P.splits > 1 ? P.counters_bytes + static_cast<int64_t>(P.tiles) * P.splits * kGvRows * 32 * 4 : 0;
+    P.ws_bytes = (P.splits > 1 && !P.cluster)
+                     ? P.counters_bytes + static_cast<int64_t>(P.tiles) * P.splits * kGvRows * 32 * 4
+                     : 0;
     return P;
 }
 
@@ -1186,6 +1320,7 @@ int gemv_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     gp.yperm = yperm ? 1 : 0;
     gp.xperm = xperm ? 1 : 0;
     gp.early_w = early_w ? 1 : 0;
+    gp.cluster = P.cluster;
     if (kv != nullptr) {
         gp.kv_codes[0] = static_cast<uint8_t*>(kv->cache->k_codes);
         gp.kv_codes[1] = static_cast<uint8_t*>(kv->cache->v_codes);
@@ -1200,11 +1335,25 @@ int gemv_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
         gp.kv_bits = kv->cache->cfg.num_bits;
         gp.kv_gs = kv->cache->cfg.group_size;
     }
-    const dim3 grid(P.tiles, P.splits);
-#define GEMV_LAUNCH(NT_)                                                                            \
-    do {                                                                                            \
-        set_smem_once(gemv_kernel<NT_>, static_cast<int>(P.smem));                                  \
-        launch_k(gemv_kernel<NT_>, grid, dim3(kGvThreads), P.smem, st, true, gp);                   \
+    // programmatic dependent launch, and the K splits of a tile as one cluster
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(P.tiles, P.splits);
+    cfg.blockDim = dim3(kGvThreads);
+    cfg.dynamicSmemBytes = P.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = P.splits;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.cluster ? 2 : 1;
+#define GEMV_LAUNCH(NT_)                                         \
+    do {                                                         \
+        set_smem_once(gemv_kernel<NT_>, static_cast<int>(P.smem)); \
+        cudaLaunchKernelEx(&cfg, gemv_kernel<NT_>, gp);          \
     } while (0)
     switch (P.nt) {
         case 1: GEMV_LAUNCH(1); break;

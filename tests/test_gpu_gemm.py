@@ -107,6 +107,23 @@ def test_gemm_split_k_repeatable(M):
         assert int(ws[:256].view(torch.int32).abs().sum()) == 0
 
 
+@pytest.mark.parametrize("M,N,K", [(8, 128, 8192), (32, 128, 16384), (3, 256, 8192)])
+def test_gemv_many_splits(M, N, K):
+    """A narrow, deep GEMV splits K more ways than one cluster holds (16 or 32 splits),
+    so its partials go through the workspace and the ticket: parity with the oracle,
+    identical bits on a second call, tickets back at zero."""
+    x, w, b, _, y1, ws = _run(M, N, K, fq.FLEX_EPI_NONE, seed=K + M)
+    need = fq.flex_gemm_ws_bytes(M, N, K)
+    assert need > 0
+    assert_layer_close(y1, _oracle_gemm(x, w, b, None, fq.FLEX_EPI_NONE, 4), f"gemv {M}x{N}x{K}")
+    W = fq.CompressedWeight(torch.from_numpy(w).cuda(), 4, 64)
+    y2 = torch.empty_like(y1)
+    fq.flex_dequant_gemm(torch.from_numpy(x).cuda(), W, torch.from_numpy(b).cuda(), None, y2, M, 0, ws)
+    sync_status()
+    assert torch.equal(y1, y2)
+    assert int(ws[:256].view(torch.int32).abs().sum()) == 0
+
+
 @pytest.mark.parametrize("name,M,N,K", [("opt-1.3b qkv decode", 32, 6144, 2048),
                                         ("opt-1.3b fc2 decode", 32, 2048, 8192),
                                         ("opt-30b fc1 gpu-batch", 48, 28672, 7168),
@@ -138,15 +155,15 @@ def test_gemm_bad_args():
     W = fq.CompressedWeight(w)
     y = torch.empty((4, 256), dtype=torch.float16, device="cuda")
     x = torch.zeros((4, 512), dtype=torch.float16, device="cuda")
-    # a shape split along K: if the device needs the workspace reduction for it, a
-    # missing workspace is refused before launch
-    if fq.flex_gemm_ws_bytes(32, 2048, 2048) > 0:
-        W2 = fq.CompressedWeight(torch.zeros((2048, 2048), dtype=torch.float16, device="cuda"))
-        x2 = torch.zeros((32, 2048), dtype=torch.float16, device="cuda")
-        y2 = torch.empty((32, 2048), dtype=torch.float16, device="cuda")
-        with pytest.raises(fq.FlexError) as e:
-            fq.flex_dequant_gemm(x2, W2, None, None, y2, 32, fq.FLEX_EPI_NONE, None)
-        assert e.value.code == fq.FLEX_ERR_WORKSPACE
+    # a narrow, deep shape split along K into more parts than one cluster holds needs
+    # the workspace reduction: a missing workspace is refused before launch
+    assert fq.flex_gemm_ws_bytes(8, 128, 8192) > 0
+    W2 = fq.CompressedWeight(torch.zeros((128, 8192), dtype=torch.float16, device="cuda"))
+    x2 = torch.zeros((8, 8192), dtype=torch.float16, device="cuda")
+    y2 = torch.empty((8, 128), dtype=torch.float16, device="cuda")
+    with pytest.raises(fq.FlexError) as e:
+        fq.flex_dequant_gemm(x2, W2, None, None, y2, 8, fq.FLEX_EPI_NONE, None)
+    assert e.value.code == fq.FLEX_ERR_WORKSPACE
     with pytest.raises(fq.FlexError) as e:
         fq.flex_dequant_gemm(x, W, None, None, y, 4, fq.FLEX_EPI_RESIDUAL, None)
     assert e.value.code == fq.FLEX_ERR_INVALID_ARG

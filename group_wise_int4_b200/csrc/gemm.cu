@@ -702,13 +702,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // mma.sync m16n8k16.
 //
 // A CTA owns kGvRows = 64 weight rows and a range of K groups (all of K, or 1/splits of
-// it). Its warps form a 4 x kGvKq grid: warp (rb, kq) owns rows 16rb .. 16rb+15 and the
+// it). Its warps form a kGvRowWarps x kGvKq grid: warp (rb, kq) owns kGvMt m16 tiles of
+// rows (16 kGvMt rows from 16 kGvMt rb; the tiles share each activation fragment) and the
 // kq-th share of the 8 code words of every group, so each warp's dependent chain per
 // stage is 8/kGvKq words long and the SM holds enough warps to hide the latencies. The
 // group's codes, metadata and activation slice pass through a kGvStages-deep cp.async
 // ring in shared memory, so several groups are always in flight. A warp turns each
-// 32-bit word of codes into 4
-// fp16 pairs in registers (lop3, hsub2, hfma2; the pairs come out in the order (e0,e4)
+// 32-bit word of codes into 4 fp16 pairs in registers (lop3, hsub2, hfma2; the pairs come out in the order (e0,e4)
 // (e1,e5) (e2,e6) (e3,e7)) and uses them directly as A fragments - thread (g, t) holds
 // K positions [16t, 16t+16) of rows g and g+8 - with the activations of the same K
 // positions as B fragments (an interleaved activation row gives them as plain 16-byte
@@ -717,12 +717,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // writes its partial tile to the workspace and the last split of a tile to finish
 // (atomic ticket) adds them in split order, so results do not depend on scheduling. The epilogue is the GEMM's (bias, q-scale, ReLU, residual,
 // interleaved output, fused store_cache).
-constexpr int kGvRowWarps = 4;             // warps across the rows (16 rows each)
+constexpr int kGvMt = 1;                   // m16 row tiles per warp (they share the B fragments)
+constexpr int kGvRowWarps = 4 / kGvMt;     // warps across the rows (16 kGvMt rows each)
 constexpr int kGvKq = 4;                   // warps across the 8 code words of a group
 constexpr int kGvWords = 8 / kGvKq;        // code words per warp per group
 constexpr int kGvThreads = kGvRowWarps * kGvKq * 32;
 constexpr int kGvCtasPerSm = 1;
-constexpr int kGvRows = 16 * kGvRowWarps;  // 64 weight rows per CTA
+constexpr int kGvRows = 16 * kGvMt * kGvRowWarps;  // 64 weight rows per CTA
+static_assert(kGvRows == 64, "the epilogue and the fused store_cache assume 64-row tiles");
 constexpr int kGvStages = 5;               // ring of stages of 4 groups (256 K)
 static_assert(8 * 32 <= kGvThreads, "every epilogue item (activation row, 8 rows) has its own thread");
 
@@ -756,9 +758,6 @@ __device__ __forceinline__ void hmma16816(float (&c)[4], uint32_t a0, uint32_t a
 __device__ __forceinline__ void gv_cp16(uint32_t dst, const void* src, bool pred) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(pred ? 16 : 0)
                  : "memory");
-}
-__device__ __forceinline__ void gv_cp4(uint32_t dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void gv_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void gv_wait() {
@@ -922,59 +921,69 @@ __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm) gemv_kernel(const Ge
 
     // two accumulator sets (the two MMAs of every code word go to different sets), so
     // each set's dependent mma.sync chain is half as long
-    float acc[NT][4], acc2[NT][4];
+    float acc[kGvMt][NT][4], acc2[kGvMt][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int mt = 0; mt < kGvMt; ++mt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[nt][j] = acc2[nt][j] = 0.f;
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[mt][nt][j] = acc2[mt][nt][j] = 0.f;
     // thread (g, t): rows r0 and r0 + 8 of the tile, group t of every stage, code words
     // [kq kGvWords, (kq + 1) kGvWords) of it (8 K positions each); the MMA's K order is
     // free as long as A and B agree
-    const int r0 = 16 * rb + g;
+    const int r0 = 16 * kGvMt * rb + g;       // rows r0 + 16 mt and r0 + 16 mt + 8
     for (int i = 0; i < nst; ++i) {
+        // stage i has landed once all but the newest kGvStages - 2 copy groups are done;
+        // the barrier publishes it and also tells that every warp has finished stage
+        // i - 1, whose slot is refilled right after (one barrier per stage)
+        gv_wait();
+        __syncthreads();
         if (i + kGvStages - 1 < nst) {
             load_weights(i + kGvStages - 1);
             load_x(i + kGvStages - 1);
         }
         gv_commit();
-        gv_wait();
-        __syncthreads();
         const uint32_t st = sbase + (i % kGvStages) * STAGE;
-        uint32_t wa[kGvWords], wb[kGvWords];
-        {
-            const uint32_t ra = st + r0 * CROW + t * 32 + kq * kGvWords * 4, rbb = ra + 8 * CROW;
+        uint32_t wa[kGvMt][kGvWords], wb[kGvMt][kGvWords], s2[kGvMt][2], m2[kGvMt][2];
+#pragma unroll
+        for (int mt = 0; mt < kGvMt; ++mt) {
+            const int ra_row = r0 + 16 * mt;
+            const uint32_t ra = st + ra_row * CROW + t * 32 + kq * kGvWords * 4, rbb = ra + 8 * CROW;
 #pragma unroll
             for (int v = 0; v < kGvWords; v += 4) {
                 if (kGvWords >= 4) {
                     const uint4 a = lds128v(ra + 4 * v), b = lds128v(rbb + 4 * v);
-                    wa[v] = a.x; wa[v + 1] = a.y; wa[v + 2] = a.z; wa[v + 3] = a.w;
-                    wb[v] = b.x; wb[v + 1] = b.y; wb[v + 2] = b.z; wb[v + 3] = b.w;
+                    wa[mt][v] = a.x; wa[mt][v + 1] = a.y; wa[mt][v + 2] = a.z; wa[mt][v + 3] = a.w;
+                    wb[mt][v] = b.x; wb[mt][v + 1] = b.y; wb[mt][v + 2] = b.z; wb[mt][v + 3] = b.w;
                 }
             }
             if (kGvWords == 2) {
                 const uint2 a = lds64(ra), b = lds64(rbb);
-                wa[0] = a.x; wa[kGvWords - 1] = a.y; wb[0] = b.x; wb[kGvWords - 1] = b.y;
+                wa[mt][0] = a.x; wa[mt][kGvWords - 1] = a.y; wb[mt][0] = b.x; wb[mt][kGvWords - 1] = b.y;
             }
-            if (kGvWords == 1) { wa[0] = lds32(ra); wb[0] = lds32(rbb); }
-        }
-        const uint32_t mw0 = lds32(st + CODES + r0 * 16 + t * 4), mw1 = lds32(st + CODES + (r0 + 8) * 16 + t * 4);
-        uint32_t s2[2], m2[2];
+            if (kGvWords == 1) { wa[mt][0] = lds32(ra); wb[mt][0] = lds32(rbb); }
+            const uint32_t mw0 = lds32(st + CODES + ra_row * 16 + t * 4), mw1 = lds32(st + CODES + (ra_row + 8) * 16 + t * 4);
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const uint32_t mwr = r ? mw1 : mw0;
-            const __half mn = __ushort_as_half(static_cast<unsigned short>(mwr & 0xFFFFu));
-            const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mwr >> 16)));
-            const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
-            const __half2 sh = __half2half2(step), mh = __half2half2(mn);
-            s2[r] = *reinterpret_cast<const uint32_t*>(&sh);
-            m2[r] = *reinterpret_cast<const uint32_t*>(&mh);
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t mwr = r ? mw1 : mw0;
+                const __half mn = __ushort_as_half(static_cast<unsigned short>(mwr & 0xFFFFu));
+                const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mwr >> 16)));
+                const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
+                const __half2 sh = __half2half2(step), mh = __half2half2(mn);
+                s2[mt][r] = *reinterpret_cast<const uint32_t*>(&sh);
+                m2[mt][r] = *reinterpret_cast<const uint32_t*>(&mh);
+            }
         }
         const uint32_t xs = st + CODES + META + (g * 4 + t) * XSEG + kq * kGvWords * 16;
 #pragma unroll
         for (int w = 0; w < kGvWords; ++w) {
             // K positions 8w .. 8w+7 of group t: A pairs (e0,e4) (e1,e5) (e2,e6) (e3,e7)
-            const uint4 d0 = dequant8_4bit_il(wa[w], s2[0], m2[0]);    // row r0
-            const uint4 d1 = dequant8_4bit_il(wb[w], s2[1], m2[1]);    // row r0 + 8
+            uint4 d0[kGvMt], d1[kGvMt];
+#pragma unroll
+            for (int mt = 0; mt < kGvMt; ++mt) {
+                d0[mt] = dequant8_4bit_il(wa[mt][w], s2[mt][0], m2[mt][0]);    // row r0 + 16 mt
+                d1[mt] = dequant8_4bit_il(wb[mt][w], s2[mt][1], m2[mt][1]);    // row r0 + 16 mt + 8
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 // activations of row 8 nt + g at the same K positions, as the pairs
@@ -983,17 +992,21 @@ __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm) gemv_kernel(const Ge
                 if (!p.xperm)
                     xv = make_uint4(prmt(xv.x, xv.z, 0x5410u), prmt(xv.x, xv.z, 0x7632u), prmt(xv.y, xv.w, 0x5410u),
                                     prmt(xv.y, xv.w, 0x7632u));
-                hmma16816(acc[nt], d0.x, d1.x, d0.y, d1.y, xv.x, xv.y);
-                hmma16816(acc2[nt], d0.z, d1.z, d0.w, d1.w, xv.z, xv.w);
+#pragma unroll
+                for (int mt = 0; mt < kGvMt; ++mt) {
+                    hmma16816(acc[mt][nt], d0[mt].x, d1[mt].x, d0[mt].y, d1[mt].y, xv.x, xv.y);
+                    hmma16816(acc2[mt][nt], d0[mt].z, d1[mt].z, d0[mt].w, d1[mt].w, xv.z, xv.w);
+                }
             }
         }
-        __syncthreads();                   // the stage is refilled by the next iteration
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int mt = 0; mt < kGvMt; ++mt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[nt][j] += acc2[nt][j];
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[mt][nt][j] += acc2[mt][nt][j];
 
     // ---- the tile (64 rows x MC activation rows) through shared memory: one
     // [64][MC + 1] partial per word share kq, added in kq order
@@ -1002,10 +1015,12 @@ __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm) gemv_kernel(const Ge
     static_assert(kGvKq * RED * 4 <= STAGE * kGvStages, "reduction tile exceeds the ring");
     __syncthreads();
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int mt = 0; mt < kGvMt; ++mt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            red[kq * RED + (r0 + 8 * (j >> 1)) * (MC + 1) + 8 * nt + 2 * t + (j & 1)] = acc[nt][j];
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                red[kq * RED + (r0 + 16 * mt + 8 * (j >> 1)) * (MC + 1) + 8 * nt + 2 * t + (j & 1)] = acc[mt][nt][j];
     __syncthreads();
     // (activation row m, rows 8c .. 8c+7): 8 MC items
     for (int item = threadIdx.x; item < 8 * MC; item += kGvThreads) {

@@ -69,56 +69,58 @@ __global__ void __launch_bounds__(kThreads) compress_contig_kernel(const __half*
     }
 }
 
-// contiguous decompress: one thread per 16 bytes of codes (32 values at 4 bits,
-// 16 values at 8 bits).
+// contiguous decompress: one item = 8 consecutive values (4 or 8 code bytes in, one
+// 16-byte vector out), so a warp's loads and stores each cover one contiguous span.
+constexpr int kDecUnroll = 8;
+
 template <int BITS, int GS>
 __global__ void __launch_bounds__(kThreads) decompress_contig_kernel(const uint8_t* __restrict__ codes,
                                                                      const uint32_t* __restrict__ meta,
                                                                      __half* __restrict__ y,
-                                                                     int64_t chunks) {
-    constexpr int EPT = 128 / BITS;  // values per 16-byte chunk
+                                                                     int64_t items) {
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
-    for (int64_t base = tid; base < chunks; base += nthreads * kUnroll) {
-        uint4 c[kUnroll];
+    for (int64_t base = tid; base < items; base += nthreads * kDecUnroll) {
+        uint2 c[kDecUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t ch = base + u * nthreads;
-            c[u] = ch < chunks ? ld_stream_v4(codes + ch * 16) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t ch = base + u * nthreads;
-            if (ch >= chunks) continue;
-            const int64_t e0 = ch * EPT;
-            // a chunk lies inside one group when EPT <= GS (always: EPT <= 32 <= GS)
-            const uint32_t m = __ldg(meta + e0 / GS);
-            const float mn = h2f_lo(m);
-            const float step = group_step(__ushort_as_half(static_cast<unsigned short>(m >> 16)));
-            const uint32_t w[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
-            uint32_t out[EPT / 2];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
+        for (int u = 0; u < kDecUnroll; ++u) {
+            const int64_t it = base + u * nthreads;
+            c[u] = make_uint2(0u, 0u);
+            if (it < items) {
                 if (BITS == 4) {
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const uint32_t byte = (w[k] >> (8 * b)) & 0xFFu;
-                        out[k * 4 + b] = pack_half2_bits(dequant_one(byte & 15u, step, mn),
-                                                         dequant_one(byte >> 4, step, mn));
-                    }
+                    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(c[u].x) : "l"(codes + it * 4));
                 } else {
-#pragma unroll
-                    for (int b = 0; b < 2; ++b) {
-                        const uint32_t pair = (w[k] >> (16 * b)) & 0xFFFFu;
-                        out[k * 2 + b] = pack_half2_bits(dequant_one(pair & 0xFFu, step, mn),
-                                                         dequant_one(pair >> 8, step, mn));
-                    }
+                    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                                 : "=r"(c[u].x), "=r"(c[u].y)
+                                 : "l"(codes + it * 8));
                 }
             }
-            uint4* dst = reinterpret_cast<uint4*>(y + e0);
+        }
 #pragma unroll
-            for (int q = 0; q < EPT / 8; ++q)
-                st_stream_v4(dst + q, make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]));
+        for (int u = 0; u < kDecUnroll; ++u) {
+            const int64_t it = base + u * nthreads;
+            if (it >= items) continue;
+            // the 8 values lie in one group (GS >= 32)
+            const uint32_t m = __ldg(meta + (it * 8) / GS);
+            const float mn = h2f_lo(m);
+            const float step = group_step(__ushort_as_half(static_cast<unsigned short>(m >> 16)));
+            uint32_t out[4];
+            if (step == 0.0f) {                  // constant group: every value is min
+#pragma unroll
+                for (int k = 0; k < 4; ++k) out[k] = (m & 0xFFFFu) * 0x10001u;
+            } else if (BITS == 4) {
+                const uint32_t w = c[u].x;       // byte k = q[2k] | q[2k+1] << 4
+#pragma unroll
+                for (int k = 0; k < 4; ++k) out[k] = dequant_two((w >> (8 * k)) & 15u, (w >> (8 * k + 4)) & 15u, step, mn);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t w = k < 2 ? c[u].x : c[u].y;
+                    const int sh = 16 * (k & 1);
+                    out[k] = dequant_two((w >> sh) & 0xFFu, (w >> (sh + 8)) & 0xFFu, step, mn);
+                }
+            }
+            st_stream_v4(y + it * 8, make_uint4(out[0], out[1], out[2], out[3]));
         }
     }
 }
@@ -339,8 +341,21 @@ int validate(int32_t ndim, const int64_t* shape, const flexq_config& cfg, Geomet
     return FLEX_OK;
 }
 
+// Grid of a grid-stride kernel: enough blocks for `work_threads`, capped at what the
+// device holds resident at once (blocks per SM from the kernel's registers, times the SM
+// count), so that no block waits for a second wave while the others stream.
+template <auto Kernel>
 unsigned grid_for(int64_t work_threads) {
-    const int64_t cap = static_cast<int64_t>(sm_count()) * (2048 / kThreads);
+    static int per_sm = 0;   // one cached value per kernel (all devices are one type)
+    if (per_sm == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, kThreads, 0) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = 1;
+        }
+        per_sm = n;
+    }
+    const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
     int64_t blocks = (work_threads + kThreads - 1) / kThreads;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
@@ -353,17 +368,17 @@ int launch_compress(const Geometry& g, const __half* x, uint8_t* codes, uint32_t
     if (g.inner == 1) {
         const int64_t G = g.outer * g.ng;
         const int64_t lanes = G * (GS / 8);
-        compress_contig_kernel<BITS, GS><<<grid_for((lanes + kUnroll - 1) / kUnroll), kThreads, 0, st>>>(
-            x, codes, meta, G);
+        const unsigned grid = grid_for<compress_contig_kernel<BITS, GS>>((lanes + kUnroll - 1) / kUnroll);
+        compress_contig_kernel<BITS, GS><<<grid, kThreads, 0, st>>>(x, codes, meta, G);
     } else {
         const bool vec = (g.inner % 8 == 0);
         const int64_t items = g.outer * g.ng * (vec ? g.inner / 8 : g.inner);
         if (vec)
-            compress_strided_kernel<BITS, GS, 8><<<grid_for(items), kThreads, 0, st>>>(x, codes, meta, g.outer,
-                                                                                     g.ng, g.inner);
+            compress_strided_kernel<BITS, GS, 8>
+                <<<grid_for<compress_strided_kernel<BITS, GS, 8>>(items), kThreads, 0, st>>>(x, codes, meta, g.outer, g.ng, g.inner);
         else
-            compress_strided_kernel<BITS, GS, 1><<<grid_for(items), kThreads, 0, st>>>(x, codes, meta, g.outer,
-                                                                                     g.ng, g.inner);
+            compress_strided_kernel<BITS, GS, 1>
+                <<<grid_for<compress_strided_kernel<BITS, GS, 1>>(items), kThreads, 0, st>>>(x, codes, meta, g.outer, g.ng, g.inner);
     }
     return launch_status();
 }
@@ -372,18 +387,18 @@ template <int BITS, int GS>
 int launch_decompress(const Geometry& g, const uint8_t* codes, const uint32_t* meta, __half* y,
                       cudaStream_t st) {
     if (g.inner == 1) {
-        const int64_t chunks = g.n * BITS / 8 / 16;
-        decompress_contig_kernel<BITS, GS><<<grid_for((chunks + kUnroll - 1) / kUnroll), kThreads, 0, st>>>(
-            codes, meta, y, chunks);
+        const int64_t items = g.n / 8;       // n is a multiple of the group size (>= 32)
+        const unsigned grid = grid_for<decompress_contig_kernel<BITS, GS>>((items + kDecUnroll - 1) / kDecUnroll);
+        decompress_contig_kernel<BITS, GS><<<grid, kThreads, 0, st>>>(codes, meta, y, items);
     } else {
         const bool vec = (g.inner % 8 == 0);
         const int64_t items = g.outer * g.ng * (vec ? g.inner / 8 : g.inner);
         if (vec)
-            decompress_strided_kernel<BITS, GS, 8><<<grid_for(items), kThreads, 0, st>>>(codes, meta, y, g.outer,
-                                                                                       g.ng, g.inner);
+            decompress_strided_kernel<BITS, GS, 8>
+                <<<grid_for<decompress_strided_kernel<BITS, GS, 8>>(items), kThreads, 0, st>>>(codes, meta, y, g.outer, g.ng, g.inner);
         else
-            decompress_strided_kernel<BITS, GS, 1><<<grid_for(items), kThreads, 0, st>>>(codes, meta, y, g.outer,
-                                                                                       g.ng, g.inner);
+            decompress_strided_kernel<BITS, GS, 1>
+                <<<grid_for<decompress_strided_kernel<BITS, GS, 1>>(items), kThreads, 0, st>>>(codes, meta, y, g.outer, g.ng, g.inner);
     }
     return launch_status();
 }

@@ -22,6 +22,7 @@ SMALL = [
     ((128, 77), 0, 64, 4), ((64, 5), 0, 32, 8),            # ragged widths: scalar path
     ((3, 5, 7, 128), 3, 64, 4), ((3, 5, 128, 6), 2, 32, 4), ((2, 64, 3, 8), 1, 64, 8),
     ((4096,), 0, 64, 4), ((64,), 0, 64, 4), ((1, 64), 1, 64, 8),
+    ((7, 4160), 1, 64, 4), ((9, 2080), 1, 32, 8), ((5, 3200), 1, 128, 4),   # ragged last staged chunk
 ]
 
 

@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=None, help="stack depth (default: per workload)")
     ap.add_argument("--no-parts", action="store_true", help="skip the per-part measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--codec-only", action="store_true",
+                    help="measure only flexq_compress / flexq_decompress on 1 GiB and print them as one JSON line")
     return ap.parse_args()
 
 
@@ -380,6 +382,40 @@ def _traffic(kernel_key, sha):
     return e.get("dram_bytes_per_launch")
 
 
+def measure_codec(fq, torch, synth, dev, hbm):
+    """flexq_compress / flexq_decompress on 1 GiB of fp16 [131072, 4096], 4-bit group 64,
+    grouped along the contiguous and the strided dimension: GB/s of algorithmic bytes
+    (fp16 in or out, codes, metadata) over 10 back-to-back calls (the tensor is 8x L2)."""
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    codec = {}
+    for gd in (1, 0):
+        shape = (131072, 4096)
+        xt = synth.codec_tensor(shape, gd, 64, 9, device=dev)
+        cfgq = fq.config(4, 64, gd)
+        codes, meta = fq.flexq_compress(xt, cfgq)
+        yt = fq.flexq_decompress(codes, meta, shape, cfgq)
+        n = xt.numel()
+        nbytes = n * 2 + n // 2 + n // 64 * 4
+        for opname, fn in (("compress", lambda: fq.flexq_compress(xt, cfgq, codes, meta)),
+                           ("decompress", lambda: fq.flexq_decompress(codes, meta, shape, cfgq, yt))):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(10):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / 10
+            key = f"{opname}_{'contiguous' if gd == 1 else 'strided'}"
+            codec[key] = {"gbs": nbytes / (ms * 1e6), "frac_hbm": nbytes / (ms * 1e6) / hbm, "ms": ms,
+                          "bytes": nbytes}
+        del xt, codes, meta, yt
+        torch.cuda.empty_cache()
+    return codec
+
+
 def measure_parts(fq, torch, synth, cfg, layers, caches, ws_dec, stream, peaks, dev, prefill_stack, ws_pre):
     """Each kernel of the decode step on its own (same launch configuration, cycling
     over the stack so nothing stays in L2), the prefill, and the codec."""
@@ -493,32 +529,7 @@ def measure_parts(fq, torch, synth, cfg, layers, caches, ws_dec, stream, peaks, 
                "tflops": flops / (pms * 1e9), "frac_tensor_peak": flops / (pms * 1e9) / peaks["bf16_tflops"],
                "peak_note": "fp16 tensor peak = measured bf16 cuBLAS peak (same rate)"}
 
-    # codec on 1 GiB of fp16 [131072, 4096], 4-bit group 64 (contiguous and strided)
-    codec = {}
-    for gd in (1, 0):
-        shape = (131072, 4096)
-        xt = synth.codec_tensor(shape, gd, 64, 9, device=dev)
-        cfgq = fq.config(4, 64, gd)
-        codes, meta = fq.flexq_compress(xt, cfgq)
-        yt = fq.flexq_decompress(codes, meta, shape, cfgq)
-        n = xt.numel()
-        nbytes = n * 2 + n // 2 + n // 64 * 4
-        for opname, fn in (("compress", lambda: fq.flexq_compress(xt, cfgq, codes, meta)),
-                           ("decompress", lambda: fq.flexq_decompress(codes, meta, shape, cfgq, yt))):
-            for _ in range(3):
-                fn()
-            torch.cuda.synchronize()
-            e0.record()
-            for _ in range(10):
-                fn()
-            e1.record()
-            torch.cuda.synchronize()
-            ms = e0.elapsed_time(e1) / 10
-            key = f"{opname}_{'contiguous' if gd == 1 else 'strided'}"
-            codec[key] = {"gbs": nbytes / (ms * 1e6), "frac_hbm": nbytes / (ms * 1e6) / hbm, "ms": ms,
-                          "bytes": nbytes}
-        del xt, codes, meta, yt
-        torch.cuda.empty_cache()
+    codec = measure_codec(fq, torch, synth, dev, hbm)
     rc = fq.flex_get_status()
     if rc != 0:
         raise RuntimeError(f"parts failed: {fq.flex_status_string(rc)}")
@@ -585,9 +596,26 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_codec_only():
+    import torch
+    import group_wise_int4_b200 as fq
+    import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    fq.lib()
+    hbm = measured_peaks()["hbm_gbs"]
+    codec = measure_codec(fq, torch, synth, dev, hbm)
+    rc = fq.flex_get_status()
+    if rc != 0:
+        raise RuntimeError(f"codec failed: {fq.flex_status_string(rc)}")
+    print(json.dumps({"mode": "codec", "unit": "GB/s", "peak_hbm_gbs": hbm, "codec_1gib_4bit_g64": codec}), flush=True)
+
+
 def main():
     args = parse_args()
-    if args.impl == "reference":
+    if args.codec_only:
+        run_codec_only()
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_flexq(args)

@@ -11,9 +11,11 @@
 // Two layouts:
 //   contiguous - the group dimension is the last one: the tensor is a flat sequence of
 //                groups; gs/8 lanes share a group and reduce min/max with shuffles.
-//   strided    - the group dimension has inner extent `inner` > 1 after it: a thread
-//                owns 8 adjacent columns (one 16-byte vector per row), scans the
-//                group's rows once for min/max and once more (from L2) to quantise.
+//   strided    - the group dimension has inner extent `inner` > 1 after it: gs/8
+//                lanes share 8 adjacent columns (one 16-byte vector per row), each
+//                holding 8 of the group's rows in registers; they combine min/max with
+//                shuffles and quantise their rows without reading them again (one column
+//                per thread when the width is not a multiple of 8).
 #include "quant.cuh"
 
 namespace flexq {
@@ -126,107 +128,148 @@ __global__ void __launch_bounds__(kThreads) decompress_contig_kernel(const uint8
 }
 
 // ---------------------------------------------------------------------------------
-// strided compress: x viewed as [outer][ng*GS][inner]; a work item is (o, g, 8 columns)
-// (VEC = 8) or (o, g, 1 column) (VEC = 1, ragged widths or unaligned pointers).
-template <int BITS, int GS, int VEC>
+// strided compress, one pass: x viewed as [outer][ng*GS][inner]; a work item is (o, g,
+// 8 columns) and NS = GS/8 lanes share it, each holding 8 of the group's rows in
+// registers. Lane = IPW slice + ci: a warp covers IPW = 32/NS adjacent items (ci), so
+// every load instruction reads 16 IPW contiguous bytes per row slice. The slices combine
+// min/max with shuffles (lane offsets IPW, 2 IPW, ...) and then quantise their own rows
+// with no second read.
+template <int BITS, int GS>
+__global__ void __launch_bounds__(kThreads) compress_strided_1pass_kernel(const __half* __restrict__ x,
+                                                                          uint8_t* __restrict__ codes,
+                                                                          uint32_t* __restrict__ meta, int64_t outer,
+                                                                          int64_t ng, int64_t inner) {
+    constexpr int RPS = 8;                     // rows per slice
+    constexpr int NS = GS / RPS;               // slices (lanes) per item
+    constexpr int IPW = 32 / NS;               // items per warp
+    constexpr int CB = GS * BITS / 8;          // code rows per group
+    const int lane = threadIdx.x & 31, ci = lane % IPW, slice = lane / IPW;
+    const int64_t cols = inner / 8;
+    const int64_t items = outer * ng * cols;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+    for (int64_t base = warp * IPW; base < items; base += nwarps * IPW) {
+        const int64_t it = base + ci;
+        const bool ok = it < items;            // the 8 lanes of an item agree
+        const int64_t cv = ok ? it % cols : 0, og = ok ? it / cols : 0;
+        const int64_t c0 = cv * 8;
+        const __half* src = x + (og * GS + slice * RPS) * inner + c0;
+        uint4 v[RPS];
+#pragma unroll
+        for (int r = 0; r < RPS; ++r) v[r] = ok ? ld_stream_v4(src + r * inner) : make_uint4(0u, 0u, 0u, 0u);
+        __half2 m2[4], M2[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t w0 = k == 0 ? v[0].x : (k == 1 ? v[0].y : (k == 2 ? v[0].z : v[0].w));
+            m2[k] = M2[k] = *reinterpret_cast<const __half2*>(&w0);
+        }
+#pragma unroll
+        for (int r = 1; r < RPS; ++r) {
+            const __half2* h = reinterpret_cast<const __half2*>(&v[r]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                m2[k] = __hmin2(m2[k], h[k]);
+                M2[k] = __hmax2(M2[k], h[k]);
+            }
+        }
+#pragma unroll
+        for (int off = IPW; off < 32; off <<= 1) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t a = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<const uint32_t*>(&m2[k]), off);
+                const uint32_t b = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<const uint32_t*>(&M2[k]), off);
+                m2[k] = __hmin2(m2[k], *reinterpret_cast<const __half2*>(&a));
+                M2[k] = __hmax2(M2[k], *reinterpret_cast<const __half2*>(&b));
+            }
+        }
+        if (!ok) continue;
+        float mn[8], s[8];
+        uint32_t mw[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            mn[2 * k] = __low2float(m2[k]);
+            mn[2 * k + 1] = __high2float(m2[k]);
+            const float mx0 = __low2float(M2[k]), mx1 = __high2float(M2[k]);
+            const __half s0 = group_scale16<BITS>(mn[2 * k], mx0), s1 = group_scale16<BITS>(mn[2 * k + 1], mx1);
+            s[2 * k] = __half2float(s0);
+            s[2 * k + 1] = __half2float(s1);
+            mw[2 * k] = pack_half2_bits(__float2half_rn(mn[2 * k]), s0);
+            mw[2 * k + 1] = pack_half2_bits(__float2half_rn(mn[2 * k + 1]), s1);
+        }
+        uint64_t mn2[4], s2[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            mn2[k] = f2_pack(mn[2 * k], mn[2 * k + 1]);
+            s2[k] = f2_pack(s[2 * k], s[2 * k + 1]);
+        }
+        uint8_t* dst = codes + og * CB * inner + c0;
+        if (BITS == 4) {
+#pragma unroll
+            for (int r = 0; r < RPS; r += 2) {
+                const uint32_t wa[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+                const uint32_t wb[4] = {v[r + 1].x, v[r + 1].y, v[r + 1].z, v[r + 1].w};
+                uint32_t p[8];                 // column c: q[row r] + 16 q[row r + 1] in the low byte
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    uint32_t a0, a1, b0, b1;
+                    quant_bits_pair(wa[k], mn2[k], s2[k], a0, a1);
+                    quant_bits_pair(wb[k], mn2[k], s2[k], b0, b1);
+                    p[2 * k] = a0 + (b0 << 4);
+                    p[2 * k + 1] = a1 + (b1 << 4);
+                }
+                st_stream_v2(dst + ((slice * RPS + r) / 2) * inner,
+                             make_uint2(pack_low_bytes(p[0], p[1], p[2], p[3]), pack_low_bytes(p[4], p[5], p[6], p[7])));
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < RPS; ++r) {
+                const uint32_t wa[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+                uint32_t p[8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) quant_bits_pair(wa[k], mn2[k], s2[k], p[2 * k], p[2 * k + 1]);
+                st_stream_v2(dst + (slice * RPS + r) * inner,
+                             make_uint2(pack_low_bytes(p[0], p[1], p[2], p[3]), pack_low_bytes(p[4], p[5], p[6], p[7])));
+            }
+        }
+        if (slice == 0) {
+            uint32_t* md = meta + og * inner + c0;
+            st_stream_v4(md, make_uint4(mw[0], mw[1], mw[2], mw[3]));
+            st_stream_v4(md + 4, make_uint4(mw[4], mw[5], mw[6], mw[7]));
+        }
+    }
+}
+
+// strided compress, one column per thread: x viewed as [outer][ng*GS][inner], a work
+// item is (o, g, 1 column); serves widths that are not a multiple of 8 columns.
+template <int BITS, int GS>
 __global__ void __launch_bounds__(kThreads) compress_strided_kernel(const __half* __restrict__ x,
                                                                     uint8_t* __restrict__ codes,
                                                                     uint32_t* __restrict__ meta,
                                                                     int64_t outer, int64_t ng,
                                                                     int64_t inner) {
-    const int64_t cols = inner / VEC;
-    const int64_t items = outer * ng * cols;
+    const int64_t items = outer * ng * inner;
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
     constexpr int CB = GS * BITS / 8;  // code rows per group
     for (int64_t it = tid; it < items; it += nthreads) {
-        const int64_t cv = it % cols;
-        const int64_t og = it / cols;  // o * ng + g
-        const int64_t c0 = cv * VEC;
+        const int64_t c0 = it % inner;
+        const int64_t og = it / inner;  // o * ng + g
         const __half* src = x + og * GS * inner + c0;
-        float mn[VEC], mx[VEC];
-        if (VEC == 8) {
-            __half2 m2[4], M2[4];
-            {
-                const uint4 v = ld_stream_v4(src);
-                const __half2* h = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m2[k] = M2[k] = h[k];
-            }
-#pragma unroll 8
-            for (int r = 1; r < GS; ++r) {
-                const uint4 v = *reinterpret_cast<const uint4*>(src + r * inner);
-                const __half2* h = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    m2[k] = __hmin2(m2[k], h[k]);
-                    M2[k] = __hmax2(M2[k], h[k]);
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                mn[2 * k] = __low2float(m2[k]);
-                mn[2 * k + 1] = __high2float(m2[k]);
-                mx[2 * k] = __low2float(M2[k]);
-                mx[2 * k + 1] = __high2float(M2[k]);
-            }
-        } else {
-            mn[0] = mx[0] = __half2float(src[0]);
-            for (int r = 1; r < GS; ++r) {
-                const float v = __half2float(src[r * inner]);
-                mn[0] = fminf(mn[0], v);
-                mx[0] = fmaxf(mx[0], v);
-            }
+        float mn = __half2float(src[0]), mx = mn;
+        for (int r = 1; r < GS; ++r) {
+            const float v = __half2float(src[r * inner]);
+            mn = fminf(mn, v);
+            mx = fmaxf(mx, v);
         }
-        float s[VEC];
-        uint32_t mw[VEC];
-#pragma unroll
-        for (int k = 0; k < VEC; ++k) {
-            const __half s16 = group_scale16<BITS>(mn[k], mx[k]);
-            s[k] = __half2float(s16);
-            mw[k] = pack_half2_bits(__float2half_rn(mn[k]), s16);
-        }
+        const __half s16 = group_scale16<BITS>(mn, mx);
+        const float s = __half2float(s16);
         uint8_t* dst = codes + og * CB * inner + c0;
-        if (VEC == 8) {
-#pragma unroll 4
-            for (int r = 0; r < GS; r += (BITS == 4 ? 2 : 1)) {
-                const uint4 a = *reinterpret_cast<const uint4*>(src + r * inner);
-                const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
-                uint32_t lo = 0, hi = 0;
-                if (BITS == 4) {
-                    const uint4 b = *reinterpret_cast<const uint4*>(src + (r + 1) * inner);
-                    const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t q0 = quant_one<4>(h2f_lo(wa[k]), mn[2 * k], s[2 * k]) |
-                                            (quant_one<4>(h2f_lo(wb[k]), mn[2 * k], s[2 * k]) << 4);
-                        const uint32_t q1 = quant_one<4>(h2f_hi(wa[k]), mn[2 * k + 1], s[2 * k + 1]) |
-                                            (quant_one<4>(h2f_hi(wb[k]), mn[2 * k + 1], s[2 * k + 1]) << 4);
-                        const uint32_t two = q0 | (q1 << 8);
-                        if (k < 2) lo |= two << (16 * k); else hi |= two << (16 * (k - 2));
-                    }
-                    st_stream_v2(dst + (r / 2) * inner, make_uint2(lo, hi));
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t two = quant_one<8>(h2f_lo(wa[k]), mn[2 * k], s[2 * k]) |
-                                             (quant_one<8>(h2f_hi(wa[k]), mn[2 * k + 1], s[2 * k + 1]) << 8);
-                        if (k < 2) lo |= two << (16 * k); else hi |= two << (16 * (k - 2));
-                    }
-                    st_stream_v2(dst + r * inner, make_uint2(lo, hi));
-                }
-            }
-            uint32_t* md = meta + og * inner + c0;
-            st_stream_v4(md, make_uint4(mw[0], mw[1], mw[2], mw[3]));
-            st_stream_v4(md + 4, make_uint4(mw[4], mw[5], mw[6], mw[7]));
-        } else {
-            for (int r = 0; r < GS; r += (BITS == 4 ? 2 : 1)) {
-                uint32_t q = quant_one<BITS>(__half2float(src[r * inner]), mn[0], s[0]);
-                if (BITS == 4) q |= quant_one<4>(__half2float(src[(r + 1) * inner]), mn[0], s[0]) << 4;
-                dst[(BITS == 4 ? r / 2 : r) * inner] = static_cast<uint8_t>(q);
-            }
-            meta[og * inner + c0] = mw[0];
+        for (int r = 0; r < GS; r += (BITS == 4 ? 2 : 1)) {
+            uint32_t q = quant_one<BITS>(__half2float(src[r * inner]), mn, s);
+            if (BITS == 4) q |= quant_one<4>(__half2float(src[(r + 1) * inner]), mn, s) << 4;
+            dst[(BITS == 4 ? r / 2 : r) * inner] = static_cast<uint8_t>(q);
         }
+        meta[og * inner + c0] = pack_half2_bits(__float2half_rn(mn), s16);
     }
 }
 
@@ -373,12 +416,12 @@ int launch_compress(const Geometry& g, const __half* x, uint8_t* codes, uint32_t
     } else {
         const bool vec = (g.inner % 8 == 0);
         const int64_t items = g.outer * g.ng * (vec ? g.inner / 8 : g.inner);
-        if (vec)
-            compress_strided_kernel<BITS, GS, 8>
-                <<<grid_for<compress_strided_kernel<BITS, GS, 8>>(items), kThreads, 0, st>>>(x, codes, meta, g.outer, g.ng, g.inner);
+        if (vec)   // GS/8 lanes per item
+            compress_strided_1pass_kernel<BITS, GS>
+                <<<grid_for<compress_strided_1pass_kernel<BITS, GS>>(items * (GS / 8)), kThreads, 0, st>>>(x, codes, meta, g.outer, g.ng, g.inner);
         else
-            compress_strided_kernel<BITS, GS, 1>
-                <<<grid_for<compress_strided_kernel<BITS, GS, 1>>(items), kThreads, 0, st>>>(x, codes, meta, g.outer, g.ng, g.inner);
+            compress_strided_kernel<BITS, GS>
+                <<<grid_for<compress_strided_kernel<BITS, GS>>(items), kThreads, 0, st>>>(x, codes, meta, g.outer, g.ng, g.inner);
     }
     return launch_status();
 }

@@ -95,10 +95,20 @@ __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const __half* __r
                                                                const __half* __restrict__ b,
                                                                __half* __restrict__ y, int h) {
     __shared__ float red[LN_THREADS / 32];
-    pdl_wait();
-    pdl_trigger();
     const int64_t row = blockIdx.x;
     const int nvec = h / 8;
+    // the gain and bias are parameters: fetched before waiting for the previous kernel
+    const uint4* gr = reinterpret_cast<const uint4*>(g);
+    const uint4* br = reinterpret_cast<const uint4*>(b);
+    uint4 gv[LN_VPT], bv[LN_VPT];
+#pragma unroll
+    for (int i = 0; i < LN_VPT; ++i) {
+        const int c = threadIdx.x + i * LN_THREADS;
+        gv[i] = c < nvec ? __ldg(gr + c) : make_uint4(0, 0, 0, 0);
+        bv[i] = c < nvec ? __ldg(br + c) : make_uint4(0, 0, 0, 0);
+    }
+    pdl_wait();
+    pdl_trigger();
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * h);
     uint4 v[LN_VPT];
     float sum = 0.f;
@@ -125,17 +135,14 @@ __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const __half* __r
     }
     const float var = block_sum(sq, red) / static_cast<float>(h);
     const float rstd = rsqrtf(var + 1e-5f);
-    const uint4* gr = reinterpret_cast<const uint4*>(g);
-    const uint4* br = reinterpret_cast<const uint4*>(b);
     uint4* yr = reinterpret_cast<uint4*>(y + row * h);
 #pragma unroll
     for (int i = 0; i < LN_VPT; ++i) {
         const int c = threadIdx.x + i * LN_THREADS;
         if (c >= nvec) continue;
-        const uint4 gv = __ldg(gr + c), bv = __ldg(br + c);
         const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+        const uint32_t gw[4] = {gv[i].x, gv[i].y, gv[i].z, gv[i].w};
+        const uint32_t bw[4] = {bv[i].x, bv[i].y, bv[i].z, bv[i].w};
         uint32_t o[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {

@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : 4) decode_attn_tc_ke
     const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
     const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
     float* __restrict__ part, const __half* __restrict__ k_new, const __half* __restrict__ v_new,
-    __half* __restrict__ o, int perm) {
+    __half* __restrict__ o, int perm, int early_kv) {
     constexpr int G = D / GS;              // groups per key: 1, 2 or 4
     constexpr int KB = D / 2;              // code bytes per key
     constexpr int KW = D / 32;             // QK: code words per key and thread (D/4 dims)
@@ -312,8 +312,6 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : 4) decode_attn_tc_ke
     __shared__ float sm_m[NW], sm_l[NW];
     __shared__ float sm_o[NW][D];
     __shared__ float sm_red[NW];
-    pdl_wait();
-    pdl_trigger();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -352,11 +350,21 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : 4) decode_attn_tc_ke
             cp_async4(st + 2 * CODE + META * 4 + u * 4, vm_src + off, ok);
         }
     };
+    // Inside a layer call (early_kv) the cached keys/values [0, pos) were written by
+    // kernels that completed before the previous kernel's own launch wait, and the
+    // previous kernel (the QKV projection) writes only position pos and the query: the
+    // first stages are then requested before waiting for it.
+    auto prologue = [&]() {
 #pragma unroll
-    for (int s = 0; s < DT_NS - 1; ++s) {
-        if (s < nst) load_stage(s);
-        cp_async_commit();
-    }
+        for (int s = 0; s < DT_NS - 1; ++s) {
+            if (s < nst) load_stage(s);
+            cp_async_commit();
+        }
+    };
+    if (early_kv) prologue();
+    pdl_wait();
+    pdl_trigger();
+    if (!early_kv) prologue();
 
     // ---- query: group sums and the QK B operand (this thread's D/4 dims, column g)
     const __half* qp = q + static_cast<int64_t>(b) * row_stride + head * D;
@@ -881,7 +889,8 @@ int64_t decode_attn_ws_bound(int pairs, int head_dim) {
 }
 
 int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new, const void* v_new,
-                       int64_t row_stride, void* o, int batch, int pos, void* ws, bool perm, cudaStream_t st) {
+                       int64_t row_stride, void* o, int batch, int pos, void* ws, bool perm, cudaStream_t st,
+                       bool early_kv) {
     const int pairs = batch * c->n_heads;
     const int ns = decode_attn_nsplit(pairs, pos);
     const int chunk = ns > 0 ? (pos + ns - 1) / ns : 0;
@@ -904,7 +913,7 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
              vm, c->n_heads, c->max_seq, pos, chunk, part)
 #define MMA(D_, G_)                                                                                      \
     launch_k(decode_attn_tc_kernel<D_, G_>, grid, dim3(DA_THREADS), 0, st, true, qh, row_stride, kc, km, vc, vm, \
-             c->n_heads, c->max_seq, pos, chunk, part, kn, vn, oh, perm ? 1 : 0)
+             c->n_heads, c->max_seq, pos, chunk, part, kn, vn, oh, perm ? 1 : 0, early_kv ? 1 : 0)
         if (B == 4) {
             if (D == 64 && G == 64) MMA(64, 64);
             else if (D == 64) MMA(64, 32);
@@ -979,7 +988,7 @@ extern "C" int flex_decode_attention(const flex_kv_cache* cache, const void* q, 
     const int64_t need = decode_attn_ws_bytes(batch * cache->n_heads, cache->head_dim, pos);
     FLEX_REQUIRE(ws != nullptr && ws_bytes >= need, FLEX_ERR_WORKSPACE);
     FLEX_REQUIRE(aligned16(ws), FLEX_ERR_ALIGN);
-    return decode_attn_launch(cache, q, k_new, v_new, row_stride, o, batch, pos, ws, false, as_stream(stream));
+    return decode_attn_launch(cache, q, k_new, v_new, row_stride, o, batch, pos, ws, false, as_stream(stream), false);
 }
 
 extern "C" int flex_prefill_attention(const void* q, const void* k, const void* v, int64_t row_stride, void* o,
@@ -1043,5 +1052,5 @@ extern "C" int flex_decode_attention_noalloc(const flex_kv_cache* cache, const v
     void* scratch = decode_scratch();
     FLEX_REQUIRE(scratch != nullptr, FLEX_ERR_CUDA);
     return decode_attn_launch(cache, q, k_new, v_new, row_stride, o, batch, pos, scratch, false,
-                              as_stream(stream));
+                              as_stream(stream), false);
 }

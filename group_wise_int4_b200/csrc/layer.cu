@@ -21,7 +21,8 @@ int layernorm_launch(const void* x, const void* g, const void* b, void* y, int64
 int append_kv_launch(const flex_kv_cache* c, const void* k_new, const void* v_new, int64_t row_stride, int batch,
                      int seq, int pos0, cudaStream_t st);
 int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new, const void* v_new,
-                       int64_t row_stride, void* o, int batch, int pos, void* ws, bool perm, cudaStream_t st);
+                       int64_t row_stride, void* o, int batch, int pos, void* ws, bool perm, cudaStream_t st,
+                       bool early_kv);
 int64_t decode_attn_ws_bound(int pairs, int head_dim);
 int prefill_attn_launch(const void* q, const void* k, const void* v, int64_t row_stride, void* o, int batch,
                         int seq, int n_heads, int head_dim, cudaStream_t st);
@@ -119,7 +120,7 @@ int run_layer(const flex_layer* L, const flex_kv_cache* C, const void* x_in, voi
         rc = gemm_launch(a, &L->w_qkv, L->b_qkv, nullptr, qkv, M, 0, h, qscale, true, false, gws, w.gemm_bytes, st, &kv, true);
     if (rc != FLEX_OK) return rc;
     if (dec)
-        rc = decode_attn_launch(C, qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, pos, base + w.attn, true, st);
+        rc = decode_attn_launch(C, qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, pos, base + w.attn, true, st, true);
     else
         rc = prefill_attn_launch(qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, seq, L->n_heads, L->head_dim, st);
     if (rc == FLEX_OK)

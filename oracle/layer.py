@@ -51,23 +51,63 @@ def softmax_rows(scores):
     return e / e.sum(axis=-1, keepdims=True)
 
 
+ROW_BLOCK_ELEMS = 1 << 25      # weights are processed in blocks of whole rows of at most this many elements
+
+
+def _row_blocks(rows, cols):
+    """Row ranges [r0, r1) covering a [rows][cols] weight, each at most ROW_BLOCK_ELEMS elements.
+
+    Groups run along the rows (group_dim 1), so blocks of whole rows are independent:
+    blocking changes no result, it only bounds the host memory of the large layers."""
+    step = max(1, ROW_BLOCK_ELEMS // max(1, cols))
+    return [(r0, min(rows, r0 + step)) for r0 in range(0, rows, step)]
+
+
 def compress_weights(raw, num_bits=4, group_size=64):
     """Quantise the four weight matrices of a raw parameter dict with the oracle codec.
 
-    Returns a dict with the same keys; each weight is (codes, meta, shape).
-    """
+    Returns a dict with the same keys; each weight is (codes, meta, shape)."""
     out = dict(raw)
     for k in ("w_qkv", "w_o", "w_fc1", "w_fc2"):
-        w = np.asarray(raw[k], dtype=np.float16)
-        c, m = codec.compress(w, num_bits=num_bits, group_size=group_size, group_dim=1)
-        out[k] = (c, m, w.shape)
+        w = np.asarray(raw[k])
+        if w.dtype != np.float16:
+            raise TypeError("weights must be float16")
+        rows, cols = w.shape
+        codes = np.empty((rows, cols * num_bits // 8), np.uint8)
+        meta = np.empty((rows, cols // group_size, 2), np.float16)
+        for r0, r1 in _row_blocks(rows, cols):
+            codes[r0:r1], meta[r0:r1] = codec.compress(w[r0:r1], num_bits=num_bits, group_size=group_size,
+                                                       group_dim=1)
+        out[k] = (codes, meta, w.shape)
     return out
 
 
-def dequant_weight(wq, num_bits=4, group_size=64):
+def dequant_weight(wq, num_bits=4, group_size=64, dtype=np.float64):
+    """Dequantised weight [rows][cols]: the codec's fp16 output, widened to `dtype`
+    (float16 keeps it as the codec returns it; every fp16 value is exact in float64)."""
     c, m, shape = wq
-    return codec.decompress(c, m, shape, num_bits=num_bits, group_size=group_size,
-                            group_dim=1).astype(np.float64)
+    rows, cols = shape
+    out = np.empty(shape, dtype)
+    for r0, r1 in _row_blocks(rows, cols):
+        out[r0:r1] = codec.decompress(c[r0:r1], m[r0:r1], (r1 - r0, cols), num_bits=num_bits,
+                                      group_size=group_size, group_dim=1)
+    return out
+
+
+def linear(a, w, bias=None):
+    """a @ w.T (+ bias) in float64. w is a dense [out][in] weight (float64, or float16
+    widened block by block, which gives the same products without a float64 copy of
+    the whole matrix)."""
+    a = np.asarray(a, np.float64)
+    if w.dtype == np.float64:
+        y = a @ w.T
+    else:
+        y = np.empty(a.shape[:-1] + (w.shape[0],), np.float64)
+        for r0, r1 in _row_blocks(*w.shape):
+            y[..., r0:r1] = a @ w[r0:r1].astype(np.float64).T
+    if bias is not None:
+        y += np.asarray(bias, np.float64)
+    return y
 
 
 class KVCache:
@@ -126,7 +166,7 @@ def qkv_projection(x, P, Wqkv, n_heads):
     h = x.shape[-1]
     d = h // n_heads
     a = layer_norm(x, P["ln1_g"], P["ln1_b"])
-    qkv = a @ Wqkv.T + np.asarray(P["b_qkv"], np.float64)
+    qkv = linear(a, Wqkv, P["b_qkv"])
     q = qkv[..., 0:h] / np.sqrt(d)
     k = qkv[..., h:2 * h]
     v = qkv[..., 2 * h:3 * h]
@@ -144,15 +184,17 @@ def attention_probs_prefill(q, k):
 
 def mlp_block(x, o, P, W):
     """Output projection, residual, LN2, ReLU FFN, residual (all float64)."""
-    h1 = np.asarray(x, np.float64) + o @ W["w_o"].T + np.asarray(P["b_o"], np.float64)
+    h1 = np.asarray(x, np.float64) + linear(o, W["w_o"], P["b_o"])
     a2 = layer_norm(h1, P["ln2_g"], P["ln2_b"])
-    f = np.maximum(a2 @ W["w_fc1"].T + np.asarray(P["b_fc1"], np.float64), 0.0)
-    out = h1 + f @ W["w_fc2"].T + np.asarray(P["b_fc2"], np.float64)
+    f = np.maximum(linear(a2, W["w_fc1"], P["b_fc1"]), 0.0)
+    out = h1 + linear(f, W["w_fc2"], P["b_fc2"])
     return out
 
 
-def dequant_all(PQ, num_bits=4, group_size=64):
-    return {k: dequant_weight(PQ[k], num_bits, group_size) for k in ("w_qkv", "w_o", "w_fc1", "w_fc2")}
+def dequant_all(PQ, num_bits=4, group_size=64, dtype=np.float64):
+    """The four dequantised weights; dtype=np.float16 keeps them at half the host memory
+    of float32 (the large layers), with identical values."""
+    return {k: dequant_weight(PQ[k], num_bits, group_size, dtype) for k in ("w_qkv", "w_o", "w_fc1", "w_fc2")}
 
 
 def prefill_layer(x16, PQ, cache: KVCache, n_heads, W=None):

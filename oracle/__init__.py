@@ -25,9 +25,14 @@ Modules:
   precision in which the integer codes are decided on both sides).
 * ``oracle.layer`` - the OPT decoder layer (pre-LayerNorm, fused QKV, causal softmax
   attention, output projection, ReLU FFN, residuals) in fp64 on dequantised weights.
+* ``oracle.cpp`` - access to ``oracle/cpp/flexq_oracle.cpp``, a second, plain C++17
+  statement of the quantiser and of the layer in IEEE fp32 (every operation rounded on
+  its own, no fused multiply-add), written independently of the numpy modules. It is
+  the program the benchmark times as the CPU baseline; its pins cross-check it against
+  the numpy oracle and against closed forms.
 
 Every function is pinned by the tests under ``tests/test_oracle_*.py`` against
 closed forms, hand-worked examples, invariants and brute force; none is
 "parity unpinned".
 """
-from . import codec, layer  # noqa: F401
+from . import codec, layer  # noqa: F401   (oracle.cpp is imported on demand: it compiles C++)

@@ -44,11 +44,23 @@ def layer_norm(x, g, b, eps=LN_EPS):
 
 
 def softmax_rows(scores):
-    """Max-subtracted softmax over the last axis; -inf entries get probability 0."""
+    """Max-subtracted softmax over the last axis; -inf entries get probability 0, and a
+    row with no finite entry (nothing to attend to) gets all zeros."""
     s = np.asarray(scores, dtype=np.float64)
     m = s.max(axis=-1, keepdims=True)
-    e = np.exp(s - m)
-    return e / e.sum(axis=-1, keepdims=True)
+    empty = ~np.isfinite(m)
+    e = np.exp(s - np.where(empty, 0.0, m))
+    z = e.sum(axis=-1, keepdims=True)
+    return np.where(empty, 0.0, e / np.where(empty, 1.0, z))
+
+
+def _key_visible(valid_from, batch, n_keys):
+    """[b][1][1][n_keys] bool: key j of sequence b is a real token (j >= valid_from[b]).
+    valid_from None: every key is."""
+    if valid_from is None:
+        return None
+    vf = np.asarray(valid_from, np.int64).reshape(batch, 1, 1, 1)
+    return np.arange(n_keys)[None, None, None, :] >= vf
 
 
 ROW_BLOCK_ELEMS = 1 << 25      # weights are processed in blocks of whole rows of at most this many elements
@@ -173,11 +185,16 @@ def qkv_projection(x, P, Wqkv, n_heads):
     return _split_heads(q, n_heads), _split_heads(k, n_heads), _split_heads(v, n_heads)
 
 
-def attention_probs_prefill(q, k):
-    """Causal attention probabilities [b][nh][s][s]: row i over keys j <= i."""
+def attention_probs_prefill(q, k, valid_from=None):
+    """Causal attention probabilities [b][nh][s][s]: row i over keys j <= i; with left
+    padding (valid_from[b] = first real token of sequence b) only over keys
+    valid_from[b] <= j <= i, and a pad row (i < valid_from[b]) attends to nothing."""
     s = q.shape[-2]
     scores = q @ np.swapaxes(k, -1, -2)
     mask = np.triu(np.ones((s, s), dtype=bool), k=1)
+    vis = _key_visible(valid_from, q.shape[0], s)
+    if vis is not None:
+        mask = mask | ~vis
     scores = np.where(mask, -np.inf, scores)
     return softmax_rows(scores)
 
@@ -197,59 +214,71 @@ def dequant_all(PQ, num_bits=4, group_size=64, dtype=np.float64):
     return {k: dequant_weight(PQ[k], num_bits, group_size, dtype) for k in ("w_qkv", "w_o", "w_fc1", "w_fc2")}
 
 
-def prefill_layer(x16, PQ, cache: KVCache, n_heads, W=None):
+def prefill_layer(x16, PQ, cache: KVCache, n_heads, W=None, valid_from=None):
     """Prefill (``mha``) over the prompt. x16 fp16 [b][s][h] -> fp16 [b][s][h].
 
     Attention reads the fresh float64 keys/values; the fp16 keys/values of every
-    prompt token are quantised into cache slots [0, s)."""
+    prompt token (pad tokens included) are quantised into cache slots [0, s).
+    valid_from: optional [b] first real token of each left-padded prompt."""
     W = W if W is not None else dequant_all(PQ)
     x = np.asarray(x16, np.float64)
     q, k, v = qkv_projection(x, PQ, W["w_qkv"], n_heads)
-    p = attention_probs_prefill(q, k)
+    p = attention_probs_prefill(q, k, valid_from)
     o = _merge_heads(p @ v)
     out = mlp_block(x, o, PQ, W)
     cache.store(k.astype(np.float16), v.astype(np.float16), 0)
     return out.astype(np.float16)
 
 
-def decode_layer(x16, PQ, cache: KVCache, pos, n_heads, W=None):
+def decode_layer(x16, PQ, cache: KVCache, pos, n_heads, W=None, valid_from=None):
     """Decode step (``mha_gen``) at position pos. x16 fp16 [b][h] -> fp16 [b][h].
 
     The new token attends to the dequantised cache slots [0, pos) and to its own
     fresh float64 key/value at pos; afterwards its fp16 key/value are quantised into
-    slot pos. Sequences are independent, so a cache holding a subset of a batch
-    gives that subset's rows of the full result."""
+    slot pos. With left padding (valid_from[b]) the slots below valid_from[b] are not
+    attended. Sequences are independent, so a cache holding a subset of a batch gives
+    that subset's rows of the full result."""
     W = W if W is not None else dequant_all(PQ)
     x = np.asarray(x16, np.float64)[:, None, :]             # [b][1][h]
     q, k, v = qkv_projection(x, PQ, W["w_qkv"], n_heads)    # [b][nh][1][d]
     kc, vc = cache.load(pos)                                # [b][nh][pos][d]
     keys = np.concatenate([kc, k], axis=2)
     vals = np.concatenate([vc, v], axis=2)
-    p = softmax_rows(q @ np.swapaxes(keys, -1, -2))         # [b][nh][1][pos+1]
+    scores = q @ np.swapaxes(keys, -1, -2)                  # [b][nh][1][pos+1]
+    vis = _key_visible(valid_from, x.shape[0], pos + 1)
+    if vis is not None:
+        vis = vis | (np.arange(pos + 1) == pos)             # the new token itself is real
+        scores = np.where(vis, scores, -np.inf)
+    p = softmax_rows(scores)
     o = _merge_heads(p @ vals)                              # [b][1][h]
     out = mlp_block(x, o, PQ, W)[:, 0, :]
     cache.store(k.astype(np.float16), v.astype(np.float16), pos)
     return out.astype(np.float16)
 
 
-def decode_attention(q16, k_new16, v_new16, cache: KVCache, pos):
+def decode_attention(q16, k_new16, v_new16, cache: KVCache, pos, valid_from=None):
     """Decode attention alone: q, k_new, v_new fp16 [b][nh][d] (q already scaled).
 
-    Returns o float64 [b][nh][d] = softmax(q . [cache[0,pos); k_new]) [cache[0,pos); v_new]."""
+    Returns o float64 [b][nh][d] = softmax(q . [cache[vf,pos); k_new]) [cache[vf,pos); v_new]
+    with vf = valid_from[b] (0 without padding)."""
     q = np.asarray(q16, np.float64)[:, :, None, :]
     kn = np.asarray(k_new16, np.float64)[:, :, None, :]
     vn = np.asarray(v_new16, np.float64)[:, :, None, :]
     kc, vc = cache.load(pos)
     keys = np.concatenate([kc, kn], axis=2)
     vals = np.concatenate([vc, vn], axis=2)
-    p = softmax_rows(q @ np.swapaxes(keys, -1, -2))
+    scores = q @ np.swapaxes(keys, -1, -2)
+    vis = _key_visible(valid_from, q.shape[0], pos + 1)
+    if vis is not None:
+        scores = np.where(vis | (np.arange(pos + 1) == pos), scores, -np.inf)
+    p = softmax_rows(scores)
     return (p @ vals)[:, :, 0, :]
 
 
-def prefill_attention(q16, k16, v16):
+def prefill_attention(q16, k16, v16, valid_from=None):
     """Prefill attention alone on fp16 q/k/v [b][s][nh][d] (q already scaled) -> float64 o."""
     q = np.moveaxis(np.asarray(q16, np.float64), 2, 1)
     k = np.moveaxis(np.asarray(k16, np.float64), 2, 1)
     v = np.moveaxis(np.asarray(v16, np.float64), 2, 1)
-    o = attention_probs_prefill(q, k) @ v
+    o = attention_probs_prefill(q, k, valid_from) @ v
     return np.moveaxis(o, 1, 2)

@@ -71,7 +71,7 @@ class flex_kv_cache(ctypes.Structure):
     _fields_ = [("k_codes", ctypes.c_void_p), ("k_meta", ctypes.c_void_p),
                 ("v_codes", ctypes.c_void_p), ("v_meta", ctypes.c_void_p),
                 ("batch", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("max_seq", ctypes.c_int32), ("cfg", flexq_config)]
+                ("max_seq", ctypes.c_int32), ("cfg", flexq_config), ("valid_from", ctypes.c_void_p)]
 
 
 _I32, _I64, _P = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
@@ -85,19 +85,41 @@ _SIGS = {
                                   _I32, _I32, _P, _I64, _P]),
     "flex_decode_layer": (_I32, [ctypes.POINTER(flex_layer), ctypes.POINTER(flex_kv_cache), _P, _P,
                                  _I32, _I32, _P, _I64, _P]),
+    "flex_prefill_layer_batches": (_I32, [ctypes.POINTER(flex_layer), ctypes.POINTER(flex_kv_cache), _I32, _P, _P,
+                                          _I32, _I32, _P, _I64, _P]),
+    "flex_decode_layer_batches": (_I32, [ctypes.POINTER(flex_layer), ctypes.POINTER(flex_kv_cache), _I32, _P, _P,
+                                         _I32, _I32, _P, _I64, _P]),
     "flex_append_kv": (_I32, [ctypes.POINTER(flex_kv_cache), _P, _P, _I64, _I32, _I32, _P]),
     "flex_decode_attention_ws_bytes": (_I64, [ctypes.POINTER(flex_kv_cache), _I32, _I32]),
     "flex_decode_attention": (_I32, [ctypes.POINTER(flex_kv_cache), _P, _P, _P, _I64, _P, _I32, _I32,
                                      _P, _I64, _P]),
     "flex_decode_attention_noalloc": (_I32, [ctypes.POINTER(flex_kv_cache), _P, _P, _P, _I64, _P, _I32,
                                              _I32, _P]),
-    "flex_prefill_attention": (_I32, [_P, _P, _P, _I64, _P, _I32, _I32, _I32, _I32, _P]),
+    "flex_prefill_attention": (_I32, [_P, _P, _P, _I64, _P, _I32, _I32, _I32, _I32, _P, _P]),
     "flex_gemm_ws_bytes": (_I64, [_I32, _I32, _I32]),
     "flex_dequant_gemm": (_I32, [_P, ctypes.POINTER(flexq_tensor), _P, _P, _P, _I32, _I32, _P, _I64, _P]),
     "flex_layernorm": (_I32, [_P, _P, _P, _P, _I64, _I32, _P]),
     "flex_get_status": (_I32, [_P]),
+    "flex_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "flex_status_string": (ctypes.c_char_p, [_I32]),
+    "flex_abi_layout": (_I64, [_I32, _I32]),
 }
+
+_STRUCTS = (flexq_config, flexq_tensor, flex_layer, flex_kv_cache)   # flex_abi_layout's `which` order
+
+
+def _check_layout(L):
+    """Refuse a library whose struct layouts differ from the ctypes declarations here: a
+    mismatch would make the library read past (or misread) the structs this module
+    passes, and hand the kernels wrong pointers."""
+    for which, S in enumerate(_STRUCTS):
+        fields = [f[0] for f in S._fields_]
+        theirs = [int(L.flex_abi_layout(which, -1))] + [int(L.flex_abi_layout(which, i)) for i in range(len(fields))]
+        ours = [ctypes.sizeof(S)] + [getattr(S, f).offset for f in fields]
+        extra = int(L.flex_abi_layout(which, len(fields)))
+        if theirs != ours or extra != -1:
+            raise RuntimeError(f"libflexq.so struct layout of {S.__name__} differs from the binding "
+                               f"(library {theirs}, binding {ours}); rebuild the library")
 
 _lib = None
 
@@ -116,6 +138,7 @@ def lib():
                 continue
             fn.restype = res
             fn.argtypes = args
+        _check_layout(L)
         _lib = L
     return _lib
 
@@ -262,10 +285,13 @@ class FlexLayer:
 
 class FlexKVCache:
     """Compressed KV cache of one layer: codes [b][nh][max_seq][d*bits/8] uint8 and
-    meta [b][nh][max_seq][d/gs][2] fp16 for keys and values."""
+    meta [b][nh][max_seq][d/gs][2] fp16 for keys and values. valid_from: optional int32
+    CUDA tensor [b] of left-padding starts (first real token of each sequence)."""
 
-    def __init__(self, batch, n_heads, head_dim, max_seq, num_bits=4, group_size=64, device="cuda"):
+    def __init__(self, batch, n_heads, head_dim, max_seq, num_bits=4, group_size=64, device="cuda",
+                 valid_from: Optional[torch.Tensor] = None):
         self.batch, self.n_heads, self.head_dim, self.max_seq = batch, n_heads, head_dim, max_seq
+        self.valid_from = valid_from
         self.cfg = config(num_bits, group_size, 3)
         cs = (batch, n_heads, max_seq, head_dim * num_bits // 8)
         ms = (batch, n_heads, max_seq, head_dim // group_size, 2)
@@ -283,6 +309,7 @@ class FlexKVCache:
             s.batch, s.n_heads, s.head_dim, s.max_seq = self.batch, self.n_heads, self.head_dim, self.max_seq
             s.cfg = self.cfg
             self._struct = s
+        self._struct.valid_from = None if self.valid_from is None else self.valid_from.data_ptr()
         return self._struct
 
     def fill_from(self, k16: torch.Tensor, v16: torch.Tensor, stream=None):
@@ -311,6 +338,31 @@ def flex_decode_layer(layer: FlexLayer, cache: FlexKVCache, x_in, x_out, batch, 
                                  _ptr(x_out), int(batch), int(pos), _ptr(ws),
                                  int(ws.numel() * ws.element_size()), ctypes.c_void_p(_stream(stream)))
     _check(rc, "flex_decode_layer")
+
+
+def _cache_array(caches):
+    arr = (flex_kv_cache * len(caches))()
+    for i, c in enumerate(caches):
+        arr[i] = c.struct()
+    return arr
+
+
+def flex_prefill_layer_batches(layer: FlexLayer, caches, x_in, x_out, batch, seq, ws, stream=None):
+    """len(caches) gpu-batches of `batch` sequences through one layer, one weight pass."""
+    arr = _cache_array(caches)
+    rc = lib().flex_prefill_layer_batches(ctypes.byref(layer.struct()), arr, len(caches), _ptr(x_in), _ptr(x_out),
+                                          int(batch), int(seq), _ptr(ws), int(ws.numel() * ws.element_size()),
+                                          ctypes.c_void_p(_stream(stream)))
+    _check(rc, "flex_prefill_layer_batches")
+
+
+def flex_decode_layer_batches(layer: FlexLayer, caches, x_in, x_out, batch, pos, ws, stream=None):
+    """Decode step of len(caches) gpu-batches of `batch` sequences, one weight pass."""
+    arr = _cache_array(caches)
+    rc = lib().flex_decode_layer_batches(ctypes.byref(layer.struct()), arr, len(caches), _ptr(x_in), _ptr(x_out),
+                                         int(batch), int(pos), _ptr(ws), int(ws.numel() * ws.element_size()),
+                                         ctypes.c_void_p(_stream(stream)))
+    _check(rc, "flex_decode_layer_batches")
 
 
 def flex_append_kv(cache: FlexKVCache, k_new, v_new, row_stride, batch, pos, stream=None):
@@ -342,9 +394,9 @@ def flex_decode_attention_noalloc(cache: FlexKVCache, q, k_new, v_new, row_strid
     _check(rc, "flex_decode_attention_noalloc")
 
 
-def flex_prefill_attention(q, k, v, row_stride, o, batch, seq, n_heads, head_dim, stream=None):
+def flex_prefill_attention(q, k, v, row_stride, o, batch, seq, n_heads, head_dim, valid_from=None, stream=None):
     rc = lib().flex_prefill_attention(_ptr(q), _ptr(k), _ptr(v), int(row_stride), _ptr(o), int(batch),
-                                      int(seq), int(n_heads), int(head_dim),
+                                      int(seq), int(n_heads), int(head_dim), _ptr(valid_from),
                                       ctypes.c_void_p(_stream(stream)))
     _check(rc, "flex_prefill_attention")
 
@@ -366,6 +418,15 @@ def flex_layernorm(x, g, b, y, rows, h, stream=None):
     rc = lib().flex_layernorm(_ptr(x), _ptr(g), _ptr(b), _ptr(y), int(rows), int(h),
                               ctypes.c_void_p(_stream(stream)))
     _check(rc, "flex_layernorm")
+
+
+def flex_abi_layout(which: int, field: int) -> int:
+    return int(lib().flex_abi_layout(int(which), int(field)))
+
+
+def flex_set_wait_limit_ns(ns: int) -> int:
+    """Limit of the GEMM's pipeline waits for later launches (0 = default 2 s); returns the old one."""
+    return int(lib().flex_set_wait_limit_ns(int(ns)))
 
 
 def flex_get_status(stream=None) -> int:

@@ -4,6 +4,8 @@
 // variable whose address is looked up once per device. Kernels with bounded waits
 // record FLEX_ERR_TIMEOUT there instead of trapping; flex_get_status reads and clears
 // it.
+#include <atomic>
+#include <cstddef>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -49,6 +51,13 @@ int sm_count() {
     return g_sm_count[dev];
 }
 
+namespace {
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;     // the drain waits' limit, tc::kWaitLimitNs
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+}  // namespace
+
+uint64_t pipeline_wait_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+
 int* status_word() {
     const int dev = current_device();
     if (dev < 0) return nullptr;
@@ -75,6 +84,44 @@ extern "C" int flex_get_status(void* stream) {
         if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FLEX_ERR_CUDA;
     }
     return v;
+}
+
+extern "C" uint64_t flex_set_wait_limit_ns(uint64_t ns) {
+    return flexq::g_wait_ns.exchange(ns == 0 ? flexq::kDefaultWaitNs : ns);
+}
+
+extern "C" int64_t flex_abi_layout(int32_t which, int32_t field) {
+#define FLEX_FIELDS(T, ...)                                              \
+    {                                                                    \
+        const int64_t offs[] = {__VA_ARGS__};                            \
+        if (field == -1) return static_cast<int64_t>(sizeof(T));        \
+        if (field >= 0 && field < static_cast<int32_t>(sizeof(offs) / sizeof(offs[0]))) return offs[field]; \
+        return -1;                                                       \
+    }
+    switch (which) {
+        case 0:
+            FLEX_FIELDS(flexq_config, offsetof(flexq_config, num_bits), offsetof(flexq_config, group_size),
+                        offsetof(flexq_config, group_dim), offsetof(flexq_config, symmetric))
+        case 1:
+            FLEX_FIELDS(flexq_tensor, offsetof(flexq_tensor, codes), offsetof(flexq_tensor, meta),
+                        offsetof(flexq_tensor, ndim), offsetof(flexq_tensor, shape), offsetof(flexq_tensor, cfg))
+        case 2:
+            FLEX_FIELDS(flex_layer, offsetof(flex_layer, h), offsetof(flex_layer, n_heads),
+                        offsetof(flex_layer, head_dim), offsetof(flex_layer, ffn), offsetof(flex_layer, ln1_g),
+                        offsetof(flex_layer, ln1_b), offsetof(flex_layer, ln2_g), offsetof(flex_layer, ln2_b),
+                        offsetof(flex_layer, w_qkv), offsetof(flex_layer, w_o), offsetof(flex_layer, w_fc1),
+                        offsetof(flex_layer, w_fc2), offsetof(flex_layer, b_qkv), offsetof(flex_layer, b_o),
+                        offsetof(flex_layer, b_fc1), offsetof(flex_layer, b_fc2))
+        case 3:
+            FLEX_FIELDS(flex_kv_cache, offsetof(flex_kv_cache, k_codes), offsetof(flex_kv_cache, k_meta),
+                        offsetof(flex_kv_cache, v_codes), offsetof(flex_kv_cache, v_meta),
+                        offsetof(flex_kv_cache, batch), offsetof(flex_kv_cache, n_heads),
+                        offsetof(flex_kv_cache, head_dim), offsetof(flex_kv_cache, max_seq),
+                        offsetof(flex_kv_cache, cfg), offsetof(flex_kv_cache, valid_from))
+        default:
+            return -1;
+    }
+#undef FLEX_FIELDS
 }
 
 extern "C" const char* flex_status_string(int32_t status) {

@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_split_kernel(
     const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
     const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
     const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
-    float* __restrict__ part) {
+    float* __restrict__ part, const int32_t* __restrict__ valid_from) {
     constexpr int KB = D * BITS / 8;        // code bytes per key
     constexpr int TPK = KB / 16;            // threads per key (16 bytes each)
     constexpr int EPT = 128 / BITS;         // dims per thread
@@ -138,8 +138,10 @@ __global__ void __launch_bounds__(DA_THREADS) decode_attn_split_kernel(
 #pragma unroll
         for (int e = 0; e < EPT; ++e) qsum += qv[e];
     }
-    const int j0 = split * chunk;
-    const int j1 = min(pos, j0 + chunk);
+    // keys [split * chunk, +chunk) of [0, pos), minus the left padding [0, valid_from[b])
+    const int vf = valid_from ? valid_from[b] : 0;
+    const int j0 = max(split * chunk, vf);
+    const int j1 = min(pos, split * chunk + chunk);
     const int64_t slot0 = static_cast<int64_t>(pair) * max_seq;
 
     float m = -FLT_MAX, l = 0.f, U = 0.f;
@@ -286,16 +288,26 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool pre
 // fresh key/value of the current token and writes the normalised output o (in the
 // interleaved 8-block order when perm != 0).
 constexpr int DT_KEYS = 128;
+#ifndef FLEXQ_DT_STAGES
+#define FLEXQ_DT_STAGES 2
+#endif
+constexpr int DT_STAGES = FLEXQ_DT_STAGES;  // stages of DT_KEYS keys in flight per CTA
 
-// 7 CTAs per SM at head_dim 64 (all 1024 CTAs of a 32 x 32-head decode in one wave),
-// 4 at head_dim 128
+// Dynamic shared memory of decode_attn_tc_kernel<D, GS>: the ring of stages, each the
+// codes and metadata of DT_KEYS keys and values.
+constexpr int dt_smem_bytes(int D, int GS) {
+    return DT_STAGES * (2 * DT_KEYS * (D / 2) + 2 * DT_KEYS * (D / GS) * 4);
+}
+
+// 7 CTAs per SM at head_dim 64 (all 1024 CTAs of a 32 x 32-head decode in one wave);
+// at head_dim 128 as many as the shared memory of the ring allows (3 with 3 stages)
 template <int D, int GS>
-__global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : 4) decode_attn_tc_kernel(
+__global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : (DT_STAGES >= 3 ? 3 : 4)) decode_attn_tc_kernel(
     const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
     const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
     const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int chunk,
     float* __restrict__ part, const __half* __restrict__ k_new, const __half* __restrict__ v_new,
-    __half* __restrict__ o, int perm, int early_kv) {
+    __half* __restrict__ o, int perm, int early_kv, const int32_t* __restrict__ valid_from) {
     constexpr int G = D / GS;              // groups per key: 1, 2 or 4
     constexpr int KB = D / 2;              // code bytes per key
     constexpr int KW = D / 32;             // QK: code words per key and thread (D/4 dims)
@@ -305,10 +317,11 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : 4) decode_attn_tc_ke
     constexpr int CODE = DT_KEYS * KB;     // code bytes of a stage (keys or values)
     constexpr int META = DT_KEYS * G;      // metadata words of a stage (keys or values)
     constexpr int STAGE = 2 * CODE + 2 * META * 4;
-    constexpr int DT_NS = D == 128 ? 2 : 3;   // stages in flight (static shared memory < 48 KB)
+    constexpr int DT_NS = DT_STAGES;       // ring depth (dynamic shared memory, dt_smem_bytes)
     static_assert(NW * 32 == DT_KEYS, "32 keys per warp and stage");
     static_assert(CODE % (16 * DA_THREADS) == 0 && META % DA_THREADS == 0, "whole copy rounds");
-    __shared__ __align__(16) uint8_t ring[DT_NS][STAGE];
+    extern __shared__ __align__(16) uint8_t dt_ring[];
+    auto ring = reinterpret_cast<uint8_t (*)[STAGE]>(dt_ring);
     __shared__ float sm_m[NW], sm_l[NW];
     __shared__ float sm_o[NW][D];
     __shared__ float sm_red[NW];
@@ -318,10 +331,13 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : 4) decode_attn_tc_ke
     const int pair = blockIdx.x, split = blockIdx.y, nsplit = gridDim.y;
     const int b = pair / n_heads, head = pair % n_heads;
     const int64_t slot0 = static_cast<int64_t>(pair) * max_seq;
-    const int j0 = split * chunk;
-    const int nkeys = min(pos, j0 + chunk) - j0;                  // keys of this split (> 0)
+    // keys [split * chunk, +chunk) of [0, pos), minus the left padding [0, valid_from[b]);
+    // valid_from is the caller's, written before the layer call (safe before the launch wait)
+    const int vf = valid_from ? valid_from[b] : 0;
+    const int j0 = max(split * chunk, vf);
+    const int nkeys = min(pos, split * chunk + chunk) - j0;       // keys of this split (may be <= 0)
     static_assert(D <= DA_THREADS, "one thread per output dim");
-    const int nst = (nkeys + DT_KEYS - 1) / DT_KEYS;
+    const int nst = nkeys > 0 ? (nkeys + DT_KEYS - 1) / DT_KEYS : 0;
 
     // ---- stage copies: every thread moves CODE/16/128 16-byte units of each code tensor
     // and META/128 metadata words of each metadata tensor; keys past the range are
@@ -701,7 +717,8 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* 
                                                                   const __half* __restrict__ v,
                                                                   int64_t row_stride,
                                                                   __half* __restrict__ o, int seq,
-                                                                  int n_heads) {
+                                                                  int n_heads,
+                                                                  const int32_t* __restrict__ valid_from) {
     constexpr int LD = D + 8;                  // padded smem row (halves): conflict-free ldmatrix
     pdl_wait();
     pdl_trigger();
@@ -718,6 +735,9 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* 
     const int g = lane >> 2, t = lane & 3;
     const int q0 = qb * PA_BQ;
     const int64_t base = static_cast<int64_t>(b) * seq;
+    // left padding: keys below valid_from[b] are never attended; a query row with no
+    // visible key (a pad row) gets a zero output
+    const int vf = valid_from ? min(max(valid_from[b], 0), seq) : 0;
 
     // Q tile
     for (int c = tid; c < PA_BQ * CPR; c += PA_THREADS) {
@@ -738,7 +758,8 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* 
         }
     };
     const int nkb = min((q0 + PA_BQ + PA_BK - 1) / PA_BK, (seq + PA_BK - 1) / PA_BK);
-    load_kv(0, 0);
+    const int kb0 = vf / PA_BK;                // first key block holding a real token
+    if (kb0 < nkb) load_kv(kb0, kb0 & 1);
     cp_async_commit();
 
     uint32_t qa[D / 16][4];
@@ -748,13 +769,13 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* 
     float mrow[2] = {-FLT_MAX, -FLT_MAX}, lrow[2] = {0.f, 0.f};
     constexpr float LOG2E = 1.4426950408889634f;
 
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb = kb0; kb < nkb; ++kb) {
         const int buf = kb & 1;
         if (kb + 1 < nkb) load_kv(kb + 1, buf ^ 1);
         cp_async_commit();
         cp_async_wait<1>();
         __syncthreads();
-        if (kb == 0) {
+        if (kb == kb0) {
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
                 const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -790,7 +811,7 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* 
                 const int key = k0 + nt * 8 + 2 * t + (e & 1);
                 const int qi = qrow0 + (e >> 1) * 8;
                 float val = s[nt][e] * LOG2E;
-                if (key > qi || key >= seq) val = -FLT_MAX;
+                if (key > qi || key >= seq || key < vf) val = -FLT_MAX;
                 s[nt][e] = val;
                 bmax[e >> 1] = fmaxf(bmax[e >> 1], val);
             }
@@ -842,6 +863,7 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* 
         }
         __syncthreads();
     }
+    cp_async_wait<0>();                        // a tile of pad rows visits no key block
     // finalise
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -853,7 +875,7 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* 
     for (int r = 0; r < 2; ++r) {
         const int tok = q0 + warp * 16 + g + r * 8;
         if (tok >= seq) continue;
-        const float inv = 1.f / lrow[r];
+        const float inv = lrow[r] > 0.f ? 1.f / lrow[r] : 0.f;     // a pad row: zero output
         __half* dst = o + (base + tok) * hD + head * D;
 #pragma unroll
         for (int nt = 0; nt < D / 8; ++nt) {
@@ -910,10 +932,14 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
         const dim3 grid(pairs, ns);
 #define SPLIT(D_, B_, G_)                                                                                 \
     launch_k(decode_attn_split_kernel<D_, B_, G_>, grid, dim3(DA_THREADS), 0, st, true, qh, row_stride, kc, km, vc, \
-             vm, c->n_heads, c->max_seq, pos, chunk, part)
+             vm, c->n_heads, c->max_seq, pos, chunk, part, c->valid_from)
 #define MMA(D_, G_)                                                                                      \
-    launch_k(decode_attn_tc_kernel<D_, G_>, grid, dim3(DA_THREADS), 0, st, true, qh, row_stride, kc, km, vc, vm, \
-             c->n_heads, c->max_seq, pos, chunk, part, kn, vn, oh, perm ? 1 : 0, early_kv ? 1 : 0)
+    do {                                                                                                 \
+        set_smem_once(decode_attn_tc_kernel<D_, G_>, dt_smem_bytes(D_, G_));                            \
+        launch_k(decode_attn_tc_kernel<D_, G_>, grid, dim3(DA_THREADS), dt_smem_bytes(D_, G_), st, true, qh, \
+                 row_stride, kc, km, vc, vm, c->n_heads, c->max_seq, pos, chunk, part, kn, vn, oh, perm ? 1 : 0, \
+                 early_kv ? 1 : 0, c->valid_from);                                                       \
+    } while (0)
         if (B == 4) {
             if (D == 64 && G == 64) MMA(64, 64);
             else if (D == 64) MMA(64, 32);
@@ -943,7 +969,7 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
 size_t prefill_attn_smem(int D) { return static_cast<size_t>(PA_BQ + 4 * PA_BK) * (D + 8) * 2; }
 
 int prefill_attn_launch(const void* q, const void* k, const void* v, int64_t row_stride, void* o, int batch,
-                        int seq, int n_heads, int head_dim, cudaStream_t st) {
+                        int seq, int n_heads, int head_dim, const int32_t* valid_from, cudaStream_t st) {
     if (batch == 0 || seq == 0) return FLEX_OK;
     const dim3 grid((seq + PA_BQ - 1) / PA_BQ, n_heads, batch);
     const size_t smem = prefill_attn_smem(head_dim);
@@ -954,11 +980,11 @@ int prefill_attn_launch(const void* q, const void* k, const void* v, int64_t row
     if (head_dim == 64) {
         set_smem_once(prefill_attn_kernel<64>, (int)smem);
         launch_k(prefill_attn_kernel<64>, grid, dim3(PA_THREADS), smem, st, true, qh, kh, vh, row_stride, oh, seq,
-                 n_heads);
+                 n_heads, valid_from);
     } else {
         set_smem_once(prefill_attn_kernel<128>, (int)smem);
         launch_k(prefill_attn_kernel<128>, grid, dim3(PA_THREADS), smem, st, true, qh, kh, vh, row_stride, oh, seq,
-                 n_heads);
+                 n_heads, valid_from);
     }
     return launch_status();
 }
@@ -993,14 +1019,15 @@ extern "C" int flex_decode_attention(const flex_kv_cache* cache, const void* q, 
 
 extern "C" int flex_prefill_attention(const void* q, const void* k, const void* v, int64_t row_stride, void* o,
                                       int32_t batch, int32_t seq, int32_t n_heads, int32_t head_dim,
-                                      void* stream) {
+                                      const int32_t* valid_from, void* stream) {
     FLEX_REQUIRE(q && k && v && o, FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(batch >= 0 && seq >= 0 && n_heads > 0, FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(head_dim == 64 || head_dim == 128, FLEX_ERR_UNSUPPORTED);
     FLEX_REQUIRE(row_stride >= static_cast<int64_t>(n_heads) * head_dim && row_stride % 8 == 0,
                  FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(o), FLEX_ERR_ALIGN);
-    return prefill_attn_launch(q, k, v, row_stride, o, batch, seq, n_heads, head_dim, as_stream(stream));
+    FLEX_REQUIRE(valid_from == nullptr || (reinterpret_cast<uintptr_t>(valid_from) & 3u) == 0, FLEX_ERR_ALIGN);
+    return prefill_attn_launch(q, k, v, row_stride, o, batch, seq, n_heads, head_dim, valid_from, as_stream(stream));
 }
 
 // ---- decode attention with library-owned scratch ---------------------------------------

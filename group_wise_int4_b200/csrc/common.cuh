@@ -54,16 +54,52 @@ inline void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
     cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-// store_cache fused into the QKV projection's epilogue (see gemm.cu).
+// store_cache fused into the QKV projection's epilogue (see gemm.cu). The activation
+// rows may belong to several gpu-batches, each with its own cache: row m is row
+// m % rows of the cache m / rows.
+constexpr int kMaxKvBatches = 8;
 struct KvFuse {
-    const flex_kv_cache* cache;
+    const flex_kv_cache* caches;   // ncaches caches of identical geometry
+    int ncaches;
+    int rows;    // activation rows per cache (its batch * seq)
     int h;       // hidden size: features [h, 2h) keys, [2h, 3h) values
     int seq;     // tokens per sequence in this call
     int pos0;    // cache slot of token 0
 };
 
+// Kernel-side form of KvFuse. codes[0][0] == nullptr: no fused store.
+struct KvTarget {
+    uint8_t* codes[kMaxKvBatches][2];      // [cache][keys, values]
+    uint32_t* meta[kMaxKvBatches][2];
+    int rows, h, hd, nh, max_seq, seq, pos0, bits, gs;
+};
+
+inline void fill_kv_target(KvTarget& t, const KvFuse* kv) {
+    t = KvTarget{};
+    if (kv == nullptr) return;
+    for (int c = 0; c < kv->ncaches && c < kMaxKvBatches; ++c) {
+        t.codes[c][0] = static_cast<uint8_t*>(kv->caches[c].k_codes);
+        t.codes[c][1] = static_cast<uint8_t*>(kv->caches[c].v_codes);
+        t.meta[c][0] = static_cast<uint32_t*>(kv->caches[c].k_meta);
+        t.meta[c][1] = static_cast<uint32_t*>(kv->caches[c].v_meta);
+    }
+    const flex_kv_cache& c0 = kv->caches[0];
+    t.rows = kv->rows;
+    t.h = kv->h;
+    t.hd = c0.head_dim;
+    t.nh = c0.n_heads;
+    t.max_seq = c0.max_seq;
+    t.seq = kv->seq;
+    t.pos0 = kv->pos0;
+    t.bits = c0.cfg.num_bits;
+    t.gs = c0.cfg.group_size;
+}
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
+// Limit of the tensor-core GEMM's pipeline waits for kernels launched from now on
+// (flex_set_wait_limit_ns).
+uint64_t pipeline_wait_ns();
 // Device status word of the current device (created on first use; see flex_get_status).
 int* status_word();
 

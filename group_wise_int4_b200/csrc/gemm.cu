@@ -63,10 +63,11 @@ constexpr int kACols = kTmemCols - kACol0;
 constexpr int kMaxSplits = 8;      // K splits of a tile form one cluster (portable size)
 // Split-K tickets: a fixed region at the start of every GEMM workspace (the partials
 // follow it), so that GEMMs of different tile counts sharing one workspace never write
-// partials over each other's tickets. Split plans have at most 2 * SMs tiles.
+// partials over each other's tickets. A split plan has at most kTicketBytes / 4 tiles.
 constexpr int64_t kTicketBytes = 2048;
 
 struct GemmParams {
+    uint64_t wait_ns;      // limit of the pipeline waits (drain waits keep tc::kWaitLimitNs)
     const __half* bias;
     const __half* residual;
     __half* y;
@@ -94,12 +95,10 @@ struct GemmParams {
     int* counters;
     uint32_t off_x, off_c, off_m, off_bar;
     uint32_t tmem_cols;
-    // fused store_cache (QKV projection): output features [kv_h, 2 kv_h) are the keys and
-    // [2 kv_h, 3 kv_h) the values; token m = b * kv_seq + t goes to cache slot kv_pos0 + t
-    // of sequence b. kv_codes[0] == nullptr: off.
-    uint8_t* kv_codes[2];
-    uint32_t* kv_meta[2];
-    int kv_h, kv_hd, kv_nh, kv_max_seq, kv_seq, kv_pos0, kv_bits, kv_gs;
+    // fused store_cache (QKV projection): output features [kv.h, 2 kv.h) are the keys and
+    // [2 kv.h, 3 kv.h) the values; row m is row r = m % kv.rows of cache m / kv.rows, and
+    // r = b * kv.seq + t goes to slot kv.pos0 + t of that cache's sequence b
+    KvTarget kv;
 };
 
 struct Bars {
@@ -186,9 +185,9 @@ __device__ __forceinline__ uint2 dequant4_8bit(uint32_t w, uint32_t step2, uint3
 template <int BITS>
 __device__ __forceinline__ void kv_store8_bits(const GemmParams& p, const __half (&o16)[8], int col, int m0, int n0,
                                                int n, int warp, int lane, uint32_t* kv_red) {
-    const int sec = (n0 - p.kv_h) / p.kv_h;                // 0 keys, 1 values
-    const int f = n - p.kv_h - sec * p.kv_h;
-    const int head = f / p.kv_hd, dim = f % p.kv_hd;
+    const int sec = (n0 - p.kv.h) / p.kv.h;                // 0 keys, 1 values
+    const int f = n - p.kv.h - sec * p.kv.h;
+    const int head = f / p.kv.hd, dim = f % p.kv.hd;
     // min / max of the 8 columns as 4 half2 pairs
     __half2 mn2[4], mx2[4];
 #pragma unroll
@@ -202,7 +201,7 @@ __device__ __forceinline__ void kv_store8_bits(const GemmParams& p, const __half
             mn2[k] = __hmin2(mn2[k], *reinterpret_cast<const __half2*>(&a));
             mx2[k] = __hmax2(mx2[k], *reinterpret_cast<const __half2*>(&b));
         }
-    if (p.kv_gs == 64) {
+    if (p.kv.gs == 64) {
         const int w = warp - 4, pairbar = 2 + (w >> 1);
         if (lane == 0)
 #pragma unroll
@@ -220,9 +219,7 @@ __device__ __forceinline__ void kv_store8_bits(const GemmParams& p, const __half
         }
         asm volatile("bar.sync %0, 64;" ::"r"(pairbar) : "memory");   // kv_red is reused by the next call
     }
-    uint8_t* codes = p.kv_codes[sec];
-    uint32_t* meta = p.kv_meta[sec];
-    const int gph = p.kv_hd / p.kv_gs;
+    const int gph = p.kv.hd / p.kv.gs;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int m = m0 + col + j;
@@ -232,20 +229,23 @@ __device__ __forceinline__ void kv_store8_bits(const GemmParams& p, const __half
         const uint32_t q = quant_one<BITS>(__half2float(o16[j]), mn, __half2float(s16));
         const uint32_t qn = __shfl_down_sync(0xffffffffu, q, 1);
         if (m >= p.M) continue;
-        const int b = m / p.kv_seq, t = m - b * p.kv_seq;
-        const int64_t slot = (static_cast<int64_t>(b) * p.kv_nh + head) * p.kv_max_seq + p.kv_pos0 + t;
+        const int c = m / p.kv.rows, r = m - c * p.kv.rows;
+        const int b = r / p.kv.seq, t = r - b * p.kv.seq;
+        uint8_t* codes = p.kv.codes[c][sec];
+        uint32_t* meta = p.kv.meta[c][sec];
+        const int64_t slot = (static_cast<int64_t>(b) * p.kv.nh + head) * p.kv.max_seq + p.kv.pos0 + t;
         if (BITS == 4) {
-            if ((lane & 1) == 0) codes[slot * (p.kv_hd / 2) + dim / 2] = static_cast<uint8_t>(q | (qn << 4));
+            if ((lane & 1) == 0) codes[slot * (p.kv.hd / 2) + dim / 2] = static_cast<uint8_t>(q | (qn << 4));
         } else {
-            codes[slot * p.kv_hd + dim] = static_cast<uint8_t>(q);
+            codes[slot * p.kv.hd + dim] = static_cast<uint8_t>(q);
         }
-        if (dim % p.kv_gs == 0) meta[slot * gph + dim / p.kv_gs] = pack_half2_bits(__float2half_rn(mn), s16);
+        if (dim % p.kv.gs == 0) meta[slot * gph + dim / p.kv.gs] = pack_half2_bits(__float2half_rn(mn), s16);
     }
 }
 
 __device__ __forceinline__ void kv_store8(const GemmParams& p, const __half (&o16)[8], int col, int m0, int n0, int n,
                                           int warp, int lane, uint32_t* kv_red) {
-    if (p.kv_bits == 4)
+    if (p.kv.bits == 4)
         kv_store8_bits<4>(p, o16, col, m0, n0, n, warp, lane, kv_red);
     else
         kv_store8_bits<8>(p, o16, col, m0, n0, n, warp, lane, kv_red);
@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     // interleaved output: element k of every 8-block goes to position 2(k%4) + (k/4)%2
     const int n_out = p.yperm ? ((n & ~7) | ((n & 3) << 1) | ((n >> 2) & 1)) : n;
     // fused store_cache: this tile lies inside the key or the value block (h % 128 == 0)
-    const bool kv_on = p.kv_codes[0] != nullptr && n0 >= p.kv_h;
+    const bool kv_on = p.kv.codes[0][0] != nullptr && n0 >= p.kv.h;
     float bias_n = 0.f;                           // read by the epilogue after its PDL wait
     uint32_t all_ok = 0;                          // epilogue warps: the main loop completed
     // bias, q-scale, ReLU, residual, fp16 store (and store_cache) of 8 columns of row n
@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             int st = 0, s = 0;
             uint32_t ph = 0;
             for (; st < nsteps; ++st) {
-                if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ph ^ 1, abort, p.status)) break;
+                if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ph ^ 1, abort, p.status, p.wait_ns)) break;
                 const int c = c_begin + st * KU;
                 tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CSTAGE + MSTAGE);
                 tc::tma_load_2d(sC + s * CSTAGE, &tm_codes, c * CROW, n0, B.codes_full + 8 * s);
@@ -403,7 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 if (u >= NSX) {
                     // the stage last held unit u - NSX: wait for the MMAs of the step that read it
                     const int pj = ((u - NSX) * XU) / KU;
-                    if (!tc::bar_wait(B.mma_done + 8 * (pj % kDoneRing), (pj / kDoneRing) & 1, abort, p.status))
+                    if (!tc::bar_wait(B.mma_done + 8 * (pj % kDoneRing), (pj / kDoneRing) & 1, abort, p.status,
+                                      p.wait_ns))
                         break;
                 }
                 tc::bar_arrive_expect_tx(B.x_full + 8 * s, XU * xbytes);
@@ -434,13 +435,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             int xs = 0;
             uint32_t xph = 0;
             bool ok = true;
-            for (int j = 0; j < nsteps && ok; ++j) {
+            int j = 0;
+            for (; j < nsteps && ok; ++j) {
                 const int sa = j % NSLOT;
-                if (!tc::bar_wait(B.a_full + 8 * sa, (j / NSLOT) & 1, abort, p.status)) { ok = false; break; }
+                if (!tc::bar_wait(B.a_full + 8 * sa, (j / NSLOT) & 1, abort, p.status, p.wait_ns)) { ok = false; break; }
                 tc::fence_after_sync();
                 const uint32_t a_tm = tmem + kACol0 + sa * SLOT_COLS;
                 for (int c0 = 0; c0 < KU && ok; c0 += XU) {
-                    if (!tc::bar_wait(B.x_full + 8 * xs, xph, abort, p.status)) { ok = false; break; }
+                    if (!tc::bar_wait(B.x_full + 8 * xs, xph, abort, p.status, p.wait_ns)) { ok = false; break; }
                     const uint32_t xb = sX + static_cast<uint32_t>(xs * XU) * xbytes;
                     for (int c2 = 0; c2 < XU; ++c2) {
                         const int c = c0 + c2;
@@ -460,21 +462,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 // are the accumulator-ready signal.
                 tc::mma_commit(j + 1 < nsteps ? B.mma_done + 8 * (j % kDoneRing) : B.acc_full);
             }
+            // Every commit's mbarrier arrival must have landed before the CTA exits: a late
+            // arrival would hit the barriers of the next CTA on this SM, which live at the
+            // same shared-memory addresses. Steps [0, committed) were committed to the
+            // mma_done ring; after an abort a final commit drains whatever is still on the
+            // tensor cores.
+            volatile int never = 0;
+            const int committed = ok ? nsteps - 1 : j;   // (the last step of a full run went to acc_full)
             if (!ok) {
-                // nothing of this thread's may still run on the tensor cores at exit
                 tc::mma_commit(B.drain + 8 * ii);
-                volatile int never = 0;
                 tc::bar_wait(B.drain + 8 * ii, 0, &never, p.status);
-            } else {
-                // every commit's mbarrier arrival must have landed before the CTA exits: a
-                // late arrival would hit the barriers of the next CTA on this SM, which
-                // live at the same shared-memory addresses
-                volatile int never = 0;
-                const int last = nsteps - 1;             // committed to acc_full (waited in the epilogue)
-                for (int c = last - kDoneRing > 0 ? last - kDoneRing : 0; c < last; ++c)
-                    tc::bar_wait(B.mma_done + 8 * (c % kDoneRing), (c / kDoneRing) & 1, &never, p.status);
-                tc::bar_wait(B.acc_full, 0, &never, p.status);
             }
+            for (int c = committed - kDoneRing > 0 ? committed - kDoneRing : 0; c < committed; ++c)
+                tc::bar_wait(B.mma_done + 8 * (c % kDoneRing), (c / kDoneRing) & 1, &never, p.status);
+            if (ok) tc::bar_wait(B.acc_full, 0, &never, p.status);
         }
         __syncwarp();
     } else if (warp >= 4) {
@@ -491,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         int s = 0;
         uint32_t cph = 0;
         for (int st = 0; st < nsteps && ok; ++st) {
-            if (!tc::bar_wait(B.codes_full + 8 * s, cph, abort, p.status)) { ok = false; break; }
+            if (!tc::bar_wait(B.codes_full + 8 * s, cph, abort, p.status, p.wait_ns)) { ok = false; break; }
             // codes of the stage (the tile was stored with the 128-byte swizzle: 16-byte
             // unit u of row r sits at unit u ^ (r % 8))
             const uint32_t crow = sC + s * CSTAGE + row * 128;
@@ -509,7 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const int sa = st % NSLOT;
             if (st >= NSLOT) {
                 const int pj = st - NSLOT;
-                if (!tc::bar_wait(B.mma_done + 8 * (pj % kDoneRing), (pj / kDoneRing) & 1, abort, p.status)) {
+                if (!tc::bar_wait(B.mma_done + 8 * (pj % kDoneRing), (pj / kDoneRing) & 1, abort, p.status,
+                                  p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -612,23 +614,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                     for (int j = 0; j < 8; ++j) tc::st_shared_f32(sX + ((col + j) * kBM + irow) * 4, v[j]);
                 }
             } else {
-                // partial tile to the workspace; the last split of the tile to arrive adds
-                // all partials in split order and finishes the tile
-                const int et = (warp - 4) * 32 + lane;
-                const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-                float* mine = p.part + (static_cast<int64_t>(tile) * p.splits + split) * p.BN * kBM;
+                // partial tile to the workspace (the ticket exchange follows below)
+                float* mine = p.part + (static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * p.splits + split) *
+                                           p.BN * kBM;
                 for (int col = cbeg; col < cend; col += 8) {
                     float v[8];
                     acc8(col, v);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) mine[(col + j) * kBM + irow] = v[j];
                 }
+            }
+        }
+        if (p.splits > 1 && !p.cluster) {
+            // Ticket: every split of the tile takes one, also a split whose main loop gave
+            // up, so that the tile's counter always returns to zero; the last split to
+            // arrive adds all partials in split order and finishes the tile (all_ok is one
+            // value for the 256 threads, so the named barriers stay uniform).
+            const int et = (warp - 4) * 32 + lane;
+            const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+            __threadfence();
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (et == 0) *last_flag = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (*last_flag) {
                 __threadfence();
-                asm volatile("bar.sync 1, 256;" ::: "memory");
-                if (et == 0) *last_flag = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
-                asm volatile("bar.sync 1, 256;" ::: "memory");
-                if (*last_flag) {
-                    __threadfence();
+                if (all_ok) {
+                    const int cbeg = ch * (p.BN / 2), cend = cbeg + p.BN / 2;
                     const float* all = p.part + static_cast<int64_t>(tile) * p.splits * p.BN * kBM;
                     for (int col = cbeg; col < cend; col += 8) {
                         float acc[8];
@@ -651,8 +662,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                         }
                         finish8(col, acc);
                     }
-                    if (et == 0) p.counters[tile] = 0;
                 }
+                if (et == 0) p.counters[tile] = 0;
             }
         }
     }
@@ -742,9 +753,7 @@ struct GemvParams {
     float qscale;
     int relu, yperm, xperm, early_w;
     int cluster;                           // K splits reduced inside a thread-block cluster
-    uint8_t* kv_codes[2];
-    uint32_t* kv_meta[2];
-    int kv_h, kv_hd, kv_nh, kv_max_seq, kv_seq, kv_pos0, kv_bits, kv_gs;
+    KvTarget kv;                           // fused store_cache, as in GemmParams
 };
 
 __device__ __forceinline__ void hmma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -807,36 +816,37 @@ __device__ __forceinline__ void gemv_finish(const GemvParams& p, int n0, int c, 
             make_uint4(pack_half2_bits(op[0], op[1]), pack_half2_bits(op[2], op[3]), pack_half2_bits(op[4], op[5]),
                        pack_half2_bits(op[6], op[7]));
     }
-    if (p.kv_codes[0] != nullptr && n0 >= p.kv_h && valid) {
+    if (p.kv.codes[0][0] != nullptr && n0 >= p.kv.h && valid) {
         // fused store_cache: the 8 values are dims [dim, dim+8) of one head; a group of gs
         // dims is the gs/8 lanes of consecutive c for this m (all 8 lanes of m are here)
         const uint4 nv = make_uint4(pack_half2_bits(o16[0], o16[1]), pack_half2_bits(o16[2], o16[3]),
                                     pack_half2_bits(o16[4], o16[5]), pack_half2_bits(o16[6], o16[7]));
-        const int sec = (n0 - p.kv_h) / p.kv_h;                 // 0 keys, 1 values
-        const int f = nb - p.kv_h - sec * p.kv_h;
-        const int head = f / p.kv_hd, dim = f % p.kv_hd;
+        const int sec = (n0 - p.kv.h) / p.kv.h;                 // 0 keys, 1 values
+        const int f = nb - p.kv.h - sec * p.kv.h;
+        const int head = f / p.kv.hd, dim = f % p.kv.hd;
         __half2 mn2, mx2;
         minmax8(nv, mn2, mx2);
         float mn = hmin_of(mn2), mx = hmax_of(mx2);
         const unsigned lanes = 0xFFu << (lane & 24);
-        const unsigned gmask = p.kv_gs == 64 ? 7u : 3u;
+        const unsigned gmask = p.kv.gs == 64 ? 7u : 3u;
         for (unsigned off = 1; off <= gmask; off <<= 1) {
             mn = fminf(mn, __shfl_xor_sync(lanes, mn, off));
             mx = fmaxf(mx, __shfl_xor_sync(lanes, mx, off));
         }
-        const int b = m / p.kv_seq, tt = m - b * p.kv_seq;
-        const int64_t slot = (static_cast<int64_t>(b) * p.kv_nh + head) * p.kv_max_seq + p.kv_pos0 + tt;
-        uint8_t* codes = p.kv_codes[sec];
-        uint32_t* meta = p.kv_meta[sec];
-        const int gph = p.kv_hd / p.kv_gs;
-        if (p.kv_bits == 4) {
+        const int c = m / p.kv.rows, r = m - c * p.kv.rows;
+        const int b = r / p.kv.seq, tt = r - b * p.kv.seq;
+        const int64_t slot = (static_cast<int64_t>(b) * p.kv.nh + head) * p.kv.max_seq + p.kv.pos0 + tt;
+        uint8_t* codes = p.kv.codes[c][sec];
+        uint32_t* meta = p.kv.meta[c][sec];
+        const int gph = p.kv.hd / p.kv.gs;
+        if (p.kv.bits == 4) {
             const __half s16 = group_scale16<4>(mn, mx);
-            *reinterpret_cast<uint32_t*>(codes + slot * (p.kv_hd / 2) + dim / 2) = quant8_4bit(nv, mn, __half2float(s16));
-            if (dim % p.kv_gs == 0) meta[slot * gph + dim / p.kv_gs] = pack_half2_bits(__float2half_rn(mn), s16);
+            *reinterpret_cast<uint32_t*>(codes + slot * (p.kv.hd / 2) + dim / 2) = quant8_4bit(nv, mn, __half2float(s16));
+            if (dim % p.kv.gs == 0) meta[slot * gph + dim / p.kv.gs] = pack_half2_bits(__float2half_rn(mn), s16);
         } else {
             const __half s16 = group_scale16<8>(mn, mx);
-            *reinterpret_cast<uint2*>(codes + slot * p.kv_hd + dim) = quant8_8bit(nv, mn, __half2float(s16));
-            if (dim % p.kv_gs == 0) meta[slot * gph + dim / p.kv_gs] = pack_half2_bits(__float2half_rn(mn), s16);
+            *reinterpret_cast<uint2*>(codes + slot * p.kv.hd + dim) = quant8_8bit(nv, mn, __half2float(s16));
+            if (dim % p.kv.gs == 0) meta[slot * gph + dim / p.kv.gs] = pack_half2_bits(__float2half_rn(mn), s16);
         }
     }
 }
@@ -1178,12 +1188,26 @@ Plan make_plan(int M, int N, int K, int bits) {
     const int nk = K / kBK;
     const int tiles = P.tiles_n * P.tiles_m;
     const int sms = sm_count();
-    int splits = 1;
-    if (tiles < sms) splits = sms / tiles;
     int max_splits = nk / kMetaChunks;
     if (max_splits > kMaxSplits) max_splits = kMaxSplits;
     if (max_splits < 1) max_splits = 1;
-    if (splits > max_splits) splits = max_splits;
+    // K splits per tile: the count whose waves of (tile, split) units take the least
+    // time, one unit costing its K steps plus a fixed overhead (prologue, pipeline fill,
+    // epilogue; more when partials must be added), so that a grid of 96 tiles on 148
+    // SMs is not left at 65% occupancy. One CTA per SM.
+    const double steps_total = static_cast<double>(nk) / (128 / (kBK * bits / 8));
+    int splits = 1;
+    double best = 0.0;
+    for (int s = 1; s <= max_splits; ++s) {
+        if (s > 1 && tiles > static_cast<int>(kTicketBytes / sizeof(int))) break;   // one ticket per tile
+        const int64_t units = static_cast<int64_t>(tiles) * s;
+        const int64_t waves = (units + sms - 1) / sms;
+        const double t = static_cast<double>(waves) * (steps_total / s + (s > 1 ? 5.0 : 3.0));
+        if (s == 1 || t < best * 0.97) {
+            best = t;
+            splits = s;
+        }
+    }
     int cps = (nk + splits - 1) / splits;
     cps = ((cps + kMetaChunks - 1) / kMetaChunks) * kMetaChunks;
     splits = (nk + cps - 1) / cps;
@@ -1336,20 +1360,7 @@ int gemv_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     gp.xperm = xperm ? 1 : 0;
     gp.early_w = early_w ? 1 : 0;
     gp.cluster = P.cluster;
-    if (kv != nullptr) {
-        gp.kv_codes[0] = static_cast<uint8_t*>(kv->cache->k_codes);
-        gp.kv_codes[1] = static_cast<uint8_t*>(kv->cache->v_codes);
-        gp.kv_meta[0] = static_cast<uint32_t*>(kv->cache->k_meta);
-        gp.kv_meta[1] = static_cast<uint32_t*>(kv->cache->v_meta);
-        gp.kv_h = kv->h;
-        gp.kv_hd = kv->cache->head_dim;
-        gp.kv_nh = kv->cache->n_heads;
-        gp.kv_max_seq = kv->cache->max_seq;
-        gp.kv_seq = kv->seq;
-        gp.kv_pos0 = kv->pos0;
-        gp.kv_bits = kv->cache->cfg.num_bits;
-        gp.kv_gs = kv->cache->cfg.group_size;
-    }
+    fill_kv_target(gp.kv, kv);
     // programmatic dependent launch, and the K splits of a tile as one cluster
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(P.tiles, P.splits);
@@ -1419,6 +1430,7 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != FLEX_OK) return rc;
     GemmParams gp{};
+    gp.wait_ns = pipeline_wait_ns();
     gp.bias = static_cast<const __half*>(bias);
     gp.residual = static_cast<const __half*>(residual);
     gp.y = static_cast<__half*>(y);
@@ -1447,20 +1459,7 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     gp.off_m = P.off_m;
     gp.off_bar = P.off_bar;
     gp.tmem_cols = P.tmem_cols;
-    if (kv != nullptr) {
-        gp.kv_codes[0] = static_cast<uint8_t*>(kv->cache->k_codes);
-        gp.kv_codes[1] = static_cast<uint8_t*>(kv->cache->v_codes);
-        gp.kv_meta[0] = static_cast<uint32_t*>(kv->cache->k_meta);
-        gp.kv_meta[1] = static_cast<uint32_t*>(kv->cache->v_meta);
-        gp.kv_h = kv->h;
-        gp.kv_hd = kv->cache->head_dim;
-        gp.kv_nh = kv->cache->n_heads;
-        gp.kv_max_seq = kv->cache->max_seq;
-        gp.kv_seq = kv->seq;
-        gp.kv_pos0 = kv->pos0;
-        gp.kv_bits = kv->cache->cfg.num_bits;
-        gp.kv_gs = kv->cache->cfg.group_size;
-    }
+    fill_kv_target(gp.kv, kv);
     const dim3 grid(P.tiles_n, P.tiles_m, P.splits);
     // programmatic dependent launch, and the K splits of a tile as one cluster
     cudaLaunchConfig_t cfg = {};

@@ -203,6 +203,7 @@ int validate_cache(const flex_kv_cache* c) {
     FLEX_REQUIRE(aligned16(c->k_codes) && aligned16(c->v_codes) && aligned16(c->k_meta) &&
                      aligned16(c->v_meta),
                  FLEX_ERR_ALIGN);
+    FLEX_REQUIRE(c->valid_from == nullptr || (reinterpret_cast<uintptr_t>(c->valid_from) & 3u) == 0, FLEX_ERR_ALIGN);
     return FLEX_OK;
 }
 

@@ -25,7 +25,7 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
                        bool early_kv);
 int64_t decode_attn_ws_bound(int pairs, int head_dim);
 int prefill_attn_launch(const void* q, const void* k, const void* v, int64_t row_stride, void* o, int batch,
-                        int seq, int n_heads, int head_dim, cudaStream_t st);
+                        int seq, int n_heads, int head_dim, const int32_t* valid_from, cudaStream_t st);
 int64_t gemm_ws_bytes(int M, int N, int K, int bits);
 int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const void* residual, void* y, int M,
                 int relu, int nq, float qscale, bool xperm, bool yperm, void* ws, int64_t ws_bytes, cudaStream_t st,
@@ -91,20 +91,26 @@ WsLayout layout(const flex_layer* L, int batch, int seq) {
     return w;
 }
 
-int run_layer(const flex_layer* L, const flex_kv_cache* C, const void* x_in, void* x_out, int batch, int seq, int pos,
-              void* ws, int64_t ws_bytes, cudaStream_t st) {
-    const WsLayout w = layout(L, batch, seq);
+// One layer call over `nc` gpu-batches of `batch` sequences each, gpu-batch c with its
+// own cache C[c]: the LayerNorms and the four weight GEMMs run once over all nc * batch
+// * seq activation rows (each weight is streamed once for all gpu-batches), attention
+// runs per gpu-batch on its own cache, and the QKV epilogue stores every row's key and
+// value into its gpu-batch's cache.
+int run_layer(const flex_layer* L, const flex_kv_cache* C, int nc, const void* x_in, void* x_out, int batch, int seq,
+              int pos, void* ws, int64_t ws_bytes, cudaStream_t st) {
+    const WsLayout w = layout(L, nc * batch, seq);
     FLEX_REQUIRE(ws != nullptr && ws_bytes >= w.total, FLEX_ERR_WORKSPACE);
     FLEX_REQUIRE(aligned16(ws), FLEX_ERR_ALIGN);
     char* base = static_cast<char*>(ws);
     void* a = base + w.a;
     __half* qkv = reinterpret_cast<__half*>(base + w.qkv);
-    void* o = base + w.o;
+    __half* o = reinterpret_cast<__half*>(base + w.o);
     void* h1 = base + w.h1;
     void* a2 = base + w.a2;
     void* f = base + w.f;
     void* gws = base + w.gemm;
-    const int64_t T = static_cast<int64_t>(batch) * seq;
+    const int64_t T = static_cast<int64_t>(nc) * batch * seq;
+    const int64_t Tc = static_cast<int64_t>(batch) * seq;      // rows of one gpu-batch
     const int M = static_cast<int>(T);
     const int h = L->h;
     const float qscale = 1.0f / sqrtf(static_cast<float>(L->head_dim));
@@ -114,15 +120,19 @@ int run_layer(const flex_layer* L, const flex_kv_cache* C, const void* x_in, voi
     const bool dec = (seq == 1);
     // the QKV epilogue also quantises the new keys/values into their cache slots
     // (store_cache): slot pos for a decode step, slots [0, seq) for a prompt
-    const KvFuse kv{C, h, seq, dec ? pos : 0};
+    const KvFuse kv{C, nc, static_cast<int>(Tc), h, seq, dec ? pos : 0};
     int rc = layernorm_launch(x_in, L->ln1_g, L->ln1_b, a, T, h, true, st);
     if (rc == FLEX_OK)
         rc = gemm_launch(a, &L->w_qkv, L->b_qkv, nullptr, qkv, M, 0, h, qscale, true, false, gws, w.gemm_bytes, st, &kv, true);
-    if (rc != FLEX_OK) return rc;
-    if (dec)
-        rc = decode_attn_launch(C, qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, pos, base + w.attn, true, st, true);
-    else
-        rc = prefill_attn_launch(qkv, qkv + h, qkv + 2 * h, 3LL * h, o, batch, seq, L->n_heads, L->head_dim, st);
+    for (int c = 0; c < nc && rc == FLEX_OK; ++c) {
+        const __half* qc = qkv + c * Tc * 3 * h;
+        __half* oc = o + c * Tc * h;
+        if (dec)
+            rc = decode_attn_launch(&C[c], qc, qc + h, qc + 2 * h, 3LL * h, oc, batch, pos, base + w.attn, true, st, true);
+        else
+            rc = prefill_attn_launch(qc, qc + h, qc + 2 * h, 3LL * h, oc, batch, seq, L->n_heads, L->head_dim,
+                                     C[c].valid_from, st);
+    }
     if (rc == FLEX_OK)
         rc = gemm_launch(o, &L->w_o, L->b_o, x_in, h1, M, 0, 0, 1.f, dec, false, gws, w.gemm_bytes, st, nullptr, true);
     if (rc == FLEX_OK) rc = layernorm_launch(h1, L->ln2_g, L->ln2_b, a2, T, h, true, st);
@@ -140,6 +150,43 @@ int check_cache_for_layer(const flex_layer* L, const flex_kv_cache* C) {
     return FLEX_OK;
 }
 
+// Every cache valid for the layer and of the same geometry as the first; batch fits.
+int check_caches(const flex_layer* L, const flex_kv_cache* C, int nc, int batch, bool exact_batch) {
+    FLEX_REQUIRE(C != nullptr && nc >= 1 && nc <= kMaxKvBatches, FLEX_ERR_INVALID_ARG);
+    for (int c = 0; c < nc; ++c) {
+        const int rc = check_cache_for_layer(L, &C[c]);
+        if (rc != FLEX_OK) return rc;
+        FLEX_REQUIRE(C[c].max_seq == C[0].max_seq && C[c].cfg.num_bits == C[0].cfg.num_bits &&
+                         C[c].cfg.group_size == C[0].cfg.group_size,
+                     FLEX_ERR_SHAPE);
+        FLEX_REQUIRE(batch > 0 && (exact_batch ? batch == C[c].batch : batch <= C[c].batch), FLEX_ERR_INVALID_ARG);
+    }
+    return FLEX_OK;
+}
+
+int prefill(const flex_layer* L, const flex_kv_cache* C, int nc, const void* x_in, void* x_out, int32_t batch,
+            int32_t seq, void* ws, int64_t ws_bytes, void* stream) {
+    int rc = validate_layer(L);
+    if (rc == FLEX_OK) rc = check_caches(L, C, nc, batch, true);
+    if (rc != FLEX_OK) return rc;
+    FLEX_REQUIRE(x_in && x_out && x_in != x_out, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(aligned16(x_in) && aligned16(x_out), FLEX_ERR_ALIGN);
+    FLEX_REQUIRE(seq > 0 && seq <= C[0].max_seq, FLEX_ERR_SHAPE);
+    FLEX_REQUIRE(static_cast<int64_t>(nc) * batch * seq < (1LL << 31), FLEX_ERR_SHAPE);
+    return run_layer(L, C, nc, x_in, x_out, batch, seq, 0, ws, ws_bytes, as_stream(stream));
+}
+
+int decode(const flex_layer* L, const flex_kv_cache* C, int nc, const void* x_in, void* x_out, int32_t batch,
+           int32_t pos, void* ws, int64_t ws_bytes, void* stream) {
+    int rc = validate_layer(L);
+    if (rc == FLEX_OK) rc = check_caches(L, C, nc, batch, false);
+    if (rc != FLEX_OK) return rc;
+    FLEX_REQUIRE(x_in && x_out && x_in != x_out, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(aligned16(x_in) && aligned16(x_out), FLEX_ERR_ALIGN);
+    FLEX_REQUIRE(pos >= 0 && pos < C[0].max_seq, FLEX_ERR_SHAPE);
+    return run_layer(L, C, nc, x_in, x_out, batch, 1, pos, ws, ws_bytes, as_stream(stream));
+}
+
 }  // namespace
 }  // namespace flexq
 
@@ -155,24 +202,22 @@ extern "C" int64_t flex_workspace_bytes(const flex_layer* L, int32_t batch, int3
 
 extern "C" int flex_prefill_layer(const flex_layer* L, const flex_kv_cache* cache, const void* x_in, void* x_out,
                                   int32_t batch, int32_t seq, void* ws, int64_t ws_bytes, void* stream) {
-    int rc = validate_layer(L);
-    if (rc == FLEX_OK) rc = check_cache_for_layer(L, cache);
-    if (rc != FLEX_OK) return rc;
-    FLEX_REQUIRE(x_in && x_out && x_in != x_out, FLEX_ERR_INVALID_ARG);
-    FLEX_REQUIRE(aligned16(x_in) && aligned16(x_out), FLEX_ERR_ALIGN);
-    FLEX_REQUIRE(batch > 0 && batch == cache->batch, FLEX_ERR_INVALID_ARG);
-    FLEX_REQUIRE(seq > 0 && seq <= cache->max_seq, FLEX_ERR_SHAPE);
-    return run_layer(L, cache, x_in, x_out, batch, seq, 0, ws, ws_bytes, as_stream(stream));
+    return prefill(L, cache, 1, x_in, x_out, batch, seq, ws, ws_bytes, stream);
 }
 
 extern "C" int flex_decode_layer(const flex_layer* L, const flex_kv_cache* cache, const void* x_in, void* x_out,
                                  int32_t batch, int32_t pos, void* ws, int64_t ws_bytes, void* stream) {
-    int rc = validate_layer(L);
-    if (rc == FLEX_OK) rc = check_cache_for_layer(L, cache);
-    if (rc != FLEX_OK) return rc;
-    FLEX_REQUIRE(x_in && x_out && x_in != x_out, FLEX_ERR_INVALID_ARG);
-    FLEX_REQUIRE(aligned16(x_in) && aligned16(x_out), FLEX_ERR_ALIGN);
-    FLEX_REQUIRE(batch > 0 && batch <= cache->batch, FLEX_ERR_INVALID_ARG);
-    FLEX_REQUIRE(pos >= 0 && pos < cache->max_seq, FLEX_ERR_SHAPE);
-    return run_layer(L, cache, x_in, x_out, batch, 1, pos, ws, ws_bytes, as_stream(stream));
+    return decode(L, cache, 1, x_in, x_out, batch, pos, ws, ws_bytes, stream);
+}
+
+extern "C" int flex_prefill_layer_batches(const flex_layer* L, const flex_kv_cache* caches, int32_t num_batches,
+                                          const void* x_in, void* x_out, int32_t batch, int32_t seq, void* ws,
+                                          int64_t ws_bytes, void* stream) {
+    return prefill(L, caches, num_batches, x_in, x_out, batch, seq, ws, ws_bytes, stream);
+}
+
+extern "C" int flex_decode_layer_batches(const flex_layer* L, const flex_kv_cache* caches, int32_t num_batches,
+                                         const void* x_in, void* x_out, int32_t batch, int32_t pos, void* ws,
+                                         int64_t ws_bytes, void* stream) {
+    return decode(L, caches, num_batches, x_in, x_out, batch, pos, ws, ws_bytes, stream);
 }

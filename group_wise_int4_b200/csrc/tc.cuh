@@ -31,14 +31,14 @@ __device__ __forceinline__ void bar_arrive_expect_tx(uint32_t bar, uint32_t byte
 // until the phase completes instead of spinning and taking issue slots from the
 // warps that do the work.
 constexpr uint32_t kSuspendHintNs = 200000;
-__device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns = kSuspendHintNs) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
@@ -52,20 +52,23 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // try_wait loop (each try_wait sleeps until the phase completes or the hint runs out);
 // every 16 polls it checks *abort (raised by another role of the CTA) and the elapsed
 // time.
-// After kWaitLimitNs it records FLEX_ERR_TIMEOUT in the device status word, raises
-// *abort and returns false.
+// After limit_ns (kWaitLimitNs unless the caller passes a limit) it records
+// FLEX_ERR_TIMEOUT in the device status word, raises *abort and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
-    if (bar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                         uint64_t limit_ns = kWaitLimitNs) {
+    // the sleep of one poll stays well below the limit (16 polls between time checks)
+    const uint32_t hint = limit_ns >= 64ull * kSuspendHintNs ? kSuspendHintNs : static_cast<uint32_t>(limit_ns / 64);
+    if (bar_try_wait(bar, parity, hint)) return true;
     uint64_t t0 = 0;
     for (uint32_t n = 1;; ++n) {
-        if (bar_try_wait(bar, parity)) return true;
+        if (bar_try_wait(bar, parity, hint)) return true;
         if ((n & 15u) == 0) {
             if (*abort) return false;
             const uint64_t t = globaltimer_ns();
             if (t0 == 0) {
                 t0 = t;
-            } else if (t - t0 > kWaitLimitNs) {
+            } else if (t - t0 > limit_ns) {
                 *abort = 1;
                 set_status(status, FLEX_ERR_TIMEOUT);
                 return false;

@@ -16,8 +16,9 @@
  *   - All tensor pointers are DEVICE pointers (cudaMalloc / torch CUDA memory) unless
  *     a parameter says otherwise. The caller owns and allocates every buffer:
  *     inputs, outputs, codes, metadata, caches and workspaces. The library keeps no
- *     per-call state; its only global state is one device status word per device,
- *     created on first use (see flex_get_status).
+ *     per-call state; its global state is one device status word per device, created
+ *     on first use (see flex_get_status), the wait limit of flex_set_wait_limit_ns, and
+ *     the scratch buffer of flex_decode_attention_noalloc.
  *   - fp16 means IEEE binary16, "half2" a pair of binary16 stored as 4 bytes.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Every call only enqueues work on `stream` and returns; none synchronises,
@@ -114,11 +115,21 @@ typedef struct {
 /* Compressed KV cache of one layer (section 6.3: KV grouped along the head dim).
  *   k_codes, v_codes: uint8 [batch][n_heads][max_seq][head_dim*bits/8]
  *   k_meta,  v_meta : half2 [batch][n_heads][max_seq][head_dim/group_size]
- *   cfg: num_bits 4 or 8, group_size 32/64 (dividing head_dim), group_dim = 3.   */
+ *   cfg: num_bits 4 or 8, group_size 32/64 (dividing head_dim), group_dim = 3.
+ *   valid_from: NULL, or a device int32 [batch] (4-byte aligned): prompts padded on the
+ *     left to a common length (the source-notes page «FlexGen» (PtirisNote), "Flex Opt":
+ *     the attention_mask buffer of the generation loop; the walkthrough page, section
+ *     3.1: HELM prompts padded to pad_to_seq_len). Sequence b's real tokens start at
+ *     slot valid_from[b]: no query attends to a slot below it, and a query that is
+ *     itself a pad token (prefill rows below it) gets a zero attention output. The
+ *     pad tokens still run through the layer and are stored in the cache. NULL (or
+ *     zeros) = no padding. Read by the kernels at run time, so it may change between
+ *     replays of a captured graph.                                                  */
 typedef struct {
     void *k_codes, *k_meta, *v_codes, *v_meta;
     int32_t batch, n_heads, head_dim, max_seq;
     flexq_config cfg;
+    const int32_t* valid_from;
 } flex_kv_cache;
 
 /* Workspace bytes that flex_prefill_layer (seq > 1) or flex_decode_layer (seq == 1)
@@ -146,6 +157,25 @@ int flex_decode_layer(const flex_layer* L, const flex_kv_cache* cache, const voi
                       void* x_out, int32_t batch, int32_t pos, void* ws, int64_t ws_bytes,
                       void* stream);
 
+/* Several gpu-batches through one layer with one pass over its weights (the walkthrough
+ * page, sections 2.3 and 6.1: gpu_batch_size x num_gpu_batches, e.g. 48 x 3, where one
+ * weight load serves every gpu-batch of the block; the source-notes page «FlexGen»
+ * (PtirisNote), "Flex Opt": the loop over gpu-batches inside each layer).
+ *   caches: num_batches caches (1..8) of identical geometry, cache c holding gpu-batch c.
+ *   x_in, x_out: fp16 [num_batches][batch][seq][h] (prefill) or [num_batches][batch][h]
+ *   (decode), gpu-batch c at rows [c*batch*seq, (c+1)*batch*seq).
+ *   The LayerNorms and the four weight GEMMs run once over all num_batches * batch * seq
+ *   rows; attention runs per gpu-batch on its own cache; each row's key/value go to its
+ *   gpu-batch's cache. Results equal num_batches separate calls up to summation order.
+ *   ws: flex_workspace_bytes(L, num_batches * batch, seq) bytes. Prefill needs
+ *   batch == every cache's batch; decode batch <= every cache's batch. */
+int flex_prefill_layer_batches(const flex_layer* L, const flex_kv_cache* caches, int32_t num_batches,
+                               const void* x_in, void* x_out, int32_t batch, int32_t seq, void* ws,
+                               int64_t ws_bytes, void* stream);
+int flex_decode_layer_batches(const flex_layer* L, const flex_kv_cache* caches, int32_t num_batches,
+                              const void* x_in, void* x_out, int32_t batch, int32_t pos, void* ws,
+                              int64_t ws_bytes, void* stream);
+
 /* ---- hot-path steps, callable one by one ------------------------------------- */
 
 /* store_cache: quantise k_new / v_new (fp16 [batch][n_heads][head_dim], rows of
@@ -156,8 +186,9 @@ int flex_append_kv(const flex_kv_cache* cache, const void* k_new, const void* v_
                    int64_t row_stride, int32_t batch, int32_t pos, void* stream);
 
 /* Decode attention (`mha_gen` core): per sequence b < batch and head:
- *   o = softmax([q.k_0 .. q.k_{pos-1}, q.k_new]) [v_0 .. v_{pos-1}, v_new]
- * with k_j, v_j the dequantised cache slots [0, pos). q, k_new, v_new: fp16 rows of
+ *   o = softmax([q.k_vf .. q.k_{pos-1}, q.k_new]) [v_vf .. v_{pos-1}, v_new]
+ * with k_j, v_j the dequantised cache slots [vf, pos), vf = cache->valid_from[b]
+ * (0 without padding; clamped to [0, pos]). q, k_new, v_new: fp16 rows of
  * `row_stride` elements per sequence, head h at offset h*head_dim (q is used as
  * given: callers pre-scale it). o: fp16 [batch][n_heads*head_dim].
  * ws: at least flex_decode_attention_ws_bytes(cache, batch, pos) bytes. */
@@ -180,7 +211,10 @@ int flex_decode_attention(const flex_kv_cache* cache, const void* q, const void*
  *   - Set-up: the first call on a device, made with that device current, looks up the
  *     buffer's device address with a CUDA runtime query (with lazy module loading the
  *     driver may load the library's device code, buffer included, at that moment);
- *     make that first call before any stream capture begins on the device.
+ *     make that first call before any stream capture begins on the device. The address
+ *     is kept for the life of the process: after cudaDeviceReset (or anything else that
+ *     destroys the device's primary context) it no longer names the buffer, and this
+ *     entry point must not be called again in that process.
  *   - Nothing in the buffer has to start at zero: each call writes every partial it
  *     reads.
  *   - One buffer per device, shared by all calls: two calls on one device that may run
@@ -194,10 +228,12 @@ int flex_decode_attention_noalloc(const flex_kv_cache* cache, const void* q, con
 /* Prefill attention (`mha` core): causal softmax attention on fresh fp16 q, k, v,
  * each [batch][seq][n_heads][head_dim] inside rows of `row_stride` elements per
  * token (token t of sequence b at (b*seq + t)*row_stride). o: fp16
- * [batch][seq][n_heads*head_dim]. head_dim 64 or 128. */
+ * [batch][seq][n_heads*head_dim]. head_dim 64 or 128. valid_from: NULL or a device
+ * int32 [batch] of left-padding starts, as in flex_kv_cache (keys below it are not
+ * attended; rows below it get zeros). */
 int flex_prefill_attention(const void* q, const void* k, const void* v, int64_t row_stride,
                            void* o, int32_t batch, int32_t seq, int32_t n_heads,
-                           int32_t head_dim, void* stream);
+                           int32_t head_dim, const int32_t* valid_from, void* stream);
 
 /* Dequant-fused weight GEMM: y[m][n] = epi( sum_k x[m][k] * W^[n][k] + bias[n] )
  *   x fp16 [M][K] row-major, W compressed [N][K] (group 64 along K, 4 or 8 bits),
@@ -229,8 +265,26 @@ int flex_layernorm(const void* x, const void* g, const void* b, void* y, int64_t
 
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: FLEX_OK, or FLEX_ERR_TIMEOUT if a kernel's bounded wait gave up
- * since the last call, or FLEX_ERR_CUDA if the stream reports an error. */
+ * since the last call, or FLEX_ERR_CUDA if the stream reports an error. The word's
+ * device address is looked up once per device and kept for the life of the process,
+ * so the library must not be used on a device after cudaDeviceReset (or any other
+ * destruction of its primary context) in the same process. */
 int flex_get_status(void* stream);
+
+/* Failure detection: limit, in nanoseconds, after which a wait inside the pipeline of
+ * the tensor-core GEMM kernel (operand stages, dequantised tiles, MMA completion) gives
+ * up. The kernel then records FLEX_ERR_TIMEOUT (read by flex_get_status), stops, lets
+ * every copy and MMA it issued finish (those drain waits keep the default limit), and
+ * exits; its outputs are unspecified, and the device stays usable. Applies to kernels
+ * launched after the call (a captured CUDA graph keeps the limit of its capture time);
+ * process-wide. ns = 0 restores the default of 2 s. Returns the previous limit. */
+uint64_t flex_set_wait_limit_ns(uint64_t ns);
+
+/* Layout of the ABI structs as this library was compiled: which = 0 flexq_config,
+ * 1 flexq_tensor, 2 flex_layer, 3 flex_kv_cache; field = -1 returns sizeof, field = i
+ * the byte offset of the struct's i-th field (declaration order). -1 if out of range.
+ * Bindings compare these with their own declarations before any call. */
+int64_t flex_abi_layout(int32_t which, int32_t field);
 
 /* Static English text for a status code. */
 const char* flex_status_string(int32_t status);

@@ -103,3 +103,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(fq, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="missing"):
         fq.lib()
+
+
+def test_struct_layouts_match_the_library():
+    """The binding's ctypes structs have the library's sizes and field offsets."""
+    L = fq.lib()
+    fq._check_layout(L)
+    assert int(L.flex_abi_layout(3, -1)) == ctypes.sizeof(fq.flex_kv_cache)
+    assert int(L.flex_abi_layout(9, -1)) == -1
+
+
+def test_layout_mismatch_is_refused(monkeypatch):
+    """A binding struct that lacks a field the library has (here flex_kv_cache without
+    valid_from) is refused before any call could pass it to the library."""
+    class short_cache(ctypes.Structure):
+        _fields_ = [f for f in fq.flex_kv_cache._fields_ if f[0] != "valid_from"]
+    monkeypatch.setattr(fq, "_STRUCTS", (fq.flexq_config, fq.flexq_tensor, fq.flex_layer, short_cache))
+    with pytest.raises(RuntimeError, match="layout"):
+        fq._check_layout(fq.lib())

@@ -2,20 +2,24 @@
 """Benchmark of the flexq hot path on B200.
 
 Metric: decode tokens/s per OPT layer-step (and int4 compress/decompress GB/s), as a
-fraction of the HBM roofline.
+fraction of the roofline.
 
-Default workload (``opt-1.3b``): OPT-1.3B-shaped decoder layers (h 2048, 32 heads x 64,
-FFN 8192), a stack of 24 distinct layers with their own weights and int4 KV caches,
-batch 32, prompt 512 then 32 decode steps; weights int4 group 64, KV int4 group 64,
-seeded synthetic data. The prompt is prefilled once (setup); one benchmark *step*
-is the whole decode phase of that workload - 32 new tokens for the 32 sequences
-through the 24-layer stack (positions 512..543), i.e. 24,576 layer-tokens, replayed
-from CUDA graphs. The stack touches ~1.6 GB per token step, more than L2, so no
-flush is needed between steps.
+Default workload (``opt-175b``): OPT-175B-shaped decoder layers (h 12288, 96 heads x
+128, FFN 49152), 4 distinct layers with their own int4 weights and int4 KV caches
+(about 2 GB per layer, so nothing stays in the 126 MB L2), batch 144, prompt 512 then
+32 decode steps; weights int4 group 64, KV int4 group 64, seeded synthetic data. The
+prompt is prefilled once (setup); one benchmark *step* is the whole decode phase - 32
+new tokens for the 144 sequences through the 4 layers (positions 512..543), i.e.
+18,432 layer-tokens, replayed from CUDA graphs.
 
-Also measured in the same run (``parts``): the prefill of the prompt through the
-stack, the codec on a 1 GiB tensor, and every kernel of the decode step timed on its
-own in the launch configuration the step uses (this gives the roofline object).
+``--workload opt-30b`` runs the 3 x 48 schedule of that shape (three gpu-batches of 48
+sequences, each with its own caches, one layer call per gpu-batch), ``opt-1.3b`` a
+24-layer stack at batch 32, ``opt-125m`` one layer at batch 4.
+
+Also measured in the same run (``parts``): every kernel of the decode step timed on its
+own in the launch configuration the step uses (this gives the roofline object), the
+prefill of the prompt, the opt-30b 3 x 48 schedule (default run only) and the codec at
+1 GiB. ``--codec-only`` runs the whole compress/decompress sweep instead.
 
 ``--impl reference`` times the CPU oracle (the only other implementation; there is no
 installable reference) on a bounded sample of the same workload.
@@ -38,20 +42,26 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode tokens/s per OPT layer-step"
 UNIT = "layer-tokens/s"
+WORKLOADS = ["opt-125m", "opt-1.3b", "opt-30b", "opt-175b"]
+KERNELS = ["gemm_qkv", "gemm_out", "gemm_fc1", "gemm_fc2", "decode_attention", "layernorm", "decode_layer",
+           "prefill_layer", "compress", "decompress"]
 
 
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="flexq", choices=["flexq", "reference"])
-    ap.add_argument("--workload", default="opt-1.3b", choices=["opt-125m", "opt-1.3b", "opt-30b", "opt-175b"])
+    ap.add_argument("--workload", default="opt-175b", choices=WORKLOADS)
     ap.add_argument("--layers", type=int, default=None, help="stack depth (default: per workload)")
     ap.add_argument("--no-parts", action="store_true", help="skip the per-part measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--codec-only", action="store_true",
-                    help="measure only flexq_compress / flexq_decompress on 1 GiB and print them as one JSON line")
+                    help="measure only flexq_compress / flexq_decompress over the sweep (one JSON line)")
+    ap.add_argument("--kernel", default=None, choices=KERNELS,
+                    help="run only this step, 3 times, at the workload's decode shape on one layer "
+                         "(a small case for ncu captures); prints one JSON line")
     return ap.parse_args()
 
 
@@ -147,40 +157,195 @@ def whole_job_value(world, units_per_step, steps, ms):
     return world * units_per_step * steps / (ms / 1e3)
 
 
-def bench_config(args, cfg, world):
-    L, b, s, nsteps = cfg["layers"], cfg["batch"], cfg["prompt"], cfg["decode_steps"]
-    return {"workload": f"{args.workload} decode: {L} distinct layers, batch {b}, prompt {s}, "
-                        f"{nsteps} decode steps (positions {s}..{s + nsteps - 1}), int4 g64 weights and KV",
-            "batch": b, "prompt": s, "decode_steps": nsteps, "layers": L, "h": cfg["h"],
-            "units_per_step": b * nsteps * L,
-            "l2": "not flushed: each token step streams ~%.1f GB (> 126 MB L2)" %
-                  (decode_bytes_per_layer_step(cfg, s) * L / 1e9),
-            "parallelism": f"replicas x{world}"}
-
-
 def workload_cfg(name, layers=None):
     import synth
     cfg = dict(synth.WORKLOADS[name])
     if layers is not None:
         cfg["layers"] = layers
+    cfg["name"] = name
+    cfg["call_batch"] = cfg.get("gpu_batch", cfg["batch"])       # sequences per layer call
+    cfg["calls"] = cfg["batch"] // cfg["call_batch"]              # layer calls per layer-step
     return cfg
 
 
-def decode_bytes_per_layer_step(cfg, pos, bits=4):
-    """Algorithmic HBM bytes of one decode layer-step at position pos (int4 g64):
-    weights 12h^2*0.5625, KV read 2*b*pos*h*0.5625, KV write 2*b*h*0.5625,
-    activations in/out 4*b*h, biases and LayerNorm ~(9h + ffn)*2."""
+def bench_config(cfg, world):
+    L, b, s, nsteps = cfg["layers"], cfg["batch"], cfg["prompt"], cfg["decode_steps"]
+    sched = (f"{cfg['calls']} gpu-batches of {cfg['call_batch']}, each with its own caches, sharing one pass over "
+             f"each layer's weights (flex_decode_layer_batches)" if cfg["calls"] > 1
+             else f"batch {b} in one layer call")
+    return {"workload": f"{cfg['name']} decode: {L} distinct layers (own int4 weights and KV caches), {sched}, "
+                        f"prompt {s}, {nsteps} decode steps (positions {s}..{s + nsteps - 1}), int4 g64 weights "
+                        f"and KV",
+            "h": cfg["h"], "heads": cfg["n_heads"], "head_dim": cfg["head_dim"], "ffn": cfg["ffn"],
+            "batch": b, "call_batch": cfg["call_batch"], "prompt": s, "decode_steps": nsteps, "layers": L,
+            "units_per_step": b * nsteps * L,
+            "l2": "not flushed: each token step streams ~%.2f GB (> 126 MB L2)" %
+                  (step_cost(cfg, s, 1.0, 1.0)["bytes"] * L / 1e9),
+            "parallelism": f"replicas x{world}"}
+
+
+def step_cost(cfg, pos, hbm_gbs, tflops, bits=4):
+    """Algorithmic cost of one decode layer-step at position pos (int4 g64) for all the
+    step's sequences (with several gpu-batches the weights are streamed once for all of
+    them): bytes (weights 12h^2*0.5625, KV read 2*b*pos*h*0.5625, KV write 2*b*h*0.5625,
+    q/k/v in and o out 8*b*h, activations of the GEMMs and LayerNorms, biases and
+    LayerNorm ~(9h + ffn)*2), flops (weight GEMMs 2*b*(4h^2 + 2h*ffn), attention
+    4*b*(pos+1)*h), and two bounds: pure HBM (bytes / bandwidth) and attainable (per
+    kernel the larger of bytes / bandwidth and flops / tensor peak, summed)."""
     h, ffn, b = cfg["h"], cfg["ffn"], cfg["batch"]
     per = 0.5 + 4 / 64 if bits == 4 else 1 + 4 / 64
-    w = (3 * h * h + h * h + 2 * h * ffn) * per
-    kv = 2 * b * pos * h * per + 2 * b * h * per
-    act = 4 * b * h
-    small = (9 * h + ffn) * 2
-    return w + kv + act + small
+    bw, pk = hbm_gbs * 1e9, tflops * 1e12
+    tot_bytes = tot_flops = attain = 0.0
+    for n, k in ((3 * h, h), (h, h), (ffn, h), (h, ffn)):
+        by = n * k * per + b * k * 2 + b * n * 2
+        fl = 2.0 * b * n * k
+        tot_bytes += by
+        tot_flops += fl
+        attain += max(by / bw, fl / pk)
+    kv = 2 * b * pos * h * per + 2 * b * h * per + 4 * b * h * 2      # + q, k, v in, o out
+    small = (9 * h + ffn) * 2 + 2 * (2 * b * h * 2)                 # params, two LayerNorms
+    tot_bytes += kv + small
+    tot_flops += 4.0 * b * (pos + 1) * h
+    attain += (kv + small) / bw
+    return {"bytes": tot_bytes, "flops": tot_flops, "hbm_s": tot_bytes / bw, "attainable_s": attain}
+
+
+# ---------------------------------------------------------------------------------
+def graph_kernel_counts(g):
+    """{kernel name: launches} of a captured CUDA graph (its kernel nodes), read back
+    through the CUDA driver API; None if the graph cannot be inspected. A node whose
+    name cannot be read is counted under "?"."""
+    try:
+        from cuda.bindings import driver as cd
+        ok = cd.CUresult.CUDA_SUCCESS
+        graph = cd.CUgraph(init_value=int(g.raw_cuda_graph()))
+        err, _, n = cd.cuGraphGetNodes(graph, 0)
+        if err != ok:
+            return None
+        err, nodes, n = cd.cuGraphGetNodes(graph, n)
+        if err != ok:
+            return None
+        counts = {}
+        for node in nodes[:n]:
+            err, t = cd.cuGraphNodeGetType(node)
+            if err != ok or t != cd.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL:
+                continue
+            name = "?"
+            err, prm = cd.cuGraphKernelNodeGetParams(node)
+            if err == ok:
+                for getter, handle in ((getattr(cd, "cuFuncGetName", None), getattr(prm, "func", None)),
+                                       (getattr(cd, "cuKernelGetName", None), getattr(prm, "kern", None))):
+                    if getter is None or handle is None or int(handle) == 0:
+                        continue
+                    e2, nm = getter(handle)
+                    if e2 == ok and nm:
+                        name = nm.decode() if isinstance(nm, bytes) else str(nm)
+                        break
+            counts[name] = counts.get(name, 0) + 1
+        return counts
+    except Exception:
+        return None
+
+
+def short_kernel_name(name):
+    """Kernel name without namespace, template arguments or parameters, from a plain
+    ('void flexq::(anonymous namespace)::gemm_tc_kernel<4, true>(...)') or a mangled
+    ('_ZN5flexq..14gemm_tc_kernelILi4ELb1EEEv...') name."""
+    import re
+    if name.startswith("_Z"):                 # mangled: length-prefixed identifiers
+        i, found = 0, None
+        while i < len(name):
+            m = re.match(r"\d+", name[i:])
+            if m:
+                n = int(m.group(0))
+                ident = name[i + len(m.group(0)):i + len(m.group(0)) + n]
+                if ident.endswith("_kernel"):
+                    found = ident
+                i += len(m.group(0)) + (n if len(ident) == n else 0)
+            else:
+                i += 1
+        if found:
+            return found
+    m = re.search(r"([A-Za-z0-9_]*_kernel)\b", name)
+    return m.group(1) if m else name.split("(")[0].split("<")[0].split("::")[-1].strip()
+
+
+class Stack:
+    """L distinct layers of one workload on the device, each with its own compressed
+    weights and, per gpu-batch, its own int4 KV cache; prefilled with the prompt."""
+
+    def __init__(self, fq, torch, synth, cfg, dev):
+        L, b, s, h = cfg["layers"], cfg["call_batch"], cfg["prompt"], cfg["h"]
+        nh, d = cfg["n_heads"], cfg["head_dim"]
+        self.fq, self.torch, self.cfg, self.dev = fq, torch, cfg, dev
+        self.max_seq = s + cfg["decode_steps"]
+        self.layers, self.caches = [], []
+        for l in range(L):
+            raw = synth.layer_params(h, cfg["ffn"], cfg["seed"] * 100 + l, device=dev)
+            self.layers.append(fq.FlexLayer(raw, nh, device=dev))
+            del raw
+            self.caches.append([fq.FlexKVCache(b, nh, d, self.max_seq, device=dev) for _ in range(cfg["calls"])])
+        torch.cuda.synchronize()
+        nc = cfg["calls"]
+        self.ws_pre = torch.zeros(fq.flex_workspace_bytes(self.layers[0], nc * b, s), dtype=torch.uint8, device=dev)
+        self.x_pre = synth.activations((nc, b, s, h), cfg["seed"] * 10, device=dev)
+        self.y_pre = torch.empty_like(self.x_pre)
+        self.ws_dec = torch.zeros(fq.flex_workspace_bytes(self.layers[0], nc * b, 1), dtype=torch.uint8, device=dev)
+
+    def prefill(self):
+        """Prompt of every gpu-batch through the stack (writes cache slots [0, prompt));
+        several gpu-batches share one pass over each layer's weights."""
+        fq, cfg = self.fq, self.cfg
+        src, dst = self.x_pre, self.y_pre
+        for l in range(cfg["layers"]):
+            if cfg["calls"] == 1:
+                fq.flex_prefill_layer(self.layers[l], self.caches[l][0], src, dst, cfg["call_batch"], cfg["prompt"],
+                                      self.ws_pre)
+            else:
+                fq.flex_prefill_layer_batches(self.layers[l], self.caches[l], src, dst, cfg["call_batch"],
+                                              cfg["prompt"], self.ws_pre)
+            src, dst = dst, src
+        # the last layer's output is not kept: a synthetic stack has no LM head
+
+    def free_prefill(self):
+        del self.ws_pre, self.x_pre, self.y_pre
+        self.torch.cuda.empty_cache()
+
+
+def build_decode_graphs(fq, torch, stack, stream, inputs, y_out, positions):
+    """One CUDA graph per position: all sequences through every layer, chained through
+    two activation buffers. With several gpu-batches (the pages' gpu_batch_size x
+    num_gpu_batches block) each layer is one flex_decode_layer_batches call, so its
+    weights are streamed once for all gpu-batches. inputs [T][batch][h], y_out [batch][h]."""
+    cfg = stack.cfg
+    L, b, calls = cfg["layers"], cfg["call_batch"], cfg["calls"]
+    bufs = [torch.empty((calls * b, cfg["h"]), dtype=torch.float16, device=stack.dev) for _ in range(2)]
+
+    def token(t, pos):
+        src = inputs[t]
+        for l in range(L):
+            dst = y_out if l == L - 1 else bufs[l % 2]
+            if calls == 1:
+                fq.flex_decode_layer(stack.layers[l], stack.caches[l][0], src, dst, b, pos, stack.ws_dec)
+            else:
+                fq.flex_decode_layer_batches(stack.layers[l], stack.caches[l], src, dst, b, pos, stack.ws_dec)
+            src = dst
+
+    with torch.cuda.stream(stream):
+        token(0, positions[0])                     # eager first call (kernel attributes, tensor maps)
+    stream.synchronize()
+    graphs = []
+    for t, pos in enumerate(positions):
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(g, stream=stream):
+            token(t, pos)
+        g.instantiate()
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs, bufs
 
 
 def run_flexq(args):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -197,75 +362,37 @@ def run_flexq(args):
 
     peaks = measured_peaks()
     cfg = workload_cfg(args.workload, args.layers)
-    L, b, s, h, nh, d = cfg["layers"], cfg["batch"], cfg["prompt"], cfg["h"], cfg["n_heads"], cfg["head_dim"]
+    L, b, s, h = cfg["layers"], cfg["batch"], cfg["prompt"], cfg["h"]
     nsteps = cfg["decode_steps"]
-    max_seq = s + nsteps
-    seed = cfg["seed"]
 
-    # ---- build the stack: compressed weights (flexq_compress on the GPU) and caches
-    layers, caches = [], []
-    for l in range(L):
-        raw = synth.layer_params(h, cfg["ffn"], seed * 100 + l, device=dev)
-        layers.append(fq.FlexLayer(raw, nh, device=dev))
-        del raw
-        caches.append(fq.FlexKVCache(b, nh, d, max_seq, device=dev))
-    torch.cuda.synchronize()
-
-    # ---- prefill (also measured as a part)
-    ws_pre = torch.zeros(fq.flex_workspace_bytes(layers[0], b, s), dtype=torch.uint8, device=dev)
-    xa = synth.activations((b, s, h), seed, device=dev)
-    xb = torch.empty_like(xa)
-
-    def prefill_stack():
-        src, dst = xa, xb
-        for l in range(L):
-            fq.flex_prefill_layer(layers[l], caches[l], src, dst, b, s, ws_pre)
-            src, dst = dst, src
-
-    prefill_stack()
+    stack = Stack(fq, torch, synth, cfg, dev)
+    stack.prefill()
     torch.cuda.synchronize()
     rc = fq.flex_get_status()
     if rc != 0:
         raise RuntimeError(f"prefill failed: {fq.flex_status_string(rc)}")
 
-    # ---- decode: one graph per position, the 24-layer stack chained through 2 buffers
-    ws_dec = torch.zeros(fq.flex_workspace_bytes(layers[0], b, 1), dtype=torch.uint8, device=dev)
-    inputs = torch.stack([synth.decode_inputs(b, h, t, seed, device=dev) for t in range(nsteps)])
-    buf = [torch.empty((b, h), dtype=torch.float16, device=dev) for _ in range(2)]
-    y_out = torch.empty((b, h), dtype=torch.float16, device=dev)
-
-    def decode_token(t):
-        src = inputs[t]
-        for l in range(L):
-            dst = y_out if l == L - 1 else buf[l % 2]
-            fq.flex_decode_layer(layers[l], caches[l], src, dst, b, s + t, ws_dec)
-            src = dst
-
     stream = torch.cuda.Stream(device=dev)
-    with torch.cuda.stream(stream):
-        decode_token(0)                        # eager first call (kernel attributes, tensor maps)
-    stream.synchronize()
-    graphs = []
-    for t in range(nsteps):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            decode_token(t)
-        graphs.append(g)
-    torch.cuda.synchronize()
+    inputs = torch.stack([synth.decode_inputs(b, h, t, cfg["seed"], device=dev) for t in range(nsteps)])
+    y_out = torch.empty((b, h), dtype=torch.float16, device=dev)
+    positions = [s + t for t in range(nsteps)]
+    graphs, _bufs = build_decode_graphs(fq, torch, stack, stream, inputs, y_out, positions)
+
+    # kernels per decode phase, read back from the captured graphs
+    launch_counts = {}
+    for g in graphs:
+        c = graph_kernel_counts(g)
+        if c is None:
+            launch_counts = None
+            break
+        for k, v in c.items():
+            launch_counts[k] = launch_counts.get(k, 0) + v
 
     def decode_phase():
         for g in graphs:
             g.replay()
 
-    # LN1, QKV (+store_cache), attention, out, LN2, fc1, fc2, plus the attention combine
-    # when a (sequence, head) key range is split across CTAs (the library splits when the
-    # pairs alone fill fewer than 4 CTAs per SM; a split keeps at least 128 keys)
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    pairs = b * nh
-    splits = [max(1, min((4 * sms + pairs - 1) // pairs, (s + t + 127) // 128)) for t in range(nsteps)]
-    launches_per_token = [L * (7 if ns == 1 else 8) for ns in splits]
     units_per_step = b * nsteps * L
-
     for _ in range(args.warmup):
         with torch.cuda.stream(stream):
             decode_phase()
@@ -326,36 +453,58 @@ def run_flexq(args):
     if rc != 0:
         raise RuntimeError(f"timed region failed: {fq.flex_status_string(rc)}")
     assert bool(torch.isfinite(y_out).all())
+    del graphs
+
+    # ---- bounds of the step (summed over its positions and layers)
+    costs = [step_cost(cfg, p, peaks["hbm_gbs"], peaks["bf16_tflops"]) for p in positions]
+    step_s = ms / args.steps / 1e3
+    hbm_s = sum(c["hbm_s"] for c in costs) * L
+    att_s = sum(c["attainable_s"] for c in costs) * L
+    step_bounds = {"hbm_bound_ms": hbm_s * 1e3, "attainable_bound_ms": att_s * 1e3, "measured_ms": step_s * 1e3,
+                   "frac_of_hbm_bound": hbm_s / step_s, "frac_of_attainable_bound": att_s / step_s,
+                   "note": "hbm: algorithmic bytes / measured copy bandwidth; attainable: per kernel max(bytes / "
+                           "bandwidth, flops / tensor peak), summed"}
 
     parts, roofline = {}, None
     if rank == 0 and not args.no_parts:
-        parts, roofline = measure_parts(fq, torch, synth, cfg, layers, caches, ws_dec, stream, peaks, dev,
-                                        prefill_stack, ws_pre)
+        parts, roofline = measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev)
+        if args.workload == "opt-175b":
+            del stack
+            torch.cuda.empty_cache()
+            parts["opt-30b_3x48"] = measure_secondary_decode(fq, torch, synth, "opt-30b", peaks, dev)
+        codec = measure_codec(fq, torch, synth, dev, peaks["hbm_gbs"], points=CODEC_POINTS_DEFAULT)
+        parts["codec"] = codec
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(cfg)
+        if "codec" in parts:
+            parts["codec"]["cpu_baseline"] = codec_cpu_baseline()
     if world > 1:
         dist.barrier()
 
-    hbm_bound_ms = sum(decode_bytes_per_layer_step(cfg, s + t) for t in range(nsteps)) * L / (peaks["hbm_gbs"] * 1e6)
+    ours = None
+    if launch_counts is not None:
+        # every kernel node of the decode graphs is one of the library's; names show which
+        ours = {short_kernel_name(k) if k != "?" else "unnamed kernel node": v for k, v in launch_counts.items()}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16 x int4 (fp32 accumulate)", "data": "synthetic",
-        "config": bench_config(args, cfg, world),
-        "hbm_roofline_frac_of_step": hbm_bound_ms / (ms / args.steps),
+        "config": bench_config(cfg, world),
         "roofline": roofline,
+        "step_bounds": step_bounds,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(host_in.numel() * 2),
                 "d2h_bytes_per_step": int(host_out.numel() * 2)},
-        "gpu_launches": sum(launches_per_token) * args.steps,
+        "gpu_launches": (sum(ours.values()) * args.steps) if ours else None,
+        "gpu_launches_per_step_by_kernel": ours,
+        "gpu_launches_source": "kernel nodes of the captured decode graphs replayed in the timed region",
         "clocks": clocks,
         "peaks": peaks,
         "parts": parts,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs
     if world > 1:
         dist.destroy_process_group()
 
@@ -382,21 +531,41 @@ def _traffic(kernel_key, sha):
     return e.get("dram_bytes_per_launch")
 
 
-def measure_codec(fq, torch, synth, dev, hbm):
-    """flexq_compress / flexq_decompress on 1 GiB of fp16 [131072, 4096], 4-bit group 64,
-    grouped along the contiguous and the strided dimension: GB/s of algorithmic bytes
-    (fp16 in or out, codes, metadata) over 10 back-to-back calls (the tensor is 8x L2)."""
+# ---- codec ---------------------------------------------------------------------------
+# (rows of [R, 4096] fp16 or a 3-D shape, group_dim, bits, group size)
+CODEC_POINTS_DEFAULT = [((131072, 4096), 1, 4, 64), ((131072, 4096), 0, 4, 64), ((131072, 4096), 1, 8, 64),
+                        ((131072, 4096), 1, 4, 32), ((131072, 4096), 1, 4, 128)]
+
+
+def codec_sweep_points():
+    pts = []
+    for mb in (16, 256, 1024, 4096):
+        rows = mb * (1 << 20) // (2 * 4096)
+        for gd in (1, 0):
+            for bits in (4, 8):
+                for gs in (32, 64, 128):
+                    pts.append(((rows, 4096), gd, bits, gs))
+    pts.append(((544, 144 * 96, 128), 2, 4, 64))         # KV-shaped: [tokens][seq x heads][head_dim]
+    return pts
+
+
+def measure_codec(fq, torch, synth, dev, hbm, points):
+    """flexq_compress / flexq_decompress: GB/s of algorithmic bytes (fp16 in or out,
+    codes, metadata) over 10 back-to-back calls per point (each input is at least 2x L2,
+    except the 16 MB points, which are L2-resident and marked so)."""
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    codec = {}
-    for gd in (1, 0):
-        shape = (131072, 4096)
-        xt = synth.codec_tensor(shape, gd, 64, 9, device=dev)
-        cfgq = fq.config(4, 64, gd)
+    out = {}
+    for shape, gd, bits, gs in points:
+        xt = synth.codec_tensor(shape, gd, gs, 9, device=dev)
+        cfgq = fq.config(bits, gs, gd)
         codes, meta = fq.flexq_compress(xt, cfgq)
         yt = fq.flexq_decompress(codes, meta, shape, cfgq)
         n = xt.numel()
-        nbytes = n * 2 + n // 2 + n // 64 * 4
+        nbytes = n * 2 + n * bits // 8 + n // gs * 4
+        layout = {1: "contiguous", 0: "strided"}.get(gd, f"dim{gd}") if len(shape) == 2 else f"kv-dim{gd}"
+        key = f"{'x'.join(map(str, shape))}_{layout}_{bits}bit_g{gs}"
+        entry = {"mb": round(n * 2 / (1 << 20)), "bytes": nbytes}
         for opname, fn in (("compress", lambda: fq.flexq_compress(xt, cfgq, codes, meta)),
                            ("decompress", lambda: fq.flexq_decompress(codes, meta, shape, cfgq, yt))):
             for _ in range(3):
@@ -408,21 +577,31 @@ def measure_codec(fq, torch, synth, dev, hbm):
             e1.record()
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / 10
-            key = f"{opname}_{'contiguous' if gd == 1 else 'strided'}"
-            codec[key] = {"gbs": nbytes / (ms * 1e6), "frac_hbm": nbytes / (ms * 1e6) / hbm, "ms": ms,
-                          "bytes": nbytes}
+            entry[opname] = {"gbs": nbytes / (ms * 1e6), "frac_hbm": nbytes / (ms * 1e6) / hbm, "us": ms * 1e3}
+        if n * 2 < 2 * 126 * (1 << 20):
+            entry["note"] = "L2-resident"
+        out[key] = entry
         del xt, codes, meta, yt
         torch.cuda.empty_cache()
-    return codec
+    rc = fq.flex_get_status()
+    if rc != 0:
+        raise RuntimeError(f"codec failed: {fq.flex_status_string(rc)}")
+    return out
 
 
-def measure_parts(fq, torch, synth, cfg, layers, caches, ws_dec, stream, peaks, dev, prefill_stack, ws_pre):
+# ---- parts ---------------------------------------------------------------------------
+def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
     """Each kernel of the decode step on its own (same launch configuration, cycling
-    over the stack so nothing stays in L2), the prefill, and the codec."""
-    L, b, s, h, nh, d, ffn = cfg["layers"], cfg["batch"], cfg["prompt"], cfg["h"], cfg["n_heads"], cfg["head_dim"], cfg["ffn"]
+    over the stack so nothing stays in L2) and the prefill."""
+    L, b, s, h, nh, d, ffn = (cfg["layers"], cfg["call_batch"], cfg["prompt"], cfg["h"], cfg["n_heads"],
+                              cfg["head_dim"], cfg["ffn"])
+    calls = cfg["calls"]
     pos = s + cfg["decode_steps"] // 2
-    hbm = peaks["hbm_gbs"]
+    hbm, tpk = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    ridge = tpk * 1e12 / (hbm * 1e9)               # flop per byte where the two bounds meet
     reps = 20
+    layers = stack.layers
+    caches = [cs[0] for cs in stack.caches]
 
     def time_cycle(fn, reps=reps):
         """ms per call of fn, from a CUDA graph that calls fn once per layer (so the
@@ -451,125 +630,212 @@ def measure_parts(fq, torch, synth, cfg, layers, caches, ws_dec, stream, peaks, 
         return e0.elapsed_time(e1) / (reps * L)      # ms per launch(-group)
 
     x = synth.activations((b, 3 * h), 5, device=dev)
+    x[:, :h] *= d ** -0.5
     xf = synth.activations((b, ffn), 6, device=dev)
     o = torch.empty((b, h), dtype=torch.float16, device=dev)
     yq = torch.empty((b, 3 * h), dtype=torch.float16, device=dev)
     yf = torch.empty((b, ffn), dtype=torch.float16, device=dev)
     gws = torch.zeros(max(16, max(fq.flex_gemm_ws_bytes(b, n, k) for n, k in
                                   ((3 * h, h), (h, h), (ffn, h), (h, ffn)))), dtype=torch.uint8, device=dev)
-    aws = torch.zeros(fq.flex_decode_attention_ws_bytes(caches[0], b, pos), dtype=torch.uint8, device=dev)
+    aws = torch.zeros(max(16, fq.flex_decode_attention_ws_bytes(caches[0], b, pos)), dtype=torch.uint8, device=dev)
     per = 0.5625
+    # the library splits a (sequence, head) key range over CTAs only when the pairs alone
+    # fill fewer than 4 CTAs per SM; then a combine kernel merges the splits
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    attn_launches = 1 if b * nh >= 4 * sms else 2
     kern = {}
     kern["decode_attention"] = dict(
         ms=time_cycle(lambda l: fq.flex_decode_attention(caches[l], x[:, :h], x[:, h:], x[:, 2 * h:], 3 * h, o, b,
                                                          pos, aws, stream=stream)),
-        bytes=2 * b * pos * h * per + 3 * b * h * 2 + b * h * 2, launches_per_layer_step=2,
-        source=["attention.cu"])
+        bytes=2 * b * pos * h * per + 3 * b * h * 2 + b * h * 2, flops=4.0 * b * (pos + 1) * h,
+        launches_per_call=attn_launches, source=["attention.cu"])
+    gemm_kernel = "gemv_kernel" if b <= 32 else "gemm_tc_kernel"   # the library's dispatch by batch
     for name, (n, k, xin, yout, epi) in {"gemm_qkv": (3 * h, h, x[:, :h], yq, 0), "gemm_out": (h, h, x[:, :h], o, 0),
                                           "gemm_fc1": (ffn, h, x[:, :h], yf, 1),
                                           "gemm_fc2": (h, ffn, xf, o, 0)}.items():
         wkey = {"gemm_qkv": "w_qkv", "gemm_out": "w_o", "gemm_fc1": "w_fc1", "gemm_fc2": "w_fc2"}[name]
         kern[name] = dict(
             # the layer hands every GEMM its activations in the interleaved 8-block order
-            ms=time_cycle(lambda l, n=n, xin=xin, yout=yout, epi=epi, wkey=wkey:
+            ms=time_cycle(lambda l, xin=xin, yout=yout, epi=epi, wkey=wkey:
                           fq.flex_dequant_gemm(xin, layers[l].w[wkey], None, None, yout, b,
                                                epi | fq.FLEX_GEMM_X_INTERLEAVED, gws, stream=stream)),
-            bytes=n * k * per + b * k * 2 + b * n * 2, launches_per_layer_step=1, source=["gemm.cu", "tc.cuh"])
+            bytes=n * k * per + b * k * 2 + b * n * 2, flops=2.0 * b * n * k, launches_per_call=1,
+            kernel=gemm_kernel, source=["gemm.cu", "tc.cuh"])
     kern["store_cache"] = dict(
         ms=time_cycle(lambda l: fq.flex_append_kv(caches[l], x[:, h:], x[:, 2 * h:], 3 * h, b, pos, stream=stream)),
-        bytes=2 * b * h * 2 + 2 * b * h * per, launches_per_layer_step=0, source=["kv_ln.cu"],
+        bytes=2 * b * h * 2 + 2 * b * h * per, flops=0.0, launches_per_call=0, source=["kv_ln.cu"],
         note="standalone store_cache entry; inside a layer it is fused into the QKV GEMM epilogue")
     kern["layernorm"] = dict(
         ms=time_cycle(lambda l: fq.flex_layernorm(x[:, :h], layers[l].vec["ln1_g"], layers[l].vec["ln1_b"], o, b, h,
                                                   stream=stream)),
-        bytes=2 * b * h * 2 + 2 * h * 2, launches_per_layer_step=2, source=["kv_ln.cu"])
+        bytes=2 * b * h * 2 + 2 * h * 2, flops=0.0, launches_per_call=2, source=["kv_ln.cu"])
     for k, v in kern.items():
+        v["us"] = v["ms"] * 1e3
         v["gbs"] = v["bytes"] / (v["ms"] * 1e6)
         v["frac_hbm"] = v["gbs"] / hbm
-        v["us"] = v["ms"] * 1e3
-    # per kernel (the four GEMMs are launches of one kernel, gemm_tc_kernel): time per
-    # layer step, and bytes and duration per launch averaged over its launches
+        if v["flops"]:
+            v["tflops"] = v["flops"] / (v["ms"] * 1e9)
+            v["frac_tensor"] = v["tflops"] / tpk
+    # per kernel (the four GEMMs are launches of one kernel): time per layer call, and
+    # bytes / flops / duration per launch averaged over its launches
     gemms = ["gemm_qkv", "gemm_out", "gemm_fc1", "gemm_fc2"]
-    gemm_kernel = "gemv_kernel" if b <= 32 else "gemm_tc_kernel"   # the library's dispatch by batch
     per_kernel = {
-        gemm_kernel: dict(launches=4, ms=sum(kern[g]["ms"] for g in gemms),
-                               bytes=sum(kern[g]["bytes"] for g in gemms), source=["gemm.cu", "tc.cuh"]),
-        "decode_attention": dict(launches=2, ms=kern["decode_attention"]["ms"],
-                                 bytes=kern["decode_attention"]["bytes"], source=["attention.cu"]),
+        gemm_kernel: dict(launches=4, ms=sum(kern[g]["ms"] for g in gemms), bytes=sum(kern[g]["bytes"] for g in gemms),
+                          flops=sum(kern[g]["flops"] for g in gemms), source=["gemm.cu", "tc.cuh"]),
+        "decode_attn_tc_kernel": dict(launches=attn_launches, ms=kern["decode_attention"]["ms"],
+                                      bytes=kern["decode_attention"]["bytes"], flops=kern["decode_attention"]["flops"],
+                                      source=["attention.cu"]),
         "layernorm_kernel": dict(launches=2, ms=2 * kern["layernorm"]["ms"], bytes=2 * kern["layernorm"]["bytes"],
-                                 source=["kv_ln.cu"]),
+                                 flops=0.0, source=["kv_ln.cu"]),
     }
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"])
     dk = per_kernel[dom]
-    gbs = dk["bytes"] / (dk["ms"] * 1e6)
     sha = _kernel_sha(*dk["source"])
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
-                "frac": gbs / hbm, "traffic": _traffic(dom, sha),
-                "launches_per_layer_step": dk["launches"],
+    intensity = dk["flops"] / dk["bytes"]
+    tensor_bound = intensity > ridge
+    achieved = dk["flops"] / (dk["ms"] * 1e9) if tensor_bound else dk["bytes"] / (dk["ms"] * 1e6)
+    peak = tpk if tensor_bound else hbm
+    roofline = {"kernel": dom, "bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s" if tensor_bound else "GB/s", "frac": achieved / peak,
+                "traffic": _traffic(f"{dom}@{cfg['name']}", sha),
+                "launches_per_layer_call": dk["launches"],
                 "algorithmic_bytes_per_launch": dk["bytes"] / dk["launches"],
+                "algorithmic_flops_per_launch": dk["flops"] / dk["launches"],
+                "intensity_flop_per_byte": intensity, "ridge_flop_per_byte": ridge,
                 "avg_launch_us": dk["ms"] * 1e3 / dk["launches"],
+                "frac_hbm": dk["bytes"] / (dk["ms"] * 1e6) / hbm,
+                "frac_tensor": dk["flops"] / (dk["ms"] * 1e9) / tpk,
                 "share_of_layer_step_parts": dk["ms"] / sum(v["ms"] for v in per_kernel.values()),
-                "peak_source": f"{peaks['source']} hbm_gbs (copy)", "source_sha": sha}
+                "peak_source": f"{peaks['source']} " + ("bf16_tflops (cuBLAS burst; fp16 dense has the same rate)"
+                                                        if tensor_bound else "hbm_gbs (copy)"),
+                "timing": "CUDA events around a graph of one launch per layer of the stack, replayed 20 times",
+                "source_sha": sha}
 
     # prefill through the stack
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    prefill_stack()
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(2):
-        prefill_stack()
-    e1.record()
-    torch.cuda.synchronize()
-    pms = e0.elapsed_time(e1) / (2 * L)
-    T = b * s
-    flops = 2 * T * (4 * h * h + 2 * h * ffn) + 2 * b * nh * s * s * d       # causal: half of 4*b*s^2*h
-    prefill = {"tokens_per_s_per_layer": T / (pms / 1e3), "ms_per_layer": pms,
-               "tflops": flops / (pms * 1e9), "frac_tensor_peak": flops / (pms * 1e9) / peaks["bf16_tflops"],
-               "peak_note": "fp16 tensor peak = measured bf16 cuBLAS peak (same rate)"}
-
-    codec = measure_codec(fq, torch, synth, dev, hbm)
+    stack_ok = hasattr(stack, "ws_pre")
+    prefill = None
+    if stack_ok:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        stack.prefill()
+        torch.cuda.synchronize()
+        e0.record()
+        stack.prefill()
+        e1.record()
+        torch.cuda.synchronize()
+        pms = e0.elapsed_time(e1) / (L * calls)
+        T = b * s
+        flops = 2 * T * (4 * h * h + 2 * h * ffn) + 2 * b * nh * s * s * d       # causal: half of 4*b*s^2*h
+        prefill = {"tokens_per_s_per_layer": T / (pms / 1e3), "ms_per_layer_call": pms,
+                   "tflops": flops / (pms * 1e9), "frac_tensor_peak": flops / (pms * 1e9) / tpk,
+                   "peak_note": "fp16 tensor peak = measured bf16 cuBLAS peak (same rate)"}
     rc = fq.flex_get_status()
     if rc != 0:
         raise RuntimeError(f"parts failed: {fq.flex_status_string(rc)}")
-    return {"kernels": kern, "prefill": prefill, "codec_1gib_4bit_g64": codec}, roofline
+    return {"kernels": kern, "per_kernel_per_layer_call": per_kernel, "prefill": prefill}, roofline
+
+
+def measure_secondary_decode(fq, torch, synth, name, peaks, dev, ntok=8, reps=5):
+    """Decode of another workload's schedule (e.g. opt-30b as 3 gpu-batches of 48): a
+    1-layer stack prefilled with the prompt, then graphs of `ntok` positions replayed
+    `reps` times. layer-tokens/s and the step bounds."""
+    cfg = workload_cfg(name)
+    stack = Stack(fq, torch, synth, cfg, dev)
+    stack.prefill()
+    stack.free_prefill()
+    stream = torch.cuda.Stream(device=dev)
+    b, h, s = cfg["batch"], cfg["h"], cfg["prompt"]
+    inputs = torch.stack([synth.decode_inputs(b, h, t, cfg["seed"], device=dev) for t in range(ntok)])
+    y_out = torch.empty((b, h), dtype=torch.float16, device=dev)
+    positions = [s + t for t in range(ntok)]
+    graphs, _ = build_decode_graphs(fq, torch, stack, stream, inputs, y_out, positions)
+    with torch.cuda.stream(stream):
+        for g in graphs:
+            g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            for g in graphs:
+                g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    rc = fq.flex_get_status()
+    if rc != 0:
+        raise RuntimeError(f"{name} decode failed: {fq.flex_status_string(rc)}")
+    ms = e0.elapsed_time(e1) / (reps * ntok * cfg["layers"])          # per layer-step
+    costs = [step_cost(cfg, p, peaks["hbm_gbs"], peaks["bf16_tflops"]) for p in positions]
+    hbm_s = sum(c["hbm_s"] for c in costs) / ntok
+    att_s = sum(c["attainable_s"] for c in costs) / ntok
+    out = {"workload": bench_config(cfg, 1)["workload"], "layer_tokens_per_s": b / (ms / 1e3),
+           "ms_per_layer_step": ms, "frac_of_hbm_bound": hbm_s / (ms / 1e3),
+           "frac_of_attainable_bound": att_s / (ms / 1e3), "positions": f"{s}..{s + ntok - 1}"}
+    del graphs, stack
+    torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------------------
-def _oracle_sample(cfg, nseq, nsteps_cpu, budget_s=20.0):
-    """Decode of `nseq` sequences through one oracle layer, one position after another,
-    until about budget_s of work. Returns (layer-tokens, seconds, threads)."""
-    import numpy as np
-    from threadpoolctl import threadpool_info
-
+def _oracle_sample(cfg, nseq, nsteps_cpu, budget_s=15.0, nthreads=None):
+    """Decode of `nseq` sequences through one layer of the C++ fp32 oracle, one position
+    after another from `prompt` on, until about budget_s of work (at least one step).
+    Returns (layer-tokens, seconds, threads, steps)."""
     import synth
-    from oracle import layer as ol
+    from oracle import cpp
     h, nh, d, s = cfg["h"], cfg["n_heads"], cfg["head_dim"], cfg["prompt"]
+    nthreads = nthreads or cpp.threads()
     raw = {k: v.numpy() for k, v in synth.layer_params(h, cfg["ffn"], cfg["seed"] * 100).items()}
-    PQ = ol.compress_weights(raw)
-    W = ol.dequant_all(PQ)
-    cache = ol.KVCache(nseq, nh, s + cfg["decode_steps"], d)
+    layer = cpp.Layer(raw, nh, nthreads=nthreads)
+    del raw
+    cache = cpp.KVCache(nseq, nh, s + cfg["decode_steps"], d)
     kh, vh = synth.kv_history(nseq, nh, s, d, cfg["seed"])
-    cache.store(kh.numpy(), vh.numpy(), 0)
-    done, t0 = 0, time.perf_counter()
+    for name, t in (("k", kh), ("v", vh)):
+        c, m = cpp.compress(t.numpy(), 4, 64, 3, nthreads)
+        getattr(cache, f"{name}_codes")[:, :, :s] = c
+        getattr(cache, f"{name}_meta")[:, :, :s] = m
+    done, steps, t0 = 0, 0, time.perf_counter()
     for t in range(nsteps_cpu):
         x = synth.decode_inputs(nseq, h, t, cfg["seed"]).numpy()
-        ol.decode_layer(x, PQ, cache, s + t, nh, W=W)
+        cpp.decode_layer(x, layer, cache, s + t % cfg["decode_steps"], nthreads)
         done += nseq
+        steps += 1
         if time.perf_counter() - t0 > budget_s:
             break
-    secs = time.perf_counter() - t0
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    return done, secs, threads
+    return done, time.perf_counter() - t0, nthreads, steps
 
 
 def cpu_baseline(cfg):
-    nseq = min(8, cfg["batch"])
-    done, secs, threads = _oracle_sample(cfg, nseq, cfg["decode_steps"], budget_s=15.0)
+    nseq = min(16, cfg["call_batch"])
+    done, secs, threads, _ = _oracle_sample(cfg, nseq, cfg["decode_steps"], budget_s=12.0)
     return {"value": done / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{done} layer-tokens: {nseq} sequences of the {cfg['h']}-wide layer decoded at positions "
-                      f"{cfg['prompt']}.. through one oracle layer (numpy fp64, BLAS threads {threads})"}
+                      f"{cfg['prompt']}.. through one layer of the C++ fp32 oracle ({threads} threads)"}
+
+
+def codec_cpu_baseline():
+    """The C++ oracle's compress / decompress of a 256 MiB fp16 [32768, 4096] tensor (4-bit
+    g64, contiguous groups), on one thread and on every host core: GB/s with the GPU's
+    byte accounting."""
+    import synth
+    from oracle import cpp
+    x = synth.codec_tensor((32768, 4096), 1, 64, 9).numpy()
+    n = x.size
+    nbytes = n * 2 + n // 2 + n // 64 * 4
+    out = {}
+    for th in (1, cpp.threads()):
+        t0 = time.perf_counter()
+        c, m = cpp.compress(x, 4, 64, 1, nthreads=th)
+        t1 = time.perf_counter()
+        cpp.decompress(c, m, x.shape, 4, 64, 1, nthreads=th)
+        t2 = time.perf_counter()
+        out[f"threads_{th}"] = {"compress_gbs": nbytes / (t1 - t0) / 1e9, "decompress_gbs": nbytes / (t2 - t1) / 1e9}
+    out["kind"] = "oracle"
+    out["sample"] = "256 MiB fp16 [32768, 4096], 4-bit g64 along the contiguous dim, C++ fp32 oracle"
+    out["cores"] = cpp.threads()
+    return out
 
 
 def run_reference(args):
@@ -578,20 +844,20 @@ def run_reference(args):
     if rank != 0:
         return
     cfg = workload_cfg(args.workload, args.layers)
-    nseq = 4
+    nseq = min(16, cfg["call_batch"])
     # warm-up and timed steps: each step = one decode position for `nseq` sequences
-    from oracle import layer as ol  # noqa: F401  (the oracle is the reference arm)
-    done, secs, threads = _oracle_sample(cfg, nseq, args.warmup + args.steps, budget_s=1e9)
-    per_step = secs / (args.warmup + args.steps)
+    n_all = args.warmup + args.steps
+    done, secs, threads, steps = _oracle_sample(cfg, nseq, n_all, budget_s=1e9)
+    per_step = secs / steps
     value = nseq / per_step
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-            "config": bench_config(args, cfg, world),
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (C++ oracle)", "data": "synthetic",
+            "config": bench_config(cfg, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": f"each step: {nseq} sequences of the {cfg['h']}-wide layer decoded one "
-                                       f"position through one oracle layer (numpy fp64); "
-                                       f"{args.warmup + args.steps} steps"},
+                                       f"position through one layer of the C++ fp32 oracle ({threads} threads); "
+                                       f"{n_all} steps"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -604,16 +870,86 @@ def run_codec_only():
     torch.cuda.set_device(dev)
     fq.lib()
     hbm = measured_peaks()["hbm_gbs"]
-    codec = measure_codec(fq, torch, synth, dev, hbm)
+    codec = measure_codec(fq, torch, synth, dev, hbm, points=codec_sweep_points())
+    print(json.dumps({"mode": "codec", "unit": "GB/s", "peak_hbm_gbs": hbm, "codec": codec}), flush=True)
+
+
+def run_kernel_only(args):
+    """One step of the decode layer (or the codec on 1 GiB) 3 times on one layer of the
+    workload, with a device synchronisation after each call: the small case that the
+    ncu captures under profiles/ run."""
+    import torch
+    import group_wise_int4_b200 as fq
+    import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = workload_cfg(args.workload, 1)
+    b, s, h, nh, d, ffn = cfg["call_batch"], cfg["prompt"], cfg["h"], cfg["n_heads"], cfg["head_dim"], cfg["ffn"]
+    pos = s + cfg["decode_steps"] // 2
+    k = args.kernel
+    if k in ("compress", "decompress"):
+        shape, cfgq = (131072, 4096), fq.config(4, 64, 1)
+        xt = synth.codec_tensor(shape, 1, 64, 9, device=dev)
+        codes, meta = fq.flexq_compress(xt, cfgq)
+        fn = ((lambda: fq.flexq_compress(xt, cfgq, codes, meta)) if k == "compress"
+              else (lambda: fq.flexq_decompress(codes, meta, shape, cfgq, xt)))
+    else:
+        layer = fq.FlexLayer(synth.layer_params(h, ffn, cfg["seed"], device=dev), nh, device=dev)
+        cache = fq.FlexKVCache(b, nh, d, s + cfg["decode_steps"], device=dev)
+        kh, vh = synth.kv_history(b, nh, pos, d, cfg["seed"], device=dev)
+        cache.fill_from(kh, vh)
+        del kh, vh
+        x = synth.activations((b, 3 * h), 5, device=dev)
+        x[:, :h] *= d ** -0.5
+        xf = synth.activations((b, ffn), 6, device=dev)
+        y = torch.empty((b, max(3 * h, ffn)), dtype=torch.float16, device=dev)
+        if k.startswith("gemm_"):
+            wkey, xin, n, epi = {"gemm_qkv": ("w_qkv", x[:, :h], 3 * h, 0), "gemm_out": ("w_o", x[:, :h], h, 0),
+                                 "gemm_fc1": ("w_fc1", x[:, :h], ffn, 1), "gemm_fc2": ("w_fc2", xf, h, 0)}[k]
+            kk = xin.shape[1]
+            ws = torch.zeros(max(16, fq.flex_gemm_ws_bytes(b, n, kk)), dtype=torch.uint8, device=dev)
+            yo = y[:, :n].contiguous()
+            fn = lambda: fq.flex_dequant_gemm(xin.contiguous(), layer.w[wkey], None, None, yo, b,
+                                              epi | fq.FLEX_GEMM_X_INTERLEAVED, ws)
+        elif k == "decode_attention":
+            ws = torch.zeros(max(16, fq.flex_decode_attention_ws_bytes(cache, b, pos)), dtype=torch.uint8, device=dev)
+            o = torch.empty((b, h), dtype=torch.float16, device=dev)
+            fn = lambda: fq.flex_decode_attention(cache, x[:, :h], x[:, h:], x[:, 2 * h:], 3 * h, o, b, pos, ws)
+        elif k == "layernorm":
+            o = torch.empty((b, h), dtype=torch.float16, device=dev)
+            fn = lambda: fq.flex_layernorm(x[:, :h], layer.vec["ln1_g"], layer.vec["ln1_b"], o, b, h)
+        elif k == "decode_layer":
+            ws = torch.zeros(fq.flex_workspace_bytes(layer, b, 1), dtype=torch.uint8, device=dev)
+            xin = synth.decode_inputs(b, h, 0, cfg["seed"], device=dev)
+            o = torch.empty((b, h), dtype=torch.float16, device=dev)
+            fn = lambda: fq.flex_decode_layer(layer, cache, xin, o, b, pos, ws)
+        else:                                            # prefill_layer, a 128-token prompt
+            sp = 128
+            ws = torch.zeros(fq.flex_workspace_bytes(layer, b, sp), dtype=torch.uint8, device=dev)
+            xin = synth.activations((b, sp, h), cfg["seed"], device=dev)
+            o = torch.empty_like(xin)
+            fn = lambda: fq.flex_prefill_layer(layer, cache, xin, o, b, sp, ws)
+    times = []
+    for _ in range(3):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
     rc = fq.flex_get_status()
     if rc != 0:
-        raise RuntimeError(f"codec failed: {fq.flex_status_string(rc)}")
-    print(json.dumps({"mode": "codec", "unit": "GB/s", "peak_hbm_gbs": hbm, "codec_1gib_4bit_g64": codec}), flush=True)
+        raise RuntimeError(f"{k} failed: {fq.flex_status_string(rc)}")
+    print(json.dumps({"mode": "kernel", "kernel": k, "workload": cfg["name"], "call_batch": b, "pos": pos,
+                      "us_per_call_cold": times}), flush=True)
 
 
 def main():
     args = parse_args()
-    if args.codec_only:
+    if args.kernel:
+        run_kernel_only(args)
+    elif args.codec_only:
         run_codec_only()
     elif args.impl == "reference":
         run_reference(args)

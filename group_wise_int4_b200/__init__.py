@@ -99,6 +99,9 @@ _SIGS = {
     "flex_gemm_ws_bytes": (_I64, [_I32, _I32, _I32]),
     "flex_dequant_gemm": (_I32, [_P, ctypes.POINTER(flexq_tensor), _P, _P, _P, _I32, _I32, _P, _I64, _P]),
     "flex_layernorm": (_I32, [_P, _P, _P, _P, _I64, _I32, _P]),
+    "flex_embed": (_I32, [ctypes.POINTER(flexq_tensor), _I32, _P, _I32, _P, _P, _I64, _P, _P]),
+    "flex_lm_head_ws_bytes": (_I64, [ctypes.POINTER(flexq_tensor), _I32, _I64, _I32]),
+    "flex_lm_head_argmax": (_I32, [ctypes.POINTER(flexq_tensor), _I32, _P, _P, _P, _I64, _P, _P, _P, _I64, _P]),
     "flex_get_status": (_I32, [_P]),
     "flex_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "flex_status_string": (ctypes.c_char_p, [_I32]),
@@ -185,16 +188,18 @@ def config(num_bits=4, group_size=64, group_dim=0, symmetric=0) -> flexq_config:
 
 # ---- codec -----------------------------------------------------------------------
 def codes_shape(shape, cfg: flexq_config):
+    """Packed codes: num_groups * group_size * bits / 8 bytes along group_dim."""
     shape = tuple(int(d) for d in shape)
     gd = cfg.group_dim % len(shape)
-    return shape[:gd] + (shape[gd] * cfg.num_bits // 8,) + shape[gd + 1:]
+    ng = -(-shape[gd] // cfg.group_size)
+    return shape[:gd] + (ng * cfg.group_size * cfg.num_bits // 8,) + shape[gd + 1:]
 
 
 def meta_shape(shape, cfg: flexq_config):
     """Metadata shape in fp16 units: one {min, scale} pair per group as a trailing 2."""
     shape = tuple(int(d) for d in shape)
     gd = cfg.group_dim % len(shape)
-    return shape[:gd] + (shape[gd] // cfg.group_size,) + shape[gd + 1:] + (2,)
+    return shape[:gd] + (-(-shape[gd] // cfg.group_size),) + shape[gd + 1:] + (2,)
 
 
 def flexq_codes_bytes(shape, cfg: flexq_config) -> int:
@@ -418,6 +423,35 @@ def flex_layernorm(x, g, b, y, rows, h, stream=None):
     rc = lib().flex_layernorm(_ptr(x), _ptr(g), _ptr(b), _ptr(y), int(rows), int(h),
                               ctypes.c_void_p(_stream(stream)))
     _check(rc, "flex_layernorm")
+
+
+# ---- whole model: embedding, output head, greedy choice ------------------------------
+def flex_embed(E: "CompressedWeight", vocab, P, tokens, positions, x=None, stream=None):
+    """x [n][h] fp16 = E^[tokens] + P[positions] (tokens/positions: int32 CUDA tensors)."""
+    n = int(tokens.numel())
+    if x is None:
+        x = torch.empty((n, E.shape[1]), dtype=torch.float16, device=tokens.device)
+    rc = lib().flex_embed(ctypes.byref(E.struct()), int(vocab), _ptr(P), int(P.shape[0]), _ptr(tokens),
+                          _ptr(positions), n, _ptr(x), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "flex_embed")
+    return x
+
+
+def flex_lm_head_ws_bytes(E: "CompressedWeight", vocab, n, with_logits=False) -> int:
+    return int(lib().flex_lm_head_ws_bytes(ctypes.byref(E.struct()), int(vocab), int(n), int(bool(with_logits))))
+
+
+def flex_lm_head_argmax(E: "CompressedWeight", vocab, lnf_g, lnf_b, x, ws, next_ids=None, logits=None,
+                        stream=None):
+    """Greedy next tokens (int32 [n]) of the rows of x; logits (fp16 [n][V_pad]) if given."""
+    n = int(x.shape[0])
+    if next_ids is None:
+        next_ids = torch.empty(n, dtype=torch.int32, device=x.device)
+    rc = lib().flex_lm_head_argmax(ctypes.byref(E.struct()), int(vocab), _ptr(lnf_g), _ptr(lnf_b), _ptr(x), n,
+                                   _ptr(next_ids), _ptr(logits), _ptr(ws), int(ws.numel() * ws.element_size()),
+                                   ctypes.c_void_p(_stream(stream)))
+    _check(rc, "flex_lm_head_argmax")
+    return next_ids
 
 
 def flex_abi_layout(which: int, field: int) -> int:

@@ -22,12 +22,24 @@ namespace flexq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+// Vectors in flight per thread (compress) and resident blocks per SM the register budget
+// is sized for: build constants, tuned by measurement.
+#ifndef FLEXQ_CODEC_UNROLL
+#define FLEXQ_CODEC_UNROLL 4
+#endif
+#ifndef FLEXQ_CODEC_MINB
+#define FLEXQ_CODEC_MINB 1
+#endif
+#ifndef FLEXQ_DEC_UNROLL
+#define FLEXQ_DEC_UNROLL 8
+#endif
+constexpr int kUnroll = FLEXQ_CODEC_UNROLL;
+constexpr int kMinBlocks = FLEXQ_CODEC_MINB;
 
 // ---------------------------------------------------------------------------------
 // contiguous compress: G groups of GS fp16, codes G x (GS*BITS/8) bytes, meta G half2
 template <int BITS, int GS>
-__global__ void __launch_bounds__(kThreads) compress_contig_kernel(const __half* __restrict__ x,
+__global__ void __launch_bounds__(kThreads, kMinBlocks) compress_contig_kernel(const __half* __restrict__ x,
                                                                    uint8_t* __restrict__ codes,
                                                                    uint32_t* __restrict__ meta,
                                                                    int64_t G) {
@@ -73,10 +85,10 @@ __global__ void __launch_bounds__(kThreads) compress_contig_kernel(const __half*
 
 // contiguous decompress: one item = 8 consecutive values (4 or 8 code bytes in, one
 // 16-byte vector out), so a warp's loads and stores each cover one contiguous span.
-constexpr int kDecUnroll = 8;
+constexpr int kDecUnroll = FLEXQ_DEC_UNROLL;
 
 template <int BITS, int GS>
-__global__ void __launch_bounds__(kThreads) decompress_contig_kernel(const uint8_t* __restrict__ codes,
+__global__ void __launch_bounds__(kThreads, kMinBlocks) decompress_contig_kernel(const uint8_t* __restrict__ codes,
                                                                      const uint32_t* __restrict__ meta,
                                                                      __half* __restrict__ y,
                                                                      int64_t items) {
@@ -135,7 +147,7 @@ __global__ void __launch_bounds__(kThreads) decompress_contig_kernel(const uint8
 // min/max with shuffles (lane offsets IPW, 2 IPW, ...) and then quantise their own rows
 // with no second read.
 template <int BITS, int GS>
-__global__ void __launch_bounds__(kThreads) compress_strided_1pass_kernel(const __half* __restrict__ x,
+__global__ void __launch_bounds__(kThreads, kMinBlocks) compress_strided_1pass_kernel(const __half* __restrict__ x,
                                                                           uint8_t* __restrict__ codes,
                                                                           uint32_t* __restrict__ meta, int64_t outer,
                                                                           int64_t ng, int64_t inner) {
@@ -353,16 +365,137 @@ __global__ void __launch_bounds__(kThreads) decompress_strided_kernel(const uint
 }
 
 // ---------------------------------------------------------------------------------
+// Codec variants (one thread per group): 3-bit codes, the symmetric (absmax) form and a
+// group dimension that is not a multiple of the group size. Readings of what the pages
+// only name - the symmetric flag and num_groups of the compression configuration (the
+// walkthrough page, section 6.3), int3/int4 group-wise quantisation (the hub page):
+//   - symmetric: B = 2^(b-1) - 1, scale = fp16(B / max|x|) (0 for an all-zero group,
+//     65504 on overflow), signed code q = clamp(rint(x * scale), -B, B) stored as q + B,
+//     metadata {0, scale}, x^ = fp16((u - B) * fp32(1/scale));
+//   - 3 bits: the codes of a group form a little-endian bit stream (code j in bits
+//     [3j, 3j + 3)), 8 codes in every 3 bytes;
+//   - a partial last group is zero-padded: the padding takes part in min/max (or
+//     max|x|) and its codes are stored; decompression writes only the real elements.
+// Item (o, g, i): group g of the dimension, outer index o, inner index i.
+__global__ void __launch_bounds__(kThreads) compress_generic_kernel(const __half* __restrict__ x,
+                                                                     uint8_t* __restrict__ codes,
+                                                                     uint32_t* __restrict__ meta, int64_t outer,
+                                                                     int64_t G, int64_t ng, int64_t inner, int gs,
+                                                                     int bits, int sym) {
+    const int64_t items = outer * ng * inner;
+    const int64_t bpg = gs * bits / 8;
+    const int levels = (1 << bits) - 1, B = (1 << (bits - 1)) - 1;
+    for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
+         it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t i = it % inner, og = it / inner, g = og % ng, o = og / ng;
+        const __half* src = x + (o * G + g * gs) * inner + i;
+        const int real = G - g * gs < gs ? static_cast<int>(G - g * gs) : gs;
+        auto val = [&](int j) { return j < real ? __half2float(src[static_cast<int64_t>(j) * inner]) : 0.0f; };
+        float s = 0.0f, mn = 0.0f;
+        __half s16 = __ushort_as_half(0);
+        if (sym) {
+            float a = 0.0f;
+            for (int j = 0; j < gs; ++j) a = fmaxf(a, fabsf(val(j)));
+            if (a > 0.0f) {
+                s16 = __float2half_rn(__fdiv_rn(static_cast<float>(B), a));
+                if (__hisinf(s16)) s16 = __ushort_as_half(0x7BFF);
+            }
+        } else {
+            float mx = val(0);
+            mn = mx;
+            for (int j = 1; j < gs; ++j) {
+                const float v = val(j);
+                mn = fminf(mn, v);
+                mx = fmaxf(mx, v);
+            }
+            const float r = __fsub_rn(mx, mn);
+            if (r > 0.0f) {
+                s16 = __float2half_rn(__fdiv_rn(static_cast<float>(levels), r));
+                if (__hisinf(s16)) s16 = __ushort_as_half(0x7BFF);
+            }
+        }
+        s = __half2float(s16);
+        uint8_t* dst = codes + (o * ng * bpg + g * bpg) * inner + i;
+        uint32_t acc = 0;          // pending bits of the 3-bit stream, or the low nibble
+        int nacc = 0;
+        int64_t byte = 0;
+        for (int j = 0; j < gs; ++j) {
+            int q;
+            if (sym) {
+                q = __float2int_rn(__fmul_rn(val(j), s));
+                q = min(max(q, -B), B) + B;
+            } else {
+                q = __float2int_rn(__fmul_rn(__fsub_rn(val(j), mn), s));
+                q = min(max(q, 0), levels);
+            }
+            if (bits == 8) {
+                dst[(byte++) * inner] = static_cast<uint8_t>(q);
+            } else {
+                acc |= static_cast<uint32_t>(q) << nacc;
+                nacc += bits;
+                while (nacc >= 8) {
+                    dst[(byte++) * inner] = static_cast<uint8_t>(acc & 0xFFu);
+                    acc >>= 8;
+                    nacc -= 8;
+                }
+            }
+        }
+        meta[(o * ng + g) * inner + i] = pack_half2_bits(sym ? __ushort_as_half(0) : __float2half_rn(mn), s16);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) decompress_generic_kernel(const uint8_t* __restrict__ codes,
+                                                                       const uint32_t* __restrict__ meta,
+                                                                       __half* __restrict__ y, int64_t outer,
+                                                                       int64_t G, int64_t ng, int64_t inner, int gs,
+                                                                       int bits, int sym) {
+    const int64_t items = outer * ng * inner;
+    const int64_t bpg = gs * bits / 8;
+    const int B = (1 << (bits - 1)) - 1;
+    const uint32_t mask = (1u << bits) - 1u;
+    for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
+         it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t i = it % inner, og = it / inner, g = og % ng, o = og / ng;
+        const uint32_t mw = meta[(o * ng + g) * inner + i];
+        const __half mn16 = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
+        const float s = h2f_hi(mw), mn = __half2float(mn16);
+        const float step = s > 0.0f ? __fdiv_rn(1.0f, s) : 0.0f;
+        const uint8_t* src = codes + (o * ng * bpg + g * bpg) * inner + i;
+        __half* dst = y + (o * G + g * gs) * inner + i;
+        const int real = G - g * gs < gs ? static_cast<int>(G - g * gs) : gs;
+        uint32_t acc = 0;
+        int nacc = 0;
+        int64_t byte = 0;
+        for (int j = 0; j < real; ++j) {
+            while (nacc < bits) {
+                acc |= static_cast<uint32_t>(src[(byte++) * inner]) << nacc;
+                nacc += 8;
+            }
+            const int q = static_cast<int>(acc & mask);
+            acc >>= bits;
+            nacc -= bits;
+            __half v;
+            if (sym)
+                v = __float2half_rn(__fmul_rn(static_cast<float>(q - B), step));
+            else
+                v = s > 0.0f ? __float2half_rn(__fadd_rn(__fmul_rn(static_cast<float>(q), step), mn)) : mn16;
+            dst[static_cast<int64_t>(j) * inner] = v;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------
 struct Geometry {
-    int64_t outer = 1, ng = 0, inner = 1, n = 0;
+    int64_t outer = 1, ng = 0, inner = 1, n = 0, G = 0;
     int gd = 0;
+    bool generic = false;      // a variant configuration (compress_/decompress_generic_kernel)
 };
 
 int validate(int32_t ndim, const int64_t* shape, const flexq_config& cfg, Geometry& geo) {
     FLEX_REQUIRE(shape != nullptr, FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(ndim >= 1 && ndim <= 4, FLEX_ERR_INVALID_ARG);
-    FLEX_REQUIRE(cfg.symmetric == 0, FLEX_ERR_UNSUPPORTED);
-    FLEX_REQUIRE(cfg.num_bits == 4 || cfg.num_bits == 8, FLEX_ERR_UNSUPPORTED);
+    FLEX_REQUIRE(cfg.symmetric == 0 || cfg.symmetric == 1, FLEX_ERR_UNSUPPORTED);
+    FLEX_REQUIRE(cfg.num_bits == 3 || cfg.num_bits == 4 || cfg.num_bits == 8, FLEX_ERR_UNSUPPORTED);
     FLEX_REQUIRE(cfg.group_size == 32 || cfg.group_size == 64 || cfg.group_size == 128,
                  FLEX_ERR_UNSUPPORTED);
     int gd = cfg.group_dim;
@@ -373,16 +506,18 @@ int validate(int32_t ndim, const int64_t* shape, const flexq_config& cfg, Geomet
         FLEX_REQUIRE(shape[i] >= 0, FLEX_ERR_INVALID_ARG);
         n *= shape[i];
     }
-    FLEX_REQUIRE(shape[gd] % cfg.group_size == 0, FLEX_ERR_SHAPE);
     geo.gd = gd;
     geo.n = n;
+    geo.G = shape[gd];
     geo.outer = 1;
     for (int i = 0; i < gd; ++i) geo.outer *= shape[i];
     geo.inner = 1;
     for (int i = gd + 1; i < ndim; ++i) geo.inner *= shape[i];
-    geo.ng = shape[gd] / cfg.group_size;
+    geo.ng = (shape[gd] + cfg.group_size - 1) / cfg.group_size;      // a partial last group is padded
+    geo.generic = cfg.num_bits == 3 || cfg.symmetric != 0 || shape[gd] % cfg.group_size != 0;
     return FLEX_OK;
 }
+
 
 // Grid of a grid-stride kernel: enough blocks for `work_threads`, capped at what the
 // device holds resident at once (blocks per SM from the kernel's registers, times the SM
@@ -403,6 +538,21 @@ unsigned grid_for(int64_t work_threads) {
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     return static_cast<unsigned>(blocks);
+}
+
+int launch_generic(const Geometry& g, const flexq_config& cfg, const __half* x, uint8_t* codes, uint32_t* meta,
+                   const uint8_t* ccodes, const uint32_t* cmeta, __half* y, cudaStream_t st) {
+    const int64_t items = g.outer * g.ng * g.inner;
+    if (x != nullptr) {
+        const unsigned grid = grid_for<compress_generic_kernel>(items);
+        compress_generic_kernel<<<grid, kThreads, 0, st>>>(x, codes, meta, g.outer, g.G, g.ng, g.inner,
+                                                           cfg.group_size, cfg.num_bits, cfg.symmetric);
+    } else {
+        const unsigned grid = grid_for<decompress_generic_kernel>(items);
+        decompress_generic_kernel<<<grid, kThreads, 0, st>>>(ccodes, cmeta, y, g.outer, g.G, g.ng, g.inner,
+                                                             cfg.group_size, cfg.num_bits, cfg.symmetric);
+    }
+    return launch_status();
 }
 
 template <int BITS, int GS>
@@ -455,7 +605,7 @@ extern "C" int64_t flexq_codes_bytes(int32_t ndim, const int64_t* shape, flexq_c
     Geometry g;
     const int rc = validate(ndim, shape, cfg, g);
     if (rc != FLEX_OK) return rc;
-    return g.n * cfg.num_bits / 8;
+    return g.outer * g.ng * cfg.group_size * cfg.num_bits / 8 * g.inner;
 }
 
 extern "C" int64_t flexq_meta_bytes(int32_t ndim, const int64_t* shape, flexq_config cfg) {
@@ -477,6 +627,7 @@ extern "C" int flexq_compress(const void* x, int32_t ndim, const int64_t* shape,
     const __half* xh = static_cast<const __half*>(x);
     uint8_t* c = static_cast<uint8_t*>(codes);
     uint32_t* m = static_cast<uint32_t*>(meta);
+    if (g.generic) return launch_generic(g, cfg, xh, c, m, nullptr, nullptr, nullptr, st);
 #define CALL_C(B, S) launch_compress<B, S>(g, xh, c, m, st)
     if (cfg.num_bits == 4) {
         if (cfg.group_size == 32) return CALL_C(4, 32);
@@ -501,6 +652,7 @@ extern "C" int flexq_decompress(const void* codes, const void* meta, int32_t ndi
     const uint8_t* c = static_cast<const uint8_t*>(codes);
     const uint32_t* m = static_cast<const uint32_t*>(meta);
     __half* yh = static_cast<__half*>(y);
+    if (g.generic) return launch_generic(g, cfg, nullptr, nullptr, nullptr, c, m, yh, st);
 #define CALL_D(B, S) launch_decompress<B, S>(g, c, m, yh, st)
     if (cfg.num_bits == 4) {
         if (cfg.group_size == 32) return CALL_D(4, 32);

@@ -87,6 +87,7 @@ struct GemmParams {
     int nsx, nsc;          // activation / code ring depths
     int xu;                // K chunks per activation stage
     int nacc, acc_stride;  // independent TMEM accumulators and their column spacing
+    int nslot, a_col0;     // gemm_tc2_kernel: A slots (one chunk per tile) and their first TMEM column
     // K splits (splits > 1): cluster = 1 reduces them through distributed shared memory
     // inside one thread-block cluster per tile; cluster = 0 through fp32 partials in the
     // workspace, the last CTA of a tile (atomic ticket) finishing it
@@ -709,6 +710,413 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------------------------------
+// 256 weight rows per CTA (two 128-row tiles, t = 0, 1), for N a multiple of 256 and up
+// to 192 activation rows per tile (BN). Each activation tile brought in from L2 then
+// feeds both weight tiles, which halves the activation traffic per weight row: with 128
+// rows per CTA the re-read activations, not the weights or the MMAs, set the pace.
+//
+//   warp 0      TMA: code tiles [256 rows][128 B] and metadata [256 rows][4 groups]
+//   warp 1      TMA: activation tiles [BN rows][64] fp16 (128-byte swizzle), XU chunks per stage
+//   warps 2, 3  one thread each issues the MMAs of tile 0 / tile 1 into its own TMEM
+//               accumulator (warp 2 also allocates TMEM)
+//   warps 4-11  warp w dequantises rows 128 t + 32 (w % 4) + lane, t = (w - 4) / 4, one
+//               whole 64-wide K chunk at a time into that tile's A slot in TMEM
+//               (tcgen05.st), then runs the epilogue of the same rows
+//
+// TMEM: accumulator of tile t at columns [t acc_stride, t acc_stride + BN); from a_col0 on,
+// nslot A slots of one chunk per tile (slot s of tile t at a_col0 + (s * 2 + t) * 32). A
+// "unit" is one chunk: one A slot fill, one MMA issue round per tile, one commit per
+// issuer (the mma_done ring counts units). Everything else - bounded waits, abort and
+// drain, split-K through clusters or tickets, the epilogue and the fused store_cache - is
+// as in gemm_tc_kernel.
+constexpr int kRT = 2;                  // 128-row tiles per CTA
+constexpr int kRows2 = kRT * kBM;       // 256
+constexpr int kDoneRing2 = 16;          // mma_done barriers (units)
+
+template <int BITS, bool XPERM>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_constant__ CUtensorMap tm_codes,
+                                                               const __grid_constant__ CUtensorMap tm_meta,
+                                                               const __grid_constant__ CUtensorMap tm_x,
+                                                               const GemmParams p) {
+    constexpr int CROW = kBK * BITS / 8;          // code bytes per row and K chunk (32 or 64)
+    constexpr int KU = 128 / CROW;                // K chunks per code stage (4 or 2)
+    constexpr int CSTAGE = kRows2 * 128;          // code bytes per stage: 256 rows x 128 B
+    constexpr int MSTAGE = kRows2 * kMetaChunks * 4;
+    constexpr int WPC = CROW / 16;                // 16-byte code vectors per row and chunk (2 or 4)
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = tc::smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* const gbase = smem_raw + (base - raw);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kRows2, m0 = blockIdx.y * p.BN, split = blockIdx.z;
+    const int nk_total = p.K / kBK;
+    const int c_begin = split * p.cps;                            // multiple of kMetaChunks
+    const int nk = min(nk_total, c_begin + p.cps) - c_begin;      // chunks = units of this CTA
+    const int nsteps = nk / KU;
+    const int XU = p.xu;
+    const int nxu = nk / XU;
+    const int NSLOT = p.nslot;
+
+    const uint32_t sX = base, sC = base + p.off_c, sM = base + p.off_m;
+    const uint32_t sb = base + p.off_bar;
+    const int NSX = p.nsx, NSC = p.nsc;
+    const uint32_t xbytes = static_cast<uint32_t>(p.BN) * 128;
+    Bars B;
+    B.codes_full = sb;
+    B.codes_empty = B.codes_full + 8 * NSC;
+    B.x_full = B.codes_empty + 8 * NSC;
+    B.a_full = B.x_full + 8 * NSX;
+    B.mma_done = B.a_full + 8 * NSLOT;
+    B.acc_full = B.mma_done + 8 * kDoneRing2;
+    B.drain = B.acc_full + 8;
+    const uint32_t misc = B.drain + 8 * 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (misc - base));
+    volatile int* abort = reinterpret_cast<volatile int*>(gbase + (misc - base) + 4);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(gbase + (misc - base) + 8);
+    uint32_t* kv_red = reinterpret_cast<uint32_t*>(gbase + (misc - base) + 16);   // [8 warps][4 pairs][2]
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSC; ++s) {
+            tc::bar_init(B.codes_full + 8 * s, 1);
+            tc::bar_init(B.codes_empty + 8 * s, kDequantThreads);
+        }
+        for (int s = 0; s < NSX; ++s) tc::bar_init(B.x_full + 8 * s, 1);
+        for (int s = 0; s < NSLOT; ++s) tc::bar_init(B.a_full + 8 * s, kDequantThreads);
+        for (int s = 0; s < kDoneRing2; ++s) tc::bar_init(B.mma_done + 8 * s, kRT);   // both issuers commit each unit
+        tc::bar_init(B.acc_full, kRT);
+        for (int i = 0; i < 4; ++i) tc::bar_init(B.drain + 8 * i, 1);
+        *abort = 0;
+        *last_flag = 0;
+        tc::bar_fence_init();
+    }
+    if (warp == 2) {
+        tc::tmem_alloc(misc, kTmemCols);
+        tc::tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tc::tma_prefetch(&tm_codes);
+        tc::tma_prefetch(&tm_meta);
+    }
+    if (warp == 1 && lane == 0) tc::tma_prefetch(&tm_x);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    // epilogue / dequantisation mapping (warps 4-11): TMEM lane quarter lq, tile tt
+    const int lq = warp & 3, tt = (warp - 4) >> 2;
+    const int row = tt * kBM + lq * 32 + lane;                    // row of the CTA's 256
+    const int n = n0 + row;
+    const int n0t = n0 + tt * kBM;                                // first row of this thread's tile
+    const float scale_n = n < p.nq ? p.qscale : 1.f;
+    const int n_out = p.yperm ? ((n & ~7) | ((n & 3) << 1) | ((n >> 2) & 1)) : n;
+    const bool kv_on = p.kv.codes[0][0] != nullptr && n0t >= p.kv.h;
+    float bias_n = 0.f;
+    uint32_t all_ok = 0;
+    auto finish8 = [&](int col, const float (&v)[8]) {
+        float r[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int m = m0 + col + j;
+            r[j] = (p.residual && m < p.M) ? __half2float(p.residual[static_cast<int64_t>(m) * p.N + n]) : 0.f;
+        }
+        __half o16[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int m = m0 + col + j;
+            float x = (v[j] + bias_n) * scale_n;
+            if (p.relu) x = fmaxf(x, 0.f);
+            o16[j] = __float2half_rn(x + r[j]);
+            if (m < p.M) p.y[static_cast<int64_t>(m) * p.N + n_out] = o16[j];
+        }
+        if (kv_on) kv_store8(p, o16, col, m0, n0t, n, warp, lane, kv_red);
+    };
+
+    if (warp == 0) {
+        // ---------------- code + metadata producer: one stage = KU chunks of 256 rows ----------------
+        if (lane == 0) {
+            if (!p.early_w) pdl_wait();
+            int st = 0, s = 0;
+            uint32_t ph = 0;
+            for (; st < nsteps; ++st) {
+                if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ph ^ 1, abort, p.status, p.wait_ns)) break;
+                const int c = c_begin + st * KU;
+                tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CSTAGE + MSTAGE);
+                tc::tma_load_2d(sC + s * CSTAGE, &tm_codes, c * CROW, n0, B.codes_full + 8 * s);
+                tc::tma_load_2d(sM + s * MSTAGE, &tm_meta, c & ~(kMetaChunks - 1), n0, B.codes_full + 8 * s);
+                if (++s == NSC) { s = 0; ph ^= 1; }
+            }
+            for (int s2 = 0; s2 < NSC && s2 < st; ++s2) {
+                const int last = s2 + ((st - 1 - s2) / NSC) * NSC;
+                volatile int never = 0;
+                tc::bar_wait(B.codes_full + 8 * s2, (last / NSC) & 1, &never, p.status);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- activation producer: one stage = XU chunks ----------------
+        if (lane == 0) {
+            pdl_wait();
+            int u = 0, s = 0;
+            for (; u < nxu; ++u) {
+                if (u >= NSX) {
+                    // the stage last held chunks [(u - NSX) XU, +XU): wait for the MMAs of its last unit
+                    const int ul = (u - NSX) * XU + XU - 1;
+                    if (!tc::bar_wait(B.mma_done + 8 * (ul % kDoneRing2), (ul / kDoneRing2) & 1, abort, p.status,
+                                      p.wait_ns))
+                        break;
+                }
+                tc::bar_arrive_expect_tx(B.x_full + 8 * s, XU * xbytes);
+                for (int c = 0; c < XU; ++c)
+                    tc::tma_load_2d(sX + (s * XU + c) * xbytes, &tm_x, (c_begin + u * XU + c) * kBK, m0,
+                                    B.x_full + 8 * s);
+                if (++s == NSX) s = 0;
+            }
+            const int issued = u;
+            for (int s2 = 0; s2 < NSX && s2 < issued; ++s2) {
+                const int last = s2 + ((issued - 1 - s2) / NSX) * NSX;
+                volatile int never = 0;
+                tc::bar_wait(B.x_full + 8 * s2, (last / NSX) & 1, &never, p.status);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2 || warp == 3) {
+        // ---------------- MMA issuers: warp 2 tile 0, warp 3 tile 1 ----------------
+        const int t = warp - 2;
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_f16_f32(kBM, p.BN);
+            const uint32_t d_acc = tmem + static_cast<uint32_t>(t * p.acc_stride);
+            int xs = 0, xc = 0;                 // activation stage and chunk within it
+            uint32_t xph = 0;
+            bool ok = true;
+            int u = 0;
+            for (; u < nk; ++u) {
+                const int sa = u % NSLOT;
+                if (!tc::bar_wait(B.a_full + 8 * sa, (u / NSLOT) & 1, abort, p.status, p.wait_ns)) { ok = false; break; }
+                if (xc == 0 && !tc::bar_wait(B.x_full + 8 * xs, xph, abort, p.status, p.wait_ns)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint32_t a_tm = tmem + static_cast<uint32_t>(p.a_col0 + (sa * kRT + t) * 32);
+                const uint64_t bd = tc::desc_k_sw128(sX + static_cast<uint32_t>(xs * XU + xc) * xbytes);
+                issue_ksteps<1>(d_acc, a_tm, bd, idesc, 0, u == 0);
+                if (++xc == XU) {
+                    xc = 0;
+                    if (++xs == NSX) { xs = 0; xph ^= 1; }
+                }
+                tc::mma_commit(u + 1 < nk ? B.mma_done + 8 * (u % kDoneRing2) : B.acc_full);
+            }
+            volatile int never = 0;
+            const int committed = ok ? nk - 1 : u;
+            if (!ok) {
+                tc::mma_commit(B.drain + 8 * t);
+                tc::bar_wait(B.drain + 8 * t, 0, &never, p.status);
+            }
+            for (int c = committed - kDoneRing2 > 0 ? committed - kDoneRing2 : 0; c < committed; ++c)
+                tc::bar_wait(B.mma_done + 8 * (c % kDoneRing2), (c / kDoneRing2) & 1, &never, p.status);
+            if (ok) tc::bar_wait(B.acc_full, 0, &never, p.status);
+        }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 12) {
+        // ---------------- dequantisation into TMEM, one chunk (unit) at a time ----------------
+        const int sw = row & 7;
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(lq * 32) << 16);
+        bool ok = true;
+        int s = 0;
+        uint32_t cph = 0;
+        for (int st = 0; st < nsteps && ok; ++st) {
+            if (!tc::bar_wait(B.codes_full + 8 * s, cph, abort, p.status, p.wait_ns)) { ok = false; break; }
+            const uint32_t crow = sC + s * CSTAGE + row * 128;
+            uint4 cw[KU][WPC];
+#pragma unroll
+            for (int c = 0; c < KU; ++c)
+#pragma unroll
+                for (int v = 0; v < WPC; ++v) cw[c][v] = tc::lds128(crow + (((c * WPC + v) ^ sw) << 4));
+            const uint4 mrow = tc::lds128(sM + s * MSTAGE + row * 16);
+            const int moff = (c_begin + st * KU) & (kMetaChunks - 1);
+#pragma unroll
+            for (int c = 0; c < KU; ++c) {
+                const int u = st * KU + c;
+                const int sa = u % NSLOT;
+                if (u >= NSLOT) {
+                    const int pu = u - NSLOT;
+                    if (!tc::bar_wait(B.mma_done + 8 * (pu % kDoneRing2), (pu / kDoneRing2) & 1, abort, p.status,
+                                      p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                }
+                const int mi = (moff + c) & 3;
+                const uint32_t mw = mi == 0 ? mrow.x : (mi == 1 ? mrow.y : (mi == 2 ? mrow.z : mrow.w));
+                const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
+                const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
+                const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
+                const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
+                const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
+                const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
+                const uint32_t a_col = p.a_col0 + (sa * kRT + tt) * 32;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {          // two halves of the chunk: 32 values each
+                    uint32_t r[16];
+                    if (BITS == 4) {
+                        const uint4 q = cw[c][hh];
+                        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2) : dequant8_4bit(w[j], step2, mnv2);
+                            r[4 * j] = v.x;
+                            r[4 * j + 1] = v.y;
+                            r[4 * j + 2] = v.z;
+                            r[4 * j + 3] = v.w;
+                        }
+                    } else {
+                        const uint4 q0 = cw[c][2 * hh], q1 = cw[c][2 * hh + 1];
+                        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint4 v;
+                            if (XPERM) {
+                                v = dequant8_8bit_il(w[2 * j], w[2 * j + 1], step2, mnv2);
+                            } else {
+                                const uint2 a = dequant4_8bit(w[2 * j], step2, mnv2);
+                                const uint2 b = dequant4_8bit(w[2 * j + 1], step2, mnv2);
+                                v = make_uint4(a.x, a.y, b.x, b.y);
+                            }
+                            r[4 * j] = v.x;
+                            r[4 * j + 1] = v.y;
+                            r[4 * j + 2] = v.z;
+                            r[4 * j + 3] = v.w;
+                        }
+                    }
+                    tc::tmem_st16(t_lane + a_col + hh * 16, r);
+                }
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                tc::bar_arrive(B.a_full + 8 * sa);
+            }
+            if (!ok) break;
+            // every value of the code stage has been used: the next TMA may refill it
+            tc::bar_arrive(B.codes_empty + 8 * s);
+            if (++s == NSC) { s = 0; cph ^= 1; }
+        }
+        // ---------------- epilogue ----------------
+        pdl_wait();
+        pdl_trigger();
+        bias_n = p.bias ? __half2float(p.bias[n]) : 0.f;
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (ok && !*abort) ok = tc::bar_wait(B.acc_full, 0, abort, p.status);
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\t"
+            "setp.ne.u32 p, %1, 0;\n\t"
+            "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
+            "selp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(all_ok)
+            : "r"((ok && !*abort) ? 1u : 0u)
+            : "memory");
+        const uint32_t taddr = t_lane + static_cast<uint32_t>(tt * p.acc_stride);
+        if (all_ok) {
+            tc::fence_after_sync();
+            if (p.splits == 1) {
+                for (int col = 0; col < p.BN; col += 8) {
+                    float v[8];
+                    tc::tmem_ld8(taddr + col, v);
+                    finish8(col, v);
+                }
+            } else if (p.cluster) {
+                // this split's fp32 partial [BN][256] into this CTA's shared memory (the rings
+                // are drained: every copy has landed and every MMA has completed)
+                for (int col = 0; col < p.BN; col += 8) {
+                    float v[8];
+                    tc::tmem_ld8(taddr + col, v);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) tc::st_shared_f32(base + ((col + j) * kRows2 + row) * 4, v[j]);
+                }
+            } else {
+                float* mine = p.part + (static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * p.splits + split) *
+                                           p.BN * kRows2;
+                for (int col = 0; col < p.BN; col += 8) {
+                    float v[8];
+                    tc::tmem_ld8(taddr + col, v);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) mine[(col + j) * kRows2 + row] = v[j];
+                }
+            }
+        }
+        if (p.splits > 1 && !p.cluster) {
+            // ticket, taken by every split (see gemm_tc_kernel); the last adds the partials in split order
+            const int et = (warp - 4) * 32 + lane;
+            const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+            __threadfence();
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (et == 0) *last_flag = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (*last_flag) {
+                __threadfence();
+                if (all_ok) {
+                    const float* all = p.part + static_cast<int64_t>(tile) * p.splits * p.BN * kRows2;
+                    for (int col = 0; col < p.BN; col += 8) {
+                        float acc[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+                        for (int s0 = 0; s0 < p.splits; s0 += 8) {
+                            float tv[8][8];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    tv[u][j] = (s0 + u < p.splits)
+                                                   ? __ldcg(all + (static_cast<int64_t>(s0 + u) * p.BN + col + j) * kRows2 + row)
+                                                   : 0.f;
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) acc[j] += tv[u][j];
+                        }
+                        finish8(col, acc);
+                    }
+                }
+                if (et == 0) p.counters[tile] = 0;
+            }
+        }
+    }
+
+    if (p.splits > 1 && p.cluster) {
+        // split-K across the cluster: CTA r finishes the 8-column groups v = r, r + S, ...
+        // of every row, adding the splits' partials in split order; the second barrier keeps
+        // each CTA's shared memory alive until its peers are done. All threads of every CTA
+        // take part in both barriers.
+        tc::cluster_sync();
+        if (warp >= 4 && warp < 12 && all_ok) {
+            const int S = p.splits;
+            const int rank = static_cast<int>(tc::cluster_rank());
+            for (int v = rank; v < p.BN / 8; v += S) {
+                const int col = v * 8;
+                float acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+                for (int sp = 0; sp < S; ++sp) {
+                    const uint32_t peer = tc::map_peer(base + (col * kRows2 + row) * 4, static_cast<uint32_t>(sp));
+                    float tv[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) tv[j] = tc::ld_peer_f32(peer + j * kRows2 * 4);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[j] += tv[j];
+                }
+                finish8(col, acc);
+            }
+        }
+        tc::cluster_sync();
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 2) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // Small-batch path (up to 32 activation rows, 4-bit weights): dequant-fused GEMV on
 // mma.sync m16n8k16.
 //
@@ -1143,16 +1551,19 @@ EncodeTiledFn encode_fn() {
 
 // Thread-block clusters of `splits` CTAs of this kernel that can be resident at once on
 // the current device (cached per device and size); 0 if the query fails.
-int max_active_clusters(int splits, uint32_t smem) {
-    static std::map<std::tuple<int, int, uint32_t>, int> cache;
+int max_active_clusters(int splits, uint32_t smem, bool rows256 = false) {
+    static std::map<std::tuple<int, int, uint32_t, bool>, int> cache;
     static std::mutex mu;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
     std::lock_guard<std::mutex> lock(mu);
-    const auto key = std::make_tuple(dev, splits, smem);
+    const auto key = std::make_tuple(dev, splits, smem, rows256);
     const auto it = cache.find(key);
     if (it != cache.end()) return it->second;
+    const void* kfn = rows256 ? reinterpret_cast<const void*>(gemm_tc2_kernel<4, true>)
+                              : reinterpret_cast<const void*>(gemm_tc_kernel<4, true>);
     set_smem_once(gemm_tc_kernel<4, true>, 227 * 1024);
+    set_smem_once(gemm_tc2_kernel<4, true>, 227 * 1024);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1, 1, splits);
     cfg.blockDim = dim3(kThreads);
@@ -1165,12 +1576,102 @@ int max_active_clusters(int splits, uint32_t smem) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<4, true>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess) {
         cudaGetLastError();
         n = 0;
     }
     cache[key] = n;
     return n;
+}
+
+// K splits per tile: the count whose waves of (tile, split) units take the least time,
+// one unit costing its K steps plus a fixed overhead (prologue, pipeline fill, epilogue;
+// more when partials must be added). One CTA per SM.
+int choose_splits(int tiles, int nk, int bits) {
+    const int sms = sm_count();
+    int max_splits = nk / kMetaChunks;
+    if (max_splits > kMaxSplits) max_splits = kMaxSplits;
+    if (max_splits < 1) max_splits = 1;
+    const double steps_total = static_cast<double>(nk) / (128 / (kBK * bits / 8));
+    int splits = 1;
+    double best = 0.0;
+    for (int s = 1; s <= max_splits; ++s) {
+        if (s > 1 && tiles > static_cast<int>(kTicketBytes / sizeof(int))) break;   // one ticket per tile
+        const int64_t units = static_cast<int64_t>(tiles) * s;
+        const int64_t waves = (units + sms - 1) / sms;
+        const double t = static_cast<double>(waves) * (steps_total / s + (s > 1 ? 5.0 : 3.0));
+        if (s == 1 || t < best * 0.97) {
+            best = t;
+            splits = s;
+        }
+    }
+    return splits;
+}
+
+struct Plan2 {
+    int BN, tiles_n, tiles_m, splits, cps, nsx, nsc, xu, nslot, acc_stride, a_col0, cluster;
+    uint32_t off_c, off_m, off_bar, smem;
+    int64_t ws_bytes, counters_bytes;
+};
+
+// gemm_tc2_kernel serves every weight with N a multiple of 256 (two 128-row tiles per
+// CTA); its activation tile is at most 192 rows (M <= 192 in one tile, else tiles of 128).
+bool tc2_eligible(int N) {
+#ifdef FLEXQ_GEMM_ROWS128_ONLY
+    (void)N;
+    return false;
+#else
+    return N % kRows2 == 0;
+#endif
+}
+
+Plan2 make_plan2(int M, int N, int K, int bits) {
+    Plan2 P{};
+    P.BN = M <= 192 ? ((M + 15) / 16) * 16 : 128;
+    if (P.BN < 16) P.BN = 16;
+    P.tiles_n = N / kRows2;
+    P.tiles_m = (M + P.BN - 1) / P.BN;
+    const int nk = K / kBK;
+    const int tiles = P.tiles_n * P.tiles_m;
+    int splits = choose_splits(tiles, nk, bits);
+    int cps = (nk + splits - 1) / splits;
+    cps = ((cps + kMetaChunks - 1) / kMetaChunks) * kMetaChunks;
+    P.splits = (nk + cps - 1) / cps;
+    P.cps = cps;
+    P.acc_stride = ((P.BN + 31) / 32) * 32;
+    P.a_col0 = kRT * P.acc_stride;
+    P.nslot = (kTmemCols - P.a_col0) / (kRT * 32);
+    // shared memory: code stages (256 rows x 128 B + metadata) and activation stages of
+    // XU chunks (BN rows x 128 B each), within about 220 KB
+    const int ku = 128 / (kBK * bits / 8);
+    const uint32_t cstage = kRows2 * 128 + kRows2 * kMetaChunks * 4;
+    int xu = ku;
+    while (xu > 1 && static_cast<uint32_t>(xu) * P.BN * 128 > 56u * 1024u) xu >>= 1;
+    const uint32_t xstage = static_cast<uint32_t>(xu) * P.BN * 128;
+    const uint32_t budget = 220u * 1024u;
+    int nsc = 3;
+    int nsx = static_cast<int>((budget - nsc * cstage) / xstage);
+    if (nsx < 2) {
+        nsc = 2;
+        nsx = static_cast<int>((budget - nsc * cstage) / xstage);
+    }
+    if (nsx > 6) nsx = 6;
+    P.xu = xu;
+    P.nsx = nsx;
+    P.nsc = nsc;
+    P.off_c = nsx * xstage;
+    P.off_m = P.off_c + nsc * kRows2 * 128;
+    P.off_bar = P.off_m + nsc * kRows2 * kMetaChunks * 4;
+    P.smem = P.off_bar + 8 * (2 * nsc + nsx + P.nslot + kDoneRing2 + 1 + 4) + 16 + 256 + 1024;
+    // split-K through distributed shared memory when the partial tile fits in the drained
+    // rings and every tile's cluster can be resident at once, else workspace and tickets
+    const bool fits = static_cast<uint32_t>(P.BN) * kRows2 * 4 <= P.off_bar;
+    P.cluster = (P.splits > 1 && fits && max_active_clusters(P.splits, P.smem, true) >= tiles) ? 1 : 0;
+    P.counters_bytes = kTicketBytes;
+    P.ws_bytes = (P.splits > 1 && !P.cluster)
+                     ? P.counters_bytes + static_cast<int64_t>(tiles) * P.splits * P.BN * kRows2 * 4
+                     : 0;
+    return P;
 }
 
 struct Plan {
@@ -1187,27 +1688,7 @@ Plan make_plan(int M, int N, int K, int bits) {
     P.tiles_m = (M + P.BN - 1) / P.BN;
     const int nk = K / kBK;
     const int tiles = P.tiles_n * P.tiles_m;
-    const int sms = sm_count();
-    int max_splits = nk / kMetaChunks;
-    if (max_splits > kMaxSplits) max_splits = kMaxSplits;
-    if (max_splits < 1) max_splits = 1;
-    // K splits per tile: the count whose waves of (tile, split) units take the least
-    // time, one unit costing its K steps plus a fixed overhead (prologue, pipeline fill,
-    // epilogue; more when partials must be added), so that a grid of 96 tiles on 148
-    // SMs is not left at 65% occupancy. One CTA per SM.
-    const double steps_total = static_cast<double>(nk) / (128 / (kBK * bits / 8));
-    int splits = 1;
-    double best = 0.0;
-    for (int s = 1; s <= max_splits; ++s) {
-        if (s > 1 && tiles > static_cast<int>(kTicketBytes / sizeof(int))) break;   // one ticket per tile
-        const int64_t units = static_cast<int64_t>(tiles) * s;
-        const int64_t waves = (units + sms - 1) / sms;
-        const double t = static_cast<double>(waves) * (steps_total / s + (s > 1 ? 5.0 : 3.0));
-        if (s == 1 || t < best * 0.97) {
-            best = t;
-            splits = s;
-        }
-    }
+    int splits = choose_splits(tiles, nk, bits);
     int cps = (nk + splits - 1) / splits;
     cps = ((cps + kMetaChunks - 1) / kMetaChunks) * kMetaChunks;
     splits = (nk + cps - 1) / cps;
@@ -1329,7 +1810,8 @@ int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, 
 }
 
 int64_t gemm_ws_bytes(int M, int N, int K, int bits) {
-    return gemv_eligible(M, N, bits) ? gemv_plan(M, N, K).ws_bytes : make_plan(M, N, K, bits).ws_bytes;
+    if (gemv_eligible(M, N, bits)) return gemv_plan(M, N, K).ws_bytes;
+    return tc2_eligible(N) ? make_plan2(M, N, K, bits).ws_bytes : make_plan(M, N, K, bits).ws_bytes;
 }
 
 namespace {
@@ -1392,6 +1874,88 @@ int gemv_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
 }
 }  // namespace
 
+namespace {
+// The 256-row tensor-core GEMM (gemm_tc2_kernel); same arguments as gemm_launch.
+int gemm2_launch(const void* x, const flexq_tensor* W, const void* bias, const void* residual, void* y, int M,
+                 int relu, int nq, float qscale, bool xperm, bool yperm, void* ws, int64_t ws_bytes, cudaStream_t st,
+                 const KvFuse* kv, bool early_w) {
+    const int N = static_cast<int>(W->shape[0]), K = static_cast<int>(W->shape[1]);
+    const int bits = W->cfg.num_bits;
+    const Plan2 P = make_plan2(M, N, K, bits);
+    if (P.ws_bytes > 0 && (ws == nullptr || ws_bytes < P.ws_bytes)) return FLEX_ERR_WORKSPACE;
+    CUtensorMap tm_codes, tm_meta, tm_x;
+    // code tiles: 256 rows x 128 bytes (4 K chunks at 4 bits, 2 at 8 bits), 128-byte swizzle
+    int rc = make_tmap_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, static_cast<uint64_t>(K) * bits / 8,
+                          N, static_cast<uint64_t>(K) * bits / 8, 128, kRows2, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != FLEX_OK) return rc;
+    rc = make_tmap_2d(&tm_meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, W->meta, K / kBK, N,
+                      static_cast<uint64_t>(K / kBK) * 4, kMetaChunks, kRows2, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc != FLEX_OK) return rc;
+    rc = make_tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, static_cast<uint64_t>(K) * 2, kBK, P.BN,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != FLEX_OK) return rc;
+    GemmParams gp{};
+    gp.wait_ns = pipeline_wait_ns();
+    gp.bias = static_cast<const __half*>(bias);
+    gp.residual = static_cast<const __half*>(residual);
+    gp.y = static_cast<__half*>(y);
+    gp.status = status_word();
+    gp.M = M;
+    gp.N = N;
+    gp.K = K;
+    gp.BN = P.BN;
+    gp.splits = P.splits;
+    gp.cps = P.cps;
+    gp.nq = nq;
+    gp.qscale = qscale;
+    gp.relu = relu;
+    gp.early_w = early_w ? 1 : 0;
+    gp.yperm = yperm ? 1 : 0;
+    gp.nsx = P.nsx;
+    gp.nsc = P.nsc;
+    gp.xu = P.xu;
+    gp.cluster = P.cluster;
+    gp.counters = static_cast<int*>(ws);
+    gp.part = reinterpret_cast<float*>(static_cast<char*>(ws) + P.counters_bytes);
+    gp.nacc = 1;
+    gp.acc_stride = P.acc_stride;
+    gp.nslot = P.nslot;
+    gp.a_col0 = P.a_col0;
+    gp.off_x = 0;
+    gp.off_c = P.off_c;
+    gp.off_m = P.off_m;
+    gp.off_bar = P.off_bar;
+    gp.tmem_cols = kTmemCols;
+    fill_kv_target(gp.kv, kv);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(P.tiles_n, P.tiles_m, P.splits);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = P.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = P.splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.cluster ? 2 : 1;
+#define GEMM2_LAUNCH(B_, XP_)                                                                \
+    do {                                                                                     \
+        set_smem_once(gemm_tc2_kernel<B_, XP_>, 227 * 1024);                                 \
+        cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<B_, XP_>, tm_codes, tm_meta, tm_x, gp);     \
+    } while (0)
+    if (bits == 4) {
+        if (xperm) GEMM2_LAUNCH(4, true); else GEMM2_LAUNCH(4, false);
+    } else {
+        if (xperm) GEMM2_LAUNCH(8, true); else GEMM2_LAUNCH(8, false);
+    }
+#undef GEMM2_LAUNCH
+    return launch_status();
+}
+}  // namespace
+
 int validate_weight(const flexq_tensor* W) {
     FLEX_REQUIRE(W != nullptr && W->codes && W->meta, FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(W->ndim == 2, FLEX_ERR_INVALID_ARG);
@@ -1416,6 +1980,8 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     // small batches of int4 weights: the register-dequant GEMV on mma.sync
     if (gemv_eligible(M, N, bits))
         return gemv_launch(x, W, bias, residual, y, M, relu, nq, qscale, xperm, yperm, ws, ws_bytes, st, kv, early_w);
+    if (tc2_eligible(N))
+        return gemm2_launch(x, W, bias, residual, y, M, relu, nq, qscale, xperm, yperm, ws, ws_bytes, st, kv, early_w);
     const Plan P = make_plan(M, N, K, bits);
     if (P.ws_bytes > 0 && (ws == nullptr || ws_bytes < P.ws_bytes)) return FLEX_ERR_WORKSPACE;
     CUtensorMap tm_codes, tm_meta, tm_x;

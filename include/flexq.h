@@ -41,10 +41,10 @@ extern "C" {
 /* ---- status codes ------------------------------------------------------------ */
 #define FLEX_OK               0
 #define FLEX_ERR_INVALID_ARG (-1)  /* null pointer, negative size, bad rank       */
-#define FLEX_ERR_UNSUPPORTED (-2)  /* bits not 4/8, group not 32/64/128,
-                                      symmetric != 0, head_dim not 64/128, ...    */
-#define FLEX_ERR_SHAPE       (-3)  /* dim not a multiple of group_size,
-                                      pos >= max_seq, seq > max_seq, ...          */
+#define FLEX_ERR_UNSUPPORTED (-2)  /* bits not 3/4/8 (4/8 outside the codec), group
+                                      not 32/64/128, head_dim not 64/128, ...     */
+#define FLEX_ERR_SHAPE       (-3)  /* a weight or cache dim not a multiple of the
+                                      group, pos >= max_seq, seq > max_seq, ...   */
 #define FLEX_ERR_ALIGN       (-4)  /* pointer not 16-byte aligned                 */
 #define FLEX_ERR_WORKSPACE   (-5)  /* workspace missing or too small              */
 #define FLEX_ERR_CUDA        (-6)  /* a CUDA launch or runtime call failed        */
@@ -55,10 +55,10 @@ extern "C" {
 
 /* ---- compression configuration (CompressionConfig of section 6.3) ------------ */
 typedef struct {
-    int32_t num_bits;    /* 4 or 8                                                 */
+    int32_t num_bits;    /* 4 or 8; the codec (flexq_*) also takes 3                */
     int32_t group_size;  /* 32, 64 or 128                                          */
     int32_t group_dim;   /* dimension the groups run along; negative counts back  */
-    int32_t symmetric;   /* must be 0: the min/max (asymmetric) form               */
+    int32_t symmetric;   /* 0: the min/max form; 1 (codec only): the absmax form   */
 } flexq_config;
 
 /* A compressed tensor: the pages' (data, scale, config) triple.
@@ -88,12 +88,26 @@ int64_t flexq_meta_bytes(int32_t ndim, const int64_t* shape, flexq_config cfg);
  *   65504 on overflow); q = clamp(rint((x - min) * scale16), 0, 2^b - 1), the
  *   subtraction and the product each rounded in fp32, ties to even.
  * Bit-exact and deterministic. Any rank 1..4; the group dimension may be the
- * contiguous one or a strided one. Tensors of any size (64-bit indexing). */
+ * contiguous one or a strided one. Tensors of any size (64-bit indexing).
+ * Variants (readings of what the pages only name: the symmetric flag and num_groups of
+ * the configuration, section 6.3; "int3/int4" on the hub page «FlexLLMGen»):
+ *   - num_bits 3: the codes of a group form a little-endian bit stream, code j in bits
+ *     [3j, 3j+3) of the group's gs*3/8 bytes;
+ *   - symmetric 1: B = 2^(b-1) - 1, scale16 = fp16(B / max|x|) (0 for an all-zero group,
+ *     65504 on overflow), signed code clamp(rint(x * scale16), -B, B) stored as code + B,
+ *     meta {0, scale16};
+ *   - a group_dim extent that is not a multiple of group_size: ceil(extent / group_size)
+ *     groups, the last one zero-padded (the padding takes part in min/max and its codes
+ *     are stored; codes and meta are sized for the padded extent).
+ * These variants run one thread per group (correct for any layout, not tuned); the
+ * layer calls take only 4- and 8-bit min/max tensors. */
 int flexq_compress(const void* x, int32_t ndim, const int64_t* shape, flexq_config cfg,
                    void* codes, void* meta, void* stream);
 
 /* decompress: codes + meta -> y (fp16, `shape`):
- *   y = fp16(fp32(fp32(q * fp32(1/scale16)) + min)), or y = min when scale16 == 0. */
+ *   y = fp16(fp32(fp32(q * fp32(1/scale16)) + min)), or y = min when scale16 == 0;
+ *   symmetric: y = fp16(fp32((u - B) * fp32(1/scale16))), 0 when scale16 == 0.
+ * A zero-padded last group writes only the real elements. */
 int flexq_decompress(const void* codes, const void* meta, int32_t ndim, const int64_t* shape,
                      flexq_config cfg, void* y, void* stream);
 
@@ -175,6 +189,33 @@ int flex_prefill_layer_batches(const flex_layer* L, const flex_kv_cache* caches,
 int flex_decode_layer_batches(const flex_layer* L, const flex_kv_cache* caches, int32_t num_batches,
                               const void* x_in, void* x_out, int32_t batch, int32_t pos, void* ws,
                               int64_t ws_bytes, void* stream);
+
+/* ---- the whole model around the layers: embedding, output head, greedy choice --- */
+/* The source-notes page «FlexGen» (PtirisNote), "Flex Opt": the model is an embedding,
+ * N transformer layers and an output head (OptLM.generate runs the loop); "Pytorch
+ * Backend": opt_input_embed / opt_output_embed are the embedding layers. The walkthrough
+ * page, section 4.1: generate(..., do_sample, ...); do_sample = False is greedy.
+ * E: the token table, fp16 [V_pad][h] compressed with {4 bits, group 64, group_dim 1}
+ * like the layer weights (V_pad a multiple of 128 and h of 256; rows >= vocab are
+ * padding that no token uses); it is also the output head (logits = LN(h) E^T). */
+
+/* x[r] = fp16(E^[tokens[r]] + P[positions[r]]), r < n: E^ the codec's dequantisation of
+ * the table row, P an fp16 position table [max_pos][h]; the sum of the two fp16 values
+ * is rounded once. tokens, positions: device int32 [n]; x: fp16 [n][h]. An id outside
+ * [0, vocab) or a position outside [0, max_pos) is clamped into range and reported as
+ * FLEX_ERR_INVALID_ARG by flex_get_status. */
+int flex_embed(const flexq_tensor* E, int32_t vocab, const void* P, int32_t max_pos,
+               const int32_t* tokens, const int32_t* positions, int64_t n, void* x, void* stream);
+
+/* Output head and greedy choice for n rows x (fp16 [n][h], natural order):
+ * logits = LN(x; lnf_g, lnf_b) E^T (eps 1e-5), next[r] = the column of the largest
+ * logit among columns [0, vocab), the lowest column among equal fp16 values. next:
+ * device int32 [n]. logits: fp16 [n][V_pad] to keep them, or NULL (then they live in
+ * the workspace). ws: flex_lm_head_ws_bytes(E, vocab, n, logits != NULL) bytes. */
+int64_t flex_lm_head_ws_bytes(const flexq_tensor* E, int32_t vocab, int64_t n, int32_t with_logits);
+int flex_lm_head_argmax(const flexq_tensor* E, int32_t vocab, const void* lnf_g, const void* lnf_b,
+                        const void* x, int64_t n, int32_t* next, void* logits, void* ws,
+                        int64_t ws_bytes, void* stream);
 
 /* ---- hot-path steps, callable one by one ------------------------------------- */
 

@@ -81,6 +81,28 @@ def layer_params(h: int, ffn: int, seed: int, device="cpu") -> dict:
     return p
 
 
+OPT_VOCAB = 50272     # token ids of the OPT family's tokenizer
+
+
+def model_params(vocab: int, h: int, max_pos: int, seed: int, vocab_pad: int = None, device="cpu") -> dict:
+    """Token table E [vocab_pad][h] (rows >= vocab zero: padding no token uses), position
+    table P [max_pos][h], both N(0, 0.02) fp16, and the final LayerNorm's gain
+    1 + N(0, 0.02) and bias N(0, 0.02)."""
+    s = int(seed) * 1000 + 900
+    vocab_pad = vocab_pad or vocab
+    E = torch.zeros((vocab_pad, h), dtype=torch.float16, device=device)
+    E[:vocab] = normal_f16((vocab, h), s + 1, WEIGHT_STD, device=device)
+    return {"E": E, "P": normal_f16((max_pos, h), s + 2, WEIGHT_STD, device=device),
+            "lnf_g": normal_f16((h,), s + 3, PARAM_STD, mean=1.0, device=device),
+            "lnf_b": normal_f16((h,), s + 4, PARAM_STD, device=device)}
+
+
+def token_ids(shape, vocab: int, seed: int, device="cpu") -> torch.Tensor:
+    """Uniform token ids in [0, vocab), int32."""
+    g = _gen(int(seed) * 1000 + 950, device)
+    return torch.randint(0, int(vocab), tuple(shape), generator=g, device=device, dtype=torch.int64).to(torch.int32)
+
+
 def activations(shape, seed: int, device="cpu") -> torch.Tensor:
     """Layer input activations, N(0, 1) fp16."""
     return normal_f16(shape, int(seed) * 1000 + 500, 1.0, device=device)
@@ -140,5 +162,6 @@ def ceil_div(a: int, b: int) -> int:
 
 __all__ = [
     "WORKLOADS", "normal_f16", "layer_params", "activations", "decode_inputs",
-    "kv_history", "codec_tensor", "codec_rows_for_bytes", "ceil_div", "math",
+    "kv_history", "codec_tensor", "codec_rows_for_bytes", "ceil_div", "math", "OPT_VOCAB", "model_params",
+    "token_ids",
 ]

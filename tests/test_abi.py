@@ -39,10 +39,15 @@ def test_size_queries():
     assert L.flexq_meta_bytes(2, _shape((4096, 4096)), cfg) == 4096 * 64 * 4
     assert L.flexq_codes_bytes(2, _shape((64, 96)), fq.config(8, 32, 0)) == 64 * 96
     assert L.flexq_meta_bytes(2, _shape((64, 96)), fq.config(8, 32, 0)) == 2 * 96 * 4
-    assert L.flexq_codes_bytes(2, _shape((4, 100)), cfg) == fq.FLEX_ERR_SHAPE
-    assert L.flexq_codes_bytes(2, _shape((4, 128)), fq.config(3, 64, 1)) == fq.FLEX_ERR_UNSUPPORTED
+    # a partial last group is padded: ceil(100 / 64) = 2 groups per row
+    assert L.flexq_codes_bytes(2, _shape((4, 100)), cfg) == 4 * 2 * 64 // 2
+    assert L.flexq_meta_bytes(2, _shape((4, 100)), cfg) == 4 * 2 * 4
+    # 3-bit codes: 3/8 byte per element; the symmetric form has the same sizes
+    assert L.flexq_codes_bytes(2, _shape((4, 128)), fq.config(3, 64, 1)) == 4 * 128 * 3 // 8
+    assert L.flexq_codes_bytes(2, _shape((4, 128)), fq.config(4, 64, 1, 1)) == 4 * 64
+    assert L.flexq_codes_bytes(2, _shape((4, 128)), fq.config(5, 64, 1)) == fq.FLEX_ERR_UNSUPPORTED
     assert L.flexq_codes_bytes(2, _shape((4, 128)), fq.config(4, 48, 1)) == fq.FLEX_ERR_UNSUPPORTED
-    assert L.flexq_codes_bytes(2, _shape((4, 128)), fq.config(4, 64, 1, 1)) == fq.FLEX_ERR_UNSUPPORTED
+    assert L.flexq_codes_bytes(2, _shape((4, 128)), fq.config(4, 64, 1, 2)) == fq.FLEX_ERR_UNSUPPORTED
     assert L.flexq_codes_bytes(5, _shape((4, 128)), cfg) == fq.FLEX_ERR_INVALID_ARG
     assert L.flexq_codes_bytes(2, _shape((4, 128)), fq.config(4, 64, 2)) == fq.FLEX_ERR_INVALID_ARG
     # negative group_dim counts from the back
@@ -58,7 +63,8 @@ def test_codec_argument_errors_are_host_side():
     assert L.flexq_compress(P(4096), 2, shp, cfg, P(4097), P(8192), None) == fq.FLEX_ERR_ALIGN
     assert L.flexq_compress(P(4104), 2, shp, cfg, P(4096), P(8192), None) == fq.FLEX_ERR_ALIGN
     assert L.flexq_decompress(P(4096), P(8192), 2, shp, cfg, P(4100), None) == fq.FLEX_ERR_ALIGN
-    assert L.flexq_compress(P(4096), 2, _shape((4, 96)), cfg, P(4096), P(8192), None) == fq.FLEX_ERR_SHAPE
+    assert L.flexq_compress(P(4096), 2, _shape((4, 96)), fq.config(4, 64, 1, 3), P(4096), P(8192), None) == \
+        fq.FLEX_ERR_UNSUPPORTED
     # an empty tensor is a valid no-op
     assert L.flexq_compress(P(4096), 2, _shape((0, 128)), cfg, P(4096), P(8192), None) == fq.FLEX_OK
 

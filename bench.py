@@ -604,9 +604,10 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
     caches = [cs[0] for cs in stack.caches]
 
     def time_cycle(fn, reps=reps):
-        """ms per call of fn, from a CUDA graph that calls fn once per layer (so the
-        operands rotate through the whole stack and do not stay in L2), replayed
-        `reps` times between two events on the launching stream."""
+        """(ms per call of fn, {kernel: launches per call}), from a CUDA graph that calls
+        fn once per layer (so the operands rotate through the whole stack and do not
+        stay in L2), replayed `reps` times between two events on the launching stream;
+        the kernel names are read from the captured graph (None if it cannot be read)."""
         with torch.cuda.stream(stream):
             for l in range(L):
                 fn(l)
@@ -615,6 +616,8 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
         with torch.cuda.graph(g, stream=stream):
             for l in range(L):
                 fn(l)
+        counts = graph_kernel_counts(g)
+        names = None if counts is None else {short_kernel_name(k): v / L for k, v in counts.items()}
         with torch.cuda.stream(stream):
             g.replay()
         torch.cuda.synchronize()
@@ -627,7 +630,15 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
             e1.record(stream)
         torch.cuda.synchronize()
         del g
-        return e0.elapsed_time(e1) / (reps * L)      # ms per launch(-group)
+        return e0.elapsed_time(e1) / (reps * L), names      # ms per launch(-group)
+
+    def main_kernel(names, expected):
+        """The part's working kernel: its most-launched kernel that is not a combine
+        step (the expected name when the graph could not be read)."""
+        if not names:
+            return expected
+        work = {k: v for k, v in names.items() if "combine" not in k} or names
+        return max(sorted(work), key=lambda k: work[k])
 
     x = synth.activations((b, 3 * h), 5, device=dev)
     x[:, :h] *= d ** -0.5
@@ -642,33 +653,33 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
     # the library splits a (sequence, head) key range over CTAs only when the pairs alone
     # fill fewer than 4 CTAs per SM; then a combine kernel merges the splits
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    attn_launches = 1 if b * nh >= 4 * sms else 2
     kern = {}
+    ms, names = time_cycle(lambda l: fq.flex_decode_attention(caches[l], x[:, :h], x[:, h:], x[:, 2 * h:], 3 * h, o,
+                                                              b, pos, aws, stream=stream))
     kern["decode_attention"] = dict(
-        ms=time_cycle(lambda l: fq.flex_decode_attention(caches[l], x[:, :h], x[:, h:], x[:, 2 * h:], 3 * h, o, b,
-                                                         pos, aws, stream=stream)),
-        bytes=2 * b * pos * h * per + 3 * b * h * 2 + b * h * 2, flops=4.0 * b * (pos + 1) * h,
-        launches_per_call=attn_launches, source=["attention.cu"])
-    gemm_kernel = "gemv_kernel" if b <= 32 else "gemm_tc_kernel"   # the library's dispatch by batch
+        ms=ms, bytes=2 * b * pos * h * per + 3 * b * h * 2 + b * h * 2, flops=4.0 * b * (pos + 1) * h,
+        launches_per_call=int(round(sum(names.values()))) if names else (1 if b * nh >= 4 * sms else 2),
+        kernel=main_kernel(names, "decode_attn_tc_kernel"), kernels=names, source=["attention.cu"])
+    gemm_kernel = "gemv_kernel" if b <= 32 else "gemm_tc_kernel"   # only if the graph cannot be read
     for name, (n, k, xin, yout, epi) in {"gemm_qkv": (3 * h, h, x[:, :h], yq, 0), "gemm_out": (h, h, x[:, :h], o, 0),
                                           "gemm_fc1": (ffn, h, x[:, :h], yf, 1),
                                           "gemm_fc2": (h, ffn, xf, o, 0)}.items():
         wkey = {"gemm_qkv": "w_qkv", "gemm_out": "w_o", "gemm_fc1": "w_fc1", "gemm_fc2": "w_fc2"}[name]
-        kern[name] = dict(
-            # the layer hands every GEMM its activations in the interleaved 8-block order
-            ms=time_cycle(lambda l, xin=xin, yout=yout, epi=epi, wkey=wkey:
-                          fq.flex_dequant_gemm(xin, layers[l].w[wkey], None, None, yout, b,
-                                               epi | fq.FLEX_GEMM_X_INTERLEAVED, gws, stream=stream)),
-            bytes=n * k * per + b * k * 2 + b * n * 2, flops=2.0 * b * n * k, launches_per_call=1,
-            kernel=gemm_kernel, source=["gemm.cu", "tc.cuh"])
+        # the layer hands every GEMM its activations in the interleaved 8-block order
+        ms, names = time_cycle(lambda l, xin=xin, yout=yout, epi=epi, wkey=wkey:
+                               fq.flex_dequant_gemm(xin, layers[l].w[wkey], None, None, yout, b,
+                                                    epi | fq.FLEX_GEMM_X_INTERLEAVED, gws, stream=stream))
+        kern[name] = dict(ms=ms, bytes=n * k * per + b * k * 2 + b * n * 2, flops=2.0 * b * n * k, launches_per_call=1,
+                          kernel=main_kernel(names, gemm_kernel), kernels=names, source=["gemm.cu", "tc.cuh"])
+    ms, names = time_cycle(lambda l: fq.flex_append_kv(caches[l], x[:, h:], x[:, 2 * h:], 3 * h, b, pos,
+                                                       stream=stream))
     kern["store_cache"] = dict(
-        ms=time_cycle(lambda l: fq.flex_append_kv(caches[l], x[:, h:], x[:, 2 * h:], 3 * h, b, pos, stream=stream)),
-        bytes=2 * b * h * 2 + 2 * b * h * per, flops=0.0, launches_per_call=0, source=["kv_ln.cu"],
-        note="standalone store_cache entry; inside a layer it is fused into the QKV GEMM epilogue")
-    kern["layernorm"] = dict(
-        ms=time_cycle(lambda l: fq.flex_layernorm(x[:, :h], layers[l].vec["ln1_g"], layers[l].vec["ln1_b"], o, b, h,
-                                                  stream=stream)),
-        bytes=2 * b * h * 2 + 2 * h * 2, flops=0.0, launches_per_call=2, source=["kv_ln.cu"])
+        ms=ms, bytes=2 * b * h * 2 + 2 * b * h * per, flops=0.0, launches_per_call=0, kernels=names,
+        source=["kv_ln.cu"], note="standalone store_cache entry; inside a layer it is fused into the QKV GEMM epilogue")
+    ms, names = time_cycle(lambda l: fq.flex_layernorm(x[:, :h], layers[l].vec["ln1_g"], layers[l].vec["ln1_b"], o, b,
+                                                       h, stream=stream))
+    kern["layernorm"] = dict(ms=ms, bytes=2 * b * h * 2 + 2 * h * 2, flops=0.0, launches_per_call=2,
+                             kernel=main_kernel(names, "layernorm_kernel"), kernels=names, source=["kv_ln.cu"])
     for k, v in kern.items():
         v["us"] = v["ms"] * 1e3
         v["gbs"] = v["bytes"] / (v["ms"] * 1e6)
@@ -678,16 +689,19 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
             v["frac_tensor"] = v["tflops"] / tpk
     # per kernel (the four GEMMs are launches of one kernel): time per layer call, and
     # bytes / flops / duration per launch averaged over its launches
-    gemms = ["gemm_qkv", "gemm_out", "gemm_fc1", "gemm_fc2"]
-    per_kernel = {
-        gemm_kernel: dict(launches=4, ms=sum(kern[g]["ms"] for g in gemms), bytes=sum(kern[g]["bytes"] for g in gemms),
-                          flops=sum(kern[g]["flops"] for g in gemms), source=["gemm.cu", "tc.cuh"]),
-        "decode_attn_tc_kernel": dict(launches=attn_launches, ms=kern["decode_attention"]["ms"],
-                                      bytes=kern["decode_attention"]["bytes"], flops=kern["decode_attention"]["flops"],
-                                      source=["attention.cu"]),
-        "layernorm_kernel": dict(launches=2, ms=2 * kern["layernorm"]["ms"], bytes=2 * kern["layernorm"]["bytes"],
-                                 flops=0.0, source=["kv_ln.cu"]),
-    }
+    # each part's time goes to its working kernel (the attention's combine step, when the
+    # key range is split, is timed with it); one layer call runs 4 GEMMs, 1 attention, 2 LNs
+    per_kernel = {}
+    for part, calls in (("gemm_qkv", 1), ("gemm_out", 1), ("gemm_fc1", 1), ("gemm_fc2", 1),
+                        ("decode_attention", 1), ("layernorm", 2)):
+        v = kern[part]
+        e = per_kernel.setdefault(v["kernel"], dict(launches=0, ms=0.0, bytes=0.0, flops=0.0, parts=[],
+                                                    source=v["source"]))
+        e["launches"] += calls
+        e["ms"] += calls * v["ms"]
+        e["bytes"] += calls * v["bytes"]
+        e["flops"] += calls * v["flops"]
+        e["parts"].append(part)
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"])
     dk = per_kernel[dom]
     sha = _kernel_sha(*dk["source"])

@@ -28,7 +28,7 @@ constexpr int kThreads = 256;
 #define FLEXQ_CODEC_UNROLL 4
 #endif
 #ifndef FLEXQ_CODEC_MINB
-#define FLEXQ_CODEC_MINB 1
+#define FLEXQ_CODEC_MINB 4
 #endif
 #ifndef FLEXQ_DEC_UNROLL
 #define FLEXQ_DEC_UNROLL 8
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) compress_contig_kernel(c
                 } else {
                     st_stream_v2(codes + g * GS + sub * 8, quant8_8bit(v[u], mn, s));
                 }
-                if (sub == 0) meta[g] = pack_half2_bits(__float2half_rn(mn), s16);
+                if (sub == 0) meta[g] = pack_half2_bits(stored_min16(mn), s16);
             }
         }
     }
@@ -205,8 +205,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) compress_strided_1pass_k
             const __half s0 = group_scale16<BITS>(mn[2 * k], mx0), s1 = group_scale16<BITS>(mn[2 * k + 1], mx1);
             s[2 * k] = __half2float(s0);
             s[2 * k + 1] = __half2float(s1);
-            mw[2 * k] = pack_half2_bits(__float2half_rn(mn[2 * k]), s0);
-            mw[2 * k + 1] = pack_half2_bits(__float2half_rn(mn[2 * k + 1]), s1);
+            mw[2 * k] = pack_half2_bits(stored_min16(mn[2 * k]), s0);
+            mw[2 * k + 1] = pack_half2_bits(stored_min16(mn[2 * k + 1]), s1);
         }
         uint64_t mn2[4], s2[4];
 #pragma unroll
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kThreads) compress_strided_kernel(const __half
             if (BITS == 4) q |= quant_one<4>(__half2float(src[(r + 1) * inner]), mn, s) << 4;
             dst[(BITS == 4 ? r / 2 : r) * inner] = static_cast<uint8_t>(q);
         }
-        meta[og * inner + c0] = pack_half2_bits(__float2half_rn(mn), s16);
+        meta[og * inner + c0] = pack_half2_bits(stored_min16(mn), s16);
     }
 }
 
@@ -440,7 +440,7 @@ __global__ void __launch_bounds__(kThreads) compress_generic_kernel(const __half
                 }
             }
         }
-        meta[(o * ng + g) * inner + i] = pack_half2_bits(sym ? __ushort_as_half(0) : __float2half_rn(mn), s16);
+        meta[(o * ng + g) * inner + i] = pack_half2_bits(sym ? __ushort_as_half(0) : stored_min16(mn), s16);
     }
 }
 

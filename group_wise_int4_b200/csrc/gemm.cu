@@ -240,7 +240,7 @@ __device__ __forceinline__ void kv_store8_bits(const GemmParams& p, const __half
         } else {
             codes[slot * p.kv.hd + dim] = static_cast<uint8_t>(q);
         }
-        if (dim % p.kv.gs == 0) meta[slot * gph + dim / p.kv.gs] = pack_half2_bits(__float2half_rn(mn), s16);
+        if (dim % p.kv.gs == 0) meta[slot * gph + dim / p.kv.gs] = pack_half2_bits(stored_min16(mn), s16);
     }
 }
 
@@ -1250,11 +1250,11 @@ __device__ __forceinline__ void gemv_finish(const GemvParams& p, int n0, int c, 
         if (p.kv.bits == 4) {
             const __half s16 = group_scale16<4>(mn, mx);
             *reinterpret_cast<uint32_t*>(codes + slot * (p.kv.hd / 2) + dim / 2) = quant8_4bit(nv, mn, __half2float(s16));
-            if (dim % p.kv.gs == 0) meta[slot * gph + dim / p.kv.gs] = pack_half2_bits(__float2half_rn(mn), s16);
+            if (dim % p.kv.gs == 0) meta[slot * gph + dim / p.kv.gs] = pack_half2_bits(stored_min16(mn), s16);
         } else {
             const __half s16 = group_scale16<8>(mn, mx);
             *reinterpret_cast<uint2*>(codes + slot * p.kv.hd + dim) = quant8_8bit(nv, mn, __half2float(s16));
-            if (dim % p.kv.gs == 0) meta[slot * gph + dim / p.kv.gs] = pack_half2_bits(__float2half_rn(mn), s16);
+            if (dim % p.kv.gs == 0) meta[slot * gph + dim / p.kv.gs] = pack_half2_bits(stored_min16(mn), s16);
         }
     }
 }

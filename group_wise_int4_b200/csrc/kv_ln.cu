@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(256) append_kv_kernel(const __half* __restrict
         *reinterpret_cast<uint32_t*>(codes + sub * 4) = quant8_4bit(v, mn, s);
     else
         *reinterpret_cast<uint2*>(codes + sub * 8) = quant8_8bit(v, mn, s);
-    if (sub == 0) *meta = pack_half2_bits(__float2half_rn(mn), s16);
+    if (sub == 0) *meta = pack_half2_bits(stored_min16(mn), s16);
 }
 
 // LayerNorm: one CTA of LN_THREADS per row, each thread keeps up to LN_VPT 16-byte

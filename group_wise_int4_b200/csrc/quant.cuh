@@ -24,6 +24,11 @@ __device__ __forceinline__ __half group_scale16(float mn, float mx) {
     return s16;
 }
 
+// The stored fp16 minimum of a group: a zero minimum is stored as +0. A group holding
+// both +0 and -0 has no defined sign for its smallest value; +0 is the one kept, so
+// every kernel writes the same bits (dequantised values do not depend on it).
+__device__ __forceinline__ __half stored_min16(float mn) { return __float2half_rn(__fadd_rn(mn, 0.0f)); }
+
 // ---- packed fp32 pairs ---------------------------------------------------------------
 // sm_100 executes add / sub / mul on two fp32 lanes held in one 64-bit register, each
 // lane rounded like the scalar instruction; the quantiser's per-value arithmetic runs on

@@ -230,8 +230,9 @@ int flex_append_kv(const flex_kv_cache* cache, const void* k_new, const void* v_
  *   o = softmax([q.k_vf .. q.k_{pos-1}, q.k_new]) [v_vf .. v_{pos-1}, v_new]
  * with k_j, v_j the dequantised cache slots [vf, pos), vf = cache->valid_from[b]
  * (0 without padding; clamped to [0, pos]). q, k_new, v_new: fp16 rows of
- * `row_stride` elements per sequence, head h at offset h*head_dim (q is used as
- * given: callers pre-scale it). o: fp16 [batch][n_heads*head_dim].
+ * `row_stride` elements per sequence (a multiple of 8, else FLEX_ERR_ALIGN), head h
+ * at offset h*head_dim (q is used as given: callers pre-scale it). o: fp16
+ * [batch][n_heads*head_dim].
  * ws: at least flex_decode_attention_ws_bytes(cache, batch, pos) bytes. */
 int64_t flex_decode_attention_ws_bytes(const flex_kv_cache* cache, int32_t batch, int32_t pos);
 int flex_decode_attention(const flex_kv_cache* cache, const void* q, const void* k_new,

@@ -98,7 +98,7 @@ def _groups(x, gd, group_size):
 def group_params(g32, num_bits):
     """Per group: min, fp16 scale. g32: float32 array [..., group_size]."""
     levels = np.float32((1 << num_bits) - 1)
-    mn = g32.min(axis=-1)
+    mn = g32.min(axis=-1) + np.float32(0)                  # a zero minimum is +0 (reading R26)
     mx = g32.max(axis=-1)
     r = mx - mn                                            # fp32, rounded once
     with np.errstate(divide="ignore", over="ignore", invalid="ignore"):

@@ -129,7 +129,7 @@ void quantise_group(const float* v, int gs, int bits, uint8_t* q, uint16_t* mn16
         if (c > levels) c = levels;
         q[j] = static_cast<uint8_t>(c);
     }
-    *mn16 = float_to_half(mn);                                 // mn is an fp16 value: exact
+    *mn16 = float_to_half(mn + 0.0f);                          // exact; a zero minimum is stored as +0
     *s16 = sc;
 }
 

@@ -80,3 +80,37 @@ def test_prefill_attention(batch, seq, nh, d):
     ref = ol.prefill_attention(q[..., :h].reshape(batch, seq, nh, d), q[..., h:2 * h].reshape(batch, seq, nh, d),
                                q[..., 2 * h:].reshape(batch, seq, nh, d))
     assert_layer_close(o, ref.reshape(batch, seq, h), f"prefill attn s={seq}")
+
+
+@pytest.mark.parametrize("batch,nh,d,gs,pos,padded", [
+    (20, 40, 128, 64, 300, True),      # 800 pairs: beyond one wave of 4 CTAs x 148 SMs
+    (20, 40, 128, 32, 257, False),     # a one-key last stage
+    (40, 32, 64, 64, 200, True),       # 1280 pairs: beyond one wave of 7 CTAs x 148 SMs
+    (40, 32, 64, 32, 128, False),      # exactly one stage per pair
+])
+def test_decode_attention_many_pairs_every_row(batch, nh, d, gs, pos, padded):
+    """Single-split decode with more (sequence, head) pairs than one wave of CTAs: each
+    CTA walks several pairs with one copy ring running across them. Every row is
+    compared (not a sample), so a pair that picks up its neighbour's keys, query or
+    fresh key/value, or a stale softmax state, fails."""
+    h = nh * d
+    vf = [(37 * b) % (pos + 1) if padded else 0 for b in range(batch)]
+    if padded:
+        vf[1] = pos                    # only the new token is visible
+    vft = torch.tensor(vf, dtype=torch.int32, device="cuda") if padded else None
+    kh, vh = synth.kv_history(batch, nh, pos, d, pos + d + gs)
+    cache = fq.FlexKVCache(batch, nh, d, pos + 1, 4, gs, valid_from=vft)
+    cache.fill_from(kh.cuda(), vh.cuda())
+    oc = ol.KVCache(batch, nh, pos + 1, d, 4, gs)
+    oc.store(kh.numpy(), vh.numpy(), 0)
+    qkv = synth.activations((batch, 3 * h), pos + 5)
+    qkv[:, :h] *= d ** -0.5
+    g = qkv.cuda()
+    o = torch.full((batch, h), float("nan"), dtype=torch.float16, device="cuda")
+    ws = torch.empty(max(16, fq.flex_decode_attention_ws_bytes(cache, batch, pos)), dtype=torch.uint8, device="cuda")
+    fq.flex_decode_attention(cache, g[:, :h], g[:, h:2 * h], g[:, 2 * h:], 3 * h, o, batch, pos, ws)
+    sync_status()
+    q = qkv.numpy()
+    ref = ol.decode_attention(q[:, :h].reshape(-1, nh, d), q[:, h:2 * h].reshape(-1, nh, d),
+                              q[:, 2 * h:].reshape(-1, nh, d), oc, pos, valid_from=vf if padded else None)
+    assert_layer_close(o, ref.reshape(batch, h), f"decode attention, {batch * nh} pairs, pos={pos}")

@@ -21,7 +21,12 @@ workload. A decode step that follows each side's own prefill is not compared at 
 widths: the two prefills round the keys/values to fp16 differently in the last place,
 the int4 codes then differ in about 0.5% of places, and at h 7168 the oracle's own
 output moves by about 3x the tolerance under such a perturbation (an oracle-only
-experiment), so the comparison would measure the rounding, not the kernels.
+experiment), so the comparison would measure the rounding, not the kernels. The same
+holds, on a smaller scale, for the one slot a decode step writes: at h 12288 the
+second step moved by about 1.1x the tolerance when each side kept its own slot 512.
+So each step checks the slot the layer wrote (flexq_compress of the layer's own fp16
+key/value, bit for bit) and then overwrites it, on both sides, with the next slot of
+the shared seeded history before the following step.
 """
 import numpy as np
 import pytest
@@ -131,15 +136,25 @@ def test_large_layer_prefill(name, batch, rows, prompt):
 def test_large_layer_decode(name, batch, rows, pos, steps):
     M = _model(name)
     h, nh, d, seed = M.h, M.nh, M.d, M.cfg["seed"]
-    kh, vh = synth.kv_history(batch, nh, pos, d, seed + 50, device="cuda")
+    n_hist = pos + steps - 1                      # the shared history also supplies later steps' slots
+    kh, vh = synth.kv_history(batch, nh, n_hist, d, seed + 50, device="cuda")
     cache = fq.FlexKVCache(batch, nh, d, MAX_SEQ)
-    cache.fill_from(kh, vh)
+    cache.fill_from(kh[:, :, :pos], vh[:, :, :pos])
     ocache = ol.KVCache(len(rows), nh, MAX_SEQ, d)
-    ocache.store(to_np(kh[rows]), to_np(vh[rows]), 0)
+    ocache.store(to_np(kh[rows, :, :pos]), to_np(vh[rows, :, :pos]), 0)
+    k_next, v_next = kh[:, :, pos:].contiguous(), vh[:, :, pos:].contiguous()
     del kh, vh
     torch.cuda.empty_cache()
     wsd = _ws(M.layer, batch, 1)
     for t in range(steps):
+        if t > 0:                                 # slot pos + t - 1 from the shared history, both sides
+            sl = slice(t - 1, t)
+            for src, codes, meta in ((k_next[:, :, sl], cache.k_codes, cache.k_meta),
+                                     (v_next[:, :, sl], cache.v_codes, cache.v_meta)):
+                c, m = fq.flexq_compress(src.contiguous(), cache.cfg)
+                codes[:, :, pos + t - 1:pos + t].copy_(c)
+                meta[:, :, pos + t - 1:pos + t].copy_(m)
+            ocache.store(to_np(k_next[rows, :, sl]), to_np(v_next[rows, :, sl]), pos + t - 1)
         xd = synth.decode_inputs(batch, h, t, seed)
         yd = torch.empty((batch, h), dtype=torch.float16, device="cuda")
         fq.flex_decode_layer(M.layer, cache, xd.cuda(), yd, batch, pos + t, wsd)

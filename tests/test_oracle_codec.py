@@ -224,3 +224,23 @@ def test_saturated_scale():
     assert float(m[0, 1]) == 65504.0                    # 15/2^-14 overflows fp16
     assert int(c[2] >> 4) == 4                          # element 5: 2^-14 * 65504 = 3.998 -> 4
     assert int(c[2] & 15) == 0 and int(c[0]) == 0
+
+
+@pytest.mark.parametrize("order", [(-0.0, 0.0), (0.0, -0.0)])
+@pytest.mark.parametrize("bits", [3, 4, 8])
+def test_zero_minimum_is_stored_as_plus_zero(order, bits):
+    """A group whose smallest value is a zero (both signs present, in either order, or
+    -0 alone) stores min = +0 (bits 0x0000); the codes and the decoded values are those
+    of the same group with every -0 replaced by +0."""
+    x = np.array([0.5, order[0], 1.0, order[1]] + [0.25] * 28, np.float16)
+    c, m = codec.compress(x, bits, 32, 0)
+    assert np.ascontiguousarray(m).view(np.uint16)[0, 0] == 0
+    xp = np.where(x == 0, np.float16(0.0), x)
+    cp, mp = codec.compress(xp, bits, 32, 0)
+    assert np.array_equal(c, cp) and np.array_equal(np.ascontiguousarray(m).view(np.uint16),
+                                                    np.ascontiguousarray(mp).view(np.uint16))
+    y = codec.decompress(c, m, x.shape, bits, 32, 0)
+    assert y[1] == 0 and y[3] == 0 and not np.signbit(y[1]) and not np.signbit(y[3])
+    xn = np.full(32, -0.0, np.float16)                   # an all -0 group: constant, min +0
+    _, mn = codec.compress(xn, bits, 32, 0)
+    assert np.ascontiguousarray(mn).view(np.uint16)[0, 0] == 0

@@ -67,7 +67,7 @@ def test_codec_matches_numpy_oracle_bit_for_bit(shape, gd, bits, gs):
     if shape[gd] % gs:
         pytest.skip("group does not divide")
     x = synth.codec_tensor(shape, gd, gs, seed=len(shape) * 10 + bits + gs).numpy()
-    x.reshape(-1)[:7] = np.float16([3e-5, 3.01e-5, 3.02e-5, 0, 0, 0, 0])       # tiny ranges
+    x.reshape(-1)[:7] = np.float16([3e-5, 3.01e-5, 3.02e-5, 0, -0.0, 0, -0.0])  # tiny ranges, signed zeros
     c1, m1 = codec.compress(x, bits, gs, gd)
     c2, m2 = cpp.compress(x, bits, gs, gd, nthreads=3)
     assert np.array_equal(c1, c2)

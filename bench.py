@@ -612,10 +612,11 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
             for l in range(L):
                 fn(l)
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)        # the graph stays readable after capture
         with torch.cuda.graph(g, stream=stream):
             for l in range(L):
                 fn(l)
+        g.instantiate()
         counts = graph_kernel_counts(g)
         names = None if counts is None else {short_kernel_name(k): v / L for k, v in counts.items()}
         with torch.cuda.stream(stream):

@@ -104,6 +104,8 @@ _SIGS = {
     "flex_lm_head_argmax": (_I32, [ctypes.POINTER(flexq_tensor), _I32, _P, _P, _P, _I64, _P, _P, _P, _I64, _P]),
     "flex_get_status": (_I32, [_P]),
     "flex_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
+    "flex_set_gemm_gate": (_P, [_P]),
+    "flex_gemm_plan": (_I32, [_I32, _I32, _I32, _I32, _P]),
     "flex_status_string": (ctypes.c_char_p, [_I32]),
     "flex_abi_layout": (_I64, [_I32, _I32]),
 }
@@ -461,6 +463,20 @@ def flex_abi_layout(which: int, field: int) -> int:
 def flex_set_wait_limit_ns(ns: int) -> int:
     """Limit of the GEMM's pipeline waits for later launches (0 = default 2 s); returns the old one."""
     return int(lib().flex_set_wait_limit_ns(int(ns)))
+
+
+def flex_gemm_plan(M: int, N: int, K: int, bits: int = 4) -> dict:
+    """The launch plan of flex_dequant_gemm for this problem on the current device."""
+    out = (ctypes.c_int32 * 4)()
+    _check(lib().flex_gemm_plan(int(M), int(N), int(K), int(bits), ctypes.cast(out, ctypes.c_void_p)), "flex_gemm_plan")
+    return {"kernel": ("gemv", "tc128", "tc256")[out[0]], "tiles": out[1], "splits": out[2], "cluster": bool(out[3])}
+
+
+def flex_set_gemm_gate(gate) -> int:
+    """Gate of the tensor-core GEMM's weight loads for later launches (a device int32
+    tensor, or None to remove it); returns the previous gate's address (0 if none)."""
+    prev = lib().flex_set_gemm_gate(None if gate is None else _ptr(gate))
+    return int(prev or 0)
 
 
 def flex_get_status(stream=None) -> int:

@@ -58,6 +58,12 @@ std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 
 uint64_t pipeline_wait_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
+namespace {
+std::atomic<const int32_t*> g_gate{nullptr};
+}  // namespace
+
+const int32_t* gemm_gate() { return g_gate.load(std::memory_order_relaxed); }
+
 int* status_word() {
     const int dev = current_device();
     if (dev < 0) return nullptr;
@@ -89,6 +95,8 @@ extern "C" int flex_get_status(void* stream) {
 extern "C" uint64_t flex_set_wait_limit_ns(uint64_t ns) {
     return flexq::g_wait_ns.exchange(ns == 0 ? flexq::kDefaultWaitNs : ns);
 }
+
+extern "C" const int32_t* flex_set_gemm_gate(const int32_t* gate) { return flexq::g_gate.exchange(gate); }
 
 extern "C" int64_t flex_abi_layout(int32_t which, int32_t field) {
 #define FLEX_FIELDS(T, ...)                                              \

@@ -299,9 +299,6 @@ constexpr int dt_smem_bytes(int D, int GS) {
     return DT_STAGES * (2 * DT_KEYS * (D / 2) + 2 * DT_KEYS * (D / GS) * 4);
 }
 
-// ... and of decode_attn_pk_kernel<D, GS>, whose stages also carry the pair's q, k_new, v_new
-constexpr int dp_smem_bytes(int D, int GS) { return dt_smem_bytes(D, GS) + DT_STAGES * 3 * D * 2; }
-
 // 7 CTAs per SM at head_dim 64 (all 1024 CTAs of a 32 x 32-head decode in one wave);
 // at head_dim 128 FLEXQ_DT_MINB_128 (a build constant, tuned by measurement)
 #ifndef FLEXQ_DT_MINB_128
@@ -674,371 +671,6 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
     }
 }
 
-// ---------------------------------------------------------------------------------
-// Persistent form of decode_attn_tc_kernel for the single-split case (a CTA's worth of
-// keys per (sequence, head) pair): a grid of a few CTAs per SM walks the pairs
-// p = blockIdx.x, blockIdx.x + gridDim.x, ..., and one cp.async ring of stages runs
-// across pairs, so that the next pair's first keys are already in flight while this
-// pair's last stage and its epilogue run (a CTA per pair pays the ring's fill and the
-// epilogue on every pair). The first stage of a pair also carries the pair's q, k_new
-// and v_new rows. The per-stage arithmetic, the reduction over the warps and the fold of
-// the fresh key/value are those of decode_attn_tc_kernel.
-template <int D, int GS>
-__global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) decode_attn_pk_kernel(
-    const __half* __restrict__ q, int64_t row_stride, const uint8_t* __restrict__ k_codes,
-    const uint32_t* __restrict__ k_meta, const uint8_t* __restrict__ v_codes,
-    const uint32_t* __restrict__ v_meta, int n_heads, int max_seq, int pos, int npairs,
-    const __half* __restrict__ k_new, const __half* __restrict__ v_new, __half* __restrict__ o, int perm,
-    const int32_t* __restrict__ valid_from) {
-    constexpr int G = D / GS;
-    constexpr int KB = D / 2;
-    constexpr int KW = D / 32;
-    constexpr int VW = D / 64;
-    constexpr int NMT = D / 16;
-    constexpr int NW = DA_THREADS / 32;
-    constexpr int CODE = DT_KEYS * KB;
-    constexpr int META = DT_KEYS * G;
-    constexpr int HDR = 3 * D * 2;                 // q, k_new, v_new of the pair (fp16)
-    constexpr int STAGE = 2 * CODE + 2 * META * 4 + HDR;
-    constexpr int DT_NS = DT_STAGES;
-    static_assert(NW * 32 == DT_KEYS, "32 keys per warp and stage");
-    static_assert(CODE % (16 * DA_THREADS) == 0 && META % DA_THREADS == 0, "whole copy rounds");
-    static_assert(3 * (D / 8) <= DA_THREADS, "one header copy per thread");
-    extern __shared__ __align__(16) uint8_t dt_ring[];
-    auto ring = reinterpret_cast<uint8_t (*)[STAGE]>(dt_ring);
-    __shared__ float sm_m[NW], sm_l[NW];
-    __shared__ float sm_o[NW][D];
-    __shared__ float sm_red[NW];
-    __shared__ __align__(16) __half hdr[3][D];           // q, k_new, v_new of the current pair
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int npk = blockIdx.x < npairs ? (npairs - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
-    // keys of a pair: slots [vf, pos), vf its sequence's left-padding start
-    auto pair_vf = [&](int pair) {
-        return valid_from ? min(max(valid_from[pair / n_heads], 0), pos) : 0;
-    };
-    auto pair_nst = [&](int pk) {                  // stages of the CTA's pk-th pair (at least one)
-        const int nk = pos - pair_vf(static_cast<int>(blockIdx.x) + pk * static_cast<int>(gridDim.x));
-        return nk > DT_KEYS ? (nk + DT_KEYS - 1) / DT_KEYS : 1;
-    };
-    auto load_stage = [&](int slot, int pk, int s) {
-        const int pair = static_cast<int>(blockIdx.x) + pk * static_cast<int>(gridDim.x);
-        const int vf = pair_vf(pair), nk = pos - vf;
-        const int64_t sl = static_cast<int64_t>(pair) * max_seq + vf;
-        uint8_t* st = ring[slot];
-        const int kbase = s * DT_KEYS;
-#pragma unroll
-        for (int i = 0; i < CODE / (16 * DA_THREADS); ++i) {
-            const int u = threadIdx.x + i * DA_THREADS;
-            const bool ok = kbase + (u * 16) / KB < nk;
-            const int64_t off = ok ? (sl + kbase) * KB + u * 16 : 0;
-            cp_async16(st + u * 16, k_codes + off, ok);
-            cp_async16(st + CODE + u * 16, v_codes + off, ok);
-        }
-#pragma unroll
-        for (int i = 0; i < META / DA_THREADS; ++i) {
-            const int u = threadIdx.x + i * DA_THREADS;
-            const bool ok = kbase + u / G < nk;
-            const int64_t off = ok ? (sl + kbase) * G + u : 0;
-            cp_async4(st + 2 * CODE + u * 4, k_meta + off, ok);
-            cp_async4(st + 2 * CODE + META * 4 + u * 4, v_meta + off, ok);
-        }
-        if (s == 0 && threadIdx.x < 3 * (D / 8)) {
-            const int which = threadIdx.x / (D / 8), part = threadIdx.x % (D / 8);
-            const __half* src = (which == 0 ? q : (which == 1 ? k_new : v_new)) +
-                                static_cast<int64_t>(pair / n_heads) * row_stride + (pair % n_heads) * D + part * 8;
-            cp_async16(st + 2 * CODE + 2 * META * 4 + which * D * 2 + part * 16, src, true);
-        }
-    };
-
-    // q / k_new / v_new come from the previous kernel: everything waits for it
-    pdl_wait();
-    pdl_trigger();
-    int pk_i = 0, s_i = 0, nst_i = npk > 0 ? pair_nst(0) : 0;     // issue cursor
-    auto issue = [&](int slot) {
-        if (pk_i < npk) {
-            load_stage(slot, pk_i, s_i);
-            if (++s_i == nst_i) {
-                s_i = 0;
-                if (++pk_i < npk) nst_i = pair_nst(pk_i);
-            }
-        }
-        cp_async_commit();
-    };
-#pragma unroll
-    for (int i = 0; i < DT_NS - 1; ++i) issue(i);
-
-    const int tgrp = (t * (D / 4)) / GS;
-    const int own_n = (G == 4) ? t : t % G;
-    const int own_h = (G == 4) ? 0 : t / G;
-    const bool owner = (G == 4) || (t < 2 * G);
-    const int gn = g < G ? g : 0;
-    const int src_a0 = 4 * (2 * t) + gn;
-    const int src_a1 = 4 * (2 * t + 1) + gn;
-    const int src_b0 = 4 * (2 * t) + ((G == 4) ? gn : G + gn);
-    const int src_b1 = 4 * (2 * t + 1) + ((G == 4) ? gn : G + gn);
-    const __half sixteenth = __float2half(0.0625f);
-
-    int gidx = 0;                                  // global stage index of this CTA
-    for (int ip = 0; ip < npk; ++ip) {
-        const int pair = static_cast<int>(blockIdx.x) + ip * static_cast<int>(gridDim.x);
-        const int b = pair / n_heads, head = pair % n_heads;
-        const int nkeys = pos - pair_vf(pair);
-        const int nst = pair_nst(ip);
-        float Qg[G], QC[G];
-        uint32_t bq[2 * KW][2];
-        float m = -FLT_MAX, lsum = 0.f, Wl = 0.f, Ul = 0.f;
-        float oacc[NMT][4];
-#pragma unroll
-        for (int i = 0; i < NMT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-        for (int s = 0; s < nst; ++s, ++gidx) {
-            issue((gidx + DT_NS - 1) % DT_NS);
-            cp_async_wait<DT_NS - 1>();
-            __syncthreads();
-            if (s == 0) {
-                // the pair's query (group sums and the QK B operand) from the stage header;
-                // its fresh key/value kept for the epilogue
-                const __half* hq = reinterpret_cast<const __half*>(ring[gidx % DT_NS] + 2 * CODE + 2 * META * 4);
-#pragma unroll
-                for (int n = 0; n < G; ++n) Qg[n] = QC[n] = 0.f;
-#pragma unroll
-                for (int v = 0; v < D / 8; ++v) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(hq + 8 * v);
-                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float lo = h2f_lo(ww[k]), hi = h2f_hi(ww[k]);
-                        Qg[(8 * v) / GS] += lo + hi;
-                        QC[(8 * v) / GS] += 1024.f * lo + 64.f * hi;
-                    }
-                }
-#pragma unroll
-                for (int ks = 0; ks < 2 * KW; ++ks) {
-                    const int d = t * (D / 4) + 8 * (ks / 2) + 2 * (ks % 2);
-                    if (g == tgrp) {
-                        bq[ks][0] = pack_half2_bits(hq[d], hq[d + 4]);
-                        bq[ks][1] = pack_half2_bits(__hmul(hq[d + 1], sixteenth), __hmul(hq[d + 5], sixteenth));
-                    } else {
-                        bq[ks][0] = bq[ks][1] = 0u;
-                    }
-                }
-                if (threadIdx.x < 3 * (D / 8))      // the slot is reused: keep the header for the epilogue
-                    reinterpret_cast<uint4*>(&hdr[0][0])[threadIdx.x] = reinterpret_cast<const uint4*>(hq)[threadIdx.x];
-            }
-        const int kw0 = s * DT_KEYS + warp * 32;                 // the warp's first key
-        if (kw0 < nkeys) {
-            const uint8_t* st = ring[gidx % DT_NS];
-            const uint32_t* kmeta = reinterpret_cast<const uint32_t*>(st + 2 * CODE) + warp * 32 * G;
-            const uint32_t* vmeta = reinterpret_cast<const uint32_t*>(st + 2 * CODE + META * 4) + warp * 32 * G;
-            // ---- scores of the two tiles: keys (tile 16 + g) and (tile 16 + g + 8)
-            float sc[2][2];
-#pragma unroll
-            for (int tile = 0; tile < 2; ++tile) {
-                const uint8_t* kc = st + (warp * 32 + tile * 16) * KB + t * (D / 8);
-                uint32_t x0[KW], x8[KW];
-                if (KW == 4) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(kc + g * KB);
-                    const uint4 c = *reinterpret_cast<const uint4*>(kc + (g + 8) * KB);
-                    x0[0] = a.x; x0[1 % KW] = a.y; x0[2 % KW] = a.z; x0[3 % KW] = a.w;
-                    x8[0] = c.x; x8[1 % KW] = c.y; x8[2 % KW] = c.z; x8[3 % KW] = c.w;
-                } else {
-                    const uint2 a = *reinterpret_cast<const uint2*>(kc + g * KB);
-                    const uint2 c = *reinterpret_cast<const uint2*>(kc + (g + 8) * KB);
-                    x0[0] = a.x; x0[1 % KW] = a.y;
-                    x8[0] = c.x; x8[1 % KW] = c.y;
-                }
-                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int w = 0; w < KW; ++w) {
-                    const uint32_t y0 = x0[w] >> 8, y8 = x8[w] >> 8;
-                    const uint32_t a0[4] = {nib_lo(x0[w]), nib_lo(x8[w]), nib_hi(x0[w]), nib_hi(x8[w])};
-                    mma16816(sacc, a0, bq[2 * w][0], bq[2 * w][1]);
-                    const uint32_t a1[4] = {nib_lo(y0), nib_lo(y8), nib_hi(y0), nib_hi(y8)};
-                    mma16816(sacc, a1, bq[2 * w + 1][0], bq[2 * w + 1][1]);
-                }
-                // per key: sum over the groups this lane holds (columns 2t, 2t+1)
-                float s0 = 0.f, s8 = 0.f;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int n = 2 * t + u;
-                    if (n < G) {
-                        const uint32_t m0 = kmeta[(tile * 16 + g) * G + n], m8 = kmeta[(tile * 16 + g + 8) * G + n];
-                        const float qc = pick(QC, n), qg = pick(Qg, n);
-                        const float st0 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(m0 >> 16)));
-                        const float st8 = group_step_fast(__ushort_as_half(static_cast<unsigned short>(m8 >> 16)));
-                        s0 += fmaf(st0, sacc[u] - qc, h2f_lo(m0) * qg);
-                        s8 += fmaf(st8, sacc[2 + u] - qc, h2f_lo(m8) * qg);
-                    }
-                }
-                if (G == 4) {
-                    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-                    s8 += __shfl_xor_sync(0xffffffffu, s8, 1);
-                }
-                s0 = __shfl_sync(0xffffffffu, s0, lane & ~3);
-                s8 = __shfl_sync(0xffffffffu, s8, lane & ~3);
-                const int kt = kw0 + tile * 16;
-                sc[tile][0] = (kt + g < nkeys) ? s0 : -FLT_MAX;
-                sc[tile][1] = (kt + g + 8 < nkeys) ? s8 : -FLT_MAX;
-            }
-            // ---- one online-softmax update for the 32 keys
-            float tmax = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
-            if (tmax > m) {                        // warp-uniform
-                const float alpha = __expf(m - tmax);
-                m = tmax;
-                lsum *= alpha;
-                Wl *= alpha;
-                Ul *= alpha;
-#pragma unroll
-                for (int i = 0; i < NMT; ++i) {
-                    oacc[i][0] *= alpha;
-                    oacc[i][1] *= alpha;
-                    oacc[i][2] *= alpha;
-                    oacc[i][3] *= alpha;
-                }
-            }
-            float pr[2][2];
-#pragma unroll
-            for (int tile = 0; tile < 2; ++tile)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) pr[tile][h] = sc[tile][h] == -FLT_MAX ? 0.f : __expf(sc[tile][h] - m);
-            if (t == 0) lsum += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-            // ---- values
-#pragma unroll
-            for (int tile = 0; tile < 2; ++tile) {
-                // owner lanes: w = fp16(p step) of (key g + 8 h, group n); running W, U
-                uint32_t wb[2] = {0u, 0u};
-#pragma unroll
-                for (int hh = 0; hh < ((G == 4) ? 2 : 1); ++hh) {
-                    const int h = (G == 4) ? hh : own_h;
-                    if (owner) {
-                        const uint32_t mv = vmeta[(tile * 16 + g + 8 * h) * G + own_n];
-                        const float stp = group_step_fast(__ushort_as_half(static_cast<unsigned short>(mv >> 16)));
-                        const float pk = h ? pr[tile][1] : pr[tile][0];
-                        const __half w16 = __float2half_rn(pk * stp);
-                        Wl += __half2float(w16);
-                        Ul = fmaf(pk, h2f_lo(mv), Ul);
-                        wb[hh] = static_cast<uint32_t>(__half_as_ushort(w16));
-                    }
-                }
-                // gather the B operand: keys 2t, 2t+1 (b0) and 2t+8, 2t+9 (b1) of group g
-                const uint32_t lo_a = __shfl_sync(0xffffffffu, wb[0], src_a0);
-                const uint32_t lo_b = __shfl_sync(0xffffffffu, wb[0], src_a1);
-                const uint32_t hi_a = __shfl_sync(0xffffffffu, wb[(G == 4) ? 1 : 0], src_b0);
-                const uint32_t hi_b = __shfl_sync(0xffffffffu, wb[(G == 4) ? 1 : 0], src_b1);
-                const uint32_t b0 = g < G ? (lo_a | (lo_b << 16)) : 0u;
-                const uint32_t b1 = g < G ? (hi_a | (hi_b << 16)) : 0u;
-                // A: transposed codes; thread g holds D/16 bytes (dims D/8 g ..) of keys
-                // 2t, 2t+1, 2t+8, 2t+9
-                const uint8_t* vc = st + CODE + (warp * 32 + tile * 16) * KB + g * (D / 16);
-                uint32_t vk[4][VW > 0 ? VW : 1];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int key = 2 * t + (u & 1) + 8 * (u >> 1);
-                    if (VW == 2) {
-                        const uint2 a = *reinterpret_cast<const uint2*>(vc + key * KB);
-                        vk[u][0] = a.x;
-                        vk[u][1 % (VW > 0 ? VW : 1)] = a.y;
-                    } else {
-                        vk[u][0] = *reinterpret_cast<const uint32_t*>(vc + key * KB);
-                    }
-                }
-#pragma unroll
-                for (int mt = 0; mt < NMT; ++mt) {
-                    const int wi = mt / 4, by = mt % 4;
-                    // byte `by` of key 2t -> bytes 0,1 and of key 2t+1 -> bytes 2,3
-                    const uint32_t sel = static_cast<uint32_t>(by * 0x11 + (4 + by) * 0x1100);
-                    const uint32_t x1 = prmt_sel(vk[0][wi], vk[1][wi], sel);
-                    const uint32_t x2 = prmt_sel(vk[2][wi], vk[3][wi], sel);
-                    const uint32_t a[4] = {nib_lo(x1), nib_hi(x1), nib_lo(x2), nib_hi(x2)};
-                    mma16816(oacc[mt], a, b0, b1);
-                }
-            }
-        }
-            __syncthreads();                   // the slot is refilled by a later issue
-        }
-        const __half* hdr_q = hdr[0];
-        const __half* hdr_k = hdr[1];
-        const __half* hdr_v = hdr[2];
-    // ---- warp result: W_n, U_n per group (sum over the owner lanes), then the rows
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-        Wl += __shfl_xor_sync(0xffffffffu, Wl, off);
-        Ul += __shfl_xor_sync(0xffffffffu, Ul, off);
-    }
-    if (G == 1) {                          // owners t = 0, 1 (t = 2, 3 hold 0)
-        Wl += __shfl_xor_sync(0xffffffffu, Wl, 1);
-        Ul += __shfl_xor_sync(0xffffffffu, Ul, 1);
-        Wl += __shfl_xor_sync(0xffffffffu, Wl, 2);
-        Ul += __shfl_xor_sync(0xffffffffu, Ul, 2);
-    } else if (G == 2) {                   // owners of group t % 2: t and t ^ 2
-        Wl += __shfl_xor_sync(0xffffffffu, Wl, 2);
-        Ul += __shfl_xor_sync(0xffffffffu, Ul, 2);
-    }
-    // now lane t of every quad holds W, U of group t (G = 1: all lanes hold group 0)
-    float Wn[2], Un[2];                    // groups 2t and 2t + 1
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int n = (2 * t + u) < G ? 2 * t + u : 0;
-        Wn[u] = __shfl_sync(0xffffffffu, Wl, (lane & ~3) | (G == 1 ? 0 : n));
-        Un[u] = __shfl_sync(0xffffffffu, Ul, (lane & ~3) | (G == 1 ? 0 : n));
-    }
-#pragma unroll
-    for (int mt = 0; mt < NMT; ++mt) {
-        const int de = 2 * (g * (D / 16) + mt);        // even dim of row g; row g + 8 is de + 1
-        const int n = de / GS;
-        if (n / 2 == t) {
-            // static register indices only (a runtime index would move oacc to local memory)
-            const bool odd_col = (n % 2) != 0;
-            const float ev = odd_col ? oacc[mt][1] : oacc[mt][0];
-            const float od = odd_col ? oacc[mt][3] : oacc[mt][2];
-            const float W = odd_col ? Wn[1] : Wn[0], U = odd_col ? Un[1] : Un[0];
-            sm_o[warp][de] = ev - 1024.f * W + U;
-            sm_o[warp][de + 1] = (od - 1024.f * W) * 0.0625f + U;
-        }
-    }
-    if (lane == 0) {
-        sm_m[warp] = m;
-        sm_l[warp] = lsum;
-    }
-    __syncthreads();
-    {
-        // single split: the combine step here. Fresh score q . k_new (one dim per thread).
-        const int d = threadIdx.x;
-        float sn = d < D ? __half2float(hdr_q[d]) * __half2float(hdr_k[d]) : 0.f;
-#pragma unroll
-        for (int w = 16; w > 0; w >>= 1) sn += __shfl_xor_sync(0xffffffffu, sn, w);
-        if (lane == 0) sm_red[warp] = sn;
-        __syncthreads();
-        float snew = 0.f;
-#pragma unroll
-        for (int i = 0; i < NW; ++i) snew += sm_red[i];
-        float M = snew;
-#pragma unroll
-        for (int i = 0; i < NW; ++i)
-            if (sm_l[i] > 0.f) M = fmaxf(M, sm_m[i]);
-        if (d < D) {
-            const float fn = __expf(snew - M);
-            float L = fn, acc = fn * __half2float(hdr_v[d]);
-#pragma unroll
-            for (int i = 0; i < NW; ++i) {
-                if (!(sm_l[i] > 0.f)) continue;
-                const float f = __expf(sm_m[i] - M);
-                L = fmaf(f, sm_l[i], L);
-                acc = fmaf(f, sm_o[i][d], acc);
-            }
-            // perm: interleaved 8-block order for the next GEMM (element k -> 2(k%4) + (k/4)%2)
-            const int dd = perm ? ((d & ~7) | ((d & 3) << 1) | ((d >> 2) & 1)) : d;
-            o[static_cast<int64_t>(b) * n_heads * D + head * D + dd] = __float2half_rn(acc / L);
-        }
-        }
-    }
-    cp_async_wait<0>();
-}
-
 // combine the split partials with the fresh key/value of the current token
 template <int D>
 __global__ void __launch_bounds__(D) decode_attn_combine_kernel(const __half* __restrict__ q,
@@ -1260,29 +892,6 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __half* 
 
 int validate_cache(const flex_kv_cache* c);
 
-// Decode attention with a single split and more (sequence, head) pairs than one wave of
-// CTAs runs as the persistent decode_attn_pk_kernel (FLEXQ_PERSISTENT_ATTN=0 builds
-// without it, for comparison).
-#ifndef FLEXQ_PERSISTENT_ATTN
-#define FLEXQ_PERSISTENT_ATTN 1
-#endif
-constexpr bool kPersistentAttn = FLEXQ_PERSISTENT_ATTN != 0;
-
-// Resident CTAs per SM of decode_attn_pk_kernel<D, GS> (once per process; 0 if it cannot run).
-template <int D, int GS>
-int pk_ctas_per_sm() {
-    static int n = -1;
-    if (n < 0) {
-        set_smem_once(decode_attn_pk_kernel<D, GS>, dp_smem_bytes(D, GS));
-        int v = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, decode_attn_pk_kernel<D, GS>, DA_THREADS,
-                                                          dp_smem_bytes(D, GS)) != cudaSuccess)
-            v = 0;
-        n = v;
-    }
-    return n;
-}
-
 int decode_attn_nsplit(int pairs, int pos) {
     if (pos <= 0) return 0;
     const int target = 4 * sm_count();
@@ -1329,13 +938,6 @@ int decode_attn_launch(const flex_kv_cache* c, const void* q, const void* k_new,
              vm, c->n_heads, c->max_seq, pos, chunk, part, c->valid_from)
 #define MMA(D_, G_)                                                                                      \
     do {                                                                                                 \
-        const int per_wave = ns == 1 && kPersistentAttn ? pk_ctas_per_sm<D_, G_>() * sm_count() : 0;    \
-        if (pairs > per_wave && per_wave > 0) {                                                          \
-            launch_k(decode_attn_pk_kernel<D_, G_>, dim3(per_wave), dim3(DA_THREADS), dp_smem_bytes(D_, G_), st, \
-                     true, qh, row_stride, kc, km, vc, vm, c->n_heads, c->max_seq, pos, pairs, kn, vn, oh,    \
-                     perm ? 1 : 0, c->valid_from);                                                       \
-            break;                                                                                       \
-        }                                                                                                \
         set_smem_once(decode_attn_tc_kernel<D_, G_>, dt_smem_bytes(D_, G_));                            \
         launch_k(decode_attn_tc_kernel<D_, G_>, grid, dim3(DA_THREADS), dt_smem_bytes(D_, G_), st, true, qh, \
                  row_stride, kc, km, vc, vm, c->n_heads, c->max_seq, pos, chunk, part, kn, vn, oh, perm ? 1 : 0, \

@@ -100,6 +100,9 @@ int sm_count();
 // Limit of the tensor-core GEMM's pipeline waits for kernels launched from now on
 // (flex_set_wait_limit_ns).
 uint64_t pipeline_wait_ns();
+// Gate of the tensor-core GEMM's weight loads for kernels launched from now on
+// (flex_set_gemm_gate; nullptr = none).
+const int32_t* gemm_gate();
 // Device status word of the current device (created on first use; see flex_get_status).
 int* status_word();
 

@@ -68,6 +68,9 @@ constexpr int64_t kTicketBytes = 2048;
 
 struct GemmParams {
     uint64_t wait_ns;      // limit of the pipeline waits (drain waits keep tc::kWaitLimitNs)
+    // nullptr, or a device flag the code producer waits on (bounded by wait_ns) before its
+    // first weight load (flex_set_gemm_gate)
+    const volatile int* gate;
     const __half* bias;
     const __half* residual;
     __half* y;
@@ -264,6 +267,81 @@ __device__ __forceinline__ void issue_ksteps(uint32_t d_acc, uint32_t a_chunk, u
     }
 }
 
+// Split-K partials in the workspace: per (tile, split) a block of BN x R fp32 (R = the
+// tile's weight rows) laid out [col / 8][row][8], so a thread (one row) moves 8 columns
+// as two 16-byte accesses and a warp (32 consecutive rows) covers 1 KB contiguously.
+__device__ __forceinline__ void part_store8(float* blk, int R, int row, int col, const float (&v)[8]) {
+    float4* d = reinterpret_cast<float4*>(blk + (static_cast<int64_t>(col >> 3) * R + row) * 8);
+    __stcg(d, make_float4(v[0], v[1], v[2], v[3]));
+    __stcg(d + 1, make_float4(v[4], v[5], v[6], v[7]));
+}
+// Requests the 8 columns (col..col+7) of `row` of splits s0..s0+3 (zeros past `splits`).
+__device__ __forceinline__ void part_load4(const float* all, int64_t split_stride, int splits, int s0, int R, int row,
+                                           int col, float4 (&t)[4][2]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (s0 + u < splits) {
+            const float4* q = reinterpret_cast<const float4*>(all + (s0 + u) * split_stride +
+                                                              (static_cast<int64_t>(col >> 3) * R + row) * 8);
+            t[u][0] = __ldcg(q);
+            t[u][1] = __ldcg(q + 1);
+        } else {
+            t[u][0] = t[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+}
+__device__ __forceinline__ void part_add4(float (&acc)[8], const float4 (&t)[4][2]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {           // split order
+        acc[0] += t[u][0].x;
+        acc[1] += t[u][0].y;
+        acc[2] += t[u][0].z;
+        acc[3] += t[u][0].w;
+        acc[4] += t[u][1].x;
+        acc[5] += t[u][1].y;
+        acc[6] += t[u][1].z;
+        acc[7] += t[u][1].w;
+    }
+}
+// The last split of a tile: for every 8-column group in [cbeg, cend) of `row`, the sum of
+// all splits' partials in split order, handed to finish(col, acc). With at most 4 splits
+// the next group's partials are requested before the current group is finished, so the
+// loop pays about one memory round trip per two groups instead of one per group.
+template <typename Finish>
+__device__ __forceinline__ void part_reduce(const float* all, int64_t split_stride, int splits, int R, int row,
+                                            int cbeg, int cend, Finish&& finish) {
+    if (splits <= 4) {
+        float4 nx[4][2];
+        if (cbeg < cend) part_load4(all, split_stride, splits, 0, R, row, cbeg, nx);
+        for (int col = cbeg; col < cend; col += 8) {
+            float4 cu[4][2];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                cu[u][0] = nx[u][0];
+                cu[u][1] = nx[u][1];
+            }
+            if (col + 8 < cend) part_load4(all, split_stride, splits, 0, R, row, col + 8, nx);
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            part_add4(acc, cu);
+            finish(col, acc);
+        }
+    } else {
+        for (int col = cbeg; col < cend; col += 8) {
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            for (int s0 = 0; s0 < splits; s0 += 4) {
+                float4 t[4][2];
+                part_load4(all, split_stride, splits, s0, R, row, col, t);
+                part_add4(acc, t);
+            }
+            finish(col, acc);
+        }
+    }
+}
+
 template <int BITS, bool XPERM>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                               const __grid_constant__ CUtensorMap tm_meta,
@@ -379,7 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             // by the runtime ring depth on this thread's path
             int st = 0, s = 0;
             uint32_t ph = 0;
-            for (; st < nsteps; ++st) {
+            const bool go = p.gate == nullptr || tc::gate_wait(p.gate, abort, p.status, p.wait_ns);
+            for (; go && st < nsteps; ++st) {
                 if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ph ^ 1, abort, p.status, p.wait_ns)) break;
                 const int c = c_begin + st * KU;
                 tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CSTAGE + MSTAGE);
@@ -621,8 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 for (int col = cbeg; col < cend; col += 8) {
                     float v[8];
                     acc8(col, v);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) mine[(col + j) * kBM + irow] = v[j];
+                    part_store8(mine, kBM, irow, col, v);
                 }
             }
         }
@@ -642,27 +720,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 if (all_ok) {
                     const int cbeg = ch * (p.BN / 2), cend = cbeg + p.BN / 2;
                     const float* all = p.part + static_cast<int64_t>(tile) * p.splits * p.BN * kBM;
-                    for (int col = cbeg; col < cend; col += 8) {
-                        float acc[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-                        // up to 8 splits' 8 values in flight at once, added in split order
-                        for (int s0 = 0; s0 < p.splits; s0 += 8) {
-                            float t[8][8];
-#pragma unroll
-                            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                                for (int j = 0; j < 8; ++j)
-                                    t[u][j] = (s0 + u < p.splits)
-                                                  ? __ldcg(all + (static_cast<int64_t>(s0 + u) * p.BN + col + j) * kBM + irow)
-                                                  : 0.f;
-#pragma unroll
-                            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                                for (int j = 0; j < 8; ++j) acc[j] += t[u][j];
-                        }
-                        finish8(col, acc);
-                    }
+                    part_reduce(all, static_cast<int64_t>(p.BN) * kBM, p.splits, kBM, irow, cbeg, cend,
+                                [&](int col, const float (&acc)[8]) { finish8(col, acc); });
                 }
                 if (et == 0) p.counters[tile] = 0;
             }
@@ -839,7 +898,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
             if (!p.early_w) pdl_wait();
             int st = 0, s = 0;
             uint32_t ph = 0;
-            for (; st < nsteps; ++st) {
+            const bool go = p.gate == nullptr || tc::gate_wait(p.gate, abort, p.status, p.wait_ns);
+            for (; go && st < nsteps; ++st) {
                 if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ph ^ 1, abort, p.status, p.wait_ns)) break;
                 const int c = c_begin + st * KU;
                 tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CSTAGE + MSTAGE);
@@ -889,11 +949,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
             const uint32_t d_acc = tmem + static_cast<uint32_t>(t * p.acc_stride);
             int xs = 0, xc = 0;                 // activation stage and chunk within it
             uint32_t xph = 0;
+            int sa = 0;                         // A slot of unit u and its phase bit (no division by NSLOT)
+            uint32_t aph = 0;
             bool ok = true;
             int u = 0;
             for (; u < nk; ++u) {
-                const int sa = u % NSLOT;
-                if (!tc::bar_wait(B.a_full + 8 * sa, (u / NSLOT) & 1, abort, p.status, p.wait_ns)) { ok = false; break; }
+                if (!tc::bar_wait(B.a_full + 8 * sa, aph, abort, p.status, p.wait_ns)) { ok = false; break; }
                 if (xc == 0 && !tc::bar_wait(B.x_full + 8 * xs, xph, abort, p.status, p.wait_ns)) { ok = false; break; }
                 tc::fence_after_sync();
                 const uint32_t a_tm = tmem + static_cast<uint32_t>(p.a_col0 + (sa * kRT + t) * 32);
@@ -904,6 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
                     if (++xs == NSX) { xs = 0; xph ^= 1; }
                 }
                 tc::mma_commit(u + 1 < nk ? B.mma_done + 8 * (u % kDoneRing2) : B.acc_full);
+                if (++sa == NSLOT) { sa = 0; aph ^= 1; }
             }
             volatile int never = 0;
             const int committed = ok ? nk - 1 : u;
@@ -923,6 +985,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
         bool ok = true;
         int s = 0;
         uint32_t cph = 0;
+        int dq_slot = 0;                   // A slot of the next unit (no division by NSLOT)
         for (int st = 0; st < nsteps && ok; ++st) {
             if (!tc::bar_wait(B.codes_full + 8 * s, cph, abort, p.status, p.wait_ns)) { ok = false; break; }
             const uint32_t crow = sC + s * CSTAGE + row * 128;
@@ -936,7 +999,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
 #pragma unroll
             for (int c = 0; c < KU; ++c) {
                 const int u = st * KU + c;
-                const int sa = u % NSLOT;
+                const int sa = dq_slot;
+                if (++dq_slot == NSLOT) dq_slot = 0;
                 if (u >= NSLOT) {
                     const int pu = u - NSLOT;
                     if (!tc::bar_wait(B.mma_done + 8 * (pu % kDoneRing2), (pu / kDoneRing2) & 1, abort, p.status,
@@ -1037,8 +1101,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
                 for (int col = 0; col < p.BN; col += 8) {
                     float v[8];
                     tc::tmem_ld8(taddr + col, v);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) mine[(col + j) * kRows2 + row] = v[j];
+                    part_store8(mine, kRows2, row, col, v);
                 }
             }
         }
@@ -1054,26 +1117,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
                 __threadfence();
                 if (all_ok) {
                     const float* all = p.part + static_cast<int64_t>(tile) * p.splits * p.BN * kRows2;
-                    for (int col = 0; col < p.BN; col += 8) {
-                        float acc[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-                        for (int s0 = 0; s0 < p.splits; s0 += 8) {
-                            float tv[8][8];
-#pragma unroll
-                            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                                for (int j = 0; j < 8; ++j)
-                                    tv[u][j] = (s0 + u < p.splits)
-                                                   ? __ldcg(all + (static_cast<int64_t>(s0 + u) * p.BN + col + j) * kRows2 + row)
-                                                   : 0.f;
-#pragma unroll
-                            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                                for (int j = 0; j < 8; ++j) acc[j] += tv[u][j];
-                        }
-                        finish8(col, acc);
-                    }
+                    part_reduce(all, static_cast<int64_t>(p.BN) * kRows2, p.splits, kRows2, row, 0, p.BN,
+                                [&](int col, const float (&acc)[8]) { finish8(col, acc); });
                 }
                 if (et == 0) p.counters[tile] = 0;
             }
@@ -1614,14 +1659,18 @@ struct Plan2 {
     int64_t ws_bytes, counters_bytes;
 };
 
-// gemm_tc2_kernel serves every weight with N a multiple of 256 (two 128-row tiles per
-// CTA); its activation tile is at most 192 rows (M <= 192 in one tile, else tiles of 128).
-bool tc2_eligible(int N) {
+// gemm_tc2_kernel serves weights with N a multiple of 256 (two 128-row tiles per CTA)
+// for more than 128 activation rows; its activation tile is at most 192 rows (M <= 192
+// in one tile, else tiles of 128). Up to 128 rows the 128-row kernel was faster in every
+// weight shape of the OPT-175B layer (its CTAs are half as long, so split-K and the
+// waves over 148 SMs come out better).
+bool tc2_eligible(int M, int N) {
 #ifdef FLEXQ_GEMM_ROWS128_ONLY
+    (void)M;
     (void)N;
     return false;
 #else
-    return N % kRows2 == 0;
+    return M > 128 && N % kRows2 == 0;
 #endif
 }
 
@@ -1811,7 +1860,7 @@ int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, 
 
 int64_t gemm_ws_bytes(int M, int N, int K, int bits) {
     if (gemv_eligible(M, N, bits)) return gemv_plan(M, N, K).ws_bytes;
-    return tc2_eligible(N) ? make_plan2(M, N, K, bits).ws_bytes : make_plan(M, N, K, bits).ws_bytes;
+    return tc2_eligible(M, N) ? make_plan2(M, N, K, bits).ws_bytes : make_plan(M, N, K, bits).ws_bytes;
 }
 
 namespace {
@@ -1896,6 +1945,7 @@ int gemm2_launch(const void* x, const flexq_tensor* W, const void* bias, const v
     if (rc != FLEX_OK) return rc;
     GemmParams gp{};
     gp.wait_ns = pipeline_wait_ns();
+    gp.gate = reinterpret_cast<const volatile int*>(gemm_gate());
     gp.bias = static_cast<const __half*>(bias);
     gp.residual = static_cast<const __half*>(residual);
     gp.y = static_cast<__half*>(y);
@@ -1980,7 +2030,7 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     // small batches of int4 weights: the register-dequant GEMV on mma.sync
     if (gemv_eligible(M, N, bits))
         return gemv_launch(x, W, bias, residual, y, M, relu, nq, qscale, xperm, yperm, ws, ws_bytes, st, kv, early_w);
-    if (tc2_eligible(N))
+    if (tc2_eligible(M, N))
         return gemm2_launch(x, W, bias, residual, y, M, relu, nq, qscale, xperm, yperm, ws, ws_bytes, st, kv, early_w);
     const Plan P = make_plan(M, N, K, bits);
     if (P.ws_bytes > 0 && (ws == nullptr || ws_bytes < P.ws_bytes)) return FLEX_ERR_WORKSPACE;
@@ -1997,6 +2047,7 @@ int gemm_launch(const void* x, const flexq_tensor* W, const void* bias, const vo
     if (rc != FLEX_OK) return rc;
     GemmParams gp{};
     gp.wait_ns = pipeline_wait_ns();
+    gp.gate = reinterpret_cast<const volatile int*>(gemm_gate());
     gp.bias = static_cast<const __half*>(bias);
     gp.residual = static_cast<const __half*>(residual);
     gp.y = static_cast<__half*>(y);
@@ -2065,6 +2116,32 @@ extern "C" int64_t flex_gemm_ws_bytes(int32_t M, int32_t N, int32_t K) {
     FLEX_REQUIRE(N % kBM == 0 && K % 256 == 0, FLEX_ERR_SHAPE);
     const int64_t a = gemm_ws_bytes(M, N, K, 4), b = gemm_ws_bytes(M, N, K, 8);
     return a > b ? a : b;
+}
+
+extern "C" int flex_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t bits, int32_t* out) {
+    FLEX_REQUIRE(out != nullptr && M > 0 && N > 0 && K > 0, FLEX_ERR_INVALID_ARG);
+    FLEX_REQUIRE(bits == 4 || bits == 8, FLEX_ERR_UNSUPPORTED);
+    FLEX_REQUIRE(N % kBM == 0 && K % 256 == 0, FLEX_ERR_SHAPE);
+    if (gemv_eligible(M, N, bits)) {
+        const GemvPlan P = gemv_plan(M, N, K);
+        out[0] = 0;
+        out[1] = P.tiles;
+        out[2] = P.splits;
+        out[3] = P.cluster;
+    } else if (tc2_eligible(M, N)) {
+        const Plan2 P = make_plan2(M, N, K, bits);
+        out[0] = 2;
+        out[1] = P.tiles_n * P.tiles_m;
+        out[2] = P.splits;
+        out[3] = P.cluster;
+    } else {
+        const Plan P = make_plan(M, N, K, bits);
+        out[0] = 1;
+        out[1] = P.tiles_n * P.tiles_m;
+        out[2] = P.splits;
+        out[3] = P.cluster;
+    }
+    return FLEX_OK;
 }
 
 extern "C" int flex_dequant_gemm(const void* x, const flexq_tensor* W, const void* bias, const void* residual,

@@ -42,14 +42,27 @@ __device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity, uint
         : "memory");
     return ok != 0;
 }
+// Non-blocking test of the phase (no suspend): the cheap check for a phase that is
+// usually complete already.
+__device__ __forceinline__ bool bar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
     return t;
 }
 
-// Wait for the phase of `bar` with the given parity to complete. The common path is a
-// try_wait loop (each try_wait sleeps until the phase completes or the hint runs out);
+// Wait for the phase of `bar` with the given parity to complete. A non-blocking test
+// comes first; then a try_wait loop (each try_wait sleeps until the phase completes or the hint runs out);
 // every 16 polls it checks *abort (raised by another role of the CTA) and the elapsed
 // time.
 // After limit_ns (kWaitLimitNs unless the caller passes a limit) it records
@@ -57,6 +70,7 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
                                          uint64_t limit_ns = kWaitLimitNs) {
+    if (bar_test_wait(bar, parity)) return true;          // usually complete already: no suspend
     // the sleep of one poll stays well below the limit (16 polls between time checks)
     const uint32_t hint = limit_ns >= 64ull * kSuspendHintNs ? kSuspendHintNs : static_cast<uint32_t>(limit_ns / 64);
     if (bar_try_wait(bar, parity, hint)) return true;
@@ -75,6 +89,23 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile
             }
         }
     }
+}
+
+// Wait until *gate != 0, with the same limit and abort protocol as bar_wait: after
+// limit_ns it records FLEX_ERR_TIMEOUT, raises *abort and returns false.
+__device__ __forceinline__ bool gate_wait(const volatile int* gate, volatile int* abort, int* status,
+                                          uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (*gate == 0) {
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort = 1;
+            set_status(status, FLEX_ERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(500);
+    }
+    return true;
 }
 
 // ---- thread-block cluster ------------------------------------------------------------

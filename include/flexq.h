@@ -294,6 +294,13 @@ int flex_prefill_attention(const void* q, const void* k, const void* v, int64_t 
  * the next (and in which the GEMM needs no permutation of its own). */
 #define FLEX_GEMM_X_INTERLEAVED 0x10
 int64_t flex_gemm_ws_bytes(int32_t M, int32_t N, int32_t K);
+/* The launch plan flex_dequant_gemm takes for this problem on the current device:
+ * out[0] the kernel (0 the small-batch GEMV on mma.sync, 1 the 128-row tcgen05 GEMM,
+ * 2 the 256-row tcgen05 GEMM), out[1] its output tiles, out[2] the K splits per tile,
+ * out[3] 1 if the splits reduce inside a thread-block cluster, 0 through the workspace
+ * (or no split). Needs a current CUDA device (the plan depends on its SM count and
+ * cluster occupancy). */
+int flex_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t bits, int32_t* out);
 int flex_dequant_gemm(const void* x, const flexq_tensor* W, const void* bias,
                       const void* residual, void* y, int32_t M, int32_t epilogue,
                       void* ws, int64_t ws_bytes, void* stream);
@@ -321,6 +328,14 @@ int flex_get_status(void* stream);
  * launched after the call (a captured CUDA graph keeps the limit of its capture time);
  * process-wide. ns = 0 restores the default of 2 s. Returns the previous limit. */
 uint64_t flex_set_wait_limit_ns(uint64_t ns);
+
+/* Failure-detection test hook: while `gate` is not NULL, every tensor-core GEMM launched
+ * waits, before its first weight load, until the device int32 *gate is non-zero. The
+ * wait has the limit of flex_set_wait_limit_ns; when it runs out the kernel takes the
+ * timeout path described above. A flag that nothing sets thus makes that path run
+ * without breaking any kernel. Process-wide; returns the previous gate. gate must stay
+ * valid while kernels launched with it may run. Pass NULL to remove it. */
+const int32_t* flex_set_gemm_gate(const int32_t* gate);
 
 /* Layout of the ABI structs as this library was compiled: which = 0 flexq_config,
  * 1 flexq_tensor, 2 flex_layer, 3 flex_kv_cache; field = -1 returns sizeof, field = i

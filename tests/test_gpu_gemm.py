@@ -215,3 +215,47 @@ def test_gemm_interleaved_activations(M, N, K):
         assert torch.equal(y1, y2)
     else:
         assert (y1.float() - y2.float()).abs().max().item() <= 1e-2 * y1.float().abs().max().item() + 1e-3
+
+
+def _plan_cases():
+    """(M, N, K) candidates whose plans cover the split-K reduction paths: for each of
+    the two tensor-core kernels, no split, splits through a thread-block cluster, and
+    splits through the workspace ticket with at most 4 and with more than 4 splits."""
+    cands = []
+    for M in (48, 144):
+        for tiles in (1, 2, 6, 12, 20, 24, 28, 40, 96):
+            for K in (2048, 12288, 49152):
+                N = tiles * (256 if M > 128 else 128)
+                cands.append((M, N, K))
+    return cands
+
+
+def test_gemm_split_reduction_paths():
+    """Every split-K reduction path the device's plans reach is parity-checked against
+    the oracle on sampled output features and gives identical bits on a second call;
+    the workspace tickets are back at zero. The ticket path with at most 4 splits and
+    the one with more (the partials are added 4 splits at a time) are required."""
+    seen = {}
+    for M, N, K in _plan_cases():
+        pl = fq.flex_gemm_plan(M, N, K)
+        path = (pl["kernel"], "none" if pl["splits"] == 1 else ("cluster" if pl["cluster"] else
+                                                              ("ticket<=4" if pl["splits"] <= 4 else "ticket>4")))
+        if path not in seen or N * K < seen[path][1] * seen[path][2]:
+            seen[path] = (M, N, K)
+    for k in ("tc128", "tc256"):
+        assert (k, "ticket<=4") in seen and (k, "ticket>4") in seen, sorted(seen)
+    for path, (M, N, K) in sorted(seen.items()):
+        x = synth.activations((M, K), 90, device="cuda")
+        w = synth.normal_f16((N, K), 91, 0.02, device="cuda")
+        W = fq.CompressedWeight(w, 4, 64)
+        ws = torch.zeros(max(16, fq.flex_gemm_ws_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
+        y1 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        y2 = torch.empty_like(y1)
+        fq.flex_dequant_gemm(x, W, None, None, y1, M, fq.FLEX_EPI_NONE, ws)
+        fq.flex_dequant_gemm(x, W, None, None, y2, M, fq.FLEX_EPI_NONE, ws)
+        sync_status()
+        assert torch.equal(y1, y2), path
+        assert int(ws[:2048].view(torch.int32).abs().sum()) == 0, path
+        rows = np.unique(np.linspace(0, N - 1, 24).astype(np.int64))
+        ref = _oracle_gemm(to_np(x), to_np(w), None, None, fq.FLEX_EPI_NONE, 4, rows=rows)
+        assert_layer_close(y1[:, torch.from_numpy(rows).cuda()], ref, f"{path} {M}x{N}x{K}")

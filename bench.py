@@ -292,18 +292,25 @@ class Stack:
         self.y_pre = torch.empty_like(self.x_pre)
         self.ws_dec = torch.zeros(fq.flex_workspace_bytes(self.layers[0], nc * b, 1), dtype=torch.uint8, device=dev)
 
-    def prefill(self):
+    def prefill(self, stream=None, events=None):
         """Prompt of every gpu-batch through the stack (writes cache slots [0, prompt));
-        several gpu-batches share one pass over each layer's weights."""
-        fq, cfg = self.fq, self.cfg
+        several gpu-batches share one pass over each layer's weights. With `events`
+        (a list), a pair of CUDA events on `stream` brackets each layer call."""
+        fq, cfg, torch = self.fq, self.cfg, self.torch
         src, dst = self.x_pre, self.y_pre
         for l in range(cfg["layers"]):
+            if events is not None:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
             if cfg["calls"] == 1:
                 fq.flex_prefill_layer(self.layers[l], self.caches[l][0], src, dst, cfg["call_batch"], cfg["prompt"],
-                                      self.ws_pre)
+                                      self.ws_pre, stream=stream)
             else:
                 fq.flex_prefill_layer_batches(self.layers[l], self.caches[l], src, dst, cfg["call_batch"],
-                                              cfg["prompt"], self.ws_pre)
+                                              cfg["prompt"], self.ws_pre, stream=stream)
+            if events is not None:
+                e1.record(stream)
+                events.append((e0, e1))
             src, dst = dst, src
         # the last layer's output is not kept: a synthetic stack has no LM head
 
@@ -693,15 +700,15 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
     # each part's time goes to its working kernel (the attention's combine step, when the
     # key range is split, is timed with it); one layer call runs 4 GEMMs, 1 attention, 2 LNs
     per_kernel = {}
-    for part, calls in (("gemm_qkv", 1), ("gemm_out", 1), ("gemm_fc1", 1), ("gemm_fc2", 1),
-                        ("decode_attention", 1), ("layernorm", 2)):
+    for part, per_call in (("gemm_qkv", 1), ("gemm_out", 1), ("gemm_fc1", 1), ("gemm_fc2", 1),
+                           ("decode_attention", 1), ("layernorm", 2)):
         v = kern[part]
         e = per_kernel.setdefault(v["kernel"], dict(launches=0, ms=0.0, bytes=0.0, flops=0.0, parts=[],
                                                     source=v["source"]))
-        e["launches"] += calls
-        e["ms"] += calls * v["ms"]
-        e["bytes"] += calls * v["bytes"]
-        e["flops"] += calls * v["flops"]
+        e["launches"] += per_call
+        e["ms"] += per_call * v["ms"]
+        e["bytes"] += per_call * v["bytes"]
+        e["flops"] += per_call * v["flops"]
         e["parts"].append(part)
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"])
     dk = per_kernel[dom]
@@ -731,18 +738,18 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
     stack_ok = hasattr(stack, "ws_pre")
     prefill = None
     if stack_ok:
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        stack.prefill()
+        stack.prefill(stream)
         torch.cuda.synchronize()
-        e0.record()
-        stack.prefill()
-        e1.record()
+        evs = []
+        with torch.cuda.stream(stream):
+            stack.prefill(stream, evs)
         torch.cuda.synchronize()
-        pms = e0.elapsed_time(e1) / (L * calls)
+        each = [e_a.elapsed_time(e_b) for e_a, e_b in evs]             # ms per layer call
+        pms = sum(each) / (L * calls)
         T = b * s
         flops = 2 * T * (4 * h * h + 2 * h * ffn) + 2 * b * nh * s * s * d       # causal: half of 4*b*s^2*h
         prefill = {"tokens_per_s_per_layer": T / (pms / 1e3), "ms_per_layer_call": pms,
+                   "ms_each_layer_call": each,
                    "tflops": flops / (pms * 1e9), "frac_tensor_peak": flops / (pms * 1e9) / tpk,
                    "peak_note": "fp16 tensor peak = measured bf16 cuBLAS peak (same rate)"}
     rc = fq.flex_get_status()

@@ -107,6 +107,7 @@ struct GemmParams {
 
 struct Bars {
     uint32_t codes_full, codes_empty, x_full, a_full, mma_done, acc_full, drain;   // drain: one per issuer
+    uint32_t red;          // gemm_tc2_kernel: two barriers of the split-K reduction's bulk loads
 };
 
 __device__ __forceinline__ uint32_t dequant_pair(uint32_t raw_pair_bits, uint32_t step2, uint32_t mn2) {
@@ -829,7 +830,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
     B.mma_done = B.a_full + 8 * NSLOT;
     B.acc_full = B.mma_done + 8 * kDoneRing2;
     B.drain = B.acc_full + 8;
-    const uint32_t misc = B.drain + 8 * 4;
+    B.red = B.drain + 8 * 4;
+    const uint32_t misc = B.red + 8 * 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (misc - base));
     volatile int* abort = reinterpret_cast<volatile int*>(gbase + (misc - base) + 4);
     volatile int* last_flag = reinterpret_cast<volatile int*>(gbase + (misc - base) + 8);
@@ -845,6 +847,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
         for (int s = 0; s < kDoneRing2; ++s) tc::bar_init(B.mma_done + 8 * s, kRT);   // both issuers commit each unit
         tc::bar_init(B.acc_full, kRT);
         for (int i = 0; i < 4; ++i) tc::bar_init(B.drain + 8 * i, 1);
+        tc::bar_init(B.red, 1);
+        tc::bar_init(B.red + 8, 1);
         *abort = 0;
         *last_flag = 0;
         tc::bar_fence_init();
@@ -873,6 +877,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
     const bool kv_on = p.kv.codes[0][0] != nullptr && n0t >= p.kv.h;
     float bias_n = 0.f;
     uint32_t all_ok = 0;
+    // the fp32 partial of this split fits in the rings (drained by then): staged there for one
+    // bulk store, and the reduction's bulk loads use the same space
+    const bool stage_ok = static_cast<uint32_t>(p.BN) * kRows2 * 4 <= p.off_bar;
     auto finish8 = [&](int col, const float (&v)[8]) {
         float r[8];
 #pragma unroll
@@ -1098,10 +1105,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
             } else {
                 float* mine = p.part + (static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * p.splits + split) *
                                            p.BN * kRows2;
-                for (int col = 0; col < p.BN; col += 8) {
-                    float v[8];
-                    tc::tmem_ld8(taddr + col, v);
-                    part_store8(mine, kRows2, row, col, v);
+                if (stage_ok) {
+                    // the partial, in its workspace layout, into the drained rings; one bulk
+                    // store (issued with the ticket below) moves it to the workspace
+                    for (int col = 0; col < p.BN; col += 8) {
+                        float v[8];
+                        tc::tmem_ld8(taddr + col, v);
+                        const uint32_t sa = base + ((col >> 3) * kRows2 + row) * 32;
+                        tc::sts128(sa, v[0], v[1], v[2], v[3]);
+                        tc::sts128(sa + 16, v[4], v[5], v[6], v[7]);
+                    }
+                    tc::fence_proxy_async_smem();
+                } else {
+                    for (int col = 0; col < p.BN; col += 8) {
+                        float v[8];
+                        tc::tmem_ld8(taddr + col, v);
+                        part_store8(mine, kRows2, row, col, v);
+                    }
                 }
             }
         }
@@ -1109,15 +1129,98 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
             // ticket, taken by every split (see gemm_tc_kernel); the last adds the partials in split order
             const int et = (warp - 4) * 32 + lane;
             const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+            const int64_t pstride = static_cast<int64_t>(p.BN) * kRows2;     // floats per partial
             __threadfence();
             asm volatile("bar.sync 1, 256;" ::: "memory");
-            if (et == 0) *last_flag = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+            if (et == 0) {
+                if (all_ok && stage_ok) {
+                    tc::bulk_store(p.part + (static_cast<int64_t>(tile) * p.splits + split) * pstride, base,
+                                   static_cast<uint32_t>(pstride * 4));
+                    tc::bulk_commit();
+                    tc::bulk_wait_all();
+                    tc::fence_proxy_async_global();
+                    __threadfence();
+                }
+                *last_flag = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+            }
             asm volatile("bar.sync 1, 256;" ::: "memory");
             if (*last_flag) {
                 __threadfence();
-                if (all_ok) {
-                    const float* all = p.part + static_cast<int64_t>(tile) * p.splits * p.BN * kRows2;
-                    part_reduce(all, static_cast<int64_t>(p.BN) * kRows2, p.splits, kRows2, row, 0, p.BN,
+                const float* all = p.part + static_cast<int64_t>(tile) * p.splits * pstride;
+                if (all_ok && stage_ok && (p.off_bar / 2) >= static_cast<uint32_t>(p.splits) * kRows2 * 32) {
+                    // the partials in batches of C column groups (8 KB each per split), bulk-
+                    // loaded into two alternating halves of the drained rings; each thread adds
+                    // its row's 8 values of every split in split order
+                    const int ng = p.BN / 8;
+                    const uint32_t half = (p.off_bar / 2) & ~15u;
+                    int C = static_cast<int>(half / (static_cast<uint32_t>(p.splits) * kRows2 * 32));
+                    if (C > ng) C = ng;
+                    const int nb = (ng + C - 1) / C;
+                    auto issue = [&](int bi) {
+                        const int g0 = bi * C, gc = min(C, ng - g0);
+                        const uint32_t dst = base + (bi & 1) * half;
+                        const uint32_t bytes = static_cast<uint32_t>(gc) * kRows2 * 32;
+                        tc::bar_arrive_expect_tx(B.red + 8 * (bi & 1), bytes * p.splits);
+                        for (int sp = 0; sp < p.splits; ++sp)
+                            tc::bulk_load(dst + sp * static_cast<uint32_t>(C) * kRows2 * 32,
+                                          all + sp * pstride + static_cast<int64_t>(g0) * kRows2 * 8, bytes,
+                                          B.red + 8 * (bi & 1));
+                    };
+                    if (et == 0) {
+                        tc::fence_proxy_async_global();
+                        issue(0);
+                        if (nb > 1) issue(1);
+                    }
+                    int waited = 0;
+                    bool rok = true;
+                    for (int bi = 0; bi < nb; ++bi) {
+                        const bool w = tc::bar_wait(B.red + 8 * (bi & 1), (bi >> 1) & 1, abort, p.status, p.wait_ns);
+                        // one decision for all 256 threads (the loop has named barriers)
+                        uint32_t wall;
+                        asm volatile(
+                            "{\n\t.reg .pred p, q;\n\t"
+                            "setp.ne.u32 p, %1, 0;\n\t"
+                            "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
+                            "selp.u32 %0, 1, 0, q;\n\t}"
+                            : "=r"(wall)
+                            : "r"(w ? 1u : 0u)
+                            : "memory");
+                        if (!wall) {
+                            rok = false;
+                            break;
+                        }
+                        waited = bi + 1;
+                        const uint32_t src = base + (bi & 1) * half;
+                        const int g0 = bi * C, gc = min(C, ng - g0);
+                        for (int gi = 0; gi < gc; ++gi) {
+                            float acc[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+                            for (int sp = 0; sp < p.splits; ++sp) {          // split order
+                                const uint32_t q = src + ((sp * C + gi) * kRows2 + row) * 32;
+                                const float4 lo = tc::lds128f(q), hi = tc::lds128f(q + 16);
+                                acc[0] += lo.x;
+                                acc[1] += lo.y;
+                                acc[2] += lo.z;
+                                acc[3] += lo.w;
+                                acc[4] += hi.x;
+                                acc[5] += hi.y;
+                                acc[6] += hi.z;
+                                acc[7] += hi.w;
+                            }
+                            finish8((g0 + gi) * 8, acc);
+                        }
+                        asm volatile("bar.sync 1, 256;" ::: "memory");       // this half is free again
+                        if (et == 0 && bi + 2 < nb) issue(bi + 2);
+                    }
+                    // a wait that gave up: let the copies already issued land before the CTA exits
+                    const int issued = rok ? nb : min(nb, waited + 2);
+                    for (int bi = waited; bi < issued; ++bi) {
+                        volatile int never = 0;
+                        tc::bar_wait(B.red + 8 * (bi & 1), (bi >> 1) & 1, &never, p.status);
+                    }
+                } else if (all_ok) {
+                    part_reduce(all, pstride, p.splits, kRows2, row, 0, p.BN,
                                 [&](int col, const float (&acc)[8]) { finish8(col, acc); });
                 }
                 if (et == 0) p.counters[tile] = 0;
@@ -1711,7 +1814,7 @@ Plan2 make_plan2(int M, int N, int K, int bits) {
     P.off_c = nsx * xstage;
     P.off_m = P.off_c + nsc * kRows2 * 128;
     P.off_bar = P.off_m + nsc * kRows2 * kMetaChunks * 4;
-    P.smem = P.off_bar + 8 * (2 * nsc + nsx + P.nslot + kDoneRing2 + 1 + 4) + 16 + 256 + 1024;
+    P.smem = P.off_bar + 8 * (2 * nsc + nsx + P.nslot + kDoneRing2 + 1 + 4 + 2) + 16 + 256 + 1024;
     // split-K through distributed shared memory when the partial tile fits in the drained
     // rings and every tile's cluster can be resident at once, else workspace and tickets
     const bool fits = static_cast<uint32_t>(P.BN) * kRows2 * 4 <= P.off_bar;

@@ -281,17 +281,33 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool pre
 }
 
 // One CTA (4 warps) streams the key range [j0, j1) of one (sequence, head) in stages of
-// DT_KEYS keys through a cp.async ring (3 stages deep at head_dim 64, 2 at 128); in a stage warp w owns keys
+// DT_KEYS keys through a cp.async ring of DT_STAGES stages; in a stage warp w owns keys
 // [32 w, 32 w + 32) as two 16-key tiles, with one online-softmax update per stage.
 // Writes the split's partial {max, sum, unnormalised output} for the combine kernel;
 // with a single split (gridDim.y == 1) it does the combine step itself: it folds in the
 // fresh key/value of the current token and writes the normalised output o (in the
 // interleaved 8-block order when perm != 0).
 constexpr int DT_KEYS = 128;
+
+// Position, in 16-byte chunks, of chunk u (key u / 4, chunk u % 4) of a stage's value
+// codes at head_dim 128. In the PV step the 16 lanes of a half-warp read 8 bytes each
+// from chunks 0-1 (or 2-3) of four keys of one parity; stored in key order those all
+// fall in the same 8 banks (a 4-way conflict). Swapping keys 2j and 2j+1 when bit 1 of
+// the key is set, and chunks c and c ^ 2 when bit 2 is set, spreads them over all 32
+// banks. Bits 1 and 2 of the key index are the same in the stage and in its 16-key
+// tile, so the reader applies the same map to its tile-local key. head_dim 64 keeps the
+// plain order.
+template <int D>
+__device__ __forceinline__ int v_chunk(int u) {
+    if (D != 128) return u;
+    const int key = u >> 2, c = u & 3;
+    return ((key ^ ((key >> 1) & 1)) << 2) | (c ^ (((key >> 2) & 1) << 1));
+}
 #ifndef FLEXQ_DT_STAGES
 #define FLEXQ_DT_STAGES 2
 #endif
 constexpr int DT_STAGES = FLEXQ_DT_STAGES;  // stages of DT_KEYS keys in flight per CTA
+static_assert(DT_STAGES >= 2, "the stage loop refills the slot of the previous stage");
 
 // Dynamic shared memory of decode_attn_tc_kernel<D, GS>: the ring of stages, each the
 // codes and metadata of DT_KEYS keys and values.
@@ -358,7 +374,7 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
             const bool ok = kbase + (u * 16) / KB < nkeys;
             const int64_t off = ok ? static_cast<int64_t>(kbase) * KB + u * 16 : 0;
             cp_async16(st + u * 16, kc_src + off, ok);
-            cp_async16(st + CODE + u * 16, vc_src + off, ok);
+            cp_async16(st + CODE + v_chunk<D>(u) * 16, vc_src + off, ok);
         }
 #pragma unroll
         for (int i = 0; i < META / DA_THREADS; ++i) {
@@ -385,21 +401,34 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
     pdl_trigger();
     if (!early_kv) prologue();
 
-    // ---- query: group sums and the QK B operand (this thread's D/4 dims, column g)
+    // ---- query: group sums (Qg = sum of q, QC = sum of 1024 q_even + 64 q_odd over the
+    // group's dims), shared out by the warp: lane l takes dims [DPL l, DPL l + DPL), the
+    // LPG lanes of a group add theirs, and every lane reads each group's total
     const __half* qp = q + static_cast<int64_t>(b) * row_stride + head * D;
+    constexpr int DPL = D / 32;            // dims per lane (4 or 2)
+    constexpr int LPG = GS / DPL;          // lanes per group
+    float qg_l = 0.f, qc_l = 0.f;
+    if (DPL == 4) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(qp) + lane);
+        const float e0 = h2f_lo(w.x), o0 = h2f_hi(w.x), e1 = h2f_lo(w.y), o1 = h2f_hi(w.y);
+        qg_l = (e0 + o0) + (e1 + o1);
+        qc_l = 1024.f * (e0 + e1) + 64.f * (o0 + o1);
+    } else {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(qp) + lane);
+        const float e0 = h2f_lo(w), o0 = h2f_hi(w);
+        qg_l = e0 + o0;
+        qc_l = 1024.f * e0 + 64.f * o0;
+    }
+#pragma unroll
+    for (int off = LPG / 2; off > 0; off >>= 1) {
+        qg_l += __shfl_xor_sync(0xffffffffu, qg_l, off);
+        qc_l += __shfl_xor_sync(0xffffffffu, qc_l, off);
+    }
     float Qg[G], QC[G];
 #pragma unroll
-    for (int n = 0; n < G; ++n) Qg[n] = QC[n] = 0.f;
-#pragma unroll
-    for (int v = 0; v < D / 8; ++v) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(qp) + v);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float lo = h2f_lo(ww[k]), hi = h2f_hi(ww[k]);     // even, odd dim
-            Qg[(8 * v) / GS] += lo + hi;
-            QC[(8 * v) / GS] += 1024.f * lo + 64.f * hi;
-        }
+    for (int n = 0; n < G; ++n) {
+        Qg[n] = __shfl_sync(0xffffffffu, qg_l, n * LPG);
+        QC[n] = __shfl_sync(0xffffffffu, qc_l, n * LPG);
     }
     const int tgrp = (t * (D / 4)) / GS;   // group of this thread's QK dims
     const __half sixteenth = __float2half(0.0625f);
@@ -434,11 +463,13 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
 #pragma unroll
     for (int i = 0; i < NMT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
 
+    // One barrier per stage: after it, stage s has landed for every thread and every warp
+    // has finished stage s - 1, whose slot then takes stage s + DT_NS - 1.
     for (int s = 0; s < nst; ++s) {
+        cp_async_wait<DT_NS - 2>();
+        __syncthreads();
         if (s + DT_NS - 1 < nst) load_stage(s + DT_NS - 1);
         cp_async_commit();
-        cp_async_wait<DT_NS - 1>();
-        __syncthreads();
         const int kw0 = s * DT_KEYS + warp * 32;                 // the warp's first key
         if (kw0 < nkeys) {
             const uint8_t* st = ring[s % DT_NS];
@@ -551,7 +582,10 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
                 for (int u = 0; u < 4; ++u) {
                     const int key = 2 * t + (u & 1) + 8 * (u >> 1);
                     if (VW == 2) {
-                        const uint2 a = *reinterpret_cast<const uint2*>(vc + key * KB);
+                        // 16-byte chunk g/2 of the key sits where v_chunk put it
+                        const int pk = key ^ ((key >> 1) & 1), pc = (g >> 1) ^ (((key >> 2) & 1) << 1);
+                        const uint2 a = *reinterpret_cast<const uint2*>(st + CODE + (warp * 32 + tile * 16 + pk) * KB +
+                                                                        pc * 16 + (g & 1) * 8);
                         vk[u][0] = a.x;
                         vk[u][1 % (VW > 0 ? VW : 1)] = a.y;
                     } else {
@@ -570,7 +604,6 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
                 }
             }
         }
-        __syncthreads();                   // the slot is refilled by the next iteration
     }
     cp_async_wait<0>();
 

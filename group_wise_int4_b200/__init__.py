@@ -106,6 +106,7 @@ _SIGS = {
     "flex_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "flex_set_gemm_gate": (_P, [_P]),
     "flex_gemm_plan": (_I32, [_I32, _I32, _I32, _I32, _P]),
+    "flex_set_gemm_streamk": (_I32, [_I32]),
     "flex_status_string": (ctypes.c_char_p, [_I32]),
     "flex_abi_layout": (_I64, [_I32, _I32]),
 }
@@ -469,7 +470,13 @@ def flex_gemm_plan(M: int, N: int, K: int, bits: int = 4) -> dict:
     """The launch plan of flex_dequant_gemm for this problem on the current device."""
     out = (ctypes.c_int32 * 4)()
     _check(lib().flex_gemm_plan(int(M), int(N), int(K), int(bits), ctypes.cast(out, ctypes.c_void_p)), "flex_gemm_plan")
-    return {"kernel": ("gemv", "tc128", "tc256")[out[0]], "tiles": out[1], "splits": out[2], "cluster": bool(out[3])}
+    return {"kernel": ("gemv", "tc128", "tc256")[out[0]], "tiles": out[1], "splits": out[2],
+            "reduce": "none" if out[2] == 1 and out[3] == 0 else ("ticket", "cluster", "streamk")[out[3]]}
+
+
+def flex_set_gemm_streamk(enable: bool) -> bool:
+    """Stream-K schedule of the 256-row GEMM for later plans; returns the previous setting."""
+    return bool(lib().flex_set_gemm_streamk(1 if enable else 0))
 
 
 def flex_set_gemm_gate(gate) -> int:

@@ -51,6 +51,13 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pr
     const int n = pred ? 16 : 0;
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(n) : "memory");
 }
+// unpredicated forms (the whole 16 / 4 bytes are always copied)
+__device__ __forceinline__ void cp_async16u(uint32_t s, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4u(uint32_t s, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(s), "l"(gmem) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -368,6 +375,27 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
     auto load_stage = [&](int s) {
         uint8_t* st = ring[s % DT_NS];
         const int kbase = s * DT_KEYS;
+        if (kbase + DT_KEYS <= nkeys) {
+            // a whole stage: no per-copy predicate or clamped address
+            const uint32_t s0 = static_cast<uint32_t>(__cvta_generic_to_shared(st));
+            const uint8_t* kc = kc_src + static_cast<int64_t>(kbase) * KB;
+            const uint8_t* vc = vc_src + static_cast<int64_t>(kbase) * KB;
+            const uint32_t* km = km_src + static_cast<int64_t>(kbase) * G;
+            const uint32_t* vm = vm_src + static_cast<int64_t>(kbase) * G;
+#pragma unroll
+            for (int i = 0; i < CODE / (16 * DA_THREADS); ++i) {
+                const int u = threadIdx.x + i * DA_THREADS;
+                cp_async16u(s0 + u * 16, kc + u * 16);
+                cp_async16u(s0 + CODE + v_chunk<D>(u) * 16, vc + u * 16);
+            }
+#pragma unroll
+            for (int i = 0; i < META / DA_THREADS; ++i) {
+                const int u = threadIdx.x + i * DA_THREADS;
+                cp_async4u(s0 + 2 * CODE + u * 4, km + u);
+                cp_async4u(s0 + 2 * CODE + META * 4 + u * 4, vm + u);
+            }
+            return;
+        }
 #pragma unroll
         for (int i = 0; i < CODE / (16 * DA_THREADS); ++i) {
             const int u = threadIdx.x + i * DA_THREADS;

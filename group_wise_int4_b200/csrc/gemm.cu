@@ -35,6 +35,7 @@
 // on scheduling. Every mbarrier wait is bounded: on
 // expiry the CTA records FLEX_ERR_TIMEOUT in the device status word, drains its own
 // copies and MMAs, frees TMEM and exits (still taking part in the cluster barriers).
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -97,6 +98,10 @@ struct GemmParams {
     int cluster;
     float* part;
     int* counters;
+    // gemm_tc2_kernel stream-K schedule (sk = 1): the tiles' K steps laid end to end,
+    // sk_total of them, shared out evenly over the grid; tiles numbered tm * sk_tiles_n + tn
+    int sk, sk_tiles_n;
+    int64_t sk_total;
     uint32_t off_x, off_c, off_m, off_bar;
     uint32_t tmem_cols;
     // fused store_cache (QKV projection): output features [kv.h, 2 kv.h) are the keys and
@@ -193,44 +198,54 @@ __device__ __forceinline__ void kv_store8_bits(const GemmParams& p, const __half
     const int sec = (n0 - p.kv.h) / p.kv.h;                // 0 keys, 1 values
     const int f = n - p.kv.h - sec * p.kv.h;
     const int head = f / p.kv.hd, dim = f % p.kv.hd;
-    // min / max of the 8 columns as 4 half2 pairs
-    __half2 mn2[4], mx2[4];
+    // {min, max} of each of the 8 columns over the warp's 32 rows, as half2 (min low, max
+    // high), reduced and scattered: after the xor-16/8/4 rounds lane l holds column
+    // (l >> 2) & 7 over 8 lanes, and the xor-2/1 rounds finish it over all 32
+    auto comb = [](uint32_t a, uint32_t b) -> uint32_t {
+        const __half2 lo = __hmin2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+        const __half2 hi = __hmax2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+        return prmt(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi), 0x7610u);
+    };
+    uint32_t v[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) mn2[k] = mx2[k] = __halves2half2(o16[2 * k], o16[2 * k + 1]);
+    for (int j = 0; j < 8; ++j) v[j] = pack_half2_bits(o16[j], o16[j]);
+    const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0, b2 = (lane & 4) != 0;
+    uint32_t w[4], x[2];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t got = __shfl_xor_sync(0xffffffffu, b4 ? v[k] : v[k + 4], 16);
+        w[k] = comb(b4 ? v[k + 4] : v[k], got);
+    }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t a = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t*>(&mn2[k]), off);
-            const uint32_t b = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t*>(&mx2[k]), off);
-            mn2[k] = __hmin2(mn2[k], *reinterpret_cast<const __half2*>(&a));
-            mx2[k] = __hmax2(mx2[k], *reinterpret_cast<const __half2*>(&b));
-        }
+    for (int k = 0; k < 2; ++k) {
+        const uint32_t got = __shfl_xor_sync(0xffffffffu, b3 ? w[k] : w[k + 2], 8);
+        x[k] = comb(b3 ? w[k + 2] : w[k], got);
+    }
+    uint32_t y = comb(b2 ? x[1] : x[0], __shfl_xor_sync(0xffffffffu, b2 ? x[0] : x[1], 4));
+    y = comb(y, __shfl_xor_sync(0xffffffffu, y, 2));
+    y = comb(y, __shfl_xor_sync(0xffffffffu, y, 1));
+    const int jc = (lane >> 2) & 7;                        // the column this lane now holds
     if (p.kv.gs == 64) {
-        const int w = warp - 4, pairbar = 2 + (w >> 1);
-        if (lane == 0)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                kv_red[(w * 4 + k) * 2] = *reinterpret_cast<uint32_t*>(&mn2[k]);
-                kv_red[(w * 4 + k) * 2 + 1] = *reinterpret_cast<uint32_t*>(&mx2[k]);
-            }
+        // a group of 64 rows spans the two warps of a pair: add the partner's column
+        const int wi = warp - 4, pairbar = 2 + (wi >> 1);
+        if ((lane & 3) == 0) kv_red[wi * 8 + jc] = y;
         asm volatile("bar.sync %0, 64;" ::"r"(pairbar) : "memory");
-        const int pw = w ^ 1;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t a = kv_red[(pw * 4 + k) * 2], b = kv_red[(pw * 4 + k) * 2 + 1];
-            mn2[k] = __hmin2(mn2[k], *reinterpret_cast<const __half2*>(&a));
-            mx2[k] = __hmax2(mx2[k], *reinterpret_cast<const __half2*>(&b));
-        }
+        y = comb(y, kv_red[(wi ^ 1) * 8 + jc]);
         asm volatile("bar.sync %0, 64;" ::"r"(pairbar) : "memory");   // kv_red is reused by the next call
     }
+    // this lane's column: scale (one division per lane), then every column's {min, scale}
+    // to every lane
+    const __half mnh = __ushort_as_half(static_cast<unsigned short>(y & 0xFFFFu));
+    const __half mxh = __ushort_as_half(static_cast<unsigned short>(y >> 16));
+    const __half s16c = group_scale16<BITS>(__half2float(mnh), __half2float(mxh));
+    const uint32_t ms = pack_half2_bits(mnh, s16c);
     const int gph = p.kv.hd / p.kv.gs;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
+        const uint32_t msj = __shfl_sync(0xffffffffu, ms, 4 * j);
         const int m = m0 + col + j;
-        const float mn = (j & 1) ? __high2float(mn2[j >> 1]) : __low2float(mn2[j >> 1]);
-        const float mx = (j & 1) ? __high2float(mx2[j >> 1]) : __low2float(mx2[j >> 1]);
-        const __half s16 = group_scale16<BITS>(mn, mx);
+        const float mn = h2f_lo(msj);
+        const __half s16 = __ushort_as_half(static_cast<unsigned short>(msj >> 16));
         const uint32_t q = quant_one<BITS>(__half2float(o16[j]), mn, __half2float(s16));
         const uint32_t qn = __shfl_down_sync(0xffffffffu, q, 1);
         if (m >= p.M) continue;
@@ -771,9 +786,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 
 // ---------------------------------------------------------------------------------------
 // 256 weight rows per CTA (two 128-row tiles, t = 0, 1), for N a multiple of 256 and up
-// to 192 activation rows per tile (BN). Each activation tile brought in from L2 then
-// feeds both weight tiles, which halves the activation traffic per weight row: with 128
-// rows per CTA the re-read activations, not the weights or the MMAs, set the pace.
+// to 192 activation rows per tile (BN). Each activation tile brought in from L2 feeds
+// both weight tiles (half the activation traffic per weight row of the 128-row kernel),
+// and the two tiles' MMA issuers run side by side. Above 128 activation rows this kernel
+// was the faster of the two at every OPT-175B weight shape measured.
 //
 //   warp 0      TMA: code tiles [256 rows][128 B] and metadata [256 rows][4 groups]
 //   warp 1      TMA: activation tiles [BN rows][64] fp16 (128-byte swizzle), XU chunks per stage
@@ -786,20 +802,82 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // TMEM: accumulator of tile t at columns [t acc_stride, t acc_stride + BN); from a_col0 on,
 // nslot A slots of one chunk per tile (slot s of tile t at a_col0 + (s * 2 + t) * 32). A
 // "unit" is one chunk: one A slot fill, one MMA issue round per tile, one commit per
-// issuer (the mma_done ring counts units). Everything else - bounded waits, abort and
-// drain, split-K through clusters or tickets, the epilogue and the fused store_cache - is
-// as in gemm_tc_kernel.
+// issuer (the mma_done ring counts units, across all segments of the CTA). A CTA works
+// through one or more segments (see SegWalk); between segments the issuers wait for the
+// epilogue to have read the accumulators (acc_full, one phase per segment). Bounded waits,
+// abort and drain, split-K through clusters or tickets and the fused store_cache are as
+// in gemm_tc_kernel.
 constexpr int kRT = 2;                  // 128-row tiles per CTA
+// 12 warps: 0 code TMA, 1 activation TMA, 2 and 3 the MMA issuers of tiles 0 and 1,
+// 4-11 dequantisation and the epilogue. One CTA per SM, so a thread may hold up to 168
+// registers (the epilogue with the fused store_cache needs about 140).
+constexpr int kThreads2 = 384;
 constexpr int kRows2 = kRT * kBM;       // 256
 constexpr int kDoneRing2 = 16;          // mma_done barriers (units)
+constexpr int kMaxPieces = 8;           // stream-K: later pieces of one tile that its owner adds
+
+// A CTA's work, as segments of K steps of one tile. A classic launch gives each CTA one
+// segment: tile (blockIdx.x, blockIdx.y), the steps of K split blockIdx.z. A stream-K
+// launch (p.sk) lays the tiles' steps end to end and gives CTA c the contiguous share
+// [c total / G, (c + 1) total / G): a run of segments that may start and end inside a
+// tile. A segment that covers its whole tile finishes it directly. A tile shared by
+// several CTAs is finished by the CTA holding its first steps (the owner; always its
+// CTA's last segment), after the later pieces - each the first segment of one of the
+// next CTAs, written to that CTA's partial slot early in its run - have been published.
+struct Seg {
+    int tn, tm;            // tile (256-row block of N, BN-column block of M)
+    int k0, k1;            // steps [k0, k1) of the tile's nst steps
+    bool whole, owner;     // covers the tile / first piece of a shared tile
+};
+
+struct SegWalk {
+    int64_t pos, end;      // stream-K: the next step and the end of this CTA's share
+    int nst, tiles_n;
+    bool sk, done;
+    __device__ SegWalk(const GemmParams& p, int nst_) : nst(nst_), tiles_n(p.sk_tiles_n), sk(p.sk != 0), done(false) {
+        if (sk) {
+            pos = static_cast<int64_t>(blockIdx.x) * p.sk_total / gridDim.x;
+            end = static_cast<int64_t>(blockIdx.x + 1) * p.sk_total / gridDim.x;
+        } else {
+            pos = end = 0;
+        }
+    }
+    __device__ bool next(const GemmParams& p, int KU, Seg& sg) {
+        if (done) return false;
+        if (!sk) {
+            done = true;
+            sg.tn = blockIdx.x;
+            sg.tm = blockIdx.y;
+            sg.k0 = blockIdx.z * (p.cps / KU);
+            sg.k1 = min(nst, sg.k0 + p.cps / KU);
+            sg.whole = p.splits == 1;
+            sg.owner = false;
+            return sg.k1 > sg.k0;
+        }
+        if (pos >= end) {
+            done = true;
+            return false;
+        }
+        const int t = static_cast<int>(pos / nst);
+        sg.tn = t % tiles_n;
+        sg.tm = t / tiles_n;
+        sg.k0 = static_cast<int>(pos - static_cast<int64_t>(t) * nst);
+        const int64_t room = end - pos;
+        sg.k1 = room < static_cast<int64_t>(nst - sg.k0) ? sg.k0 + static_cast<int>(room) : nst;
+        sg.whole = sg.k0 == 0 && sg.k1 == nst;
+        sg.owner = sg.k0 == 0 && sg.k1 < nst;
+        pos += sg.k1 - sg.k0;
+        return true;
+    }
+};
 
 template <int BITS, bool XPERM>
-__global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_constant__ CUtensorMap tm_codes,
+__global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                                const __grid_constant__ CUtensorMap tm_meta,
                                                                const __grid_constant__ CUtensorMap tm_x,
                                                                const GemmParams p) {
     constexpr int CROW = kBK * BITS / 8;          // code bytes per row and K chunk (32 or 64)
-    constexpr int KU = 128 / CROW;                // K chunks per code stage (4 or 2)
+    constexpr int KU = 128 / CROW;                // K chunks (units) per step = per code stage (4 or 2)
     constexpr int CSTAGE = kRows2 * 128;          // code bytes per stage: 256 rows x 128 B
     constexpr int MSTAGE = kRows2 * kMetaChunks * 4;
     constexpr int WPC = CROW / 16;                // 16-byte code vectors per row and chunk (2 or 4)
@@ -809,13 +887,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
     uint8_t* const gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * kRows2, m0 = blockIdx.y * p.BN, split = blockIdx.z;
-    const int nk_total = p.K / kBK;
-    const int c_begin = split * p.cps;                            // multiple of kMetaChunks
-    const int nk = min(nk_total, c_begin + p.cps) - c_begin;      // chunks = units of this CTA
-    const int nsteps = nk / KU;
+    const int nst = p.K / (kBK * KU);             // steps per tile
     const int XU = p.xu;
-    const int nxu = nk / XU;
     const int NSLOT = p.nslot;
 
     const uint32_t sX = base, sC = base + p.off_c, sM = base + p.off_m;
@@ -828,7 +901,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
     B.x_full = B.codes_empty + 8 * NSC;
     B.a_full = B.x_full + 8 * NSX;
     B.mma_done = B.a_full + 8 * NSLOT;
-    B.acc_full = B.mma_done + 8 * kDoneRing2;
+    B.acc_full = B.mma_done + 8 * kDoneRing2;     // here: the accumulators are free again (one phase per segment)
     B.drain = B.acc_full + 8;
     B.red = B.drain + 8 * 4;
     const uint32_t misc = B.red + 8 * 2;
@@ -845,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
         for (int s = 0; s < NSX; ++s) tc::bar_init(B.x_full + 8 * s, 1);
         for (int s = 0; s < NSLOT; ++s) tc::bar_init(B.a_full + 8 * s, kDequantThreads);
         for (int s = 0; s < kDoneRing2; ++s) tc::bar_init(B.mma_done + 8 * s, kRT);   // both issuers commit each unit
-        tc::bar_init(B.acc_full, kRT);
+        tc::bar_init(B.acc_full, kDequantThreads);
         for (int i = 0; i < 4; ++i) tc::bar_init(B.drain + 8 * i, 1);
         tc::bar_init(B.red, 1);
         tc::bar_init(B.red + 8, 1);
@@ -870,52 +943,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
     // epilogue / dequantisation mapping (warps 4-11): TMEM lane quarter lq, tile tt
     const int lq = warp & 3, tt = (warp - 4) >> 2;
     const int row = tt * kBM + lq * 32 + lane;                    // row of the CTA's 256
-    const int n = n0 + row;
-    const int n0t = n0 + tt * kBM;                                // first row of this thread's tile
-    const float scale_n = n < p.nq ? p.qscale : 1.f;
-    const int n_out = p.yperm ? ((n & ~7) | ((n & 3) << 1) | ((n >> 2) & 1)) : n;
-    const bool kv_on = p.kv.codes[0][0] != nullptr && n0t >= p.kv.h;
-    float bias_n = 0.f;
     uint32_t all_ok = 0;
-    // the fp32 partial of this split fits in the rings (drained by then): staged there for one
-    // bulk store, and the reduction's bulk loads use the same space
+    // the rings hold a whole fp32 partial (staged for one bulk store) once they are drained
     const bool stage_ok = static_cast<uint32_t>(p.BN) * kRows2 * 4 <= p.off_bar;
-    auto finish8 = [&](int col, const float (&v)[8]) {
-        float r[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int m = m0 + col + j;
-            r[j] = (p.residual && m < p.M) ? __half2float(p.residual[static_cast<int64_t>(m) * p.N + n]) : 0.f;
-        }
-        __half o16[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int m = m0 + col + j;
-            float x = (v[j] + bias_n) * scale_n;
-            if (p.relu) x = fmaxf(x, 0.f);
-            o16[j] = __float2half_rn(x + r[j]);
-            if (m < p.M) p.y[static_cast<int64_t>(m) * p.N + n_out] = o16[j];
-        }
-        if (kv_on) kv_store8(p, o16, col, m0, n0t, n, warp, lane, kv_red);
-    };
 
     if (warp == 0) {
-        // ---------------- code + metadata producer: one stage = KU chunks of 256 rows ----------------
+        // ---------------- code + metadata producer: one stage = one step (KU chunks of 256 rows) ----------------
         if (lane == 0) {
             if (!p.early_w) pdl_wait();
-            int st = 0, s = 0;
+            int s = 0, issued = 0;
             uint32_t ph = 0;
-            const bool go = p.gate == nullptr || tc::gate_wait(p.gate, abort, p.status, p.wait_ns);
-            for (; go && st < nsteps; ++st) {
-                if (st >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ph ^ 1, abort, p.status, p.wait_ns)) break;
-                const int c = c_begin + st * KU;
-                tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CSTAGE + MSTAGE);
-                tc::tma_load_2d(sC + s * CSTAGE, &tm_codes, c * CROW, n0, B.codes_full + 8 * s);
-                tc::tma_load_2d(sM + s * MSTAGE, &tm_meta, c & ~(kMetaChunks - 1), n0, B.codes_full + 8 * s);
-                if (++s == NSC) { s = 0; ph ^= 1; }
+            bool go = p.gate == nullptr || tc::gate_wait(p.gate, abort, p.status, p.wait_ns);
+            SegWalk walk(p, nst);
+            Seg sg;
+            while (go && walk.next(p, KU, sg)) {
+                const int n0 = sg.tn * kRows2;
+                for (int st = sg.k0; st < sg.k1; ++st) {
+                    if (issued >= NSC && !tc::bar_wait(B.codes_empty + 8 * s, ph ^ 1, abort, p.status, p.wait_ns)) {
+                        go = false;
+                        break;
+                    }
+                    const int c = st * KU;
+                    tc::bar_arrive_expect_tx(B.codes_full + 8 * s, CSTAGE + MSTAGE);
+                    tc::tma_load_2d(sC + s * CSTAGE, &tm_codes, c * CROW, n0, B.codes_full + 8 * s);
+                    tc::tma_load_2d(sM + s * MSTAGE, &tm_meta, c & ~(kMetaChunks - 1), n0, B.codes_full + 8 * s);
+                    ++issued;
+                    if (++s == NSC) { s = 0; ph ^= 1; }
+                }
             }
-            for (int s2 = 0; s2 < NSC && s2 < st; ++s2) {
-                const int last = s2 + ((st - 1 - s2) / NSC) * NSC;
+            // drain: every copy this thread issued has landed before the CTA can exit
+            for (int s2 = 0; s2 < NSC && s2 < issued; ++s2) {
+                const int last = s2 + ((issued - 1 - s2) / NSC) * NSC;
                 volatile int never = 0;
                 tc::bar_wait(B.codes_full + 8 * s2, (last / NSC) & 1, &never, p.status);
             }
@@ -925,24 +983,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
         // ---------------- activation producer: one stage = XU chunks ----------------
         if (lane == 0) {
             pdl_wait();
-            int u = 0, s = 0;
-            for (; u < nxu; ++u) {
-                if (u >= NSX) {
-                    // the stage last held chunks [(u - NSX) XU, +XU): wait for the MMAs of its last unit
-                    const int ul = (u - NSX) * XU + XU - 1;
-                    if (!tc::bar_wait(B.mma_done + 8 * (ul % kDoneRing2), (ul / kDoneRing2) & 1, abort, p.status,
-                                      p.wait_ns))
-                        break;
+            int s = 0, gx = 0;                    // ring slot; stages issued so far (all segments)
+            bool go = true;
+            SegWalk walk(p, nst);
+            Seg sg;
+            while (go && walk.next(p, KU, sg)) {
+                const int m0 = sg.tm * p.BN;
+                for (int xi = sg.k0 * KU / XU; xi < sg.k1 * KU / XU; ++xi) {
+                    if (gx >= NSX) {
+                        // the slot last held units [(gx - NSX) XU, +XU): wait for the MMAs of its last unit
+                        const int ul = (gx - NSX) * XU + XU - 1;
+                        if (!tc::bar_wait(B.mma_done + 8 * (ul % kDoneRing2), (ul / kDoneRing2) & 1, abort, p.status,
+                                          p.wait_ns)) {
+                            go = false;
+                            break;
+                        }
+                    }
+                    tc::bar_arrive_expect_tx(B.x_full + 8 * s, XU * xbytes);
+                    for (int c = 0; c < XU; ++c)
+                        tc::tma_load_2d(sX + (s * XU + c) * xbytes, &tm_x, (xi * XU + c) * kBK, m0, B.x_full + 8 * s);
+                    ++gx;
+                    if (++s == NSX) s = 0;
                 }
-                tc::bar_arrive_expect_tx(B.x_full + 8 * s, XU * xbytes);
-                for (int c = 0; c < XU; ++c)
-                    tc::tma_load_2d(sX + (s * XU + c) * xbytes, &tm_x, (c_begin + u * XU + c) * kBK, m0,
-                                    B.x_full + 8 * s);
-                if (++s == NSX) s = 0;
             }
-            const int issued = u;
-            for (int s2 = 0; s2 < NSX && s2 < issued; ++s2) {
-                const int last = s2 + ((issued - 1 - s2) / NSX) * NSX;
+            for (int s2 = 0; s2 < NSX && s2 < gx; ++s2) {
+                const int last = s2 + ((gx - 1 - s2) / NSX) * NSX;
                 volatile int never = 0;
                 tc::bar_wait(B.x_full + 8 * s2, (last / NSX) & 1, &never, p.status);
             }
@@ -956,156 +1021,371 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
             const uint32_t d_acc = tmem + static_cast<uint32_t>(t * p.acc_stride);
             int xs = 0, xc = 0;                 // activation stage and chunk within it
             uint32_t xph = 0;
-            int sa = 0;                         // A slot of unit u and its phase bit (no division by NSLOT)
+            int sa = 0;                         // A slot of the next unit and its phase bit
             uint32_t aph = 0;
             bool ok = true;
-            int u = 0;
-            for (; u < nk; ++u) {
-                if (!tc::bar_wait(B.a_full + 8 * sa, aph, abort, p.status, p.wait_ns)) { ok = false; break; }
-                if (xc == 0 && !tc::bar_wait(B.x_full + 8 * xs, xph, abort, p.status, p.wait_ns)) { ok = false; break; }
-                tc::fence_after_sync();
-                const uint32_t a_tm = tmem + static_cast<uint32_t>(p.a_col0 + (sa * kRT + t) * 32);
-                const uint64_t bd = tc::desc_k_sw128(sX + static_cast<uint32_t>(xs * XU + xc) * xbytes);
-                issue_ksteps<1>(d_acc, a_tm, bd, idesc, 0, u == 0);
-                if (++xc == XU) {
-                    xc = 0;
-                    if (++xs == NSX) { xs = 0; xph ^= 1; }
+            int g = 0;                          // units committed so far (all segments)
+            int seg_i = 0;
+            SegWalk walk(p, nst);
+            Seg sg;
+            while (ok && walk.next(p, KU, sg)) {
+                // the previous segment's epilogue has read the accumulators
+                if (seg_i > 0 && !tc::bar_wait(B.acc_full, (seg_i - 1) & 1, abort, p.status, p.wait_ns)) {
+                    ok = false;
+                    break;
                 }
-                tc::mma_commit(u + 1 < nk ? B.mma_done + 8 * (u % kDoneRing2) : B.acc_full);
-                if (++sa == NSLOT) { sa = 0; aph ^= 1; }
+                const int nu = (sg.k1 - sg.k0) * KU;
+                for (int u = 0; u < nu; ++u) {
+                    if (!tc::bar_wait(B.a_full + 8 * sa, aph, abort, p.status, p.wait_ns)) { ok = false; break; }
+                    if (xc == 0 && !tc::bar_wait(B.x_full + 8 * xs, xph, abort, p.status, p.wait_ns)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t a_tm = tmem + static_cast<uint32_t>(p.a_col0 + (sa * kRT + t) * 32);
+                    const uint64_t bd = tc::desc_k_sw128(sX + static_cast<uint32_t>(xs * XU + xc) * xbytes);
+                    issue_ksteps<1>(d_acc, a_tm, bd, idesc, 0, u == 0);
+                    if (++xc == XU) {
+                        xc = 0;
+                        if (++xs == NSX) { xs = 0; xph ^= 1; }
+                    }
+                    tc::mma_commit(B.mma_done + 8 * (g % kDoneRing2));
+                    ++g;
+                    if (++sa == NSLOT) { sa = 0; aph ^= 1; }
+                }
+                ++seg_i;
             }
             volatile int never = 0;
-            const int committed = ok ? nk - 1 : u;
             if (!ok) {
                 tc::mma_commit(B.drain + 8 * t);
                 tc::bar_wait(B.drain + 8 * t, 0, &never, p.status);
             }
-            for (int c = committed - kDoneRing2 > 0 ? committed - kDoneRing2 : 0; c < committed; ++c)
+            // every commit arrival lands before the CTA exits
+            for (int c = g - kDoneRing2 > 0 ? g - kDoneRing2 : 0; c < g; ++c)
                 tc::bar_wait(B.mma_done + 8 * (c % kDoneRing2), (c / kDoneRing2) & 1, &never, p.status);
-            if (ok) tc::bar_wait(B.acc_full, 0, &never, p.status);
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 12) {
-        // ---------------- dequantisation into TMEM, one chunk (unit) at a time ----------------
+        // ---------------- dequantisation into TMEM, one chunk (unit) at a time; epilogues ----------------
         const int sw = row & 7;
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(lq * 32) << 16);
+        const uint32_t taddr = t_lane + static_cast<uint32_t>(tt * p.acc_stride);
+        const int et = (warp - 4) * 32 + lane;
         bool ok = true;
         int s = 0;
         uint32_t cph = 0;
-        int dq_slot = 0;                   // A slot of the next unit (no division by NSLOT)
-        for (int st = 0; st < nsteps && ok; ++st) {
-            if (!tc::bar_wait(B.codes_full + 8 * s, cph, abort, p.status, p.wait_ns)) { ok = false; break; }
-            const uint32_t crow = sC + s * CSTAGE + row * 128;
-            uint4 cw[KU][WPC];
+        int dq_slot = 0;                   // A slot of the next unit
+        int g = 0;                         // units dequantised so far (all segments)
+        int seg_i = 0;
+        bool pdl_done = false;
+        SegWalk walk(p, nst);
+        Seg sg;
+        while (walk.next(p, KU, sg)) {
+            for (int st = sg.k0; st < sg.k1 && ok; ++st) {
+                if (!tc::bar_wait(B.codes_full + 8 * s, cph, abort, p.status, p.wait_ns)) { ok = false; break; }
+                const uint32_t crow = sC + s * CSTAGE + row * 128;
+                uint4 cw[KU][WPC];
 #pragma unroll
-            for (int c = 0; c < KU; ++c)
+                for (int c = 0; c < KU; ++c)
 #pragma unroll
-                for (int v = 0; v < WPC; ++v) cw[c][v] = tc::lds128(crow + (((c * WPC + v) ^ sw) << 4));
-            const uint4 mrow = tc::lds128(sM + s * MSTAGE + row * 16);
-            const int moff = (c_begin + st * KU) & (kMetaChunks - 1);
+                    for (int v = 0; v < WPC; ++v) cw[c][v] = tc::lds128(crow + (((c * WPC + v) ^ sw) << 4));
+                const uint4 mrow = tc::lds128(sM + s * MSTAGE + row * 16);
+                const int moff = (st * KU) & (kMetaChunks - 1);
 #pragma unroll
-            for (int c = 0; c < KU; ++c) {
-                const int u = st * KU + c;
-                const int sa = dq_slot;
-                if (++dq_slot == NSLOT) dq_slot = 0;
-                if (u >= NSLOT) {
-                    const int pu = u - NSLOT;
-                    if (!tc::bar_wait(B.mma_done + 8 * (pu % kDoneRing2), (pu / kDoneRing2) & 1, abort, p.status,
-                                      p.wait_ns)) {
-                        ok = false;
+                for (int c = 0; c < KU; ++c) {
+                    const int u = g;
+                    const int sa = dq_slot;
+                    if (++dq_slot == NSLOT) dq_slot = 0;
+                    if (u >= NSLOT) {
+                        const int pu = u - NSLOT;
+                        if (!tc::bar_wait(B.mma_done + 8 * (pu % kDoneRing2), (pu / kDoneRing2) & 1, abort, p.status,
+                                          p.wait_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+                    }
+                    const int mi = (moff + c) & 3;
+                    const uint32_t mw = mi == 0 ? mrow.x : (mi == 1 ? mrow.y : (mi == 2 ? mrow.z : mrow.w));
+                    const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
+                    const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
+                    const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
+                    const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
+                    const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
+                    const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
+                    const uint32_t a_col = p.a_col0 + (sa * kRT + tt) * 32;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {          // two halves of the chunk: 32 values each
+                        uint32_t r[16];
+                        if (BITS == 4) {
+                            const uint4 q = cw[c][hh];
+                            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2)
+                                                      : dequant8_4bit(w[j], step2, mnv2);
+                                r[4 * j] = v.x;
+                                r[4 * j + 1] = v.y;
+                                r[4 * j + 2] = v.z;
+                                r[4 * j + 3] = v.w;
+                            }
+                        } else {
+                            const uint4 q0 = cw[c][2 * hh], q1 = cw[c][2 * hh + 1];
+                            const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                uint4 v;
+                                if (XPERM) {
+                                    v = dequant8_8bit_il(w[2 * j], w[2 * j + 1], step2, mnv2);
+                                } else {
+                                    const uint2 a = dequant4_8bit(w[2 * j], step2, mnv2);
+                                    const uint2 b = dequant4_8bit(w[2 * j + 1], step2, mnv2);
+                                    v = make_uint4(a.x, a.y, b.x, b.y);
+                                }
+                                r[4 * j] = v.x;
+                                r[4 * j + 1] = v.y;
+                                r[4 * j + 2] = v.z;
+                                r[4 * j + 3] = v.w;
+                            }
+                        }
+                        tc::tmem_st16(t_lane + a_col + hh * 16, r);
+                    }
+                    tc::tmem_wait_st();
+                    tc::fence_before_sync();
+                    tc::bar_arrive(B.a_full + 8 * sa);
+                    ++g;
+                }
+                if (!ok) break;
+                // every value of the code stage has been used: the next TMA may refill it
+                tc::bar_arrive(B.codes_empty + 8 * s);
+                if (++s == NSC) { s = 0; cph ^= 1; }
+            }
+
+            // ---------------- epilogue of this segment ----------------
+            const int n0 = sg.tn * kRows2, m0 = sg.tm * p.BN;
+            const int n = n0 + row;
+            const int n0t = n0 + tt * kBM;                            // first row of this thread's tile
+            const float scale_n = n < p.nq ? p.qscale : 1.f;
+            const int n_out = p.yperm ? ((n & ~7) | ((n & 3) << 1) | ((n >> 2) & 1)) : n;
+            const bool kv_on = p.kv.codes[0][0] != nullptr && n0t >= p.kv.h;
+            if (!pdl_done) {
+                pdl_wait();
+                pdl_trigger();
+                pdl_done = true;
+            }
+            const float bias_n = p.bias ? __half2float(p.bias[n]) : 0.f;
+            auto finish8 = [&](int col, const float (&v)[8]) {
+                float r[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int m = m0 + col + j;
+                    r[j] = (p.residual && m < p.M) ? __half2float(p.residual[static_cast<int64_t>(m) * p.N + n]) : 0.f;
+                }
+                __half o16[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int m = m0 + col + j;
+                    float x = (v[j] + bias_n) * scale_n;
+                    if (p.relu) x = fmaxf(x, 0.f);
+                    o16[j] = __float2half_rn(x + r[j]);
+                    if (m < p.M) p.y[static_cast<int64_t>(m) * p.N + n_out] = o16[j];
+                }
+                if (kv_on) kv_store8(p, o16, col, m0, n0t, n, warp, lane, kv_red);
+            };
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (ok && !*abort && g > 0) {
+                const int gl = g - 1;                                 // the segment's last unit: both tiles' MMAs done
+                ok = tc::bar_wait(B.mma_done + 8 * (gl % kDoneRing2), (gl / kDoneRing2) & 1, abort, p.status);
+            }
+            asm volatile(
+                "{\n\t.reg .pred p, q;\n\t"
+                "setp.ne.u32 p, %1, 0;\n\t"
+                "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
+                "selp.u32 %0, 1, 0, q;\n\t}"
+                : "=r"(all_ok)
+                : "r"((ok && !*abort) ? 1u : 0u)
+                : "memory");
+            if (all_ok) tc::fence_after_sync();
+            const int64_t pstride = static_cast<int64_t>(p.BN) * kRows2;     // floats per partial
+
+            // Sum, for every 8-column group of `row`, of `own` (this CTA's accumulator, when
+            // set) and the partial blocks src[0..np) in that order, handed to finish8. The
+            // blocks pass through the drained rings in batches of C column groups, bulk-
+            // loaded into two alternating halves. Returns false if a wait gave up.
+            auto reduce_blocks = [&](const float* const* src, int np, bool own) -> bool {
+                const int ng = p.BN / 8;
+                const uint32_t half = (p.off_bar / 2) & ~15u;
+                int C = static_cast<int>(half / (static_cast<uint32_t>(np) * kRows2 * 32));
+                if (C > ng) C = ng;
+                const int nb = (ng + C - 1) / C;
+                auto issue = [&](int bi) {
+                    const int g0 = bi * C, gc = min(C, ng - g0);
+                    const uint32_t dst = base + (bi & 1) * half;
+                    const uint32_t bytes = static_cast<uint32_t>(gc) * kRows2 * 32;
+                    tc::bar_arrive_expect_tx(B.red + 8 * (bi & 1), bytes * np);
+                    for (int sp = 0; sp < np; ++sp)
+                        tc::bulk_load(dst + sp * static_cast<uint32_t>(C) * kRows2 * 32,
+                                      src[sp] + static_cast<int64_t>(g0) * kRows2 * 8, bytes, B.red + 8 * (bi & 1));
+                };
+                if (et == 0) {
+                    tc::fence_proxy_async_global();
+                    issue(0);
+                    if (nb > 1) issue(1);
+                }
+                int waited = 0;
+                bool rok = true;
+                for (int bi = 0; bi < nb; ++bi) {
+                    const bool w = tc::bar_wait(B.red + 8 * (bi & 1), (bi >> 1) & 1, abort, p.status, p.wait_ns);
+                    uint32_t wall;                                    // one decision for the 256 threads
+                    asm volatile(
+                        "{\n\t.reg .pred p, q;\n\t"
+                        "setp.ne.u32 p, %1, 0;\n\t"
+                        "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
+                        "selp.u32 %0, 1, 0, q;\n\t}"
+                        : "=r"(wall)
+                        : "r"(w ? 1u : 0u)
+                        : "memory");
+                    if (!wall) {
+                        rok = false;
                         break;
                     }
-                    tc::fence_after_sync();
-                }
-                const int mi = (moff + c) & 3;
-                const uint32_t mw = mi == 0 ? mrow.x : (mi == 1 ? mrow.y : (mi == 2 ? mrow.z : mrow.w));
-                const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
-                const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
-                const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
-                const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
-                const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
-                const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
-                const uint32_t a_col = p.a_col0 + (sa * kRT + tt) * 32;
+                    waited = bi + 1;
+                    const uint32_t sbuf = base + (bi & 1) * half;
+                    const int g0 = bi * C, gc = min(C, ng - g0);
+                    for (int gi = 0; gi < gc; ++gi) {
+                        float acc[8];
+                        if (own) {
+                            tc::tmem_ld8(taddr + (g0 + gi) * 8, acc);
+                        } else {
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {          // two halves of the chunk: 32 values each
-                    uint32_t r[16];
-                    if (BITS == 4) {
-                        const uint4 q = cw[c][hh];
-                        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2) : dequant8_4bit(w[j], step2, mnv2);
-                            r[4 * j] = v.x;
-                            r[4 * j + 1] = v.y;
-                            r[4 * j + 2] = v.z;
-                            r[4 * j + 3] = v.w;
+                            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
                         }
-                    } else {
-                        const uint4 q0 = cw[c][2 * hh], q1 = cw[c][2 * hh + 1];
-                        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint4 v;
-                            if (XPERM) {
-                                v = dequant8_8bit_il(w[2 * j], w[2 * j + 1], step2, mnv2);
-                            } else {
-                                const uint2 a = dequant4_8bit(w[2 * j], step2, mnv2);
-                                const uint2 b = dequant4_8bit(w[2 * j + 1], step2, mnv2);
-                                v = make_uint4(a.x, a.y, b.x, b.y);
+                        for (int sp = 0; sp < np; ++sp) {                 // block order
+                            const uint32_t q = sbuf + ((sp * C + gi) * kRows2 + row) * 32;
+                            const float4 lo = tc::lds128f(q), hi = tc::lds128f(q + 16);
+                            acc[0] += lo.x;
+                            acc[1] += lo.y;
+                            acc[2] += lo.z;
+                            acc[3] += lo.w;
+                            acc[4] += hi.x;
+                            acc[5] += hi.y;
+                            acc[6] += hi.z;
+                            acc[7] += hi.w;
+                        }
+                        finish8((g0 + gi) * 8, acc);
+                    }
+                    asm volatile("bar.sync 1, 256;" ::: "memory");       // this half is free again
+                    if (et == 0 && bi + 2 < nb) issue(bi + 2);
+                }
+                // a wait that gave up: the copies already issued land before the CTA exits
+                const int issued = rok ? nb : min(nb, waited + 2);
+                for (int bi = waited; bi < issued; ++bi) {
+                    volatile int never = 0;
+                    tc::bar_wait(B.red + 8 * (bi & 1), (bi >> 1) & 1, &never, p.status);
+                }
+                return rok;
+            };
+
+            if (p.sk) {
+                if (all_ok && sg.whole) {
+                    for (int col = 0; col < p.BN; col += 8) {
+                        float v[8];
+                        tc::tmem_ld8(taddr + col, v);
+                        finish8(col, v);
+                    }
+                } else if (all_ok && !sg.owner) {
+                    // a later piece of a shared tile (this CTA's first segment): partial to this
+                    // CTA's slot, then published (the rings still feed the next segment, so the
+                    // partial goes straight from the accumulator to the workspace)
+                    float* mine = p.part + static_cast<int64_t>(blockIdx.x) * pstride;
+                    for (int col = 0; col < p.BN; col += 8) {
+                        float v[8];
+                        tc::tmem_ld8(taddr + col, v);
+                        part_store8(mine, kRows2, row, col, v);
+                    }
+                    __threadfence();
+                    asm volatile("bar.sync 1, 256;" ::: "memory");
+                    if (et == 0) atomicExch(p.counters + blockIdx.x, 1);
+                } else if (all_ok) {
+                    // the owner: its accumulator plus the later pieces, CTAs blockIdx.x + 1, ...
+                    // up to the tile's last step, in K order
+                    const int64_t tile_end = (static_cast<int64_t>(sg.tm) * p.sk_tiles_n + sg.tn + 1) * nst;
+                    const float* srcs[kMaxPieces];
+                    int np = 0;
+                    for (int c2 = blockIdx.x + 1; c2 < static_cast<int>(gridDim.x) && np < kMaxPieces; ++c2) {
+                        if (static_cast<int64_t>(c2) * p.sk_total / gridDim.x >= tile_end) break;
+                        srcs[np++] = p.part + static_cast<int64_t>(c2) * pstride;
+                    }
+                    // wait until every piece is published (its CTA started earlier in K order
+                    // and runs on another SM; the wait is bounded all the same)
+                    bool pub = true;
+                    if (et == 0) {
+                        const uint64_t t0 = tc::globaltimer_ns();
+                        for (int i = 0; i < np && pub; ++i) {
+                            volatile int* f = p.counters + blockIdx.x + 1 + i;
+                            while (*f == 0) {
+                                if (*abort || tc::globaltimer_ns() - t0 > p.wait_ns) {
+                                    *abort = 1;
+                                    set_status(p.status, FLEX_ERR_TIMEOUT);
+                                    pub = false;
+                                    break;
+                                }
+                                __nanosleep(256);
                             }
-                            r[4 * j] = v.x;
-                            r[4 * j + 1] = v.y;
-                            r[4 * j + 2] = v.z;
-                            r[4 * j + 3] = v.w;
+                        }
+                        __threadfence();
+                    }
+                    uint32_t pall;
+                    asm volatile(
+                        "{\n\t.reg .pred p, q;\n\t"
+                        "setp.ne.u32 p, %1, 0;\n\t"
+                        "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
+                        "selp.u32 %0, 1, 0, q;\n\t}"
+                        : "=r"(pall)
+                        : "r"(pub ? 1u : 0u)
+                        : "memory");
+                    if (pall && stage_ok && (p.off_bar / 2) >= static_cast<uint32_t>(np) * kRows2 * 32) {
+                        __threadfence();
+                        reduce_blocks(srcs, np, true);
+                    } else if (pall) {
+                        __threadfence();
+                        for (int col = 0; col < p.BN; col += 8) {
+                            float acc[8];
+                            tc::tmem_ld8(taddr + col, acc);
+                            for (int i = 0; i < np; ++i) {
+                                const float4* q = reinterpret_cast<const float4*>(
+                                    srcs[i] + (static_cast<int64_t>(col >> 3) * kRows2 + row) * 8);
+                                const float4 lo = __ldcg(q), hi = __ldcg(q + 1);
+                                acc[0] += lo.x;
+                                acc[1] += lo.y;
+                                acc[2] += lo.z;
+                                acc[3] += lo.w;
+                                acc[4] += hi.x;
+                                acc[5] += hi.y;
+                                acc[6] += hi.z;
+                                acc[7] += hi.w;
+                            }
+                            finish8(col, acc);
                         }
                     }
-                    tc::tmem_st16(t_lane + a_col + hh * 16, r);
+                    asm volatile("bar.sync 1, 256;" ::: "memory");
+                    if (et == 0)
+                        for (int i = 0; i < np; ++i) p.counters[blockIdx.x + 1 + i] = 0;   // ready for the next call
                 }
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
-                tc::bar_arrive(B.a_full + 8 * sa);
-            }
-            if (!ok) break;
-            // every value of the code stage has been used: the next TMA may refill it
-            tc::bar_arrive(B.codes_empty + 8 * s);
-            if (++s == NSC) { s = 0; cph ^= 1; }
-        }
-        // ---------------- epilogue ----------------
-        pdl_wait();
-        pdl_trigger();
-        bias_n = p.bias ? __half2float(p.bias[n]) : 0.f;
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (ok && !*abort) ok = tc::bar_wait(B.acc_full, 0, abort, p.status);
-        asm volatile(
-            "{\n\t.reg .pred p, q;\n\t"
-            "setp.ne.u32 p, %1, 0;\n\t"
-            "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
-            "selp.u32 %0, 1, 0, q;\n\t}"
-            : "=r"(all_ok)
-            : "r"((ok && !*abort) ? 1u : 0u)
-            : "memory");
-        const uint32_t taddr = t_lane + static_cast<uint32_t>(tt * p.acc_stride);
-        if (all_ok) {
-            tc::fence_after_sync();
-            if (p.splits == 1) {
-                for (int col = 0; col < p.BN; col += 8) {
-                    float v[8];
-                    tc::tmem_ld8(taddr + col, v);
-                    finish8(col, v);
-                }
-            } else if (p.cluster) {
-                // this split's fp32 partial [BN][256] into this CTA's shared memory (the rings
-                // are drained: every copy has landed and every MMA has completed)
-                for (int col = 0; col < p.BN; col += 8) {
-                    float v[8];
-                    tc::tmem_ld8(taddr + col, v);
+            } else if (all_ok) {
+                if (p.splits == 1) {
+                    for (int col = 0; col < p.BN; col += 8) {
+                        float v[8];
+                        tc::tmem_ld8(taddr + col, v);
+                        finish8(col, v);
+                    }
+                } else if (p.cluster) {
+                    // this split's fp32 partial [BN][256] into this CTA's shared memory (the rings
+                    // are drained: every copy has landed and every MMA has completed)
+                    for (int col = 0; col < p.BN; col += 8) {
+                        float v[8];
+                        tc::tmem_ld8(taddr + col, v);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) tc::st_shared_f32(base + ((col + j) * kRows2 + row) * 4, v[j]);
-                }
-            } else {
-                float* mine = p.part + (static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * p.splits + split) *
-                                           p.BN * kRows2;
-                if (stage_ok) {
+                        for (int j = 0; j < 8; ++j) tc::st_shared_f32(base + ((col + j) * kRows2 + row) * 4, v[j]);
+                    }
+                } else if (stage_ok) {
                     // the partial, in its workspace layout, into the drained rings; one bulk
                     // store (issued with the ticket below) moves it to the workspace
                     for (int col = 0; col < p.BN; col += 8) {
@@ -1117,6 +1397,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
                     }
                     tc::fence_proxy_async_smem();
                 } else {
+                    float* mine = p.part + (static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * p.splits +
+                                            blockIdx.z) * pstride;
                     for (int col = 0; col < p.BN; col += 8) {
                         float v[8];
                         tc::tmem_ld8(taddr + col, v);
@@ -1124,111 +1406,47 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
                     }
                 }
             }
-        }
-        if (p.splits > 1 && !p.cluster) {
-            // ticket, taken by every split (see gemm_tc_kernel); the last adds the partials in split order
-            const int et = (warp - 4) * 32 + lane;
-            const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-            const int64_t pstride = static_cast<int64_t>(p.BN) * kRows2;     // floats per partial
-            __threadfence();
-            asm volatile("bar.sync 1, 256;" ::: "memory");
-            if (et == 0) {
-                if (all_ok && stage_ok) {
-                    tc::bulk_store(p.part + (static_cast<int64_t>(tile) * p.splits + split) * pstride, base,
-                                   static_cast<uint32_t>(pstride * 4));
-                    tc::bulk_commit();
-                    tc::bulk_wait_all();
-                    tc::fence_proxy_async_global();
-                    __threadfence();
-                }
-                *last_flag = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
-            }
-            asm volatile("bar.sync 1, 256;" ::: "memory");
-            if (*last_flag) {
+            if (!p.sk && p.splits > 1 && !p.cluster) {
+                // ticket, taken by every split (see gemm_tc_kernel); the last adds the partials in split order
+                const int tile = blockIdx.y * gridDim.x + blockIdx.x;
                 __threadfence();
-                const float* all = p.part + static_cast<int64_t>(tile) * p.splits * pstride;
-                if (all_ok && stage_ok && (p.off_bar / 2) >= static_cast<uint32_t>(p.splits) * kRows2 * 32) {
-                    // the partials in batches of C column groups (8 KB each per split), bulk-
-                    // loaded into two alternating halves of the drained rings; each thread adds
-                    // its row's 8 values of every split in split order
-                    const int ng = p.BN / 8;
-                    const uint32_t half = (p.off_bar / 2) & ~15u;
-                    int C = static_cast<int>(half / (static_cast<uint32_t>(p.splits) * kRows2 * 32));
-                    if (C > ng) C = ng;
-                    const int nb = (ng + C - 1) / C;
-                    auto issue = [&](int bi) {
-                        const int g0 = bi * C, gc = min(C, ng - g0);
-                        const uint32_t dst = base + (bi & 1) * half;
-                        const uint32_t bytes = static_cast<uint32_t>(gc) * kRows2 * 32;
-                        tc::bar_arrive_expect_tx(B.red + 8 * (bi & 1), bytes * p.splits);
-                        for (int sp = 0; sp < p.splits; ++sp)
-                            tc::bulk_load(dst + sp * static_cast<uint32_t>(C) * kRows2 * 32,
-                                          all + sp * pstride + static_cast<int64_t>(g0) * kRows2 * 8, bytes,
-                                          B.red + 8 * (bi & 1));
-                    };
-                    if (et == 0) {
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                if (et == 0) {
+                    if (all_ok && stage_ok) {
+                        tc::bulk_store(p.part + (static_cast<int64_t>(tile) * p.splits + blockIdx.z) * pstride, base,
+                                       static_cast<uint32_t>(pstride * 4));
+                        tc::bulk_commit();
+                        tc::bulk_wait_all();
                         tc::fence_proxy_async_global();
-                        issue(0);
-                        if (nb > 1) issue(1);
+                        __threadfence();
                     }
-                    int waited = 0;
-                    bool rok = true;
-                    for (int bi = 0; bi < nb; ++bi) {
-                        const bool w = tc::bar_wait(B.red + 8 * (bi & 1), (bi >> 1) & 1, abort, p.status, p.wait_ns);
-                        // one decision for all 256 threads (the loop has named barriers)
-                        uint32_t wall;
-                        asm volatile(
-                            "{\n\t.reg .pred p, q;\n\t"
-                            "setp.ne.u32 p, %1, 0;\n\t"
-                            "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
-                            "selp.u32 %0, 1, 0, q;\n\t}"
-                            : "=r"(wall)
-                            : "r"(w ? 1u : 0u)
-                            : "memory");
-                        if (!wall) {
-                            rok = false;
-                            break;
-                        }
-                        waited = bi + 1;
-                        const uint32_t src = base + (bi & 1) * half;
-                        const int g0 = bi * C, gc = min(C, ng - g0);
-                        for (int gi = 0; gi < gc; ++gi) {
-                            float acc[8];
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-                            for (int sp = 0; sp < p.splits; ++sp) {          // split order
-                                const uint32_t q = src + ((sp * C + gi) * kRows2 + row) * 32;
-                                const float4 lo = tc::lds128f(q), hi = tc::lds128f(q + 16);
-                                acc[0] += lo.x;
-                                acc[1] += lo.y;
-                                acc[2] += lo.z;
-                                acc[3] += lo.w;
-                                acc[4] += hi.x;
-                                acc[5] += hi.y;
-                                acc[6] += hi.z;
-                                acc[7] += hi.w;
-                            }
-                            finish8((g0 + gi) * 8, acc);
-                        }
-                        asm volatile("bar.sync 1, 256;" ::: "memory");       // this half is free again
-                        if (et == 0 && bi + 2 < nb) issue(bi + 2);
-                    }
-                    // a wait that gave up: let the copies already issued land before the CTA exits
-                    const int issued = rok ? nb : min(nb, waited + 2);
-                    for (int bi = waited; bi < issued; ++bi) {
-                        volatile int never = 0;
-                        tc::bar_wait(B.red + 8 * (bi & 1), (bi >> 1) & 1, &never, p.status);
-                    }
-                } else if (all_ok) {
-                    part_reduce(all, pstride, p.splits, kRows2, row, 0, p.BN,
-                                [&](int col, const float (&acc)[8]) { finish8(col, acc); });
+                    *last_flag = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
                 }
-                if (et == 0) p.counters[tile] = 0;
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                if (*last_flag) {
+                    __threadfence();
+                    const float* all = p.part + static_cast<int64_t>(tile) * p.splits * pstride;
+                    if (all_ok && stage_ok && (p.off_bar / 2) >= static_cast<uint32_t>(p.splits) * kRows2 * 32) {
+                        const float* srcs[kMaxSplits];
+                        for (int sp = 0; sp < p.splits; ++sp) srcs[sp] = all + sp * pstride;
+                        reduce_blocks(srcs, p.splits, false);
+                    } else if (all_ok) {
+                        part_reduce(all, pstride, p.splits, kRows2, row, 0, p.BN,
+                                    [&](int col, const float (&acc)[8]) { finish8(col, acc); });
+                    }
+                    if (et == 0) p.counters[tile] = 0;
+                }
             }
+            // the accumulators are free for the next segment's MMAs
+            tc::fence_before_sync();
+            tc::bar_arrive(B.acc_full);
+            ++seg_i;
+            if (!all_ok) break;
         }
+        (void)seg_i;
     }
 
-    if (p.splits > 1 && p.cluster) {
+    if (!p.sk && p.splits > 1 && p.cluster) {
         // split-K across the cluster: CTA r finishes the 8-column groups v = r, r + S, ...
         // of every row, adding the splits' partials in split order; the second barrier keeps
         // each CTA's shared memory alive until its peers are done. All threads of every CTA
@@ -1237,6 +1455,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
         if (warp >= 4 && warp < 12 && all_ok) {
             const int S = p.splits;
             const int rank = static_cast<int>(tc::cluster_rank());
+            const int n = blockIdx.x * kRows2 + row;
+            const int n0t = blockIdx.x * kRows2 + tt * kBM;
+            const int m0 = blockIdx.y * p.BN;
+            const float scale_n = n < p.nq ? p.qscale : 1.f;
+            const int n_out = p.yperm ? ((n & ~7) | ((n & 3) << 1) | ((n >> 2) & 1)) : n;
+            const bool kv_on = p.kv.codes[0][0] != nullptr && n0t >= p.kv.h;
+            const float bias_n = p.bias ? __half2float(p.bias[n]) : 0.f;
             for (int v = rank; v < p.BN / 8; v += S) {
                 const int col = v * 8;
                 float acc[8];
@@ -1250,7 +1475,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
 #pragma unroll
                     for (int j = 0; j < 8; ++j) acc[j] += tv[j];
                 }
-                finish8(col, acc);
+                float r[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int m = m0 + col + j;
+                    r[j] = (p.residual && m < p.M) ? __half2float(p.residual[static_cast<int64_t>(m) * p.N + n]) : 0.f;
+                }
+                __half o16[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int m = m0 + col + j;
+                    float x = (acc[j] + bias_n) * scale_n;
+                    if (p.relu) x = fmaxf(x, 0.f);
+                    o16[j] = __float2half_rn(x + r[j]);
+                    if (m < p.M) p.y[static_cast<int64_t>(m) * p.N + n_out] = o16[j];
+                }
+                if (kv_on) kv_store8(p, o16, col, m0, n0t, n, warp, lane, kv_red);
             }
         }
         tc::cluster_sync();
@@ -1714,7 +1954,7 @@ int max_active_clusters(int splits, uint32_t smem, bool rows256 = false) {
     set_smem_once(gemm_tc2_kernel<4, true>, 227 * 1024);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1, 1, splits);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(rows256 ? kThreads2 : kThreads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1758,9 +1998,14 @@ int choose_splits(int tiles, int nk, int bits) {
 
 struct Plan2 {
     int BN, tiles_n, tiles_m, splits, cps, nsx, nsc, xu, nslot, acc_stride, a_col0, cluster;
+    int sk, grid;                          // stream-K schedule over `grid` CTAs
+    int64_t sk_total;
     uint32_t off_c, off_m, off_bar, smem;
     int64_t ws_bytes, counters_bytes;
 };
+
+// Stream-K for the 256-row kernel (flex_set_gemm_streamk): on unless switched off.
+std::atomic<int> g_streamk{1};
 
 // gemm_tc2_kernel serves weights with N a multiple of 256 (two 128-row tiles per CTA)
 // for more than 128 activation rows; its activation tile is at most 192 rows (M <= 192
@@ -1823,6 +2068,28 @@ Plan2 make_plan2(int M, int N, int K, int bits) {
     P.ws_bytes = (P.splits > 1 && !P.cluster)
                      ? P.counters_bytes + static_cast<int64_t>(tiles) * P.splits * P.BN * kRows2 * 4
                      : 0;
+    // Where the split plan would reduce through the workspace in more than one wave of
+    // CTAs, a stream-K schedule instead: one CTA per SM, each taking an equal share of all
+    // tiles' K steps; a tile is cut only where one CTA's share ends, so at most one partial
+    // per CTA crosses the workspace, and the CTAs' fills and epilogues are paid once per CTA,
+    // not once per (tile, split). Taken when every CTA gets at least 8 steps and no tile is
+    // spread over more than kMaxPieces + 1 CTAs. (With the splits in one wave the ticket
+    // plan measured faster: at OPT-175B shapes, 48 tiles x 3 splits, 62 against 72 us.)
+    P.sk = 0;
+    P.grid = tiles * P.splits;
+    P.sk_total = 0;
+    if (g_streamk.load(std::memory_order_relaxed) && P.splits > 1 && !P.cluster && tiles * P.splits > sm_count()) {
+        const int sms = sm_count();
+        const int nst = nk / ku;
+        const int64_t total = static_cast<int64_t>(tiles) * nst;
+        const int64_t qmin = total / sms;
+        if (qmin >= 8 && (nst + qmin - 1) / qmin <= kMaxPieces) {
+            P.sk = 1;
+            P.grid = sms;
+            P.sk_total = total;
+            P.ws_bytes = P.counters_bytes + static_cast<int64_t>(sms) * P.BN * kRows2 * 4;
+        }
+    }
     return P;
 }
 
@@ -2079,10 +2346,13 @@ int gemm2_launch(const void* x, const flexq_tensor* W, const void* bias, const v
     gp.off_m = P.off_m;
     gp.off_bar = P.off_bar;
     gp.tmem_cols = kTmemCols;
+    gp.sk = P.sk;
+    gp.sk_tiles_n = P.tiles_n;
+    gp.sk_total = P.sk_total;
     fill_kv_target(gp.kv, kv);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(P.tiles_n, P.tiles_m, P.splits);
-    cfg.blockDim = dim3(kThreads);
+    cfg.gridDim = P.sk ? dim3(P.grid, 1, 1) : dim3(P.tiles_n, P.tiles_m, P.splits);
+    cfg.blockDim = dim3(kThreads2);
     cfg.dynamicSmemBytes = P.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -2221,6 +2491,8 @@ extern "C" int64_t flex_gemm_ws_bytes(int32_t M, int32_t N, int32_t K) {
     return a > b ? a : b;
 }
 
+extern "C" int32_t flex_set_gemm_streamk(int32_t enable) { return g_streamk.exchange(enable ? 1 : 0); }
+
 extern "C" int flex_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t bits, int32_t* out) {
     FLEX_REQUIRE(out != nullptr && M > 0 && N > 0 && K > 0, FLEX_ERR_INVALID_ARG);
     FLEX_REQUIRE(bits == 4 || bits == 8, FLEX_ERR_UNSUPPORTED);
@@ -2235,8 +2507,8 @@ extern "C" int flex_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t bits, int
         const Plan2 P = make_plan2(M, N, K, bits);
         out[0] = 2;
         out[1] = P.tiles_n * P.tiles_m;
-        out[2] = P.splits;
-        out[3] = P.cluster;
+        out[2] = P.sk ? P.grid : P.splits;
+        out[3] = P.sk ? 2 : P.cluster;
     } else {
         const Plan P = make_plan(M, N, K, bits);
         out[0] = 1;

@@ -296,11 +296,17 @@ int flex_prefill_attention(const void* q, const void* k, const void* v, int64_t 
 int64_t flex_gemm_ws_bytes(int32_t M, int32_t N, int32_t K);
 /* The launch plan flex_dequant_gemm takes for this problem on the current device:
  * out[0] the kernel (0 the small-batch GEMV on mma.sync, 1 the 128-row tcgen05 GEMM,
- * 2 the 256-row tcgen05 GEMM), out[1] its output tiles, out[2] the K splits per tile,
- * out[3] 1 if the splits reduce inside a thread-block cluster, 0 through the workspace
- * (or no split). Needs a current CUDA device (the plan depends on its SM count and
- * cluster occupancy). */
+ * 2 the 256-row tcgen05 GEMM), out[1] its output tiles, out[2] the K splits per tile
+ * (stream-K: the CTAs that share the tiles' K steps), out[3] how split results are
+ * added: 0 through workspace partials and a ticket (or no split), 1 inside a
+ * thread-block cluster, 2 stream-K (a tile's first CTA adds the later pieces). Needs a
+ * current CUDA device (the plan depends on its SM count and cluster occupancy). */
 int flex_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t bits, int32_t* out);
+
+/* Stream-K schedule of the 256-row GEMM (on by default): enable = 0 makes later plans
+ * use K splits with workspace tickets instead, e.g. for comparison. Process-wide;
+ * returns the previous setting. */
+int32_t flex_set_gemm_streamk(int32_t enable);
 int flex_dequant_gemm(const void* x, const flexq_tensor* W, const void* bias,
                       const void* residual, void* y, int32_t M, int32_t epilogue,
                       void* ws, int64_t ws_bytes, void* stream);

@@ -218,44 +218,63 @@ def test_gemm_interleaved_activations(M, N, K):
 
 
 def _plan_cases():
-    """(M, N, K) candidates whose plans cover the split-K reduction paths: for each of
-    the two tensor-core kernels, no split, splits through a thread-block cluster, and
-    splits through the workspace ticket with at most 4 and with more than 4 splits."""
+    """(M, N, K) candidates whose plans cover the split-K reduction paths of the two
+    tensor-core kernels: no split, splits through a thread-block cluster, through the
+    workspace ticket with at most 4 and with more than 4 splits, and stream-K."""
     cands = []
     for M in (48, 144):
-        for tiles in (1, 2, 6, 12, 20, 24, 28, 40, 96):
+        for tiles in (1, 2, 6, 12, 20, 24, 28, 40, 96, 192):
             for K in (2048, 12288, 49152):
                 N = tiles * (256 if M > 128 else 128)
                 cands.append((M, N, K))
     return cands
 
 
-def test_gemm_split_reduction_paths():
+def _path(pl):
+    if pl["reduce"] in ("none", "cluster", "streamk"):
+        return (pl["kernel"], pl["reduce"])
+    return (pl["kernel"], "ticket<=4" if pl["splits"] <= 4 else "ticket>4")
+
+
+@pytest.mark.parametrize("streamk", [True, False])
+def test_gemm_split_reduction_paths(streamk):
     """Every split-K reduction path the device's plans reach is parity-checked against
     the oracle on sampled output features and gives identical bits on a second call;
-    the workspace tickets are back at zero. The ticket path with at most 4 splits and
-    the one with more (the partials are added 4 splits at a time) are required."""
-    seen = {}
-    for M, N, K in _plan_cases():
-        pl = fq.flex_gemm_plan(M, N, K)
-        path = (pl["kernel"], "none" if pl["splits"] == 1 else ("cluster" if pl["cluster"] else
-                                                              ("ticket<=4" if pl["splits"] <= 4 else "ticket>4")))
-        if path not in seen or N * K < seen[path][1] * seen[path][2]:
-            seen[path] = (M, N, K)
-    for k in ("tc128", "tc256"):
-        assert (k, "ticket<=4") in seen and (k, "ticket>4") in seen, sorted(seen)
-    for path, (M, N, K) in sorted(seen.items()):
-        x = synth.activations((M, K), 90, device="cuda")
-        w = synth.normal_f16((N, K), 91, 0.02, device="cuda")
-        W = fq.CompressedWeight(w, 4, 64)
-        ws = torch.zeros(max(16, fq.flex_gemm_ws_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
-        y1 = torch.empty((M, N), dtype=torch.float16, device="cuda")
-        y2 = torch.empty_like(y1)
-        fq.flex_dequant_gemm(x, W, None, None, y1, M, fq.FLEX_EPI_NONE, ws)
-        fq.flex_dequant_gemm(x, W, None, None, y2, M, fq.FLEX_EPI_NONE, ws)
-        sync_status()
-        assert torch.equal(y1, y2), path
-        assert int(ws[:2048].view(torch.int32).abs().sum()) == 0, path
-        rows = np.unique(np.linspace(0, N - 1, 24).astype(np.int64))
-        ref = _oracle_gemm(to_np(x), to_np(w), None, None, fq.FLEX_EPI_NONE, 4, rows=rows)
-        assert_layer_close(y1[:, torch.from_numpy(rows).cuda()], ref, f"{path} {M}x{N}x{K}")
+    the workspace tickets and stream-K flags are back at zero. Required: both ticket
+    paths (at most 4 splits, and more: the partials are added 4 at a time) of the
+    128-row kernel, stream-K of the 256-row kernel, and with stream-K switched off the
+    256-row kernel's ticket path."""
+    old = fq.flex_set_gemm_streamk(streamk)
+    try:
+        seen = {}
+        for M, N, K in _plan_cases():
+            path = _path(fq.flex_gemm_plan(M, N, K))
+            if path not in seen or N * K < seen[path][1] * seen[path][2]:
+                seen[path] = (M, N, K)
+        need = [("tc128", "ticket<=4"), ("tc128", "ticket>4")]
+        need += [("tc256", "streamk")] if streamk else [("tc256", "ticket<=4")]
+        for k in need:
+            assert k in seen, sorted(seen)
+        for path, (M, N, K) in sorted(seen.items()):
+            x = synth.activations((M, K), 90, device="cuda")
+            w = synth.normal_f16((N, K), 91, 0.02, device="cuda")
+            W = fq.CompressedWeight(w, 4, 64)
+            ws = torch.zeros(max(16, fq.flex_gemm_ws_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
+            y1 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+            y2 = torch.empty_like(y1)
+            fq.flex_dequant_gemm(x, W, None, None, y1, M, fq.FLEX_EPI_NONE, ws)
+            fq.flex_dequant_gemm(x, W, None, None, y2, M, fq.FLEX_EPI_NONE, ws)
+            sync_status()
+            assert torch.equal(y1, y2), path
+            assert int(ws[:2048].view(torch.int32).abs().sum()) == 0, path
+            rows = np.unique(np.linspace(0, N - 1, 24).astype(np.int64))
+            ref = _oracle_gemm(to_np(x), to_np(w), None, None, fq.FLEX_EPI_NONE, 4, rows=rows)
+            assert_layer_close(y1[:, torch.from_numpy(rows).cuda()], ref, f"{path} {M}x{N}x{K}")
+            # every tile of the whole output is finished: full-row check of a few tokens
+            mrows = [0, M // 2, M - 1]
+            wd = fq.flexq_decompress(W.codes, W.meta, W.shape, W.cfg).float()
+            full = x[mrows].float() @ wd.t()
+            err = (y1[mrows].float() - full).abs().max().item()
+            assert err <= 1e-2 * full.abs().max().item() + 1e-3, (path, err)
+    finally:
+        fq.flex_set_gemm_streamk(old)

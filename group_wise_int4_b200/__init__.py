@@ -471,7 +471,7 @@ def flex_gemm_plan(M: int, N: int, K: int, bits: int = 4) -> dict:
     out = (ctypes.c_int32 * 4)()
     _check(lib().flex_gemm_plan(int(M), int(N), int(K), int(bits), ctypes.cast(out, ctypes.c_void_p)), "flex_gemm_plan")
     return {"kernel": ("gemv", "tc128", "tc256")[out[0]], "tiles": out[1], "splits": out[2],
-            "reduce": "none" if out[2] == 1 and out[3] == 0 else ("ticket", "cluster", "streamk")[out[3]]}
+            "reduce": "none" if out[2] == 1 and out[3] == 0 else ("ticket", "cluster", "streamk", "exchange")[out[3]]}
 
 
 def flex_set_gemm_streamk(enable: bool) -> bool:

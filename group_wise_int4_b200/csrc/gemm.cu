@@ -102,6 +102,9 @@ struct GemmParams {
     // sk_total of them, shared out evenly over the grid; tiles numbered tm * sk_tiles_n + tn
     int sk, sk_tiles_n;
     int64_t sk_total;
+    // gemm_tc2_kernel, splits in one wave without a cluster: the splits of a tile exchange
+    // their partials and each finishes a share of the columns (xchg = 1) instead of a ticket
+    int xchg;
     uint32_t off_x, off_c, off_m, off_bar;
     uint32_t tmem_cols;
     // fused store_cache (QKV projection): output features [kv.h, 2 kv.h) are the keys and
@@ -1284,26 +1287,31 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
             };
 
             if (p.sk) {
-                if (all_ok && sg.whole) {
-                    for (int col = 0; col < p.BN; col += 8) {
-                        float v[8];
-                        tc::tmem_ld8(taddr + col, v);
-                        finish8(col, v);
-                    }
-                } else if (all_ok && !sg.owner) {
+                // (every CTA keeps the flag protocol even after a wait gave up, so the flags
+                // are back at zero when the kernel ends; the data is then unspecified)
+                if (sg.whole) {
+                    if (all_ok)
+                        for (int col = 0; col < p.BN; col += 8) {
+                            float v[8];
+                            tc::tmem_ld8(taddr + col, v);
+                            finish8(col, v);
+                        }
+                } else if (!sg.owner) {
                     // a later piece of a shared tile (this CTA's first segment): partial to this
                     // CTA's slot, then published (the rings still feed the next segment, so the
                     // partial goes straight from the accumulator to the workspace)
-                    float* mine = p.part + static_cast<int64_t>(blockIdx.x) * pstride;
-                    for (int col = 0; col < p.BN; col += 8) {
-                        float v[8];
-                        tc::tmem_ld8(taddr + col, v);
-                        part_store8(mine, kRows2, row, col, v);
+                    if (all_ok) {
+                        float* mine = p.part + static_cast<int64_t>(blockIdx.x) * pstride;
+                        for (int col = 0; col < p.BN; col += 8) {
+                            float v[8];
+                            tc::tmem_ld8(taddr + col, v);
+                            part_store8(mine, kRows2, row, col, v);
+                        }
                     }
                     __threadfence();
                     asm volatile("bar.sync 1, 256;" ::: "memory");
                     if (et == 0) atomicExch(p.counters + blockIdx.x, 1);
-                } else if (all_ok) {
+                } else {
                     // the owner: its accumulator plus the later pieces, CTAs blockIdx.x + 1, ...
                     // up to the tile's last step, in K order
                     const int64_t tile_end = (static_cast<int64_t>(sg.tm) * p.sk_tiles_n + sg.tn + 1) * nst;
@@ -1321,7 +1329,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
                         for (int i = 0; i < np && pub; ++i) {
                             volatile int* f = p.counters + blockIdx.x + 1 + i;
                             while (*f == 0) {
-                                if (*abort || tc::globaltimer_ns() - t0 > p.wait_ns) {
+                                if (tc::globaltimer_ns() - t0 > p.wait_ns) {     // (peers publish even after an abort)
                                     *abort = 1;
                                     set_status(p.status, FLEX_ERR_TIMEOUT);
                                     pub = false;
@@ -1339,7 +1347,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
                         "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
                         "selp.u32 %0, 1, 0, q;\n\t}"
                         : "=r"(pall)
-                        : "r"(pub ? 1u : 0u)
+                        : "r"((pub && all_ok) ? 1u : 0u)
                         : "memory");
                     if (pall && stage_ok && (p.off_bar / 2) >= static_cast<uint32_t>(np) * kRows2 * 32) {
                         __threadfence();
@@ -1385,6 +1393,20 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
 #pragma unroll
                         for (int j = 0; j < 8; ++j) tc::st_shared_f32(base + ((col + j) * kRows2 + row) * 4, v[j]);
                     }
+                } else if (p.xchg) {
+                    // the column groups other splits finish (v % splits != this split), in
+                    // workspace layout, packed into the drained rings for the bulk stores below
+                    int j = 0;
+                    for (int v = 0; v < p.BN / 8; ++v) {
+                        if (v % p.splits == static_cast<int>(blockIdx.z)) continue;
+                        float x8[8];
+                        tc::tmem_ld8(taddr + v * 8, x8);
+                        const uint32_t sa = base + (j * kRows2 + row) * 32;
+                        tc::sts128(sa, x8[0], x8[1], x8[2], x8[3]);
+                        tc::sts128(sa + 16, x8[4], x8[5], x8[6], x8[7]);
+                        ++j;
+                    }
+                    tc::fence_proxy_async_smem();
                 } else if (stage_ok) {
                     // the partial, in its workspace layout, into the drained rings; one bulk
                     // store (issued with the ticket below) moves it to the workspace
@@ -1406,7 +1428,123 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
                     }
                 }
             }
-            if (!p.sk && p.splits > 1 && !p.cluster) {
+            if (!p.sk && p.splits > 1 && !p.cluster && p.xchg) {
+                // Exchange (all of the grid is resident at once: one wave, one CTA per SM):
+                // split z finishes the column groups v with v % S == z. Each split publishes
+                // the groups the others finish, waits for the others' copies of its own
+                // groups and adds all splits in split order (its own from TMEM). A split that
+                // gave up still publishes and counts itself done, so nobody waits for it.
+                const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+                const int S = p.splits, z = blockIdx.z, ng = p.BN / 8;
+                const int nown = (ng - z + S - 1) / S;                // groups z, z + S, ...
+                const int nmax = (ng + S - 1) / S;                    // slots per peer in the load area
+                int* flags = p.counters + tile * S;
+                int* done = p.counters + gridDim.x * gridDim.y * S + tile;
+                float* mine = p.part + (static_cast<int64_t>(tile) * S + z) * pstride;
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                if (et == 0) {
+                    if (all_ok) {
+                        int j = 0;
+                        for (int v = 0; v < ng; ++v) {
+                            if (v % S == z) continue;
+                            tc::bulk_store(mine + static_cast<int64_t>(v) * kRows2 * 8, base + j * kRows2 * 32,
+                                           kRows2 * 32);
+                            ++j;
+                        }
+                        tc::bulk_commit();
+                        tc::bulk_wait_all();
+                        tc::fence_proxy_async_global();
+                    }
+                    __threadfence();
+                    atomicExch(flags + z, 1);
+                }
+                bool pub = true;
+                if (et == 0) {
+                    const uint64_t t0 = tc::globaltimer_ns();
+                    for (int s2 = 0; s2 < S && pub; ++s2) {
+                        if (s2 == z) continue;
+                        volatile int* f = flags + s2;
+                        while (*f == 0) {
+                            if (tc::globaltimer_ns() - t0 > p.wait_ns) {         // (peers publish even after an abort)
+                                *abort = 1;
+                                set_status(p.status, FLEX_ERR_TIMEOUT);
+                                pub = false;
+                                break;
+                            }
+                            __nanosleep(128);
+                        }
+                    }
+                    __threadfence();
+                }
+                uint32_t pall;
+                asm volatile(
+                    "{\n\t.reg .pred p, q;\n\t"
+                    "setp.ne.u32 p, %1, 0;\n\t"
+                    "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
+                    "selp.u32 %0, 1, 0, q;\n\t}"
+                    : "=r"(pall)
+                    : "r"((pub && all_ok) ? 1u : 0u)
+                    : "memory");
+                if (pall && nown > 0) {
+                    // the peers' copies of this split's groups: peer slot k (peers in split
+                    // order, skipping z), group i at base + (k nmax + i) 8 KB
+                    if (et == 0) {
+                        tc::fence_proxy_async_global();
+                        tc::bar_arrive_expect_tx(B.red, static_cast<uint32_t>((S - 1) * nown) * kRows2 * 32);
+                        int k = 0;
+                        for (int s2 = 0; s2 < S; ++s2) {
+                            if (s2 == z) continue;
+                            const float* peer = p.part + (static_cast<int64_t>(tile) * S + s2) * pstride;
+                            for (int i = 0; i < nown; ++i)
+                                tc::bulk_load(base + (k * nmax + i) * kRows2 * 32,
+                                              peer + static_cast<int64_t>(z + i * S) * kRows2 * 8, kRows2 * 32, B.red);
+                            ++k;
+                        }
+                    }
+                    const bool w = tc::bar_wait(B.red, 0, abort, p.status, p.wait_ns);
+                    uint32_t wall;
+                    asm volatile(
+                        "{\n\t.reg .pred p, q;\n\t"
+                        "setp.ne.u32 p, %1, 0;\n\t"
+                        "barrier.cta.red.and.pred q, 1, 256, p;\n\t"
+                        "selp.u32 %0, 1, 0, q;\n\t}"
+                        : "=r"(wall)
+                        : "r"(w ? 1u : 0u)
+                        : "memory");
+                    if (wall) {
+                        for (int i = 0; i < nown; ++i) {
+                            const int v = z + i * S;
+                            float acc[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+                            int k = 0;
+                            for (int s2 = 0; s2 < S; ++s2) {              // split order
+                                float t8[8];
+                                if (s2 == z) {
+                                    tc::tmem_ld8(taddr + v * 8, t8);
+                                } else {
+                                    const uint32_t q = base + ((k * nmax + i) * kRows2 + row) * 32;
+                                    const float4 lo = tc::lds128f(q), hi = tc::lds128f(q + 16);
+                                    t8[0] = lo.x; t8[1] = lo.y; t8[2] = lo.z; t8[3] = lo.w;
+                                    t8[4] = hi.x; t8[5] = hi.y; t8[6] = hi.z; t8[7] = hi.w;
+                                    ++k;
+                                }
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) acc[j] += t8[j];
+                            }
+                            finish8(v * 8, acc);
+                        }
+                    } else {
+                        volatile int never = 0;                         // the copies land before exit
+                        tc::bar_wait(B.red, 0, &never, p.status);
+                    }
+                }
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                if (et == 0 && atomicAdd(done, 1) == S - 1) {            // the last split out resets
+                    for (int s2 = 0; s2 < S; ++s2) flags[s2] = 0;
+                    *done = 0;
+                }
+            } else if (!p.sk && p.splits > 1 && !p.cluster) {
                 // ticket, taken by every split (see gemm_tc_kernel); the last adds the partials in split order
                 const int tile = blockIdx.y * gridDim.x + blockIdx.x;
                 __threadfence();
@@ -2000,6 +2138,7 @@ struct Plan2 {
     int BN, tiles_n, tiles_m, splits, cps, nsx, nsc, xu, nslot, acc_stride, a_col0, cluster;
     int sk, grid;                          // stream-K schedule over `grid` CTAs
     int64_t sk_total;
+    int xchg;                              // one-wave splits exchange partials (no ticket)
     uint32_t off_c, off_m, off_bar, smem;
     int64_t ws_bytes, counters_bytes;
 };
@@ -2078,6 +2217,18 @@ Plan2 make_plan2(int M, int N, int K, int bits) {
     P.sk = 0;
     P.grid = tiles * P.splits;
     P.sk_total = 0;
+    // Splits that all run in one wave (one CTA per SM, so every CTA of the grid is resident
+    // at once) exchange partials: each split finishes 1/splits of the columns, instead of
+    // the last split adding all of them after the others.
+    {
+        const int ng = P.BN / 8, nmax = (ng + P.splits - 1) / P.splits;
+        P.xchg = (P.splits > 1 && !P.cluster && tiles * P.splits <= sm_count() &&
+                  static_cast<uint32_t>(P.BN) * kRows2 * 4 <= P.off_bar &&
+                  static_cast<uint32_t>((P.splits - 1) * nmax) * kRows2 * 32 <= P.off_bar &&
+                  tiles * (P.splits + 1) <= static_cast<int>(kTicketBytes / sizeof(int)))
+                     ? 1
+                     : 0;
+    }
     if (g_streamk.load(std::memory_order_relaxed) && P.splits > 1 && !P.cluster && tiles * P.splits > sm_count()) {
         const int sms = sm_count();
         const int nst = nk / ku;
@@ -2349,6 +2500,7 @@ int gemm2_launch(const void* x, const flexq_tensor* W, const void* bias, const v
     gp.sk = P.sk;
     gp.sk_tiles_n = P.tiles_n;
     gp.sk_total = P.sk_total;
+    gp.xchg = P.sk ? 0 : P.xchg;
     fill_kv_target(gp.kv, kv);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = P.sk ? dim3(P.grid, 1, 1) : dim3(P.tiles_n, P.tiles_m, P.splits);
@@ -2508,7 +2660,7 @@ extern "C" int flex_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t bits, int
         out[0] = 2;
         out[1] = P.tiles_n * P.tiles_m;
         out[2] = P.sk ? P.grid : P.splits;
-        out[3] = P.sk ? 2 : P.cluster;
+        out[3] = P.sk ? 2 : (P.cluster ? 1 : (P.xchg && P.splits > 1 ? 3 : 0));
     } else {
         const Plan P = make_plan(M, N, K, bits);
         out[0] = 1;

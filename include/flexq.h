@@ -299,7 +299,8 @@ int64_t flex_gemm_ws_bytes(int32_t M, int32_t N, int32_t K);
  * 2 the 256-row tcgen05 GEMM), out[1] its output tiles, out[2] the K splits per tile
  * (stream-K: the CTAs that share the tiles' K steps), out[3] how split results are
  * added: 0 through workspace partials and a ticket (or no split), 1 inside a
- * thread-block cluster, 2 stream-K (a tile's first CTA adds the later pieces). Needs a
+ * thread-block cluster, 2 stream-K (a tile's first CTA adds the later pieces), 3 an
+ * exchange (splits in one wave: each finishes a share of the columns). Needs a
  * current CUDA device (the plan depends on its SM count and cluster occupancy). */
 int flex_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t bits, int32_t* out);
 

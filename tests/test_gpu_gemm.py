@@ -231,7 +231,7 @@ def _plan_cases():
 
 
 def _path(pl):
-    if pl["reduce"] in ("none", "cluster", "streamk"):
+    if pl["reduce"] in ("none", "cluster", "streamk", "exchange"):
         return (pl["kernel"], pl["reduce"])
     return (pl["kernel"], "ticket<=4" if pl["splits"] <= 4 else "ticket>4")
 
@@ -242,8 +242,8 @@ def test_gemm_split_reduction_paths(streamk):
     the oracle on sampled output features and gives identical bits on a second call;
     the workspace tickets and stream-K flags are back at zero. Required: both ticket
     paths (at most 4 splits, and more: the partials are added 4 at a time) of the
-    128-row kernel, stream-K of the 256-row kernel, and with stream-K switched off the
-    256-row kernel's ticket path."""
+    128-row kernel; stream-K and the one-wave exchange of the 256-row kernel (and its
+    ticket path wherever the candidates reach it)."""
     old = fq.flex_set_gemm_streamk(streamk)
     try:
         seen = {}
@@ -252,7 +252,8 @@ def test_gemm_split_reduction_paths(streamk):
             if path not in seen or N * K < seen[path][1] * seen[path][2]:
                 seen[path] = (M, N, K)
         need = [("tc128", "ticket<=4"), ("tc128", "ticket>4")]
-        need += [("tc256", "streamk")] if streamk else [("tc256", "ticket<=4")]
+        need += ([("tc256", "streamk"), ("tc256", "exchange")] if streamk
+                 else [("tc256", "exchange"), ("tc256", "ticket<=4")])
         for k in need:
             assert k in seen, sorted(seen)
         for path, (M, N, K) in sorted(seen.items()):

@@ -14,10 +14,12 @@ GPU: every wait keeps a limit, and every thread still reaches every barrier.
 no timeout: an mbarrier try_wait may suspend until the phase completes, so waits that
 complete within one poll never run out.)
 
-Covered: the 256-row kernel with no split (148 CTAs), with splits reduced through
-workspace tickets (96 tiles x 3 splits) and with splits reduced inside a thread-block
-cluster (1 tile x 8 splits); the 128-row kernel (N not a multiple of 256) with and
-without a split."""
+Covered: the 256-row kernel with no split (148 CTAs), with the stream-K schedule (96
+tiles of 3 splits' worth of work), with splits exchanging partials in one wave (48 tiles
+x 3 splits) and with splits reduced inside a thread-block cluster (1 tile x 8 splits);
+the 128-row kernel (N not a multiple of 256) with and without a split. (A wait that
+gives up in the exchange or in stream-K still publishes this CTA's flag, so no peer
+waits for it past its own limit.)"""
 import pytest
 import torch
 
@@ -29,7 +31,8 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("M,N,K", [(144, 148 * 256, 1024),      # 256-row tiles, one per SM, no split
-                                   (144, 96 * 256, 12288),      # 96 tiles x 3 splits, ticket reduction
+                                   (144, 96 * 256, 12288),      # 96 tiles x 3 splits in 2 waves: stream-K
+                                   (144, 48 * 256, 12288),      # 48 x 3 splits in one wave: exchange
                                    (144, 256, 49152),           # 1 tile x 8 splits in one cluster
                                    (144, 37 * 128, 1024),       # 128-row kernel
                                    (144, 128, 49152)])          # 128-row kernel, 1 tile x 8 splits

@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
     constexpr int STAGE = 2 * CODE + 2 * META * 4;
     constexpr int DT_NS = DT_STAGES;       // ring depth (dynamic shared memory, dt_smem_bytes)
     static_assert(NW * 32 == DT_KEYS, "32 keys per warp and stage");
-    static_assert(CODE % (16 * DA_THREADS) == 0 && META % DA_THREADS == 0, "whole copy rounds");
+    static_assert((32 * KB / 16) % 32 == 0 && (32 * G) % 32 == 0, "whole copy rounds per warp");
     extern __shared__ __align__(16) uint8_t dt_ring[];
     auto ring = reinterpret_cast<uint8_t (*)[STAGE]>(dt_ring);
     __shared__ float sm_m[NW], sm_l[NW];
@@ -372,45 +372,51 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
     const uint8_t* vc_src = v_codes + (slot0 + j0) * KB;
     const uint32_t* km_src = k_meta + (slot0 + j0) * G;
     const uint32_t* vm_src = v_meta + (slot0 + j0) * G;
+    // Each warp copies and later reads only its own 32 keys of a stage (the K and V code
+    // rows and metadata of keys [32 w, 32 w + 32)), so a stage needs no CTA barrier: the
+    // warp's own copies are waited for, then shared across its lanes by __syncwarp.
+    constexpr int WCH = 32 * KB / 16;                 // 16-byte code chunks per warp and stage
+    constexpr int WMETA = 32 * G;                     // metadata words per warp and stage
     auto load_stage = [&](int s) {
         uint8_t* st = ring[s % DT_NS];
-        const int kbase = s * DT_KEYS;
-        if (kbase + DT_KEYS <= nkeys) {
-            // a whole stage: no per-copy predicate or clamped address
+        const int kbase = s * DT_KEYS + warp * 32;    // this warp's first key of the stage
+        const int c0 = warp * WCH, m0w = warp * WMETA;
+        if (kbase + 32 <= nkeys) {
+            // all 32 keys present: no per-copy predicate or clamped address
             const uint32_t s0 = static_cast<uint32_t>(__cvta_generic_to_shared(st));
             const uint8_t* kc = kc_src + static_cast<int64_t>(kbase) * KB;
             const uint8_t* vc = vc_src + static_cast<int64_t>(kbase) * KB;
             const uint32_t* km = km_src + static_cast<int64_t>(kbase) * G;
             const uint32_t* vm = vm_src + static_cast<int64_t>(kbase) * G;
 #pragma unroll
-            for (int i = 0; i < CODE / (16 * DA_THREADS); ++i) {
-                const int u = threadIdx.x + i * DA_THREADS;
-                cp_async16u(s0 + u * 16, kc + u * 16);
-                cp_async16u(s0 + CODE + v_chunk<D>(u) * 16, vc + u * 16);
+            for (int i = 0; i < WCH / 32; ++i) {
+                const int ul = lane + i * 32;
+                cp_async16u(s0 + (c0 + ul) * 16, kc + ul * 16);
+                cp_async16u(s0 + CODE + v_chunk<D>(c0 + ul) * 16, vc + ul * 16);
             }
 #pragma unroll
-            for (int i = 0; i < META / DA_THREADS; ++i) {
-                const int u = threadIdx.x + i * DA_THREADS;
-                cp_async4u(s0 + 2 * CODE + u * 4, km + u);
-                cp_async4u(s0 + 2 * CODE + META * 4 + u * 4, vm + u);
+            for (int i = 0; i < WMETA / 32; ++i) {
+                const int ul = lane + i * 32;
+                cp_async4u(s0 + 2 * CODE + (m0w + ul) * 4, km + ul);
+                cp_async4u(s0 + 2 * CODE + META * 4 + (m0w + ul) * 4, vm + ul);
             }
             return;
         }
 #pragma unroll
-        for (int i = 0; i < CODE / (16 * DA_THREADS); ++i) {
-            const int u = threadIdx.x + i * DA_THREADS;
-            const bool ok = kbase + (u * 16) / KB < nkeys;
-            const int64_t off = ok ? static_cast<int64_t>(kbase) * KB + u * 16 : 0;
-            cp_async16(st + u * 16, kc_src + off, ok);
-            cp_async16(st + CODE + v_chunk<D>(u) * 16, vc_src + off, ok);
+        for (int i = 0; i < WCH / 32; ++i) {
+            const int ul = lane + i * 32;
+            const bool ok = kbase + (ul * 16) / KB < nkeys;
+            const int64_t off = ok ? static_cast<int64_t>(kbase) * KB + ul * 16 : 0;
+            cp_async16(st + (c0 + ul) * 16, kc_src + off, ok);
+            cp_async16(st + CODE + v_chunk<D>(c0 + ul) * 16, vc_src + off, ok);
         }
 #pragma unroll
-        for (int i = 0; i < META / DA_THREADS; ++i) {
-            const int u = threadIdx.x + i * DA_THREADS;
-            const bool ok = kbase + u / G < nkeys;
-            const int64_t off = ok ? static_cast<int64_t>(kbase) * G + u : 0;
-            cp_async4(st + 2 * CODE + u * 4, km_src + off, ok);
-            cp_async4(st + 2 * CODE + META * 4 + u * 4, vm_src + off, ok);
+        for (int i = 0; i < WMETA / 32; ++i) {
+            const int ul = lane + i * 32;
+            const bool ok = kbase + ul / G < nkeys;
+            const int64_t off = ok ? static_cast<int64_t>(kbase) * G + ul : 0;
+            cp_async4(st + 2 * CODE + (m0w + ul) * 4, km_src + off, ok);
+            cp_async4(st + 2 * CODE + META * 4 + (m0w + ul) * 4, vm_src + off, ok);
         }
     };
     // Inside a layer call (early_kv) the cached keys/values [0, pos) were written by
@@ -491,11 +497,11 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
 #pragma unroll
     for (int i = 0; i < NMT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
 
-    // One barrier per stage: after it, stage s has landed for every thread and every warp
-    // has finished stage s - 1, whose slot then takes stage s + DT_NS - 1.
+    // Per warp and stage: after __syncwarp, stage s has landed for every lane and every
+    // lane has finished stage s - 1, whose slot then takes stage s + DT_NS - 1.
     for (int s = 0; s < nst; ++s) {
         cp_async_wait<DT_NS - 2>();
-        __syncthreads();
+        __syncwarp();
         if (s + DT_NS - 1 < nst) load_stage(s + DT_NS - 1);
         cp_async_commit();
         const int kw0 = s * DT_KEYS + warp * 32;                 // the warp's first key

@@ -141,17 +141,22 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decompress_contig_kernel
 
 // ---------------------------------------------------------------------------------
 // strided compress, one pass: x viewed as [outer][ng*GS][inner]; a work item is (o, g,
-// 8 columns) and NS = GS/8 lanes share it, each holding 8 of the group's rows in
+// 8 columns) and NS = GS/RPS lanes share it, each holding RPS of the group's rows in
 // registers. Lane = IPW slice + ci: a warp covers IPW = 32/NS adjacent items (ci), so
 // every load instruction reads 16 IPW contiguous bytes per row slice. The slices combine
 // min/max with shuffles (lane offsets IPW, 2 IPW, ...) and then quantise their own rows
 // with no second read.
+// Rows per slice: 8, or 16 for groups of 128 rows, so that a slice still spans at most 8
+// lanes and a warp reads at least 64 contiguous bytes of every row (with 8 rows per slice
+// a 128-row group took 16 lanes and left 32-byte row pieces: about 1.3-2.3 TB/s).
+constexpr int strided_rps(int gs) { return gs >= 128 ? 16 : 8; }
+
 template <int BITS, int GS>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) compress_strided_1pass_kernel(const __half* __restrict__ x,
+__global__ void __launch_bounds__(kThreads, GS >= 128 ? 2 : kMinBlocks) compress_strided_1pass_kernel(const __half* __restrict__ x,
                                                                           uint8_t* __restrict__ codes,
                                                                           uint32_t* __restrict__ meta, int64_t outer,
                                                                           int64_t ng, int64_t inner) {
-    constexpr int RPS = 8;                     // rows per slice
+    constexpr int RPS = strided_rps(GS);       // rows per slice
     constexpr int NS = GS / RPS;               // slices (lanes) per item
     constexpr int IPW = 32 / NS;               // items per warp
     constexpr int CB = GS * BITS / 8;          // code rows per group
@@ -566,9 +571,10 @@ int launch_compress(const Geometry& g, const __half* x, uint8_t* codes, uint32_t
     } else {
         const bool vec = (g.inner % 8 == 0);
         const int64_t items = g.outer * g.ng * (vec ? g.inner / 8 : g.inner);
-        if (vec)   // GS/8 lanes per item
+        if (vec)   // GS / strided_rps(GS) lanes per item
             compress_strided_1pass_kernel<BITS, GS>
-                <<<grid_for<compress_strided_1pass_kernel<BITS, GS>>(items * (GS / 8)), kThreads, 0, st>>>(x, codes, meta, g.outer, g.ng, g.inner);
+                <<<grid_for<compress_strided_1pass_kernel<BITS, GS>>(items * (GS / strided_rps(GS))), kThreads, 0, st>>>(
+                    x, codes, meta, g.outer, g.ng, g.inner);
         else
             compress_strided_kernel<BITS, GS>
                 <<<grid_for<compress_strided_kernel<BITS, GS>>(items), kThreads, 0, st>>>(x, codes, meta, g.outer, g.ng, g.inner);

@@ -688,6 +688,17 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
                                                        h, stream=stream))
     kern["layernorm"] = dict(ms=ms, bytes=2 * b * h * 2 + 2 * h * 2, flops=0.0, launches_per_call=2,
                              kernel=main_kernel(names, "layernorm_kernel"), kernels=names, source=["kv_ln.cu"])
+    # the whole layer call in the same regime (a graph of one call per layer, replayed):
+    # against the sum of its kernels' parts it shows what the kernel boundaries cost
+    xl = synth.decode_inputs(b * calls, h, 0, cfg["seed"], device=dev)
+    yl = torch.empty((b * calls, h), dtype=torch.float16, device=dev)
+    ms_layer, names = time_cycle(lambda l: (fq.flex_decode_layer(layers[l], caches[l], xl, yl, b, pos, stack.ws_dec,
+                                                                  stream=stream) if calls == 1 else
+                                            fq.flex_decode_layer_batches(layers[l], stack.caches[l], xl, yl, b, pos,
+                                                                         stack.ws_dec, stream=stream)))
+    layer_call = {"us": ms_layer * 1e3, "kernels": names,
+                  "note": "one decode layer call (all its kernels, programmatic-launch chained), graph-timed "
+                          "like the parts"}
     for k, v in kern.items():
         v["us"] = v["ms"] * 1e3
         v["gbs"] = v["bytes"] / (v["ms"] * 1e6)
@@ -755,7 +766,8 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
     rc = fq.flex_get_status()
     if rc != 0:
         raise RuntimeError(f"parts failed: {fq.flex_status_string(rc)}")
-    return {"kernels": kern, "per_kernel_per_layer_call": per_kernel, "prefill": prefill}, roofline
+    return {"kernels": kern, "per_kernel_per_layer_call": per_kernel, "layer_call": layer_call,
+            "prefill": prefill}, roofline
 
 
 def measure_secondary_decode(fq, torch, synth, name, peaks, dev, ntok=8, reps=5):

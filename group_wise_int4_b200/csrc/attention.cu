@@ -349,7 +349,9 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
     extern __shared__ __align__(16) uint8_t dt_ring[];
     auto ring = reinterpret_cast<uint8_t (*)[STAGE]>(dt_ring);
     __shared__ float sm_m[NW], sm_l[NW];
-    __shared__ float sm_o[NW][D];
+    // the warps' output rows reuse the ring once every warp is done with its stages
+    float (*const sm_o)[D] = reinterpret_cast<float (*)[D]>(dt_ring);
+    static_assert(NW * D * 4 <= DT_NS * STAGE, "the output rows fit in the ring");
     __shared__ float sm_red[NW];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -640,6 +642,7 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
         }
     }
     cp_async_wait<0>();
+    __syncthreads();                       // every warp is done with the ring (sm_o reuses it)
 
     // ---- warp result: W_n, U_n per group (sum over the owner lanes), then the rows
 #pragma unroll

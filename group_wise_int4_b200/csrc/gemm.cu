@@ -815,6 +815,13 @@ constexpr int kRT = 2;                  // 128-row tiles per CTA
 // 4-11 dequantisation and the epilogue. One CTA per SM, so a thread may hold up to 168
 // registers (the epilogue with the fused store_cache needs about 140).
 constexpr int kThreads2 = 384;
+// MMA issuing threads: 2 (warp 2 tile 0, warp 3 tile 1) or 1 (warp 2 both tiles, one
+// commit per unit); a build constant, chosen by measurement.
+#ifndef FLEXQ_TC2_ISSUERS
+#define FLEXQ_TC2_ISSUERS 2
+#endif
+constexpr int kIssuers2 = FLEXQ_TC2_ISSUERS;
+static_assert(kIssuers2 == 1 || kIssuers2 == 2, "one or two issuers");
 constexpr int kRows2 = kRT * kBM;       // 256
 constexpr int kDoneRing2 = 16;          // mma_done barriers (units)
 constexpr int kMaxPieces = 8;           // stream-K: later pieces of one tile that its owner adds
@@ -920,7 +927,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
         }
         for (int s = 0; s < NSX; ++s) tc::bar_init(B.x_full + 8 * s, 1);
         for (int s = 0; s < NSLOT; ++s) tc::bar_init(B.a_full + 8 * s, kDequantThreads);
-        for (int s = 0; s < kDoneRing2; ++s) tc::bar_init(B.mma_done + 8 * s, kRT);   // both issuers commit each unit
+        for (int s = 0; s < kDoneRing2; ++s) tc::bar_init(B.mma_done + 8 * s, kIssuers2);   // every issuer commits each unit
         tc::bar_init(B.acc_full, kDequantThreads);
         for (int i = 0; i < 4; ++i) tc::bar_init(B.drain + 8 * i, 1);
         tc::bar_init(B.red, 1);
@@ -1017,9 +1024,9 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
         }
         __syncwarp();
     } else if (warp == 2 || warp == 3) {
-        // ---------------- MMA issuers: warp 2 tile 0, warp 3 tile 1 ----------------
+        // ---------------- MMA issuers: warp 2 tile 0, warp 3 tile 1 (or warp 2 both) ----------------
         const int t = warp - 2;
-        if (lane == 0) {
+        if (lane == 0 && t < kIssuers2) {
             const uint32_t idesc = tc::idesc_f16_f32(kBM, p.BN);
             const uint32_t d_acc = tmem + static_cast<uint32_t>(t * p.acc_stride);
             int xs = 0, xc = 0;                 // activation stage and chunk within it
@@ -1045,6 +1052,8 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
                     const uint32_t a_tm = tmem + static_cast<uint32_t>(p.a_col0 + (sa * kRT + t) * 32);
                     const uint64_t bd = tc::desc_k_sw128(sX + static_cast<uint32_t>(xs * XU + xc) * xbytes);
                     issue_ksteps<1>(d_acc, a_tm, bd, idesc, 0, u == 0);
+                    if (kIssuers2 == 1)                 // tile 1 too, same activation stage
+                        issue_ksteps<1>(tmem + static_cast<uint32_t>(p.acc_stride), a_tm + 32, bd, idesc, 0, u == 0);
                     if (++xc == XU) {
                         xc = 0;
                         if (++xs == NSX) { xs = 0; xph ^= 1; }

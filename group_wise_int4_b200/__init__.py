@@ -107,6 +107,7 @@ _SIGS = {
     "flex_set_gemm_gate": (_P, [_P]),
     "flex_gemm_plan": (_I32, [_I32, _I32, _I32, _I32, _P]),
     "flex_set_gemm_streamk": (_I32, [_I32]),
+    "flex_set_gemm_gemv": (_I32, [_I32]),
     "flex_status_string": (ctypes.c_char_p, [_I32]),
     "flex_abi_layout": (_I64, [_I32, _I32]),
 }
@@ -477,6 +478,11 @@ def flex_gemm_plan(M: int, N: int, K: int, bits: int = 4) -> dict:
 def flex_set_gemm_streamk(enable: bool) -> bool:
     """Stream-K schedule of the 256-row GEMM for later plans; returns the previous setting."""
     return bool(lib().flex_set_gemm_streamk(1 if enable else 0))
+
+
+def flex_set_gemm_gemv(enable: bool) -> bool:
+    """Small-batch GEMV route for later launches; returns the previous setting."""
+    return bool(lib().flex_set_gemm_gemv(1 if enable else 0))
 
 
 def flex_set_gemm_gate(gate) -> int:

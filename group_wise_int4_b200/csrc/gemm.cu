@@ -2308,8 +2308,12 @@ Plan make_plan(int M, int N, int K, int bits) {
 }
 
 // The register-dequant GEMV serves int4 weights for up to 32 activation rows (one tile
-// of n-tiles); larger batches and prefill go to the tcgen05 GEMM.
-bool gemv_eligible(int M, int N, int bits) { return bits == 4 && M >= 1 && M <= 32 && N % kGvRows == 0; }
+// of n-tiles) unless switched off (flex_set_gemm_gemv); larger batches and prefill go to
+// the tcgen05 GEMM.
+std::atomic<int> g_gemv{1};
+bool gemv_eligible(int M, int N, int bits) {
+    return g_gemv.load(std::memory_order_relaxed) && bits == 4 && M >= 1 && M <= 32 && N % kGvRows == 0;
+}
 
 struct GemvPlan {
     int nt, tiles, splits, gps, cluster;
@@ -2653,6 +2657,8 @@ extern "C" int64_t flex_gemm_ws_bytes(int32_t M, int32_t N, int32_t K) {
 }
 
 extern "C" int32_t flex_set_gemm_streamk(int32_t enable) { return g_streamk.exchange(enable ? 1 : 0); }
+
+extern "C" int32_t flex_set_gemm_gemv(int32_t enable) { return g_gemv.exchange(enable ? 1 : 0); }
 
 extern "C" int flex_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t bits, int32_t* out) {
     FLEX_REQUIRE(out != nullptr && M > 0 && N > 0 && K > 0, FLEX_ERR_INVALID_ARG);

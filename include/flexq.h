@@ -308,6 +308,11 @@ int flex_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t bits, int32_t* out);
  * use K splits with workspace tickets instead, e.g. for comparison. Process-wide;
  * returns the previous setting. */
 int32_t flex_set_gemm_streamk(int32_t enable);
+/* The small-batch GEMV route (on by default: int4 weights, at most 32 activation rows):
+ * enable = 0 sends those problems to the 128-row tcgen05 GEMM as well, e.g. for
+ * comparison. Process-wide; returns the previous setting. A workspace sized under one
+ * setting may be too small under the other (FLEX_ERR_WORKSPACE). */
+int32_t flex_set_gemm_gemv(int32_t enable);
 int flex_dequant_gemm(const void* x, const flexq_tensor* W, const void* bias,
                       const void* residual, void* y, int32_t M, int32_t epilogue,
                       void* ws, int64_t ws_bytes, void* stream);

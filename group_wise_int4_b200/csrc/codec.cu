@@ -25,7 +25,7 @@ constexpr int kThreads = 256;
 // Vectors in flight per thread (compress) and resident blocks per SM the register budget
 // is sized for: build constants, tuned by measurement.
 #ifndef FLEXQ_CODEC_UNROLL
-#define FLEXQ_CODEC_UNROLL 4
+#define FLEXQ_CODEC_UNROLL 2
 #endif
 #ifndef FLEXQ_CODEC_MINB
 #define FLEXQ_CODEC_MINB 4
@@ -51,24 +51,21 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) compress_contig_kernel(c
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     const int64_t stride = nwarps * GPW;
 
-    for (int64_t base = warp * GPW; base < G; base += stride * kUnroll) {
-        uint4 v[kUnroll];
+    auto load = [&](uint4 (&v)[kUnroll], int64_t base) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t g = base + u * stride + lane / L;
             v[u] = g < G ? ld_stream_v4(x + g * GS + sub * 8) : make_uint4(0, 0, 0, 0);
         }
+    };
+    auto process = [&](const uint4 (&v)[kUnroll], int64_t base) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t g = base + u * stride + lane / L;
             __half2 hmn, hmx;
             minmax8(v[u], hmn, hmx);
-            float mn = hmin_of(hmn), mx = hmax_of(hmx);
-#pragma unroll
-            for (int off = 1; off < L; off <<= 1) {
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            }
+            float mn, mx;
+            group_minmax<L>(hmn, hmx, mn, mx);
             const __half s16 = group_scale16<BITS>(mn, mx);
             const float s = __half2float(s16);
             if (g < G) {
@@ -80,6 +77,20 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) compress_contig_kernel(c
                 if (sub == 0) meta[g] = pack_half2_bits(stored_min16(mn), s16);
             }
         }
+    };
+    // software pipelined: the next step's vectors are requested before this step's are
+    // quantised, so the loads of one step overlap the arithmetic of the previous one
+    int64_t base = warp * GPW;
+    uint4 v[kUnroll];
+    load(v, base);
+    while (base < G) {
+        const int64_t next = base + stride * kUnroll;
+        uint4 nv[kUnroll];
+        load(nv, next);
+        process(v, base);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) v[u] = nv[u];
+        base = next;
     }
 }
 
@@ -95,11 +106,16 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decompress_contig_kernel
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
     for (int64_t base = tid; base < items; base += nthreads * kDecUnroll) {
+        // codes and the group's metadata word are both requested before any is used: the
+        // metadata of a tensor larger than L2 comes from DRAM too, and a load issued only
+        // when its item is converted would add one memory round trip per item
         uint2 c[kDecUnroll];
+        uint32_t mw[kDecUnroll];
 #pragma unroll
         for (int u = 0; u < kDecUnroll; ++u) {
             const int64_t it = base + u * nthreads;
             c[u] = make_uint2(0u, 0u);
+            mw[u] = 0u;
             if (it < items) {
                 if (BITS == 4) {
                     asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(c[u].x) : "l"(codes + it * 4));
@@ -108,14 +124,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decompress_contig_kernel
                                  : "=r"(c[u].x), "=r"(c[u].y)
                                  : "l"(codes + it * 8));
                 }
+                // the 8 values lie in one group (GS >= 32)
+                mw[u] = __ldg(meta + (it * 8) / GS);
             }
         }
 #pragma unroll
         for (int u = 0; u < kDecUnroll; ++u) {
             const int64_t it = base + u * nthreads;
             if (it >= items) continue;
-            // the 8 values lie in one group (GS >= 32)
-            const uint32_t m = __ldg(meta + (it * 8) / GS);
+            const uint32_t m = mw[u];
             const float mn = h2f_lo(m);
             const float step = group_step(__ushort_as_half(static_cast<unsigned short>(m >> 16)));
             uint32_t out[4];

@@ -30,9 +30,9 @@ __device__ __forceinline__ __half group_scale16(float mn, float mx) {
 __device__ __forceinline__ __half stored_min16(float mn) { return __float2half_rn(__fadd_rn(mn, 0.0f)); }
 
 // ---- packed fp32 pairs ---------------------------------------------------------------
-// sm_100 executes add / sub / mul on two fp32 lanes held in one 64-bit register, each
-// lane rounded like the scalar instruction; the quantiser's per-value arithmetic runs on
-// pairs of values this way.
+// sm_100 executes add / mul on two fp32 lanes held in one 64-bit register, each lane
+// rounded like the scalar instruction; the quantiser's per-value arithmetic runs on pairs
+// of values this way.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
     uint64_t r;
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -40,11 +40,6 @@ __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
 }
 __device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
 }
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     uint64_t d;
@@ -72,10 +67,18 @@ __device__ __forceinline__ uint32_t quant_bits(float x, float mn, float s) {
 }
 
 // quant_bits of the two fp16 values of a half2 word (low value first), with min and
-// scale given as packed pairs {min, min} and {scale, scale}.
+// scale given as packed pairs {min_lo, min_hi} and {scale_lo, scale_hi} (the two values
+// may belong to different groups).
+// fl(x - min) is formed by the mixed-precision subtract (fp16 operand, fp32 operand and
+// result): the fp16 value enters exactly, as after a conversion, and the difference is
+// rounded once - the same bits as converting first, one instruction fewer per value.
 __device__ __forceinline__ void quant_bits_pair(uint32_t w, uint64_t mn2, uint64_t s2, uint32_t& lo, uint32_t& hi) {
-    float a, b;
-    f2_unpack(f2_mul(f2_sub(f2_pack(h2f_lo(w), h2f_hi(w)), mn2), s2), a, b);
+    float a, b, mn, mn_hi;
+    f2_unpack(mn2, mn, mn_hi);
+    asm("{.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tsub.rn.f32.f16 %0, l, %3;\n\tsub.rn.f32.f16 %1, h, %4;}"
+        : "=f"(a), "=f"(b)
+        : "r"(w), "f"(mn), "f"(mn_hi));
+    f2_unpack(f2_mul(f2_pack(a, b), s2), a, b);
     f2_unpack(f2_add(f2_pack(fmaxf(a, 0.0f), fmaxf(b, 0.0f)), f2_pack(12582912.0f, 12582912.0f)), a, b);
     lo = __float_as_uint(a);
     hi = __float_as_uint(b);
@@ -124,6 +127,23 @@ __device__ __forceinline__ void minmax8(uint4 v, __half2& mn, __half2& mx) {
     const __half2 d = *reinterpret_cast<const __half2*>(&v.w);
     mn = __hmin2(__hmin2(a, b), __hmin2(c, d));
     mx = __hmax2(__hmax2(a, b), __hmax2(c, d));
+}
+
+// min and max over the L lanes of a group (L a power of two, lanes aligned to L) from
+// each lane's half2 min/max pair: {min, -max} travel as one half2 word, so every
+// shuffle round is one shuffle and one packed min (exact: selects and a negation).
+template <int L>
+__device__ __forceinline__ void group_minmax(__half2 hmn, __half2 hmx, float& mn, float& mx) {
+    const __half2 a = __halves2half2(__low2half(hmn), __hneg(__low2half(hmx)));
+    const __half2 b = __halves2half2(__high2half(hmn), __hneg(__high2half(hmx)));
+    __half2 r = __hmin2(a, b);
+#pragma unroll
+    for (int off = 1; off < L; off <<= 1) {
+        const uint32_t o = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<const uint32_t*>(&r), off);
+        r = __hmin2(r, *reinterpret_cast<const __half2*>(&o));
+    }
+    mn = __low2float(r);
+    mx = -__high2float(r);
 }
 
 // Reduce a half2 min/max pair to scalars (exact: min/max select, no rounding).

@@ -528,15 +528,18 @@ __global__ void __launch_bounds__(DA_THREADS, D == 64 ? 7 : FLEXQ_DT_MINB_128) d
                     x0[0] = a.x; x0[1 % KW] = a.y;
                     x8[0] = c.x; x8[1 % KW] = c.y;
                 }
-                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+                // two accumulator sets (even and odd k-steps) halve the dependent MMA chain
+                float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int w = 0; w < KW; ++w) {
                     const uint32_t y0 = x0[w] >> 8, y8 = x8[w] >> 8;
                     const uint32_t a0[4] = {nib_lo(x0[w]), nib_lo(x8[w]), nib_hi(x0[w]), nib_hi(x8[w])};
                     mma16816(sacc, a0, bq[2 * w][0], bq[2 * w][1]);
                     const uint32_t a1[4] = {nib_lo(y0), nib_lo(y8), nib_hi(y0), nib_hi(y8)};
-                    mma16816(sacc, a1, bq[2 * w + 1][0], bq[2 * w + 1][1]);
+                    mma16816(sacc2, a1, bq[2 * w + 1][0], bq[2 * w + 1][1]);
                 }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sacc[i] += sacc2[i];
                 // per key: sum over the groups this lane holds (columns 2t, 2t+1)
                 float s0 = 0.f, s8 = 0.f;
 #pragma unroll

@@ -148,22 +148,60 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
-// 8 codes of 4 bits (one u32, element e in bits 4e..4e+3) -> 8 fp16 in natural order.
-__device__ __forceinline__ uint4 dequant8_4bit(uint32_t w, uint32_t step2, uint32_t mn2) {
-    const uint32_t p0 = dequant_pair(lop_nib(w), step2, mn2);         // (e0, e4)
-    const uint32_t p1 = dequant_pair(lop_nib(w >> 4), step2, mn2);    // (e1, e5)
-    const uint32_t p2 = dequant_pair(lop_nib(w >> 8), step2, mn2);    // (e2, e6)
-    const uint32_t p3 = dequant_pair(lop_nib(w >> 12), step2, mn2);   // (e3, e7)
-    return make_uint4(prmt(p0, p1, 0x5410u), prmt(p2, p3, 0x5410u), prmt(p0, p1, 0x7632u), prmt(p2, p3, 0x7632u));
+__device__ __forceinline__ uint32_t lop_nib_hi(uint32_t w) {
+    // (w & 0x00F000F0) | 0x64006400: the high nibbles of bytes 0 and 2 left in place, as
+    // fp16 1024 + 16 q
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(0x00F000F0u), "r"(0x64006400u));
+    return r;
+}
+
+// Dequantisation constants of one group from its metadata word {min, scale}, each packed
+// twice: step = fp16(1/scale) (0 for a constant group, which then decodes to min), step/16
+// for codes read in place from a byte's high nibble (fp16 16 q: 16 q * step/16 = q * step,
+// exactly while step/16 is a normal fp16), and min.
+struct DqConst {
+    uint32_t step2, step2_16, mn2;
+};
+__device__ __forceinline__ DqConst dq_const(uint32_t mw) {
+    const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
+    const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
+    const float r = sc32 > 0.f ? rcp_approx(sc32) : 0.f;
+    const __half2 s = __float2half2_rn(r), s16 = __float2half2_rn(r * 0.0625f), m = __half2half2(mn);
+    DqConst k;
+    k.step2 = *reinterpret_cast<const uint32_t*>(&s);
+    k.step2_16 = *reinterpret_cast<const uint32_t*>(&s16);
+    k.mn2 = *reinterpret_cast<const uint32_t*>(&m);
+    return k;
+}
+
+// 8 codes of 4 bits (one u32, element e in bits 4e..4e+3) as the four pairs (e0,e4)
+// (e1,e5) (e2,e6) (e3,e7): low nibbles masked out directly, high nibbles in place, one
+// shift for the upper byte of each half.
+__device__ __forceinline__ void dequant8_4bit_pairs(uint32_t w, const DqConst& k, uint32_t (&p)[4]) {
+    const uint32_t w8 = w >> 8;
+    p[0] = dequant_pair(lop_nib(w), k.step2, k.mn2);           // (e0, e4)
+    p[1] = dequant_pair(lop_nib_hi(w), k.step2_16, k.mn2);     // (e1, e5)
+    p[2] = dequant_pair(lop_nib(w8), k.step2, k.mn2);          // (e2, e6)
+    p[3] = dequant_pair(lop_nib_hi(w8), k.step2_16, k.mn2);    // (e3, e7)
+}
+
+// 8 codes of 4 bits -> 8 fp16 in natural order.
+__device__ __forceinline__ uint4 dequant8_4bit(uint32_t w, const DqConst& k) {
+    uint32_t p[4];
+    dequant8_4bit_pairs(w, k, p);
+    return make_uint4(prmt(p[0], p[1], 0x5410u), prmt(p[2], p[3], 0x5410u), prmt(p[0], p[1], 0x7632u),
+                      prmt(p[2], p[3], 0x7632u));
 }
 
 // Same 8 codes, left in the pair order the unpack produces: (e0,e4) (e1,e5) (e2,e6)
 // (e3,e7), i.e. positions [e0 e4 e1 e5 e2 e6 e3 e7]. The activation operand must then
 // use the same order inside every 8-block of K (the "interleaved" activation layout the
 // layer kernels write), and the MMA sees matching K positions on both sides.
-__device__ __forceinline__ uint4 dequant8_4bit_il(uint32_t w, uint32_t step2, uint32_t mn2) {
-    return make_uint4(dequant_pair(lop_nib(w), step2, mn2), dequant_pair(lop_nib(w >> 4), step2, mn2),
-                      dequant_pair(lop_nib(w >> 8), step2, mn2), dequant_pair(lop_nib(w >> 12), step2, mn2));
+__device__ __forceinline__ uint4 dequant8_4bit_il(uint32_t w, const DqConst& k) {
+    uint32_t p[4];
+    dequant8_4bit_pairs(w, k, p);
+    return make_uint4(p[0], p[1], p[2], p[3]);
 }
 
 __device__ __forceinline__ uint32_t lop_byte(uint32_t x) {
@@ -616,25 +654,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 }
                 tc::fence_after_sync();
             }
+            // the step's groups (moff + c) % 4 of the metadata tile, decoded together (a
+            // select per word: a runtime array index would put them in local memory)
+            DqConst kc[KU];
 #pragma unroll
             for (int c = 0; c < KU; ++c) {
-                // group (moff + c) % 4 of the metadata tile (a select: a runtime array index
-                // would put the words in local memory)
                 const int mi = (moff + c) & 3;
-                const uint32_t mw = mi == 0 ? mrow.x : (mi == 1 ? mrow.y : (mi == 2 ? mrow.z : mrow.w));
-                const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
-                const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
-                // step = fp16(1/scale); a constant group (scale 0) gets step 0 and decodes to min
-                const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
-                const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
-                const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
-                const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
+                kc[c] = dq_const(mi == 0 ? mrow.x : (mi == 1 ? mrow.y : (mi == 2 ? mrow.z : mrow.w)));
+            }
+#pragma unroll
+            for (int c = 0; c < KU; ++c) {
+                const uint32_t step2 = kc[c].step2, mnv2 = kc[c].mn2;
                 uint32_t r[16];
                 if (BITS == 4) {
                     const uint32_t w[4] = {cw[c][0].x, cw[c][0].y, cw[c][0].z, cw[c][0].w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2) : dequant8_4bit(w[j], step2, mnv2);
+                        const uint4 v = XPERM ? dequant8_4bit_il(w[j], kc[c]) : dequant8_4bit(w[j], kc[c]);
                         r[4 * j] = v.x;
                         r[4 * j + 1] = v.y;
                         r[4 * j + 2] = v.z;
@@ -805,7 +841,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // TMEM: accumulator of tile t at columns [t acc_stride, t acc_stride + BN); from a_col0 on,
 // nslot A slots of one chunk per tile (slot s of tile t at a_col0 + (s * 2 + t) * 32). A
 // "unit" is one chunk: one A slot fill, one MMA issue round per tile, one commit per
-// issuer (the mma_done ring counts units, across all segments of the CTA). A CTA works
+// issuer (the mma_done ring counts units, across all segments of the CTA). The A-slot and
+// mma_done barriers are per tile: a tile's issuer waits only for its own 4 dequantising
+// warps, and they only for its commits, so one tile's issuer keeps the tensor pipe busy
+// while the other waits (two threads issuing back to back are what it takes to keep the
+// pipe full at these N: one thread issues an MMA every ~130-160 cycles, a 128 x 144 x 16
+// MMA occupies the pipe for 72). A CTA works
 // through one or more segments (see SegWalk); between segments the issuers wait for the
 // epilogue to have read the accumulators (acc_full, one phase per segment). Bounded waits,
 // abort and drain, split-K through clusters or tickets and the fused store_cache are as
@@ -815,13 +856,6 @@ constexpr int kRT = 2;                  // 128-row tiles per CTA
 // 4-11 dequantisation and the epilogue. One CTA per SM, so a thread may hold up to 168
 // registers (the epilogue with the fused store_cache needs about 140).
 constexpr int kThreads2 = 384;
-// MMA issuing threads: 2 (warp 2 tile 0, warp 3 tile 1) or 1 (warp 2 both tiles, one
-// commit per unit); a build constant, chosen by measurement.
-#ifndef FLEXQ_TC2_ISSUERS
-#define FLEXQ_TC2_ISSUERS 2
-#endif
-constexpr int kIssuers2 = FLEXQ_TC2_ISSUERS;
-static_assert(kIssuers2 == 1 || kIssuers2 == 2, "one or two issuers");
 constexpr int kRows2 = kRT * kBM;       // 256
 constexpr int kDoneRing2 = 16;          // mma_done barriers (units)
 constexpr int kMaxPieces = 8;           // stream-K: later pieces of one tile that its owner adds
@@ -909,9 +943,11 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
     B.codes_full = sb;
     B.codes_empty = B.codes_full + 8 * NSC;
     B.x_full = B.codes_empty + 8 * NSC;
+    // per tile: a_full of (slot s, tile t) at a_full + 8 (2 s + t); mma_done of (unit u, tile t)
+    // at mma_done + 8 (2 (u % kDoneRing2) + t)
     B.a_full = B.x_full + 8 * NSX;
-    B.mma_done = B.a_full + 8 * NSLOT;
-    B.acc_full = B.mma_done + 8 * kDoneRing2;     // here: the accumulators are free again (one phase per segment)
+    B.mma_done = B.a_full + 8 * kRT * NSLOT;
+    B.acc_full = B.mma_done + 8 * kRT * kDoneRing2;   // here: the accumulators are free again (one phase per segment)
     B.drain = B.acc_full + 8;
     B.red = B.drain + 8 * 4;
     const uint32_t misc = B.red + 8 * 2;
@@ -926,8 +962,8 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
             tc::bar_init(B.codes_empty + 8 * s, kDequantThreads);
         }
         for (int s = 0; s < NSX; ++s) tc::bar_init(B.x_full + 8 * s, 1);
-        for (int s = 0; s < NSLOT; ++s) tc::bar_init(B.a_full + 8 * s, kDequantThreads);
-        for (int s = 0; s < kDoneRing2; ++s) tc::bar_init(B.mma_done + 8 * s, kIssuers2);   // every issuer commits each unit
+        for (int s = 0; s < kRT * NSLOT; ++s) tc::bar_init(B.a_full + 8 * s, kDequantThreads / kRT);   // a tile's 4 warps
+        for (int s = 0; s < kRT * kDoneRing2; ++s) tc::bar_init(B.mma_done + 8 * s, 1);   // the tile's issuer
         tc::bar_init(B.acc_full, kDequantThreads);
         for (int i = 0; i < 4; ++i) tc::bar_init(B.drain + 8 * i, 1);
         tc::bar_init(B.red, 1);
@@ -1001,10 +1037,13 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
                 const int m0 = sg.tm * p.BN;
                 for (int xi = sg.k0 * KU / XU; xi < sg.k1 * KU / XU; ++xi) {
                     if (gx >= NSX) {
-                        // the slot last held units [(gx - NSX) XU, +XU): wait for the MMAs of its last unit
+                        // the slot last held units [(gx - NSX) XU, +XU): wait for the MMAs of its
+                        // last unit, both tiles
                         const int ul = (gx - NSX) * XU + XU - 1;
-                        if (!tc::bar_wait(B.mma_done + 8 * (ul % kDoneRing2), (ul / kDoneRing2) & 1, abort, p.status,
-                                          p.wait_ns)) {
+                        const uint32_t md = B.mma_done + 8 * (kRT * (ul % kDoneRing2));
+                        const uint32_t par = (ul / kDoneRing2) & 1;
+                        if (!tc::bar_wait(md, par, abort, p.status, p.wait_ns) ||
+                            !tc::bar_wait(md + 8, par, abort, p.status, p.wait_ns)) {
                             go = false;
                             break;
                         }
@@ -1024,9 +1063,11 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
         }
         __syncwarp();
     } else if (warp == 2 || warp == 3) {
-        // ---------------- MMA issuers: warp 2 tile 0, warp 3 tile 1 (or warp 2 both) ----------------
+        // ---------------- MMA issuers: warp 2 tile 0, warp 3 tile 1 ----------------
+        // Each issuer waits only for its own tile's A slot and commits to its own tile's
+        // mma_done ring, so the two tiles' pipelines need not wait for each other.
         const int t = warp - 2;
-        if (lane == 0 && t < kIssuers2) {
+        if (lane == 0) {
             const uint32_t idesc = tc::idesc_f16_f32(kBM, p.BN);
             const uint32_t d_acc = tmem + static_cast<uint32_t>(t * p.acc_stride);
             int xs = 0, xc = 0;                 // activation stage and chunk within it
@@ -1046,19 +1087,20 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
                 }
                 const int nu = (sg.k1 - sg.k0) * KU;
                 for (int u = 0; u < nu; ++u) {
-                    if (!tc::bar_wait(B.a_full + 8 * sa, aph, abort, p.status, p.wait_ns)) { ok = false; break; }
+                    if (!tc::bar_wait(B.a_full + 8 * (kRT * sa + t), aph, abort, p.status, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
                     if (xc == 0 && !tc::bar_wait(B.x_full + 8 * xs, xph, abort, p.status, p.wait_ns)) { ok = false; break; }
                     tc::fence_after_sync();
                     const uint32_t a_tm = tmem + static_cast<uint32_t>(p.a_col0 + (sa * kRT + t) * 32);
                     const uint64_t bd = tc::desc_k_sw128(sX + static_cast<uint32_t>(xs * XU + xc) * xbytes);
                     issue_ksteps<1>(d_acc, a_tm, bd, idesc, 0, u == 0);
-                    if (kIssuers2 == 1)                 // tile 1 too, same activation stage
-                        issue_ksteps<1>(tmem + static_cast<uint32_t>(p.acc_stride), a_tm + 32, bd, idesc, 0, u == 0);
                     if (++xc == XU) {
                         xc = 0;
                         if (++xs == NSX) { xs = 0; xph ^= 1; }
                     }
-                    tc::mma_commit(B.mma_done + 8 * (g % kDoneRing2));
+                    tc::mma_commit(B.mma_done + 8 * (kRT * (g % kDoneRing2) + t));
                     ++g;
                     if (++sa == NSLOT) { sa = 0; aph ^= 1; }
                 }
@@ -1071,7 +1113,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
             }
             // every commit arrival lands before the CTA exits
             for (int c = g - kDoneRing2 > 0 ? g - kDoneRing2 : 0; c < g; ++c)
-                tc::bar_wait(B.mma_done + 8 * (c % kDoneRing2), (c / kDoneRing2) & 1, &never, p.status);
+                tc::bar_wait(B.mma_done + 8 * (kRT * (c % kDoneRing2) + t), (c / kDoneRing2) & 1, &never, p.status);
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 12) {
@@ -1100,6 +1142,13 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
                     for (int v = 0; v < WPC; ++v) cw[c][v] = tc::lds128(crow + (((c * WPC + v) ^ sw) << 4));
                 const uint4 mrow = tc::lds128(sM + s * MSTAGE + row * 16);
                 const int moff = (st * KU) & (kMetaChunks - 1);
+                // the step's groups, decoded together before the first unit
+                DqConst kc[KU];
+#pragma unroll
+                for (int c = 0; c < KU; ++c) {
+                    const int mi = (moff + c) & 3;
+                    kc[c] = dq_const(mi == 0 ? mrow.x : (mi == 1 ? mrow.y : (mi == 2 ? mrow.z : mrow.w)));
+                }
 #pragma unroll
                 for (int c = 0; c < KU; ++c) {
                     const int u = g;
@@ -1107,32 +1156,27 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
                     if (++dq_slot == NSLOT) dq_slot = 0;
                     if (u >= NSLOT) {
                         const int pu = u - NSLOT;
-                        if (!tc::bar_wait(B.mma_done + 8 * (pu % kDoneRing2), (pu / kDoneRing2) & 1, abort, p.status,
-                                          p.wait_ns)) {
+                        if (!tc::bar_wait(B.mma_done + 8 * (kRT * (pu % kDoneRing2) + tt), (pu / kDoneRing2) & 1,
+                                          abort, p.status, p.wait_ns)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after_sync();
                     }
-                    const int mi = (moff + c) & 3;
-                    const uint32_t mw = mi == 0 ? mrow.x : (mi == 1 ? mrow.y : (mi == 2 ? mrow.z : mrow.w));
-                    const __half mn = __ushort_as_half(static_cast<unsigned short>(mw & 0xFFFFu));
-                    const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mw >> 16)));
-                    const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
-                    const __half2 s2h = __half2half2(step), m2h = __half2half2(mn);
-                    const uint32_t step2 = *reinterpret_cast<const uint32_t*>(&s2h);
-                    const uint32_t mnv2 = *reinterpret_cast<const uint32_t*>(&m2h);
+                    const uint32_t step2 = kc[c].step2, mnv2 = kc[c].mn2;
                     const uint32_t a_col = p.a_col0 + (sa * kRT + tt) * 32;
+                    // the whole chunk (64 values, 32 columns) goes to TMEM in one store: a
+                    // tcgen05.st costs about as much issue time as two of half the width
+                    uint32_t r32[32];
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {          // two halves of the chunk: 32 values each
-                        uint32_t r[16];
+                        uint32_t (&r)[16] = *reinterpret_cast<uint32_t (*)[16]>(&r32[16 * hh]);
                         if (BITS == 4) {
                             const uint4 q = cw[c][hh];
                             const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
-                                const uint4 v = XPERM ? dequant8_4bit_il(w[j], step2, mnv2)
-                                                      : dequant8_4bit(w[j], step2, mnv2);
+                                const uint4 v = XPERM ? dequant8_4bit_il(w[j], kc[c]) : dequant8_4bit(w[j], kc[c]);
                                 r[4 * j] = v.x;
                                 r[4 * j + 1] = v.y;
                                 r[4 * j + 2] = v.z;
@@ -1157,11 +1201,11 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
                                 r[4 * j + 3] = v.w;
                             }
                         }
-                        tc::tmem_st16(t_lane + a_col + hh * 16, r);
                     }
+                    tc::tmem_st32(t_lane + a_col, r32);
                     tc::tmem_wait_st();
                     tc::fence_before_sync();
-                    tc::bar_arrive(B.a_full + 8 * sa);
+                    tc::bar_arrive(B.a_full + 8 * (kRT * sa + tt));
                     ++g;
                 }
                 if (!ok) break;
@@ -1204,7 +1248,9 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_tc2_kernel(const __grid_con
             asm volatile("bar.sync 1, 256;" ::: "memory");
             if (ok && !*abort && g > 0) {
                 const int gl = g - 1;                                 // the segment's last unit: both tiles' MMAs done
-                ok = tc::bar_wait(B.mma_done + 8 * (gl % kDoneRing2), (gl / kDoneRing2) & 1, abort, p.status);
+                const uint32_t md = B.mma_done + 8 * (kRT * (gl % kDoneRing2));
+                ok = tc::bar_wait(md, (gl / kDoneRing2) & 1, abort, p.status) &&
+                     tc::bar_wait(md + 8, (gl / kDoneRing2) & 1, abort, p.status);
             }
             asm volatile(
                 "{\n\t.reg .pred p, q;\n\t"
@@ -1897,7 +1943,8 @@ __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm) gemv_kernel(const Ge
         }
         gv_commit();
         const uint32_t st = sbase + (i % kGvStages) * STAGE;
-        uint32_t wa[kGvMt][kGvWords], wb[kGvMt][kGvWords], s2[kGvMt][2], m2[kGvMt][2];
+        uint32_t wa[kGvMt][kGvWords], wb[kGvMt][kGvWords];
+        DqConst kd[kGvMt][2];
 #pragma unroll
         for (int mt = 0; mt < kGvMt; ++mt) {
             const int ra_row = r0 + 16 * mt;
@@ -1916,16 +1963,8 @@ __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm) gemv_kernel(const Ge
             }
             if (kGvWords == 1) { wa[mt][0] = lds32(ra); wb[mt][0] = lds32(rbb); }
             const uint32_t mw0 = lds32(st + CODES + ra_row * 16 + t * 4), mw1 = lds32(st + CODES + (ra_row + 8) * 16 + t * 4);
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const uint32_t mwr = r ? mw1 : mw0;
-                const __half mn = __ushort_as_half(static_cast<unsigned short>(mwr & 0xFFFFu));
-                const float sc32 = __half2float(__ushort_as_half(static_cast<unsigned short>(mwr >> 16)));
-                const __half step = __float2half_rn(sc32 > 0.f ? rcp_approx(sc32) : 0.f);
-                const __half2 sh = __half2half2(step), mh = __half2half2(mn);
-                s2[mt][r] = *reinterpret_cast<const uint32_t*>(&sh);
-                m2[mt][r] = *reinterpret_cast<const uint32_t*>(&mh);
-            }
+            kd[mt][0] = dq_const(mw0);
+            kd[mt][1] = dq_const(mw1);
         }
         const uint32_t xs = st + CODES + META + (g * 4 + t) * XSEG + kq * kGvWords * 16;
 #pragma unroll
@@ -1934,8 +1973,8 @@ __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm) gemv_kernel(const Ge
             uint4 d0[kGvMt], d1[kGvMt];
 #pragma unroll
             for (int mt = 0; mt < kGvMt; ++mt) {
-                d0[mt] = dequant8_4bit_il(wa[mt][w], s2[mt][0], m2[mt][0]);    // row r0 + 16 mt
-                d1[mt] = dequant8_4bit_il(wb[mt][w], s2[mt][1], m2[mt][1]);    // row r0 + 16 mt + 8
+                d0[mt] = dequant8_4bit_il(wa[mt][w], kd[mt][0]);    // row r0 + 16 mt
+                d1[mt] = dequant8_4bit_il(wb[mt][w], kd[mt][1]);    // row r0 + 16 mt + 8
             }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -2207,7 +2246,7 @@ Plan2 make_plan2(int M, int N, int K, int bits) {
     P.off_c = nsx * xstage;
     P.off_m = P.off_c + nsc * kRows2 * 128;
     P.off_bar = P.off_m + nsc * kRows2 * kMetaChunks * 4;
-    P.smem = P.off_bar + 8 * (2 * nsc + nsx + P.nslot + kDoneRing2 + 1 + 4 + 2) + 16 + 256 + 1024;
+    P.smem = P.off_bar + 8 * (2 * nsc + nsx + kRT * P.nslot + kRT * kDoneRing2 + 1 + 4 + 2) + 16 + 256 + 1024;
     // split-K through distributed shared memory when the partial tile fits in the drained
     // rings and every tile's cluster can be resident at once, else workspace and tickets
     const bool fits = static_cast<uint32_t>(P.BN) * kRows2 * 4 <= P.off_bar;

@@ -166,14 +166,18 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decompress_contig_kernel
 // Rows per slice: 8, or 16 for groups of 128 rows, so that a slice still spans at most 8
 // lanes and a warp reads at least 64 contiguous bytes of every row (with 8 rows per slice
 // a 128-row group took 16 lanes and left 32-byte row pieces: about 1.3-2.3 TB/s).
-constexpr int strided_rps(int gs) { return gs >= 128 ? 16 : 8; }
+// 8-bit codes take 16 rows per slice at every group size: with 8 (and a register budget for
+// 4 blocks per SM) the kernel spilled and fell from 5.0 to 2.9 TB/s between 1 and 4 GiB
+// tensors at g64; with 16 rows per slice (and 2 blocks per SM) it holds 5.1-5.6 TB/s.
+template <int BITS>
+constexpr int strided_rps(int gs) { return (gs >= 128 || BITS == 8) ? 16 : 8; }
 
 template <int BITS, int GS>
-__global__ void __launch_bounds__(kThreads, GS >= 128 ? 2 : kMinBlocks) compress_strided_1pass_kernel(const __half* __restrict__ x,
+__global__ void __launch_bounds__(kThreads, (GS >= 128 || BITS == 8) ? 2 : kMinBlocks) compress_strided_1pass_kernel(const __half* __restrict__ x,
                                                                           uint8_t* __restrict__ codes,
                                                                           uint32_t* __restrict__ meta, int64_t outer,
                                                                           int64_t ng, int64_t inner) {
-    constexpr int RPS = strided_rps(GS);       // rows per slice
+    constexpr int RPS = strided_rps<BITS>(GS);       // rows per slice
     constexpr int NS = GS / RPS;               // slices (lanes) per item
     constexpr int IPW = 32 / NS;               // items per warp
     constexpr int CB = GS * BITS / 8;          // code rows per group
@@ -588,9 +592,9 @@ int launch_compress(const Geometry& g, const __half* x, uint8_t* codes, uint32_t
     } else {
         const bool vec = (g.inner % 8 == 0);
         const int64_t items = g.outer * g.ng * (vec ? g.inner / 8 : g.inner);
-        if (vec)   // GS / strided_rps(GS) lanes per item
+        if (vec)   // GS / strided_rps<BITS>(GS) lanes per item
             compress_strided_1pass_kernel<BITS, GS>
-                <<<grid_for<compress_strided_1pass_kernel<BITS, GS>>(items * (GS / strided_rps(GS))), kThreads, 0, st>>>(
+                <<<grid_for<compress_strided_1pass_kernel<BITS, GS>>(items * (GS / strided_rps<BITS>(GS))), kThreads, 0, st>>>(
                     x, codes, meta, g.outer, g.ng, g.inner);
         else
             compress_strided_kernel<BITS, GS>

@@ -319,11 +319,13 @@ class Stack:
         self.torch.cuda.empty_cache()
 
 
-def build_decode_graphs(fq, torch, stack, stream, inputs, y_out, positions):
+def build_decode_graphs(fq, torch, stack, stream, inputs, y_outs, positions):
     """One CUDA graph per position: all sequences through every layer, chained through
     two activation buffers. With several gpu-batches (the pages' gpu_batch_size x
     num_gpu_batches block) each layer is one flex_decode_layer_batches call, so its
-    weights are streamed once for all gpu-batches. inputs [T][batch][h], y_out [batch][h]."""
+    weights are streamed once for all gpu-batches. inputs [T][batch][h]; the graph of
+    position t writes its output to y_outs[t % len(y_outs)] ([batch][h] each), so that a
+    copy of one token's output can run while the next token computes."""
     cfg = stack.cfg
     L, b, calls = cfg["layers"], cfg["call_batch"], cfg["calls"]
     bufs = [torch.empty((calls * b, cfg["h"]), dtype=torch.float16, device=stack.dev) for _ in range(2)]
@@ -331,7 +333,7 @@ def build_decode_graphs(fq, torch, stack, stream, inputs, y_out, positions):
     def token(t, pos):
         src = inputs[t]
         for l in range(L):
-            dst = y_out if l == L - 1 else bufs[l % 2]
+            dst = y_outs[t % len(y_outs)] if l == L - 1 else bufs[l % 2]
             if calls == 1:
                 fq.flex_decode_layer(stack.layers[l], stack.caches[l][0], src, dst, b, pos, stack.ws_dec)
             else:
@@ -381,9 +383,9 @@ def run_flexq(args):
 
     stream = torch.cuda.Stream(device=dev)
     inputs = torch.stack([synth.decode_inputs(b, h, t, cfg["seed"], device=dev) for t in range(nsteps)])
-    y_out = torch.empty((b, h), dtype=torch.float16, device=dev)
+    y_outs = [torch.empty((b, h), dtype=torch.float16, device=dev) for _ in range(2)]
     positions = [s + t for t in range(nsteps)]
-    graphs, _bufs = build_decode_graphs(fq, torch, stack, stream, inputs, y_out, positions)
+    graphs, _bufs = build_decode_graphs(fq, torch, stack, stream, inputs, y_outs, positions)
 
     # kernels per decode phase, read back from the captured graphs
     launch_counts = {}
@@ -436,16 +438,43 @@ def run_flexq(args):
     t_end = time.time()
     value = whole_job_value(world, units_per_step, args.steps, ms)
 
-    # ---- end to end: per step H2D of the step's inputs from pinned memory, graphs,
-    #      D2H of the step's result
+    # ---- end to end: every token's inputs copied from pinned host memory and its output
+    #      copied back, inside the timed region. The copies run on their own stream:
+    #      token t + 1's inputs while token t computes, token t's output while token t + 1
+    #      computes (outputs alternate between two buffers). Each graph waits for its
+    #      inputs, and a graph reuses an output buffer only once its earlier copy is done.
     host_in = inputs.cpu().pin_memory()
     host_out = torch.empty((nsteps, b, h), dtype=torch.float16).pin_memory()
+    copy_stream = torch.cuda.Stream(device=dev)
+    T = len(graphs)
 
     def e2e_phase():
+        ev_in = [torch.cuda.Event() for _ in range(T)]
+        ev_out = [torch.cuda.Event() for _ in range(T)]
+        start = torch.cuda.Event()
+        start.record(stream)                       # every earlier graph has finished here
+        copy_stream.wait_event(start)
+        with torch.cuda.stream(copy_stream):
+            inputs[0].copy_(host_in[0], non_blocking=True)
+            ev_in[0].record(copy_stream)
         for t, g in enumerate(graphs):
-            inputs[t].copy_(host_in[t], non_blocking=True)
+            stream.wait_event(ev_in[t])
+            if t >= 2:
+                stream.wait_event(ev_out[t - 2])   # y_outs[t % 2] has been copied out
+            ev_run = torch.cuda.Event()
+            ev_run.record(stream)                  # graph t - 1, the last reader of inputs[t + 1] before, is done
             g.replay()
-            host_out[t].copy_(y_out, non_blocking=True)
+            ev_done = torch.cuda.Event()
+            ev_done.record(stream)
+            with torch.cuda.stream(copy_stream):
+                if t + 1 < T:
+                    copy_stream.wait_event(ev_run)
+                    inputs[t + 1].copy_(host_in[t + 1], non_blocking=True)
+                    ev_in[t + 1].record(copy_stream)
+                copy_stream.wait_event(ev_done)
+                host_out[t].copy_(y_outs[t % 2], non_blocking=True)
+                ev_out[t].record(copy_stream)
+        stream.wait_event(ev_out[T - 1])           # the timed region ends after the last copy
 
     for _ in range(2):
         with torch.cuda.stream(stream):
@@ -459,7 +488,7 @@ def run_flexq(args):
     rc = fq.flex_get_status()
     if rc != 0:
         raise RuntimeError(f"timed region failed: {fq.flex_status_string(rc)}")
-    assert bool(torch.isfinite(y_out).all())
+    assert all(bool(torch.isfinite(y).all()) for y in y_outs)
     del graphs
 
     # ---- bounds of the step (summed over its positions and layers)
@@ -783,7 +812,7 @@ def measure_secondary_decode(fq, torch, synth, name, peaks, dev, ntok=8, reps=5)
     inputs = torch.stack([synth.decode_inputs(b, h, t, cfg["seed"], device=dev) for t in range(ntok)])
     y_out = torch.empty((b, h), dtype=torch.float16, device=dev)
     positions = [s + t for t in range(ntok)]
-    graphs, _ = build_decode_graphs(fq, torch, stack, stream, inputs, y_out, positions)
+    graphs, _ = build_decode_graphs(fq, torch, stack, stream, inputs, [y_out], positions)
     with torch.cuda.stream(stream):
         for g in graphs:
             g.replay()

@@ -717,6 +717,43 @@ def measure_parts(fq, torch, synth, cfg, stack, stream, peaks, dev):
                                                        h, stream=stream))
     kern["layernorm"] = dict(ms=ms, bytes=2 * b * h * 2 + 2 * h * 2, flops=0.0, launches_per_call=2,
                              kernel=main_kernel(names, "layernorm_kernel"), kernels=names, source=["kv_ln.cu"])
+    # left padding (valid_from): sequence i starts at key (i % 4) * 128, so its first keys
+    # are neither read nor attended (the same kernel, fewer keys)
+    vf = torch.clamp((torch.arange(b, device=dev, dtype=torch.int32) % 4) * 128, max=pos)
+    for c in caches:
+        c.valid_from = vf
+    ms, names = time_cycle(lambda l: fq.flex_decode_attention(caches[l], x[:, :h], x[:, h:], x[:, 2 * h:], 3 * h, o,
+                                                              b, pos, aws, stream=stream))
+    for c in caches:
+        c.valid_from = None
+    kept = float(torch.clamp(pos - vf, min=0).sum().item())
+    kern["decode_attention_padded"] = dict(
+        ms=ms, bytes=2 * kept * h * per + 3 * b * h * 2 + b * h * 2, flops=4.0 * (kept + b) * h,
+        launches_per_call=int(round(sum(names.values()))) if names else 1, kernels=names, source=["attention.cu"],
+        note="left-padded batch: sequence i skips its first (i % 4) * 128 keys; bytes count the keys read")
+    # the model around the layers: input embedding of the next tokens, then the output head
+    # (final LayerNorm, logits over the 4-bit token table, greedy choice) - OPT vocabulary
+    vocab = synth.OPT_VOCAB
+    vpad = (vocab + 255) // 256 * 256
+    mp = synth.model_params(vocab, h, 2048, cfg["seed"], vpad, device=dev)
+    E = fq.CompressedWeight(mp.pop("E"))
+    tok = synth.token_ids((b,), vocab, 7, device=dev)
+    tpos = torch.full((b,), pos, dtype=torch.int32, device=dev)
+    xe = torch.empty((b, h), dtype=torch.float16, device=dev)
+    ids = torch.empty(b, dtype=torch.int32, device=dev)
+    hws = torch.zeros(max(16, fq.flex_lm_head_ws_bytes(E, vocab, b)), dtype=torch.uint8, device=dev)
+
+    def model_io(_l):
+        fq.flex_embed(E, vocab, mp["P"], tok, tpos, xe, stream=stream)
+        fq.flex_lm_head_argmax(E, vocab, mp["lnf_g"], mp["lnf_b"], xe, hws, ids, stream=stream)
+    ms, names = time_cycle(model_io)
+    kern["embed_and_head"] = dict(
+        ms=ms, bytes=vpad * h * per + b * h * (per + 2 + 2) + 3 * b * h * 2 + b * vpad * 2 * 2,
+        flops=2.0 * b * vpad * h, launches_per_call=int(round(sum(names.values()))) if names else 4, kernels=names,
+        source=["model.cu", "gemm.cu"],
+        note="flex_embed of the next tokens + flex_lm_head_argmax (final LayerNorm, logits over the 4-bit token "
+             "table, greedy id) for the whole batch; not part of the layer step")
+    del E, mp, hws
     # the whole layer call in the same regime (a graph of one call per layer, replayed):
     # against the sum of its kernels' parts it shows what the kernel boundaries cost
     xl = synth.decode_inputs(b * calls, h, 0, cfg["seed"], device=dev)

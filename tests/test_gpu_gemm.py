@@ -279,3 +279,19 @@ def test_gemm_split_reduction_paths(streamk):
             assert err <= 1e-2 * full.abs().max().item() + 1e-3, (path, err)
     finally:
         fq.flex_set_gemm_streamk(old)
+
+
+@pytest.mark.parametrize("M,N,K", [(4, 256, 512), (32, 512, 2048)])
+def test_small_batches_on_the_tensor_core_gemm(M, N, K):
+    """flex_set_gemm_gemv(False) sends batches of up to 32 rows to the 128-row tcgen05
+    GEMM (the comparison the route switch exists for); it must give the same result
+    within the tolerance, and the default route comes back afterwards."""
+    assert fq.flex_gemm_plan(M, N, K)["kernel"] == "gemv"
+    old = fq.flex_set_gemm_gemv(False)
+    try:
+        assert fq.flex_gemm_plan(M, N, K)["kernel"] == "tc128"
+        x, w, b, _, y, _ = _run(M, N, K, fq.FLEX_EPI_NONE, seed=M + 31)
+    finally:
+        fq.flex_set_gemm_gemv(old)
+    assert fq.flex_gemm_plan(M, N, K)["kernel"] == "gemv"
+    assert_layer_close(y, _oracle_gemm(x, w, b, None, fq.FLEX_EPI_NONE, 4), f"tc128 {M}x{N}x{K}")

@@ -582,6 +582,11 @@ def codec_sweep_points():
                 for gs in (32, 64, 128):
                     pts.append(((rows, 4096), gd, bits, gs))
     pts.append(((544, 144 * 96, 128), 2, 4, 64))         # KV-shaped: [tokens][seq x heads][head_dim]
+    # codec variants (the generic kernels), 1 GiB: 3-bit codes, the symmetric form, and a
+    # group dimension that is not a multiple of the group size (last group padded)
+    rows = 1024 * (1 << 20) // (2 * 4096)
+    pts += [((rows, 4096), 1, 3, 64, 0), ((rows, 4096), 1, 4, 64, 1), ((rows, 4096), 1, 8, 64, 1),
+            ((rows, 4000), 1, 4, 64, 0)]
     return pts
 
 
@@ -592,15 +597,21 @@ def measure_codec(fq, torch, synth, dev, hbm, points):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     out = {}
-    for shape, gd, bits, gs in points:
-        xt = synth.codec_tensor(shape, gd, gs, 9, device=dev)
-        cfgq = fq.config(bits, gs, gd)
+    for shape, gd, bits, gs, *rest in points:
+        sym = rest[0] if rest else 0
+        if shape[gd] % gs:                     # partial last group: a slice of a whole-group tensor
+            full = list(shape)
+            full[gd] = (shape[gd] + gs - 1) // gs * gs
+            xt = synth.codec_tensor(tuple(full), gd, gs, 9, device=dev).narrow(gd, 0, shape[gd]).contiguous()
+        else:
+            xt = synth.codec_tensor(shape, gd, gs, 9, device=dev)
+        cfgq = fq.config(bits, gs, gd, sym)
         codes, meta = fq.flexq_compress(xt, cfgq)
         yt = fq.flexq_decompress(codes, meta, shape, cfgq)
         n = xt.numel()
-        nbytes = n * 2 + n * bits // 8 + n // gs * 4
+        nbytes = n * 2 + codes.numel() + meta.numel() * meta.element_size()
         layout = {1: "contiguous", 0: "strided"}.get(gd, f"dim{gd}") if len(shape) == 2 else f"kv-dim{gd}"
-        key = f"{'x'.join(map(str, shape))}_{layout}_{bits}bit_g{gs}"
+        key = f"{'x'.join(map(str, shape))}_{layout}_{bits}bit_g{gs}" + ("_symmetric" if sym else "")
         entry = {"mb": round(n * 2 / (1 << 20)), "bytes": nbytes}
         for opname, fn in (("compress", lambda: fq.flexq_compress(xt, cfgq, codes, meta)),
                            ("decompress", lambda: fq.flexq_decompress(codes, meta, shape, cfgq, yt))):

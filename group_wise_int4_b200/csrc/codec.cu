@@ -511,6 +511,300 @@ __global__ void __launch_bounds__(kThreads) decompress_generic_kernel(const uint
 }
 
 // ---------------------------------------------------------------------------------
+// Codec variants on contiguous groups (group_dim the last one, its extent G a multiple of
+// 8): the layout of the main contiguous kernels - gs/8 lanes per group, 8 values per
+// lane from one 16-byte load - with the variants' arithmetic, bit for bit that of the
+// one-thread-per-group kernels above. A lane whose 8 values lie past G (the padding of a
+// partial last group; G % 8 == 0, so a lane is wholly in or out) takes zeros, which count
+// in min/max and max|x|, and its codes are stored like any other. 3-bit codes: the 8 of
+// a lane are bits [24 l, 24 l + 24) of its group's little-endian stream, i.e. 3 whole
+// bytes at byte 3 l.
+template <int BITS, int SYM>
+__device__ __forceinline__ uint32_t var_quant8(uint4 v, float mn, float s) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t q[8];
+    if (SYM) {
+        // q = rint(fl(x * s)) in [-B, B] (|x * s| <= B (1 + 2^-10) < B + 0.5 by the
+        // choice of s), stored as q + B; a NaN product gives q = 0 like the conversion
+        constexpr int B = (1 << (BITS - 1)) - 1;
+        const uint64_t s2 = f2_pack(s, s);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float a, b;
+            f2_unpack(f2_mul(f2_pack(h2f_lo(w[k]), h2f_hi(w[k])), s2), a, b);
+            a = (a == a) ? a : 0.0f;
+            b = (b == b) ? b : 0.0f;
+            f2_unpack(f2_add(f2_pack(a, b), f2_pack(12582912.0f, 12582912.0f)), a, b);
+            q[2 * k] = (__float_as_uint(a) + B) & ((1u << BITS) - 1u);
+            q[2 * k + 1] = (__float_as_uint(b) + B) & ((1u << BITS) - 1u);
+        }
+    } else {
+        const uint64_t mn2 = f2_pack(mn, mn), s2 = f2_pack(s, s);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            quant_bits_pair(w[k], mn2, s2, q[2 * k], q[2 * k + 1]);
+            q[2 * k] &= (1u << BITS) - 1u;
+            q[2 * k + 1] &= (1u << BITS) - 1u;
+        }
+    }
+    uint32_t u = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) u |= q[k] << (BITS * k);     // BITS <= 4: fits 32 bits
+    return u;
+}
+
+// Division of a group index by the groups per row, ng, fixed for a launch: Granlund and
+// Montgomery's unsigned division by a run-time invariant integer ("Division by Invariant
+// Integers using Multiplication", 1994, figure 4.1). With l = ceil(log2 ng) and
+// m = floor(2^32 (2^l - ng) / ng) + 1, every 32-bit n gives
+//   n / ng = (t + ((n - t) >> 1)) >> (l - 1),  t = umulhi(m, n)   (ng >= 2).
+struct DivU32 {
+    uint32_t m = 0;
+    int l = 0;                                 // 0: ng == 1
+};
+inline DivU32 make_div(int64_t ng) {
+    DivU32 d;
+    if (ng < 2 || ng >= 0x7FFFFFFF) return d;
+    const uint32_t dv = static_cast<uint32_t>(ng);
+    int l = 0;
+    while ((1ull << l) < dv) ++l;
+    d.l = l;
+    d.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << l) - dv)) / dv + 1);
+    return d;
+}
+__device__ __forceinline__ uint32_t div_u32(uint32_t n, const DivU32& d) {
+    const uint32_t t = __umulhi(d.m, n);
+    return (t + ((n - t) >> 1)) >> (d.l - 1);
+}
+
+// Address of lane `sub` of group q: flat when every group is whole (ng GS == G), else
+// through the row (a partial last group leaves a gap of padding in the group index).
+template <int GS>
+__device__ __forceinline__ int64_t var_col(int64_t q, int sub, int64_t G, int64_t ng, bool whole, const DivU32& dv,
+                                           bool& ok) {
+    if (whole) {
+        ok = true;
+        return q * GS + sub * 8;
+    }
+    const int64_t o = ng == 1 ? q
+                      : (dv.l > 0 && q < 0x7FFFFFFF) ? static_cast<int64_t>(div_u32(static_cast<uint32_t>(q), dv))
+                                                     : q / ng;
+    const int64_t gi = q - o * ng, col = gi * GS + sub * 8;
+    ok = col < G;
+    return o * G + col;
+}
+
+template <int BITS, int GS, int SYM>
+__global__ void __launch_bounds__(kThreads) compress_var_contig_kernel(const __half* __restrict__ x,
+                                                                        uint8_t* __restrict__ codes,
+                                                                        uint32_t* __restrict__ meta, int64_t rows,
+                                                                        int64_t G, int64_t ng, DivU32 dv) {
+    constexpr int L = GS / 8;                  // lanes per group
+    constexpr int GPW = 32 / L;                // groups per warp and step
+    constexpr int CB = GS * BITS / 8;          // code bytes per group
+    const int lane = threadIdx.x & 31, sub = lane % L;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+    const int64_t total = rows * ng;
+    const bool whole = ng * GS == G;
+    auto load = [&](int64_t base) {
+        const int64_t q = base + lane / L;
+        bool ok = false;
+        const int64_t at = q < total ? var_col<GS>(q, sub, G, ng, whole, dv, ok) : 0;
+        return (q < total && ok) ? ld_stream_v4(x + at) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    // software pipelined: the next step's vector is requested before this one is quantised
+    int64_t base = warp * GPW;
+    uint4 v = load(base);
+    while (base < total) {
+        const int64_t next = base + nwarps * GPW;
+        const uint4 nv = load(next);
+        const int64_t q = base + lane / L;
+        float mn = 0.0f;
+        __half s16 = __ushort_as_half(0);
+        if (SYM) {
+            const __half2* h = reinterpret_cast<const __half2*>(&v);
+            __half2 a2 = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
+#pragma unroll
+            for (int off = 1; off < L; off <<= 1) {
+                const uint32_t o2 = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<const uint32_t*>(&a2), off);
+                a2 = __hmax2(a2, *reinterpret_cast<const __half2*>(&o2));
+            }
+            const float a = fmaxf(__low2float(a2), __high2float(a2));
+            if (a > 0.0f) {
+                s16 = __float2half_rn(__fdiv_rn(static_cast<float>((1 << (BITS - 1)) - 1), a));
+                if (__hisinf(s16)) s16 = __ushort_as_half(0x7BFF);
+            }
+        } else {
+            __half2 hmn, hmx;
+            minmax8(v, hmn, hmx);
+            float mx;
+            group_minmax<L>(hmn, hmx, mn, mx);
+            s16 = group_scale16<BITS>(mn, mx);
+        }
+        if (q < total) {
+            const uint32_t u = var_quant8<BITS, SYM>(v, mn, __half2float(s16));
+            uint8_t* dst = codes + q * CB + sub * BITS;
+            if (BITS == 4) {
+                *reinterpret_cast<uint32_t*>(dst) = u;
+            } else {                           // 3 bytes, little-endian
+                dst[0] = static_cast<uint8_t>(u);
+                dst[1] = static_cast<uint8_t>(u >> 8);
+                dst[2] = static_cast<uint8_t>(u >> 16);
+            }
+            if (sub == 0) meta[q] = pack_half2_bits(SYM ? __ushort_as_half(0) : stored_min16(mn), s16);
+        }
+        v = nv;
+        base = next;
+    }
+}
+
+// 8-bit codes of the contiguous variants (8 code bytes per lane): the symmetric form, or
+// the min/max form of a partial last group.
+template <int GS, int SYM>
+__global__ void __launch_bounds__(kThreads) compress_var8_contig_kernel(const __half* __restrict__ x,
+                                                                         uint8_t* __restrict__ codes,
+                                                                         uint32_t* __restrict__ meta, int64_t rows,
+                                                                         int64_t G, int64_t ng, DivU32 dv) {
+    constexpr int L = GS / 8, GPW = 32 / L, B = 127;
+    const int lane = threadIdx.x & 31, sub = lane % L;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+    const int64_t total = rows * ng;
+    const bool whole = ng * GS == G;
+    for (int64_t base = warp * GPW; base < total; base += nwarps * GPW) {
+        const int64_t q = base + lane / L;
+        const bool okg = q < total;
+        bool okv = false;
+        const int64_t at = okg ? var_col<GS>(q, sub, G, ng, whole, dv, okv) : 0;
+        const uint4 v = (okg && okv) ? ld_stream_v4(x + at) : make_uint4(0u, 0u, 0u, 0u);
+        float mn = 0.0f;
+        __half s16 = __ushort_as_half(0);
+        if (SYM) {
+            const __half2* h = reinterpret_cast<const __half2*>(&v);
+            __half2 a2 = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
+#pragma unroll
+            for (int off = 1; off < L; off <<= 1) {
+                const uint32_t o2 = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<const uint32_t*>(&a2), off);
+                a2 = __hmax2(a2, *reinterpret_cast<const __half2*>(&o2));
+            }
+            const float a = fmaxf(__low2float(a2), __high2float(a2));
+            if (a > 0.0f) {
+                s16 = __float2half_rn(__fdiv_rn(static_cast<float>(B), a));
+                if (__hisinf(s16)) s16 = __ushort_as_half(0x7BFF);
+            }
+        } else {
+            __half2 hmn, hmx;
+            minmax8(v, hmn, hmx);
+            float mx;
+            group_minmax<L>(hmn, hmx, mn, mx);
+            s16 = group_scale16<8>(mn, mx);
+        }
+        if (!okg) continue;
+        const float s = __half2float(s16);
+        uint2 out;
+        if (SYM) {
+            const uint64_t s2 = f2_pack(s, s);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t b8[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float p0, p1;
+                f2_unpack(f2_mul(f2_pack(h2f_lo(w[k]), h2f_hi(w[k])), s2), p0, p1);
+                p0 = (p0 == p0) ? p0 : 0.0f;
+                p1 = (p1 == p1) ? p1 : 0.0f;
+                f2_unpack(f2_add(f2_pack(p0, p1), f2_pack(12582912.0f, 12582912.0f)), p0, p1);
+                b8[2 * k] = (__float_as_uint(p0) + B) & 0xFFu;
+                b8[2 * k + 1] = (__float_as_uint(p1) + B) & 0xFFu;
+            }
+            out = make_uint2(pack_low_bytes(b8[0], b8[1], b8[2], b8[3]), pack_low_bytes(b8[4], b8[5], b8[6], b8[7]));
+        } else {
+            out = quant8_8bit(v, mn, s);
+        }
+        *reinterpret_cast<uint2*>(codes + q * GS + sub * 8) = out;
+        if (sub == 0) meta[q] = pack_half2_bits(SYM ? __ushort_as_half(0) : stored_min16(mn), s16);
+    }
+}
+
+// Decompression of the contiguous variants: one item = 8 values of one group (BITS bytes
+// of codes in, one 16-byte store out); items past G (padding) write nothing. Four items
+// per thread and step, their codes and metadata requested before any is converted.
+template <int BITS, int GS, int SYM>
+__global__ void __launch_bounds__(kThreads) decompress_var_contig_kernel(const uint8_t* __restrict__ codes,
+                                                                          const uint32_t* __restrict__ meta,
+                                                                          __half* __restrict__ y, int64_t rows,
+                                                                          int64_t G, int64_t ng, DivU32 dv) {
+    constexpr int L = GS / 8;
+    constexpr int CB = GS * BITS / 8;
+    constexpr int B = (1 << (BITS - 1)) - 1;
+    constexpr int U = 4;
+    const int64_t items = rows * ng * L;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
+    const bool whole = ng * GS == G;
+    for (int64_t base = tid; base < items; base += nthreads * U) {
+        uint32_t c0[U], c1[U], mw[U];
+        int64_t at[U];
+        bool ok[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t it = base + u * nthreads;
+            const int64_t q = it / L;                       // L is a power of two
+            const int sub = static_cast<int>(it & (L - 1));
+            ok[u] = false;
+            at[u] = it < items ? var_col<GS>(q, sub, G, ng, whole, dv, ok[u]) : 0;
+            ok[u] = ok[u] && it < items;
+            c0[u] = c1[u] = mw[u] = 0u;
+            if (ok[u]) {
+                const uint8_t* src = codes + q * CB + sub * BITS;
+                if (BITS == 8) {
+                    const uint2 c = __ldg(reinterpret_cast<const uint2*>(src));
+                    c0[u] = c.x;
+                    c1[u] = c.y;
+                } else if (BITS == 4) {
+                    c0[u] = __ldg(reinterpret_cast<const uint32_t*>(src));
+                } else {
+                    c0[u] = static_cast<uint32_t>(__ldg(src)) | (static_cast<uint32_t>(__ldg(src + 1)) << 8) |
+                            (static_cast<uint32_t>(__ldg(src + 2)) << 16);
+                }
+                mw[u] = __ldg(meta + q);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (!ok[u]) continue;
+            const uint32_t m = mw[u];
+            const float step = group_step(__ushort_as_half(static_cast<unsigned short>(m >> 16)));
+            const uint32_t cw[2] = {c0[u], c1[u]};
+            uint32_t out[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                uint32_t q0, q1;
+                if (BITS == 8) {
+                    q0 = (cw[k / 2] >> (16 * (k % 2))) & 0xFFu;
+                    q1 = (cw[k / 2] >> (16 * (k % 2) + 8)) & 0xFFu;
+                } else {
+                    q0 = (cw[0] >> (BITS * 2 * k)) & ((1u << BITS) - 1u);
+                    q1 = (cw[0] >> (BITS * (2 * k + 1))) & ((1u << BITS) - 1u);
+                }
+                if (SYM) {
+                    // x^ = fp16(fl((u - B) * step)); an all-zero group (step 0) gives 0
+                    const __half2 hv =
+                        __floats2half2_rn(__fmul_rn(static_cast<float>(static_cast<int>(q0) - B), step),
+                                          __fmul_rn(static_cast<float>(static_cast<int>(q1) - B), step));
+                    out[k] = *reinterpret_cast<const uint32_t*>(&hv);
+                } else if (step == 0.0f) {
+                    out[k] = (m & 0xFFFFu) * 0x10001u;
+                } else {
+                    out[k] = dequant_two(q0, q1, step, h2f_lo(m));
+                }
+            }
+            st_stream_v4(y + at[u], make_uint4(out[0], out[1], out[2], out[3]));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------
 struct Geometry {
     int64_t outer = 1, ng = 0, inner = 1, n = 0, G = 0;
     int gd = 0;
@@ -623,6 +917,54 @@ int launch_decompress(const Geometry& g, const uint8_t* codes, const uint32_t* m
     return launch_status();
 }
 
+// The contiguous-group variants (3-bit, symmetric, partial last group with G % 8 == 0).
+template <int BITS, int GS, int SYM>
+int launch_var(const Geometry& g, const __half* x, uint8_t* codes, uint32_t* meta, const uint8_t* ccodes,
+               const uint32_t* cmeta, __half* y, cudaStream_t st) {
+    const int64_t lanes = g.outer * g.ng * (GS / 8);
+    const DivU32 dv = make_div(g.ng);
+    if (x != nullptr) {
+        if constexpr (BITS == 8) {
+            compress_var8_contig_kernel<GS, SYM>
+                <<<grid_for<compress_var8_contig_kernel<GS, SYM>>(lanes), kThreads, 0, st>>>(x, codes, meta, g.outer,
+                                                                                              g.G, g.ng, dv);
+        } else {
+            compress_var_contig_kernel<BITS, GS, SYM>
+                <<<grid_for<compress_var_contig_kernel<BITS, GS, SYM>>(lanes), kThreads, 0, st>>>(x, codes, meta,
+                                                                                                   g.outer, g.G, g.ng, dv);
+        }
+    } else {
+        decompress_var_contig_kernel<BITS, GS, SYM>
+            <<<grid_for<decompress_var_contig_kernel<BITS, GS, SYM>>(lanes), kThreads, 0, st>>>(ccodes, cmeta, y,
+                                                                                                 g.outer, g.G, g.ng, dv);
+    }
+    return launch_status();
+}
+
+template <int BITS, int SYM>
+int launch_var_gs(const Geometry& g, int gs, const __half* x, uint8_t* codes, uint32_t* meta, const uint8_t* ccodes,
+                  const uint32_t* cmeta, __half* y, cudaStream_t st) {
+    if (gs == 32) return launch_var<BITS, 32, SYM>(g, x, codes, meta, ccodes, cmeta, y, st);
+    if (gs == 64) return launch_var<BITS, 64, SYM>(g, x, codes, meta, ccodes, cmeta, y, st);
+    return launch_var<BITS, 128, SYM>(g, x, codes, meta, ccodes, cmeta, y, st);
+}
+
+// A variant configuration: the contiguous-group kernels when the group dimension is the
+// last one and its extent a multiple of 8, else the one-thread-per-group kernels.
+int launch_variant(const Geometry& g, const flexq_config& cfg, const __half* x, uint8_t* codes, uint32_t* meta,
+                   const uint8_t* ccodes, const uint32_t* cmeta, __half* y, cudaStream_t st) {
+    if (g.inner != 1 || g.G % 8 != 0) return launch_generic(g, cfg, x, codes, meta, ccodes, cmeta, y, st);
+    const int gs = cfg.group_size;
+    if (cfg.symmetric) {
+        if (cfg.num_bits == 3) return launch_var_gs<3, 1>(g, gs, x, codes, meta, ccodes, cmeta, y, st);
+        if (cfg.num_bits == 4) return launch_var_gs<4, 1>(g, gs, x, codes, meta, ccodes, cmeta, y, st);
+        return launch_var_gs<8, 1>(g, gs, x, codes, meta, ccodes, cmeta, y, st);
+    }
+    if (cfg.num_bits == 3) return launch_var_gs<3, 0>(g, gs, x, codes, meta, ccodes, cmeta, y, st);
+    if (cfg.num_bits == 4) return launch_var_gs<4, 0>(g, gs, x, codes, meta, ccodes, cmeta, y, st);
+    return launch_var_gs<8, 0>(g, gs, x, codes, meta, ccodes, cmeta, y, st);
+}
+
 }  // namespace
 }  // namespace flexq
 
@@ -654,7 +996,7 @@ extern "C" int flexq_compress(const void* x, int32_t ndim, const int64_t* shape,
     const __half* xh = static_cast<const __half*>(x);
     uint8_t* c = static_cast<uint8_t*>(codes);
     uint32_t* m = static_cast<uint32_t*>(meta);
-    if (g.generic) return launch_generic(g, cfg, xh, c, m, nullptr, nullptr, nullptr, st);
+    if (g.generic) return launch_variant(g, cfg, xh, c, m, nullptr, nullptr, nullptr, st);
 #define CALL_C(B, S) launch_compress<B, S>(g, xh, c, m, st)
     if (cfg.num_bits == 4) {
         if (cfg.group_size == 32) return CALL_C(4, 32);
@@ -679,7 +1021,7 @@ extern "C" int flexq_decompress(const void* codes, const void* meta, int32_t ndi
     const uint8_t* c = static_cast<const uint8_t*>(codes);
     const uint32_t* m = static_cast<const uint32_t*>(meta);
     __half* yh = static_cast<__half*>(y);
-    if (g.generic) return launch_generic(g, cfg, nullptr, nullptr, nullptr, c, m, yh, st);
+    if (g.generic) return launch_variant(g, cfg, nullptr, nullptr, nullptr, c, m, yh, st);
 #define CALL_D(B, S) launch_decompress<B, S>(g, c, m, yh, st)
     if (cfg.num_bits == 4) {
         if (cfg.group_size == 32) return CALL_D(4, 32);

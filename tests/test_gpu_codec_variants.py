@@ -1,6 +1,9 @@
 """flexq_compress / flexq_decompress for the codec variants - 3-bit codes, the symmetric
 (absmax) form and zero-padded partial groups - bit-exact against the oracle codec on
-contiguous, strided and KV-shaped tensors, small and at 256 MB (sampled)."""
+contiguous, strided and KV-shaped tensors, small and at 256 MB (sampled). Contiguous
+groups whose extent is a multiple of 8 (the last three small shapes, partial last groups
+included, and the 256 MB contiguous cases) take the vectorised variant kernels; the
+other shapes take the one-thread-per-group kernels."""
 import numpy as np
 import pytest
 import torch
@@ -22,7 +25,8 @@ def _run(x, bits, gs, gd, sym):
 
 
 @pytest.mark.parametrize("shape,gd", [((16, 256), 1), ((256, 24), 0), ((3, 100), 1), ((70, 5), 0),
-                                      ((2, 5, 96, 3), 2), ((4, 3, 130), -1)])
+                                      ((2, 5, 96, 3), 2), ((4, 3, 130), -1),
+                                      ((5, 200), 1), ((6, 1000), -1), ((3, 7, 136), 2)])
 @pytest.mark.parametrize("bits,sym", [(3, False), (3, True), (4, True), (8, True), (4, False), (8, False)])
 @pytest.mark.parametrize("gs", [32, 64, 128])
 def test_variants_bit_exact(shape, gd, bits, sym, gs):
@@ -37,7 +41,7 @@ def test_variants_bit_exact(shape, gd, bits, sym, gs):
     assert_bits_equal(y, oc.decompress(rc, rm, x.shape, bits, gs, gd, symmetric=sym), "decompressed")
 
 
-@pytest.mark.parametrize("bits,sym,gd", [(3, False, 1), (4, True, 1), (3, True, 0)])
+@pytest.mark.parametrize("bits,sym,gd", [(3, False, 1), (4, True, 1), (3, True, 0), (8, True, 1), (3, True, 1)])
 def test_variants_256mb_sampled(bits, sym, gd):
     """256 MB fp16 [32768, 4096]: sampled groups equal the oracle's."""
     shape = (32768, 4096)

@@ -10,7 +10,8 @@
 //
 // Two layouts:
 //   contiguous - the group dimension is the last one: the tensor is a flat sequence of
-//                groups; gs/8 lanes share a group and reduce min/max with shuffles.
+//                groups; a group's lanes (one or two vectors each) reduce min/max
+//                with shuffles.
 //   strided    - the group dimension has inner extent `inner` > 1 after it: gs/8
 //                lanes share 8 adjacent columns (one 16-byte vector per row), each
 //                holding 8 of the group's rows in registers; they combine min/max with
@@ -22,10 +23,10 @@ namespace flexq {
 namespace {
 
 constexpr int kThreads = 256;
-// Vectors in flight per thread (compress) and resident blocks per SM the register budget
-// is sized for: build constants, tuned by measurement.
+// Pairs of vectors in flight per thread (contiguous compress) and resident blocks per SM
+// the register budget is sized for: build constants, tuned by measurement.
 #ifndef FLEXQ_CODEC_UNROLL
-#define FLEXQ_CODEC_UNROLL 2
+#define FLEXQ_CODEC_UNROLL 1
 #endif
 #ifndef FLEXQ_CODEC_MINB
 #define FLEXQ_CODEC_MINB 4
@@ -72,42 +73,67 @@ __device__ __forceinline__ void divmod(int64_t n, int64_t d, const DivU32& dv, i
 }
 
 // ---------------------------------------------------------------------------------
-// contiguous compress: G groups of GS fp16, codes G x (GS*BITS/8) bytes, meta G half2
+// contiguous compress: G groups of GS fp16, codes G x (GS*BITS/8) bytes, meta G half2.
+// With 4-bit codes a lane holds two 16-byte vectors of one group, vectors sub and
+// sub + L, so that each load instruction of a warp still covers whole 32-byte sectors,
+// while the group's min/max shuffle reduction and its scale (an fp32 division) are
+// computed once per 16 values instead of once per 8: the 4-bit kernel is bound by instruction
+// issue about as much as by HBM, and those two steps were a fifth of its instructions
+// (76% -> 92% of HBM at group 64, 72% -> 95% at group 128). With 8-bit codes, whose
+// stores are twice as wide, splitting a lane's codes in two cost 4%, so there a lane
+// holds one vector of each of two groups.
+template <int BITS>
+constexpr int contig_vpl() { return BITS == 4 ? 2 : 1; }
+
 template <int BITS, int GS>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) compress_contig_kernel(const __half* __restrict__ x,
                                                                    uint8_t* __restrict__ codes,
                                                                    uint32_t* __restrict__ meta,
                                                                    int64_t G) {
-    constexpr int L = GS / 8;      // lanes per group
-    constexpr int GPW = 32 / L;    // groups per warp and step
+    constexpr int V = contig_vpl<BITS>();   // vectors per lane and group
+    constexpr int L = GS / (8 * V);         // lanes per group
+    constexpr int GPW = 32 / L;             // groups per warp and step
+    constexpr int U = kUnroll * 2 / V;      // groups per lane and step
     const int lane = threadIdx.x & 31;
     const int sub = lane % L;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     const int64_t stride = nwarps * GPW;
 
-    auto load = [&](uint4 (&v)[kUnroll], int64_t base) {
+    auto load = [&](uint4 (&v)[U][V], int64_t base) {
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int64_t g = base + u * stride + lane / L;
-            v[u] = g < G ? ld_stream_v4(x + g * GS + sub * 8) : make_uint4(0, 0, 0, 0);
+            const __half* p = x + g * GS + sub * 8;
+#pragma unroll
+            for (int j = 0; j < V; ++j) v[u][j] = g < G ? ld_stream_v4(p + j * L * 8) : make_uint4(0, 0, 0, 0);
         }
     };
-    auto process = [&](const uint4 (&v)[kUnroll], int64_t base) {
+    auto process = [&](const uint4 (&v)[U][V], int64_t base) {
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int64_t g = base + u * stride + lane / L;
             __half2 hmn, hmx;
-            minmax8(v[u], hmn, hmx);
+            minmax8(v[u][0], hmn, hmx);
+#pragma unroll
+            for (int j = 1; j < V; ++j) {
+                __half2 mn1, mx1;
+                minmax8(v[u][j], mn1, mx1);
+                hmn = __hmin2(hmn, mn1);
+                hmx = __hmax2(hmx, mx1);
+            }
             float mn, mx;
             group_minmax<L>(hmn, hmx, mn, mx);
             const __half s16 = group_scale16<BITS>(mn, mx);
             const float s = __half2float(s16);
             if (g < G) {
-                if (BITS == 4) {
-                    st_stream_u32(codes + g * (GS / 2) + sub * 4, quant8_4bit(v[u], mn, s));
-                } else {
-                    st_stream_v2(codes + g * GS + sub * 8, quant8_8bit(v[u], mn, s));
+#pragma unroll
+                for (int j = 0; j < V; ++j) {
+                    if (BITS == 4) {
+                        st_stream_u32(codes + g * (GS / 2) + (sub + j * L) * 4, quant8_4bit(v[u][j], mn, s));
+                    } else {
+                        st_stream_v2(codes + g * GS + (sub + j * L) * 8, quant8_8bit(v[u][j], mn, s));
+                    }
                 }
                 if (sub == 0) meta[g] = pack_half2_bits(stored_min16(mn), s16);
             }
@@ -116,15 +142,17 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) compress_contig_kernel(c
     // software pipelined: the next step's vectors are requested before this step's are
     // quantised, so the loads of one step overlap the arithmetic of the previous one
     int64_t base = warp * GPW;
-    uint4 v[kUnroll];
+    uint4 v[U][V];
     load(v, base);
     while (base < G) {
-        const int64_t next = base + stride * kUnroll;
-        uint4 nv[kUnroll];
+        const int64_t next = base + stride * U;
+        uint4 nv[U][V];
         load(nv, next);
         process(v, base);
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) v[u] = nv[u];
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int j = 0; j < V; ++j) v[u][j] = nv[u][j];
         base = next;
     }
 }
@@ -623,12 +651,14 @@ __device__ __forceinline__ int64_t var_col(int64_t q, int sub, int64_t G, int64_
     return o * G + col;
 }
 
+// Like the main 4-bit kernel, a lane holds two vectors of its group (vectors sub and
+// sub + L), so the group's reduction and scale division are done once per 16 values.
 template <int BITS, int GS, int SYM>
 __global__ void __launch_bounds__(kThreads) compress_var_contig_kernel(const __half* __restrict__ x,
                                                                         uint8_t* __restrict__ codes,
                                                                         uint32_t* __restrict__ meta, int64_t rows,
                                                                         int64_t G, int64_t ng, DivU32 dv) {
-    constexpr int L = GS / 8;                  // lanes per group
+    constexpr int L = GS / 16;                 // lanes per group
     constexpr int GPW = 32 / L;                // groups per warp and step
     constexpr int CB = GS * BITS / 8;          // code bytes per group
     const int lane = threadIdx.x & 31, sub = lane % L;
@@ -636,24 +666,31 @@ __global__ void __launch_bounds__(kThreads) compress_var_contig_kernel(const __h
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     const int64_t total = rows * ng;
     const bool whole = ng * GS == G;
-    auto load = [&](int64_t base) {
+    auto load = [&](uint4 (&v)[2], int64_t base) {
         const int64_t q = base + lane / L;
-        bool ok = false;
-        const int64_t at = q < total ? var_col<GS>(q, sub, G, ng, whole, dv, ok) : 0;
-        return (q < total && ok) ? ld_stream_v4(x + at) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            bool ok = false;
+            const int64_t at = q < total ? var_col<GS>(q, sub + j * L, G, ng, whole, dv, ok) : 0;
+            v[j] = (q < total && ok) ? ld_stream_v4(x + at) : make_uint4(0u, 0u, 0u, 0u);
+        }
     };
-    // software pipelined: the next step's vector is requested before this one is quantised
+    // software pipelined: the next step's vectors are requested before these are quantised
     int64_t base = warp * GPW;
-    uint4 v = load(base);
+    uint4 v[2];
+    load(v, base);
     while (base < total) {
         const int64_t next = base + nwarps * GPW;
-        const uint4 nv = load(next);
+        uint4 nv[2];
+        load(nv, next);
         const int64_t q = base + lane / L;
         float mn = 0.0f;
         __half s16 = __ushort_as_half(0);
         if (SYM) {
-            const __half2* h = reinterpret_cast<const __half2*>(&v);
-            __half2 a2 = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
+            const __half2* h = reinterpret_cast<const __half2*>(&v[0]);
+            const __half2* k = reinterpret_cast<const __half2*>(&v[1]);
+            __half2 a2 = __hmax2(__hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3]))),
+                                 __hmax2(__hmax2(__habs2(k[0]), __habs2(k[1])), __hmax2(__habs2(k[2]), __habs2(k[3]))));
 #pragma unroll
             for (int off = 1; off < L; off <<= 1) {
                 const uint32_t o2 = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<const uint32_t*>(&a2), off);
@@ -665,25 +702,30 @@ __global__ void __launch_bounds__(kThreads) compress_var_contig_kernel(const __h
                 if (__hisinf(s16)) s16 = __ushort_as_half(0x7BFF);
             }
         } else {
-            __half2 hmn, hmx;
-            minmax8(v, hmn, hmx);
+            __half2 hmn, hmx, mn1, mx1;
+            minmax8(v[0], hmn, hmx);
+            minmax8(v[1], mn1, mx1);
             float mx;
-            group_minmax<L>(hmn, hmx, mn, mx);
+            group_minmax<L>(__hmin2(hmn, mn1), __hmax2(hmx, mx1), mn, mx);
             s16 = group_scale16<BITS>(mn, mx);
         }
         if (q < total) {
-            const uint32_t u = var_quant8<BITS, SYM>(v, mn, __half2float(s16));
-            uint8_t* dst = codes + q * CB + sub * BITS;
-            if (BITS == 4) {
-                *reinterpret_cast<uint32_t*>(dst) = u;
-            } else {                           // 3 bytes, little-endian
-                dst[0] = static_cast<uint8_t>(u);
-                dst[1] = static_cast<uint8_t>(u >> 8);
-                dst[2] = static_cast<uint8_t>(u >> 16);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const uint32_t u = var_quant8<BITS, SYM>(v[j], mn, __half2float(s16));
+                uint8_t* dst = codes + q * CB + (sub + j * L) * BITS;
+                if (BITS == 4) {
+                    *reinterpret_cast<uint32_t*>(dst) = u;
+                } else {                           // 3 bytes, little-endian
+                    dst[0] = static_cast<uint8_t>(u);
+                    dst[1] = static_cast<uint8_t>(u >> 8);
+                    dst[2] = static_cast<uint8_t>(u >> 16);
+                }
             }
             if (sub == 0) meta[q] = pack_half2_bits(SYM ? __ushort_as_half(0) : stored_min16(mn), s16);
         }
-        v = nv;
+        v[0] = nv[0];
+        v[1] = nv[1];
         base = next;
     }
 }
@@ -909,8 +951,9 @@ int launch_compress(const Geometry& g, const __half* x, uint8_t* codes, uint32_t
                     cudaStream_t st) {
     if (g.inner == 1) {
         const int64_t G = g.outer * g.ng;
-        const int64_t lanes = G * (GS / 8);
-        const unsigned grid = grid_for<compress_contig_kernel<BITS, GS>>((lanes + kUnroll - 1) / kUnroll);
+        constexpr int U = kUnroll * 2 / contig_vpl<BITS>();     // groups per lane and step
+        const int64_t lanes = G * (GS / (8 * contig_vpl<BITS>()));
+        const unsigned grid = grid_for<compress_contig_kernel<BITS, GS>>((lanes + U - 1) / U);
         compress_contig_kernel<BITS, GS><<<grid, kThreads, 0, st>>>(x, codes, meta, G);
     } else {
         const bool vec = (g.inner % 8 == 0);
@@ -959,9 +1002,9 @@ int launch_var(const Geometry& g, const __half* x, uint8_t* codes, uint32_t* met
             compress_var8_contig_kernel<GS, SYM>
                 <<<grid_for<compress_var8_contig_kernel<GS, SYM>>(lanes), kThreads, 0, st>>>(x, codes, meta, g.outer,
                                                                                               g.G, g.ng, dv);
-        } else {
+        } else {                               // two vectors per lane
             compress_var_contig_kernel<BITS, GS, SYM>
-                <<<grid_for<compress_var_contig_kernel<BITS, GS, SYM>>(lanes), kThreads, 0, st>>>(x, codes, meta,
+                <<<grid_for<compress_var_contig_kernel<BITS, GS, SYM>>(lanes / 2), kThreads, 0, st>>>(x, codes, meta,
                                                                                                    g.outer, g.G, g.ng, dv);
         }
     } else {

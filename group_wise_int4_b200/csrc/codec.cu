@@ -383,8 +383,20 @@ __global__ void __launch_bounds__(kThreads) compress_strided_kernel(const __half
     }
 }
 
+// Resident blocks per SM the strided decompress is compiled for, and code rows in flight
+// per thread: measured per configuration. 4-bit codes at group 32 / 64 gain 2-5% from a
+// fifth block per SM (a few registers spill) and lose 3% at group 128; 8-bit codes gain 4%
+// from 8 rows in flight, 4-bit ones lose 2-7%. (The other counts only keep each kernel at
+// the registers it takes without a bound: an explicit bound of 1 lets it take ~95.)
 template <int BITS, int GS, int VEC>
-__global__ void __launch_bounds__(kThreads) decompress_strided_kernel(const uint8_t* __restrict__ codes,
+constexpr int strided_dec_minb() {
+    return VEC == 1 ? (BITS == 4 ? 8 : 6) : BITS == 8 ? 5 : GS < 128 ? 5 : 4;
+}
+template <int BITS>
+constexpr int strided_dec_rows() { return BITS == 8 ? 8 : 4; }
+
+template <int BITS, int GS, int VEC>
+__global__ void __launch_bounds__(kThreads, strided_dec_minb<BITS, GS, VEC>()) decompress_strided_kernel(const uint8_t* __restrict__ codes,
                                                                       const uint32_t* __restrict__ meta,
                                                                       __half* __restrict__ y,
                                                                       int64_t outer, int64_t ng,
@@ -425,7 +437,8 @@ __global__ void __launch_bounds__(kThreads) decompress_strided_kernel(const uint
         const uint8_t* src = codes + og * CB * inner + c0;
         __half* dst = y + og * GS * inner + c0;
         if (VEC == 8) {
-#pragma unroll 4
+            constexpr int JU = strided_dec_rows<BITS>();
+#pragma unroll JU
             for (int j = 0; j < CB; ++j) {
                 uint2 cw;
                 asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"

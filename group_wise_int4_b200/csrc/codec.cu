@@ -647,30 +647,59 @@ __device__ __forceinline__ uint32_t var_quant8(uint4 v, float mn, float s) {
     return u;
 }
 
-// Address of lane `sub` of group q: flat when every group is whole (ng GS == G), else
-// through the row (a partial last group leaves a gap of padding in the group index).
-template <int GS>
-__device__ __forceinline__ int64_t var_col(int64_t q, int sub, int64_t G, int64_t ng, bool whole, const DivU32& dv,
-                                           bool& ok) {
-    if (whole) {
-        ok = true;
-        return q * GS + sub * 8;
+// Group q of the [rows][ng] grid of groups, with its row o = q / ng and its index gi = q %
+// ng in the row. A thread's groups form an arithmetic sequence (its grid stride is a
+// multiple of the lanes per group), so the walk advances (o, gi) by (D / ng, D % ng), taken
+// once per thread, and one conditional subtraction, instead of dividing for every group.
+// When every group is whole (ng GS == G, the WHOLE instantiation) the address is flat and
+// only q is kept: the row state would cost registers and resident blocks (3-11% measured).
+// (gi + dr < 2 ng and the stride fit 31 bits: the stride is at most the threads of a
+// resident grid, and the launcher routes ng >= 2^30 to the generic kernels.)
+template <int GS, bool WHOLE>
+struct GroupWalk {
+    int64_t q, o;
+    int32_t gi, dq, dr, D;
+    __device__ __forceinline__ GroupWalk(int64_t q0, int64_t stride, int64_t ng) : q(q0), D(static_cast<int32_t>(stride)) {
+        if constexpr (!WHOLE) {
+            o = q0 / ng;
+            gi = static_cast<int32_t>(q0 - o * ng);
+            dq = static_cast<int32_t>(stride / ng);
+            dr = static_cast<int32_t>(stride - static_cast<int64_t>(dq) * ng);
+        }
     }
-    const int64_t o = ng == 1 ? q
-                      : (dv.l > 0 && q < 0x7FFFFFFF) ? static_cast<int64_t>(div_u32(static_cast<uint32_t>(q), dv))
-                                                     : q / ng;
-    const int64_t gi = q - o * ng, col = gi * GS + sub * 8;
-    ok = col < G;
-    return o * G + col;
-}
+    __device__ __forceinline__ void step(int64_t ng) {
+        q += D;
+        if constexpr (!WHOLE) {
+            o += dq;
+            gi += dr;
+            if (gi >= static_cast<int32_t>(ng)) {
+                gi -= static_cast<int32_t>(ng);
+                ++o;
+            }
+        }
+    }
+    // Element offset of the 8 values at position `sub` (in units of 8) of the walk's group,
+    // passed again as gq (a caller that knows it saves the walk's copy), and whether they
+    // lie inside the row (a partial last group leaves padding).
+    __device__ __forceinline__ int64_t at(int64_t gq, int sub, int64_t G, bool& ok) const {
+        if constexpr (WHOLE) {
+            ok = true;
+            return gq * GS + sub * 8;
+        } else {
+            const int64_t col = static_cast<int64_t>(gi) * GS + sub * 8;
+            ok = col < G;
+            return o * G + col;
+        }
+    }
+};
 
 // Like the main 4-bit kernel, a lane holds two vectors of its group (vectors sub and
 // sub + L), so the group's reduction and scale division are done once per 16 values.
-template <int BITS, int GS, int SYM>
+template <int BITS, int GS, int SYM, bool WHOLE>
 __global__ void __launch_bounds__(kThreads) compress_var_contig_kernel(const __half* __restrict__ x,
                                                                         uint8_t* __restrict__ codes,
                                                                         uint32_t* __restrict__ meta, int64_t rows,
-                                                                        int64_t G, int64_t ng, DivU32 dv) {
+                                                                        int64_t G, int64_t ng) {
     constexpr int L = GS / 16;                 // lanes per group
     constexpr int GPW = 32 / L;                // groups per warp and step
     constexpr int CB = GS * BITS / 8;          // code bytes per group
@@ -678,15 +707,16 @@ __global__ void __launch_bounds__(kThreads) compress_var_contig_kernel(const __h
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     const int64_t total = rows * ng;
-    const bool whole = ng * GS == G;
+    GroupWalk<GS, WHOLE> walk(warp * GPW + lane / L, nwarps * GPW, ng);   // the group of the next load
     auto load = [&](uint4 (&v)[2], int64_t base) {
         const int64_t q = base + lane / L;
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             bool ok = false;
-            const int64_t at = q < total ? var_col<GS>(q, sub + j * L, G, ng, whole, dv, ok) : 0;
+            const int64_t at = q < total ? walk.at(q, sub + j * L, G, ok) : 0;
             v[j] = (q < total && ok) ? ld_stream_v4(x + at) : make_uint4(0u, 0u, 0u, 0u);
         }
+        walk.step(ng);
     };
     // software pipelined: the next step's vectors are requested before these are quantised
     int64_t base = warp * GPW;
@@ -745,23 +775,32 @@ __global__ void __launch_bounds__(kThreads) compress_var_contig_kernel(const __h
 
 // 8-bit codes of the contiguous variants (8 code bytes per lane): the symmetric form, or
 // the min/max form of a partial last group.
-template <int GS, int SYM>
+template <int GS, int SYM, bool WHOLE>
 __global__ void __launch_bounds__(kThreads) compress_var8_contig_kernel(const __half* __restrict__ x,
                                                                          uint8_t* __restrict__ codes,
                                                                          uint32_t* __restrict__ meta, int64_t rows,
-                                                                         int64_t G, int64_t ng, DivU32 dv) {
+                                                                         int64_t G, int64_t ng) {
     constexpr int L = GS / 8, GPW = 32 / L, B = 127;
     const int lane = threadIdx.x & 31, sub = lane % L;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     const int64_t total = rows * ng;
-    const bool whole = ng * GS == G;
-    for (int64_t base = warp * GPW; base < total; base += nwarps * GPW) {
+    GroupWalk<GS, WHOLE> walk(warp * GPW + lane / L, nwarps * GPW, ng);   // the group of the next load
+    auto load = [&](int64_t base) {
+        const int64_t q = base + lane / L;
+        bool okv = false;
+        const int64_t at = q < total ? walk.at(q, sub, G, okv) : 0;
+        walk.step(ng);
+        return (q < total && okv) ? ld_stream_v4(x + at) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    // software pipelined: the next step's vector is requested before this one is quantised
+    int64_t base = warp * GPW;
+    uint4 v = load(base);
+    while (base < total) {
+        const int64_t next = base + nwarps * GPW;
+        const uint4 nv = load(next);
         const int64_t q = base + lane / L;
         const bool okg = q < total;
-        bool okv = false;
-        const int64_t at = okg ? var_col<GS>(q, sub, G, ng, whole, dv, okv) : 0;
-        const uint4 v = (okg && okv) ? ld_stream_v4(x + at) : make_uint4(0u, 0u, 0u, 0u);
         float mn = 0.0f;
         __half s16 = __ushort_as_half(0);
         if (SYM) {
@@ -784,40 +823,43 @@ __global__ void __launch_bounds__(kThreads) compress_var8_contig_kernel(const __
             group_minmax<L>(hmn, hmx, mn, mx);
             s16 = group_scale16<8>(mn, mx);
         }
-        if (!okg) continue;
-        const float s = __half2float(s16);
-        uint2 out;
-        if (SYM) {
-            const uint64_t s2 = f2_pack(s, s);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t b8[8];
+        if (okg) {
+            const float s = __half2float(s16);
+            uint2 out;
+            if (SYM) {
+                const uint64_t s2 = f2_pack(s, s);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t b8[8];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float p0, p1;
-                f2_unpack(f2_mul(f2_pack(h2f_lo(w[k]), h2f_hi(w[k])), s2), p0, p1);
-                p0 = (p0 == p0) ? p0 : 0.0f;
-                p1 = (p1 == p1) ? p1 : 0.0f;
-                f2_unpack(f2_add(f2_pack(p0, p1), f2_pack(12582912.0f, 12582912.0f)), p0, p1);
-                b8[2 * k] = (__float_as_uint(p0) + B) & 0xFFu;
-                b8[2 * k + 1] = (__float_as_uint(p1) + B) & 0xFFu;
+                for (int k = 0; k < 4; ++k) {
+                    float p0, p1;
+                    f2_unpack(f2_mul(f2_pack(h2f_lo(w[k]), h2f_hi(w[k])), s2), p0, p1);
+                    p0 = (p0 == p0) ? p0 : 0.0f;
+                    p1 = (p1 == p1) ? p1 : 0.0f;
+                    f2_unpack(f2_add(f2_pack(p0, p1), f2_pack(12582912.0f, 12582912.0f)), p0, p1);
+                    b8[2 * k] = (__float_as_uint(p0) + B) & 0xFFu;
+                    b8[2 * k + 1] = (__float_as_uint(p1) + B) & 0xFFu;
+                }
+                out = make_uint2(pack_low_bytes(b8[0], b8[1], b8[2], b8[3]), pack_low_bytes(b8[4], b8[5], b8[6], b8[7]));
+            } else {
+                out = quant8_8bit(v, mn, s);
             }
-            out = make_uint2(pack_low_bytes(b8[0], b8[1], b8[2], b8[3]), pack_low_bytes(b8[4], b8[5], b8[6], b8[7]));
-        } else {
-            out = quant8_8bit(v, mn, s);
+            *reinterpret_cast<uint2*>(codes + q * GS + sub * 8) = out;
+            if (sub == 0) meta[q] = pack_half2_bits(SYM ? __ushort_as_half(0) : stored_min16(mn), s16);
         }
-        *reinterpret_cast<uint2*>(codes + q * GS + sub * 8) = out;
-        if (sub == 0) meta[q] = pack_half2_bits(SYM ? __ushort_as_half(0) : stored_min16(mn), s16);
+        v = nv;
+        base = next;
     }
 }
 
 // Decompression of the contiguous variants: one item = 8 values of one group (BITS bytes
 // of codes in, one 16-byte store out); items past G (padding) write nothing. Four items
 // per thread and step, their codes and metadata requested before any is converted.
-template <int BITS, int GS, int SYM>
+template <int BITS, int GS, int SYM, bool WHOLE>
 __global__ void __launch_bounds__(kThreads) decompress_var_contig_kernel(const uint8_t* __restrict__ codes,
                                                                           const uint32_t* __restrict__ meta,
                                                                           __half* __restrict__ y, int64_t rows,
-                                                                          int64_t G, int64_t ng, DivU32 dv) {
+                                                                          int64_t G, int64_t ng) {
     constexpr int L = GS / 8;
     constexpr int CB = GS * BITS / 8;
     constexpr int B = (1 << (BITS - 1)) - 1;
@@ -825,7 +867,10 @@ __global__ void __launch_bounds__(kThreads) decompress_var_contig_kernel(const u
     const int64_t items = rows * ng * L;
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
-    const bool whole = ng * GS == G;
+    // item it = tid + m nthreads (m = 0, 1, ...): group tid / L + m (nthreads / L), position
+    // tid % L in it (nthreads is a multiple of L, a power of two)
+    const int sub = static_cast<int>(tid & (L - 1));
+    GroupWalk<GS, WHOLE> walk(tid / L, nthreads / L, ng);
     for (int64_t base = tid; base < items; base += nthreads * U) {
         uint32_t c0[U], c1[U], mw[U];
         int64_t at[U];
@@ -833,11 +878,11 @@ __global__ void __launch_bounds__(kThreads) decompress_var_contig_kernel(const u
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t it = base + u * nthreads;
-            const int64_t q = it / L;                       // L is a power of two
-            const int sub = static_cast<int>(it & (L - 1));
+            const int64_t q = WHOLE ? it / L : walk.q;      // L is a power of two
             ok[u] = false;
-            at[u] = it < items ? var_col<GS>(q, sub, G, ng, whole, dv, ok[u]) : 0;
+            at[u] = it < items ? walk.at(q, sub, G, ok[u]) : 0;
             ok[u] = ok[u] && it < items;
+            walk.step(ng);
             c0[u] = c1[u] = mw[u] = 0u;
             if (ok[u]) {
                 const uint8_t* src = codes + q * CB + sub * BITS;
@@ -1005,27 +1050,33 @@ int launch_decompress(const Geometry& g, const uint8_t* codes, const uint32_t* m
 }
 
 // The contiguous-group variants (3-bit, symmetric, partial last group with G % 8 == 0).
+template <int BITS, int GS, int SYM, bool WHOLE>
+int launch_var_w(const Geometry& g, const __half* x, uint8_t* codes, uint32_t* meta, const uint8_t* ccodes,
+                 const uint32_t* cmeta, __half* y, cudaStream_t st) {
+    const int64_t lanes = g.outer * g.ng * (GS / 8);
+    if (x != nullptr) {
+        if constexpr (BITS == 8) {
+            compress_var8_contig_kernel<GS, SYM, WHOLE>
+                <<<grid_for<compress_var8_contig_kernel<GS, SYM, WHOLE>>(lanes), kThreads, 0, st>>>(x, codes, meta, g.outer,
+                                                                                                     g.G, g.ng);
+        } else {                               // two vectors per lane
+            compress_var_contig_kernel<BITS, GS, SYM, WHOLE>
+                <<<grid_for<compress_var_contig_kernel<BITS, GS, SYM, WHOLE>>(lanes / 2), kThreads, 0, st>>>(
+                    x, codes, meta, g.outer, g.G, g.ng);
+        }
+    } else {
+        decompress_var_contig_kernel<BITS, GS, SYM, WHOLE>
+            <<<grid_for<decompress_var_contig_kernel<BITS, GS, SYM, WHOLE>>(lanes), kThreads, 0, st>>>(ccodes, cmeta, y,
+                                                                                                        g.outer, g.G, g.ng);
+    }
+    return launch_status();
+}
+
 template <int BITS, int GS, int SYM>
 int launch_var(const Geometry& g, const __half* x, uint8_t* codes, uint32_t* meta, const uint8_t* ccodes,
                const uint32_t* cmeta, __half* y, cudaStream_t st) {
-    const int64_t lanes = g.outer * g.ng * (GS / 8);
-    const DivU32 dv = make_div(g.ng);
-    if (x != nullptr) {
-        if constexpr (BITS == 8) {
-            compress_var8_contig_kernel<GS, SYM>
-                <<<grid_for<compress_var8_contig_kernel<GS, SYM>>(lanes), kThreads, 0, st>>>(x, codes, meta, g.outer,
-                                                                                              g.G, g.ng, dv);
-        } else {                               // two vectors per lane
-            compress_var_contig_kernel<BITS, GS, SYM>
-                <<<grid_for<compress_var_contig_kernel<BITS, GS, SYM>>(lanes / 2), kThreads, 0, st>>>(x, codes, meta,
-                                                                                                   g.outer, g.G, g.ng, dv);
-        }
-    } else {
-        decompress_var_contig_kernel<BITS, GS, SYM>
-            <<<grid_for<decompress_var_contig_kernel<BITS, GS, SYM>>(lanes), kThreads, 0, st>>>(ccodes, cmeta, y,
-                                                                                                 g.outer, g.G, g.ng, dv);
-    }
-    return launch_status();
+    if (g.ng * GS == g.G) return launch_var_w<BITS, GS, SYM, true>(g, x, codes, meta, ccodes, cmeta, y, st);
+    return launch_var_w<BITS, GS, SYM, false>(g, x, codes, meta, ccodes, cmeta, y, st);
 }
 
 template <int BITS, int SYM>
@@ -1040,7 +1091,8 @@ int launch_var_gs(const Geometry& g, int gs, const __half* x, uint8_t* codes, ui
 // last one and its extent a multiple of 8, else the one-thread-per-group kernels.
 int launch_variant(const Geometry& g, const flexq_config& cfg, const __half* x, uint8_t* codes, uint32_t* meta,
                    const uint8_t* ccodes, const uint32_t* cmeta, __half* y, cudaStream_t st) {
-    if (g.inner != 1 || g.G % 8 != 0) return launch_generic(g, cfg, x, codes, meta, ccodes, cmeta, y, st);
+    if (g.inner != 1 || g.G % 8 != 0 || g.ng >= (int64_t{1} << 30))
+        return launch_generic(g, cfg, x, codes, meta, ccodes, cmeta, y, st);
     const int gs = cfg.group_size;
     if (cfg.symmetric) {
         if (cfg.num_bits == 3) return launch_var_gs<3, 1>(g, gs, x, codes, meta, ccodes, cmeta, y, st);

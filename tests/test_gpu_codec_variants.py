@@ -67,3 +67,25 @@ def test_variants_256mb_sampled(bits, sym, gd):
             assert_bits_equal(meta[g:g + 1][:, cols], rm, "meta")
             assert_bits_equal(y[g * 64:(g + 1) * 64][:, cols], oc.decompress(rc, rm, xs.shape, bits, 64, 0,
                                                                             symmetric=sym), "y")
+
+
+@pytest.mark.parametrize("bits,sym,gs", [(4, False, 64), (8, False, 64), (3, True, 128)])
+def test_variants_partial_groups_large_sampled(bits, sym, gs):
+    """[65536, 1000] (131 MB fp16): every row ends in a partial group, and each thread of
+    the variant kernels walks about ten groups across row boundaries (grid stride), so
+    the row and in-row index it steps forward are checked; 66 sampled rows equal the
+    oracle's."""
+    shape = (65536, 1000)
+    full = (shape[0], -(-shape[1] // gs) * gs)
+    x = synth.codec_tensor(full, 1, gs, seed=12, device="cuda")[:, :shape[1]].contiguous()
+    cfg = fq.config(bits, gs, 1, int(sym))
+    codes, meta = fq.flexq_compress(x, cfg)
+    y = fq.flexq_decompress(codes, meta, shape, cfg)
+    sync_status()
+    rng = np.random.default_rng(5)
+    rows = sorted({0, 1, shape[0] - 1, *rng.integers(0, shape[0], 63).tolist()})
+    xs = to_np(x[rows])
+    rc, rm = oc.compress(xs, bits, gs, 1, symmetric=sym)
+    assert_bits_equal(codes[rows], rc, "codes")
+    assert_bits_equal(meta[rows], rm, "meta")
+    assert_bits_equal(y[rows], oc.decompress(rc, rm, xs.shape, bits, gs, 1, symmetric=sym), "y")

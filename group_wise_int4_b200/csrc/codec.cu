@@ -606,13 +606,14 @@ __global__ void __launch_bounds__(kThreads) decompress_generic_kernel(const uint
 
 // ---------------------------------------------------------------------------------
 // Codec variants on contiguous groups (group_dim the last one, its extent G a multiple of
-// 8): the layout of the main contiguous kernels - gs/8 lanes per group, 8 values per
-// lane from one 16-byte load - with the variants' arithmetic, bit for bit that of the
-// one-thread-per-group kernels above. A lane whose 8 values lie past G (the padding of a
-// partial last group; G % 8 == 0, so a lane is wholly in or out) takes zeros, which count
-// in min/max and max|x|, and its codes are stored like any other. 3-bit codes: the 8 of
-// a lane are bits [24 l, 24 l + 24) of its group's little-endian stream, i.e. 3 whole
-// bytes at byte 3 l.
+// 8): the layout of the main contiguous kernels - 8 values per 16-byte load, the lanes of
+// a group reducing min/max (or max|x|) with shuffles; compress with 3- and 4-bit codes
+// gives a lane two vectors of its group - with the variants' arithmetic, bit for bit
+// that of the one-thread-per-group kernels above. A vector whose 8 values lie past G (the
+// padding of a partial last group; G % 8 == 0, so a vector is wholly in or out) is taken
+// as zeros, which count in min/max and max|x|, and its codes are stored like any other.
+// 3-bit codes: the 8 codes of vector l of a group are bits [24 l, 24 l + 24) of the
+// group's little-endian stream, i.e. 3 whole bytes at byte 3 l.
 template <int BITS, int SYM>
 __device__ __forceinline__ uint32_t var_quant8(uint4 v, float mn, float s) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};

@@ -853,18 +853,21 @@ __global__ void __launch_bounds__(kThreads) compress_var8_contig_kernel(const __
     }
 }
 
-// Decompression of the contiguous variants: one item = 8 values of one group (BITS bytes
-// of codes in, one 16-byte store out); items past G (padding) write nothing. Four items
-// per thread and step, their codes and metadata requested before any is converted.
+// Decompression of the contiguous variants: one item = vectors sub and sub + L of one
+// group (L = GS / 16 lanes per group; BITS bytes of codes in and one 16-byte store out per
+// vector), so the group's step (an fp32 division) and the index arithmetic are done once
+// per 16 values, as in compression: the kernel is bound by instruction issue. A vector
+// past G (padding) writes nothing. Two items per thread and step, their codes and
+// metadata requested before any is converted.
 template <int BITS, int GS, int SYM, bool WHOLE>
 __global__ void __launch_bounds__(kThreads) decompress_var_contig_kernel(const uint8_t* __restrict__ codes,
                                                                           const uint32_t* __restrict__ meta,
                                                                           __half* __restrict__ y, int64_t rows,
                                                                           int64_t G, int64_t ng) {
-    constexpr int L = GS / 8;
+    constexpr int L = GS / 16;
     constexpr int CB = GS * BITS / 8;
     constexpr int B = (1 << (BITS - 1)) - 1;
-    constexpr int U = 4;
+    constexpr int U = 2;
     const int64_t items = rows * ng * L;
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
@@ -873,63 +876,72 @@ __global__ void __launch_bounds__(kThreads) decompress_var_contig_kernel(const u
     const int sub = static_cast<int>(tid & (L - 1));
     GroupWalk<GS, WHOLE> walk(tid / L, nthreads / L, ng);
     for (int64_t base = tid; base < items; base += nthreads * U) {
-        uint32_t c0[U], c1[U], mw[U];
-        int64_t at[U];
-        bool ok[U];
+        uint2 c[U][2];
+        uint32_t mw[U];
+        int64_t at[U][2];
+        bool ok[U][2];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t it = base + u * nthreads;
             const int64_t q = WHOLE ? it / L : walk.q;      // L is a power of two
-            ok[u] = false;
-            at[u] = it < items ? walk.at(q, sub, G, ok[u]) : 0;
-            ok[u] = ok[u] && it < items;
-            walk.step(ng);
-            c0[u] = c1[u] = mw[u] = 0u;
-            if (ok[u]) {
-                const uint8_t* src = codes + q * CB + sub * BITS;
-                if (BITS == 8) {
-                    const uint2 c = __ldg(reinterpret_cast<const uint2*>(src));
-                    c0[u] = c.x;
-                    c1[u] = c.y;
-                } else if (BITS == 4) {
-                    c0[u] = __ldg(reinterpret_cast<const uint32_t*>(src));
-                } else {
-                    c0[u] = static_cast<uint32_t>(__ldg(src)) | (static_cast<uint32_t>(__ldg(src + 1)) << 8) |
-                            (static_cast<uint32_t>(__ldg(src + 2)) << 16);
+            const bool in = it < items;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                ok[u][j] = false;
+                at[u][j] = in ? walk.at(q, sub + j * L, G, ok[u][j]) : 0;
+                ok[u][j] = ok[u][j] && in;
+                c[u][j] = make_uint2(0u, 0u);
+                if (ok[u][j]) {
+                    const uint8_t* src = codes + q * CB + (sub + j * L) * BITS;
+                    if (BITS == 8) {
+                        c[u][j] = __ldg(reinterpret_cast<const uint2*>(src));
+                    } else if (BITS == 4) {
+                        c[u][j].x = __ldg(reinterpret_cast<const uint32_t*>(src));
+                    } else {
+                        c[u][j].x = static_cast<uint32_t>(__ldg(src)) | (static_cast<uint32_t>(__ldg(src + 1)) << 8) |
+                                    (static_cast<uint32_t>(__ldg(src + 2)) << 16);
+                    }
                 }
-                mw[u] = __ldg(meta + q);
             }
+            // vector sub + L lies further along the row than vector sub: if sub is padding,
+            // so is sub + L
+            mw[u] = ok[u][0] ? __ldg(meta + q) : 0u;
+            walk.step(ng);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            if (!ok[u]) continue;
+            if (!ok[u][0]) continue;
             const uint32_t m = mw[u];
             const float step = group_step(__ushort_as_half(static_cast<unsigned short>(m >> 16)));
-            const uint32_t cw[2] = {c0[u], c1[u]};
-            uint32_t out[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                uint32_t q0, q1;
-                if (BITS == 8) {
-                    q0 = (cw[k / 2] >> (16 * (k % 2))) & 0xFFu;
-                    q1 = (cw[k / 2] >> (16 * (k % 2) + 8)) & 0xFFu;
-                } else {
-                    q0 = (cw[0] >> (BITS * 2 * k)) & ((1u << BITS) - 1u);
-                    q1 = (cw[0] >> (BITS * (2 * k + 1))) & ((1u << BITS) - 1u);
+            for (int j = 0; j < 2; ++j) {
+                if (!ok[u][j]) continue;
+                const uint32_t cw[2] = {c[u][j].x, c[u][j].y};
+                uint32_t out[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    uint32_t q0, q1;
+                    if (BITS == 8) {
+                        q0 = (cw[k / 2] >> (16 * (k % 2))) & 0xFFu;
+                        q1 = (cw[k / 2] >> (16 * (k % 2) + 8)) & 0xFFu;
+                    } else {
+                        q0 = (cw[0] >> (BITS * 2 * k)) & ((1u << BITS) - 1u);
+                        q1 = (cw[0] >> (BITS * (2 * k + 1))) & ((1u << BITS) - 1u);
+                    }
+                    if (SYM) {
+                        // x^ = fp16(fl((u - B) * step)); an all-zero group (step 0) gives 0
+                        const __half2 hv =
+                            __floats2half2_rn(__fmul_rn(static_cast<float>(static_cast<int>(q0) - B), step),
+                                              __fmul_rn(static_cast<float>(static_cast<int>(q1) - B), step));
+                        out[k] = *reinterpret_cast<const uint32_t*>(&hv);
+                    } else if (step == 0.0f) {
+                        out[k] = (m & 0xFFFFu) * 0x10001u;
+                    } else {
+                        out[k] = dequant_two(q0, q1, step, h2f_lo(m));
+                    }
                 }
-                if (SYM) {
-                    // x^ = fp16(fl((u - B) * step)); an all-zero group (step 0) gives 0
-                    const __half2 hv =
-                        __floats2half2_rn(__fmul_rn(static_cast<float>(static_cast<int>(q0) - B), step),
-                                          __fmul_rn(static_cast<float>(static_cast<int>(q1) - B), step));
-                    out[k] = *reinterpret_cast<const uint32_t*>(&hv);
-                } else if (step == 0.0f) {
-                    out[k] = (m & 0xFFFFu) * 0x10001u;
-                } else {
-                    out[k] = dequant_two(q0, q1, step, h2f_lo(m));
-                }
+                st_stream_v4(y + at[u][j], make_uint4(out[0], out[1], out[2], out[3]));
             }
-            st_stream_v4(y + at[u], make_uint4(out[0], out[1], out[2], out[3]));
         }
     }
 }
@@ -1066,8 +1078,8 @@ int launch_var_w(const Geometry& g, const __half* x, uint8_t* codes, uint32_t* m
                     x, codes, meta, g.outer, g.G, g.ng);
         }
     } else {
-        decompress_var_contig_kernel<BITS, GS, SYM, WHOLE>
-            <<<grid_for<decompress_var_contig_kernel<BITS, GS, SYM, WHOLE>>(lanes), kThreads, 0, st>>>(ccodes, cmeta, y,
+        decompress_var_contig_kernel<BITS, GS, SYM, WHOLE>      // two vectors per lane
+            <<<grid_for<decompress_var_contig_kernel<BITS, GS, SYM, WHOLE>>(lanes / 2), kThreads, 0, st>>>(ccodes, cmeta, y,
                                                                                                         g.outer, g.G, g.ng);
     }
     return launch_status();
